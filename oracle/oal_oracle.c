@@ -1,0 +1,226 @@
+/*
+ * oal_oracle.c -- plain fp64 CPU oracle for OAL causal grouped positive-quadratic attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path links, loads or calls this file:
+ * only the test suite, the smoke check and the CPU-baseline leg of the benchmark use it.
+ * It shares no code, header, table or helper with the CUDA library.
+ *
+ * Source of every formula: "OAL: 按 QK 离群贡献分组的正二次注意力核" (daiwk auto-research
+ * reproduction note of arXiv 2610.13674), section 核心公式 (core formulas):
+ *   eq. (2)  s_g = sum_{r in G_g} q_r k_r / sqrt(d_h),   sbar = [1, s_1, ..., s_G]
+ *   eq. (3)  kappa(q, k) = eps + sbar^T L L^T sbar  (> 0)
+ *   eq. (4)  H0_i = sum_{j<=i} [v_j; 1],  H1_{i,r} = sum_{j<=i} k_{j,r} [v_j; 1],
+ *            H2_{i,rt} = sum_{j<=i} k_{j,r} k_{j,t} [v_j; 1]
+ *   eq. (5)  u_i = a H0_i + (1/sqrt(d_h)) sum_r b_r q_{i,r} H1_{i,r}
+ *                 + (1/d_h) sum_{r,t} C_rt q_{i,r} q_{i,t} H2_{i,rt},
+ *            yhat_i = u_{i,1:dv} / u_{i,dv+1}
+ *
+ * Readings where the page is silent (each is also listed in the design notes):
+ *  - a, b_r, C_rt are not printed.  Expanding eq. (3) with sbar_0 = 1 gives
+ *    a = eps + M_00, b_r = 2 M_{0,g(r)}, C_rt = M_{g(r),g(t)} with M = L L^T; this is the
+ *    only choice that makes eq. (5) equal eq. (3) summed over j <= i.
+ *  - causality is inclusive (j <= i), as written in eq. (4).
+ *  - group ids run 1..G; index 0 of sbar is the constant 1.
+ *  - L is used exactly as given (M = L L^T over the leading (G+1)x(G+1) block of a
+ *    (Gmax+1)x(Gmax+1) row-major array); it need not be triangular.
+ *  - GQA: query head h reads key/value head floor(h * Hkv / Hq).
+ *
+ * Two independent evaluations are provided: the dense O(T^2) definition (eqs. 2-3, summed
+ * over j <= i and normalised) and the H0/H1/H2 recurrence (eqs. 4-5), run token by token
+ * with full (unpacked) d_h x d_h second-order states.
+ *
+ * Layouts (all row-major, contiguous):
+ *   q [B][Hq][T][dh], k [B][Hkv][T][dh], v [B][Hkv][T][dv], y [B][Hq][T][dv]
+ *   group_id [Hq][dh] (values 1..G[h]), L [Hq][Gmax+1][Gmax+1], G [Hq]
+ *   states H0 [B][Hkv][dv+1], H1 [B][Hkv][dh][dv+1], H2 [B][Hkv][dh][dh][dv+1]
+ * Return value: 0 on success, -1 on bad arguments, -2 on allocation failure.
+ */
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* M = L L^T over the leading (G+1)x(G+1) block; L row-major with leading dimension ld. */
+static void gram_llt(const double* L, int G, int ld, double* M)
+{
+    for (int a = 0; a <= G; ++a)
+        for (int b = 0; b <= G; ++b) {
+            double acc = 0.0;
+            for (int m = 0; m <= G; ++m) acc += L[a * ld + m] * L[b * ld + m];
+            M[a * (G + 1) + b] = acc;
+        }
+}
+
+static int check_args(int B, int Hq, int Hkv, int T, int dh, int dv, const int* gid,
+                      const int* G, int Gmax)
+{
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || T < 0 || dh <= 0 || dv <= 0 || Gmax < 1) return -1;
+    if (Hq % Hkv != 0) return -1;
+    for (int h = 0; h < Hq; ++h) {
+        if (G[h] < 1 || G[h] > Gmax) return -1;
+        for (int r = 0; r < dh; ++r)
+            if (gid[h * dh + r] < 1 || gid[h * dh + r] > G[h]) return -1;
+    }
+    return 0;
+}
+
+/* kappa(q_i, k_j) for one head, every (i, j) pair, no causal mask: eqs. (2)-(3). */
+int oal_oracle_kappa(int Tq, int Tk, int dh, const double* q, const double* k,
+                     const int* gid, const double* L, int G, int Gmax, double eps,
+                     double* kappa)
+{
+    if (G < 1 || G > Gmax || dh <= 0) return -1;
+    double* M = (double*)malloc(sizeof(double) * (G + 1) * (G + 1));
+    double* sbar = (double*)malloc(sizeof(double) * (G + 1));
+    if (!M || !sbar) { free(M); free(sbar); return -2; }
+    gram_llt(L, G, Gmax + 1, M);
+    const double inv_sqrt_d = 1.0 / sqrt((double)dh);
+    for (int i = 0; i < Tq; ++i)
+        for (int j = 0; j < Tk; ++j) {
+            sbar[0] = 1.0;
+            for (int g = 1; g <= G; ++g) sbar[g] = 0.0;
+            for (int r = 0; r < dh; ++r)
+                sbar[gid[r]] += q[i * dh + r] * k[j * dh + r] * inv_sqrt_d;
+            double quad = 0.0;
+            for (int a = 0; a <= G; ++a)
+                for (int b = 0; b <= G; ++b) quad += sbar[a] * M[a * (G + 1) + b] * sbar[b];
+            kappa[i * Tk + j] = eps + quad;
+        }
+    free(M);
+    free(sbar);
+    return 0;
+}
+
+/* Dense causal form: yhat_i = sum_{j<=i} kappa_ij v_j / sum_{j<=i} kappa_ij.
+ * den (optional, [B][Hq][T]) receives the normaliser sum_{j<=i} kappa_ij. */
+int oal_oracle_dense(int B, int Hq, int Hkv, int T, int dh, int dv, const double* q,
+                     const double* k, const double* v, const int* gid, const double* L,
+                     const int* G, int Gmax, double eps, double* y, double* den)
+{
+    if (check_args(B, Hq, Hkv, T, dh, dv, gid, G, Gmax)) return -1;
+    const int group = Hq / Hkv;
+    int status = 0;
+#pragma omp parallel for schedule(dynamic) reduction(min : status)
+    for (int bh = 0; bh < B * Hq; ++bh) {
+        const int b = bh / Hq, h = bh % Hq, kv = h / group;
+        const double* qh = q + ((size_t)b * Hq + h) * T * dh;
+        const double* kh = k + ((size_t)b * Hkv + kv) * T * dh;
+        const double* vh = v + ((size_t)b * Hkv + kv) * T * dv;
+        double* yh = y + ((size_t)b * Hq + h) * T * dv;
+        double* kap = (double*)malloc(sizeof(double) * (T > 0 ? T : 1));
+        double* num = (double*)malloc(sizeof(double) * dv);
+        if (!kap || !num) { free(kap); free(num); status = -2; continue; }
+        for (int i = 0; i < T; ++i) {
+            /* one query row against keys 0..i */
+            oal_oracle_kappa(1, i + 1, dh, qh + (size_t)i * dh, kh, gid + h * dh,
+                             L + (size_t)h * (Gmax + 1) * (Gmax + 1), G[h], Gmax, eps, kap);
+            double z = 0.0;
+            for (int n = 0; n < dv; ++n) num[n] = 0.0;
+            for (int j = 0; j <= i; ++j) {
+                z += kap[j];
+                for (int n = 0; n < dv; ++n) num[n] += kap[j] * vh[(size_t)j * dv + n];
+            }
+            for (int n = 0; n < dv; ++n) yh[(size_t)i * dv + n] = num[n] / z;
+            if (den) den[((size_t)b * Hq + h) * T + i] = z;
+        }
+        free(kap);
+        free(num);
+    }
+    return status;
+}
+
+/* Recurrent form, eqs. (4)-(5), one token at a time.  The prefix state is kept per
+ * key/value head.  H*_in (all three or none) give the state of the tokens before this call;
+ * NULL starts from zero (a fresh prefill).  H*_out (all three or none) receive the state
+ * after all T tokens; they must not alias the inputs.  Each query head keeps a private
+ * copy of its key/value head's state, exactly as eq. (4) defines it per head; heads of one
+ * GQA group therefore end with identical states, and the first head of each group writes
+ * it out. */
+int oal_oracle_recurrent(int B, int Hq, int Hkv, int T, int dh, int dv, const double* q,
+                         const double* k, const double* v, const int* gid, const double* L,
+                         const int* G, int Gmax, double eps, const double* H0_in,
+                         const double* H1_in, const double* H2_in, double* H0_out,
+                         double* H1_out, double* H2_out, double* y)
+{
+    if (check_args(B, Hq, Hkv, T, dh, dv, gid, G, Gmax)) return -1;
+    const int have_in = (H0_in != NULL) && (H1_in != NULL) && (H2_in != NULL);
+    const int have_out = (H0_out != NULL) && (H1_out != NULL) && (H2_out != NULL);
+    if (!have_in && (H0_in || H1_in || H2_in)) return -1;
+    if (!have_out && (H0_out || H1_out || H2_out)) return -1;
+    const int group = Hq / Hkv;
+    const int w = dv + 1;
+    const size_t n0 = (size_t)w, n1 = (size_t)dh * w, n2 = (size_t)dh * dh * w;
+    int status = 0;
+#pragma omp parallel for schedule(dynamic) reduction(min : status)
+    for (int bh = 0; bh < B * Hq; ++bh) {
+        const int b = bh / Hq, h = bh % Hq, kv = h / group;
+        const double* qh = q + ((size_t)b * Hq + h) * T * dh;
+        const double* kh = k + ((size_t)b * Hkv + kv) * T * dh;
+        const double* vh = v + ((size_t)b * Hkv + kv) * T * dv;
+        double* yh = y + ((size_t)b * Hq + h) * T * dv;
+        const int Gh = G[h];
+        double* h0 = (double*)calloc(n0, sizeof(double));
+        double* h1 = (double*)calloc(n1, sizeof(double));
+        double* h2 = (double*)calloc(n2, sizeof(double));
+        double* M = (double*)malloc(sizeof(double) * (Gh + 1) * (Gh + 1));
+        double* bco = (double*)malloc(sizeof(double) * dh);
+        double* Cco = (double*)malloc(sizeof(double) * dh * dh);
+        double* vv = (double*)malloc(sizeof(double) * w);
+        double* u = (double*)malloc(sizeof(double) * w);
+        if (!h0 || !h1 || !h2 || !M || !bco || !Cco || !vv || !u) {
+            free(h0); free(h1); free(h2); free(M); free(bco); free(Cco); free(vv); free(u);
+            status = -2;
+            continue;
+        }
+        const size_t s = (size_t)b * Hkv + kv;
+        if (have_in) {
+            memcpy(h0, H0_in + s * n0, n0 * sizeof(double));
+            memcpy(h1, H1_in + s * n1, n1 * sizeof(double));
+            memcpy(h2, H2_in + s * n2, n2 * sizeof(double));
+        }
+        /* coefficients of eq. (5) from M = L L^T and the group ids */
+        gram_llt(L + (size_t)h * (Gmax + 1) * (Gmax + 1), Gh, Gmax + 1, M);
+        const int* g = gid + h * dh;
+        const double a = eps + M[0];
+        for (int r = 0; r < dh; ++r) bco[r] = 2.0 * M[0 * (Gh + 1) + g[r]];
+        for (int r = 0; r < dh; ++r)
+            for (int t = 0; t < dh; ++t) Cco[r * dh + t] = M[g[r] * (Gh + 1) + g[t]];
+        const double inv_sqrt_d = 1.0 / sqrt((double)dh), inv_d = 1.0 / (double)dh;
+
+        for (int i = 0; i < T; ++i) {
+            const double* ki = kh + (size_t)i * dh;
+            const double* qi = qh + (size_t)i * dh;
+            for (int n = 0; n < dv; ++n) vv[n] = vh[(size_t)i * dv + n];
+            vv[dv] = 1.0;
+            /* eq. (4): add token i to the prefix sums */
+            for (int n = 0; n < w; ++n) h0[n] += vv[n];
+            for (int r = 0; r < dh; ++r)
+                for (int n = 0; n < w; ++n) h1[(size_t)r * w + n] += ki[r] * vv[n];
+            for (int r = 0; r < dh; ++r)
+                for (int t = 0; t < dh; ++t) {
+                    const double kk = ki[r] * ki[t];
+                    double* row = h2 + ((size_t)r * dh + t) * w;
+                    for (int n = 0; n < w; ++n) row[n] += kk * vv[n];
+                }
+            /* eq. (5): read out and normalise */
+            for (int n = 0; n < w; ++n) u[n] = a * h0[n];
+            for (int r = 0; r < dh; ++r) {
+                const double c1 = inv_sqrt_d * bco[r] * qi[r];
+                for (int n = 0; n < w; ++n) u[n] += c1 * h1[(size_t)r * w + n];
+            }
+            for (int r = 0; r < dh; ++r)
+                for (int t = 0; t < dh; ++t) {
+                    const double c2 = inv_d * Cco[r * dh + t] * qi[r] * qi[t];
+                    const double* row = h2 + ((size_t)r * dh + t) * w;
+                    for (int n = 0; n < w; ++n) u[n] += c2 * row[n];
+                }
+            for (int n = 0; n < dv; ++n) yh[(size_t)i * dv + n] = u[n] / u[dv];
+        }
+        if (have_out && (h % group) == 0) {
+            memcpy(H0_out + s * n0, h0, n0 * sizeof(double));
+            memcpy(H1_out + s * n1, h1, n1 * sizeof(double));
+            memcpy(H2_out + s * n2, h2, n2 * sizeof(double));
+        }
+        free(h0); free(h1); free(h2); free(M); free(bco); free(Cco); free(vv); free(u);
+    }
+    return status;
+}
