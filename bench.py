@@ -1,0 +1,421 @@
+#!/usr/bin/env python
+"""Benchmark of the OAL causal grouped positive-quadratic attention library on B200.
+
+Headline (one JSON line on rank 0):
+  value  = causal PREFILL tokens/s on a Qwen2.5-0.5B-shaped layer: B=1, T=4096, 14 query /
+           2 key-value heads, d_h = dv = 64, bf16 inputs (seeded synthetic, same recipe as the
+           parity tests), chunk 128.  One step = one oal_prefill call = the whole prefill
+           hot path (coefficient expansion, chunk-state builder, readout with the intra-chunk
+           dense kernel).  Inputs are resident in HBM; L2 (126 MB) is flushed by writing a
+           256 MB buffer between steps, outside the timed events.
+  e2e    = the same metric through the public Python API with pinned HOST buffers: every
+           step copies q/k/v host->device, runs the prefill and copies yhat device->host.
+  decode = autoregressive decode tokens/s: batch 64, 4096-token context prefilled into the
+           packed fp32 states, then single-token steps (L2 flushed between steps).
+  roofline = the dominant prefill kernel's achieved rate from the library's CUDA-event trace
+           (recorded on the launching stream during the timed steps) against the measured
+           peak in MEASURED_PEAKS.json; likewise for the decode kernel against HBM.
+  cpu_baseline = the fp64 oracle (oracle/, plain C + OpenMP) on this host's cores, on a
+           bounded sample of the same workload (rank 0, N=1 only).
+
+Multi-GPU: one process per GPU (torchrun).  Every rank prefills its own replica of the
+layer (independent problems, no data-path collective): weak scaling.  Timing is the max over
+ranks of the summed per-step device time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "OAL causal prefill tokens/s and decode tokens/s on 1 B200; % of roofline"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+F, W = 2145, 65
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--chunk", type=int, default=128)
+    ap.add_argument("--decode-steps", type=int, default=256)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="config1", choices=["config1", "config3_16k",
+                                                              "config3_32k", "config3_64k"],
+                    help="prefill workload (config1 is the headline)")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu)], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        time.sleep(0.2)
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != gpus:
+        raise SystemExit(f"--gpus {gpus} but WORLD_SIZE={world}")
+    return world, rank, local
+
+
+def workload(name):
+    from positive_quadratic_b200 import inputs as I
+    if name == "config1":
+        return I.config1(), "qwen2.5-0.5b-layer-prefill B=1 T=4096 Hq=14 Hkv=2 d=64 bf16"
+    T = {"config3_16k": 16384, "config3_32k": 32768, "config3_64k": 65536}[name]
+    return I.config3(T), f"long-context prefill B=1 T={T} Hq=14 Hkv=2 d=64 bf16"
+
+
+def to_dev(p, dev, torch):
+    dt = torch.bfloat16 if p.dtype == "bf16" else torch.float32
+    t = lambda a, d=None: torch.from_numpy(np.ascontiguousarray(a)).to(dev, d)  # noqa: E731
+    return t(p.q, dt), t(p.k, dt), t(p.v, dt), t(p.group_id), t(p.L), t(p.G)
+
+
+def prefill_flops(B, T, Hq, Hkv):
+    """Algorithmic prefill work: the eq. (4) state update per key/value head plus the eq. (5)
+    readout per query head over D = 2145 packed features and dv + 1 = 65 columns."""
+    return 2.0 * B * T * F * W * (Hq + Hkv)
+
+
+def cpu_baseline(p, budget_s=12.0):
+    import oracle
+    tokens, t0, runs = 0, time.perf_counter(), 0
+    while True:
+        oracle.recurrent(p.q, p.k, p.v, p.group_id, p.L, p.G, p.eps)
+        runs += 1
+        tokens += p.q.shape[0] * p.q.shape[2]
+        el = time.perf_counter() - t0
+        if el >= budget_s or runs >= 3:
+            break
+    return {"value": tokens / el, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"fp64 oracle (H0/H1/H2 recurrence, OpenMP) on the full layer "
+                      f"B={p.q.shape[0]} T={p.q.shape[2]} Hq={p.q.shape[1]} x{runs} run(s), "
+                      f"{el:.1f} s", "seconds": el}
+
+
+def run_reference(args):
+    """The reference arm: the fp64 oracle timed on this host's cores (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    p, desc = workload(args.workload)
+    sample_T = 512
+    s = p.slice_tokens(0, sample_T)
+    for _ in range(args.warmup):
+        oracle.recurrent(s.q, s.k, s.v, s.group_id, s.L, s.G, s.eps)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.recurrent(s.q, s.k, s.v, s.group_id, s.L, s.G, s.eps)
+        times.append(time.perf_counter() - t0)
+    tot = sum(times)
+    value = args.steps * sample_T * s.q.shape[0] / tot
+    out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic", "impl": "reference",
+           "config": {"workload": desc, "sample": f"first {sample_T} tokens, all heads",
+                      "chunk": args.chunk},
+           "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.threads(),
+                            "kind": "oracle",
+                            "sample": f"fp64 oracle recurrence on the first {sample_T} tokens "
+                                      f"of the layer (all 14 heads) per step"},
+           "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    import torch.distributed as dist
+    from positive_quadratic_b200 import oal
+
+    world, rank, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=dev)
+    pk, pk_kind = peaks()
+    oal.lib()
+
+    p, desc = workload(args.workload)
+    B, Hq, T, _ = p.q.shape
+    Hkv = p.k.shape[1]
+    q, k, v, g, L, G = to_dev(p, dev, torch)
+    out, state = oal.prefill(q, k, v, g, L, G, p.eps, args.chunk)
+    ws = oal.empty_workspace(oal.prefill_workspace_bytes(
+        oal.make_shape(B, T, Hq, Hkv, args.chunk, oal.OAL_BF16)), dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def step():
+        oal.prefill(q, k, v, g, L, G, p.eps, args.chunk, out=out, state=state, workspace=ws)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+        flush.zero_()
+    torch.cuda.synchronize()
+    assert oal.device_error() == 0
+
+    # ---- timed prefill (device-resident inputs) ----
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    oal.profile_read()
+    oal.profile_enable(True)
+    barrier()
+    torch.cuda.synchronize()
+    n0 = oal.launch_count()
+    with ClockSampler(local) as clk:
+        for s0, s1 in evs:
+            s0.record(stream)
+            step()
+            s1.record(stream)
+            flush.zero_()
+        torch.cuda.synchronize()
+    n_launch = oal.launch_count() - n0
+    barrier()
+    oal.profile_enable(False)
+    prof = oal.profile_read()
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    total_ms = sum(step_ms)
+    tmax = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
+    total_ms = float(tmax.item())
+    value = world * args.steps * B * T / (total_ms / 1e3)
+
+    # roofline of the dominant prefill kernel
+    flops_state = 2.0 * B * T * F * W * Hkv
+    flops_read = 2.0 * B * T * F * W * Hq
+    dom = max(prof.items(), key=lambda kv: kv[1][1]) if prof else None
+    roof = None
+    if dom is not None:
+        name, (nl, ms) = dom
+        per = ms / nl
+        algo = flops_read if name.startswith("readout") else (
+            flops_state if name.startswith("state") else prefill_flops(B, T, Hq, Hkv))
+        tensor = name.endswith("_tc")
+        if tensor:
+            peak, unit, bound = pk["bf16_tflops"], "TFLOP/s", "tensor"
+        else:
+            # fp32 FMA on CUDA cores: 148 SMs x 128 lanes x 2 flop x max SM clock
+            peak, unit, bound = 148 * 128 * 2 * pk.get("sm_max_mhz", 1965.0) * 1e6 / 1e12, \
+                "TFLOP/s", "alu"
+        ach = algo / (per / 1e3) / 1e12
+        roof = {"bound": bound, "achieved": ach, "peak": peak, "unit": unit, "frac": ach / peak,
+                "traffic": None, "kernel": name, "avg_launch_ms": per,
+                "algorithmic_flop_per_launch": algo, "peak_kind": pk_kind,
+                "kernel_shares": {n: round(t / sum(x[1] for x in prof.values()), 4)
+                                  for n, (c, t) in prof.items()},
+                "whole_step_frac_of_bf16_peak": prefill_flops(B, T, Hq, Hkv) /
+                (total_ms / args.steps / 1e3) / 1e12 / pk["bf16_tflops"]}
+
+    # ---- e2e through the public API with pinned host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        hq = q.cpu().pin_memory()
+        hk = k.cpu().pin_memory()
+        hv = v.cpu().pin_memory()
+        bufs = oal.alloc_prefill_buffers(hq, hk, hv, g, L, G, args.chunk, device=dev)
+        hout = torch.empty(out.shape, dtype=torch.float32, pin_memory=True)
+        for _ in range(3):
+            oal.prefill_host(hq, hk, hv, g, L, G, p.eps, args.chunk, bufs, hout)
+            flush.zero_()
+        evs2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(args.steps)]
+        barrier()
+        torch.cuda.synchronize()
+        for s0, s1 in evs2:
+            s0.record(stream)
+            oal.prefill_host(hq, hk, hv, g, L, G, p.eps, args.chunk, bufs, hout)
+            s1.record(stream)
+            flush.zero_()
+        torch.cuda.synchronize()
+        e_ms = sum(a.elapsed_time(b) for a, b in evs2)
+        te = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": world * args.steps * B * T / (float(te.item()) / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": int(hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2),
+               "d2h_bytes_per_step": int(hout.numel() * 4)}
+
+    # ---- decode ----
+    decode = None
+    if not args.no_decode:
+        decode = run_decode(args, dev, torch, oal, pk, pk_kind, flush, world, barrier)
+
+    base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        base = cpu_baseline(p)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": desc, "chunk": args.chunk,
+                           "l2": "flushed between steps (256 MB write, outside timed events)",
+                           "parallelism": f"replicas x{world}"},
+                "roofline": roof, "e2e": e2e, "gpu_launches": int(n_launch),
+                "clocks": clk.summary(), "decode": decode, "cpu_baseline": base,
+                "step_ms_min": min(step_ms), "step_ms_median": statistics.median(step_ms)}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_decode(args, dev, torch, oal, pk, pk_kind, flush, world, barrier):
+    """batch 64, context 4096 prefilled (untimed), then args.decode_steps single-token steps."""
+    from positive_quadratic_b200 import inputs as I
+    nsteps = args.decode_steps
+    p = I.config4(batch=64, context=4096, steps=nsteps)
+    B, Hq, Ttot, _ = p.q.shape
+    Hkv = p.k.shape[1]
+    q, k, v, g, L, G = to_dev(p, dev, torch)
+    ctx = 4096
+    _, state = oal.prefill(q[:, :, :ctx].contiguous(), k[:, :, :ctx].contiguous(),
+                           v[:, :, :ctx].contiguous(), g, L, G, p.eps, args.chunk)
+    ws = oal.decode_workspace(B, Hq, Hkv, dev)
+    qs = [q[:, :, t:t + 1].contiguous() for t in range(ctx, Ttot)]
+    ks = [k[:, :, t:t + 1].contiguous() for t in range(ctx, Ttot)]
+    vs = [v[:, :, t:t + 1].contiguous() for t in range(ctx, Ttot)]
+    del q, k, v
+    out = torch.empty(B, Hq, 1, 64, dtype=torch.float32, device=dev)
+    state0 = state.clone()
+    stream = torch.cuda.current_stream()
+    for i in range(3):  # warm-up on a scratch copy of the state
+        oal.decode_step(qs[i], ks[i], vs[i], state0, ws, out=out)
+    torch.cuda.synchronize()
+    del state0
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(nsteps)]
+    oal.profile_read()
+    oal.profile_enable(True)
+    barrier()
+    torch.cuda.synchronize()
+    for i, (s0, s1) in enumerate(evs):
+        s0.record(stream)
+        oal.decode_step(qs[i], ks[i], vs[i], state, ws, out=out)
+        s1.record(stream)
+        flush.zero_()
+    torch.cuda.synchronize()
+    oal.profile_enable(False)
+    prof = oal.profile_read()
+    assert oal.device_error() == 0
+    ms = sum(a.elapsed_time(b) for a, b in evs)
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    state_bytes = 2.0 * B * Hkv * F * W * 4   # every packed row read and written once
+    io_bytes = B * (Hq + 2 * Hkv) * 64 * 2 + B * Hq * 64 * 4
+    kern = prof.get("decode")
+    roof = None
+    if kern:
+        per = kern[1] / kern[0]
+        gbs = (state_bytes + io_bytes) / (per / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": gbs / pk["hbm_gbs"], "frac_of_8tbs": gbs / 8000.0, "traffic": None,
+                "kernel": "decode", "avg_launch_ms": per, "peak_kind": pk_kind,
+                "algorithmic_bytes_per_launch": state_bytes + io_bytes}
+    return {"value": world * B * nsteps / (ms / 1e3), "unit": UNIT,
+            "ms_per_token_step": ms / nsteps, "batch": B, "context": 4096, "steps": nsteps,
+            "roofline": roof,
+            "workload": "decode batch 64, context 4096, Hq=14 Hkv=2 d=64 bf16 q/k/v, fp32 state"}
+
+
+if __name__ == "__main__":
+    main()

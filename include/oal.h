@@ -1,0 +1,171 @@
+/*
+ * oal.h -- C ABI of the B200 (sm_100a) library for OAL causal grouped positive-quadratic
+ * attention.
+ *
+ * What it computes.  "OAL: 按 QK 离群贡献分组的正二次注意力核" (reproduction note of arXiv
+ * 2610.13674), section 核心公式, equations in order of appearance:
+ *   (2) s_g = sum_{r in G_g} q_r k_r / sqrt(d_h),  sbar = [1, s_1, ..., s_G]
+ *   (3) kappa(q, k) = eps + sbar^T L L^T sbar > 0
+ *   (4) H0_i = sum_{j<=i} [v_j; 1],  H1_{i,r} = sum_{j<=i} k_{j,r} [v_j; 1],
+ *       H2_{i,rt} = sum_{j<=i} k_{j,r} k_{j,t} [v_j; 1]
+ *   (5) u_i = a H0_i + (1/sqrt(d_h)) sum_r b_r q_{i,r} H1_{i,r}
+ *             + (1/d_h) sum_{r,t} C_rt q_{i,r} q_{i,t} H2_{i,rt},   yhat_i = u_{i,1:dv}/u_{i,dv+1}
+ * i.e. yhat_i = sum_{j<=i} kappa(q_i,k_j) v_j / sum_{j<=i} kappa(q_i,k_j) (causal, j <= i
+ * inclusive).  The coefficients are a = eps + M_00, b_r = 2 M_{0,g(r)}, C_rt = M_{g(r),g(t)}
+ * with M = L L^T (the pages do not print them; this expansion is the one that makes (5) equal
+ * (3) summed over j).  The abstract of arXiv 2610.13674 states the linear-time evaluation in
+ * sequence length for a fixed head dimension that oal_prefill and oal_decode_step implement.
+ *
+ * Conventions for every entry point:
+ *  - All tensor arguments are DEVICE pointers to contiguous row-major arrays, allocated and
+ *    owned by the caller (for example through PyTorch).  The library allocates no device
+ *    memory and keeps no pointer after a call returns.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL = legacy
+ *    default stream).  A return of OAL_OK means the work was validated and enqueued.
+ *  - Return value: OAL_OK (0) or a negative oal_status.  Nothing aborts or throws.  Argument
+ *    errors are found on the host before anything is enqueued.  Errors that only the device
+ *    can see (a group id outside 1..G[h], G[h] outside 1..OAL_G_MAX, a bounded wait that ran
+ *    out) set a device-side error word instead; read and clear it with oal_device_error().
+ *  - Layouts: q [B][Hq][T][dh], k [B][Hkv][T][dh], v [B][Hkv][T][dv] in the element type of
+ *    oal_shape.dtype; out [B][Hq][T][dv] fp32.  Query head h reads key/value head
+ *    floor(h * Hkv / Hq) (grouped-query attention; Hq must be a multiple of Hkv).
+ *    group_id [Hq][dh] int32 with values 1..G[h]; G [Hq] int32 in 1..OAL_G_MAX;
+ *    L [Hq][OAL_G_MAX+1][OAL_G_MAX+1] fp32, of which the leading (G[h]+1)x(G[h]+1) block is
+ *    used as given (M = L L^T; L need not be triangular).
+ *  - Supported sizes: dh = dv = 64; Hq/Hkv <= 8; chunk in {64, 128, 256}; B, T >= 0 with
+ *    B*Hq*T < 2^31.  Pointers must be 16-byte aligned.  When B*T == 0 the q, k, v and out
+ *    pointers are not used and may be NULL.
+ */
+#ifndef OAL_H
+#define OAL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define OAL_ABI_VERSION 1
+#define OAL_HEAD_DIM 64
+#define OAL_VALUE_DIM 64
+#define OAL_G_MAX 8
+/* packed features of the prefix state: the upper triangle of qhat qhat^T, qhat = [q; 1] */
+#define OAL_FEATURES 2145
+#define OAL_FEATURES_PAD 2176
+
+typedef enum { OAL_F32 = 0, OAL_BF16 = 1 } oal_dtype;
+
+typedef enum {
+    OAL_OK = 0,
+    OAL_ERR_NULL = -1,        /* a required pointer is NULL */
+    OAL_ERR_SHAPE = -2,       /* inconsistent or out-of-range sizes */
+    OAL_ERR_UNSUPPORTED = -3, /* valid but unsupported (dh/dv != 64, chunk size, dtype) */
+    OAL_ERR_ALIGN = -4,       /* a pointer is not 16-byte aligned */
+    OAL_ERR_GROUPS = -5,      /* device: group id or G out of range (inputs were clamped) */
+    OAL_ERR_CUDA = -6,        /* a CUDA launch or runtime call failed */
+    OAL_ERR_TIMEOUT = -7,     /* device: a bounded wait gave up */
+    OAL_ERR_WORKSPACE = -8,   /* workspace NULL or smaller than the query function says */
+    OAL_ERR_STATE = -9        /* state buffer does not match the shape */
+} oal_status;
+
+/* Problem description shared by every call. */
+typedef struct {
+    int32_t B;     /* batch */
+    int32_t T;     /* tokens per sequence (oal_decode_step: ignored, one token) */
+    int32_t Hq;    /* query heads */
+    int32_t Hkv;   /* key/value heads; Hq % Hkv == 0 */
+    int32_t dh;    /* head dim of q and k (64) */
+    int32_t dv;    /* head dim of v (64) */
+    int32_t chunk; /* prefill chunk size C in {64, 128, 256}; ignored by decode and dense */
+    int32_t dtype; /* oal_dtype of q, k, v */
+} oal_shape;
+
+/* Size in bytes of the recurrent state buffer for `s` (B, Hq, Hkv used).
+ * Layout: a 256-byte header; then the readout coefficients of every query head,
+ * coef [Hq][OAL_FEATURES_PAD] fp32 (padded to 256 bytes); then, per (b, kv) in row-major
+ * order, Hv [OAL_FEATURES_PAD][dv] fp32 followed by z [OAL_FEATURES_PAD] fp32.  Row f of
+ * (Hv | z) is sum_j psi_f(k_j) [v_j; 1] over the tokens seen so far, where psi_f(k) =
+ * khat_r khat_t for the f-th pair (r <= t) of khat = [k; 1] (index 64 is the constant 1) in
+ * this packed order:
+ *   f in [0, 1792):     28 off-diagonal 8x8 blocks, (R, T) with R < T over the 8 blocks of 8
+ *                       dims in lexicographic order; f = 64*block + 8*a + b <-> (8R+a, 8T+b)
+ *   f in [1792, 2080):  8 diagonal blocks of 36 rows: (8R+a, 8R+b), a <= b, a-major
+ *   f in [2080, 2144):  (r, 64): sum_j k_{j,r} [v_j; 1]   (H1 of eq. (4))
+ *   f = 2144:           (64, 64): sum_j [v_j; 1]           (H0 of eq. (4))
+ *   f in [2145, 2176):  zero padding
+ * so rows with r, t < 64 hold H2_rt (= H2_tr) of eq. (4).  coef[h][f] is the readout weight
+ * of row f for head h: (r == t ? 1 : 2) * M_{g(r),g(t)} * s_r * s_t with g(64) = 0,
+ * s_r = 1/sqrt(dh) for r < 64, s_64 = 1, plus eps on f = 2144; u = sum_f coef[h][f] *
+ * qhat_r qhat_t * (Hv | z)[f].  The header holds magic 0x534C414F ("OALS"), the ABI version,
+ * B, Hq, Hkv, dh, dv, OAL_FEATURES_PAD (int32 each), the token count (int64 at byte 32) and
+ * eps (fp32 at byte 40).  The buffer is the resumable artifact of a sequence: copying it
+ * saves the sequence, copying it back resumes it. */
+int oal_state_bytes(const oal_shape* s, size_t* bytes);
+
+/* Scratch needed by oal_prefill for `s` (all fields used).  The contents need no
+ * initialisation and are meaningless after the call. */
+int oal_prefill_workspace_bytes(const oal_shape* s, size_t* bytes);
+
+/* Scratch needed by oal_decode_step for `s` (B, Hq, Hkv used).  It MUST be zero-filled once
+ * before the first decode call.  Its first 256-byte-aligned block holds one completion ticket
+ * per (b, kv) that every completed call returns to zero; the rest is per-call scratch. */
+int oal_decode_workspace_bytes(const oal_shape* s, size_t* bytes);
+
+/* Causal prefill of T tokens: writes out = yhat for every token (eqs. (2)-(5)) and fills
+ * `state` (oal_state_bytes) with the prefix state after the last token plus the readout
+ * coefficients, ready for oal_decode_step.  Chunked evaluation: within each chunk of C tokens
+ * the kernel kappa is evaluated densely (eqs. (2)-(3)); across chunks the exclusive prefix
+ * state of eq. (4) is built and read out with eq. (5).  Linear in T for fixed d_h.
+ * bf16 inputs run on tcgen05 tensor cores (fp32 accumulation); fp32 inputs run in fp32 on
+ * CUDA cores.  `workspace` must hold oal_prefill_workspace_bytes(s) bytes. */
+int oal_prefill(const void* q, const void* k, const void* v, const int32_t* group_id,
+                const float* L, const int32_t* G, float eps, float* out, void* state,
+                void* workspace, size_t workspace_bytes, const oal_shape* s, void* stream);
+
+/* One autoregressive step for every sequence of the batch: q [B][Hq][1][dh],
+ * k [B][Hkv][1][dh], v [B][Hkv][1][dv] (dtype of s).  Adds the new token to `state`
+ * (eq. (4), rank-one update of every packed row) and writes out [B][Hq][1][dv] = yhat of the
+ * new token (eq. (5), inclusive of it).  `state` must come from oal_prefill with the same
+ * B, Hq, Hkv.  Memory-bound: every state row is read and written once. */
+int oal_decode_step(const void* q, const void* k, const void* v, void* state, float* out,
+                    void* workspace, size_t workspace_bytes, const oal_shape* s,
+                    void* stream);
+
+/* The exact O(T^2) dense form (eqs. (2)-(3) summed over j <= i and normalised), for
+ * cross-checking and timing against the linear-time path.  Same arguments as oal_prefill
+ * without the state; `chunk` is ignored.  Computes in fp32 for both dtypes. */
+int oal_dense_ref_gpu(const void* q, const void* k, const void* v, const int32_t* group_id,
+                      const float* L, const int32_t* G, float eps, float* out,
+                      const oal_shape* s, void* stream);
+
+/* Reads the device-side error word (OAL_OK or a negative oal_status set by a kernel since
+ * the last read), synchronising `stream`, and clears it. */
+int oal_device_error(int* code, void* stream);
+
+/* Tracing.  Every kernel launch of the library is counted; while tracing is on, each launch
+ * also records a CUDA event pair on its own stream.  oal_profile_read waits for the recorded
+ * events, returns per-kernel totals (launches, summed device time) since the previous read,
+ * and forgets them.  Tracing costs two event records per launch; leave it off in production. */
+typedef struct {
+    char name[40];
+    int32_t launches;
+    double total_ms;
+} oal_kernel_stat;
+
+int oal_profile_enable(int on);
+int oal_profile_read(oal_kernel_stat* stats, int max_stats, int* n_stats);
+/* Kernels launched by this library since it was loaded (all devices, all streams). */
+unsigned long long oal_launch_count(void);
+
+/* Static description of a status code. */
+const char* oal_status_string(int status);
+
+/* OAL_ABI_VERSION of the loaded library. */
+int oal_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* OAL_H */

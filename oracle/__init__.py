@@ -54,7 +54,13 @@ def _load():
             lib.oal_oracle_recurrent.argtypes = [ctypes.c_int] * 6 + [_D, _D, _D, _I, _D, _I,
                                                                       ctypes.c_int,
                                                                       ctypes.c_double] + [_D] * 7
-            for f in (lib.oal_oracle_kappa, lib.oal_oracle_dense, lib.oal_oracle_recurrent):
+            lib.oal_oracle_dense_rows.argtypes = [ctypes.c_int] * 6 + [_D, _D, _D, _I, _D, _I,
+                                                                       ctypes.c_int,
+                                                                       ctypes.c_double,
+                                                                       ctypes.c_int, _I, _I, _I,
+                                                                       _D]
+            for f in (lib.oal_oracle_kappa, lib.oal_oracle_dense, lib.oal_oracle_recurrent,
+                      lib.oal_oracle_dense_rows):
                 f.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -115,6 +121,20 @@ def dense(q, k, v, group_id, L, G, eps, return_den: bool = False):
                                   float(eps), _d(y), _d(den))
     _check(rc, "dense")
     return (y, den) if return_den else y
+
+
+def dense_rows(q, k, v, group_id, L, G, eps, rows):
+    """Dense-definition outputs for selected (b, h, i) triples only -> [len(rows), dv]."""
+    q, k, v, group_id, L, G, (B, Hq, Hkv, T, dh, dv, Gmax) = _common(q, k, v, group_id, L, G)
+    rows = np.asarray(rows, dtype=np.int64).reshape(-1, 3)
+    rb, rh, ri = (_i32(rows[:, c]) for c in range(3))
+    y = np.empty((rows.shape[0], dv), np.float64)
+    rc = _load().oal_oracle_dense_rows(B, Hq, Hkv, T, dh, dv, _d(q), _d(k), _d(v),
+                                       group_id.ctypes.data_as(_I), _d(L), G.ctypes.data_as(_I),
+                                       Gmax, float(eps), rows.shape[0], rb.ctypes.data_as(_I),
+                                       rh.ctypes.data_as(_I), ri.ctypes.data_as(_I), _d(y))
+    _check(rc, "dense_rows")
+    return y
 
 
 class State:

@@ -224,3 +224,41 @@ int oal_oracle_recurrent(int B, int Hq, int Hkv, int T, int dh, int dv, const do
     }
     return status;
 }
+
+/* Dense causal form for selected outputs only: row n is (b = rows_b[n], h = rows_h[n],
+ * i = rows_i[n]); y [nrows][dv] receives yhat_i of that head.  Same definition as
+ * oal_oracle_dense, one row at a time, so single rows of very long sequences stay cheap. */
+int oal_oracle_dense_rows(int B, int Hq, int Hkv, int T, int dh, int dv, const double* q,
+                          const double* k, const double* v, const int* gid, const double* L,
+                          const int* G, int Gmax, double eps, int nrows, const int* rows_b,
+                          const int* rows_h, const int* rows_i, double* y)
+{
+    if (check_args(B, Hq, Hkv, T, dh, dv, gid, G, Gmax)) return -1;
+    for (int n = 0; n < nrows; ++n)
+        if (rows_b[n] < 0 || rows_b[n] >= B || rows_h[n] < 0 || rows_h[n] >= Hq ||
+            rows_i[n] < 0 || rows_i[n] >= T)
+            return -1;
+    const int group = Hq / Hkv;
+    int status = 0;
+#pragma omp parallel for schedule(dynamic) reduction(min : status)
+    for (int n = 0; n < nrows; ++n) {
+        const int b = rows_b[n], h = rows_h[n], i = rows_i[n], kv = h / group;
+        const double* qi = q + (((size_t)b * Hq + h) * T + i) * dh;
+        const double* kh = k + ((size_t)b * Hkv + kv) * T * dh;
+        const double* vh = v + ((size_t)b * Hkv + kv) * T * dv;
+        double* kap = (double*)malloc(sizeof(double) * (i + 1));
+        double* num = (double*)calloc(dv, sizeof(double));
+        if (!kap || !num) { free(kap); free(num); status = -2; continue; }
+        oal_oracle_kappa(1, i + 1, dh, qi, kh, gid + h * dh,
+                         L + (size_t)h * (Gmax + 1) * (Gmax + 1), G[h], Gmax, eps, kap);
+        double z = 0.0;
+        for (int j = 0; j <= i; ++j) {
+            z += kap[j];
+            for (int c = 0; c < dv; ++c) num[c] += kap[j] * vh[(size_t)j * dv + c];
+        }
+        for (int c = 0; c < dv; ++c) y[(size_t)n * dv + c] = num[c] / z;
+        free(kap);
+        free(num);
+    }
+    return status;
+}

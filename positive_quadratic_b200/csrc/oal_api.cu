@@ -1,0 +1,222 @@
+// oal_api.cu -- the extern "C" boundary declared in include/oal.h: argument validation on the
+// host, workspace layout, and dispatch to the kernels.  No device memory is allocated here.
+#include <cstring>
+
+#include "oal_common.cuh"
+#include "oal_kernels.cuh"
+
+using namespace oal;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// q, k, v, out: required and aligned only when there is at least one token to process.
+int check_io(const oal_shape* s, const void* q, const void* k, const void* v, const void* out)
+{
+    if ((long long)s->B * s->T == 0) return OAL_OK;
+    if (!q || !k || !v || !out) return OAL_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return OAL_ERR_ALIGN;
+    return OAL_OK;
+}
+
+int check_common(const oal_shape* s)
+{
+    if (!s) return OAL_ERR_NULL;
+    if (s->B < 0 || s->T < 0 || s->Hq < 1 || s->Hkv < 1 || s->Hq % s->Hkv != 0)
+        return OAL_ERR_SHAPE;
+    if (s->dh != OAL_HEAD_DIM || s->dv != OAL_VALUE_DIM) return OAL_ERR_UNSUPPORTED;
+    if (s->Hq / s->Hkv > kMaxGroup) return OAL_ERR_UNSUPPORTED;
+    if (s->dtype != OAL_F32 && s->dtype != OAL_BF16) return OAL_ERR_UNSUPPORTED;
+    const long long rows = (long long)s->B * s->Hq * (long long)(s->T > 0 ? s->T : 1);
+    if (rows >= (1LL << 31)) return OAL_ERR_SHAPE;
+    return OAL_OK;
+}
+
+int check_chunk(const oal_shape* s)
+{
+    return (s->chunk == 64 || s->chunk == 128 || s->chunk == 256) ? OAL_OK
+                                                                   : OAL_ERR_UNSUPPORTED;
+}
+
+size_t simt_chunk_state_bytes(const oal_shape* s)
+{
+    const size_t NC = s->T > 0 ? size_t((s->T + s->chunk - 1) / s->chunk) : 0;
+    return size_t(s->B) * s->Hkv * NC * kW * kFP * sizeof(float);
+}
+
+size_t decode_ticket_bytes(const oal_shape* s) { return align256(size_t(s->B) * s->Hkv * 4); }
+
+size_t decode_part_bytes(const oal_shape* s)
+{
+    return size_t(s->B) * s->Hkv * decode_slabs() * (s->Hq / s->Hkv) * kW * sizeof(float);
+}
+
+}  // namespace
+
+extern "C" {
+
+int oal_abi_version(void) { return OAL_ABI_VERSION; }
+
+const char* oal_status_string(int status)
+{
+    switch (status) {
+    case OAL_OK: return "ok";
+    case OAL_ERR_NULL: return "a required pointer is NULL";
+    case OAL_ERR_SHAPE: return "inconsistent or out-of-range sizes";
+    case OAL_ERR_UNSUPPORTED: return "unsupported size, chunk or dtype";
+    case OAL_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case OAL_ERR_GROUPS: return "group id or group count out of range (clamped on device)";
+    case OAL_ERR_CUDA: return "CUDA launch or runtime error";
+    case OAL_ERR_TIMEOUT: return "a bounded device wait gave up";
+    case OAL_ERR_WORKSPACE: return "workspace missing or too small";
+    case OAL_ERR_STATE: return "state buffer does not match the shape";
+    default: return "unknown status";
+    }
+}
+
+int oal_state_bytes(const oal_shape* s, size_t* bytes)
+{
+    const int rc = check_common(s);
+    if (rc) return rc;
+    if (!bytes) return OAL_ERR_NULL;
+    *bytes = state_bytes(s->B, s->Hq, s->Hkv);
+    return OAL_OK;
+}
+
+int oal_prefill_workspace_bytes(const oal_shape* s, size_t* bytes)
+{
+    int rc = check_common(s);
+    if (rc) return rc;
+    if ((rc = check_chunk(s))) return rc;
+    if (!bytes) return OAL_ERR_NULL;
+    *bytes = simt_chunk_state_bytes(s);
+    if (*bytes == 0) *bytes = 256;
+    return OAL_OK;
+}
+
+int oal_decode_workspace_bytes(const oal_shape* s, size_t* bytes)
+{
+    const int rc = check_common(s);
+    if (rc) return rc;
+    if (!bytes) return OAL_ERR_NULL;
+    *bytes = decode_ticket_bytes(s) + decode_part_bytes(s);
+    return OAL_OK;
+}
+
+int oal_prefill(const void* q, const void* k, const void* v, const int32_t* group_id,
+                const float* L, const int32_t* G, float eps, float* out, void* state,
+                void* workspace, size_t workspace_bytes, const oal_shape* s, void* stream)
+{
+    int rc = check_common(s);
+    if (rc) return rc;
+    if ((rc = check_chunk(s))) return rc;
+    if (!group_id || !L || !G || !state) return OAL_ERR_NULL;
+    if ((rc = check_io(s, q, k, v, out))) return rc;
+    if (!aligned16(state) || !aligned16(group_id) || !aligned16(L) || !aligned16(G))
+        return OAL_ERR_ALIGN;
+    size_t need = 0;
+    oal_prefill_workspace_bytes(s, &need);
+    if (!workspace || workspace_bytes < need) return OAL_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return OAL_ERR_ALIGN;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    rc = launch_prep(group_id, L, G, eps, state, s->B, s->Hq, s->Hkv, s->T, st);
+    if (rc) return rc;
+    if (s->B == 0) return OAL_OK;
+    return launch_prefill_simt(q, k, v, group_id, L, G, eps, out, state,
+                               static_cast<float*>(workspace), s->B, s->T, s->Hq, s->Hkv,
+                               s->chunk, s->dtype, st);
+}
+
+int oal_decode_step(const void* q, const void* k, const void* v, void* state, float* out,
+                    void* workspace, size_t workspace_bytes, const oal_shape* s, void* stream)
+{
+    int rc = check_common(s);
+    if (rc) return rc;
+    oal_shape one = *s;
+    one.T = 1;
+    if (!state) return OAL_ERR_NULL;
+    if ((rc = check_io(&one, q, k, v, out))) return rc;
+    if (!aligned16(state)) return OAL_ERR_ALIGN;
+    size_t need = 0;
+    oal_decode_workspace_bytes(s, &need);
+    if (!workspace || workspace_bytes < need) return OAL_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return OAL_ERR_ALIGN;
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    return launch_decode(q, k, v, state, out,
+                         reinterpret_cast<float*>(ws + decode_ticket_bytes(s)),
+                         reinterpret_cast<unsigned int*>(ws), s->B, s->Hq, s->Hkv, s->dtype,
+                         static_cast<cudaStream_t>(stream));
+}
+
+int oal_dense_ref_gpu(const void* q, const void* k, const void* v, const int32_t* group_id,
+                      const float* L, const int32_t* G, float eps, float* out,
+                      const oal_shape* s, void* stream)
+{
+    int rc = check_common(s);
+    if (rc) return rc;
+    if (!group_id || !L || !G) return OAL_ERR_NULL;
+    if ((rc = check_io(s, q, k, v, out))) return rc;
+    if (!aligned16(group_id) || !aligned16(L) || !aligned16(G)) return OAL_ERR_ALIGN;
+    if ((long long)s->B * s->T == 0) return OAL_OK;
+    return launch_dense(q, k, v, group_id, L, G, eps, out, s->B, s->T, s->Hq, s->Hkv, s->dtype,
+                        static_cast<cudaStream_t>(stream));
+}
+
+unsigned long long oal_launch_count(void) { return tracer().launches.load(); }
+
+int oal_profile_enable(int on)
+{
+    Tracer& t = tracer();
+    if (on) {
+        std::lock_guard<std::mutex> g(t.mu);
+        if (!tracer_fill_pool(t)) return OAL_ERR_CUDA;
+    }
+    t.enabled.store(on ? 1 : 0);
+    return OAL_OK;
+}
+
+int oal_profile_read(oal_kernel_stat* stats, int max_stats, int* n_stats)
+{
+    if (!n_stats || (max_stats > 0 && !stats)) return OAL_ERR_NULL;
+    Tracer& t = tracer();
+    std::vector<TraceRecord> recs;
+    {
+        std::lock_guard<std::mutex> g(t.mu);
+        recs.swap(t.records);
+    }
+    std::vector<cudaEvent_t> back;
+    int n = 0, rc = OAL_OK;
+    for (const TraceRecord& r : recs) {
+        float ms = 0.f;
+        if (cudaEventSynchronize(r.stop) != cudaSuccess ||
+            cudaEventElapsedTime(&ms, r.start, r.stop) != cudaSuccess)
+            rc = OAL_ERR_CUDA;
+        back.push_back(r.start);
+        back.push_back(r.stop);
+        int i = 0;
+        while (i < n && std::strncmp(stats[i].name, r.name, sizeof(stats[i].name)) != 0) ++i;
+        if (i == n) {
+            if (n == max_stats) continue;
+            std::memset(&stats[n], 0, sizeof(stats[n]));
+            std::strncpy(stats[n].name, r.name, sizeof(stats[n].name) - 1);
+            ++n;
+        }
+        stats[i].launches += 1;
+        stats[i].total_ms += ms;
+    }
+    {
+        std::lock_guard<std::mutex> g(t.mu);
+        t.pool.insert(t.pool.end(), back.begin(), back.end());
+    }
+    *n_stats = n;
+    return rc;
+}
+
+int oal_device_error(int* code, void* stream)
+{
+    if (!code) return OAL_ERR_NULL;
+    return read_device_error(code, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

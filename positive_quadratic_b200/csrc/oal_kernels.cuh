@@ -1,0 +1,30 @@
+// oal_kernels.cuh -- internal launchers behind the C ABI (not part of the public header).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace oal {
+
+int launch_prep(const int32_t* gid, const float* L, const int32_t* G, float eps, void* state,
+                int B, int Hq, int Hkv, long long tokens, cudaStream_t st);
+
+int launch_prefill_simt(const void* q, const void* k, const void* v, const int32_t* gid,
+                        const float* L, const int32_t* G, float eps, float* out, void* state,
+                        float* Hc, int B, int T, int Hq, int Hkv, int C, int dtype,
+                        cudaStream_t st);
+
+int launch_dense(const void* q, const void* k, const void* v, const int32_t* gid, const float* L,
+                 const int32_t* G, float eps, float* out, int B, int T, int Hq, int Hkv,
+                 int dtype, cudaStream_t st);
+
+int decode_slabs();
+
+int launch_decode(const void* q, const void* k, const void* v, void* state, float* out,
+                  float* part, unsigned int* tickets, int B, int Hq, int Hkv, int dtype,
+                  cudaStream_t st);
+
+int read_device_error(int* code, cudaStream_t st);
+
+}  // namespace oal

@@ -1,0 +1,5 @@
+// oal_lib.cu -- the whole library as one translation unit, so that device symbols shared by
+// all kernels (the error word) exist exactly once without relocatable device code.
+#include "oal_common.cuh"
+#include "oal_simt.cu"
+#include "oal_api.cu"

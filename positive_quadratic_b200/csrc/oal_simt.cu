@@ -1,0 +1,613 @@
+// oal_simt.cu -- CUDA-core kernels of the OAL library: coefficient expansion, the fp32
+// chunked prefill (state builder + readout with the intra-chunk dense kernel), the O(T^2)
+// dense form, and the memory-bound decode step.
+//
+// Equations cited are those of "OAL: 按 QK 离群贡献分组的正二次注意力核" (reproduction note of
+// arXiv 2610.13674), section 核心公式, numbered in order of appearance: (2) grouped score,
+// (3) kernel kappa, (4) prefix states H0/H1/H2, (5) readout.  The packed feature map that
+// merges H0/H1/H2 into one state is described in oal_common.cuh.
+#include "oal_common.cuh"
+#include "oal_kernels.cuh"
+
+namespace oal {
+
+// ------------------------------------------------------------------------------------------
+// a1: coefficient expansion.  M = L L^T (fp64), then the packed readout coefficients
+// Cp_f (oal_common.cuh) per query head, written into the state buffer's coefficient table;
+// block 0 also writes the state header.  Group ids and G are validated; out-of-range values
+// raise OAL_ERR_GROUPS and are clamped so that nothing reads outside M.
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) prep_kernel(const int32_t* __restrict__ gid,
+                                                   const float* __restrict__ L,
+                                                   const int32_t* __restrict__ G, float eps,
+                                                   unsigned char* __restrict__ state, int B,
+                                                   int Hq, int Hkv, long long tokens)
+{
+    const int h = blockIdx.x, tid = threadIdx.x;
+    __shared__ double M[kGM1][kGM1];
+    __shared__ int g[kDA];
+    __shared__ int sG;
+    if (tid == 0) {
+        int Gh = G[h];
+        if (Gh < 1 || Gh > kGMax) {
+            raise_error(OAL_ERR_GROUPS);
+            Gh = Gh < 1 ? 1 : kGMax;
+        }
+        sG = Gh;
+    }
+    __syncthreads();
+    const int Gh = sG;
+    if (tid < kD) {
+        int x = gid[h * kD + tid];
+        if (x < 1 || x > Gh) {
+            raise_error(OAL_ERR_GROUPS);
+            x = x < 1 ? 1 : Gh;
+        }
+        g[tid] = x;
+    } else if (tid < kDA) {
+        g[tid] = 0;  // the constant slot (index 64) belongs to sbar_0; 65 is padding
+    }
+    if (tid < kGM1 * kGM1) {
+        const int a = tid / kGM1, c = tid % kGM1;
+        double acc = 0.0;
+        if (a <= Gh && c <= Gh) {
+            const float* Lh = L + size_t(h) * kGM1 * kGM1;
+            for (int m = 0; m <= Gh; ++m) acc += double(Lh[a * kGM1 + m]) * double(Lh[c * kGM1 + m]);
+        }
+        M[a][c] = acc;
+    }
+    __syncthreads();
+    float* coef = reinterpret_cast<float*>(state + kHeaderBytes) + size_t(h) * kFP;
+    for (int f = tid; f < kFP; f += blockDim.x) {
+        double val = 0.0;
+        if (f < kF) {
+            const RT rt = feature_rt(f);
+            const double sr = rt.r < kD ? 0.125 : 1.0, st = rt.t < kD ? 0.125 : 1.0;
+            val = (rt.r == rt.t ? 1.0 : 2.0) * M[g[rt.r]][g[rt.t]] * sr * st;
+            if (f == kConstRow) val += double(eps);
+        }
+        coef[f] = float(val);
+    }
+    if (h == 0 && tid == 0) {
+        StateHeader* hd = reinterpret_cast<StateHeader*>(state);
+        hd->magic = kStateMagic;
+        hd->abi = OAL_ABI_VERSION;
+        hd->B = B;
+        hd->Hq = Hq;
+        hd->Hkv = Hkv;
+        hd->dh = kD;
+        hd->dv = kDV;
+        hd->feat_pad = kFP;
+        hd->tokens = tokens;
+        hd->eps = eps;
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// a5-a7 (fp32 path): chunk states.  One block owns 64 packed rows of one (b, kv) state and
+// walks the chunks in order.  Before adding chunk c it stores the exclusive prefix
+// S_c = sum_{j < cC} psi(k_j) [v_j; 1] (eq. (4)) to Hc[(bkv*NC + c)][n][f] (fp32, column
+// major); after the last chunk it writes the inclusive state into the state buffer.
+// ------------------------------------------------------------------------------------------
+template <typename Tin>
+__global__ void __launch_bounds__(256) state_simt_kernel(const Tin* __restrict__ k,
+                                                         const Tin* __restrict__ v, int T,
+                                                         int C, int NC, float* __restrict__ Hc,
+                                                         float* __restrict__ body)
+{
+    const int slab = blockIdx.x, bkv = blockIdx.y;
+    const int tid = threadIdx.x, fi = tid & 63, cg = tid >> 6;
+    const int f = slab * 64 + fi;
+    const RT rt = feature_rt(f);
+    __shared__ float ks[64][kDA + 1];
+    __shared__ float vs[64][kW];
+    const Tin* kb = k + size_t(bkv) * T * kD;
+    const Tin* vb = v + size_t(bkv) * T * kDV;
+    float run[17], acc[17];
+#pragma unroll
+    for (int u = 0; u < 17; ++u) run[u] = 0.f;
+    for (int c = 0; c < NC; ++c) {
+        if (Hc) {
+            float* dst = Hc + (size_t(bkv) * NC + c) * kW * kFP;
+#pragma unroll
+            for (int u = 0; u < 17; ++u) {
+                const int n = cg + 4 * u;
+                if (n < kW) dst[size_t(n) * kFP + f] = run[u];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 17; ++u) acc[u] = 0.f;
+        const int t0 = c * C, t1 = min(t0 + C, T);
+        for (int s0 = t0; s0 < t1; s0 += 64) {
+            for (int e = tid; e < 64 * kD; e += 256) {
+                const int j = e / kD, r = e % kD, tok = s0 + j;
+                ks[j][r] = tok < t1 ? to_f32(kb[size_t(tok) * kD + r]) : 0.f;
+                vs[j][r] = tok < t1 ? to_f32(vb[size_t(tok) * kDV + r]) : 0.f;
+            }
+            if (tid < 64) {
+                const bool ok = s0 + tid < t1;
+                ks[tid][kD] = ok ? 1.f : 0.f;
+                ks[tid][kD + 1] = 0.f;
+                vs[tid][kDV] = ok ? 1.f : 0.f;
+            }
+            __syncthreads();
+            for (int j = 0; j < 64; ++j) {
+                const float psi = ks[j][rt.r] * ks[j][rt.t];
+#pragma unroll
+                for (int u = 0; u < 17; ++u) {
+                    const int n = cg + 4 * u;
+                    if (n < kW) acc[u] = fmaf(psi, vs[j][n], acc[u]);
+                }
+            }
+            __syncthreads();
+        }
+#pragma unroll
+        for (int u = 0; u < 17; ++u) run[u] += acc[u];
+    }
+    float* unit = body + size_t(bkv) * kFP * kW;
+#pragma unroll
+    for (int u = 0; u < 17; ++u) {
+        const int n = cg + 4 * u;
+        if (n < kDV) unit[size_t(f) * kDV + n] = run[u];
+        else if (n == kDV) unit[size_t(kFP) * kDV + f] = run[u];
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// a8-a10 (fp32 path) and a12: readout of 64 query rows of one (b, h).
+// inter (prefill only): u_i += phi(q_i)^T S_c with phi_f(q) = Cp_f qhat_r qhat_t (eq. (5));
+// intra: u_i += sum_j kappa(q_i, k_j) [v_j; 1] over j in [j0, i] with kappa from eqs.
+// (2)-(3) (j0 = start of the chunk for prefill, 0 for the dense form); then
+// yhat_i = u_i[0:64] / u_i[64].
+// ------------------------------------------------------------------------------------------
+struct ReadoutSmem {
+    float qs[64][kDA + 1];
+    float ps[64][65];
+    union {
+        float hs[kW][64];
+        struct {
+            float ks[64][kD + 1];
+            float vs[64][kW];
+        } kv;
+    } u;
+    float Ms[kGM1][kGM1];
+    int gperm[kD];
+    int gstart[kGM1 + 1];
+    int G;
+};
+
+template <typename Tin, bool kDense>
+__global__ void __launch_bounds__(256) readout_simt_kernel(
+    const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
+    const int32_t* __restrict__ gid, const float* __restrict__ L, const int32_t* __restrict__ G,
+    float eps, const float* __restrict__ coef, const float* __restrict__ Hc,
+    float* __restrict__ out, int Hq, int Hkv, int T, int C, int NC)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    ReadoutSmem& sm = *reinterpret_cast<ReadoutSmem*>(smem_raw);
+    const int tile = blockIdx.x, bh = blockIdx.y;
+    const int b = bh / Hq, h = bh % Hq, kv = h / (Hq / Hkv), bkv = b * Hkv + kv;
+    const int i0 = tile * 64;
+    const int tid = threadIdx.x, ri = tid & 63, cg = tid >> 6;
+    const Tin* qb = q + size_t(bh) * T * kD;
+    const Tin* kb = k + size_t(bkv) * T * kD;
+    const Tin* vb = v + size_t(bkv) * T * kDV;
+
+    for (int e = tid; e < 64 * kD; e += 256) {
+        const int j = e / kD, r = e % kD;
+        sm.qs[j][r] = i0 + j < T ? to_f32(qb[size_t(i0 + j) * kD + r]) : 0.f;
+    }
+    if (tid < 64) {
+        sm.qs[tid][kD] = 1.f;
+        sm.qs[tid][kD + 1] = 0.f;
+    }
+    if (tid == 0) {
+        int Gh = G[h];
+        if (Gh < 1 || Gh > kGMax) {
+            raise_error(OAL_ERR_GROUPS);
+            Gh = Gh < 1 ? 1 : kGMax;
+        }
+        sm.G = Gh;
+        // dims sorted by group (counting sort), so each s_g is a contiguous run
+        int cnt[kGM1 + 1];
+        for (int g = 0; g <= kGM1; ++g) cnt[g] = 0;
+        for (int r = 0; r < kD; ++r) {
+            int x = gid[h * kD + r];
+            if (x < 1 || x > Gh) {
+                raise_error(OAL_ERR_GROUPS);
+                x = x < 1 ? 1 : Gh;
+            }
+            cnt[x + 1]++;
+        }
+        for (int g = 1; g <= kGM1; ++g) cnt[g] += cnt[g - 1];
+        for (int g = 0; g <= kGM1; ++g) sm.gstart[g] = cnt[g];
+        for (int r = 0; r < kD; ++r) {
+            int x = gid[h * kD + r];
+            x = x < 1 ? 1 : (x > Gh ? Gh : x);
+            sm.gperm[cnt[x]++] = r;
+        }
+    }
+    __syncthreads();
+    const int Gh = sm.G;
+    if (tid < kGM1 * kGM1) {
+        const int a = tid / kGM1, c = tid % kGM1;
+        float acc = 0.f;
+        if (a <= Gh && c <= Gh) {
+            const float* Lh = L + size_t(h) * kGM1 * kGM1;
+            for (int m = 0; m <= Gh; ++m) acc = fmaf(Lh[a * kGM1 + m], Lh[c * kGM1 + m], acc);
+        }
+        sm.Ms[a][c] = acc;
+    }
+    __syncthreads();
+
+    float acc[17];
+#pragma unroll
+    for (int u = 0; u < 17; ++u) acc[u] = 0.f;
+
+    const int c = i0 / C;
+    if (!kDense && c > 0) {
+        const float* Hs = Hc + (size_t(bkv) * NC + c) * kW * kFP;
+        const float* cf = coef + size_t(h) * kFP;
+        for (int slab = 0; slab < kFP / 64; ++slab) {
+            const int f = slab * 64 + ri;
+            for (int n = cg; n < kW; n += 4) sm.u.hs[n][ri] = Hs[size_t(n) * kFP + f];
+            const RT rt = feature_rt(f);
+            const float cfv = cf[f];
+            for (int row = cg; row < 64; row += 4)
+                sm.ps[row][ri] = cfv * sm.qs[row][rt.r] * sm.qs[row][rt.t];
+            __syncthreads();
+            for (int ff = 0; ff < 64; ++ff) {
+                const float p = sm.ps[ri][ff];
+#pragma unroll
+                for (int u = 0; u < 17; ++u) {
+                    const int n = cg + 4 * u;
+                    if (n < kW) acc[u] = fmaf(p, sm.u.hs[n][ff], acc[u]);
+                }
+            }
+            __syncthreads();
+        }
+    }
+
+    const int j0 = kDense ? 0 : c * C;
+    const int j1 = min(i0 + 64, T);
+    for (int kb0 = j0; kb0 < j1; kb0 += 64) {
+        for (int e = tid; e < 64 * kD; e += 256) {
+            const int j = e / kD, r = e % kD, tok = kb0 + j;
+            sm.u.kv.ks[j][r] = tok < T ? to_f32(kb[size_t(tok) * kD + r]) : 0.f;
+            sm.u.kv.vs[j][r] = tok < T ? to_f32(vb[size_t(tok) * kDV + r]) : 0.f;
+        }
+        if (tid < 64) sm.u.kv.vs[tid][kDV] = 1.f;
+        __syncthreads();
+        const int i = i0 + ri;
+        for (int key = cg; key < 64; key += 4) {
+            const int j = kb0 + key;
+            float kap = 0.f;
+            if (j <= i && j < T && i < T) {
+                float sb[kGM1];
+                sb[0] = 1.f;
+#pragma unroll
+                for (int g = 1; g < kGM1; ++g) {
+                    float s = 0.f;
+                    if (g <= Gh) {
+                        for (int e = sm.gstart[g]; e < sm.gstart[g + 1]; ++e) {
+                            const int r = sm.gperm[e];
+                            s = fmaf(sm.qs[ri][r], sm.u.kv.ks[key][r], s);
+                        }
+                    }
+                    sb[g] = s * 0.125f;
+                }
+                float quad = 0.f;
+#pragma unroll
+                for (int a = 0; a < kGM1; ++a) {
+                    float row = 0.f;
+#pragma unroll
+                    for (int bb = 0; bb < kGM1; ++bb) row = fmaf(sm.Ms[a][bb], sb[bb], row);
+                    quad = fmaf(sb[a], row, quad);
+                }
+                kap = eps + quad;
+            }
+            sm.ps[ri][key] = kap;
+        }
+        __syncthreads();
+        for (int key = 0; key < 64; ++key) {
+            const float p = sm.ps[ri][key];
+#pragma unroll
+            for (int u = 0; u < 17; ++u) {
+                const int n = cg + 4 * u;
+                if (n < kW) acc[u] = fmaf(p, sm.u.kv.vs[key][n], acc[u]);
+            }
+        }
+        __syncthreads();
+    }
+
+    // normalise: the denominator u[64] lives in the cg == 0 thread (u index 16)
+#pragma unroll
+    for (int u = 0; u < 17; ++u) {
+        const int n = cg + 4 * u;
+        if (n < kW) sm.ps[ri][n] = acc[u];
+    }
+    __syncthreads();
+    const int i = i0 + ri;
+    if (i < T) {
+        const float den = sm.ps[ri][kDV];
+        float* o = out + (size_t(bh) * T + i) * kDV;
+        for (int n = cg; n < kDV; n += 4) o[n] = sm.ps[ri][n] / den;
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// a11: decode step.  Block (slab, bkv) streams 128 packed rows of one (b, kv) state once:
+// S_f += psi_f(k) [v; 1] (eq. (4) with one new token), then accumulates
+// u_h += phi_{h,f}(q_h) S_f for the Hq/Hkv query heads of that kv head (eq. (5)).  Row data
+// moves as 128-bit loads and stores (a half warp per 256-byte row).  Per-block partial u go
+// to the workspace; the last block of a (b, kv) (atomic ticket) sums them, writes yhat and
+// re-arms the ticket.
+// ------------------------------------------------------------------------------------------
+constexpr int kDecRows = 128;
+
+template <typename Tin>
+__global__ void __launch_bounds__(256) decode_kernel(const Tin* __restrict__ q,
+                                                     const Tin* __restrict__ k,
+                                                     const Tin* __restrict__ v,
+                                                     unsigned char* __restrict__ state,
+                                                     float* __restrict__ out,
+                                                     float* __restrict__ part,
+                                                     unsigned int* __restrict__ tickets, int Hq,
+                                                     int Hkv)
+{
+    const int slab = blockIdx.x, bkv = blockIdx.y, nslab = gridDim.x;
+    const int b = bkv / Hkv, kv = bkv % Hkv, grp = Hq / Hkv, h0 = kv * grp;
+    const int tid = threadIdx.x, lane4 = tid & 15, rsub = tid >> 4, warp = tid >> 5;
+    const float* coef = reinterpret_cast<const float*>(state + kHeaderBytes);
+    float* unit = reinterpret_cast<float*>(state + kHeaderBytes + coef_bytes(Hq)) +
+                  size_t(bkv) * kFP * kW;
+    float* Hv = unit;
+    float* z = unit + size_t(kFP) * kDV;
+
+    __shared__ __align__(16) float vh[kW + 3];
+    __shared__ float kh[kDA];
+    __shared__ float qh[kMaxGroup][kDA];
+    __shared__ float phis[kDecRows][kMaxGroup + 1];
+    __shared__ float psis[kDecRows];
+    __shared__ float red[8][kMaxGroup][kDV];
+    __shared__ float redz[8][kMaxGroup];
+    __shared__ float ufin[kMaxGroup][kW];
+    __shared__ int s_last;
+
+    if (tid < kD) {
+        kh[tid] = to_f32(k[size_t(bkv) * kD + tid]);
+        vh[tid] = to_f32(v[size_t(bkv) * kDV + tid]);
+    } else if (tid == kD) {
+        kh[kD] = 1.f;
+        kh[kD + 1] = 0.f;
+        vh[kDV] = 1.f;
+    }
+    for (int e = tid; e < grp * kDA; e += 256) {
+        const int g = e / kDA, r = e % kDA;
+        qh[g][r] = r < kD ? to_f32(q[(size_t(b) * Hq + h0 + g) * kD + r]) : (r == kD ? 1.f : 0.f);
+    }
+    __syncthreads();
+    const int f0 = slab * kDecRows;
+    const int nrows = min(kDecRows, kF - f0);
+    for (int row = tid; row < nrows; row += 256) {
+        const int f = f0 + row;
+        const RT rt = feature_rt(f);
+        psis[row] = kh[rt.r] * kh[rt.t];
+        for (int g = 0; g < grp; ++g)
+            phis[row][g] = coef[size_t(h0 + g) * kFP + f] * qh[g][rt.r] * qh[g][rt.t];
+    }
+    __syncthreads();
+
+    float acc[kMaxGroup][4];
+#pragma unroll
+    for (int g = 0; g < kMaxGroup; ++g) acc[g][0] = acc[g][1] = acc[g][2] = acc[g][3] = 0.f;
+    const float4 v4 = *reinterpret_cast<const float4*>(&vh[lane4 * 4]);
+#pragma unroll 4
+    for (int row = rsub; row < nrows; row += 16) {
+        float4* p = reinterpret_cast<float4*>(Hv + size_t(f0 + row) * kDV) + lane4;
+        float4 hv = *p;
+        const float psi = psis[row];
+        hv.x = fmaf(psi, v4.x, hv.x);
+        hv.y = fmaf(psi, v4.y, hv.y);
+        hv.z = fmaf(psi, v4.z, hv.z);
+        hv.w = fmaf(psi, v4.w, hv.w);
+        *p = hv;
+#pragma unroll
+        for (int g = 0; g < kMaxGroup; ++g) {
+            if (g < grp) {
+                const float ph = phis[row][g];
+                acc[g][0] = fmaf(ph, hv.x, acc[g][0]);
+                acc[g][1] = fmaf(ph, hv.y, acc[g][1]);
+                acc[g][2] = fmaf(ph, hv.z, acc[g][2]);
+                acc[g][3] = fmaf(ph, hv.w, acc[g][3]);
+            }
+        }
+    }
+    float accz[kMaxGroup];
+#pragma unroll
+    for (int g = 0; g < kMaxGroup; ++g) accz[g] = 0.f;
+    if (tid < nrows) {
+        const float zz = z[f0 + tid] + psis[tid];
+        z[f0 + tid] = zz;
+#pragma unroll
+        for (int g = 0; g < kMaxGroup; ++g)
+            if (g < grp) accz[g] = phis[tid][g] * zz;
+    }
+    // reduce: the two half-warps of a warp hold the same columns
+#pragma unroll
+    for (int g = 0; g < kMaxGroup; ++g) {
+        if (g < grp) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[g][c] += __shfl_xor_sync(0xffffffffu, acc[g][c], 16);
+            float zz = accz[g];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) zz += __shfl_xor_sync(0xffffffffu, zz, o);
+            if ((tid & 31) < 16) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) red[warp][g][lane4 * 4 + c] = acc[g][c];
+            }
+            if ((tid & 31) == 0) redz[warp][g] = zz;
+        }
+    }
+    __syncthreads();
+    float* mypart = part + (size_t(bkv) * nslab + slab) * grp * kW;
+    for (int e = tid; e < grp * kW; e += 256) {
+        const int g = e / kW, n = e % kW;
+        float s = 0.f;
+        for (int w = 0; w < 8; ++w) s += n < kDV ? red[w][g][n] : redz[w][g];
+        mypart[e] = s;
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        const unsigned int prev = atomicAdd(&tickets[bkv], 1u);
+        s_last = (prev == unsigned(nslab - 1));
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    const float* allpart = part + size_t(bkv) * nslab * grp * kW;
+    for (int e = tid; e < grp * kW; e += 256) {
+        float s = 0.f;
+        for (int sl = 0; sl < nslab; ++sl) s += __ldcg(allpart + size_t(sl) * grp * kW + e);
+        ufin[e / kW][e % kW] = s;
+    }
+    __syncthreads();
+    for (int e = tid; e < grp * kDV; e += 256) {
+        const int g = e / kDV, n = e % kDV;
+        out[(size_t(b) * Hq + h0 + g) * kDV + n] = ufin[g][n] / ufin[g][kDV];
+    }
+    if (tid == 0) {
+        tickets[bkv] = 0u;
+        if (bkv == 0) reinterpret_cast<StateHeader*>(state)->tokens += 1;
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// launchers
+// ------------------------------------------------------------------------------------------
+int launch_prep(const int32_t* gid, const float* L, const int32_t* G, float eps, void* state,
+                int B, int Hq, int Hkv, long long tokens, cudaStream_t st)
+{
+    LaunchScope ls("prep", st);
+    prep_kernel<<<Hq, 256, 0, st>>>(gid, L, G, eps, static_cast<unsigned char*>(state), B, Hq,
+                                    Hkv, tokens);
+    OAL_LAUNCH_CHECK();
+    return OAL_OK;
+}
+
+template <typename Tin>
+static int launch_prefill_simt_t(const Tin* q, const Tin* k, const Tin* v,
+                                 const int32_t* gid, const float* L, const int32_t* G,
+                                 float eps, float* out, void* state, float* Hc, int B, int T,
+                                 int Hq, int Hkv, int C, cudaStream_t st)
+{
+    const int NC = (T + C - 1) / C;
+    float* coef = reinterpret_cast<float*>(static_cast<unsigned char*>(state) + kHeaderBytes);
+    float* body = reinterpret_cast<float*>(static_cast<unsigned char*>(state) + kHeaderBytes +
+                                           coef_bytes(Hq));
+    {
+        LaunchScope ls("state_simt", st);
+        state_simt_kernel<Tin><<<dim3(kFP / 64, B * Hkv), 256, 0, st>>>(k, v, T, C, NC, Hc,
+                                                                         body);
+        OAL_LAUNCH_CHECK();
+    }
+    if (T == 0) return OAL_OK;
+    const size_t smem = sizeof(ReadoutSmem);
+    auto kern = readout_simt_kernel<Tin, false>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+        cudaSuccess)
+        return OAL_ERR_CUDA;
+    LaunchScope ls("readout_simt", st);
+    kern<<<dim3((T + 63) / 64, B * Hq), 256, smem, st>>>(q, k, v, gid, L, G, eps, coef, Hc, out,
+                                                         Hq, Hkv, T, C, NC);
+    OAL_LAUNCH_CHECK();
+    return OAL_OK;
+}
+
+int launch_prefill_simt(const void* q, const void* k, const void* v, const int32_t* gid,
+                        const float* L, const int32_t* G, float eps, float* out, void* state,
+                        float* Hc, int B, int T, int Hq, int Hkv, int C, int dtype,
+                        cudaStream_t st)
+{
+    if (dtype == OAL_BF16)
+        return launch_prefill_simt_t(static_cast<const __nv_bfloat16*>(q),
+                                     static_cast<const __nv_bfloat16*>(k),
+                                     static_cast<const __nv_bfloat16*>(v), gid, L, G, eps, out,
+                                     state, Hc, B, T, Hq, Hkv, C, st);
+    return launch_prefill_simt_t(static_cast<const float*>(q), static_cast<const float*>(k),
+                                 static_cast<const float*>(v), gid, L, G, eps, out, state, Hc,
+                                 B, T, Hq, Hkv, C, st);
+}
+
+template <typename Tin>
+static int launch_dense_t(const Tin* q, const Tin* k, const Tin* v, const int32_t* gid,
+                          const float* L, const int32_t* G, float eps, float* out, int B, int T,
+                          int Hq, int Hkv, cudaStream_t st)
+{
+    if (T == 0 || B == 0) return OAL_OK;
+    const size_t smem = sizeof(ReadoutSmem);
+    auto kern = readout_simt_kernel<Tin, true>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+        cudaSuccess)
+        return OAL_ERR_CUDA;
+    LaunchScope ls("dense_simt", st);
+    kern<<<dim3((T + 63) / 64, B * Hq), 256, smem, st>>>(q, k, v, gid, L, G, eps, nullptr,
+                                                         nullptr, out, Hq, Hkv, T, 64, 1);
+    OAL_LAUNCH_CHECK();
+    return OAL_OK;
+}
+
+int launch_dense(const void* q, const void* k, const void* v, const int32_t* gid, const float* L,
+                 const int32_t* G, float eps, float* out, int B, int T, int Hq, int Hkv,
+                 int dtype, cudaStream_t st)
+{
+    if (dtype == OAL_BF16)
+        return launch_dense_t(static_cast<const __nv_bfloat16*>(q),
+                              static_cast<const __nv_bfloat16*>(k),
+                              static_cast<const __nv_bfloat16*>(v), gid, L, G, eps, out, B, T,
+                              Hq, Hkv, st);
+    return launch_dense_t(static_cast<const float*>(q), static_cast<const float*>(k),
+                          static_cast<const float*>(v), gid, L, G, eps, out, B, T, Hq, Hkv, st);
+}
+
+int decode_slabs() { return (kF + kDecRows - 1) / kDecRows; }
+
+int launch_decode(const void* q, const void* k, const void* v, void* state, float* out,
+                  float* part, unsigned int* tickets, int B, int Hq, int Hkv, int dtype,
+                  cudaStream_t st)
+{
+    if (B == 0) return OAL_OK;
+    const dim3 grid(decode_slabs(), B * Hkv);
+    unsigned char* s = static_cast<unsigned char*>(state);
+    LaunchScope ls("decode", st);
+    if (dtype == OAL_BF16)
+        decode_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+            static_cast<const __nv_bfloat16*>(v), s, out, part, tickets, Hq, Hkv);
+    else
+        decode_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(q),
+                                                   static_cast<const float*>(k),
+                                                   static_cast<const float*>(v), s, out, part,
+                                                   tickets, Hq, Hkv);
+    OAL_LAUNCH_CHECK();
+    return OAL_OK;
+}
+
+int read_device_error(int* code, cudaStream_t st)
+{
+    int val = 0;
+    if (cudaMemcpyFromSymbolAsync(&val, g_device_error, sizeof(int), 0, cudaMemcpyDeviceToHost,
+                                  st) != cudaSuccess)
+        return OAL_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return OAL_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpyToSymbolAsync(g_device_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice,
+                                st) != cudaSuccess)
+        return OAL_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return OAL_ERR_CUDA;
+    *code = val;
+    return OAL_OK;
+}
+
+}  // namespace oal

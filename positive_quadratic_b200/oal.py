@@ -1,0 +1,275 @@
+"""Python binding of the OAL C ABI (include/oal.h): argument marshalling only.
+
+Every step of the computation runs in the CUDA library liboal.so.  PyTorch supplies device
+memory and streams.  The binding raises OALError on any non-zero status and refuses to run
+when the library is missing.  There is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+import threading
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "liboal.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "oal.h")
+
+OAL_F32, OAL_BF16 = 0, 1
+HEAD_DIM = VALUE_DIM = 64
+G_MAX = 8
+FEATURES, FEATURES_PAD = 2145, 2176
+STATUS = {0: "OAL_OK", -1: "OAL_ERR_NULL", -2: "OAL_ERR_SHAPE", -3: "OAL_ERR_UNSUPPORTED",
+          -4: "OAL_ERR_ALIGN", -5: "OAL_ERR_GROUPS", -6: "OAL_ERR_CUDA", -7: "OAL_ERR_TIMEOUT",
+          -8: "OAL_ERR_WORKSPACE", -9: "OAL_ERR_STATE"}
+
+
+class Shape(ctypes.Structure):
+    """oal_shape."""
+    _fields_ = [(n, ctypes.c_int32) for n in ("B", "T", "Hq", "Hkv", "dh", "dv", "chunk",
+                                               "dtype")]
+
+
+class KernelStat(ctypes.Structure):
+    """oal_kernel_stat."""
+    _fields_ = [("name", ctypes.c_char * 40), ("launches", ctypes.c_int32),
+                ("total_ms", ctypes.c_double)]
+
+
+class OALError(RuntimeError):
+    def __init__(self, code: int, what: str = ""):
+        self.code = code
+        super().__init__(f"{what}: {STATUS.get(code, code)} ({status_string(code)})")
+
+
+_lock = threading.Lock()
+_lib = None
+_VP, _SZ, _PS = ctypes.c_void_p, ctypes.c_size_t, ctypes.POINTER(Shape)
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded liboal.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"CUDA library not built: {LIB_PATH} is missing; run "
+                                   "python -m positive_quadratic_b200.build")
+            L = ctypes.CDLL(LIB_PATH)
+            L.oal_abi_version.restype = ctypes.c_int
+            L.oal_status_string.argtypes = [ctypes.c_int]
+            L.oal_status_string.restype = ctypes.c_char_p
+            for name in ("oal_state_bytes", "oal_prefill_workspace_bytes",
+                         "oal_decode_workspace_bytes"):
+                getattr(L, name).argtypes = [_PS, ctypes.POINTER(_SZ)]
+            L.oal_prefill.argtypes = [_VP] * 6 + [ctypes.c_float, _VP, _VP, _VP, _SZ, _PS, _VP]
+            L.oal_decode_step.argtypes = [_VP] * 6 + [_SZ, _PS, _VP]
+            L.oal_dense_ref_gpu.argtypes = [_VP] * 6 + [ctypes.c_float, _VP, _PS, _VP]
+            L.oal_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), _VP]
+            L.oal_launch_count.restype = ctypes.c_ulonglong
+            L.oal_profile_enable.argtypes = [ctypes.c_int]
+            L.oal_profile_enable.restype = ctypes.c_int
+            L.oal_profile_read.argtypes = [ctypes.POINTER(KernelStat), ctypes.c_int,
+                                           ctypes.POINTER(ctypes.c_int)]
+            L.oal_profile_read.restype = ctypes.c_int
+            for name in ("oal_state_bytes", "oal_prefill_workspace_bytes",
+                         "oal_decode_workspace_bytes", "oal_prefill", "oal_decode_step",
+                         "oal_dense_ref_gpu", "oal_device_error"):
+                getattr(L, name).restype = ctypes.c_int
+            _lib = L
+    return _lib
+
+
+def declared_symbols(header: str = HEADER):
+    """Names of the functions include/oal.h declares."""
+    text = open(header).read()
+    return sorted(set(re.findall(r"^\s*(?:int|const char\*|unsigned long long)\s+(oal_\w+)\s*\(",
+                                 text, re.M)))
+
+
+def status_string(code: int) -> str:
+    try:
+        return lib().oal_status_string(int(code)).decode()
+    except Exception:
+        return "?"
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise OALError(rc, what)
+
+
+def make_shape(B, T, Hq, Hkv, chunk=128, dtype=OAL_BF16, dh=HEAD_DIM, dv=VALUE_DIM) -> Shape:
+    return Shape(int(B), int(T), int(Hq), int(Hkv), int(dh), int(dv), int(chunk), int(dtype))
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return OAL_BF16
+    if t.dtype == torch.float32:
+        return OAL_F32
+    raise TypeError(f"q/k/v must be float32 or bfloat16, got {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def state_bytes(shape: Shape) -> int:
+    n = _SZ()
+    _check(lib().oal_state_bytes(ctypes.byref(shape), ctypes.byref(n)), "oal_state_bytes")
+    return n.value
+
+
+def prefill_workspace_bytes(shape: Shape) -> int:
+    n = _SZ()
+    _check(lib().oal_prefill_workspace_bytes(ctypes.byref(shape), ctypes.byref(n)),
+           "oal_prefill_workspace_bytes")
+    return n.value
+
+
+def decode_workspace_bytes(shape: Shape) -> int:
+    n = _SZ()
+    _check(lib().oal_decode_workspace_bytes(ctypes.byref(shape), ctypes.byref(n)),
+           "oal_decode_workspace_bytes")
+    return n.value
+
+
+def _shape_of(q, k, v, chunk):
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, v must be [B, H, T, d]")
+    B, Hq, T, dh = q.shape
+    return make_shape(B, T, Hq, k.shape[1], chunk, _dtype_code(q), dh, v.shape[3])
+
+
+def _contig_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def empty_workspace(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def prefill(q, k, v, group_id, L, G, eps: float, chunk: int = 128, out=None, state=None,
+            workspace=None, stream=None):
+    """oal_prefill on CUDA tensors.  Returns (out [B,Hq,T,dv] fp32, state uint8)."""
+    shape = _shape_of(q, k, v, chunk)
+    dev = q.device
+    if out is None:
+        out = torch.empty(q.shape[0], q.shape[1], q.shape[2], v.shape[3], dtype=torch.float32,
+                          device=dev)
+    if state is None:
+        state = torch.empty(state_bytes(shape), dtype=torch.uint8, device=dev)
+    if workspace is None:
+        workspace = empty_workspace(prefill_workspace_bytes(shape), dev)
+    _contig_cuda(q, k, v, group_id, L, G, out, state, workspace)
+    rc = lib().oal_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(group_id), _ptr(L), _ptr(G),
+                           float(eps), _ptr(out), _ptr(state), _ptr(workspace),
+                           workspace.numel() * workspace.element_size(), ctypes.byref(shape),
+                           _stream(stream))
+    _check(rc, "oal_prefill")
+    return out, state
+
+
+def decode_step(q, k, v, state, workspace, out=None, stream=None):
+    """oal_decode_step on CUDA tensors q [B,Hq,1,dh], k/v [B,Hkv,1,d]; returns out."""
+    shape = _shape_of(q, k, v, 128)
+    shape.T = 1
+    if out is None:
+        out = torch.empty(q.shape[0], q.shape[1], 1, v.shape[3], dtype=torch.float32,
+                          device=q.device)
+    _contig_cuda(q, k, v, state, workspace, out)
+    rc = lib().oal_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(state), _ptr(out),
+                               _ptr(workspace), workspace.numel() * workspace.element_size(),
+                               ctypes.byref(shape), _stream(stream))
+    _check(rc, "oal_decode_step")
+    return out
+
+
+def decode_workspace(B, Hq, Hkv, device) -> torch.Tensor:
+    """Zero-filled decode workspace (the ABI requires zeros before the first step)."""
+    n = decode_workspace_bytes(make_shape(B, 1, Hq, Hkv))
+    return torch.zeros(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def dense_ref(q, k, v, group_id, L, G, eps: float, out=None, stream=None):
+    """oal_dense_ref_gpu: the O(T^2) dense form."""
+    shape = _shape_of(q, k, v, 128)
+    if out is None:
+        out = torch.empty(q.shape[0], q.shape[1], q.shape[2], v.shape[3], dtype=torch.float32,
+                          device=q.device)
+    _contig_cuda(q, k, v, group_id, L, G, out)
+    rc = lib().oal_dense_ref_gpu(_ptr(q), _ptr(k), _ptr(v), _ptr(group_id), _ptr(L), _ptr(G),
+                                 float(eps), _ptr(out), ctypes.byref(shape), _stream(stream))
+    _check(rc, "oal_dense_ref_gpu")
+    return out
+
+
+def device_error(stream=None) -> int:
+    """Reads and clears the device-side error word (0 = none)."""
+    code = ctypes.c_int(0)
+    _check(lib().oal_device_error(ctypes.byref(code), _stream(stream)), "oal_device_error")
+    return code.value
+
+
+def prefill_host(q, k, v, group_id, L, G, eps: float, chunk: int = 128, dev_bufs=None,
+                 out_host=None, stream=None):
+    """End-to-end prefill from HOST tensors (pinned for overlap): copies q/k/v to the device,
+    runs oal_prefill, copies yhat back.  ``dev_bufs`` (from ``alloc_prefill_buffers``) reuses
+    device buffers across calls.  Returns the host output tensor."""
+    if dev_bufs is None:
+        dev_bufs = alloc_prefill_buffers(q, k, v, group_id, L, G, chunk)
+    dq, dk, dv_, dg, dL, dG, dout, dstate, dws = dev_bufs
+    s = torch.cuda.current_stream() if stream is None else stream
+    with torch.cuda.stream(s):
+        dq.copy_(q, non_blocking=True)
+        dk.copy_(k, non_blocking=True)
+        dv_.copy_(v, non_blocking=True)
+        prefill(dq, dk, dv_, dg, dL, dG, eps, chunk, dout, dstate, dws, s)
+        if out_host is None:
+            out_host = torch.empty(dout.shape, dtype=dout.dtype, pin_memory=True)
+        out_host.copy_(dout, non_blocking=True)
+    return out_host
+
+
+def alloc_prefill_buffers(q, k, v, group_id, L, G, chunk, device="cuda"):
+    """Device buffers for prefill_host (group ids, L and G are copied once here)."""
+    shape = _shape_of(q, k, v, chunk)
+    dq = torch.empty(q.shape, dtype=q.dtype, device=device)
+    dk = torch.empty(k.shape, dtype=k.dtype, device=device)
+    dv_ = torch.empty(v.shape, dtype=v.dtype, device=device)
+    dg = group_id.to(device=device, dtype=torch.int32).contiguous()
+    dL = L.to(device=device, dtype=torch.float32).contiguous()
+    dG = G.to(device=device, dtype=torch.int32).contiguous()
+    dout = torch.empty(q.shape[0], q.shape[1], q.shape[2], v.shape[3], dtype=torch.float32,
+                       device=device)
+    dstate = torch.empty(state_bytes(shape), dtype=torch.uint8, device=device)
+    dws = empty_workspace(prefill_workspace_bytes(shape), device)
+    return dq, dk, dv_, dg, dL, dG, dout, dstate, dws
+
+
+def launch_count() -> int:
+    """Kernels launched by the library since it was loaded."""
+    return int(lib().oal_launch_count())
+
+
+def profile_enable(on: bool = True):
+    _check(lib().oal_profile_enable(1 if on else 0), "oal_profile_enable")
+
+
+def profile_read() -> dict:
+    """{kernel name: (launches, total device ms)} since the previous read (waits for them)."""
+    arr = (KernelStat * 64)()
+    n = ctypes.c_int(0)
+    _check(lib().oal_profile_read(arr, 64, ctypes.byref(n)), "oal_profile_read")
+    return {arr[i].name.decode(): (int(arr[i].launches), float(arr[i].total_ms))
+            for i in range(n.value)}

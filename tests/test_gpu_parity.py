@@ -1,0 +1,249 @@
+"""GPU parity: the CUDA library (through the C ABI) against the fp64 oracle on the same seeded
+inputs.  Tolerances (row-relative max error, tests/_metrics.py): 1e-4 for fp32 inputs, 2e-2
+for bf16 inputs with fp32 accumulation.  Full-size workloads run in the benchmark's launch
+configuration and are checked on outputs the oracle can afford (sampled batch elements,
+layers or rows)."""
+import numpy as np
+import pytest
+
+import oracle
+from positive_quadratic_b200 import inputs as I
+from tests._metrics import TOL_BF16, TOL_F32, row_rel_err
+from tests._packed import F, FP, pack_oracle_state, packed_pairs, read_state
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def oal(cuda):
+    from positive_quadratic_b200 import build, oal as binding
+    build.build()
+    binding.lib()
+    return binding
+
+
+def dev_inputs(p, dev):
+    dt = torch.bfloat16 if p.dtype == "bf16" else torch.float32
+    t = lambda a, d=None: torch.from_numpy(np.ascontiguousarray(a)).to(dev, d)  # noqa: E731
+    return (t(p.q, dt), t(p.k, dt), t(p.v, dt), t(p.group_id), t(p.L), t(p.G))
+
+
+def tol(p):
+    return TOL_BF16 if p.dtype == "bf16" else TOL_F32
+
+
+def gpu_prefill(oal, p, dev, chunk=128):
+    q, k, v, g, L, G = dev_inputs(p, dev)
+    out, state = oal.prefill(q, k, v, g, L, G, p.eps, chunk)
+    torch.cuda.synchronize()
+    assert oal.device_error() == 0
+    return out.cpu().numpy(), state
+
+
+# --- config 0: tiny fp32 ---------------------------------------------------------------------
+
+@pytest.mark.parametrize("chunk", [64, 128, 256])
+def test_config0_prefill_f32(oal, cuda, chunk):
+    p = I.config0()
+    ref = oracle.dense(p.q, p.k, p.v, p.group_id, p.L, p.G, p.eps)
+    y, _ = gpu_prefill(oal, p, cuda, chunk)
+    assert row_rel_err(y, ref) <= TOL_F32
+
+
+def test_config0_dense_ref_f32(oal, cuda):
+    p = I.config0()
+    ref = oracle.dense(p.q, p.k, p.v, p.group_id, p.L, p.G, p.eps)
+    q, k, v, g, L, G = dev_inputs(p, cuda)
+    y = oal.dense_ref(q, k, v, g, L, G, p.eps).cpu().numpy()
+    assert row_rel_err(y, ref) <= TOL_F32
+
+
+# --- ragged sizes, GQA, both dtypes ---------------------------------------------------------
+
+@pytest.mark.parametrize("T", [1, 7, 63, 64, 65, 127, 128, 129, 255, 257, 700])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_ragged_prefill(oal, cuda, T, dtype):
+    p = I.small_layer(200 + T, B=2, T=T, Hq=4, Hkv=2, dtype=dtype)
+    ref = oracle.recurrent(p.q, p.k, p.v, p.group_id, p.L, p.G, p.eps)
+    for chunk in (64, 128, 256):
+        y, _ = gpu_prefill(oal, p, cuda, chunk)
+        assert row_rel_err(y, ref) <= tol(p), (chunk, row_rel_err(y, ref))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_dense_ref_gqa(oal, cuda, dtype):
+    p = I.small_layer(300, B=2, T=333, Hq=14, Hkv=2, dtype=dtype)
+    ref = oracle.dense(p.q, p.k, p.v, p.group_id, p.L, p.G, p.eps)
+    q, k, v, g, L, G = dev_inputs(p, cuda)
+    y = oal.dense_ref(q, k, v, g, L, G, p.eps).cpu().numpy()
+    assert row_rel_err(y, ref) <= tol(p)
+
+
+def test_group_count_extremes(oal, cuda):
+    rng = np.random.default_rng(5)
+    p = I.small_layer(301, B=1, T=300, Hq=4, Hkv=1, dtype="f32")
+    p.G[:] = [1, 8, 8, 2]
+    p.group_id[0] = 1
+    for h in (1, 2):
+        p.group_id[h] = rng.integers(1, 9, size=64)
+        p.group_id[h, :8] = np.arange(1, 9)
+        p.L[h] = I.random_L(rng, 8)
+    p.group_id[3] = 1
+    p.group_id[3, 5] = 2
+    p.L[0] = I.random_L(rng, 1)
+    p.L[3] = I.random_L(rng, 2)
+    ref = oracle.recurrent(p.q, p.k, p.v, p.group_id, p.L, p.G, p.eps)
+    y, _ = gpu_prefill(oal, p, cuda, 128)
+    assert row_rel_err(y, ref) <= TOL_F32
+
+
+def test_empty_inputs(oal, cuda):
+    p = I.small_layer(302, B=1, T=0, Hq=2, Hkv=1, dtype="bf16")
+    y, state = gpu_prefill(oal, p, cuda, 128)
+    assert y.shape == (1, 2, 0, 64)
+    hdr, _, S = read_state(state.cpu().numpy(), 1, 2, 1)
+    assert hdr["tokens"] == 0 and np.all(S == 0)
+    p0 = I.small_layer(303, B=0, T=16, Hq=2, Hkv=1, dtype="bf16")
+    y0, _ = gpu_prefill(oal, p0, cuda, 128)
+    assert y0.shape == (0, 2, 16, 64)
+
+
+def test_output_canary(oal, cuda):
+    """Nothing is written past the end of `out`."""
+    p = I.small_layer(304, B=1, T=190, Hq=2, Hkv=1, dtype="bf16")
+    q, k, v, g, L, G = dev_inputs(p, cuda)
+    n = 1 * 2 * 190 * 64
+    big = torch.full((n + 4096,), 12345.0, device=cuda)
+    out = big[:n].view(1, 2, 190, 64)
+    oal.prefill(q, k, v, g, L, G, p.eps, 128, out=out)
+    torch.cuda.synchronize()
+    assert torch.all(big[n:] == 12345.0)
+
+
+def test_bad_group_id_sets_error_word(oal, cuda):
+    p = I.small_layer(305, B=1, T=64, Hq=2, Hkv=1, dtype="bf16")
+    p.group_id[1, 3] = 0
+    q, k, v, g, L, G = dev_inputs(p, cuda)
+    out, _ = oal.prefill(q, k, v, g, L, G, p.eps, 128)
+    torch.cuda.synchronize()
+    assert oal.device_error() == -5
+    assert oal.device_error() == 0  # cleared by the read
+    assert torch.isfinite(out).all()
+
+
+# --- state layout, coefficients, decode ------------------------------------------------------
+
+def _coef_reference(p):
+    """Readout weights of the packed rows per include/oal.h, from L and the group ids."""
+    pairs = packed_pairs()
+    Hq = p.G.shape[0]
+    out = np.zeros((Hq, FP))
+    for h in range(Hq):
+        Gh = int(p.G[h])
+        Lh = p.L[h, :Gh + 1, :Gh + 1].astype(np.float64)
+        M = Lh @ Lh.T
+        g = np.concatenate([p.group_id[h], [0]])
+        s = np.concatenate([np.full(64, 0.125), [1.0]])
+        r, t = pairs[:, 0], pairs[:, 1]
+        out[h, :F] = np.where(r == t, 1.0, 2.0) * M[g[r], g[t]] * s[r] * s[t]
+        out[h, 2144] += p.eps
+    return out
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_state_and_coefficients(oal, cuda, dtype):
+    p = I.small_layer(306, B=2, T=333, Hq=4, Hkv=2, dtype=dtype)
+    _, st = oracle.recurrent(p.q, p.k, p.v, p.group_id, p.L, p.G, p.eps, return_state=True)
+    _, state = gpu_prefill(oal, p, cuda, 128)
+    hdr, coef, S = read_state(state.cpu().numpy(), 2, 4, 2)
+    assert hdr["magic"] == 0x534C414F and hdr["tokens"] == 333 and hdr["feat_pad"] == FP
+    assert (hdr["B"], hdr["Hq"], hdr["Hkv"], hdr["dh"], hdr["dv"]) == (2, 4, 2, 64, 64)
+    np.testing.assert_allclose(coef, _coef_reference(p), rtol=1e-6, atol=1e-9)
+    ref = pack_oracle_state(st)
+    scale = np.abs(ref).max(axis=2, keepdims=True)
+    assert np.max(np.abs(S[:, :, :F] - ref) / scale) < 1e-5
+    assert np.all(S[:, :, F:] == 0)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_decode_continuation(oal, cuda, dtype):
+    """prefill(T) + n decode steps == prefill(T + n) (outputs and state)."""
+    T0, n = 200, 6
+    p = I.small_layer(307, B=3, T=T0 + n, Hq=14, Hkv=2, dtype=dtype)
+    y_all, st_all = oracle.recurrent(p.q, p.k, p.v, p.group_id, p.L, p.G, p.eps,
+                                     return_state=True)
+    pre = p.slice_tokens(0, T0)
+    _, state = gpu_prefill(oal, pre, cuda, 128)
+    ws = oal.decode_workspace(3, 14, 2, cuda)
+    q, k, v, _, _, _ = dev_inputs(p, cuda)
+    for t in range(T0, T0 + n):
+        sl = lambda x: x[:, :, t:t + 1].contiguous()  # noqa: E731
+        y = oal.decode_step(sl(q), sl(k), sl(v), state, ws)
+        torch.cuda.synchronize()
+        assert row_rel_err(y.cpu().numpy()[:, :, 0], y_all[:, :, t]) <= tol(p)
+    assert oal.device_error() == 0
+    assert torch.all(ws[:256] == 0)  # completion tickets return to zero
+    hdr, _, S = read_state(state.cpu().numpy(), 3, 14, 2)
+    assert hdr["tokens"] == T0 + n
+    ref = pack_oracle_state(st_all)
+    assert np.max(np.abs(S[:, :, :F] - ref) / np.abs(ref).max(axis=2, keepdims=True)) < 1e-5
+
+
+def test_chunk_size_independence(oal, cuda):
+    p = I.small_layer(308, B=1, T=1000, Hq=4, Hkv=2, dtype="f32")
+    ys = [gpu_prefill(oal, p, cuda, c)[0] for c in (64, 128, 256)]
+    assert row_rel_err(ys[1], ys[0]) < 2e-5 and row_rel_err(ys[2], ys[0]) < 2e-5
+
+
+# --- full-size workloads (benchmark launch configuration), sampled checks ---------------------
+
+def test_config1_full(oal, cuda):
+    p = I.config1()
+    ref = oracle.recurrent(p.q, p.k, p.v, p.group_id, p.L, p.G, p.eps)
+    y, _ = gpu_prefill(oal, p, cuda, 128)
+    err = row_rel_err(y, ref)
+    print(f"config1 max row-relative error {err:.3e}")
+    assert err <= TOL_BF16
+
+
+@pytest.mark.parametrize("layer", [0, 17])
+def test_config2_sampled(oal, cuda, layer):
+    p = I.config2_layer(layer)
+    y, _ = gpu_prefill(oal, p, cuda, 128)
+    for b in (0, 7):
+        s = p.slice_batch(b, b + 1)
+        ref = oracle.recurrent(s.q, s.k, s.v, s.group_id, s.L, s.G, s.eps)
+        assert row_rel_err(y[b:b + 1], ref) <= TOL_BF16, (layer, b)
+
+
+@pytest.mark.parametrize("T", [16384, 65536])
+def test_config3_sampled_rows(oal, cuda, T):
+    p = I.config3(T)
+    rng = np.random.default_rng(T)
+    rows = [(0, int(h), int(i)) for h, i in zip(rng.integers(0, 14, 12), rng.integers(0, T, 12))]
+    rows += [(0, 0, 0), (0, 13, T - 1), (0, 6, T // 2)]
+    ref = oracle.dense_rows(p.q, p.k, p.v, p.group_id, p.L, p.G, p.eps, rows)
+    for chunk in ((64, 128, 256) if T == 16384 else (128,)):
+        y, _ = gpu_prefill(oal, p, cuda, chunk)
+        got = np.stack([y[b, h, i] for b, h, i in rows])
+        assert row_rel_err(got, ref) <= TOL_BF16, chunk
+
+
+def test_config4_decode_sampled(oal, cuda):
+    p = I.config4(batch=64, context=4096, steps=4)
+    pre = p.slice_tokens(0, 4096)
+    _, state = gpu_prefill(oal, pre, cuda, 128)
+    ws = oal.decode_workspace(64, 14, 2, cuda)
+    q, k, v, _, _, _ = dev_inputs(p, cuda)
+    ys = []
+    for t in range(4096, 4100):
+        sl = lambda x: x[:, :, t:t + 1].contiguous()  # noqa: E731
+        ys.append(oal.decode_step(sl(q), sl(k), sl(v), state, ws).cpu().numpy()[:, :, 0])
+    assert oal.device_error() == 0
+    for b in (0, 41):
+        s = p.slice_batch(b, b + 1)
+        ref = oracle.recurrent(s.q, s.k, s.v, s.group_id, s.L, s.G, s.eps)
+        for n, t in enumerate(range(4096, 4100)):
+            assert row_rel_err(ys[n][b:b + 1], ref[:, :, t]) <= TOL_BF16, (b, t)

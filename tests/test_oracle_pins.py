@@ -303,3 +303,13 @@ def test_golden_regression_record():
     for n, i in enumerate(rec["rows"]):
         np.testing.assert_allclose(y[0, 0, i, :8], rec["yhat_first8"][n], rtol=1e-12)
         np.testing.assert_allclose(den[0, 0, i], rec["normaliser"][n], rtol=1e-12)
+
+
+def test_dense_rows_match_dense():
+    """Sampled-row evaluation returns exactly the rows of the full dense form."""
+    p = I.small_layer(12, B=2, T=50, Hq=4, Hkv=2, dtype="bf16")
+    y = oracle.dense(p.q, p.k, p.v, p.group_id, p.L, p.G, p.eps)
+    rows = [(0, 0, 0), (1, 3, 49), (0, 2, 17), (1, 1, 33)]
+    yr = oracle.dense_rows(p.q, p.k, p.v, p.group_id, p.L, p.G, p.eps, rows)
+    for n, (b, h, i) in enumerate(rows):
+        np.testing.assert_array_equal(yr[n], y[b, h, i])
