@@ -132,6 +132,25 @@ int oal_decode_step(const void* q, const void* k, const void* v, void* state, fl
                     void* workspace, size_t workspace_bytes, const oal_shape* s,
                     void* stream);
 
+/* oal_decode_step without a workspace: allocates nothing and takes no scratch argument.
+ * The paper has no counterpart; this is an interface for callers that cannot allocate
+ * device memory: for example a serving engine that reserves all GPU memory for its own pool
+ * at start-up and forbids allocation afterwards, a host framework whose plugin interface
+ * hands an operator only its input and output buffers, or a latency-critical loop that
+ * cannot afford cudaMalloc's implicit device-wide synchronisation.
+ * Same arguments and results as oal_decode_step, minus the workspace.  The scratch is a
+ * fixed 4 MiB array inside the library (one copy on every GPU that loads the library, held
+ * until the process exits).  A step needs align256(4*B*Hkv) + 4420*B*Hq bytes of it, so
+ * B*Hq must stay at or below 948 (batch 64 x 14 heads fits); larger problems return
+ * OAL_ERR_UNSUPPORTED without launching anything.
+ * The first call on each device looks up the array's device address (cudaGetSymbolAddress);
+ * make that first call before any stream capture.  Every call shares the one array and
+ * clears the part that must start at zero itself, so calls that overlap on the GPU (on
+ * different streams, or from threads that do not order their calls) race and corrupt each
+ * other's results: issue them one after another. */
+int oal_decode_step_noalloc(const void* q, const void* k, const void* v, void* state,
+                            float* out, const oal_shape* s, void* stream);
+
 /* The exact O(T^2) dense form (eqs. (2)-(3) summed over j <= i and normalised), for
  * cross-checking and timing against the linear-time path.  Same arguments as oal_prefill
  * without the state; `chunk` is ignored.  Computes in fp32 for both dtypes. */

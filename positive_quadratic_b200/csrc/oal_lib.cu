@@ -3,3 +3,4 @@
 #include "oal_common.cuh"
 #include "oal_simt.cu"
 #include "oal_api.cu"
+#include "oal_noalloc.cu"
