@@ -158,6 +158,14 @@ int oal_dense_ref_gpu(const void* q, const void* k, const void* v, const int32_t
                       const float* L, const int32_t* G, float eps, float* out,
                       const oal_shape* s, void* stream);
 
+/* Scheduling of the tensor-core prefill (bf16, chunk 128).  1 (default): one persistent
+ * kernel pulls state-building and readout work from a single queue, so readouts of early
+ * chunks overlap the building of later chunk states; it needs every CTA resident at once and
+ * falls back to 0 when the device cannot host the grid.  0: two kernels, all chunk states
+ * first, then all readouts.  Both produce the same results.  Process-wide; returns the
+ * previous setting. */
+int oal_set_prefill_fused(int fused);
+
 /* Reads the device-side error word (OAL_OK or a negative oal_status set by a kernel since
  * the last read), synchronising `stream`, and clears it. */
 int oal_device_error(int* code, void* stream);
@@ -176,6 +184,11 @@ int oal_profile_enable(int on);
 int oal_profile_read(oal_kernel_stat* stats, int max_stats, int* n_stats);
 /* Kernels launched by this library since it was loaded (all devices, all streams). */
 unsigned long long oal_launch_count(void);
+
+/* The CUDA runtime error (cudaError_t value; 0 = none) behind the most recent OAL_ERR_CUDA
+ * returned by any call in this process, with its name and description written into buf
+ * (NUL-terminated, truncated to len bytes; buf may be NULL). */
+int oal_last_cuda_error(char* buf, size_t len);
 
 /* Static description of a status code. */
 const char* oal_status_string(int status);

@@ -1,5 +1,7 @@
 // oal_api.cu -- the extern "C" boundary declared in include/oal.h: argument validation on the
 // host, workspace layout, and dispatch to the kernels.  No device memory is allocated here.
+#include <atomic>
+#include <cstdio>
 #include <cstring>
 
 #include "oal_common.cuh"
@@ -44,6 +46,11 @@ size_t simt_chunk_state_bytes(const oal_shape* s)
     const size_t NC = s->T > 0 ? size_t((s->T + s->chunk - 1) / s->chunk) : 0;
     return size_t(s->B) * s->Hkv * NC * kW * kFP * sizeof(float);
 }
+
+// bf16 inputs with chunk 128 run on the tcgen05 kernels; everything else on CUDA cores.
+bool use_tensor_path(const oal_shape* s) { return s->dtype == OAL_BF16 && s->chunk == 128; }
+
+std::atomic<int> g_prefill_fused{1};
 
 size_t decode_ticket_bytes(const oal_shape* s) { return align256(size_t(s->B) * s->Hkv * 4); }
 
@@ -90,7 +97,8 @@ int oal_prefill_workspace_bytes(const oal_shape* s, size_t* bytes)
     if (rc) return rc;
     if ((rc = check_chunk(s))) return rc;
     if (!bytes) return OAL_ERR_NULL;
-    *bytes = simt_chunk_state_bytes(s);
+    const size_t tc = use_tensor_path(s) ? tc_workspace_bytes(s->B, s->Hkv, s->T) : 0;
+    *bytes = simt_chunk_state_bytes(s) > tc ? simt_chunk_state_bytes(s) : tc;
     if (*bytes == 0) *bytes = 256;
     return OAL_OK;
 }
@@ -123,6 +131,9 @@ int oal_prefill(const void* q, const void* k, const void* v, const int32_t* grou
     rc = launch_prep(group_id, L, G, eps, state, s->B, s->Hq, s->Hkv, s->T, st);
     if (rc) return rc;
     if (s->B == 0) return OAL_OK;
+    if (use_tensor_path(s))
+        return launch_prefill_tc(q, k, v, group_id, L, G, eps, out, state, workspace, s->B, s->T,
+                                 s->Hq, s->Hkv, g_prefill_fused.load() != 0, st);
     return launch_prefill_simt(q, k, v, group_id, L, G, eps, out, state,
                                static_cast<float*>(workspace), s->B, s->T, s->Hq, s->Hkv,
                                s->chunk, s->dtype, st);
@@ -164,6 +175,8 @@ int oal_dense_ref_gpu(const void* q, const void* k, const void* v, const int32_t
 }
 
 unsigned long long oal_launch_count(void) { return tracer().launches.load(); }
+
+int oal_set_prefill_fused(int fused) { return g_prefill_fused.exchange(fused ? 1 : 0); }
 
 int oal_profile_enable(int on)
 {
@@ -211,6 +224,17 @@ int oal_profile_read(oal_kernel_stat* stats, int max_stats, int* n_stats)
     }
     *n_stats = n;
     return rc;
+}
+
+int oal_last_cuda_error(char* buf, size_t len)
+{
+    const int e = last_cuda_error().load();
+    if (buf && len > 0) {
+        const char* name = e ? cudaGetErrorName(cudaError_t(e)) : "cudaSuccess";
+        const char* text = e ? cudaGetErrorString(cudaError_t(e)) : "no error";
+        std::snprintf(buf, len, "%s: %s", name, text);
+    }
+    return e;
 }
 
 int oal_device_error(int* code, void* stream)

@@ -19,6 +19,7 @@
 //   [2145, 2176)  padding, (65, 65) with khat_65 = qhat_65 = 0: always zero
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -65,22 +66,22 @@ __host__ __device__ constexpr size_t state_bytes(int B, int Hq, int Hkv) {
 // (r, t) of packed feature row f; padding rows map to (65, 65).
 struct RT { int r, t; };
 
-__host__ __device__ __forceinline__ RT feature_rt(int f) {
+__host__ __device__ constexpr RT feature_rt(int f) {
     if (f < kOffDiagRows) {
         int beta = f >> 6, R = 0, s = 0;
         while (beta >= s + 7 - R) { s += 7 - R; ++R; }
         const int T = R + 1 + (beta - s);
-        return {8 * R + ((f >> 3) & 7), 8 * T + (f & 7)};
+        return RT{8 * R + ((f >> 3) & 7), 8 * T + (f & 7)};
     }
     if (f < kLinStart) {
         const int e = f - kOffDiagRows, R = e / 36;
         int p = e - 36 * R, a = 0;
         while (p >= 8 - a) { p -= 8 - a; ++a; }
-        return {8 * R + a, 8 * R + a + p};
+        return RT{8 * R + a, 8 * R + a + p};
     }
-    if (f < kConstRow) return {f - kLinStart, kD};
-    if (f == kConstRow) return {kD, kD};
-    return {kD + 1, kD + 1};
+    if (f < kConstRow) return RT{f - kLinStart, kD};
+    if (f == kConstRow) return RT{kD, kD};
+    return RT{kD + 1, kD + 1};
 }
 
 // Device-side error word (OAL_OK or a negative oal_status); first error wins.  The library
@@ -95,10 +96,31 @@ template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16
     return __bfloat162float(x);
 }
 
+// The CUDA error behind the most recent OAL_ERR_CUDA (process-wide, last writer wins).
+inline std::atomic<int>& last_cuda_error()
+{
+    static std::atomic<int> e{0};
+    return e;
+}
+
+inline int cuda_fail(cudaError_t e)
+{
+    last_cuda_error().store(int(e));
+    return OAL_ERR_CUDA;
+}
+
 // Launch-side error check: returns OAL_ERR_CUDA from the calling function.
-#define OAL_LAUNCH_CHECK()                                    \
-    do {                                                      \
-        if (cudaGetLastError() != cudaSuccess) return OAL_ERR_CUDA; \
+#define OAL_LAUNCH_CHECK()                                \
+    do {                                                  \
+        const cudaError_t oal_e_ = cudaGetLastError();    \
+        if (oal_e_ != cudaSuccess) return cuda_fail(oal_e_); \
+    } while (0)
+
+// Evaluates a CUDA runtime call; on failure returns OAL_ERR_CUDA from the calling function.
+#define OAL_CUDA_TRY(call)                                \
+    do {                                                  \
+        const cudaError_t oal_e_ = (call);                \
+        if (oal_e_ != cudaSuccess) return cuda_fail(oal_e_); \
     } while (0)
 
 }  // namespace oal

@@ -2,5 +2,6 @@
 // all kernels (the error word) exist exactly once without relocatable device code.
 #include "oal_common.cuh"
 #include "oal_simt.cu"
+#include "oal_tc.cu"
 #include "oal_api.cu"
 #include "oal_noalloc.cu"

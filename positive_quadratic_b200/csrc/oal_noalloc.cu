@@ -64,7 +64,7 @@ extern "C" int oal_decode_step_noalloc(const void* q, const void* k, const void*
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     unsigned char* ws = static_cast<unsigned char*>(scratch);
     // The array keeps whatever the previous call left; the tickets must start at zero.
-    if (cudaMemsetAsync(ws, 0, decode_ticket_bytes(s), st) != cudaSuccess) return OAL_ERR_CUDA;
+    OAL_CUDA_TRY(cudaMemsetAsync(ws, 0, decode_ticket_bytes(s), st));
     return launch_decode(q, k, v, state, out,
                          reinterpret_cast<float*>(ws + decode_ticket_bytes(s)),
                          reinterpret_cast<unsigned int*>(ws), s->B, s->Hq, s->Hkv, s->dtype, st);

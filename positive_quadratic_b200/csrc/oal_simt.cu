@@ -515,9 +515,7 @@ static int launch_prefill_simt_t(const Tin* q, const Tin* k, const Tin* v,
     if (T == 0) return OAL_OK;
     const size_t smem = sizeof(ReadoutSmem);
     auto kern = readout_simt_kernel<Tin, false>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
-        cudaSuccess)
-        return OAL_ERR_CUDA;
+    OAL_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
     LaunchScope ls("readout_simt", st);
     kern<<<dim3((T + 63) / 64, B * Hq), 256, smem, st>>>(q, k, v, gid, L, G, eps, coef, Hc, out,
                                                          Hq, Hkv, T, C, NC);
@@ -548,9 +546,7 @@ static int launch_dense_t(const Tin* q, const Tin* k, const Tin* v, const int32_
     if (T == 0 || B == 0) return OAL_OK;
     const size_t smem = sizeof(ReadoutSmem);
     auto kern = readout_simt_kernel<Tin, true>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
-        cudaSuccess)
-        return OAL_ERR_CUDA;
+    OAL_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
     LaunchScope ls("dense_simt", st);
     kern<<<dim3((T + 63) / 64, B * Hq), 256, smem, st>>>(q, k, v, gid, L, G, eps, nullptr,
                                                          nullptr, out, Hq, Hkv, T, 64, 1);
@@ -597,15 +593,13 @@ int launch_decode(const void* q, const void* k, const void* v, void* state, floa
 int read_device_error(int* code, cudaStream_t st)
 {
     int val = 0;
-    if (cudaMemcpyFromSymbolAsync(&val, g_device_error, sizeof(int), 0, cudaMemcpyDeviceToHost,
-                                  st) != cudaSuccess)
-        return OAL_ERR_CUDA;
-    if (cudaStreamSynchronize(st) != cudaSuccess) return OAL_ERR_CUDA;
+    OAL_CUDA_TRY(cudaMemcpyFromSymbolAsync(&val, g_device_error, sizeof(int), 0, cudaMemcpyDeviceToHost,
+                                  st));
+    OAL_CUDA_TRY(cudaStreamSynchronize(st));
     const int zero = 0;
-    if (cudaMemcpyToSymbolAsync(g_device_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice,
-                                st) != cudaSuccess)
-        return OAL_ERR_CUDA;
-    if (cudaStreamSynchronize(st) != cudaSuccess) return OAL_ERR_CUDA;
+    OAL_CUDA_TRY(cudaMemcpyToSymbolAsync(g_device_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice,
+                                st));
+    OAL_CUDA_TRY(cudaStreamSynchronize(st));
     *code = val;
     return OAL_OK;
 }

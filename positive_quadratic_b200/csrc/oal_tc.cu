@@ -1,0 +1,1182 @@
+// oal_tc.cu -- tcgen05 / TMA kernels of the bf16 chunked prefill on B200 (sm_100a).
+//
+// Equations: "OAL: 按 QK 离群贡献分组的正二次注意力核" (reproduction note of arXiv 2610.13674),
+// section 核心公式, numbered in order of appearance: (2) grouped score, (3) kernel kappa,
+// (4) prefix states, (5) readout.  With the packed feature map of oal_common.cuh, the state
+// of a (b, kv) head after token i is S_i = sum_{j<=i} psi(k_j) [v_j; 1] (2176 x 65) and
+// u_i = phi(q_i)^T S_i.  Chunked with C = 128 tokens, the prefill is three kinds of work item:
+//
+//   chain builder (b, kv, slab): 128 packed rows of one state, walked chunk by chunk.
+//     Producer warps build bf16 psi(K_c)^T (MN-major) in shared memory; one N=80 MMA per
+//     K-step accumulates dS_c = psi(K_c)^T [V_c; 1] in TMEM (the [.; 1] column comes from a
+//     constant "ones" atom addressed through the B descriptor's leading byte offset);
+//     epilogue warps keep the running prefix in fp32 registers and store the exclusive prefix
+//     S_c of every chunk as a bf16 K-major B-operand image (bulk copy).
+//   remainder item (b, kv, slab, token segment): the same product with psi replaced by its
+//     bf16 rounding remainder psi - bf16(psi) (exact: psi = k_r k_t of two bf16 values has at
+//     most 16 significant bits).  Chain and remainders add their fp32 sums into the final
+//     state, which therefore holds the exact products accumulated in fp32.
+//   reader (b, h, chunk c): 128 query rows of one head.  phi(Q_c) is written straight into
+//     tensor memory (tcgen05.st) slice by slice and multiplied with the state image of S_c by
+//     N=80 MMAs reading A from TMEM; concurrently the intra-chunk kernel is evaluated on tensor
+//     cores in the factored form of eq. (3),
+//       kappa = eps + sum_m (L_0m + (q o w_m) . k)^2,   w_m[r] = L_{g(r),m} / sqrt(d)
+//     (= ||L^T sbar||^2), masked causally and multiplied into [V_c; 1] in the same TMEM
+//     accumulator; finally yhat = u[:64] / u[64].
+//
+// One CTA shape (18 warps, 1 CTA per SM) serves all items.  Kernels: builders + remainders,
+// readers, and a persistent kernel that pulls every item from one queue in which each reader
+// follows the chain builders it depends on; readers wait (bounded) on per-chunk counters that
+// chain builders release once an image has reached global memory.
+//
+// Every wait is bounded (1 s); one that runs out sets OAL_ERR_TIMEOUT and the CTA leaves its
+// loops in order (copies drained, MMAs committed, TMEM freed) instead of hanging.
+#include <algorithm>
+#include <mutex>
+#include <utility>
+
+#include <cuda.h>
+
+#include "oal_common.cuh"
+#include "oal_kernels.cuh"
+#include "oal_tc_util.cuh"
+
+namespace oal {
+namespace tc {
+
+constexpr int kC = 128;                                    // chunk = tile rows
+constexpr int kSlabRows = 128;                             // packed rows per builder item
+constexpr int kNumSlabs = kFP / kSlabRows;                 // 17
+constexpr int kSlices = kFP / 64;                          // 34 readout K-slices
+constexpr int kOffDiagSlices = kOffDiagRows / 64;          // 28
+constexpr int kSegChunks = 8;                              // chunks per remainder item
+constexpr uint32_t kImgSliceBytes = 80 * 64 * 2;           // K-major [80 n][64 rows]
+constexpr size_t kImgChunkBytes = size_t(kSlices) * kImgSliceBytes;
+constexpr uint32_t kTileBytes = kC * 64 * 2;               // 16384: one 128 x 64 bf16 tile
+constexpr uint32_t kOnesAtomBytes = kC * 128;              // 16384: 128 rows x 128 B
+constexpr uint16_t kBf16One = 0x3F80;
+
+constexpr int kWarps = 18;
+constexpr int kThreads = kWarps * 32;
+constexpr int kTmaWarp = 16;
+constexpr int kMmaWarp = 17;
+constexpr uint32_t kTmemCols = 512;
+
+static_assert(kFP % kSlabRows == 0 && kFP % 64 == 0, "feature padding");
+
+// ---- shared memory (offsets from a 1024-aligned base) ---------------------------------------
+// reader
+constexpr uint32_t kRdOffK = 0;           // K tile (score B operand, K-major)
+constexpr uint32_t kRdOffV = 16384;       // V tile (PV B operand, MN-major)
+constexpr uint32_t kRdOffQ = 32768;       // Q tile (bf16)
+constexpr uint32_t kRdOffQf = 49152;      // fp32 q rows [128][64], 16-byte chunks swizzled
+constexpr uint32_t kRdOffAq = 81920;      // Aq0 | Aq1 (score A operands); P tile aliases
+constexpr uint32_t kRdOffB = 114688;      // 4 x 10 KB state-image stages
+constexpr uint32_t kRdOffOnes = 155648;   // 16 KB ones atom
+constexpr uint32_t kRdOffCoef = 172032;   // 2176 fp32
+constexpr uint32_t kRdOffW = 180736;      // 9 x 64 fp32
+constexpr uint32_t kRdOffC0 = 183040;     // 9 fp32
+// builder
+constexpr uint32_t kStOffKV = 0;          // 4 x (K 16 KB + V 16 KB)
+constexpr uint32_t kStOffA = 131072;      // 2 x 16 KB psi stages
+constexpr uint32_t kStOffOnes = 163840;   // 16 KB ones atom
+constexpr uint32_t kStOffImg = 180224;    // 2 slices x 10 KB staging
+// both
+constexpr uint32_t kOffCtl = 219392;      // barriers and control words
+constexpr uint32_t kSmemBytes = kOffCtl + 512 + 1024;
+
+constexpr int kRdStages = 4;
+constexpr int kKVStages = 4;
+constexpr uint32_t kStATile = 64 * kSlabRows * 2;          // 64 tokens x 128 rows = 16 KB
+constexpr uint32_t kColU = 0, kColS0 = 128, kColA0 = 384;  // reader TMEM map
+
+struct RdBars {
+    uint64_t qkv_full, aq_full[2], s_full[2], s_empty[2], p_full;
+    uint64_t a_full[kRdStages], b_full[kRdStages], ab_empty[kRdStages];
+    uint64_t u_full, done;
+};
+struct StBars {
+    uint64_t kv_full[kKVStages], kv_empty[kKVStages], a_full[2], a_empty[2];
+    uint64_t acc_full[2], acc_empty[2], done;
+};
+struct Ctl {
+    union {
+        RdBars rd;
+        StBars st;
+        uint64_t raw[32];
+    } bar;
+    uint32_t tmem_base;
+    int abort_flag;
+    int item;
+    int G;
+};
+static_assert(sizeof(Ctl) <= 512, "control block");
+
+struct Params {
+    const CUtensorMap* tm_q;
+    const CUtensorMap* tm_k;
+    const CUtensorMap* tm_v;
+    const int32_t* gid;
+    const float* L;
+    const int32_t* G;
+    float eps;
+    const float* coef_all;   // state header coefficient table [Hq][kFP]
+    unsigned char* img;      // chunk-state images [B*Hkv][NC][34][10240]
+    float* body;             // final state (zeroed before the launch; items add into it)
+    float* out;
+    unsigned int* flags;     // [B*Hkv][NC] image-completion counters (persistent mode) or null
+    unsigned int* queue;     // work-queue head (persistent mode)
+    int B, Hq, Hkv, T, NC, nseg;
+};
+
+// ------------------------------------------------------------------------------------------
+// helpers
+// ------------------------------------------------------------------------------------------
+template <typename F, int... I>
+__device__ __forceinline__ void static_for_impl(F&& f, std::integer_sequence<int, I...>)
+{
+    (f(std::integral_constant<int, I>{}), ...);
+}
+template <int N, typename F>
+__device__ __forceinline__ void static_for(F&& f)
+{
+    static_for_impl(f, std::make_integer_sequence<int, N>{});
+}
+
+// (R, T) of off-diagonal block beta (R < T, lexicographic)
+__device__ __forceinline__ void block_rt(int beta, int& R, int& T)
+{
+    int r = 0, s = 0;
+    while (beta >= s + 7 - r) {
+        s += 7 - r;
+        ++r;
+    }
+    R = r;
+    T = r + 1 + (beta - s);
+}
+
+__device__ __forceinline__ void warp_arrive(uint64_t* bar)
+{
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
+__device__ __forceinline__ void bounded_spin_done(uint64_t* bar, uint32_t parity)
+{
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity) && globaltimer() - t0 < kWaitLimitNs) {
+    }
+}
+
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+__device__ __forceinline__ uint32_t pack2(float2 v) { return pack_bf16x2(v.x, v.y); }
+
+__device__ __forceinline__ void fence_proxy_async_global()
+{
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int* p)
+{
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void red_release_gpu_add(unsigned int* p, unsigned int v)
+{
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d)
+{
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b),
+                 "f"(c), "f"(d)
+                 : "memory");
+}
+
+// fp32 q row cache: [128 rows][16 chunks of 4 floats]; the low 3 bits of the chunk index are
+// XORed with (row & 7) so that 32 rows reading the same chunk hit every bank group
+__device__ __forceinline__ uint32_t qf_chunk(int row, int ch)
+{
+    return uint32_t(row * 256 + ((((ch ^ row) & 7)) | (ch & 8)) * 16);
+}
+
+// MN-major SW128 atom whose N-element 0 is 1 for every K row (the [.; 1] column of [V; 1])
+__device__ __forceinline__ void init_ones_atom(unsigned char* atom)
+{
+    for (int e = threadIdx.x; e < int(kOnesAtomBytes / 4); e += blockDim.x)
+        reinterpret_cast<uint32_t*>(atom)[e] = 0u;
+    __syncthreads();
+    for (int j = threadIdx.x; j < kC; j += blockDim.x)
+        *reinterpret_cast<uint16_t*>(atom + (j >> 3) * 1024 + (j & 7) * 128 + (j & 7) * 16) =
+            kBf16One;
+}
+
+__device__ __forceinline__ void inval_builder_bars(StBars& b)
+{
+    for (int i = 0; i < kKVStages; ++i) {
+        mbar_inval(&b.kv_full[i]);
+        mbar_inval(&b.kv_empty[i]);
+    }
+    for (int i = 0; i < 2; ++i) {
+        mbar_inval(&b.a_full[i]);
+        mbar_inval(&b.a_empty[i]);
+        mbar_inval(&b.acc_full[i]);
+        mbar_inval(&b.acc_empty[i]);
+    }
+    mbar_inval(&b.done);
+}
+
+__device__ __forceinline__ void inval_reader_bars(RdBars& b)
+{
+    mbar_inval(&b.qkv_full);
+    for (int i = 0; i < 2; ++i) {
+        mbar_inval(&b.aq_full[i]);
+        mbar_inval(&b.s_full[i]);
+        mbar_inval(&b.s_empty[i]);
+    }
+    mbar_inval(&b.p_full);
+    for (int i = 0; i < kRdStages; ++i) {
+        mbar_inval(&b.a_full[i]);
+        mbar_inval(&b.b_full[i]);
+        mbar_inval(&b.ab_empty[i]);
+    }
+    mbar_inval(&b.u_full);
+    mbar_inval(&b.done);
+}
+
+// ------------------------------------------------------------------------------------------
+// builder: psi producers (thread = token j of a half chunk, quarter qf of the slab's rows)
+// ------------------------------------------------------------------------------------------
+// MN-major A tile (128 rows x 64 tokens): the 8-row chunk starting at row m for token j
+__device__ __forceinline__ uint32_t st_a_off(int m, int j)
+{
+    return uint32_t((m >> 6) * 8192 + (j >> 3) * 1024 + (j & 7) * 128 +
+                    ((((m & 63) >> 3) ^ (j & 7)) << 4));
+}
+
+// bf16 of the exact product p (kLo = false) or of its rounding remainder p - bf16(p) (true)
+template <bool kLo>
+__device__ __forceinline__ uint32_t psi_pack(float2 p)
+{
+    const uint32_t h = pack2(p);
+    if (!kLo) return h;
+    return pack_bf16x2(p.x - bf16lo_to_f32(h), p.y - bf16hi_to_f32(h));
+}
+
+// off-diagonal slabs: 32 rows = 4 dims a of block R times the 8 dims of block T.  They never
+// involve the constant slot, and K rows past T are zero-filled by the copy.
+template <bool kLo>
+__device__ __forceinline__ void psi_offdiag(const unsigned char* ktile, int trow, uint32_t abase,
+                                            int j, int slab, int qf)
+{
+    int R, T;
+    block_rt(2 * slab + (qf >> 1), R, T);
+    const uint2 wa = *reinterpret_cast<const uint2*>(ktile + kmajor_chunk(trow, R) + 8 * (qf & 1));
+    const uint4 wt = *reinterpret_cast<const uint4*>(ktile + kmajor_chunk(trow, T));
+    const float ka[4] = {bf16lo_to_f32(wa.x), bf16hi_to_f32(wa.x), bf16lo_to_f32(wa.y),
+                         bf16hi_to_f32(wa.y)};
+    const float2 t0 = f2(bf16lo_to_f32(wt.x), bf16hi_to_f32(wt.x));
+    const float2 t1 = f2(bf16lo_to_f32(wt.y), bf16hi_to_f32(wt.y));
+    const float2 t2 = f2(bf16lo_to_f32(wt.z), bf16hi_to_f32(wt.z));
+    const float2 t3 = f2(bf16lo_to_f32(wt.w), bf16hi_to_f32(wt.w));
+    const int m0 = 64 * (qf >> 1) + 32 * (qf & 1);
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+        const float2 xx = f2(ka[a], ka[a]);
+        sts128(abase + st_a_off(m0 + 8 * a, j), psi_pack<kLo>(__fmul2_rn(xx, t0)),
+               psi_pack<kLo>(__fmul2_rn(xx, t1)), psi_pack<kLo>(__fmul2_rn(xx, t2)),
+               psi_pack<kLo>(__fmul2_rn(xx, t3)));
+    }
+}
+
+template <int F0>
+constexpr bool psi_chunk_needed(int ch)
+{
+    for (int i = 0; i < 32; ++i) {
+        const RT rt = feature_rt(F0 + i);
+        if ((rt.r < 64 && rt.r / 8 == ch) || (rt.t < 64 && rt.t / 8 == ch)) return true;
+    }
+    return false;
+}
+
+// diagonal / linear / constant slabs: 32 rows with compile-time (r, t)
+template <int F0, bool kLo>
+__device__ __forceinline__ void psi_static(const unsigned char* ktile, int trow, float one,
+                                           uint32_t abase, int j)
+{
+    float k[66];
+    static_for<8>([&](auto CH) {
+        constexpr int ch = decltype(CH)::value;
+        if constexpr (psi_chunk_needed<F0>(ch)) {
+            const uint4 w = *reinterpret_cast<const uint4*>(ktile + kmajor_chunk(trow, ch));
+            k[ch * 8 + 0] = bf16lo_to_f32(w.x);
+            k[ch * 8 + 1] = bf16hi_to_f32(w.x);
+            k[ch * 8 + 2] = bf16lo_to_f32(w.y);
+            k[ch * 8 + 3] = bf16hi_to_f32(w.y);
+            k[ch * 8 + 4] = bf16lo_to_f32(w.z);
+            k[ch * 8 + 5] = bf16hi_to_f32(w.z);
+            k[ch * 8 + 6] = bf16lo_to_f32(w.w);
+            k[ch * 8 + 7] = bf16hi_to_f32(w.w);
+        }
+    });
+    k[64] = one;
+    k[65] = 0.f;
+    constexpr int m0 = F0 % kSlabRows;
+    static_for<4>([&](auto CH) {
+        constexpr int ch = decltype(CH)::value;
+        uint32_t h[4];
+        static_for<4>([&](auto E) {
+            constexpr int e = decltype(E)::value;
+            constexpr RT a = feature_rt(F0 + ch * 8 + 2 * e);
+            constexpr RT b = feature_rt(F0 + ch * 8 + 2 * e + 1);
+            h[e] = psi_pack<kLo>(f2(k[a.r] * k[a.t], k[b.r] * k[b.t]));
+        });
+        sts128(abase + st_a_off(m0 + 8 * ch, j), h[0], h[1], h[2], h[3]);
+    });
+}
+
+template <bool kLo>
+__device__ __forceinline__ void psi_tile(int slab, int qf, const unsigned char* ktile, int trow,
+                                         float one, uint32_t abase, int j)
+{
+    if (slab < kOffDiagSlices / 2) {
+        psi_offdiag<kLo>(ktile, trow, abase, j, slab, qf);
+        return;
+    }
+    const int sel = (slab - kOffDiagSlices / 2) * 4 + qf;
+    static_for<(kNumSlabs - kOffDiagSlices / 2) * 4>([&](auto I) {
+        constexpr int i = decltype(I)::value;
+        if (sel == i) psi_static<kOffDiagRows + i * 32, kLo>(ktile, trow, one, abase, j);
+    });
+}
+
+// ------------------------------------------------------------------------------------------
+// builder item: chain (kLo = false, chunks [0, NC)) or remainder (kLo = true, chunks
+// [c0, c1)); warps 0-7 psi producers, 8-15 epilogue, 16 TMA, 17 MMA
+// ------------------------------------------------------------------------------------------
+template <bool kLo>
+__device__ void builder_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Params& P,
+                             int bkv, int slab, int c0, int c1)
+{
+    StBars& bar = ctl.bar.st;
+    volatile int* abort_flag = &ctl.abort_flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int NC = P.NC, T = P.T, nch = c1 - c0;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kKVStages; ++i) {
+            mbar_init(&bar.kv_full[i], 1);
+            mbar_init(&bar.kv_empty[i], 8 + 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bar.a_full[i], 8);
+            mbar_init(&bar.a_empty[i], 1);
+            mbar_init(&bar.acc_full[i], 1);
+            mbar_init(&bar.acc_empty[i], 8);
+        }
+        mbar_init(&bar.done, 1);
+        ctl.abort_flag = 0;
+        fence_mbar_init();
+    }
+    init_ones_atom(sm + kStOffOnes);
+    if (!kLo)
+        for (int e = threadIdx.x; e < int(2 * kImgSliceBytes / 4); e += blockDim.x)
+            reinterpret_cast<uint32_t*>(sm + kStOffImg)[e] = 0u;
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    if (warp == kTmaWarp) {
+        if (lane == 0) {
+            int issued = 0;
+            for (int u = 0; u < nch; ++u) {
+                const int c = c0 + u, s = u % kKVStages;
+                if (u >= kKVStages &&
+                    !mbar_wait(&bar.kv_empty[s], ((u / kKVStages) - 1) & 1, abort_flag))
+                    break;
+                unsigned char* kvs = sm + kStOffKV + s * 2 * kTileBytes;
+                mbar_expect_tx(&bar.kv_full[s], 2 * kTileBytes);
+                tma_load_3d(kvs, P.tm_k, &bar.kv_full[s], 0, c * kC, bkv);
+                tma_load_3d(kvs + kTileBytes, P.tm_v, &bar.kv_full[s], 0, c * kC, bkv);
+                ++issued;
+            }
+            for (int u = max(0, issued - kKVStages); u < issued; ++u)
+                bounded_spin_done(&bar.kv_full[u % kKVStages], (u / kKVStages) & 1);
+        }
+        __syncwarp();
+    } else if (warp == kMmaWarp) {
+        if (lane == 0) {
+            constexpr uint32_t id = idesc_bf16(128, 80, true, true);
+            const uint32_t a0 = smem_u32(sm + kStOffA), kv0 = smem_u32(sm + kStOffKV);
+            const uint32_t ones = smem_u32(sm + kStOffOnes);
+            bool ok = true;
+            for (int u = 0; u < nch && ok; ++u) {
+                const int s = kLo ? 0 : (u & 1), st = u % kKVStages;
+                if (!kLo && u >= 2) ok = mbar_wait(&bar.acc_empty[s], ((u >> 1) - 1) & 1, abort_flag);
+                if (ok) ok = mbar_wait(&bar.kv_full[st], (u / kKVStages) & 1, abort_flag);
+                if (!ok) break;
+                const uint32_t d = tmem + s * 128;
+                const uint32_t vt = kv0 + st * 2 * kTileBytes + kTileBytes;
+                const uint32_t lbo = ones - vt;  // V atom -> ones atom (N elements 64..)
+                for (int hc = 0; hc < 2; ++hc) {
+                    const int w = 2 * u + hc, as = w & 1;
+                    if (!(ok = mbar_wait(&bar.a_full[as], (w >> 1) & 1, abort_flag))) break;
+                    tc_fence_after();
+                    const uint32_t ab = a0 + as * kStATile;
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                        const uint32_t acc = (kLo ? (u | hc | ks) : (hc | ks)) ? 1u : 0u;
+                        mma_bf16(d, sdesc_sw128(ab + ks * 2048, 8192, 1024),
+                                 sdesc_sw128(vt + hc * 8192 + ks * 2048, lbo, 1024), id, acc);
+                    }
+                    mma_commit(&bar.a_empty[as]);
+                }
+                if (!ok) break;
+                if (!kLo) mma_commit(&bar.acc_full[s]);
+                mma_commit(&bar.kv_empty[st]);
+            }
+            if (kLo && ok) mma_commit(&bar.acc_full[0]);
+            mma_commit(&bar.done);
+            bounded_spin_done(&bar.done, 0);
+        }
+        __syncwarp();
+    } else if (warp < 8) {
+        const int t = threadIdx.x, j = t & 63, qf = t >> 6;
+        const uint32_t a0 = smem_u32(sm + kStOffA);
+        for (int u = 0; u < nch; ++u) {
+            const int c = c0 + u, st = u % kKVStages;
+            if (!mbar_wait(&bar.kv_full[st], (u / kKVStages) & 1, abort_flag)) break;
+            const unsigned char* kt = sm + kStOffKV + st * 2 * kTileBytes;
+            bool ok = true;
+            for (int hc = 0; hc < 2; ++hc) {
+                const int w = 2 * u + hc, as = w & 1;
+                if (w >= 2 && !mbar_wait(&bar.a_empty[as], ((w >> 1) - 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const int trow = hc * 64 + j;
+                const float one = (c * kC + trow < T) ? 1.f : 0.f;
+                psi_tile<kLo>(slab, qf, kt, trow, one, a0 + as * kStATile, j);
+                fence_proxy_async();
+                warp_arrive(&bar.a_full[as]);
+            }
+            if (!ok) break;
+            warp_arrive(&bar.kv_empty[st]);
+        }
+    } else {
+        // epilogue: thread = (packed row of the slab, column half)
+        const int q4 = warp & 3, hfe = (warp - 8) >> 2;
+        const int fl = q4 * 32 + lane, f = slab * kSlabRows + fl;
+        const int kk = fl & 63;
+        const uint32_t stage = smem_u32(sm + kStOffImg) + (fl >> 6) * kImgSliceBytes;
+        float run[33];
+#pragma unroll
+        for (int n = 0; n < 33; ++n) run[n] = 0.f;
+        const bool leader = (threadIdx.x == 8 * 32);
+        unsigned int* flags = (!kLo && P.flags) ? P.flags + size_t(bkv) * NC : nullptr;
+        const int rounds = kLo ? 1 : nch;
+        for (int u = 0; u < rounds; ++u) {
+            const int c = c0 + u, s = kLo ? 0 : (u & 1);
+            if (!kLo && c >= 1) {
+                // exclusive prefix S_c -> bf16 K-major image [80 n][64 rows] -> bulk store
+                if (leader) {
+                    if (flags && c >= 2) {
+                        bulk_wait0();  // image c-1 is in global memory: publish it
+                        fence_proxy_async_global();
+                        red_release_gpu_add(flags + (c - 1), 1u);
+                    } else {
+                        bulk_wait_read0();
+                    }
+                }
+                named_bar_sync(1, 256);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int n = 32 * hfe + i;
+                    asm volatile("st.shared.b16 [%0], %1;" ::"r"(stage + kmajor_off(n, kk)),
+                                 "h"(__bfloat16_as_ushort(__float2bfloat16_rn(run[i])))
+                                 : "memory");
+                }
+                if (hfe == 1)
+                    asm volatile("st.shared.b16 [%0], %1;" ::"r"(stage + kmajor_off(64, kk)),
+                                 "h"(__bfloat16_as_ushort(__float2bfloat16_rn(run[32])))
+                                 : "memory");
+                fence_proxy_async();
+                named_bar_sync(1, 256);
+                if (leader) {
+                    unsigned char* dst = P.img + (size_t(bkv) * NC + c) * kImgChunkBytes +
+                                         size_t(2 * slab) * kImgSliceBytes;
+                    bulk_s2g(dst, sm + kStOffImg, 2 * kImgSliceBytes);
+                    bulk_commit();
+                }
+            }
+            // all epilogue threads leave together, so no named barrier is left half-joined
+            const bool got = mbar_wait(&bar.acc_full[s], kLo ? 0 : ((u >> 1) & 1), abort_flag);
+            if (!named_bar_and(2, 256, got)) break;
+            tc_fence_after();
+            const uint32_t lanebase = tmem + (uint32_t(q4 * 32) << 16) + s * 128;
+            float v0[16], v1[16], vz[16];
+            tmem_ld16(lanebase + hfe * 32, v0);
+            tmem_ld16(lanebase + hfe * 32 + 16, v1);
+            tmem_ld16(lanebase + 64, vz);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                run[i] += v0[i];
+                run[16 + i] += v1[i];
+            }
+            if (hfe == 1) run[32] += vz[0];
+            tc_fence_before();
+            if (!kLo) warp_arrive(&bar.acc_empty[s]);
+        }
+        if (!*abort_flag) {
+            // fp32 sums into the final state (chain and remainders add into a zeroed body)
+            float* unit = P.body + size_t(bkv) * kFP * kW;
+            float* hv = unit + size_t(f) * kDV + hfe * 32;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                red_add_v4(hv + 4 * i, run[4 * i], run[4 * i + 1], run[4 * i + 2], run[4 * i + 3]);
+            if (hfe == 1) atomicAdd(unit + size_t(kFP) * kDV + f, run[32]);
+        }
+        if (leader && !kLo) {
+            bulk_wait0();
+            if (flags && NC >= 2 && !*abort_flag) {
+                fence_proxy_async_global();
+                red_release_gpu_add(flags + (NC - 1), 1u);
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// reader: phi producers (thread = query row; one slice = 64 packed rows = 32 TMEM columns)
+// ------------------------------------------------------------------------------------------
+// off-diagonal slice s = block (R, T): rows (8R + a, 8T + b), a, b = 0..7
+__device__ __forceinline__ void phi_offdiag(const unsigned char* qf, const float* coef, int s,
+                                            int row, uint32_t (&w)[32])
+{
+    int R, T;
+    block_rt(s, R, T);
+    const float4 r0 = *reinterpret_cast<const float4*>(qf + qf_chunk(row, 2 * R));
+    const float4 r1 = *reinterpret_cast<const float4*>(qf + qf_chunk(row, 2 * R + 1));
+    const float4 t0 = *reinterpret_cast<const float4*>(qf + qf_chunk(row, 2 * T));
+    const float4 t1 = *reinterpret_cast<const float4*>(qf + qf_chunk(row, 2 * T + 1));
+    const float qa[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+    const float* cf = coef + 64 * s;
+#pragma unroll
+    for (int a = 0; a < 8; ++a) {
+        const float4 c0 = *reinterpret_cast<const float4*>(cf + 8 * a);
+        const float4 c1 = *reinterpret_cast<const float4*>(cf + 8 * a + 4);
+        const float2 xx = f2(qa[a], qa[a]);
+        w[4 * a + 0] = pack2(__fmul2_rn(__fmul2_rn(xx, f2(t0.x, t0.y)), f2(c0.x, c0.y)));
+        w[4 * a + 1] = pack2(__fmul2_rn(__fmul2_rn(xx, f2(t0.z, t0.w)), f2(c0.z, c0.w)));
+        w[4 * a + 2] = pack2(__fmul2_rn(__fmul2_rn(xx, f2(t1.x, t1.y)), f2(c1.x, c1.y)));
+        w[4 * a + 3] = pack2(__fmul2_rn(__fmul2_rn(xx, f2(t1.z, t1.w)), f2(c1.z, c1.w)));
+    }
+}
+
+template <int F0>
+constexpr bool phi_chunk_needed(int ch)  // 4-float chunk of the q row
+{
+    for (int i = 0; i < 64; ++i) {
+        const RT rt = feature_rt(F0 + i);
+        if ((rt.r < 64 && rt.r / 4 == ch) || (rt.t < 64 && rt.t / 4 == ch)) return true;
+    }
+    return false;
+}
+
+// diagonal / linear / constant slices: 64 rows with compile-time (r, t)
+template <int F0>
+__device__ __forceinline__ void phi_static(const unsigned char* qf, const float* coef, int row,
+                                           uint32_t (&w)[32])
+{
+    float q[66];
+    static_for<16>([&](auto CH) {
+        constexpr int ch = decltype(CH)::value;
+        if constexpr (phi_chunk_needed<F0>(ch)) {
+            const float4 v = *reinterpret_cast<const float4*>(qf + qf_chunk(row, ch));
+            q[4 * ch + 0] = v.x;
+            q[4 * ch + 1] = v.y;
+            q[4 * ch + 2] = v.z;
+            q[4 * ch + 3] = v.w;
+        }
+    });
+    q[64] = 1.f;
+    q[65] = 0.f;
+    static_for<8>([&](auto X) {
+        constexpr int x = decltype(X)::value;
+        const float4 c0 = *reinterpret_cast<const float4*>(coef + F0 + 8 * x);
+        const float4 c1 = *reinterpret_cast<const float4*>(coef + F0 + 8 * x + 4);
+        const float cf[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        static_for<4>([&](auto E) {
+            constexpr int e = decltype(E)::value;
+            constexpr RT a = feature_rt(F0 + 8 * x + 2 * e);
+            constexpr RT b = feature_rt(F0 + 8 * x + 2 * e + 1);
+            w[4 * x + e] =
+                pack_bf16x2(cf[2 * e] * (q[a.r] * q[a.t]), cf[2 * e + 1] * (q[b.r] * q[b.t]));
+        });
+    });
+}
+
+__device__ __forceinline__ void phi_diag(const unsigned char* qf, const float* coef, int s,
+                                         int row, uint32_t (&w)[32])
+{
+    const int sel = s - kOffDiagSlices;
+    static_for<kSlices - kOffDiagSlices>([&](auto I) {
+        constexpr int i = decltype(I)::value;
+        if (sel == i) phi_static<kOffDiagRows + i * 64>(qf, coef, row, w);
+    });
+}
+
+// ------------------------------------------------------------------------------------------
+// reader item: (bh, chunk c)
+//   warps 0-7: phi (slice parity = warp >> 2, row quarter = warp & 3)
+//   warps 8-15: intra-chunk kernel (row quarter = warp & 3, key half = (warp >> 2) & 1)
+//   warp 16: TMA, warp 17: MMA
+// ------------------------------------------------------------------------------------------
+__device__ void reader_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Params& P, int bh,
+                            int c)
+{
+    RdBars& bar = ctl.bar.rd;
+    volatile int* abort_flag = &ctl.abort_flag;
+    const int Hq = P.Hq, Hkv = P.Hkv, T = P.T, NC = P.NC;
+    const int b = bh / Hq, h = bh % Hq, kv = h / (Hq / Hkv), bkv = b * Hkv + kv;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float* coef = reinterpret_cast<float*>(sm + kRdOffCoef);
+    float* wch = reinterpret_cast<float*>(sm + kRdOffW);
+    float* c0 = reinterpret_cast<float*>(sm + kRdOffC0);
+    const bool has_inter = c > 0;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bar.qkv_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bar.aq_full[i], 8);
+            mbar_init(&bar.s_full[i], 1);
+            mbar_init(&bar.s_empty[i], 8);
+        }
+        mbar_init(&bar.p_full, 8);
+        for (int i = 0; i < kRdStages; ++i) {
+            mbar_init(&bar.a_full[i], 4);
+            mbar_init(&bar.b_full[i], 1);
+            mbar_init(&bar.ab_empty[i], 1);
+        }
+        mbar_init(&bar.u_full, 1);
+        mbar_init(&bar.done, 1);
+        ctl.abort_flag = 0;
+        int Gh = P.G[h];
+        if (Gh < 1 || Gh > kGMax) {
+            raise_error(OAL_ERR_GROUPS);
+            Gh = Gh < 1 ? 1 : kGMax;
+        }
+        ctl.G = Gh;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const int G = ctl.G;
+    if (warp == kTmaWarp && lane == 0) {
+        // tiles and the coefficient table first: they do not depend on the setup below
+        mbar_expect_tx(&bar.qkv_full, 3 * kTileBytes + kFP * 4);
+        tma_load_3d(sm + kRdOffQ, P.tm_q, &bar.qkv_full, 0, c * kC, bh);
+        tma_load_3d(sm + kRdOffK, P.tm_k, &bar.qkv_full, 0, c * kC, bkv);
+        tma_load_3d(sm + kRdOffV, P.tm_v, &bar.qkv_full, 0, c * kC, bkv);
+        bulk_g2s(coef, P.coef_all + size_t(h) * kFP, kFP * 4, &bar.qkv_full);
+    }
+    init_ones_atom(sm + kRdOffOnes);
+    for (int e = threadIdx.x; e < kGM1 * 64; e += blockDim.x) {
+        const int m = e >> 6, r = e & 63;
+        int g = P.gid[h * kD + r];
+        if (g < 1 || g > G) {
+            raise_error(OAL_ERR_GROUPS);
+            g = g < 1 ? 1 : G;
+        }
+        wch[e] = (m <= G) ? P.L[size_t(h) * kGM1 * kGM1 + g * kGM1 + m] * 0.125f : 0.f;
+    }
+    if (threadIdx.x < kGM1) c0[threadIdx.x] = P.L[size_t(h) * kGM1 * kGM1 + threadIdx.x];
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    if (warp == kTmaWarp) {
+        if (lane == 0) {
+            int issued = 0;
+            bool ok = true;
+            if (has_inter && P.flags) {
+                // every slab of this chunk's state image must be in global memory
+                const unsigned int* fl = P.flags + size_t(bkv) * NC + c;
+                const uint64_t t0 = globaltimer();
+                while (ld_acquire_gpu(fl) < unsigned(kNumSlabs)) {
+                    if (*abort_flag || globaltimer() - t0 > kWaitLimitNs) {
+                        *abort_flag = 1;
+                        raise_error(OAL_ERR_TIMEOUT);
+                        ok = false;
+                        break;
+                    }
+                    __nanosleep(64);
+                }
+                fence_proxy_async_global();
+            }
+            if (has_inter && ok) {
+                const unsigned char* src = P.img + (size_t(bkv) * NC + c) * kImgChunkBytes;
+                for (int s = 0; s < kSlices; ++s) {
+                    const int bs = s % kRdStages;
+                    if (s >= kRdStages &&
+                        !mbar_wait(&bar.ab_empty[bs], ((s / kRdStages) - 1) & 1, abort_flag))
+                        break;
+                    mbar_expect_tx(&bar.b_full[bs], kImgSliceBytes);
+                    bulk_g2s(sm + kRdOffB + bs * kImgSliceBytes, src + size_t(s) * kImgSliceBytes,
+                             kImgSliceBytes, &bar.b_full[bs]);
+                    ++issued;
+                }
+            }
+            bounded_spin_done(&bar.qkv_full, 0);
+            for (int s = max(0, issued - kRdStages); s < issued; ++s)
+                bounded_spin_done(&bar.b_full[s % kRdStages], (s / kRdStages) & 1);
+        }
+        __syncwarp();
+    } else if (warp == kMmaWarp) {
+        if (lane == 0) {
+            constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);
+            constexpr uint32_t id_u = idesc_bf16(128, 80, false, false);   // A in TMEM, B K-major
+            constexpr uint32_t id_pv = idesc_bf16(128, 80, false, true);   // B = [V | ones] MN
+            const uint32_t aq0 = smem_u32(sm + kRdOffAq), kt = smem_u32(sm + kRdOffK);
+            const uint32_t vt = smem_u32(sm + kRdOffV), ones = smem_u32(sm + kRdOffOnes);
+            const uint32_t b0 = smem_u32(sm + kRdOffB);
+            auto score = [&](int m) -> bool {
+                const int sb = m & 1;
+                if (!mbar_wait(&bar.aq_full[sb], (m >> 1) & 1, abort_flag)) return false;
+                if (m >= 2 && !mbar_wait(&bar.s_empty[sb], ((m >> 1) - 1) & 1, abort_flag))
+                    return false;
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16(tmem + kColS0 + sb * 128,
+                             sdesc_sw128(aq0 + sb * kTileBytes + ks * 32, 16, 1024),
+                             sdesc_sw128(kt + ks * 32, 16, 1024), id_s, ks > 0 ? 1u : 0u);
+                mma_commit(&bar.s_full[sb]);
+                return true;
+            };
+            bool ok = mbar_wait(&bar.qkv_full, 0, abort_flag);
+            if (ok) ok = score(0) && score(1);
+            // inter-chunk readout phi(Q_c) S_c: A from TMEM, B = state image (K-major, N=80)
+            for (int s = 0; s < kSlices && ok && has_inter; ++s) {
+                const int st = s % kRdStages;
+                ok = mbar_wait(&bar.a_full[st], (s / kRdStages) & 1, abort_flag) &&
+                     mbar_wait(&bar.b_full[st], (s / kRdStages) & 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t bs = b0 + st * kImgSliceBytes;
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16_ts(tmem + kColU, tmem + kColA0 + st * 32 + ks * 8,
+                                sdesc_sw128(bs + ks * 32, 16, 1024), id_u, (s | ks) ? 1u : 0u);
+                mma_commit(&bar.ab_empty[st]);
+            }
+            for (int m = 2; m <= G && ok; ++m) ok = score(m);
+            if (ok) ok = mbar_wait(&bar.p_full, 0, abort_flag);
+            if (ok) {
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t acc = (has_inter || ks > 0) ? 1u : 0u;
+                    mma_bf16(tmem + kColU,
+                             sdesc_sw128(aq0 + (ks >> 2) * kTileBytes + (ks & 3) * 32, 16, 1024),
+                             sdesc_sw128(vt + ks * 2048, ones - vt, 1024), id_pv, acc);
+                }
+                mma_commit(&bar.u_full);
+            }
+            mma_commit(&bar.done);
+            bounded_spin_done(&bar.done, 0);
+        }
+        __syncwarp();
+    } else {
+        const int qw = warp & 3, row = qw * 32 + lane;
+        const unsigned char* qf = sm + kRdOffQf;
+        bool ok = mbar_wait(&bar.qkv_full, 0, abort_flag);
+        if (ok) {
+            // bf16 Q tile -> fp32 row cache: 16 warps, dims [16p, 16p+16) of each row
+            const int p = warp >> 2;
+            const uint32_t qf0 = smem_u32(sm + kRdOffQf);
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                const uint4 w = *reinterpret_cast<const uint4*>(sm + kRdOffQ +
+                                                                kmajor_chunk(row, 2 * p + x));
+                const int ch = 4 * p + 2 * x;
+                sts128(qf0 + qf_chunk(row, ch), __float_as_uint(bf16lo_to_f32(w.x)),
+                       __float_as_uint(bf16hi_to_f32(w.x)), __float_as_uint(bf16lo_to_f32(w.y)),
+                       __float_as_uint(bf16hi_to_f32(w.y)));
+                sts128(qf0 + qf_chunk(row, ch + 1), __float_as_uint(bf16lo_to_f32(w.z)),
+                       __float_as_uint(bf16hi_to_f32(w.z)), __float_as_uint(bf16lo_to_f32(w.w)),
+                       __float_as_uint(bf16hi_to_f32(w.w)));
+            }
+        }
+        named_bar_sync(1, 16 * 32);  // q cache complete
+
+        if (warp < 8) {
+            // ---- phi producers: slices of parity sg, written into TMEM A stages ----
+            const int sg = warp >> 2;
+            const uint32_t lanebase = tmem + (uint32_t(qw * 32) << 16);
+            for (int s = sg; s < kSlices && ok && has_inter; s += 2) {
+                const int st = s % kRdStages;
+                uint32_t w[32];
+                if (s < kOffDiagSlices) phi_offdiag(qf, coef, s, row, w);
+                else phi_diag(qf, coef, s, row, w);
+                if (s >= kRdStages &&
+                    !mbar_wait(&bar.ab_empty[st], ((s / kRdStages) - 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                tmem_st32(lanebase + kColA0 + st * 32, w);
+                tmem_st_wait();
+                tc_fence_before();
+                warp_arrive(&bar.a_full[st]);
+            }
+        } else {
+            // ---- intra-chunk kernel: keys [64hf, 64hf+64) of this row ----
+            const int hf = (warp >> 2) & 1;
+            const uint32_t aq0 = smem_u32(sm + kRdOffAq);
+            auto produce_half = [&](auto HFC, int m) {
+                constexpr int H = decltype(HFC)::value;
+                const uint32_t base = aq0 + (m & 1) * kTileBytes;
+                const float* w = wch + m * 64 + 32 * H;
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const float4 qa = *reinterpret_cast<const float4*>(qf + qf_chunk(row, 8 * H + 2 * x));
+                    const float4 qb =
+                        *reinterpret_cast<const float4*>(qf + qf_chunk(row, 8 * H + 2 * x + 1));
+                    const float4 wa = *reinterpret_cast<const float4*>(w + 8 * x);
+                    const float4 wb = *reinterpret_cast<const float4*>(w + 8 * x + 4);
+                    sts128(base + kmajor_chunk(row, 4 * H + x),
+                           pack2(__fmul2_rn(f2(qa.x, qa.y), f2(wa.x, wa.y))),
+                           pack2(__fmul2_rn(f2(qa.z, qa.w), f2(wa.z, wa.w))),
+                           pack2(__fmul2_rn(f2(qb.x, qb.y), f2(wb.x, wb.y))),
+                           pack2(__fmul2_rn(f2(qb.z, qb.w), f2(wb.z, wb.w))));
+                }
+            };
+            auto produce_aq = [&](int m) {
+                if (hf == 0) produce_half(std::integral_constant<int, 0>{}, m);
+                else produce_half(std::integral_constant<int, 1>{}, m);
+                fence_proxy_async();
+                warp_arrive(&bar.aq_full[m & 1]);
+            };
+            if (ok) {
+                produce_aq(0);
+                produce_aq(1);
+            }
+            const bool live = !(hf == 1 && qw < 2);  // keys 64..127 vs rows 0..63: all masked
+            float acc[64];
+#pragma unroll
+            for (int jj = 0; jj < 64; ++jj) acc[jj] = 0.f;
+            for (int m = 0; m <= G && ok; ++m) {
+                const int sb = m & 1;
+                if (!mbar_wait(&bar.s_full[sb], (m >> 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (live) {
+                    const float cm = c0[m];
+                    const uint32_t taddr =
+                        tmem + (uint32_t(qw * 32) << 16) + kColS0 + sb * 128 + 64 * hf;
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        float v[16];
+                        tmem_ld16(taddr + 16 * x, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 16; i += 2) {
+                            const float2 t = __fadd2_rn(f2(cm, cm), f2(v[i], v[i + 1]));
+                            const float2 a =
+                                __ffma2_rn(t, t, f2(acc[16 * x + i], acc[16 * x + i + 1]));
+                            acc[16 * x + i] = a.x;
+                            acc[16 * x + i + 1] = a.y;
+                        }
+                    }
+                }
+                tc_fence_before();
+                warp_arrive(&bar.s_empty[sb]);
+                if (m + 2 <= G) produce_aq(m + 2);
+            }
+            if (ok) {
+                // P tile (K-major, 2 K-atoms over the 128 keys; aliases Aq0 | Aq1)
+#pragma unroll
+                for (int x = 0; x < 8; ++x) {
+                    uint32_t wv[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int j0 = 64 * hf + 8 * x + 2 * e;
+                        const float k0 = (j0 <= row) ? P.eps + acc[8 * x + 2 * e] : 0.f;
+                        const float k1 = (j0 + 1 <= row) ? P.eps + acc[8 * x + 2 * e + 1] : 0.f;
+                        wv[e] = pack_bf16x2(k0, k1);
+                    }
+                    sts128(aq0 + hf * kTileBytes + kmajor_chunk(row, x), wv[0], wv[1], wv[2],
+                           wv[3]);
+                }
+                fence_proxy_async();
+                warp_arrive(&bar.p_full);
+            }
+            // epilogue: yhat = u[:64] / u[64], columns [32hf, 32hf+32) of this row
+            if (ok) ok = mbar_wait(&bar.u_full, 0, abort_flag);
+            if (ok) {
+                tc_fence_after();
+                const uint32_t taddr = tmem + (uint32_t(qw * 32) << 16) + kColU;
+                float u0[16], u1[16], dz[16];
+                tmem_ld16(taddr + 32 * hf, u0);
+                tmem_ld16(taddr + 32 * hf + 16, u1);
+                tmem_ld16(taddr + 64, dz);
+                tmem_ld_wait();
+                const int irow = c * kC + row;
+                if (irow < T) {
+                    const float inv = 1.f / dz[0];
+                    float4* o = reinterpret_cast<float4*>(P.out + (size_t(bh) * T + irow) * kDV +
+                                                          32 * hf);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        o[i] = make_float4(u0[4 * i] * inv, u0[4 * i + 1] * inv,
+                                           u0[4 * i + 2] * inv, u0[4 * i + 3] * inv);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        o[4 + i] = make_float4(u1[4 * i] * inv, u1[4 * i + 1] * inv,
+                                               u1[4 * i + 2] * inv, u1[4 * i + 3] * inv);
+                }
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// kernels: 0 = builders (grid 17 x B*Hkv x (1 + nseg): z = 0 chain, z > 0 remainder segment
+// z - 1), 1 = readers (grid NC x B*Hq), 2 = persistent queue over all items
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ void run_builder(unsigned char* sm, Ctl& ctl, uint32_t tmem,
+                                            const Params& P, int bkv, int slab, int seg)
+{
+    if (seg < 0) {
+        builder_item<false>(sm, ctl, tmem, P, bkv, slab, 0, P.NC);
+    } else {
+        const int c0 = seg * kSegChunks, c1 = min(P.NC, c0 + kSegChunks);
+        builder_item<true>(sm, ctl, tmem, P, bkv, slab, c0, c1);
+    }
+}
+
+template <int kMode>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, Params P)
+{
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* sm = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Ctl& ctl = *reinterpret_cast<Ctl*>(sm + kOffCtl);
+    const int warp = threadIdx.x >> 5;
+    P.tm_q = &tm_q;
+    P.tm_k = &tm_k;
+    P.tm_v = &tm_v;
+
+    if (warp == kMmaWarp) {
+        tmem_alloc(&ctl.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl.tmem_base;
+
+    if (kMode == 0) {
+        run_builder(sm, ctl, tmem, P, blockIdx.y, blockIdx.x, int(blockIdx.z) - 1);
+    } else if (kMode == 1) {
+        reader_item(sm, ctl, tmem, P, blockIdx.y, blockIdx.x);
+    } else {
+        // per batch element: chain builders, then readers (chunk-major), then remainders
+        const int nb = P.Hkv * kNumSlabs, nr = P.Hq * P.NC, nl = nb * P.nseg;
+        const int per_b = nb + nr + nl, total = P.B * per_b;
+        while (true) {
+            if (threadIdx.x == 0) ctl.item = int(atomicAdd(P.queue, 1u));
+            __syncthreads();
+            const int item = ctl.item;
+            if (item >= total) break;
+            const int b = item / per_b, r = item % per_b;
+            int kind;
+            if (r < nb) {
+                kind = 0;
+                run_builder(sm, ctl, tmem, P, b * P.Hkv + r / kNumSlabs, r % kNumSlabs, -1);
+            } else if (r < nb + nr) {
+                kind = 1;
+                const int rr = r - nb;
+                reader_item(sm, ctl, tmem, P, b * P.Hq + rr % P.Hq, rr / P.Hq);
+            } else {
+                kind = 0;
+                const int rr = r - nb - nr, unit = rr % nb;
+                run_builder(sm, ctl, tmem, P, b * P.Hkv + unit / kNumSlabs, unit % kNumSlabs,
+                            rr / nb);
+            }
+            tc_fence_before();
+            __syncthreads();
+            tc_fence_after();
+            // the barrier memory is reused by the next item (possibly of the other kind)
+            if (threadIdx.x == 0) {
+                if (kind == 0) inval_builder_bars(ctl.bar.st);
+                else inval_reader_bars(ctl.bar.rd);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace tc
+
+// ------------------------------------------------------------------------------------------
+// host side: tensor maps and launch
+// ------------------------------------------------------------------------------------------
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// [heads][T][64] bf16 viewed as 3D {64, T, heads}; box {64, 128, 1}; 128B swizzle; rows past
+// T read as zero.
+bool make_map(CUtensorMap* m, const void* base, int T, int heads)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {64, cuuint64_t(T), cuuint64_t(heads)};
+    const cuuint64_t strides[2] = {64 * 2, cuuint64_t(T) * 64 * 2};
+    const cuuint32_t box[3] = {64, tc::kC, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return n;
+}
+
+}  // namespace
+
+size_t tc_image_bytes(int B, int Hkv, int T)
+{
+    const size_t NC = size_t((T + tc::kC - 1) / tc::kC);
+    return size_t(B) * Hkv * NC * tc::kImgChunkBytes;
+}
+
+size_t tc_workspace_bytes(int B, int Hkv, int T)
+{
+    const size_t NC = size_t((T + tc::kC - 1) / tc::kC);
+    return tc_image_bytes(B, Hkv, T) + align256((size_t(B) * Hkv * NC + 1) * 4);
+}
+
+int launch_prefill_tc(const void* q, const void* k, const void* v, const int32_t* gid,
+                      const float* L, const int32_t* G, float eps, float* out, void* state,
+                      void* ws, int B, int T, int Hq, int Hkv, bool fused, cudaStream_t st)
+{
+    if (B == 0) return OAL_OK;
+    const int NC = (T + tc::kC - 1) / tc::kC;
+    unsigned char* sb = static_cast<unsigned char*>(state);
+    float* body = reinterpret_cast<float*>(sb + kHeaderBytes + coef_bytes(Hq));
+    // chain builders and remainder items add their sums into the final state
+    OAL_CUDA_TRY(cudaMemsetAsync(body, 0, size_t(B) * Hkv * state_unit_bytes(), st));
+    if (T == 0) return OAL_OK;
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, q, T, B * Hq) || !make_map(&mk, k, T, B * Hkv) ||
+        !make_map(&mv, v, T, B * Hkv))
+        return OAL_ERR_CUDA;
+    unsigned char* wsb = static_cast<unsigned char*>(ws);
+    tc::Params P{};
+    P.gid = gid;
+    P.L = L;
+    P.G = G;
+    P.eps = eps;
+    P.coef_all = reinterpret_cast<const float*>(sb + kHeaderBytes);
+    P.img = wsb;
+    P.body = body;
+    P.out = out;
+    P.B = B;
+    P.Hq = Hq;
+    P.Hkv = Hkv;
+    P.T = T;
+    P.NC = NC;
+    P.nseg = (NC + tc::kSegChunks - 1) / tc::kSegChunks;
+    unsigned int* ctl = reinterpret_cast<unsigned int*>(wsb + tc_image_bytes(B, Hkv, T));
+    const size_t ctl_words = size_t(B) * Hkv * NC + 1;
+    if (fused) {
+        const int items = B * (Hkv * tc::kNumSlabs * (1 + P.nseg) + Hq * NC);
+        const int grid = std::min(sm_count(), items);
+        if (grid > 0 &&
+            cudaFuncSetAttribute(tc::prefill_tc_kernel<2>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(tc::kSmemBytes)) == cudaSuccess &&
+            cudaMemsetAsync(ctl, 0, ctl_words * 4, st) == cudaSuccess) {
+            P.queue = ctl;
+            P.flags = ctl + 1;
+            cudaLaunchConfig_t cfg{};
+            cfg.gridDim = dim3(grid);
+            cfg.blockDim = dim3(tc::kThreads);
+            cfg.dynamicSmemBytes = tc::kSmemBytes;
+            cfg.stream = st;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident at once
+            attr[0].val.cooperative = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            LaunchScope ls("prefill_tc", st);
+            if (cudaLaunchKernelEx(&cfg, tc::prefill_tc_kernel<2>, mq, mk, mv, P) == cudaSuccess)
+                return OAL_OK;
+        }
+        cudaGetLastError();  // not launchable as one resident grid: use the two-kernel form
+        P.queue = nullptr;
+        P.flags = nullptr;
+    }
+    {
+        OAL_CUDA_TRY(cudaFuncSetAttribute(tc::prefill_tc_kernel<0>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(tc::kSmemBytes)));
+        LaunchScope ls("state_tc", st);
+        tc::prefill_tc_kernel<0><<<dim3(tc::kNumSlabs, B * Hkv, 1 + P.nseg), tc::kThreads,
+                                   tc::kSmemBytes, st>>>(mq, mk, mv, P);
+        OAL_LAUNCH_CHECK();
+    }
+    {
+        OAL_CUDA_TRY(cudaFuncSetAttribute(tc::prefill_tc_kernel<1>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(tc::kSmemBytes)));
+        LaunchScope ls("readout_tc", st);
+        tc::prefill_tc_kernel<1><<<dim3(NC, B * Hq), tc::kThreads, tc::kSmemBytes, st>>>(
+            mq, mk, mv, P);
+        OAL_LAUNCH_CHECK();
+    }
+    return OAL_OK;
+}
+
+}  // namespace oal

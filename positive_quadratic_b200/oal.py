@@ -41,7 +41,10 @@ class KernelStat(ctypes.Structure):
 class OALError(RuntimeError):
     def __init__(self, code: int, what: str = ""):
         self.code = code
-        super().__init__(f"{what}: {STATUS.get(code, code)} ({status_string(code)})")
+        msg = f"{what}: {STATUS.get(code, code)} ({status_string(code)})"
+        if code == -6:
+            msg += f" [{last_cuda_error()}]"
+        super().__init__(msg)
 
 
 _lock = threading.Lock()
@@ -69,6 +72,10 @@ def lib() -> ctypes.CDLL:
             L.oal_dense_ref_gpu.argtypes = [_VP] * 6 + [ctypes.c_float, _VP, _PS, _VP]
             L.oal_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), _VP]
             L.oal_launch_count.restype = ctypes.c_ulonglong
+            L.oal_last_cuda_error.argtypes = [ctypes.c_char_p, ctypes.c_size_t]
+            L.oal_last_cuda_error.restype = ctypes.c_int
+            L.oal_set_prefill_fused.argtypes = [ctypes.c_int]
+            L.oal_set_prefill_fused.restype = ctypes.c_int
             L.oal_profile_enable.argtypes = [ctypes.c_int]
             L.oal_profile_enable.restype = ctypes.c_int
             L.oal_profile_read.argtypes = [ctypes.POINTER(KernelStat), ctypes.c_int,
@@ -87,6 +94,16 @@ def declared_symbols(header: str = HEADER):
     text = open(header).read()
     return sorted(set(re.findall(r"^\s*(?:int|const char\*|unsigned long long)\s+(oal_\w+)\s*\(",
                                  text, re.M)))
+
+
+def last_cuda_error() -> str:
+    """Name and description of the CUDA error behind the most recent OAL_ERR_CUDA."""
+    try:
+        buf = ctypes.create_string_buffer(256)
+        lib().oal_last_cuda_error(buf, 256)
+        return buf.value.decode()
+    except Exception:
+        return "?"
 
 
 def status_string(code: int) -> str:
@@ -273,3 +290,9 @@ def profile_read() -> dict:
     _check(lib().oal_profile_read(arr, 64, ctypes.byref(n)), "oal_profile_read")
     return {arr[i].name.decode(): (int(arr[i].launches), float(arr[i].total_ms))
             for i in range(n.value)}
+
+
+def set_prefill_fused(fused: bool) -> bool:
+    """Select the tensor-core prefill schedule (persistent fused kernel or two kernels);
+    returns the previous setting."""
+    return bool(lib().oal_set_prefill_fused(1 if fused else 0))

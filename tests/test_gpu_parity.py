@@ -247,3 +247,40 @@ def test_config4_decode_sampled(oal, cuda):
         ref = oracle.recurrent(s.q, s.k, s.v, s.group_id, s.L, s.G, s.eps)
         for n, t in enumerate(range(4096, 4100)):
             assert row_rel_err(ys[n][b:b + 1], ref[:, :, t]) <= TOL_BF16, (b, t)
+
+
+# --- tensor-core prefill schedules --------------------------------------------------------------
+
+@pytest.mark.parametrize("fused", [True, False])
+@pytest.mark.parametrize("T,B", [(129, 1), (300, 2), (1000, 3), (2048, 1)])
+def test_tensor_prefill_schedules(oal, cuda, fused, T, B):
+    """bf16, chunk 128 runs on the tcgen05 kernels: persistent fused schedule and the
+    two-kernel schedule both match the oracle (outputs and exact final state)."""
+    p = I.small_layer(500 + T, B=B, T=T, Hq=14, Hkv=2, dtype="bf16")
+    ref, st = oracle.recurrent(p.q, p.k, p.v, p.group_id, p.L, p.G, p.eps, return_state=True)
+    prev = oal.set_prefill_fused(fused)
+    try:
+        oal.profile_read()
+        oal.profile_enable(True)
+        y, state = gpu_prefill(oal, p, cuda, 128)
+        oal.profile_enable(False)
+        names = set(oal.profile_read())
+    finally:
+        oal.set_prefill_fused(prev)
+    assert ("prefill_tc" in names) if fused else ({"state_tc", "readout_tc"} <= names), names
+    assert row_rel_err(y, ref) <= TOL_BF16
+    _, _, S = read_state(state.cpu().numpy(), B, 14, 2)
+    refS = pack_oracle_state(st)
+    assert np.max(np.abs(S[:, :, :F] - refS) / np.abs(refS).max(axis=2, keepdims=True)) < 1e-5
+
+
+def test_tensor_schedules_agree(oal, cuda):
+    p = I.config1()
+    prev = oal.set_prefill_fused(True)
+    try:
+        y1, _ = gpu_prefill(oal, p, cuda, 128)
+        oal.set_prefill_fused(False)
+        y2, _ = gpu_prefill(oal, p, cuda, 128)
+    finally:
+        oal.set_prefill_fused(prev)
+    np.testing.assert_array_equal(y1, y2)
