@@ -51,6 +51,7 @@ constexpr int kSlices = kFP / 64;                          // 34 readout K-slice
 constexpr int kOffDiagSlices = kOffDiagRows / 64;          // 28
 constexpr int kSegChunks = 8;                              // chunks per remainder item
 constexpr uint32_t kImgSliceBytes = 80 * 64 * 2;           // K-major [80 n][64 rows]
+constexpr uint32_t kImgLoadBytes = 65 * 128;               // rows 0..64 (65..79 are zero)
 constexpr size_t kImgChunkBytes = size_t(kSlices) * kImgSliceBytes;
 constexpr uint32_t kTileBytes = kC * 64 * 2;               // 16384: one 128 x 64 bf16 tile
 constexpr uint32_t kOnesAtomBytes = kC * 128;              // 16384: 128 rows x 128 B
@@ -68,31 +69,36 @@ static_assert(kFP % kSlabRows == 0 && kFP % 64 == 0, "feature padding");
 // reader
 constexpr uint32_t kRdOffK = 0;           // K tile (score B operand, K-major)
 constexpr uint32_t kRdOffV = 16384;       // V tile (PV B operand, MN-major)
-constexpr uint32_t kRdOffQ = 32768;       // Q tile (bf16)
-constexpr uint32_t kRdOffQf = 49152;      // fp32 q rows [128][64], 16-byte chunks swizzled
-constexpr uint32_t kRdOffAq = 81920;      // Aq0 | Aq1 (score A operands); P tile aliases
-constexpr uint32_t kRdOffB = 114688;      // 4 x 10 KB state-image stages
-constexpr uint32_t kRdOffOnes = 155648;   // 16 KB ones atom
-constexpr uint32_t kRdOffCoef = 172032;   // 2176 fp32
-constexpr uint32_t kRdOffW = 180736;      // 9 x 64 fp32
-constexpr uint32_t kRdOffC0 = 183040;     // 9 fp32
+constexpr uint32_t kRdOffQ = 32768;       // Q tile (bf16, K-major): phi and Aq read it
+constexpr uint32_t kRdOffAq = 49152;      // Aq0 | Aq1 (score A operands); the P tile aliases
+constexpr uint32_t kRdOffB = 81920;       // 8 x 10 KB state-image stages
+constexpr uint32_t kRdOffCoef = 180224;   // 2176 fp32 coefficients
+constexpr uint32_t kRdOffCoefH = 188928;  // 1792 bf16 coefficients of the off-diagonal rows
+constexpr uint32_t kRdOffW = 192512;      // 9 x 64 fp32
+constexpr uint32_t kRdOffC0 = 194816;     // 9 fp32
 // builder
 constexpr uint32_t kStOffKV = 0;          // 4 x (K 16 KB + V 16 KB)
 constexpr uint32_t kStOffA = 131072;      // 2 x 16 KB psi stages
-constexpr uint32_t kStOffOnes = 163840;   // 16 KB ones atom
-constexpr uint32_t kStOffImg = 180224;    // 2 slices x 10 KB staging
+constexpr uint32_t kStOffImg = 180224;    // 2 buffers x 2 slices x 10 KB image staging
 // both
-constexpr uint32_t kOffCtl = 219392;      // barriers and control words
-constexpr uint32_t kSmemBytes = kOffCtl + 512 + 1024;
+constexpr uint32_t kOffOnes = 163840;     // 16 KB ones atom, written once per CTA
+constexpr uint32_t kOffCtl = 221184;      // barriers and control words
+constexpr uint32_t kSmemBytes = kOffCtl + 1024 + 1024;
 
-constexpr int kRdStages = 4;
+constexpr int kPhiSets = 4;                                // reader warps (w >> 2) per slice
+constexpr int kRdStages = 12;                              // phi stages (TMEM)
+constexpr int kBStages = 8;                                // state-image stages (SMEM)
 constexpr int kKVStages = 4;
 constexpr uint32_t kStATile = 64 * kSlabRows * 2;          // 64 tokens x 128 rows = 16 KB
-constexpr uint32_t kColU = 0, kColS0 = 128, kColA0 = 384;  // reader TMEM map
+// reader TMEM map: U in [0, 80); score tiles S0 | S1 in [128, 384) during the intra-chunk
+// phase; phi stages of 32 columns in [128, 512) during the inter-chunk phase
+constexpr uint32_t kColU = 0, kColS0 = 128, kColA0 = 128;
+static_assert(kColA0 + 32 * kRdStages <= kTmemCols, "phi stages");
+static_assert(kRdStages % kPhiSets == 0, "a stage belongs to one phi set");
 
 struct RdBars {
     uint64_t qkv_full, aq_full[2], s_full[2], s_empty[2], p_full;
-    uint64_t a_full[kRdStages], b_full[kRdStages], ab_empty[kRdStages];
+    uint64_t a_full[kRdStages], a_empty[kRdStages], b_full[kBStages], b_empty[kBStages];
     uint64_t u_full, done;
 };
 struct StBars {
@@ -103,14 +109,16 @@ struct Ctl {
     union {
         RdBars rd;
         StBars st;
-        uint64_t raw[32];
+        uint64_t raw[64];
     } bar;
     uint32_t tmem_base;
     int abort_flag;
     int item;
     int G;
 };
-static_assert(sizeof(Ctl) <= 512, "control block");
+static_assert(sizeof(Ctl) <= 1024, "control block");
+static_assert(sizeof(RdBars) <= sizeof(uint64_t) * 64 && sizeof(StBars) <= sizeof(uint64_t) * 64,
+              "barrier block");
 
 struct Params {
     const CUtensorMap* tm_q;
@@ -195,13 +203,6 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
                  : "memory");
 }
 
-// fp32 q row cache: [128 rows][16 chunks of 4 floats]; the low 3 bits of the chunk index are
-// XORed with (row & 7) so that 32 rows reading the same chunk hit every bank group
-__device__ __forceinline__ uint32_t qf_chunk(int row, int ch)
-{
-    return uint32_t(row * 256 + ((((ch ^ row) & 7)) | (ch & 8)) * 16);
-}
-
 // MN-major SW128 atom whose N-element 0 is 1 for every K row (the [.; 1] column of [V; 1])
 __device__ __forceinline__ void init_ones_atom(unsigned char* atom)
 {
@@ -239,8 +240,11 @@ __device__ __forceinline__ void inval_reader_bars(RdBars& b)
     mbar_inval(&b.p_full);
     for (int i = 0; i < kRdStages; ++i) {
         mbar_inval(&b.a_full[i]);
+        mbar_inval(&b.a_empty[i]);
+    }
+    for (int i = 0; i < kBStages; ++i) {
         mbar_inval(&b.b_full[i]);
-        mbar_inval(&b.ab_empty[i]);
+        mbar_inval(&b.b_empty[i]);
     }
     mbar_inval(&b.u_full);
     mbar_inval(&b.done);
@@ -380,10 +384,9 @@ __device__ void builder_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const P
         ctl.abort_flag = 0;
         fence_mbar_init();
     }
-    init_ones_atom(sm + kStOffOnes);
     if (!kLo)
-        for (int e = threadIdx.x; e < int(2 * kImgSliceBytes / 4); e += blockDim.x)
-            reinterpret_cast<uint32_t*>(sm + kStOffImg)[e] = 0u;
+        for (int e = threadIdx.x; e < int(4 * kImgSliceBytes / 16); e += blockDim.x)
+            reinterpret_cast<uint4*>(sm + kStOffImg)[e] = make_uint4(0u, 0u, 0u, 0u);
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
@@ -411,7 +414,7 @@ __device__ void builder_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const P
         if (lane == 0) {
             constexpr uint32_t id = idesc_bf16(128, 80, true, true);
             const uint32_t a0 = smem_u32(sm + kStOffA), kv0 = smem_u32(sm + kStOffKV);
-            const uint32_t ones = smem_u32(sm + kStOffOnes);
+            const uint32_t ones = smem_u32(sm + kOffOnes);
             bool ok = true;
             for (int u = 0; u < nch && ok; ++u) {
                 const int s = kLo ? 0 : (u & 1), st = u % kKVStages;
@@ -471,7 +474,7 @@ __device__ void builder_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const P
         const int q4 = warp & 3, hfe = (warp - 8) >> 2;
         const int fl = q4 * 32 + lane, f = slab * kSlabRows + fl;
         const int kk = fl & 63;
-        const uint32_t stage = smem_u32(sm + kStOffImg) + (fl >> 6) * kImgSliceBytes;
+        const uint32_t stage0 = smem_u32(sm + kStOffImg) + (fl >> 6) * kImgSliceBytes;
         float run[33];
 #pragma unroll
         for (int n = 0; n < 33; ++n) run[n] = 0.f;
@@ -481,14 +484,17 @@ __device__ void builder_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const P
         for (int u = 0; u < rounds; ++u) {
             const int c = c0 + u, s = kLo ? 0 : (u & 1);
             if (!kLo && c >= 1) {
-                // exclusive prefix S_c -> bf16 K-major image [80 n][64 rows] -> bulk store
-                if (leader) {
-                    if (flags && c >= 2) {
-                        bulk_wait0();  // image c-1 is in global memory: publish it
+                // exclusive prefix S_c -> bf16 K-major image [80 n][64 rows] -> bulk store,
+                // staged in buffer c & 1.  That buffer last held image c - 2: wait for its
+                // store only (image c - 1 stays in flight), then publish image c - 2.
+                const uint32_t stage = stage0 + (c & 1) * 2 * kImgSliceBytes;
+                if (leader && c >= 3) {
+                    if (flags) {
+                        bulk_wait1();
                         fence_proxy_async_global();
-                        red_release_gpu_add(flags + (c - 1), 1u);
+                        red_release_gpu_add(flags + (c - 2), 1u);
                     } else {
-                        bulk_wait_read0();
+                        bulk_wait_read1();
                     }
                 }
                 named_bar_sync(1, 256);
@@ -508,7 +514,8 @@ __device__ void builder_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const P
                 if (leader) {
                     unsigned char* dst = P.img + (size_t(bkv) * NC + c) * kImgChunkBytes +
                                          size_t(2 * slab) * kImgSliceBytes;
-                    bulk_s2g(dst, sm + kStOffImg, 2 * kImgSliceBytes);
+                    bulk_s2g(dst, sm + kStOffImg + (c & 1) * 2 * kImgSliceBytes,
+                             2 * kImgSliceBytes);
                     bulk_commit();
                 }
             }
@@ -542,9 +549,10 @@ __device__ void builder_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const P
         }
         if (leader && !kLo) {
             bulk_wait0();
-            if (flags && NC >= 2 && !*abort_flag) {
+            if (flags && !*abort_flag) {
+                // the last two images (the loop published images up to NC - 3)
                 fence_proxy_async_global();
-                red_release_gpu_add(flags + (NC - 1), 1u);
+                for (int c = max(1, NC - 2); c < NC; ++c) red_release_gpu_add(flags + c, 1u);
             }
         }
     }
@@ -553,54 +561,75 @@ __device__ void builder_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const P
 // ------------------------------------------------------------------------------------------
 // reader: phi producers (thread = query row; one slice = 64 packed rows = 32 TMEM columns)
 // ------------------------------------------------------------------------------------------
-// off-diagonal slice s = block (R, T): rows (8R + a, 8T + b), a, b = 0..7
-__device__ __forceinline__ void phi_offdiag(const unsigned char* qf, const float* coef, int s,
+// (R, T) of the 28 off-diagonal 8 x 8 blocks (R < T, lexicographic), as 8 R + T
+#define OAL_BLOCK_RT                                                                       \
+    1, 2, 3, 4, 5, 6, 7, 10, 11, 12, 13, 14, 15, 19, 20, 21, 22, 23, 28, 29, 30, 31, 37, 38, \
+        39, 46, 47, 55
+constexpr uint8_t kBlockRT[kOffDiagSlices] = {OAL_BLOCK_RT};
+__constant__ uint8_t c_block_rt[kOffDiagSlices] = {OAL_BLOCK_RT};
+#undef OAL_BLOCK_RT
+constexpr bool block_rt_table_ok()
+{
+    for (int s = 0; s < kOffDiagSlices; ++s) {
+        const RT rt = feature_rt(64 * s);
+        if (rt.r != 8 * (kBlockRT[s] >> 3) || rt.t != 8 * (kBlockRT[s] & 7)) return false;
+    }
+    return true;
+}
+static_assert(block_rt_table_ok(), "off-diagonal block table");
+
+// off-diagonal slice s = block (R, T): rows (8R + a, 8T + b), a, b = 0..7.  Packed bf16
+// arithmetic: phi = bf16(bf16(q_r q_t) c) with c rounded to bf16 -- three roundings of 2^-9,
+// the same order as the bf16 operand rounding the tensor core sees anyway, and no fp32 ->
+// bf16 conversions (which issue at a quarter of the FMA rate).
+__device__ __forceinline__ void phi_offdiag(const unsigned char* qt, const uint32_t* coefh, int s,
                                             int row, uint32_t (&w)[32])
 {
-    int R, T;
-    block_rt(s, R, T);
-    const float4 r0 = *reinterpret_cast<const float4*>(qf + qf_chunk(row, 2 * R));
-    const float4 r1 = *reinterpret_cast<const float4*>(qf + qf_chunk(row, 2 * R + 1));
-    const float4 t0 = *reinterpret_cast<const float4*>(qf + qf_chunk(row, 2 * T));
-    const float4 t1 = *reinterpret_cast<const float4*>(qf + qf_chunk(row, 2 * T + 1));
-    const float qa[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-    const float* cf = coef + 64 * s;
+    const int rt = c_block_rt[s];
+    const uint4 qr = *reinterpret_cast<const uint4*>(qt + kmajor_chunk(row, rt >> 3));
+    const uint4 qc = *reinterpret_cast<const uint4*>(qt + kmajor_chunk(row, rt & 7));
+    const uint32_t rr[4] = {qr.x, qr.y, qr.z, qr.w};
+    const uint32_t* cf = coefh + 32 * s;
 #pragma unroll
     for (int a = 0; a < 8; ++a) {
-        const float4 c0 = *reinterpret_cast<const float4*>(cf + 8 * a);
-        const float4 c1 = *reinterpret_cast<const float4*>(cf + 8 * a + 4);
-        const float2 xx = f2(qa[a], qa[a]);
-        w[4 * a + 0] = pack2(__fmul2_rn(__fmul2_rn(xx, f2(t0.x, t0.y)), f2(c0.x, c0.y)));
-        w[4 * a + 1] = pack2(__fmul2_rn(__fmul2_rn(xx, f2(t0.z, t0.w)), f2(c0.z, c0.w)));
-        w[4 * a + 2] = pack2(__fmul2_rn(__fmul2_rn(xx, f2(t1.x, t1.y)), f2(c1.x, c1.y)));
-        w[4 * a + 3] = pack2(__fmul2_rn(__fmul2_rn(xx, f2(t1.z, t1.w)), f2(c1.z, c1.w)));
+        const uint32_t xa = (a & 1) ? dup_hi(rr[a >> 1]) : dup_lo(rr[a >> 1]);
+        const uint4 c = *reinterpret_cast<const uint4*>(cf + 4 * a);
+        w[4 * a + 0] = bmul2(bmul2(xa, qc.x), c.x);
+        w[4 * a + 1] = bmul2(bmul2(xa, qc.y), c.y);
+        w[4 * a + 2] = bmul2(bmul2(xa, qc.z), c.z);
+        w[4 * a + 3] = bmul2(bmul2(xa, qc.w), c.w);
     }
 }
 
 template <int F0>
-constexpr bool phi_chunk_needed(int ch)  // 4-float chunk of the q row
+constexpr bool phi_chunk_needed(int ch)  // 8-dim chunk of the q row
 {
     for (int i = 0; i < 64; ++i) {
         const RT rt = feature_rt(F0 + i);
-        if ((rt.r < 64 && rt.r / 4 == ch) || (rt.t < 64 && rt.t / 4 == ch)) return true;
+        if ((rt.r < 64 && rt.r / 8 == ch) || (rt.t < 64 && rt.t / 8 == ch)) return true;
     }
     return false;
 }
 
-// diagonal / linear / constant slices: 64 rows with compile-time (r, t)
+// diagonal / linear / constant slices: 64 rows with compile-time (r, t); fp32 products,
+// one rounding
 template <int F0>
-__device__ __forceinline__ void phi_static(const unsigned char* qf, const float* coef, int row,
+__device__ __forceinline__ void phi_static(const unsigned char* qt, const float* coef, int row,
                                            uint32_t (&w)[32])
 {
     float q[66];
-    static_for<16>([&](auto CH) {
+    static_for<8>([&](auto CH) {
         constexpr int ch = decltype(CH)::value;
         if constexpr (phi_chunk_needed<F0>(ch)) {
-            const float4 v = *reinterpret_cast<const float4*>(qf + qf_chunk(row, ch));
-            q[4 * ch + 0] = v.x;
-            q[4 * ch + 1] = v.y;
-            q[4 * ch + 2] = v.z;
-            q[4 * ch + 3] = v.w;
+            const uint4 v = *reinterpret_cast<const uint4*>(qt + kmajor_chunk(row, ch));
+            q[8 * ch + 0] = bf16lo_to_f32(v.x);
+            q[8 * ch + 1] = bf16hi_to_f32(v.x);
+            q[8 * ch + 2] = bf16lo_to_f32(v.y);
+            q[8 * ch + 3] = bf16hi_to_f32(v.y);
+            q[8 * ch + 4] = bf16lo_to_f32(v.z);
+            q[8 * ch + 5] = bf16hi_to_f32(v.z);
+            q[8 * ch + 6] = bf16lo_to_f32(v.w);
+            q[8 * ch + 7] = bf16hi_to_f32(v.w);
         }
     });
     q[64] = 1.f;
@@ -620,21 +649,23 @@ __device__ __forceinline__ void phi_static(const unsigned char* qf, const float*
     });
 }
 
-__device__ __forceinline__ void phi_diag(const unsigned char* qf, const float* coef, int s,
+__device__ __forceinline__ void phi_diag(const unsigned char* qt, const float* coef, int s,
                                          int row, uint32_t (&w)[32])
 {
     const int sel = s - kOffDiagSlices;
     static_for<kSlices - kOffDiagSlices>([&](auto I) {
         constexpr int i = decltype(I)::value;
-        if (sel == i) phi_static<kOffDiagRows + i * 64>(qf, coef, row, w);
+        if (sel == i) phi_static<kOffDiagRows + i * 64>(qt, coef, row, w);
     });
 }
 
 // ------------------------------------------------------------------------------------------
-// reader item: (bh, chunk c)
-//   warps 0-7: phi (slice parity = warp >> 2, row quarter = warp & 3)
-//   warps 8-15: intra-chunk kernel (row quarter = warp & 3, key half = (warp >> 2) & 1)
-//   warp 16: TMA, warp 17: MMA
+// reader item: (bh, chunk c).  Warps 0-15 (row quarter qw = w & 3, set kq = w >> 2):
+//   intra-chunk phase: Aq tiles (dims [16 kq, 16 kq + 16)), kappa over keys
+//   [32 kq, 32 kq + 32) of score tiles S_0..S_G, P tile;
+//   inter-chunk phase: phi of slices s = kq (mod 4) into TMEM stages;
+//   epilogue: yhat columns [16 kq, 16 kq + 16).
+// Warp 16: TMA, warp 17: MMA (S_0..S_G, then P [V; 1], then the 34 readout slices).
 // ------------------------------------------------------------------------------------------
 __device__ void reader_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Params& P, int bh,
                             int c)
@@ -645,6 +676,7 @@ __device__ void reader_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Pa
     const int b = bh / Hq, h = bh % Hq, kv = h / (Hq / Hkv), bkv = b * Hkv + kv;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     float* coef = reinterpret_cast<float*>(sm + kRdOffCoef);
+    uint32_t* coefh = reinterpret_cast<uint32_t*>(sm + kRdOffCoefH);
     float* wch = reinterpret_cast<float*>(sm + kRdOffW);
     float* c0 = reinterpret_cast<float*>(sm + kRdOffC0);
     const bool has_inter = c > 0;
@@ -652,15 +684,18 @@ __device__ void reader_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Pa
     if (threadIdx.x == 0) {
         mbar_init(&bar.qkv_full, 1);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&bar.aq_full[i], 8);
+            mbar_init(&bar.aq_full[i], 16);
             mbar_init(&bar.s_full[i], 1);
-            mbar_init(&bar.s_empty[i], 8);
+            mbar_init(&bar.s_empty[i], 16);
         }
-        mbar_init(&bar.p_full, 8);
+        mbar_init(&bar.p_full, 16);
         for (int i = 0; i < kRdStages; ++i) {
             mbar_init(&bar.a_full[i], 4);
+            mbar_init(&bar.a_empty[i], 1);
+        }
+        for (int i = 0; i < kBStages; ++i) {
             mbar_init(&bar.b_full[i], 1);
-            mbar_init(&bar.ab_empty[i], 1);
+            mbar_init(&bar.b_empty[i], 1);
         }
         mbar_init(&bar.u_full, 1);
         mbar_init(&bar.done, 1);
@@ -683,7 +718,12 @@ __device__ void reader_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Pa
         tma_load_3d(sm + kRdOffV, P.tm_v, &bar.qkv_full, 0, c * kC, bkv);
         bulk_g2s(coef, P.coef_all + size_t(h) * kFP, kFP * 4, &bar.qkv_full);
     }
-    init_ones_atom(sm + kRdOffOnes);
+    // state-image stages: N rows 65..79 are never loaded and must read as zero
+    for (int e = threadIdx.x; e < int(kBStages * 15 * 8); e += blockDim.x) {
+        const int st = e / 120, x = e % 120;
+        reinterpret_cast<uint4*>(sm + kRdOffB + st * kImgSliceBytes + kImgLoadBytes)[x] =
+            make_uint4(0u, 0u, 0u, 0u);
+    }
     for (int e = threadIdx.x; e < kGM1 * 64; e += blockDim.x) {
         const int m = e >> 6, r = e & 63;
         int g = P.gid[h * kD + r];
@@ -721,19 +761,19 @@ __device__ void reader_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Pa
             if (has_inter && ok) {
                 const unsigned char* src = P.img + (size_t(bkv) * NC + c) * kImgChunkBytes;
                 for (int s = 0; s < kSlices; ++s) {
-                    const int bs = s % kRdStages;
-                    if (s >= kRdStages &&
-                        !mbar_wait(&bar.ab_empty[bs], ((s / kRdStages) - 1) & 1, abort_flag))
+                    const int bs = s % kBStages;
+                    if (s >= kBStages &&
+                        !mbar_wait(&bar.b_empty[bs], ((s / kBStages) - 1) & 1, abort_flag))
                         break;
-                    mbar_expect_tx(&bar.b_full[bs], kImgSliceBytes);
+                    mbar_expect_tx(&bar.b_full[bs], kImgLoadBytes);
                     bulk_g2s(sm + kRdOffB + bs * kImgSliceBytes, src + size_t(s) * kImgSliceBytes,
-                             kImgSliceBytes, &bar.b_full[bs]);
+                             kImgLoadBytes, &bar.b_full[bs]);
                     ++issued;
                 }
             }
             bounded_spin_done(&bar.qkv_full, 0);
-            for (int s = max(0, issued - kRdStages); s < issued; ++s)
-                bounded_spin_done(&bar.b_full[s % kRdStages], (s / kRdStages) & 1);
+            for (int s = max(0, issued - kBStages); s < issued; ++s)
+                bounded_spin_done(&bar.b_full[s % kBStages], (s / kBStages) & 1);
         }
         __syncwarp();
     } else if (warp == kMmaWarp) {
@@ -742,13 +782,15 @@ __device__ void reader_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Pa
             constexpr uint32_t id_u = idesc_bf16(128, 80, false, false);   // A in TMEM, B K-major
             constexpr uint32_t id_pv = idesc_bf16(128, 80, false, true);   // B = [V | ones] MN
             const uint32_t aq0 = smem_u32(sm + kRdOffAq), kt = smem_u32(sm + kRdOffK);
-            const uint32_t vt = smem_u32(sm + kRdOffV), ones = smem_u32(sm + kRdOffOnes);
+            const uint32_t vt = smem_u32(sm + kRdOffV), ones = smem_u32(sm + kOffOnes);
             const uint32_t b0 = smem_u32(sm + kRdOffB);
-            auto score = [&](int m) -> bool {
+            bool ok = mbar_wait(&bar.qkv_full, 0, abort_flag);
+            // grouped score tiles S_m = (Q o w_m) K^T, double-buffered in TMEM
+            for (int m = 0; m <= G && ok; ++m) {
                 const int sb = m & 1;
-                if (!mbar_wait(&bar.aq_full[sb], (m >> 1) & 1, abort_flag)) return false;
-                if (m >= 2 && !mbar_wait(&bar.s_empty[sb], ((m >> 1) - 1) & 1, abort_flag))
-                    return false;
+                ok = mbar_wait(&bar.aq_full[sb], (m >> 1) & 1, abort_flag);
+                if (ok && m >= 2) ok = mbar_wait(&bar.s_empty[sb], ((m >> 1) - 1) & 1, abort_flag);
+                if (!ok) break;
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
@@ -756,192 +798,162 @@ __device__ void reader_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Pa
                              sdesc_sw128(aq0 + sb * kTileBytes + ks * 32, 16, 1024),
                              sdesc_sw128(kt + ks * 32, 16, 1024), id_s, ks > 0 ? 1u : 0u);
                 mma_commit(&bar.s_full[sb]);
-                return true;
-            };
-            bool ok = mbar_wait(&bar.qkv_full, 0, abort_flag);
-            if (ok) ok = score(0) && score(1);
-            // inter-chunk readout phi(Q_c) S_c: A from TMEM, B = state image (K-major, N=80)
-            for (int s = 0; s < kSlices && ok && has_inter; ++s) {
-                const int st = s % kRdStages;
-                ok = mbar_wait(&bar.a_full[st], (s / kRdStages) & 1, abort_flag) &&
-                     mbar_wait(&bar.b_full[st], (s / kRdStages) & 1, abort_flag);
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t bs = b0 + st * kImgSliceBytes;
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ts(tmem + kColU, tmem + kColA0 + st * 32 + ks * 8,
-                                sdesc_sw128(bs + ks * 32, 16, 1024), id_u, (s | ks) ? 1u : 0u);
-                mma_commit(&bar.ab_empty[st]);
             }
-            for (int m = 2; m <= G && ok; ++m) ok = score(m);
+            // intra-chunk term: U = P [V | 1]
             if (ok) ok = mbar_wait(&bar.p_full, 0, abort_flag);
             if (ok) {
                 tc_fence_after();
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t acc = (has_inter || ks > 0) ? 1u : 0u;
+                for (int ks = 0; ks < 8; ++ks)
                     mma_bf16(tmem + kColU,
                              sdesc_sw128(aq0 + (ks >> 2) * kTileBytes + (ks & 3) * 32, 16, 1024),
-                             sdesc_sw128(vt + ks * 2048, ones - vt, 1024), id_pv, acc);
-                }
-                mma_commit(&bar.u_full);
+                             sdesc_sw128(vt + ks * 2048, ones - vt, 1024), id_pv,
+                             ks > 0 ? 1u : 0u);
             }
+            // inter-chunk readout U += phi(Q_c) S_c: A from TMEM, B = state image (K-major)
+            for (int s = 0; s < kSlices && ok && has_inter; ++s) {
+                const int st = s % kRdStages, bsi = s % kBStages;
+                ok = mbar_wait(&bar.a_full[st], (s / kRdStages) & 1, abort_flag) &&
+                     mbar_wait(&bar.b_full[bsi], (s / kBStages) & 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t bs = b0 + bsi * kImgSliceBytes;
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16_ts(tmem + kColU, tmem + kColA0 + st * 32 + ks * 8,
+                                sdesc_sw128(bs + ks * 32, 16, 1024), id_u, 1u);
+                mma_commit(&bar.a_empty[st]);
+                mma_commit(&bar.b_empty[bsi]);
+            }
+            if (ok) mma_commit(&bar.u_full);
             mma_commit(&bar.done);
             bounded_spin_done(&bar.done, 0);
         }
         __syncwarp();
     } else {
-        const int qw = warp & 3, row = qw * 32 + lane;
-        const unsigned char* qf = sm + kRdOffQf;
+        const int qw = warp & 3, kq = warp >> 2, row = qw * 32 + lane;
+        const unsigned char* qt = sm + kRdOffQ;
+        const uint32_t aq0 = smem_u32(sm + kRdOffAq);
+        const uint32_t lanebase = tmem + (uint32_t(qw * 32) << 16);
         bool ok = mbar_wait(&bar.qkv_full, 0, abort_flag);
-        if (ok) {
-            // bf16 Q tile -> fp32 row cache: 16 warps, dims [16p, 16p+16) of each row
-            const int p = warp >> 2;
-            const uint32_t qf0 = smem_u32(sm + kRdOffQf);
+
+        // ---- intra-chunk phase ----
+        // Aq_m = Q o w_m (bf16, K-major); this warp writes dims [16 kq, 16 kq + 16)
+        auto produce_aq = [&](int m) {
+            const uint32_t base = aq0 + (m & 1) * kTileBytes;
+            const float* w = wch + m * 64;
 #pragma unroll
             for (int x = 0; x < 2; ++x) {
-                const uint4 w = *reinterpret_cast<const uint4*>(sm + kRdOffQ +
-                                                                kmajor_chunk(row, 2 * p + x));
-                const int ch = 4 * p + 2 * x;
-                sts128(qf0 + qf_chunk(row, ch), __float_as_uint(bf16lo_to_f32(w.x)),
-                       __float_as_uint(bf16hi_to_f32(w.x)), __float_as_uint(bf16lo_to_f32(w.y)),
-                       __float_as_uint(bf16hi_to_f32(w.y)));
-                sts128(qf0 + qf_chunk(row, ch + 1), __float_as_uint(bf16lo_to_f32(w.z)),
-                       __float_as_uint(bf16hi_to_f32(w.z)), __float_as_uint(bf16lo_to_f32(w.w)),
-                       __float_as_uint(bf16hi_to_f32(w.w)));
+                const int ch = 2 * kq + x;
+                const uint4 qv = *reinterpret_cast<const uint4*>(qt + kmajor_chunk(row, ch));
+                const float4 wa = *reinterpret_cast<const float4*>(w + 8 * ch);
+                const float4 wb = *reinterpret_cast<const float4*>(w + 8 * ch + 4);
+                sts128(base + kmajor_chunk(row, ch),
+                       pack2(__fmul2_rn(f2(bf16lo_to_f32(qv.x), bf16hi_to_f32(qv.x)), f2(wa.x, wa.y))),
+                       pack2(__fmul2_rn(f2(bf16lo_to_f32(qv.y), bf16hi_to_f32(qv.y)), f2(wa.z, wa.w))),
+                       pack2(__fmul2_rn(f2(bf16lo_to_f32(qv.z), bf16hi_to_f32(qv.z)), f2(wb.x, wb.y))),
+                       pack2(__fmul2_rn(f2(bf16lo_to_f32(qv.w), bf16hi_to_f32(qv.w)), f2(wb.z, wb.w))));
             }
+            fence_proxy_async();
+            warp_arrive(&bar.aq_full[m & 1]);
+        };
+        if (ok) {
+            // bf16 copy of the off-diagonal coefficients (read in the inter-chunk phase)
+            for (int i = threadIdx.x; i < kOffDiagRows / 2; i += 16 * 32)
+                coefh[i] = pack_bf16x2(coef[2 * i], coef[2 * i + 1]);
+            produce_aq(0);
+            if (G >= 1) produce_aq(1);
         }
-        named_bar_sync(1, 16 * 32);  // q cache complete
-
-        if (warp < 8) {
-            // ---- phi producers: slices of parity sg, written into TMEM A stages ----
-            const int sg = warp >> 2;
-            const uint32_t lanebase = tmem + (uint32_t(qw * 32) << 16);
-            for (int s = sg; s < kSlices && ok && has_inter; s += 2) {
-                const int st = s % kRdStages;
-                uint32_t w[32];
-                if (s < kOffDiagSlices) phi_offdiag(qf, coef, s, row, w);
-                else phi_diag(qf, coef, s, row, w);
-                if (s >= kRdStages &&
-                    !mbar_wait(&bar.ab_empty[st], ((s / kRdStages) - 1) & 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                tmem_st32(lanebase + kColA0 + st * 32, w);
-                tmem_st_wait();
-                tc_fence_before();
-                warp_arrive(&bar.a_full[st]);
+        const bool live = kq <= qw;  // keys [32 kq, 32 kq + 32) vs rows [32 qw, 32 qw + 32)
+        float acc[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc[j] = 0.f;
+        for (int m = 0; m <= G && ok; ++m) {
+            const int sb = m & 1;
+            if (!mbar_wait(&bar.s_full[sb], (m >> 1) & 1, abort_flag)) {
+                ok = false;
+                break;
             }
-        } else {
-            // ---- intra-chunk kernel: keys [64hf, 64hf+64) of this row ----
-            const int hf = (warp >> 2) & 1;
-            const uint32_t aq0 = smem_u32(sm + kRdOffAq);
-            auto produce_half = [&](auto HFC, int m) {
-                constexpr int H = decltype(HFC)::value;
-                const uint32_t base = aq0 + (m & 1) * kTileBytes;
-                const float* w = wch + m * 64 + 32 * H;
-#pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                    const float4 qa = *reinterpret_cast<const float4*>(qf + qf_chunk(row, 8 * H + 2 * x));
-                    const float4 qb =
-                        *reinterpret_cast<const float4*>(qf + qf_chunk(row, 8 * H + 2 * x + 1));
-                    const float4 wa = *reinterpret_cast<const float4*>(w + 8 * x);
-                    const float4 wb = *reinterpret_cast<const float4*>(w + 8 * x + 4);
-                    sts128(base + kmajor_chunk(row, 4 * H + x),
-                           pack2(__fmul2_rn(f2(qa.x, qa.y), f2(wa.x, wa.y))),
-                           pack2(__fmul2_rn(f2(qa.z, qa.w), f2(wa.z, wa.w))),
-                           pack2(__fmul2_rn(f2(qb.x, qb.y), f2(wb.x, wb.y))),
-                           pack2(__fmul2_rn(f2(qb.z, qb.w), f2(wb.z, wb.w))));
-                }
-            };
-            auto produce_aq = [&](int m) {
-                if (hf == 0) produce_half(std::integral_constant<int, 0>{}, m);
-                else produce_half(std::integral_constant<int, 1>{}, m);
-                fence_proxy_async();
-                warp_arrive(&bar.aq_full[m & 1]);
-            };
-            if (ok) {
-                produce_aq(0);
-                produce_aq(1);
-            }
-            const bool live = !(hf == 1 && qw < 2);  // keys 64..127 vs rows 0..63: all masked
-            float acc[64];
-#pragma unroll
-            for (int jj = 0; jj < 64; ++jj) acc[jj] = 0.f;
-            for (int m = 0; m <= G && ok; ++m) {
-                const int sb = m & 1;
-                if (!mbar_wait(&bar.s_full[sb], (m >> 1) & 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                if (live) {
-                    const float cm = c0[m];
-                    const uint32_t taddr =
-                        tmem + (uint32_t(qw * 32) << 16) + kColS0 + sb * 128 + 64 * hf;
-#pragma unroll
-                    for (int x = 0; x < 4; ++x) {
-                        float v[16];
-                        tmem_ld16(taddr + 16 * x, v);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int i = 0; i < 16; i += 2) {
-                            const float2 t = __fadd2_rn(f2(cm, cm), f2(v[i], v[i + 1]));
-                            const float2 a =
-                                __ffma2_rn(t, t, f2(acc[16 * x + i], acc[16 * x + i + 1]));
-                            acc[16 * x + i] = a.x;
-                            acc[16 * x + i + 1] = a.y;
-                        }
-                    }
-                }
-                tc_fence_before();
-                warp_arrive(&bar.s_empty[sb]);
-                if (m + 2 <= G) produce_aq(m + 2);
-            }
-            if (ok) {
-                // P tile (K-major, 2 K-atoms over the 128 keys; aliases Aq0 | Aq1)
-#pragma unroll
-                for (int x = 0; x < 8; ++x) {
-                    uint32_t wv[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int j0 = 64 * hf + 8 * x + 2 * e;
-                        const float k0 = (j0 <= row) ? P.eps + acc[8 * x + 2 * e] : 0.f;
-                        const float k1 = (j0 + 1 <= row) ? P.eps + acc[8 * x + 2 * e + 1] : 0.f;
-                        wv[e] = pack_bf16x2(k0, k1);
-                    }
-                    sts128(aq0 + hf * kTileBytes + kmajor_chunk(row, x), wv[0], wv[1], wv[2],
-                           wv[3]);
-                }
-                fence_proxy_async();
-                warp_arrive(&bar.p_full);
-            }
-            // epilogue: yhat = u[:64] / u[64], columns [32hf, 32hf+32) of this row
-            if (ok) ok = mbar_wait(&bar.u_full, 0, abort_flag);
-            if (ok) {
-                tc_fence_after();
-                const uint32_t taddr = tmem + (uint32_t(qw * 32) << 16) + kColU;
-                float u0[16], u1[16], dz[16];
-                tmem_ld16(taddr + 32 * hf, u0);
-                tmem_ld16(taddr + 32 * hf + 16, u1);
-                tmem_ld16(taddr + 64, dz);
+            tc_fence_after();
+            if (live) {
+                const float cm = c0[m];
+                const uint32_t taddr = lanebase + kColS0 + sb * 128 + 32 * kq;
+                float v[32];
+                tmem_ld16(taddr, *reinterpret_cast<float(*)[16]>(&v[0]));
+                tmem_ld16(taddr + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
                 tmem_ld_wait();
-                const int irow = c * kC + row;
-                if (irow < T) {
-                    const float inv = 1.f / dz[0];
-                    float4* o = reinterpret_cast<float4*>(P.out + (size_t(bh) * T + irow) * kDV +
-                                                          32 * hf);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        o[i] = make_float4(u0[4 * i] * inv, u0[4 * i + 1] * inv,
-                                           u0[4 * i + 2] * inv, u0[4 * i + 3] * inv);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        o[4 + i] = make_float4(u1[4 * i] * inv, u1[4 * i + 1] * inv,
-                                               u1[4 * i + 2] * inv, u1[4 * i + 3] * inv);
+                for (int i = 0; i < 32; i += 2) {
+                    const float2 t = __fadd2_rn(f2(cm, cm), f2(v[i], v[i + 1]));
+                    const float2 a = __ffma2_rn(t, t, f2(acc[i], acc[i + 1]));
+                    acc[i] = a.x;
+                    acc[i + 1] = a.y;
                 }
+            }
+            tc_fence_before();
+            warp_arrive(&bar.s_empty[sb]);
+            if (m + 2 <= G) produce_aq(m + 2);
+        }
+        if (ok) {
+            // P tile (K-major, 2 K-atoms over the 128 keys; aliases Aq0 | Aq1): keys
+            // [32 kq, 32 kq + 32) are chunks 4 (kq & 1) .. + 3 of atom kq >> 1
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                uint32_t wv[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j0 = 32 * kq + 8 * x + 2 * e;
+                    const float k0 = (j0 <= row) ? P.eps + acc[8 * x + 2 * e] : 0.f;
+                    const float k1 = (j0 + 1 <= row) ? P.eps + acc[8 * x + 2 * e + 1] : 0.f;
+                    wv[e] = pack_bf16x2(k0, k1);
+                }
+                sts128(aq0 + (kq >> 1) * kTileBytes + kmajor_chunk(row, 4 * (kq & 1) + x),
+                       wv[0], wv[1], wv[2], wv[3]);
+            }
+            fence_proxy_async();
+            warp_arrive(&bar.p_full);
+        }
+        // every score tile has been read (and coefh written) before TMEM columns 128.. are
+        // reused as phi stages
+        tc_fence_before();
+        named_bar_sync(1, 16 * 32);
+        tc_fence_after();
+
+        // ---- inter-chunk phase: phi(Q_c) slices kq, kq + 4, ... ----
+        for (int s = kq; s < kSlices && ok && has_inter; s += kPhiSets) {
+            const int st = s % kRdStages;
+            uint32_t w[32];
+            if (s < kOffDiagSlices) phi_offdiag(qt, coefh, s, row, w);
+            else phi_diag(qt, coef, s, row, w);
+            if (s >= kRdStages &&
+                !mbar_wait(&bar.a_empty[st], ((s / kRdStages) - 1) & 1, abort_flag)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            tmem_st32(lanebase + kColA0 + st * 32, w);
+            tmem_st_wait();
+            tc_fence_before();
+            warp_arrive(&bar.a_full[st]);
+        }
+
+        // ---- epilogue: yhat = u[:64] / u[64], columns [16 kq, 16 kq + 16) of this row ----
+        if (ok) ok = mbar_wait(&bar.u_full, 0, abort_flag);
+        if (ok) {
+            tc_fence_after();
+            float u[16], dz[16];
+            tmem_ld16(lanebase + kColU + 16 * kq, u);
+            tmem_ld16(lanebase + kColU + 64, dz);
+            tmem_ld_wait();
+            const int irow = c * kC + row;
+            if (irow < T) {
+                const float inv = 1.f / dz[0];
+                float4* o = reinterpret_cast<float4*>(P.out + (size_t(bh) * T + irow) * kDV +
+                                                      16 * kq);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    o[i] = make_float4(u[4 * i] * inv, u[4 * i + 1] * inv, u[4 * i + 2] * inv,
+                                       u[4 * i + 3] * inv);
             }
         }
     }
@@ -981,6 +993,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_alloc(&ctl.tmem_base, kTmemCols);
         tmem_relinquish();
     }
+    init_ones_atom(sm + kOffOnes);  // both item kinds read it; neither writes that region
+    fence_proxy_async();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();

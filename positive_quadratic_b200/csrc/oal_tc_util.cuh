@@ -126,6 +126,13 @@ __device__ __forceinline__ void bulk_wait_read0()
 
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// As above, but the most recent bulk group may still be in flight.
+__device__ __forceinline__ void bulk_wait_read1()
+{
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait1() { asm volatile("cp.async.bulk.wait_group 1;" ::: "memory"); }
+
 // Make this thread's ordinary shared-memory writes visible to the async proxy (TMA, MMA).
 __device__ __forceinline__ void fence_proxy_async()
 {
@@ -278,6 +285,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
 }
+
+// Packed bf16 product (both halves rounded to nearest even).
+__device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+// bf16x2 with both halves equal to the low (high) half of w.
+__device__ __forceinline__ uint32_t dup_lo(uint32_t w) { return __byte_perm(w, 0u, 0x1010); }
+__device__ __forceinline__ uint32_t dup_hi(uint32_t w) { return __byte_perm(w, 0u, 0x3232); }
 
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi_to_f32(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
