@@ -55,9 +55,9 @@ def parse():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--split", action="store_true",
-                    help="tensor-core prefill as two kernels (all chunk states, then all "
-                         "readouts) instead of the persistent fused schedule")
+    ap.add_argument("--no-overlap", action="store_true",
+                    help="launch the prefill's scan and readout kernels in plain stream order "
+                         "instead of as programmatic dependents")
     ap.add_argument("--workload", default="config1", choices=["config1", "config3_16k",
                                                               "config3_32k", "config3_64k"],
                     help="prefill workload (config1 is the headline)")
@@ -227,7 +227,7 @@ def main():
                                 device_id=dev)
     pk, pk_kind = peaks()
     oal.lib()
-    oal.set_prefill_fused(not args.split)
+    oal.set_prefill_overlap(not args.no_overlap)
 
     p, desc = workload(args.workload)
     B, Hq, T, _ = p.q.shape
@@ -288,10 +288,8 @@ def main():
         name, (nl, ms) = dom
         per = ms / nl
         algo = flops_read if name.startswith("readout") else (
-            flops_state if name.startswith("state") else prefill_flops(B, T, Hq, Hkv))
+            flops_state if name.startswith(("state", "delta")) else prefill_flops(B, T, Hq, Hkv))
         tensor = name.endswith("_tc")
-        if name == "prefill_tc":  # the fused kernel does the whole prefill
-            algo = prefill_flops(B, T, Hq, Hkv)
         if tensor:
             peak, unit, bound = pk["bf16_tflops"], "TFLOP/s", "tensor"
         else:
@@ -351,7 +349,8 @@ def main():
                 "ms_per_step": total_ms / args.steps, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": {"workload": desc, "chunk": args.chunk,
-                           "schedule": "two kernels" if args.split else "persistent fused",
+                           "schedule": "deltas, scan, readout" + (
+                               "" if args.no_overlap else " (programmatic dependent launch)"),
                            "l2": "flushed between steps (256 MB write, outside timed events)",
                            "parallelism": f"replicas x{world}"},
                 "roofline": roof, "e2e": e2e, "gpu_launches": int(n_launch),

@@ -158,13 +158,12 @@ int oal_dense_ref_gpu(const void* q, const void* k, const void* v, const int32_t
                       const float* L, const int32_t* G, float eps, float* out,
                       const oal_shape* s, void* stream);
 
-/* Scheduling of the tensor-core prefill (bf16, chunk 128).  1 (default): one persistent
- * kernel pulls state-building and readout work from a single queue, so readouts of early
- * chunks overlap the building of later chunk states; it needs every CTA resident at once and
- * falls back to 0 when the device cannot host the grid.  0: two kernels, all chunk states
- * first, then all readouts.  Both produce the same results.  Process-wide; returns the
- * previous setting. */
-int oal_set_prefill_fused(int fused);
+/* Launch mode of the tensor-core prefill (bf16, chunk 128), which runs as three kernels:
+ * chunk deltas, the prefix scan over chunks, and the readout.  1 (default): the scan and the
+ * readout are launched as programmatic dependents, so each is scheduled while its predecessor
+ * drains and waits for it on the device.  0: plain stream order.  Both produce identical
+ * results.  Process-wide; returns the previous setting. */
+int oal_set_prefill_overlap(int overlap);
 
 /* Reads the device-side error word (OAL_OK or a negative oal_status set by a kernel since
  * the last read), synchronising `stream`, and clears it. */

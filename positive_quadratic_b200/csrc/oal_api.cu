@@ -50,7 +50,7 @@ size_t simt_chunk_state_bytes(const oal_shape* s)
 // bf16 inputs with chunk 128 run on the tcgen05 kernels; everything else on CUDA cores.
 bool use_tensor_path(const oal_shape* s) { return s->dtype == OAL_BF16 && s->chunk == 128; }
 
-std::atomic<int> g_prefill_fused{1};
+std::atomic<int> g_prefill_overlap{1};
 
 size_t decode_ticket_bytes(const oal_shape* s) { return align256(size_t(s->B) * s->Hkv * 4); }
 
@@ -133,7 +133,7 @@ int oal_prefill(const void* q, const void* k, const void* v, const int32_t* grou
     if (s->B == 0) return OAL_OK;
     if (use_tensor_path(s))
         return launch_prefill_tc(q, k, v, group_id, L, G, eps, out, state, workspace, s->B, s->T,
-                                 s->Hq, s->Hkv, g_prefill_fused.load() != 0, st);
+                                 s->Hq, s->Hkv, g_prefill_overlap.load() != 0, st);
     return launch_prefill_simt(q, k, v, group_id, L, G, eps, out, state,
                                static_cast<float*>(workspace), s->B, s->T, s->Hq, s->Hkv,
                                s->chunk, s->dtype, st);
@@ -176,7 +176,7 @@ int oal_dense_ref_gpu(const void* q, const void* k, const void* v, const int32_t
 
 unsigned long long oal_launch_count(void) { return tracer().launches.load(); }
 
-int oal_set_prefill_fused(int fused) { return g_prefill_fused.exchange(fused ? 1 : 0); }
+int oal_set_prefill_overlap(int overlap) { return g_prefill_overlap.exchange(overlap ? 1 : 0); }
 
 int oal_profile_enable(int on)
 {

@@ -4,30 +4,23 @@
 // section 核心公式, numbered in order of appearance: (2) grouped score, (3) kernel kappa,
 // (4) prefix states, (5) readout.  With the packed feature map of oal_common.cuh, the state
 // of a (b, kv) head after token i is S_i = sum_{j<=i} psi(k_j) [v_j; 1] (2176 x 65) and
-// u_i = phi(q_i)^T S_i.  Chunked with C = 128 tokens, the prefill is three kinds of work item:
+// u_i = phi(q_i)^T S_i.  Chunked with C = 128 tokens, the prefill runs as three kernels:
 //
-//   chain builder (b, kv, slab): 128 packed rows of one state, walked chunk by chunk.
-//     Producer warps build bf16 psi(K_c)^T (MN-major) in shared memory; one N=80 MMA per
-//     K-step accumulates dS_c = psi(K_c)^T [V_c; 1] in TMEM (the [.; 1] column comes from a
-//     constant "ones" atom addressed through the B descriptor's leading byte offset);
-//     epilogue warps keep the running prefix in fp32 registers and store the exclusive prefix
-//     S_c of every chunk as a bf16 K-major B-operand image (bulk copy).
-//   remainder item (b, kv, slab, token segment): the same product with psi replaced by its
-//     bf16 rounding remainder psi - bf16(psi) (exact: psi = k_r k_t of two bf16 values has at
-//     most 16 significant bits).  Chain and remainders add their fp32 sums into the final
-//     state, which therefore holds the exact products accumulated in fp32.
-//   reader (b, h, chunk c): 128 query rows of one head.  phi(Q_c) is written straight into
-//     tensor memory (tcgen05.st) slice by slice and multiplied with the state image of S_c by
-//     N=80 MMAs reading A from TMEM; concurrently the intra-chunk kernel is evaluated on tensor
-//     cores in the factored form of eq. (3),
+//   chunk deltas (b, kv, chunk c, slab of 128 packed rows; every unit independent):
+//     producer warps build psi(K_c)^T (MN-major, bf16) in shared memory, split exactly into
+//     hi = bf16(psi) and lo = psi - hi; N=80 MMAs accumulate dS_c = psi(K_c)^T [V_c; 1] in
+//     TMEM (the [.; 1] column comes from a constant "ones" atom addressed through the B
+//     descriptor's leading byte offset) and epilogue warps store it in fp32.
+//   prefix scan (SIMT, memory bound): S_c = sum_{c' < c} dS_c' for every chunk, written as
+//     bf16 K-major B-operand images, and the final state S_NC in fp32 (eq. 4 in chunk form).
+//   readout (b, h, chunk c): 128 query rows of one head.  The intra-chunk kernel runs first
+//     on tensor cores in the factored form of eq. (3),
 //       kappa = eps + sum_m (L_0m + (q o w_m) . k)^2,   w_m[r] = L_{g(r),m} / sqrt(d)
-//     (= ||L^T sbar||^2), masked causally and multiplied into [V_c; 1] in the same TMEM
-//     accumulator; finally yhat = u[:64] / u[64].
-//
-// One CTA shape (18 warps, 1 CTA per SM) serves all items.  Kernels: builders + remainders,
-// readers, and a persistent kernel that pulls every item from one queue in which each reader
-// follows the chain builders it depends on; readers wait (bounded) on per-chunk counters that
-// chain builders release once an image has reached global memory.
+//     (= ||L^T sbar||^2): score tiles S_m = (Q o w_m) K^T in TMEM, kappa accumulated in
+//     registers, masked causally and multiplied into [V_c; 1].  Then phi(Q_c) is written
+//     straight into tensor memory (tcgen05.st) slice by slice and multiplied with the image
+//     of S_c by N=80 MMAs reading A from TMEM, into the same accumulator; finally
+//     yhat = u[:64] / u[64] (eq. 5).
 //
 // Every wait is bounded (1 s); one that runs out sets OAL_ERR_TIMEOUT and the CTA leaves its
 // loops in order (copies drained, MMAs committed, TMEM freed) instead of hanging.
@@ -49,7 +42,6 @@ constexpr int kSlabRows = 128;                             // packed rows per bu
 constexpr int kNumSlabs = kFP / kSlabRows;                 // 17
 constexpr int kSlices = kFP / 64;                          // 34 readout K-slices
 constexpr int kOffDiagSlices = kOffDiagRows / 64;          // 28
-constexpr int kSegChunks = 8;                              // chunks per remainder item
 constexpr uint32_t kImgSliceBytes = 80 * 64 * 2;           // K-major [80 n][64 rows]
 constexpr uint32_t kImgLoadBytes = 65 * 128;               // rows 0..64 (65..79 are zero)
 constexpr size_t kImgChunkBytes = size_t(kSlices) * kImgSliceBytes;
@@ -71,30 +63,38 @@ constexpr uint32_t kRdOffK = 0;           // K tile (score B operand, K-major)
 constexpr uint32_t kRdOffV = 16384;       // V tile (PV B operand, MN-major)
 constexpr uint32_t kRdOffQ = 32768;       // Q tile (bf16, K-major): phi and Aq read it
 constexpr uint32_t kRdOffAq = 49152;      // Aq0 | Aq1 (score A operands); the P tile aliases
-constexpr uint32_t kRdOffB = 81920;       // 8 x 10 KB state-image stages
-constexpr uint32_t kRdOffCoef = 180224;   // 2176 fp32 coefficients
-constexpr uint32_t kRdOffCoefH = 188928;  // 1792 bf16 coefficients of the off-diagonal rows
-constexpr uint32_t kRdOffW = 192512;      // 9 x 64 fp32
-constexpr uint32_t kRdOffC0 = 194816;     // 9 fp32
-// builder
-constexpr uint32_t kStOffKV = 0;          // 4 x (K 16 KB + V 16 KB)
-constexpr uint32_t kStOffA = 131072;      // 2 x 16 KB psi stages
-constexpr uint32_t kStOffImg = 180224;    // 2 buffers x 2 slices x 10 KB image staging
+constexpr uint32_t kRdOffA = 81920;       // 4 x 16 KB phi stages (readout A operand, K-major)
+constexpr uint32_t kRdOffB = 147456;      // 2 x 20 KB state-image stages of 2 slices (B operand)
+constexpr uint32_t kRdOffOnes = 188416;   // 16 KB ones atom
+constexpr uint32_t kRdOffCoef = 204800;   // 2176 fp32 coefficients
+constexpr uint32_t kRdOffCoefH = 213504;  // 1792 bf16 coefficients of the off-diagonal rows
+constexpr uint32_t kRdOffW = 217088;      // 9 x 64 fp32
+constexpr uint32_t kRdOffC0 = 219392;     // 9 fp32
+// chunk-delta builder
+constexpr uint32_t kStOffKV = 0;          // 3 x (K 16 KB + V 16 KB)
+constexpr uint32_t kStOffA = 98304;       // 2 x (hi 16 KB + lo 16 KB) psi stages
+constexpr uint32_t kOffOnes = 163840;     // 16 KB ones atom
 // both
-constexpr uint32_t kOffOnes = 163840;     // 16 KB ones atom, written once per CTA
-constexpr uint32_t kOffCtl = 221184;      // barriers and control words
+constexpr uint32_t kOffCtl = 219648;      // barriers and control words
 constexpr uint32_t kSmemBytes = kOffCtl + 1024 + 1024;
 
 constexpr int kPhiSets = 4;                                // reader warps (w >> 2) per slice
-constexpr int kRdStages = 12;                              // phi stages (TMEM)
-constexpr int kBStages = 8;                                // state-image stages (SMEM)
-constexpr int kKVStages = 4;
+// phi stages (SMEM, 1 slice): one per warp set, so that every wait on a stage barrier is for
+// the phase right after the one the waiter last saw complete (parity waits cannot tell
+// phases two apart)
+constexpr int kRdStages = kPhiSets;
+constexpr int kBStages = 2;                                // image stages (SMEM, 2 slices)
+constexpr uint32_t kImgPairBytes = 2 * kImgSliceBytes;     // one tensor copy: 160 rows
+constexpr uint32_t kPhiTileBytes = kC * 64 * 2;            // 128 rows x 64 packed rows, bf16
+constexpr int kKVStages = 3;
 constexpr uint32_t kStATile = 64 * kSlabRows * 2;          // 64 tokens x 128 rows = 16 KB
-// reader TMEM map: U in [0, 80); score tiles S0 | S1 in [128, 384) during the intra-chunk
-// phase; phi stages of 32 columns in [128, 512) during the inter-chunk phase
-constexpr uint32_t kColU = 0, kColS0 = 128, kColA0 = 128;
-static_assert(kColA0 + 32 * kRdStages <= kTmemCols, "phi stages");
-static_assert(kRdStages % kPhiSets == 0, "a stage belongs to one phi set");
+// reader TMEM map: U in [0, 80); score tiles S0 | S1 in [128, 384).  phi stays in shared
+// memory: warp stores into tensor memory stall concurrent MMAs, shared-memory stores do not.
+constexpr uint32_t kColU = 0, kColS0 = 128;
+static_assert(kRdOffA + kRdStages * kPhiTileBytes <= kRdOffB &&
+                  kRdOffB + kBStages * kImgPairBytes <= kRdOffOnes &&
+                  kRdOffC0 + 64 <= kOffCtl,
+              "reader shared-memory map");
 
 struct RdBars {
     uint64_t qkv_full, aq_full[2], s_full[2], s_empty[2], p_full;
@@ -124,17 +124,16 @@ struct Params {
     const CUtensorMap* tm_q;
     const CUtensorMap* tm_k;
     const CUtensorMap* tm_v;
+    const CUtensorMap* tm_img;  // chunk-state images as {64 f, slices * 80 rows}, box {64, 160}
     const int32_t* gid;
     const float* L;
     const int32_t* G;
     float eps;
     const float* coef_all;   // state header coefficient table [Hq][kFP]
-    unsigned char* img;      // chunk-state images [B*Hkv][NC][34][10240]
-    float* body;             // final state (zeroed before the launch; items add into it)
+    unsigned char* img;      // chunk-state images [B*Hkv][NC][34 slices][80 n][64 f] bf16
+    float* dS;               // chunk deltas [B*Hkv][NC][65][kFP] fp32
     float* out;
-    unsigned int* flags;     // [B*Hkv][NC] image-completion counters (persistent mode) or null
-    unsigned int* queue;     // work-queue head (persistent mode)
-    int B, Hq, Hkv, T, NC, nseg;
+    int B, Hq, Hkv, T, NC;
 };
 
 // ------------------------------------------------------------------------------------------
@@ -149,18 +148,6 @@ template <int N, typename F>
 __device__ __forceinline__ void static_for(F&& f)
 {
     static_for_impl(f, std::make_integer_sequence<int, N>{});
-}
-
-// (R, T) of off-diagonal block beta (R < T, lexicographic)
-__device__ __forceinline__ void block_rt(int beta, int& R, int& T)
-{
-    int r = 0, s = 0;
-    while (beta >= s + 7 - r) {
-        s += 7 - r;
-        ++r;
-    }
-    R = r;
-    T = r + 1 + (beta - s);
 }
 
 __device__ __forceinline__ void warp_arrive(uint64_t* bar)
@@ -214,44 +201,28 @@ __device__ __forceinline__ void init_ones_atom(unsigned char* atom)
             kBf16One;
 }
 
-__device__ __forceinline__ void inval_builder_bars(StBars& b)
+// (R, T) of the 28 off-diagonal 8 x 8 blocks (R < T, lexicographic), as 8 R + T
+#define OAL_BLOCK_RT                                                                       \
+    1, 2, 3, 4, 5, 6, 7, 10, 11, 12, 13, 14, 15, 19, 20, 21, 22, 23, 28, 29, 30, 31, 37, 38, \
+        39, 46, 47, 55
+constexpr uint8_t kBlockRT[kOffDiagSlices] = {OAL_BLOCK_RT};
+__constant__ uint8_t c_block_rt[kOffDiagSlices] = {OAL_BLOCK_RT};
+#undef OAL_BLOCK_RT
+constexpr bool block_rt_table_ok()
 {
-    for (int i = 0; i < kKVStages; ++i) {
-        mbar_inval(&b.kv_full[i]);
-        mbar_inval(&b.kv_empty[i]);
+    for (int s = 0; s < kOffDiagSlices; ++s) {
+        const RT rt = feature_rt(64 * s);
+        if (rt.r != 8 * (kBlockRT[s] >> 3) || rt.t != 8 * (kBlockRT[s] & 7)) return false;
     }
-    for (int i = 0; i < 2; ++i) {
-        mbar_inval(&b.a_full[i]);
-        mbar_inval(&b.a_empty[i]);
-        mbar_inval(&b.acc_full[i]);
-        mbar_inval(&b.acc_empty[i]);
-    }
-    mbar_inval(&b.done);
+    return true;
 }
-
-__device__ __forceinline__ void inval_reader_bars(RdBars& b)
-{
-    mbar_inval(&b.qkv_full);
-    for (int i = 0; i < 2; ++i) {
-        mbar_inval(&b.aq_full[i]);
-        mbar_inval(&b.s_full[i]);
-        mbar_inval(&b.s_empty[i]);
-    }
-    mbar_inval(&b.p_full);
-    for (int i = 0; i < kRdStages; ++i) {
-        mbar_inval(&b.a_full[i]);
-        mbar_inval(&b.a_empty[i]);
-    }
-    for (int i = 0; i < kBStages; ++i) {
-        mbar_inval(&b.b_full[i]);
-        mbar_inval(&b.b_empty[i]);
-    }
-    mbar_inval(&b.u_full);
-    mbar_inval(&b.done);
-}
+static_assert(block_rt_table_ok(), "off-diagonal block table");
 
 // ------------------------------------------------------------------------------------------
-// builder: psi producers (thread = token j of a half chunk, quarter qf of the slab's rows)
+// chunk-delta builder: psi producers (thread = token j of a half chunk, quarter qf of the
+// slab's 128 rows).  psi = k_r k_t of two bf16 values has at most 16 significant bits, so it
+// splits exactly into hi = bf16(psi) and lo = psi - hi (also a bf16 value); both are written
+// as MN-major A tiles and the MMA accumulates hi^T [V; 1] + lo^T [V; 1] in fp32.
 // ------------------------------------------------------------------------------------------
 // MN-major A tile (128 rows x 64 tokens): the 8-row chunk starting at row m for token j
 __device__ __forceinline__ uint32_t st_a_off(int m, int j)
@@ -260,38 +231,34 @@ __device__ __forceinline__ uint32_t st_a_off(int m, int j)
                     ((((m & 63) >> 3) ^ (j & 7)) << 4));
 }
 
-// bf16 of the exact product p (kLo = false) or of its rounding remainder p - bf16(p) (true)
-template <bool kLo>
-__device__ __forceinline__ uint32_t psi_pack(float2 p)
+// a * b + c on packed bf16 pairs, one rounding
+__device__ __forceinline__ uint32_t bfma2(uint32_t a, uint32_t b, uint32_t c)
 {
-    const uint32_t h = pack2(p);
-    if (!kLo) return h;
-    return pack_bf16x2(p.x - bf16lo_to_f32(h), p.y - bf16hi_to_f32(h));
+    uint32_t d;
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
 }
 
 // off-diagonal slabs: 32 rows = 4 dims a of block R times the 8 dims of block T.  They never
 // involve the constant slot, and K rows past T are zero-filled by the copy.
-template <bool kLo>
 __device__ __forceinline__ void psi_offdiag(const unsigned char* ktile, int trow, uint32_t abase,
                                             int j, int slab, int qf)
 {
-    int R, T;
-    block_rt(2 * slab + (qf >> 1), R, T);
-    const uint2 wa = *reinterpret_cast<const uint2*>(ktile + kmajor_chunk(trow, R) + 8 * (qf & 1));
-    const uint4 wt = *reinterpret_cast<const uint4*>(ktile + kmajor_chunk(trow, T));
-    const float ka[4] = {bf16lo_to_f32(wa.x), bf16hi_to_f32(wa.x), bf16lo_to_f32(wa.y),
-                         bf16hi_to_f32(wa.y)};
-    const float2 t0 = f2(bf16lo_to_f32(wt.x), bf16hi_to_f32(wt.x));
-    const float2 t1 = f2(bf16lo_to_f32(wt.y), bf16hi_to_f32(wt.y));
-    const float2 t2 = f2(bf16lo_to_f32(wt.z), bf16hi_to_f32(wt.z));
-    const float2 t3 = f2(bf16lo_to_f32(wt.w), bf16hi_to_f32(wt.w));
+    const int rt = c_block_rt[2 * slab + (qf >> 1)];
+    const uint2 wa =
+        *reinterpret_cast<const uint2*>(ktile + kmajor_chunk(trow, rt >> 3) + 8 * (qf & 1));
+    const uint4 wt = *reinterpret_cast<const uint4*>(ktile + kmajor_chunk(trow, rt & 7));
+    const uint32_t xs[4] = {dup_lo(wa.x), dup_hi(wa.x), dup_lo(wa.y), dup_hi(wa.y)};
     const int m0 = 64 * (qf >> 1) + 32 * (qf & 1);
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
-        const float2 xx = f2(ka[a], ka[a]);
-        sts128(abase + st_a_off(m0 + 8 * a, j), psi_pack<kLo>(__fmul2_rn(xx, t0)),
-               psi_pack<kLo>(__fmul2_rn(xx, t1)), psi_pack<kLo>(__fmul2_rn(xx, t2)),
-               psi_pack<kLo>(__fmul2_rn(xx, t3)));
+        const uint32_t h0 = bmul2(xs[a], wt.x), h1 = bmul2(xs[a], wt.y);
+        const uint32_t h2 = bmul2(xs[a], wt.z), h3 = bmul2(xs[a], wt.w);
+        const uint32_t off = st_a_off(m0 + 8 * a, j);
+        sts128(abase + off, h0, h1, h2, h3);
+        sts128(abase + kStATile + off, bfma2(xs[a], wt.x, h0 ^ 0x80008000u),
+               bfma2(xs[a], wt.y, h1 ^ 0x80008000u), bfma2(xs[a], wt.z, h2 ^ 0x80008000u),
+               bfma2(xs[a], wt.w, h3 ^ 0x80008000u));
     }
 }
 
@@ -305,8 +272,9 @@ constexpr bool psi_chunk_needed(int ch)
     return false;
 }
 
-// diagonal / linear / constant slabs: 32 rows with compile-time (r, t)
-template <int F0, bool kLo>
+// diagonal / linear / constant slabs: 32 rows with compile-time (r, t); fp32 products (exact)
+// split into hi and lo
+template <int F0>
 __device__ __forceinline__ void psi_static(const unsigned char* ktile, int trow, float one,
                                            uint32_t abase, int j)
 {
@@ -330,44 +298,56 @@ __device__ __forceinline__ void psi_static(const unsigned char* ktile, int trow,
     constexpr int m0 = F0 % kSlabRows;
     static_for<4>([&](auto CH) {
         constexpr int ch = decltype(CH)::value;
-        uint32_t h[4];
+        uint32_t h[4], l[4];
         static_for<4>([&](auto E) {
             constexpr int e = decltype(E)::value;
             constexpr RT a = feature_rt(F0 + ch * 8 + 2 * e);
             constexpr RT b = feature_rt(F0 + ch * 8 + 2 * e + 1);
-            h[e] = psi_pack<kLo>(f2(k[a.r] * k[a.t], k[b.r] * k[b.t]));
+            const float pa = k[a.r] * k[a.t], pb = k[b.r] * k[b.t];
+            h[e] = pack_bf16x2(pa, pb);
+            l[e] = pack_bf16x2(pa - bf16lo_to_f32(h[e]), pb - bf16hi_to_f32(h[e]));
         });
         sts128(abase + st_a_off(m0 + 8 * ch, j), h[0], h[1], h[2], h[3]);
+        sts128(abase + kStATile + st_a_off(m0 + 8 * ch, j), l[0], l[1], l[2], l[3]);
     });
 }
 
-template <bool kLo>
 __device__ __forceinline__ void psi_tile(int slab, int qf, const unsigned char* ktile, int trow,
                                          float one, uint32_t abase, int j)
 {
     if (slab < kOffDiagSlices / 2) {
-        psi_offdiag<kLo>(ktile, trow, abase, j, slab, qf);
+        psi_offdiag(ktile, trow, abase, j, slab, qf);
         return;
     }
     const int sel = (slab - kOffDiagSlices / 2) * 4 + qf;
     static_for<(kNumSlabs - kOffDiagSlices / 2) * 4>([&](auto I) {
         constexpr int i = decltype(I)::value;
-        if (sel == i) psi_static<kOffDiagRows + i * 32, kLo>(ktile, trow, one, abase, j);
+        if (sel == i) psi_static<kOffDiagRows + i * 32>(ktile, trow, one, abase, j);
     });
 }
 
+// unit u -> (bkv, chunk c, slab); slabs of one chunk are consecutive
+struct DeltaUnit {
+    int bkv, c, slab;
+};
+__device__ __forceinline__ DeltaUnit delta_unit(int u, int NC)
+{
+    const int rest = u / kNumSlabs;
+    return DeltaUnit{rest / NC, rest % NC, u % kNumSlabs};
+}
+
 // ------------------------------------------------------------------------------------------
-// builder item: chain (kLo = false, chunks [0, NC)) or remainder (kLo = true, chunks
-// [c0, c1)); warps 0-7 psi producers, 8-15 epilogue, 16 TMA, 17 MMA
+// chunk-delta item: units [u0, u1), each dS_c = psi(K_c)^T [V_c; 1] for the 128 packed rows
+// of one slab, stored in fp32 as dS[bkv][c][n][f] (n = column of [v; 1]).
+// Warps 0-7 psi producers, 8-15 epilogue, 16 TMA, 17 MMA.
 // ------------------------------------------------------------------------------------------
-template <bool kLo>
-__device__ void builder_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Params& P,
-                             int bkv, int slab, int c0, int c1)
+__device__ void delta_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Params& P, int u0,
+                           int u1)
 {
     StBars& bar = ctl.bar.st;
     volatile int* abort_flag = &ctl.abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int NC = P.NC, T = P.T, nch = c1 - c0;
+    const int NC = P.NC, T = P.T, nu = u1 - u0;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kKVStages; ++i) {
@@ -384,10 +364,6 @@ __device__ void builder_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const P
         ctl.abort_flag = 0;
         fence_mbar_init();
     }
-    if (!kLo)
-        for (int e = threadIdx.x; e < int(4 * kImgSliceBytes / 16); e += blockDim.x)
-            reinterpret_cast<uint4*>(sm + kStOffImg)[e] = make_uint4(0u, 0u, 0u, 0u);
-    fence_proxy_async();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -395,74 +371,83 @@ __device__ void builder_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const P
     if (warp == kTmaWarp) {
         if (lane == 0) {
             int issued = 0;
-            for (int u = 0; u < nch; ++u) {
-                const int c = c0 + u, s = u % kKVStages;
-                if (u >= kKVStages &&
-                    !mbar_wait(&bar.kv_empty[s], ((u / kKVStages) - 1) & 1, abort_flag))
+            for (int i = 0; i < nu; ++i) {
+                const DeltaUnit du = delta_unit(u0 + i, NC);
+                const int s = i % kKVStages;
+                if (i >= kKVStages &&
+                    !mbar_wait(&bar.kv_empty[s], ((i / kKVStages) - 1) & 1, abort_flag))
                     break;
                 unsigned char* kvs = sm + kStOffKV + s * 2 * kTileBytes;
                 mbar_expect_tx(&bar.kv_full[s], 2 * kTileBytes);
-                tma_load_3d(kvs, P.tm_k, &bar.kv_full[s], 0, c * kC, bkv);
-                tma_load_3d(kvs + kTileBytes, P.tm_v, &bar.kv_full[s], 0, c * kC, bkv);
+                tma_load_3d(kvs, P.tm_k, &bar.kv_full[s], 0, du.c * kC, du.bkv);
+                tma_load_3d(kvs + kTileBytes, P.tm_v, &bar.kv_full[s], 0, du.c * kC, du.bkv);
                 ++issued;
             }
-            for (int u = max(0, issued - kKVStages); u < issued; ++u)
-                bounded_spin_done(&bar.kv_full[u % kKVStages], (u / kKVStages) & 1);
+            for (int i = max(0, issued - kKVStages); i < issued; ++i)
+                bounded_spin_done(&bar.kv_full[i % kKVStages], (i / kKVStages) & 1);
         }
         __syncwarp();
     } else if (warp == kMmaWarp) {
-        if (lane == 0) {
-            constexpr uint32_t id = idesc_bf16(128, 80, true, true);
-            const uint32_t a0 = smem_u32(sm + kStOffA), kv0 = smem_u32(sm + kStOffKV);
-            const uint32_t ones = smem_u32(sm + kOffOnes);
-            bool ok = true;
-            for (int u = 0; u < nch && ok; ++u) {
-                const int s = kLo ? 0 : (u & 1), st = u % kKVStages;
-                if (!kLo && u >= 2) ok = mbar_wait(&bar.acc_empty[s], ((u >> 1) - 1) & 1, abort_flag);
-                if (ok) ok = mbar_wait(&bar.kv_full[st], (u / kKVStages) & 1, abort_flag);
+        // the whole warp runs the issue loop; one elected lane issues
+        constexpr uint32_t id = idesc_bf16(128, 80, true, true);
+        const uint32_t a0 = smem_u32(sm + kStOffA), kv0 = smem_u32(sm + kStOffKV);
+        const uint32_t ones = smem_u32(sm + kOffOnes);
+        bool ok = true;
+        for (int i = 0; i < nu && ok; ++i) {
+            const int s = i & 1, st = i % kKVStages;
+            if (i >= 2) ok = mbar_wait(&bar.acc_empty[s], ((i >> 1) - 1) & 1, abort_flag);
+            if (ok) ok = mbar_wait(&bar.kv_full[st], (i / kKVStages) & 1, abort_flag);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            const uint32_t d = tmem + s * 128;
+            const uint32_t vt = kv0 + st * 2 * kTileBytes + kTileBytes;
+            const uint32_t lbo = ones - vt;  // V atom -> ones atom (N elements 64..)
+            for (int hc = 0; hc < 2; ++hc) {
+                const int w = 2 * i + hc, as = w & 1;
+                ok = __all_sync(0xffffffffu, mbar_wait(&bar.a_full[as], (w >> 1) & 1, abort_flag));
                 if (!ok) break;
-                const uint32_t d = tmem + s * 128;
-                const uint32_t vt = kv0 + st * 2 * kTileBytes + kTileBytes;
-                const uint32_t lbo = ones - vt;  // V atom -> ones atom (N elements 64..)
-                for (int hc = 0; hc < 2; ++hc) {
-                    const int w = 2 * u + hc, as = w & 1;
-                    if (!(ok = mbar_wait(&bar.a_full[as], (w >> 1) & 1, abort_flag))) break;
-                    tc_fence_after();
-                    const uint32_t ab = a0 + as * kStATile;
+                tc_fence_after();
+                if (elect_one()) {
+                    const uint32_t ab = a0 + as * 2 * kStATile;
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks) {
-                        const uint32_t acc = (kLo ? (u | hc | ks) : (hc | ks)) ? 1u : 0u;
-                        mma_bf16(d, sdesc_sw128(ab + ks * 2048, 8192, 1024),
-                                 sdesc_sw128(vt + hc * 8192 + ks * 2048, lbo, 1024), id, acc);
+                    for (int x = 0; x < 8; ++x) {  // hi (x < 4), lo (x >= 4) over 4 K-steps
+                        const int ks = x & 3;
+                        mma_bf16(d, sdesc_sw128(ab + (x >> 2) * kStATile + ks * 2048, 8192, 1024),
+                                 sdesc_sw128(vt + hc * 8192 + ks * 2048, lbo, 1024), id,
+                                 (hc | x) ? 1u : 0u);
                     }
                     mma_commit(&bar.a_empty[as]);
                 }
-                if (!ok) break;
-                if (!kLo) mma_commit(&bar.acc_full[s]);
+                __syncwarp();
+            }
+            if (!ok) break;
+            if (elect_one()) {
+                mma_commit(&bar.acc_full[s]);
                 mma_commit(&bar.kv_empty[st]);
             }
-            if (kLo && ok) mma_commit(&bar.acc_full[0]);
-            mma_commit(&bar.done);
-            bounded_spin_done(&bar.done, 0);
+            __syncwarp();
         }
+        if (elect_one()) mma_commit(&bar.done);
+        __syncwarp();
+        if (lane == 0) bounded_spin_done(&bar.done, 0);
         __syncwarp();
     } else if (warp < 8) {
         const int t = threadIdx.x, j = t & 63, qf = t >> 6;
         const uint32_t a0 = smem_u32(sm + kStOffA);
-        for (int u = 0; u < nch; ++u) {
-            const int c = c0 + u, st = u % kKVStages;
-            if (!mbar_wait(&bar.kv_full[st], (u / kKVStages) & 1, abort_flag)) break;
+        for (int i = 0; i < nu; ++i) {
+            const DeltaUnit du = delta_unit(u0 + i, NC);
+            const int st = i % kKVStages;
+            if (!mbar_wait(&bar.kv_full[st], (i / kKVStages) & 1, abort_flag)) break;
             const unsigned char* kt = sm + kStOffKV + st * 2 * kTileBytes;
             bool ok = true;
             for (int hc = 0; hc < 2; ++hc) {
-                const int w = 2 * u + hc, as = w & 1;
+                const int w = 2 * i + hc, as = w & 1;
                 if (w >= 2 && !mbar_wait(&bar.a_empty[as], ((w >> 1) - 1) & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
                 const int trow = hc * 64 + j;
-                const float one = (c * kC + trow < T) ? 1.f : 0.f;
-                psi_tile<kLo>(slab, qf, kt, trow, one, a0 + as * kStATile, j);
+                const float one = (du.c * kC + trow < T) ? 1.f : 0.f;
+                psi_tile(du.slab, qf, kt, trow, one, a0 + as * 2 * kStATile, j);
                 fence_proxy_async();
                 warp_arrive(&bar.a_full[as]);
             }
@@ -472,88 +457,29 @@ __device__ void builder_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const P
     } else {
         // epilogue: thread = (packed row of the slab, column half)
         const int q4 = warp & 3, hfe = (warp - 8) >> 2;
-        const int fl = q4 * 32 + lane, f = slab * kSlabRows + fl;
-        const int kk = fl & 63;
-        const uint32_t stage0 = smem_u32(sm + kStOffImg) + (fl >> 6) * kImgSliceBytes;
-        float run[33];
-#pragma unroll
-        for (int n = 0; n < 33; ++n) run[n] = 0.f;
-        const bool leader = (threadIdx.x == 8 * 32);
-        unsigned int* flags = (!kLo && P.flags) ? P.flags + size_t(bkv) * NC : nullptr;
-        const int rounds = kLo ? 1 : nch;
-        for (int u = 0; u < rounds; ++u) {
-            const int c = c0 + u, s = kLo ? 0 : (u & 1);
-            if (!kLo && c >= 1) {
-                // exclusive prefix S_c -> bf16 K-major image [80 n][64 rows] -> bulk store,
-                // staged in buffer c & 1.  That buffer last held image c - 2: wait for its
-                // store only (image c - 1 stays in flight), then publish image c - 2.
-                const uint32_t stage = stage0 + (c & 1) * 2 * kImgSliceBytes;
-                if (leader && c >= 3) {
-                    if (flags) {
-                        bulk_wait1();
-                        fence_proxy_async_global();
-                        red_release_gpu_add(flags + (c - 2), 1u);
-                    } else {
-                        bulk_wait_read1();
-                    }
-                }
-                named_bar_sync(1, 256);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int n = 32 * hfe + i;
-                    asm volatile("st.shared.b16 [%0], %1;" ::"r"(stage + kmajor_off(n, kk)),
-                                 "h"(__bfloat16_as_ushort(__float2bfloat16_rn(run[i])))
-                                 : "memory");
-                }
-                if (hfe == 1)
-                    asm volatile("st.shared.b16 [%0], %1;" ::"r"(stage + kmajor_off(64, kk)),
-                                 "h"(__bfloat16_as_ushort(__float2bfloat16_rn(run[32])))
-                                 : "memory");
-                fence_proxy_async();
-                named_bar_sync(1, 256);
-                if (leader) {
-                    unsigned char* dst = P.img + (size_t(bkv) * NC + c) * kImgChunkBytes +
-                                         size_t(2 * slab) * kImgSliceBytes;
-                    bulk_s2g(dst, sm + kStOffImg + (c & 1) * 2 * kImgSliceBytes,
-                             2 * kImgSliceBytes);
-                    bulk_commit();
-                }
-            }
+        const int fl = q4 * 32 + lane;
+        for (int i = 0; i < nu; ++i) {
+            const DeltaUnit du = delta_unit(u0 + i, NC);
+            const int s = i & 1;
             // all epilogue threads leave together, so no named barrier is left half-joined
-            const bool got = mbar_wait(&bar.acc_full[s], kLo ? 0 : ((u >> 1) & 1), abort_flag);
+            const bool got = mbar_wait(&bar.acc_full[s], (i >> 1) & 1, abort_flag);
             if (!named_bar_and(2, 256, got)) break;
             tc_fence_after();
             const uint32_t lanebase = tmem + (uint32_t(q4 * 32) << 16) + s * 128;
             float v0[16], v1[16], vz[16];
             tmem_ld16(lanebase + hfe * 32, v0);
             tmem_ld16(lanebase + hfe * 32 + 16, v1);
-            tmem_ld16(lanebase + 64, vz);
+            if (hfe == 1) tmem_ld16(lanebase + 64, vz);
             tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                run[i] += v0[i];
-                run[16 + i] += v1[i];
-            }
-            if (hfe == 1) run[32] += vz[0];
             tc_fence_before();
-            if (!kLo) warp_arrive(&bar.acc_empty[s]);
-        }
-        if (!*abort_flag) {
-            // fp32 sums into the final state (chain and remainders add into a zeroed body)
-            float* unit = P.body + size_t(bkv) * kFP * kW;
-            float* hv = unit + size_t(f) * kDV + hfe * 32;
+            warp_arrive(&bar.acc_empty[s]);
+            float* dst = P.dS + (size_t(du.bkv) * NC + du.c) * kW * kFP + du.slab * kSlabRows + fl;
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                red_add_v4(hv + 4 * i, run[4 * i], run[4 * i + 1], run[4 * i + 2], run[4 * i + 3]);
-            if (hfe == 1) atomicAdd(unit + size_t(kFP) * kDV + f, run[32]);
-        }
-        if (leader && !kLo) {
-            bulk_wait0();
-            if (flags && !*abort_flag) {
-                // the last two images (the loop published images up to NC - 3)
-                fence_proxy_async_global();
-                for (int c = max(1, NC - 2); c < NC; ++c) red_release_gpu_add(flags + c, 1u);
+            for (int x = 0; x < 16; ++x) {
+                dst[size_t(hfe * 32 + x) * kFP] = v0[x];
+                dst[size_t(hfe * 32 + 16 + x) * kFP] = v1[x];
             }
+            if (hfe == 1) dst[size_t(64) * kFP] = vz[0];
         }
     }
 }
@@ -561,22 +487,6 @@ __device__ void builder_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const P
 // ------------------------------------------------------------------------------------------
 // reader: phi producers (thread = query row; one slice = 64 packed rows = 32 TMEM columns)
 // ------------------------------------------------------------------------------------------
-// (R, T) of the 28 off-diagonal 8 x 8 blocks (R < T, lexicographic), as 8 R + T
-#define OAL_BLOCK_RT                                                                       \
-    1, 2, 3, 4, 5, 6, 7, 10, 11, 12, 13, 14, 15, 19, 20, 21, 22, 23, 28, 29, 30, 31, 37, 38, \
-        39, 46, 47, 55
-constexpr uint8_t kBlockRT[kOffDiagSlices] = {OAL_BLOCK_RT};
-__constant__ uint8_t c_block_rt[kOffDiagSlices] = {OAL_BLOCK_RT};
-#undef OAL_BLOCK_RT
-constexpr bool block_rt_table_ok()
-{
-    for (int s = 0; s < kOffDiagSlices; ++s) {
-        const RT rt = feature_rt(64 * s);
-        if (rt.r != 8 * (kBlockRT[s] >> 3) || rt.t != 8 * (kBlockRT[s] & 7)) return false;
-    }
-    return true;
-}
-static_assert(block_rt_table_ok(), "off-diagonal block table");
 
 // off-diagonal slice s = block (R, T): rows (8R + a, 8T + b), a, b = 0..7.  Packed bf16
 // arithmetic: phi = bf16(bf16(q_r q_t) c) with c rounded to bf16 -- three roundings of 2^-9,
@@ -718,12 +628,6 @@ __device__ void reader_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Pa
         tma_load_3d(sm + kRdOffV, P.tm_v, &bar.qkv_full, 0, c * kC, bkv);
         bulk_g2s(coef, P.coef_all + size_t(h) * kFP, kFP * 4, &bar.qkv_full);
     }
-    // state-image stages: N rows 65..79 are never loaded and must read as zero
-    for (int e = threadIdx.x; e < int(kBStages * 15 * 8); e += blockDim.x) {
-        const int st = e / 120, x = e % 120;
-        reinterpret_cast<uint4*>(sm + kRdOffB + st * kImgSliceBytes + kImgLoadBytes)[x] =
-            make_uint4(0u, 0u, 0u, 0u);
-    }
     for (int e = threadIdx.x; e < kGM1 * 64; e += blockDim.x) {
         const int m = e >> 6, r = e & 63;
         int g = P.gid[h * kD + r];
@@ -743,55 +647,42 @@ __device__ void reader_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Pa
         if (lane == 0) {
             int issued = 0;
             bool ok = true;
-            if (has_inter && P.flags) {
-                // every slab of this chunk's state image must be in global memory
-                const unsigned int* fl = P.flags + size_t(bkv) * NC + c;
-                const uint64_t t0 = globaltimer();
-                while (ld_acquire_gpu(fl) < unsigned(kNumSlabs)) {
-                    if (*abort_flag || globaltimer() - t0 > kWaitLimitNs) {
-                        *abort_flag = 1;
-                        raise_error(OAL_ERR_TIMEOUT);
-                        ok = false;
-                        break;
-                    }
-                    __nanosleep(64);
-                }
-                fence_proxy_async_global();
-            }
             if (has_inter && ok) {
-                const unsigned char* src = P.img + (size_t(bkv) * NC + c) * kImgChunkBytes;
-                for (int s = 0; s < kSlices; ++s) {
-                    const int bs = s % kBStages;
-                    if (s >= kBStages &&
-                        !mbar_wait(&bar.b_empty[bs], ((s / kBStages) - 1) & 1, abort_flag))
+                // slices 2u, 2u + 1 of image (bkv, c) in one copy of 160 rows
+                const int row0 = (bkv * NC + c) * kSlices * 80;
+                for (int u = 0; u < kSlices / 2; ++u) {
+                    const int bs = u % kBStages;
+                    if (u >= kBStages &&
+                        !mbar_wait(&bar.b_empty[bs], ((u / kBStages) - 1) & 1, abort_flag))
                         break;
-                    mbar_expect_tx(&bar.b_full[bs], kImgLoadBytes);
-                    bulk_g2s(sm + kRdOffB + bs * kImgSliceBytes, src + size_t(s) * kImgSliceBytes,
-                             kImgLoadBytes, &bar.b_full[bs]);
+                    mbar_expect_tx(&bar.b_full[bs], kImgPairBytes);
+                    tma_load_2d(sm + kRdOffB + bs * kImgPairBytes, P.tm_img, &bar.b_full[bs], 0,
+                                row0 + 160 * u);
                     ++issued;
                 }
             }
             bounded_spin_done(&bar.qkv_full, 0);
-            for (int s = max(0, issued - kBStages); s < issued; ++s)
-                bounded_spin_done(&bar.b_full[s % kBStages], (s / kBStages) & 1);
+            for (int u = max(0, issued - kBStages); u < issued; ++u)
+                bounded_spin_done(&bar.b_full[u % kBStages], (u / kBStages) & 1);
         }
         __syncwarp();
     } else if (warp == kMmaWarp) {
-        if (lane == 0) {
-            constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);
-            constexpr uint32_t id_u = idesc_bf16(128, 80, false, false);   // A in TMEM, B K-major
-            constexpr uint32_t id_pv = idesc_bf16(128, 80, false, true);   // B = [V | ones] MN
-            const uint32_t aq0 = smem_u32(sm + kRdOffAq), kt = smem_u32(sm + kRdOffK);
-            const uint32_t vt = smem_u32(sm + kRdOffV), ones = smem_u32(sm + kOffOnes);
-            const uint32_t b0 = smem_u32(sm + kRdOffB);
-            bool ok = mbar_wait(&bar.qkv_full, 0, abort_flag);
-            // grouped score tiles S_m = (Q o w_m) K^T, double-buffered in TMEM
-            for (int m = 0; m <= G && ok; ++m) {
-                const int sb = m & 1;
-                ok = mbar_wait(&bar.aq_full[sb], (m >> 1) & 1, abort_flag);
-                if (ok && m >= 2) ok = mbar_wait(&bar.s_empty[sb], ((m >> 1) - 1) & 1, abort_flag);
-                if (!ok) break;
-                tc_fence_after();
+        // the whole warp runs the issue loop (waits by every lane); one elected lane issues
+        constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);
+        constexpr uint32_t id_u = idesc_bf16(128, 80, false, false);   // A, B K-major
+        constexpr uint32_t id_pv = idesc_bf16(128, 80, false, true);   // B = [V | ones] MN
+        const uint32_t aq0 = smem_u32(sm + kRdOffAq), kt = smem_u32(sm + kRdOffK);
+        const uint32_t vt = smem_u32(sm + kRdOffV), ones = smem_u32(sm + kRdOffOnes);
+        const uint32_t a0 = smem_u32(sm + kRdOffA), b0 = smem_u32(sm + kRdOffB);
+        bool ok = mbar_wait(&bar.qkv_full, 0, abort_flag);
+        // grouped score tiles S_m = (Q o w_m) K^T, double-buffered in TMEM
+        for (int m = 0; m <= G && ok; ++m) {
+            const int sb = m & 1;
+            ok = mbar_wait(&bar.aq_full[sb], (m >> 1) & 1, abort_flag);
+            if (ok && m >= 2) ok = mbar_wait(&bar.s_empty[sb], ((m >> 1) - 1) & 1, abort_flag);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            tc_fence_after();
+            if (elect_one()) {
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
                     mma_bf16(tmem + kColS0 + sb * 128,
@@ -799,10 +690,13 @@ __device__ void reader_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Pa
                              sdesc_sw128(kt + ks * 32, 16, 1024), id_s, ks > 0 ? 1u : 0u);
                 mma_commit(&bar.s_full[sb]);
             }
-            // intra-chunk term: U = P [V | 1]
-            if (ok) ok = mbar_wait(&bar.p_full, 0, abort_flag);
-            if (ok) {
-                tc_fence_after();
+            __syncwarp();
+        }
+        // intra-chunk term: U = P [V | 1]
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar.p_full, 0, abort_flag));
+        if (ok) {
+            tc_fence_after();
+            if (elect_one()) {
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
                     mma_bf16(tmem + kColU,
@@ -810,25 +704,40 @@ __device__ void reader_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Pa
                              sdesc_sw128(vt + ks * 2048, ones - vt, 1024), id_pv,
                              ks > 0 ? 1u : 0u);
             }
-            // inter-chunk readout U += phi(Q_c) S_c: A from TMEM, B = state image (K-major)
-            for (int s = 0; s < kSlices && ok && has_inter; ++s) {
-                const int st = s % kRdStages, bsi = s % kBStages;
-                ok = mbar_wait(&bar.a_full[st], (s / kRdStages) & 1, abort_flag) &&
-                     mbar_wait(&bar.b_full[bsi], (s / kBStages) & 1, abort_flag);
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t bs = b0 + bsi * kImgSliceBytes;
+            __syncwarp();
+        }
+        // inter-chunk readout U += phi(Q_c) S_c, two slices (one image stage) per round:
+        // A = phi slices 2u, 2u + 1 (stages of sets 2u % 4, (2u + 1) % 4), B = image pair u
+        for (int u = 0; u < kSlices / 2 && ok && has_inter; ++u) {
+            const int s0 = 2 * u, bs = u % kBStages;
+            ok = mbar_wait(&bar.a_full[s0 % kRdStages], (s0 / kRdStages) & 1, abort_flag) &&
+                 mbar_wait(&bar.a_full[(s0 + 1) % kRdStages], ((s0 + 1) / kRdStages) & 1,
+                           abort_flag) &&
+                 mbar_wait(&bar.b_full[bs], (u / kBStages) & 1, abort_flag);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            tc_fence_after();
+            if (elect_one()) {
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ts(tmem + kColU, tmem + kColA0 + st * 32 + ks * 8,
-                                sdesc_sw128(bs + ks * 32, 16, 1024), id_u, 1u);
-                mma_commit(&bar.a_empty[st]);
-                mma_commit(&bar.b_empty[bsi]);
+                for (int x = 0; x < 2; ++x) {
+                    const int st = (s0 + x) % kRdStages;
+                    const uint32_t bsl = b0 + bs * kImgPairBytes + x * kImgSliceBytes;
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_bf16(tmem + kColU,
+                                 sdesc_sw128(a0 + st * kPhiTileBytes + ks * 32, 16, 1024),
+                                 sdesc_sw128(bsl + ks * 32, 16, 1024), id_u, 1u);
+                    mma_commit(&bar.a_empty[st]);
+                }
+                mma_commit(&bar.b_empty[bs]);
             }
+            __syncwarp();
+        }
+        if (elect_one()) {
             if (ok) mma_commit(&bar.u_full);
             mma_commit(&bar.done);
-            bounded_spin_done(&bar.done, 0);
         }
+        __syncwarp();
+        if (lane == 0) bounded_spin_done(&bar.done, 0);
         __syncwarp();
     } else {
         const int qw = warp & 3, kq = warp >> 2, row = qw * 32 + lane;
@@ -836,6 +745,7 @@ __device__ void reader_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Pa
         const uint32_t aq0 = smem_u32(sm + kRdOffAq);
         const uint32_t lanebase = tmem + (uint32_t(qw * 32) << 16);
         bool ok = mbar_wait(&bar.qkv_full, 0, abort_flag);
+
 
         // ---- intra-chunk phase ----
         // Aq_m = Q o w_m (bf16, K-major); this warp writes dims [16 kq, 16 kq + 16)
@@ -857,10 +767,35 @@ __device__ void reader_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Pa
             fence_proxy_async();
             warp_arrive(&bar.aq_full[m & 1]);
         };
+        // phi slice s of this row -> shared stage s % 4 = kq (K-major, 128B-swizzled rows)
+        const uint32_t a0 = smem_u32(sm + kRdOffA);
+        auto produce_phi = [&](int s) -> bool {
+            const int st = s % kRdStages;
+            uint32_t w[32];
+            if (s < kOffDiagSlices) phi_offdiag(qt, coefh, s, row, w);
+            else phi_diag(qt, coef, s, row, w);
+            if (s >= kRdStages &&
+                !mbar_wait(&bar.a_empty[st], ((s / kRdStages) - 1) & 1, abort_flag))
+                return false;
+            const uint32_t base = a0 + st * kPhiTileBytes;
+#pragma unroll
+            for (int x = 0; x < 8; ++x)
+                sts128(base + kmajor_chunk(row, x), w[4 * x], w[4 * x + 1], w[4 * x + 2],
+                       w[4 * x + 3]);
+            fence_proxy_async();
+            warp_arrive(&bar.a_full[st]);
+            return true;
+        };
         if (ok) {
-            // bf16 copy of the off-diagonal coefficients (read in the inter-chunk phase)
+            // bf16 copy of the off-diagonal coefficients (read by phi)
             for (int i = threadIdx.x; i < kOffDiagRows / 2; i += 16 * 32)
                 coefh[i] = pack_bf16x2(coef[2 * i], coef[2 * i + 1]);
+        }
+        named_bar_sync(1, 16 * 32);
+        if (ok) {
+            // the first phi slice of this set is staged before the intra-chunk phase, so the
+            // readout MMAs can start as soon as the intra-chunk ones are issued
+            if (has_inter) ok = produce_phi(kq);
             produce_aq(0);
             if (G >= 1) produce_aq(1);
         }
@@ -913,29 +848,9 @@ __device__ void reader_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Pa
             fence_proxy_async();
             warp_arrive(&bar.p_full);
         }
-        // every score tile has been read (and coefh written) before TMEM columns 128.. are
-        // reused as phi stages
-        tc_fence_before();
-        named_bar_sync(1, 16 * 32);
-        tc_fence_after();
-
-        // ---- inter-chunk phase: phi(Q_c) slices kq, kq + 4, ... ----
-        for (int s = kq; s < kSlices && ok && has_inter; s += kPhiSets) {
-            const int st = s % kRdStages;
-            uint32_t w[32];
-            if (s < kOffDiagSlices) phi_offdiag(qt, coefh, s, row, w);
-            else phi_diag(qt, coef, s, row, w);
-            if (s >= kRdStages &&
-                !mbar_wait(&bar.a_empty[st], ((s / kRdStages) - 1) & 1, abort_flag)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            tmem_st32(lanebase + kColA0 + st * 32, w);
-            tmem_st_wait();
-            tc_fence_before();
-            warp_arrive(&bar.a_full[st]);
-        }
+        // ---- inter-chunk phase: phi(Q_c) slices kq + 4, kq + 8, ... ----
+        for (int s = kq + kPhiSets; s < kSlices && ok && has_inter; s += kPhiSets)
+            ok = produce_phi(s);
 
         // ---- epilogue: yhat = u[:64] / u[64], columns [16 kq, 16 kq + 16) of this row ----
         if (ok) ok = mbar_wait(&bar.u_full, 0, abort_flag);
@@ -960,25 +875,19 @@ __device__ void reader_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Pa
 }
 
 // ------------------------------------------------------------------------------------------
-// kernels: 0 = builders (grid 17 x B*Hkv x (1 + nseg): z = 0 chain, z > 0 remainder segment
-// z - 1), 1 = readers (grid NC x B*Hq), 2 = persistent queue over all items
+// kernels: 0 = chunk deltas (persistent: CTA i takes a contiguous range of units),
+// 1 = readers (grid NC x B*Hq).  Both may be launched as programmatic dependents of the
+// preceding kernel in the stream: griddepcontrol.wait orders every read of its outputs.
 // ------------------------------------------------------------------------------------------
-__device__ __forceinline__ void run_builder(unsigned char* sm, Ctl& ctl, uint32_t tmem,
-                                            const Params& P, int bkv, int slab, int seg)
-{
-    if (seg < 0) {
-        builder_item<false>(sm, ctl, tmem, P, bkv, slab, 0, P.NC);
-    } else {
-        const int c0 = seg * kSegChunks, c1 = min(P.NC, c0 + kSegChunks);
-        builder_item<true>(sm, ctl, tmem, P, bkv, slab, c0, c1);
-    }
-}
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 template <int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, Params P)
+                      const __grid_constant__ CUtensorMap tm_v,
+                      const __grid_constant__ CUtensorMap tm_img, Params P)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>(
@@ -988,55 +897,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     P.tm_q = &tm_q;
     P.tm_k = &tm_k;
     P.tm_v = &tm_v;
+    P.tm_img = &tm_img;
 
     if (warp == kMmaWarp) {
         tmem_alloc(&ctl.tmem_base, kTmemCols);
         tmem_relinquish();
     }
-    init_ones_atom(sm + kOffOnes);  // both item kinds read it; neither writes that region
+    init_ones_atom(sm + (kMode == 0 ? kOffOnes : kRdOffOnes));
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ctl.tmem_base;
+    grid_dep_launch();  // the next kernel may start its prologue
+    grid_dep_wait();    // outputs of the previous kernel are visible from here on
 
     if (kMode == 0) {
-        run_builder(sm, ctl, tmem, P, blockIdx.y, blockIdx.x, int(blockIdx.z) - 1);
-    } else if (kMode == 1) {
-        reader_item(sm, ctl, tmem, P, blockIdx.y, blockIdx.x);
+        const int units = P.B * P.Hkv * P.NC * kNumSlabs;
+        const int u0 = int((long long)units * blockIdx.x / gridDim.x);
+        const int u1 = int((long long)units * (blockIdx.x + 1) / gridDim.x);
+        if (u1 > u0) delta_item(sm, ctl, tmem, P, u0, u1);
     } else {
-        // per batch element: chain builders, then readers (chunk-major), then remainders
-        const int nb = P.Hkv * kNumSlabs, nr = P.Hq * P.NC, nl = nb * P.nseg;
-        const int per_b = nb + nr + nl, total = P.B * per_b;
-        while (true) {
-            if (threadIdx.x == 0) ctl.item = int(atomicAdd(P.queue, 1u));
-            __syncthreads();
-            const int item = ctl.item;
-            if (item >= total) break;
-            const int b = item / per_b, r = item % per_b;
-            int kind;
-            if (r < nb) {
-                kind = 0;
-                run_builder(sm, ctl, tmem, P, b * P.Hkv + r / kNumSlabs, r % kNumSlabs, -1);
-            } else if (r < nb + nr) {
-                kind = 1;
-                const int rr = r - nb;
-                reader_item(sm, ctl, tmem, P, b * P.Hq + rr % P.Hq, rr / P.Hq);
-            } else {
-                kind = 0;
-                const int rr = r - nb - nr, unit = rr % nb;
-                run_builder(sm, ctl, tmem, P, b * P.Hkv + unit / kNumSlabs, unit % kNumSlabs,
-                            rr / nb);
-            }
-            tc_fence_before();
-            __syncthreads();
-            tc_fence_after();
-            // the barrier memory is reused by the next item (possibly of the other kind)
-            if (threadIdx.x == 0) {
-                if (kind == 0) inval_builder_bars(ctl.bar.st);
-                else inval_reader_bars(ctl.bar.rd);
-            }
-        }
+        reader_item(sm, ctl, tmem, P, blockIdx.y, blockIdx.x);
     }
 
     tc_fence_before();
@@ -1044,6 +926,69 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// Exclusive prefix over chunks of one (bkv, 64-row slice, 8 columns): image_c =
+// bf16(sum_{c' < c} dS_c') for c >= 1, stored row-major as [80 n][64 f] per slice (the
+// readout's tensor copy swizzles it into the K-major B-operand layout; rows 65.. are never
+// read), final state = sum over all chunks.  Thread = (n, row pair).
+constexpr int kScanCols = 8;
+constexpr int kImgRows = 80;
+__global__ void __launch_bounds__(256) scan_kernel(const float* __restrict__ dS,
+                                                   unsigned char* __restrict__ img,
+                                                   float* __restrict__ body, int NC)
+{
+    grid_dep_launch();
+    grid_dep_wait();
+    const int sl = blockIdx.x, bkv = blockIdx.z;
+    const int nl = threadIdx.x >> 5, p = threadIdx.x & 31;
+    const int n = blockIdx.y * kScanCols + nl;
+    __shared__ float fin[kScanCols][64 + 1];
+    float a0 = 0.f, a1 = 0.f;
+    if (n >= kW && n < kImgRows) {
+        // rows 65..79 of every image: zero (the readout's N = 80 MMA reads them)
+        unsigned char* dst = img + (size_t(bkv) * NC * kSlices + sl) * kImgSliceBytes + n * 128 + 4 * p;
+        for (int c = 1; c < NC; ++c)
+            *reinterpret_cast<uint32_t*>(dst + size_t(c) * kSlices * kImgSliceBytes) = 0u;
+    }
+    if (n < kW) {
+        const float* src = dS + (size_t(bkv) * NC * kW + n) * kFP + sl * 64 + 2 * p;
+        unsigned char* dst = img + (size_t(bkv) * NC * kSlices + sl) * kImgSliceBytes +
+                             n * 128 + 4 * p;
+        const size_t sstride = size_t(kW) * kFP, dstride = size_t(kSlices) * kImgSliceBytes;
+        int c = 0;
+        for (; c + 4 <= NC; c += 4) {
+            float2 d[4];
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+                d[x] = __ldcs(reinterpret_cast<const float2*>(src + (c + x) * sstride));
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                if (c + x >= 1)
+                    *reinterpret_cast<uint32_t*>(dst + (c + x) * dstride) = pack_bf16x2(a0, a1);
+                a0 += d[x].x;
+                a1 += d[x].y;
+            }
+        }
+        for (; c < NC; ++c) {
+            const float2 d = __ldcs(reinterpret_cast<const float2*>(src + c * sstride));
+            if (c >= 1) *reinterpret_cast<uint32_t*>(dst + c * dstride) = pack_bf16x2(a0, a1);
+            a0 += d.x;
+            a1 += d.y;
+        }
+    }
+    fin[nl][2 * p] = a0;
+    fin[nl][2 * p + 1] = a1;
+    __syncthreads();
+    // final state of unit bkv: Hv[f][n] (n < 64), z[f] (n == 64)
+    float* unit = body + size_t(bkv) * kFP * kW;
+    const int fl = threadIdx.x >> 2, cq = threadIdx.x & 3;
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+        const int nn = blockIdx.y * kScanCols + 2 * cq + x;
+        if (nn < kDV) unit[size_t(sl * 64 + fl) * kDV + nn] = fin[2 * cq + x][fl];
+        else if (nn == kDV) unit[size_t(kFP) * kDV + sl * 64 + fl] = fin[2 * cq + x][fl];
     }
 }
 
@@ -1089,6 +1034,22 @@ bool make_map(CUtensorMap* m, const void* base, int T, int heads)
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// chunk-state images [slices][80 rows][64] bf16 viewed as 2D {64, slices * 80}; box {64, 160}
+// = two consecutive slices per copy (copies from L2 cost about the same per copy from 8 to
+// 20 KB, so fewer and larger ones); 128B swizzle on the way in.
+bool make_img_map(CUtensorMap* m, const void* base, size_t slices)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {64, cuuint64_t(slices) * 80};
+    const cuuint64_t strides[1] = {128};
+    const cuuint32_t box[2] = {64, 160};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int sm_count()
 {
     int dev = 0, n = 0;
@@ -1108,25 +1069,50 @@ size_t tc_image_bytes(int B, int Hkv, int T)
 size_t tc_workspace_bytes(int B, int Hkv, int T)
 {
     const size_t NC = size_t((T + tc::kC - 1) / tc::kC);
-    return tc_image_bytes(B, Hkv, T) + align256((size_t(B) * Hkv * NC + 1) * 4);
+    return tc_image_bytes(B, Hkv, T) + size_t(B) * Hkv * NC * kW * kFP * 4;
 }
+
+namespace {
+
+// Launch with the programmatic-dependent attribute: the kernel may be scheduled while its
+// predecessor in the stream is still running, and waits for it in griddepcontrol.wait.
+template <typename... Args>
+cudaError_t launch_ex(void (*kern)(Args...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                      bool dependent, Args... args)
+{
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = dependent ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+}  // namespace
 
 int launch_prefill_tc(const void* q, const void* k, const void* v, const int32_t* gid,
                       const float* L, const int32_t* G, float eps, float* out, void* state,
-                      void* ws, int B, int T, int Hq, int Hkv, bool fused, cudaStream_t st)
+                      void* ws, int B, int T, int Hq, int Hkv, bool overlap, cudaStream_t st)
 {
     if (B == 0) return OAL_OK;
     const int NC = (T + tc::kC - 1) / tc::kC;
     unsigned char* sb = static_cast<unsigned char*>(state);
     float* body = reinterpret_cast<float*>(sb + kHeaderBytes + coef_bytes(Hq));
-    // chain builders and remainder items add their sums into the final state
-    OAL_CUDA_TRY(cudaMemsetAsync(body, 0, size_t(B) * Hkv * state_unit_bytes(), st));
-    if (T == 0) return OAL_OK;
-    CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, q, T, B * Hq) || !make_map(&mk, k, T, B * Hkv) ||
-        !make_map(&mv, v, T, B * Hkv))
-        return OAL_ERR_CUDA;
+    if (T == 0) {
+        OAL_CUDA_TRY(cudaMemsetAsync(body, 0, size_t(B) * Hkv * state_unit_bytes(), st));
+        return OAL_OK;
+    }
     unsigned char* wsb = static_cast<unsigned char*>(ws);
+    CUtensorMap mq, mk, mv, mi;
+    if (!make_map(&mq, q, T, B * Hq) || !make_map(&mk, k, T, B * Hkv) ||
+        !make_map(&mv, v, T, B * Hkv) ||
+        !make_img_map(&mi, wsb, size_t(B) * Hkv * NC * tc::kSlices))
+        return OAL_ERR_CUDA;
     tc::Params P{};
     P.gid = gid;
     P.L = L;
@@ -1134,61 +1120,36 @@ int launch_prefill_tc(const void* q, const void* k, const void* v, const int32_t
     P.eps = eps;
     P.coef_all = reinterpret_cast<const float*>(sb + kHeaderBytes);
     P.img = wsb;
-    P.body = body;
+    P.dS = reinterpret_cast<float*>(wsb + tc_image_bytes(B, Hkv, T));
     P.out = out;
     P.B = B;
     P.Hq = Hq;
     P.Hkv = Hkv;
     P.T = T;
     P.NC = NC;
-    P.nseg = (NC + tc::kSegChunks - 1) / tc::kSegChunks;
-    unsigned int* ctl = reinterpret_cast<unsigned int*>(wsb + tc_image_bytes(B, Hkv, T));
-    const size_t ctl_words = size_t(B) * Hkv * NC + 1;
-    if (fused) {
-        const int items = B * (Hkv * tc::kNumSlabs * (1 + P.nseg) + Hq * NC);
-        const int grid = std::min(sm_count(), items);
-        if (grid > 0 &&
-            cudaFuncSetAttribute(tc::prefill_tc_kernel<2>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 int(tc::kSmemBytes)) == cudaSuccess &&
-            cudaMemsetAsync(ctl, 0, ctl_words * 4, st) == cudaSuccess) {
-            P.queue = ctl;
-            P.flags = ctl + 1;
-            cudaLaunchConfig_t cfg{};
-            cfg.gridDim = dim3(grid);
-            cfg.blockDim = dim3(tc::kThreads);
-            cfg.dynamicSmemBytes = tc::kSmemBytes;
-            cfg.stream = st;
-            cudaLaunchAttribute attr[1];
-            attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident at once
-            attr[0].val.cooperative = 1;
-            cfg.attrs = attr;
-            cfg.numAttrs = 1;
-            LaunchScope ls("prefill_tc", st);
-            if (cudaLaunchKernelEx(&cfg, tc::prefill_tc_kernel<2>, mq, mk, mv, P) == cudaSuccess)
-                return OAL_OK;
-        }
-        cudaGetLastError();  // not launchable as one resident grid: use the two-kernel form
-        P.queue = nullptr;
-        P.flags = nullptr;
+    const int units = B * Hkv * NC * tc::kNumSlabs;
+    const int grid0 = std::max(1, std::min(sm_count(), units));
+    OAL_CUDA_TRY(cudaFuncSetAttribute(tc::prefill_tc_kernel<0>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      int(tc::kSmemBytes)));
+    OAL_CUDA_TRY(cudaFuncSetAttribute(tc::prefill_tc_kernel<1>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      int(tc::kSmemBytes)));
+    {
+        LaunchScope ls("delta_tc", st);
+        OAL_CUDA_TRY(launch_ex(tc::prefill_tc_kernel<0>, dim3(grid0), dim3(tc::kThreads),
+                               tc::kSmemBytes, st, false, mq, mk, mv, mi, P));
     }
     {
-        OAL_CUDA_TRY(cudaFuncSetAttribute(tc::prefill_tc_kernel<0>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 int(tc::kSmemBytes)));
-        LaunchScope ls("state_tc", st);
-        tc::prefill_tc_kernel<0><<<dim3(tc::kNumSlabs, B * Hkv, 1 + P.nseg), tc::kThreads,
-                                   tc::kSmemBytes, st>>>(mq, mk, mv, P);
-        OAL_LAUNCH_CHECK();
+        LaunchScope ls("scan", st);
+        OAL_CUDA_TRY(launch_ex(tc::scan_kernel,
+                               dim3(tc::kSlices, tc::kImgRows / tc::kScanCols, B * Hkv),
+                               dim3(256), 0, st, overlap, (const float*)P.dS, P.img, body, NC));
     }
     {
-        OAL_CUDA_TRY(cudaFuncSetAttribute(tc::prefill_tc_kernel<1>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 int(tc::kSmemBytes)));
         LaunchScope ls("readout_tc", st);
-        tc::prefill_tc_kernel<1><<<dim3(NC, B * Hq), tc::kThreads, tc::kSmemBytes, st>>>(
-            mq, mk, mv, P);
-        OAL_LAUNCH_CHECK();
+        OAL_CUDA_TRY(launch_ex(tc::prefill_tc_kernel<1>, dim3(NC, B * Hq), dim3(tc::kThreads),
+                               tc::kSmemBytes, st, overlap, mq, mk, mv, mi, P));
     }
     return OAL_OK;
 }

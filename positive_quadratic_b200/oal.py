@@ -74,8 +74,8 @@ def lib() -> ctypes.CDLL:
             L.oal_launch_count.restype = ctypes.c_ulonglong
             L.oal_last_cuda_error.argtypes = [ctypes.c_char_p, ctypes.c_size_t]
             L.oal_last_cuda_error.restype = ctypes.c_int
-            L.oal_set_prefill_fused.argtypes = [ctypes.c_int]
-            L.oal_set_prefill_fused.restype = ctypes.c_int
+            L.oal_set_prefill_overlap.argtypes = [ctypes.c_int]
+            L.oal_set_prefill_overlap.restype = ctypes.c_int
             L.oal_profile_enable.argtypes = [ctypes.c_int]
             L.oal_profile_enable.restype = ctypes.c_int
             L.oal_profile_read.argtypes = [ctypes.POINTER(KernelStat), ctypes.c_int,
@@ -292,7 +292,7 @@ def profile_read() -> dict:
             for i in range(n.value)}
 
 
-def set_prefill_fused(fused: bool) -> bool:
-    """Select the tensor-core prefill schedule (persistent fused kernel or two kernels);
-    returns the previous setting."""
-    return bool(lib().oal_set_prefill_fused(1 if fused else 0))
+def set_prefill_overlap(overlap: bool) -> bool:
+    """Launch the tensor-core prefill's scan and readout kernels as programmatic dependents
+    (True) or in plain stream order (False); returns the previous setting."""
+    return bool(lib().oal_set_prefill_overlap(1 if overlap else 0))

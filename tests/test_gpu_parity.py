@@ -251,14 +251,15 @@ def test_config4_decode_sampled(oal, cuda):
 
 # --- tensor-core prefill schedules --------------------------------------------------------------
 
-@pytest.mark.parametrize("fused", [True, False])
+@pytest.mark.parametrize("overlap", [True, False])
 @pytest.mark.parametrize("T,B", [(129, 1), (300, 2), (1000, 3), (2048, 1)])
-def test_tensor_prefill_schedules(oal, cuda, fused, T, B):
-    """bf16, chunk 128 runs on the tcgen05 kernels: persistent fused schedule and the
-    two-kernel schedule both match the oracle (outputs and exact final state)."""
+def test_tensor_prefill_schedules(oal, cuda, overlap, T, B):
+    """bf16, chunk 128 runs on the tcgen05 kernels (chunk deltas, prefix scan, readout),
+    with and without programmatic dependent launch: outputs and exact final state match the
+    oracle."""
     p = I.small_layer(500 + T, B=B, T=T, Hq=14, Hkv=2, dtype="bf16")
     ref, st = oracle.recurrent(p.q, p.k, p.v, p.group_id, p.L, p.G, p.eps, return_state=True)
-    prev = oal.set_prefill_fused(fused)
+    prev = oal.set_prefill_overlap(overlap)
     try:
         oal.profile_read()
         oal.profile_enable(True)
@@ -266,8 +267,8 @@ def test_tensor_prefill_schedules(oal, cuda, fused, T, B):
         oal.profile_enable(False)
         names = set(oal.profile_read())
     finally:
-        oal.set_prefill_fused(prev)
-    assert ("prefill_tc" in names) if fused else ({"state_tc", "readout_tc"} <= names), names
+        oal.set_prefill_overlap(prev)
+    assert {"delta_tc", "scan", "readout_tc"} <= names, names
     assert row_rel_err(y, ref) <= TOL_BF16
     _, _, S = read_state(state.cpu().numpy(), B, 14, 2)
     refS = pack_oracle_state(st)
@@ -276,11 +277,11 @@ def test_tensor_prefill_schedules(oal, cuda, fused, T, B):
 
 def test_tensor_schedules_agree(oal, cuda):
     p = I.config1()
-    prev = oal.set_prefill_fused(True)
+    prev = oal.set_prefill_overlap(True)
     try:
         y1, _ = gpu_prefill(oal, p, cuda, 128)
-        oal.set_prefill_fused(False)
+        oal.set_prefill_overlap(False)
         y2, _ = gpu_prefill(oal, p, cuda, 128)
     finally:
-        oal.set_prefill_fused(prev)
+        oal.set_prefill_overlap(prev)
     np.testing.assert_array_equal(y1, y2)
