@@ -12,8 +12,9 @@
 
 namespace oal {
 
-// 4 MiB: room for the per-(b, kv) tickets and per-slab partial readouts of a decode step
-// with B*Hq up to 948 query heads in flight (batch 64 x 14 heads needs 3.96 MB).
+// 4 MiB: room for the per-(b, kv) tickets and per-slab partial readouts (9 slabs x 65 fp32
+// per query head) of a decode step with B*Hq up to 1788 query heads (batch 64 x 14 heads
+// needs 2.1 MB).
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];

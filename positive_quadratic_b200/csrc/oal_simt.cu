@@ -6,6 +6,8 @@
 // arXiv 2610.13674), section 核心公式, numbered in order of appearance: (2) grouped score,
 // (3) kernel kappa, (4) prefix states H0/H1/H2, (5) readout.  The packed feature map that
 // merges H0/H1/H2 into one state is described in oal_common.cuh.
+#include <type_traits>
+
 #include "oal_common.cuh"
 #include "oal_kernels.cuh"
 
@@ -336,28 +338,32 @@ __global__ void __launch_bounds__(256) readout_simt_kernel(
 }
 
 // ------------------------------------------------------------------------------------------
-// a11: decode step.  Block (slab, bkv) streams 128 packed rows of one (b, kv) state once:
+// a11: decode step.  Block (slab, bkv) streams 240 packed rows of one (b, kv) state once:
 // S_f += psi_f(k) [v; 1] (eq. (4) with one new token), then accumulates
 // u_h += phi_{h,f}(q_h) S_f for the Hq/Hkv query heads of that kv head (eq. (5)).  Row data
 // moves as 128-bit loads and stores (a half warp per 256-byte row).  Per-block partial u go
 // to the workspace; the last block of a (b, kv) (atomic ticket) sums them, writes yhat and
 // re-arms the ticket.
 // ------------------------------------------------------------------------------------------
-constexpr int kDecRows = 128;
+// 9 slabs of 240 packed rows per (b, kv) head: 256 threads, at most 64 registers, so four
+// blocks share an SM and a batch-64 step (1152 blocks) runs in two nearly full waves.
+constexpr int kDecRows = 240;
+constexpr int kDecThreads = 256;
 
-template <typename Tin>
-__global__ void __launch_bounds__(256) decode_kernel(const Tin* __restrict__ q,
-                                                     const Tin* __restrict__ k,
-                                                     const Tin* __restrict__ v,
-                                                     unsigned char* __restrict__ state,
-                                                     float* __restrict__ out,
-                                                     float* __restrict__ part,
-                                                     unsigned int* __restrict__ tickets, int Hq,
-                                                     int Hkv)
+template <typename Tin, int kGrp>  // kGrp = Hq / Hkv query heads per kv head
+__global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const Tin* __restrict__ q,
+                                                              const Tin* __restrict__ k,
+                                                              const Tin* __restrict__ v,
+                                                              unsigned char* __restrict__ state,
+                                                              float* __restrict__ out,
+                                                              float* __restrict__ part,
+                                                              unsigned int* __restrict__ tickets,
+                                                              int Hq, int Hkv)
 {
     const int slab = blockIdx.x, bkv = blockIdx.y, nslab = gridDim.x;
-    const int b = bkv / Hkv, kv = bkv % Hkv, grp = Hq / Hkv, h0 = kv * grp;
-    const int tid = threadIdx.x, lane4 = tid & 15, rsub = tid >> 4, warp = tid >> 5;
+    constexpr int grp = kGrp;
+    const int b = bkv / Hkv, kv = bkv % Hkv, h0 = kv * grp;
+    const int tid = threadIdx.x, lane4 = tid & 15, rsub = tid >> 4;
     const float* coef = reinterpret_cast<const float*>(state + kHeaderBytes);
     float* unit = reinterpret_cast<float*>(state + kHeaderBytes + coef_bytes(Hq)) +
                   size_t(bkv) * kFP * kW;
@@ -369,8 +375,7 @@ __global__ void __launch_bounds__(256) decode_kernel(const Tin* __restrict__ q,
     __shared__ float qh[kMaxGroup][kDA];
     __shared__ float phis[kDecRows][kMaxGroup + 1];
     __shared__ float psis[kDecRows];
-    __shared__ float red[8][kMaxGroup][kDV];
-    __shared__ float redz[8][kMaxGroup];
+    __shared__ float red[kMaxGroup][kW];
     __shared__ float ufin[kMaxGroup][kW];
     __shared__ int s_last;
 
@@ -382,14 +387,15 @@ __global__ void __launch_bounds__(256) decode_kernel(const Tin* __restrict__ q,
         kh[kD + 1] = 0.f;
         vh[kDV] = 1.f;
     }
-    for (int e = tid; e < grp * kDA; e += 256) {
+    for (int e = tid; e < grp * kDA; e += kDecThreads) {
         const int g = e / kDA, r = e % kDA;
         qh[g][r] = r < kD ? to_f32(q[(size_t(b) * Hq + h0 + g) * kD + r]) : (r == kD ? 1.f : 0.f);
     }
+    for (int e = tid; e < kMaxGroup * kW; e += kDecThreads) (&red[0][0])[e] = 0.f;
     __syncthreads();
     const int f0 = slab * kDecRows;
-    const int nrows = min(kDecRows, kF - f0);
-    for (int row = tid; row < nrows; row += 256) {
+    const int nrows = max(0, min(kDecRows, kF - f0));
+    for (int row = tid; row < nrows; row += kDecThreads) {
         const int f = f0 + row;
         const RT rt = feature_rt(f);
         psis[row] = kh[rt.r] * kh[rt.t];
@@ -398,65 +404,57 @@ __global__ void __launch_bounds__(256) decode_kernel(const Tin* __restrict__ q,
     }
     __syncthreads();
 
-    float acc[kMaxGroup][4];
+    // eq. (4) rank-1 update of Hv and eq. (5) readout, one 64-float row per half-warp
+    float acc[kGrp][4];
 #pragma unroll
-    for (int g = 0; g < kMaxGroup; ++g) acc[g][0] = acc[g][1] = acc[g][2] = acc[g][3] = 0.f;
+    for (int g = 0; g < kGrp; ++g) acc[g][0] = acc[g][1] = acc[g][2] = acc[g][3] = 0.f;
     const float4 v4 = *reinterpret_cast<const float4*>(&vh[lane4 * 4]);
 #pragma unroll 4
-    for (int row = rsub; row < nrows; row += 16) {
+    for (int row = rsub; row < nrows; row += kDecThreads / 16) {
         float4* p = reinterpret_cast<float4*>(Hv + size_t(f0 + row) * kDV) + lane4;
-        float4 hv = *p;
+        float4 hv = __ldcs(p);
         const float psi = psis[row];
         hv.x = fmaf(psi, v4.x, hv.x);
         hv.y = fmaf(psi, v4.y, hv.y);
         hv.z = fmaf(psi, v4.z, hv.z);
         hv.w = fmaf(psi, v4.w, hv.w);
-        *p = hv;
+        __stcs(p, hv);
 #pragma unroll
-        for (int g = 0; g < kMaxGroup; ++g) {
-            if (g < grp) {
-                const float ph = phis[row][g];
-                acc[g][0] = fmaf(ph, hv.x, acc[g][0]);
-                acc[g][1] = fmaf(ph, hv.y, acc[g][1]);
-                acc[g][2] = fmaf(ph, hv.z, acc[g][2]);
-                acc[g][3] = fmaf(ph, hv.w, acc[g][3]);
-            }
+        for (int g = 0; g < kGrp; ++g) {
+            const float ph = phis[row][g];
+            acc[g][0] = fmaf(ph, hv.x, acc[g][0]);
+            acc[g][1] = fmaf(ph, hv.y, acc[g][1]);
+            acc[g][2] = fmaf(ph, hv.z, acc[g][2]);
+            acc[g][3] = fmaf(ph, hv.w, acc[g][3]);
         }
     }
-    float accz[kMaxGroup];
+    float accz[kGrp];
 #pragma unroll
-    for (int g = 0; g < kMaxGroup; ++g) accz[g] = 0.f;
-    if (tid < nrows) {
-        const float zz = z[f0 + tid] + psis[tid];
-        z[f0 + tid] = zz;
+    for (int g = 0; g < kGrp; ++g) accz[g] = 0.f;
+    for (int row = tid; row < nrows; row += kDecThreads) {
+        const float zz = z[f0 + row] + psis[row];
+        z[f0 + row] = zz;
 #pragma unroll
-        for (int g = 0; g < kMaxGroup; ++g)
-            if (g < grp) accz[g] = phis[tid][g] * zz;
+        for (int g = 0; g < kGrp; ++g) accz[g] = fmaf(phis[row][g], zz, accz[g]);
     }
-    // reduce: the two half-warps of a warp hold the same columns
+    // reduce: the two half-warps of a warp hold the same columns; warps meet in shared
+    // memory through atomic adds
 #pragma unroll
-    for (int g = 0; g < kMaxGroup; ++g) {
-        if (g < grp) {
+    for (int g = 0; g < kGrp; ++g) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) acc[g][c] += __shfl_xor_sync(0xffffffffu, acc[g][c], 16);
-            float zz = accz[g];
+        for (int c = 0; c < 4; ++c) acc[g][c] += __shfl_xor_sync(0xffffffffu, acc[g][c], 16);
+        float zz = accz[g];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) zz += __shfl_xor_sync(0xffffffffu, zz, o);
-            if ((tid & 31) < 16) {
+        for (int o = 16; o > 0; o >>= 1) zz += __shfl_xor_sync(0xffffffffu, zz, o);
+        if ((tid & 31) < 16) {
 #pragma unroll
-                for (int c = 0; c < 4; ++c) red[warp][g][lane4 * 4 + c] = acc[g][c];
-            }
-            if ((tid & 31) == 0) redz[warp][g] = zz;
+            for (int c = 0; c < 4; ++c) atomicAdd(&red[g][lane4 * 4 + c], acc[g][c]);
         }
+        if ((tid & 31) == 0) atomicAdd(&red[g][kDV], zz);
     }
     __syncthreads();
     float* mypart = part + (size_t(bkv) * nslab + slab) * grp * kW;
-    for (int e = tid; e < grp * kW; e += 256) {
-        const int g = e / kW, n = e % kW;
-        float s = 0.f;
-        for (int w = 0; w < 8; ++w) s += n < kDV ? red[w][g][n] : redz[w][g];
-        mypart[e] = s;
-    }
+    for (int e = tid; e < grp * kW; e += kDecThreads) mypart[e] = red[e / kW][e % kW];
     __threadfence();
     __syncthreads();
     if (tid == 0) {
@@ -467,13 +465,13 @@ __global__ void __launch_bounds__(256) decode_kernel(const Tin* __restrict__ q,
     if (!s_last) return;
     __threadfence();
     const float* allpart = part + size_t(bkv) * nslab * grp * kW;
-    for (int e = tid; e < grp * kW; e += 256) {
+    for (int e = tid; e < grp * kW; e += kDecThreads) {
         float s = 0.f;
         for (int sl = 0; sl < nslab; ++sl) s += __ldcg(allpart + size_t(sl) * grp * kW + e);
         ufin[e / kW][e % kW] = s;
     }
     __syncthreads();
-    for (int e = tid; e < grp * kDV; e += 256) {
+    for (int e = tid; e < grp * kDV; e += kDecThreads) {
         const int g = e / kDV, n = e % kDV;
         out[(size_t(b) * Hq + h0 + g) * kDV + n] = ufin[g][n] / ufin[g][kDV];
     }
@@ -482,10 +480,6 @@ __global__ void __launch_bounds__(256) decode_kernel(const Tin* __restrict__ q,
         if (bkv == 0) reinterpret_cast<StateHeader*>(state)->tokens += 1;
     }
 }
-
-// ------------------------------------------------------------------------------------------
-// launchers
-// ------------------------------------------------------------------------------------------
 int launch_prep(const int32_t* gid, const float* L, const int32_t* G, float eps, void* state,
                 int B, int Hq, int Hkv, long long tokens, cudaStream_t st)
 {
@@ -577,15 +571,30 @@ int launch_decode(const void* q, const void* k, const void* v, void* state, floa
     const dim3 grid(decode_slabs(), B * Hkv);
     unsigned char* s = static_cast<unsigned char*>(state);
     LaunchScope ls("decode", st);
-    if (dtype == OAL_BF16)
-        decode_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
-            static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-            static_cast<const __nv_bfloat16*>(v), s, out, part, tickets, Hq, Hkv);
-    else
-        decode_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(q),
-                                                   static_cast<const float*>(k),
-                                                   static_cast<const float*>(v), s, out, part,
-                                                   tickets, Hq, Hkv);
+    const int grp = Hq / Hkv;
+    const bool bf = dtype == OAL_BF16;
+    auto go = [&](auto G) {
+        constexpr int g = decltype(G)::value;
+        if (bf)
+            decode_kernel<__nv_bfloat16, g><<<grid, kDecThreads, 0, st>>>(
+                static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                static_cast<const __nv_bfloat16*>(v), s, out, part, tickets, Hq, Hkv);
+        else
+            decode_kernel<float, g><<<grid, kDecThreads, 0, st>>>(
+                static_cast<const float*>(q), static_cast<const float*>(k),
+                static_cast<const float*>(v), s, out, part, tickets, Hq, Hkv);
+    };
+    switch (grp) {
+        case 1: go(std::integral_constant<int, 1>{}); break;
+        case 2: go(std::integral_constant<int, 2>{}); break;
+        case 3: go(std::integral_constant<int, 3>{}); break;
+        case 4: go(std::integral_constant<int, 4>{}); break;
+        case 5: go(std::integral_constant<int, 5>{}); break;
+        case 6: go(std::integral_constant<int, 6>{}); break;
+        case 7: go(std::integral_constant<int, 7>{}); break;
+        case 8: go(std::integral_constant<int, 8>{}); break;
+        default: return OAL_ERR_UNSUPPORTED;
+    }
     OAL_LAUNCH_CHECK();
     return OAL_OK;
 }

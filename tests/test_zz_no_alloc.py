@@ -55,6 +55,6 @@ def test_noalloc_decode_matches_workspace_decode(cuda):
 
 def test_noalloc_rejects_too_large(cuda):
     oal, noalloc = _noalloc_fn()
-    big = oal.make_shape(128, 1, 8, 1, 128, oal.OAL_BF16)  # B*Hq = 1024 > 948
+    big = oal.make_shape(256, 1, 8, 1, 128, oal.OAL_BF16)  # B*Hq = 2048 > 1788
     P = ctypes.c_void_p(256)
     assert noalloc(P, P, P, P, P, ctypes.byref(big), None) == -3
