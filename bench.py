@@ -131,6 +131,38 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def profiled_traffic(workload_name):
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the kernels
+    captured with ncu on the config-1 workload, from the committed profile summary."""
+    if workload_name != "config1":
+        return {}
+    path = os.path.join(ROOT, "profiles", "readout_tc_config1_full.md")
+    out = {}
+    if os.path.exists(path):
+        with open(path) as f:
+            for ln in f:
+                if ln.startswith("traffic_bytes_per_launch:"):
+                    for item in ln.split(":", 1)[1].split():
+                        name, val = item.split("=")
+                        out[name] = int(val)
+    return out
+
+
+def max_over_ranks(ms, world, device):
+    """The job's time: the slowest rank's device-timed milliseconds (all ranks call this)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(world, units_per_rank, ms):
+    """Whole-job throughput: every rank processed units_per_rank units in at most ms."""
+    return world * units_per_rank / (ms / 1e3)
+
+
 def dist_setup(gpus):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -272,12 +304,8 @@ def main():
     oal.profile_enable(False)
     prof = oal.profile_read()
     step_ms = [a.elapsed_time(b) for a, b in evs]
-    total_ms = sum(step_ms)
-    tmax = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
-    total_ms = float(tmax.item())
-    value = world * args.steps * B * T / (total_ms / 1e3)
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
+    value = job_rate(world, args.steps * B * T, total_ms)
 
     # roofline of the dominant prefill kernel
     flops_state = 2.0 * B * T * F * W * Hkv
@@ -298,7 +326,8 @@ def main():
                 "TFLOP/s", "alu"
         ach = algo / (per / 1e3) / 1e12
         roof = {"bound": bound, "achieved": ach, "peak": peak, "unit": unit, "frac": ach / peak,
-                "traffic": None, "kernel": name, "avg_launch_ms": per,
+                "traffic": profiled_traffic(args.workload).get(name), "kernel": name,
+                "avg_launch_ms": per,
                 "algorithmic_flop_per_launch": algo, "peak_kind": pk_kind,
                 "kernel_shares": {n: round(t / sum(x[1] for x in prof.values()), 4)
                                   for n, (c, t) in prof.items()},
@@ -326,11 +355,8 @@ def main():
             s1.record(stream)
             flush.zero_()
         torch.cuda.synchronize()
-        e_ms = sum(a.elapsed_time(b) for a, b in evs2)
-        te = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": world * args.steps * B * T / (float(te.item()) / 1e3), "unit": UNIT,
+        e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs2), world, dev)
+        e2e = {"value": job_rate(world, args.steps * B * T, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": int(hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2),
                "d2h_bytes_per_step": int(hout.numel() * 4)}
 
@@ -400,12 +426,7 @@ def run_decode(args, dev, torch, oal, pk, pk_kind, flush, world, barrier):
     oal.profile_enable(False)
     prof = oal.profile_read()
     assert oal.device_error() == 0
-    ms = sum(a.elapsed_time(b) for a, b in evs)
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        import torch.distributed as dist
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t.item())
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world, dev)
     state_bytes = 2.0 * B * Hkv * F * W * 4   # every packed row read and written once
     io_bytes = B * (Hq + 2 * Hkv) * 64 * 2 + B * Hq * 64 * 4
     kern = prof.get("decode")
@@ -417,7 +438,7 @@ def run_decode(args, dev, torch, oal, pk, pk_kind, flush, world, barrier):
                 "frac": gbs / pk["hbm_gbs"], "frac_of_8tbs": gbs / 8000.0, "traffic": None,
                 "kernel": "decode", "avg_launch_ms": per, "peak_kind": pk_kind,
                 "algorithmic_bytes_per_launch": state_bytes + io_bytes}
-    return {"value": world * B * nsteps / (ms / 1e3), "unit": UNIT,
+    return {"value": job_rate(world, B * nsteps, ms), "unit": UNIT,
             "ms_per_token_step": ms / nsteps, "batch": B, "context": 4096, "steps": nsteps,
             "roofline": roof,
             "workload": "decode batch 64, context 4096, Hq=14 Hkv=2 d=64 bf16 q/k/v, fp32 state"}
