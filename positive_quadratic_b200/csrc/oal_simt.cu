@@ -338,20 +338,21 @@ __global__ void __launch_bounds__(256) readout_simt_kernel(
 }
 
 // ------------------------------------------------------------------------------------------
-// a11: decode step.  Block (slab, bkv) streams 240 packed rows of one (b, kv) state once:
+// a11: decode step.  Block (slab, bkv) streams 320 packed rows of one (b, kv) state once:
 // S_f += psi_f(k) [v; 1] (eq. (4) with one new token), then accumulates
 // u_h += phi_{h,f}(q_h) S_f for the Hq/Hkv query heads of that kv head (eq. (5)).  Row data
 // moves as 128-bit loads and stores (a half warp per 256-byte row).  Per-block partial u go
 // to the workspace; the last block of a (b, kv) (atomic ticket) sums them, writes yhat and
 // re-arms the ticket.
 // ------------------------------------------------------------------------------------------
-// 9 slabs of 240 packed rows per (b, kv) head: 256 threads, at most 64 registers, so four
-// blocks share an SM and a batch-64 step (1152 blocks) runs in two nearly full waves.
-constexpr int kDecRows = 240;
+// 7 slabs of 320 packed rows per (b, kv) head: 256 threads with at most 80 registers, so
+// three blocks share an SM and a batch-64 step (896 blocks) runs in two full waves.
+constexpr int kDecRows = 320;
 constexpr int kDecThreads = 256;
+constexpr int kDecBatch = 5;  // rows in flight per thread (320 rows = 4 batches of 16 x 5)
 
 template <typename Tin, int kGrp>  // kGrp = Hq / Hkv query heads per kv head
-__global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const Tin* __restrict__ q,
+__global__ void __launch_bounds__(kDecThreads, 3) decode_kernel(const Tin* __restrict__ q,
                                                               const Tin* __restrict__ k,
                                                               const Tin* __restrict__ v,
                                                               unsigned char* __restrict__ state,
@@ -409,23 +410,38 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const Tin* __res
 #pragma unroll
     for (int g = 0; g < kGrp; ++g) acc[g][0] = acc[g][1] = acc[g][2] = acc[g][3] = 0.f;
     const float4 v4 = *reinterpret_cast<const float4*>(&vh[lane4 * 4]);
-#pragma unroll 4
-    for (int row = rsub; row < nrows; row += kDecThreads / 16) {
-        float4* p = reinterpret_cast<float4*>(Hv + size_t(f0 + row) * kDV) + lane4;
-        float4 hv = __ldcs(p);
-        const float psi = psis[row];
-        hv.x = fmaf(psi, v4.x, hv.x);
-        hv.y = fmaf(psi, v4.y, hv.y);
-        hv.z = fmaf(psi, v4.z, hv.z);
-        hv.w = fmaf(psi, v4.w, hv.w);
-        __stcs(p, hv);
+    // rows in batches of kDecBatch: every load of a batch is issued before any store (the
+    // compiler cannot move a load past a store to a possibly aliasing row by itself)
+    constexpr int kRowStep = kDecThreads / 16;
+#pragma unroll 1
+    for (int base = rsub; base < nrows; base += kRowStep * kDecBatch) {
+        float4 hv[kDecBatch];
 #pragma unroll
-        for (int g = 0; g < kGrp; ++g) {
-            const float ph = phis[row][g];
-            acc[g][0] = fmaf(ph, hv.x, acc[g][0]);
-            acc[g][1] = fmaf(ph, hv.y, acc[g][1]);
-            acc[g][2] = fmaf(ph, hv.z, acc[g][2]);
-            acc[g][3] = fmaf(ph, hv.w, acc[g][3]);
+        for (int x = 0; x < kDecBatch; ++x) {
+            const int row = base + kRowStep * x;
+            if (row < nrows)
+                hv[x] = __ldcs(reinterpret_cast<const float4*>(Hv + size_t(f0 + row) * kDV) + lane4);
+        }
+#pragma unroll
+        for (int x = 0; x < kDecBatch; ++x) {
+            const int row = base + kRowStep * x;
+            if (row < nrows) {
+                const float psi = psis[row];
+                float4 h = hv[x];
+                h.x = fmaf(psi, v4.x, h.x);
+                h.y = fmaf(psi, v4.y, h.y);
+                h.z = fmaf(psi, v4.z, h.z);
+                h.w = fmaf(psi, v4.w, h.w);
+                __stcs(reinterpret_cast<float4*>(Hv + size_t(f0 + row) * kDV) + lane4, h);
+#pragma unroll
+                for (int g = 0; g < kGrp; ++g) {
+                    const float ph = phis[row][g];
+                    acc[g][0] = fmaf(ph, h.x, acc[g][0]);
+                    acc[g][1] = fmaf(ph, h.y, acc[g][1]);
+                    acc[g][2] = fmaf(ph, h.z, acc[g][2]);
+                    acc[g][3] = fmaf(ph, h.w, acc[g][3]);
+                }
+            }
         }
     }
     float accz[kGrp];

@@ -55,6 +55,11 @@ def test_noalloc_decode_matches_workspace_decode(cuda):
 
 def test_noalloc_rejects_too_large(cuda):
     oal, noalloc = _noalloc_fn()
-    big = oal.make_shape(256, 1, 8, 1, 128, oal.OAL_BF16)  # B*Hq = 2048 > 1788
+    big = oal.make_shape(1024, 1, 8, 1, 128, oal.OAL_BF16)  # B*Hq = 8192
+    # the call below passes fake pointers: make sure the size check rejects it before any
+    # launch, i.e. that this shape really needs more than the library's 4 MiB of scratch
+    need = ctypes.c_size_t()
+    assert oal.lib().oal_decode_workspace_bytes(ctypes.byref(big), ctypes.byref(need)) == 0
+    assert need.value > (4 << 20)
     P = ctypes.c_void_p(256)
     assert noalloc(P, P, P, P, P, ctypes.byref(big), None) == -3
