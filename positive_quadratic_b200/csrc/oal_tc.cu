@@ -65,25 +65,28 @@ constexpr uint32_t kRdOffQ = 32768;       // Q tile (bf16, K-major): phi and Aq 
 constexpr uint32_t kRdOffAq = 49152;      // Aq0 | Aq1 (score A operands); the P tile aliases
 constexpr uint32_t kRdOffA = 81920;       // 4 x 16 KB phi stages (readout A operand, K-major)
 constexpr uint32_t kRdOffB = 147456;      // 2 x 20 KB state-image stages of 2 slices (B operand)
-constexpr uint32_t kRdOffOnes = 188416;   // 16 KB ones atom
-constexpr uint32_t kRdOffCoef = 204800;   // 2176 fp32 coefficients
-constexpr uint32_t kRdOffCoefH = 213504;  // 1792 bf16 coefficients of the off-diagonal rows
-constexpr uint32_t kRdOffW = 217088;      // 9 x 64 fp32
-constexpr uint32_t kRdOffC0 = 219392;     // 9 fp32
+constexpr uint32_t kRdOffCoef = 188416;   // 2176 fp32 coefficients
+constexpr uint32_t kRdOffCoefH = 197120;  // 1792 bf16 coefficients of the off-diagonal rows
+constexpr uint32_t kRdOffW = 200704;      // 9 x 64 fp32
+constexpr uint32_t kRdOffC0 = 203008;     // 9 fp32
+constexpr uint32_t kRdOffOnes = 203776;   // 16 KB ones atom; then image stage 2 (20 KB) reuses it
 // chunk-delta builder
 constexpr uint32_t kStOffKV = 0;          // 3 x (K 16 KB + V 16 KB)
 constexpr uint32_t kStOffA = 98304;       // 2 x (hi 16 KB + lo 16 KB) psi stages
 constexpr uint32_t kOffOnes = 163840;     // 16 KB ones atom
 // both
-constexpr uint32_t kOffCtl = 219648;      // barriers and control words
+constexpr uint32_t kOffCtl = 224256;      // barriers and control words
 constexpr uint32_t kSmemBytes = kOffCtl + 1024 + 1024;
 
 constexpr int kPhiSets = 4;                                // reader warps (w >> 2) per slice
-// phi stages (SMEM, 1 slice): one per warp set, so that every wait on a stage barrier is for
-// the phase right after the one the waiter last saw complete (parity waits cannot tell
-// phases two apart)
-constexpr int kRdStages = kPhiSets;
-constexpr int kBStages = 2;                                // image stages (SMEM, 2 slices)
+// phi stages (SMEM, 1 slice): two per warp set (stages kq and kq + 4), so that every wait on
+// a stage barrier is for the phase right after the one the waiter last saw complete (parity
+// waits cannot tell phases two apart).  Stages 0..3 have their own region; stages 4..7 reuse
+// the K, V and Aq | P tiles once the intra-chunk MMAs that read them have completed.
+constexpr int kRdStages = 2 * kPhiSets;
+// image stages (SMEM, 2 slices each): stages 0, 1 have their own region, stage 2 reuses the
+// ones atom once the intra-chunk P [V | 1] MMAs have completed
+constexpr int kBStages = 3;
 constexpr uint32_t kImgPairBytes = 2 * kImgSliceBytes;     // one tensor copy: 160 rows
 constexpr uint32_t kPhiTileBytes = kC * 64 * 2;            // 128 rows x 64 packed rows, bf16
 constexpr int kKVStages = 3;
@@ -91,13 +94,26 @@ constexpr uint32_t kStATile = 64 * kSlabRows * 2;          // 64 tokens x 128 ro
 // reader TMEM map: U in [0, 80); score tiles S0 | S1 in [128, 384).  phi stays in shared
 // memory: warp stores into tensor memory stall concurrent MMAs, shared-memory stores do not.
 constexpr uint32_t kColU = 0, kColS0 = 128;
-static_assert(kRdOffA + kRdStages * kPhiTileBytes <= kRdOffB &&
-                  kRdOffB + kBStages * kImgPairBytes <= kRdOffOnes &&
-                  kRdOffC0 + 64 <= kOffCtl,
+__host__ __device__ constexpr uint32_t rd_stage_off(int st)
+{
+    return st < kPhiSets ? kRdOffA + uint32_t(st) * kPhiTileBytes
+                         : (st == 4 ? kRdOffK : st == 5 ? kRdOffV : kRdOffAq + (st - 6) * kTileBytes);
+}
+static_assert(kRdOffK + kTileBytes <= kRdOffV && kRdOffV + kTileBytes <= kRdOffQ &&
+                  kRdOffAq + 2 * kTileBytes <= kRdOffA && kTileBytes == kPhiTileBytes,
+              "reused phi stages");
+__host__ __device__ constexpr uint32_t rd_bstage_off(int bs)
+{
+    return bs < 2 ? kRdOffB + uint32_t(bs) * kImgPairBytes : kRdOffOnes;
+}
+static_assert(kRdOffA + kPhiSets * kPhiTileBytes <= kRdOffB &&
+                  kRdOffB + 2 * kImgPairBytes <= kRdOffCoef && kRdOffC0 + 64 <= kRdOffOnes &&
+                  kRdOffOnes % 1024 == 0 && kRdOffOnes + kImgPairBytes <= kOffCtl &&
+                  kOnesAtomBytes <= kImgPairBytes,
               "reader shared-memory map");
 
 struct RdBars {
-    uint64_t qkv_full, aq_full[2], s_full[2], s_empty[2], p_full;
+    uint64_t qkv_full, aq_full[2], s_full[2], s_empty[2], p_full, pv_done;
     uint64_t a_full[kRdStages], a_empty[kRdStages], b_full[kBStages], b_empty[kBStages];
     uint64_t u_full, done;
 };
@@ -599,6 +615,7 @@ __device__ void reader_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Pa
             mbar_init(&bar.s_empty[i], 16);
         }
         mbar_init(&bar.p_full, 16);
+        mbar_init(&bar.pv_done, 1);
         for (int i = 0; i < kRdStages; ++i) {
             mbar_init(&bar.a_full[i], 4);
             mbar_init(&bar.a_empty[i], 1);
@@ -655,8 +672,10 @@ __device__ void reader_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Pa
                     if (u >= kBStages &&
                         !mbar_wait(&bar.b_empty[bs], ((u / kBStages) - 1) & 1, abort_flag))
                         break;
+                    // stage 2 is the ones atom until the P [V | 1] MMAs are done
+                    if (u == 2 && !mbar_wait(&bar.pv_done, 0, abort_flag)) break;
                     mbar_expect_tx(&bar.b_full[bs], kImgPairBytes);
-                    tma_load_2d(sm + kRdOffB + bs * kImgPairBytes, P.tm_img, &bar.b_full[bs], 0,
+                    tma_load_2d(sm + rd_bstage_off(bs), P.tm_img, &bar.b_full[bs], 0,
                                 row0 + 160 * u);
                     ++issued;
                 }
@@ -673,7 +692,7 @@ __device__ void reader_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Pa
         constexpr uint32_t id_pv = idesc_bf16(128, 80, false, true);   // B = [V | ones] MN
         const uint32_t aq0 = smem_u32(sm + kRdOffAq), kt = smem_u32(sm + kRdOffK);
         const uint32_t vt = smem_u32(sm + kRdOffV), ones = smem_u32(sm + kRdOffOnes);
-        const uint32_t a0 = smem_u32(sm + kRdOffA), b0 = smem_u32(sm + kRdOffB);
+        const uint32_t sm0 = smem_u32(sm);
         bool ok = mbar_wait(&bar.qkv_full, 0, abort_flag);
         // grouped score tiles S_m = (Q o w_m) K^T, double-buffered in TMEM
         for (int m = 0; m <= G && ok; ++m) {
@@ -703,11 +722,12 @@ __device__ void reader_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Pa
                              sdesc_sw128(aq0 + (ks >> 2) * kTileBytes + (ks & 3) * 32, 16, 1024),
                              sdesc_sw128(vt + ks * 2048, ones - vt, 1024), id_pv,
                              ks > 0 ? 1u : 0u);
+                mma_commit(&bar.pv_done);  // K, V, Aq | P are free for phi stages 4..7
             }
             __syncwarp();
         }
         // inter-chunk readout U += phi(Q_c) S_c, two slices (one image stage) per round:
-        // A = phi slices 2u, 2u + 1 (stages of sets 2u % 4, (2u + 1) % 4), B = image pair u
+        // A = phi slices 2u, 2u + 1 (stages (2u) % 8, (2u + 1) % 8), B = image pair u
         for (int u = 0; u < kSlices / 2 && ok && has_inter; ++u) {
             const int s0 = 2 * u, bs = u % kBStages;
             ok = mbar_wait(&bar.a_full[s0 % kRdStages], (s0 / kRdStages) & 1, abort_flag) &&
@@ -720,11 +740,11 @@ __device__ void reader_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Pa
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
                     const int st = (s0 + x) % kRdStages;
-                    const uint32_t bsl = b0 + bs * kImgPairBytes + x * kImgSliceBytes;
+                    const uint32_t bsl = sm0 + rd_bstage_off(bs) + x * kImgSliceBytes;
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
                         mma_bf16(tmem + kColU,
-                                 sdesc_sw128(a0 + st * kPhiTileBytes + ks * 32, 16, 1024),
+                                 sdesc_sw128(sm0 + rd_stage_off(st) + ks * 32, 16, 1024),
                                  sdesc_sw128(bsl + ks * 32, 16, 1024), id_u, 1u);
                     mma_commit(&bar.a_empty[st]);
                 }
@@ -767,8 +787,9 @@ __device__ void reader_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Pa
             fence_proxy_async();
             warp_arrive(&bar.aq_full[m & 1]);
         };
-        // phi slice s of this row -> shared stage s % 4 = kq (K-major, 128B-swizzled rows)
-        const uint32_t a0 = smem_u32(sm + kRdOffA);
+        // phi slice s of this row -> shared stage s % 8 (kq or kq + 4; K-major, 128B-swizzled
+        // rows)
+        const uint32_t sm0 = smem_u32(sm);
         auto produce_phi = [&](int s) -> bool {
             const int st = s % kRdStages;
             uint32_t w[32];
@@ -777,7 +798,10 @@ __device__ void reader_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Pa
             if (s >= kRdStages &&
                 !mbar_wait(&bar.a_empty[st], ((s / kRdStages) - 1) & 1, abort_flag))
                 return false;
-            const uint32_t base = a0 + st * kPhiTileBytes;
+            // first use of a reused stage: the intra-chunk MMAs must be done with it
+            if (s >= kPhiSets && s < kRdStages && !mbar_wait(&bar.pv_done, 0, abort_flag))
+                return false;
+            const uint32_t base = sm0 + rd_stage_off(st);
 #pragma unroll
             for (int x = 0; x < 8; ++x)
                 sts128(base + kmajor_chunk(row, x), w[4 * x], w[4 * x + 1], w[4 * x + 2],
