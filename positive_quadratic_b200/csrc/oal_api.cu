@@ -128,8 +128,12 @@ int oal_prefill(const void* q, const void* k, const void* v, const int32_t* grou
     if (!workspace || workspace_bytes < need) return OAL_ERR_WORKSPACE;
     if (!aligned16(workspace)) return OAL_ERR_ALIGN;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    rc = launch_prep(group_id, L, G, eps, state, s->B, s->Hq, s->Hkv, s->T, st);
-    if (rc) return rc;
+    // the tensor-core path builds the coefficient tables inside its scan kernel
+    const bool tc = use_tensor_path(s) && s->B > 0 && s->T > 0;
+    if (!tc) {
+        rc = launch_prep(group_id, L, G, eps, state, s->B, s->Hq, s->Hkv, s->T, st);
+        if (rc) return rc;
+    }
     if (s->B == 0) return OAL_OK;
     if (use_tensor_path(s))
         return launch_prefill_tc(q, k, v, group_id, L, G, eps, out, state, workspace, s->B, s->T,

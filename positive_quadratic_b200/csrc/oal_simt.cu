@@ -19,13 +19,15 @@ namespace oal {
 // block 0 also writes the state header.  Group ids and G are validated; out-of-range values
 // raise OAL_ERR_GROUPS and are clamped so that nothing reads outside M.
 // ------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) prep_kernel(const int32_t* __restrict__ gid,
-                                                   const float* __restrict__ L,
-                                                   const int32_t* __restrict__ G, float eps,
-                                                   unsigned char* __restrict__ state, int B,
-                                                   int Hq, int Hkv, long long tokens)
+// One block of 256 threads per query head h: M = L L^T in fp64, the packed coefficient table
+// of that head, and (head 0) the state header.
+__device__ __forceinline__ void prep_head(int h, const int32_t* __restrict__ gid,
+                                          const float* __restrict__ L,
+                                          const int32_t* __restrict__ G, float eps,
+                                          unsigned char* __restrict__ state, int B, int Hq,
+                                          int Hkv, long long tokens)
 {
-    const int h = blockIdx.x, tid = threadIdx.x;
+    const int tid = threadIdx.x;
     __shared__ double M[kGM1][kGM1];
     __shared__ int g[kDA];
     __shared__ int sG;
@@ -83,6 +85,15 @@ __global__ void __launch_bounds__(256) prep_kernel(const int32_t* __restrict__ g
         hd->tokens = tokens;
         hd->eps = eps;
     }
+}
+
+__global__ void __launch_bounds__(256) prep_kernel(const int32_t* __restrict__ gid,
+                                                   const float* __restrict__ L,
+                                                   const int32_t* __restrict__ G, float eps,
+                                                   unsigned char* __restrict__ state, int B,
+                                                   int Hq, int Hkv, long long tokens)
+{
+    prep_head(blockIdx.x, gid, L, G, eps, state, B, Hq, Hkv, tokens);
 }
 
 // ------------------------------------------------------------------------------------------

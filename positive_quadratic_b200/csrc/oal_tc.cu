@@ -72,8 +72,8 @@ constexpr uint32_t kRdOffC0 = 203008;     // 9 fp32
 constexpr uint32_t kRdOffOnes = 203776;   // 16 KB ones atom; then image stage 2 (20 KB) reuses it
 // chunk-delta builder
 constexpr uint32_t kStOffKV = 0;          // 3 x (K 16 KB + V 16 KB)
-constexpr uint32_t kStOffA = 98304;       // 2 x (hi 16 KB + lo 16 KB) psi stages
-constexpr uint32_t kOffOnes = 163840;     // 16 KB ones atom
+constexpr uint32_t kStOffA = 98304;       // 3 x (hi 16 KB + lo 16 KB) psi stages
+constexpr uint32_t kOffOnes = 196608;     // 16 KB ones atom
 // both
 constexpr uint32_t kOffCtl = 224256;      // barriers and control words
 constexpr uint32_t kSmemBytes = kOffCtl + 1024 + 1024;
@@ -90,10 +90,16 @@ constexpr int kBStages = 3;
 constexpr uint32_t kImgPairBytes = 2 * kImgSliceBytes;     // one tensor copy: 160 rows
 constexpr uint32_t kPhiTileBytes = kC * 64 * 2;            // 128 rows x 64 packed rows, bf16
 constexpr int kKVStages = 3;
+constexpr int kDAStages = 3;  // psi stages (hi + lo tiles of one half chunk)
+constexpr int kDAcc = 4;      // TMEM accumulators of the delta builder (128 columns each)
 constexpr uint32_t kStATile = 64 * kSlabRows * 2;          // 64 tokens x 128 rows = 16 KB
 // reader TMEM map: U in [0, 80); score tiles S0 | S1 in [128, 384).  phi stays in shared
 // memory: warp stores into tensor memory stall concurrent MMAs, shared-memory stores do not.
 constexpr uint32_t kColU = 0, kColS0 = 128;
+static_assert(kStOffKV + kKVStages * 2 * kTileBytes <= kStOffA &&
+                  kStOffA + kDAStages * 2 * kStATile <= kOffOnes &&
+                  kOffOnes + kOnesAtomBytes <= kOffCtl && kDAcc * 128 <= int(kTmemCols),
+              "delta builder shared-memory and TMEM map");
 __host__ __device__ constexpr uint32_t rd_stage_off(int st)
 {
     return st < kPhiSets ? kRdOffA + uint32_t(st) * kPhiTileBytes
@@ -118,8 +124,8 @@ struct RdBars {
     uint64_t u_full, done;
 };
 struct StBars {
-    uint64_t kv_full[kKVStages], kv_empty[kKVStages], a_full[2], a_empty[2];
-    uint64_t acc_full[2], acc_empty[2], done;
+    uint64_t kv_full[kKVStages], kv_empty[kKVStages], a_full[kDAStages], a_empty[kDAStages];
+    uint64_t acc_full[kDAcc], acc_empty[kDAcc], done;
 };
 struct Ctl {
     union {
@@ -370,9 +376,11 @@ __device__ void delta_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Par
             mbar_init(&bar.kv_full[i], 1);
             mbar_init(&bar.kv_empty[i], 8 + 1);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kDAStages; ++i) {
             mbar_init(&bar.a_full[i], 8);
             mbar_init(&bar.a_empty[i], 1);
+        }
+        for (int i = 0; i < kDAcc; ++i) {
             mbar_init(&bar.acc_full[i], 1);
             mbar_init(&bar.acc_empty[i], 8);
         }
@@ -410,16 +418,17 @@ __device__ void delta_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Par
         const uint32_t ones = smem_u32(sm + kOffOnes);
         bool ok = true;
         for (int i = 0; i < nu && ok; ++i) {
-            const int s = i & 1, st = i % kKVStages;
-            if (i >= 2) ok = mbar_wait(&bar.acc_empty[s], ((i >> 1) - 1) & 1, abort_flag);
+            const int s = i % kDAcc, st = i % kKVStages;
+            if (i >= kDAcc) ok = mbar_wait(&bar.acc_empty[s], ((i / kDAcc) - 1) & 1, abort_flag);
             if (ok) ok = mbar_wait(&bar.kv_full[st], (i / kKVStages) & 1, abort_flag);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             const uint32_t d = tmem + s * 128;
             const uint32_t vt = kv0 + st * 2 * kTileBytes + kTileBytes;
             const uint32_t lbo = ones - vt;  // V atom -> ones atom (N elements 64..)
             for (int hc = 0; hc < 2; ++hc) {
-                const int w = 2 * i + hc, as = w & 1;
-                ok = __all_sync(0xffffffffu, mbar_wait(&bar.a_full[as], (w >> 1) & 1, abort_flag));
+                const int w = 2 * i + hc, as = w % kDAStages;
+                ok = __all_sync(0xffffffffu,
+                                mbar_wait(&bar.a_full[as], (w / kDAStages) & 1, abort_flag));
                 if (!ok) break;
                 tc_fence_after();
                 if (elect_one()) {
@@ -456,8 +465,9 @@ __device__ void delta_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Par
             const unsigned char* kt = sm + kStOffKV + st * 2 * kTileBytes;
             bool ok = true;
             for (int hc = 0; hc < 2; ++hc) {
-                const int w = 2 * i + hc, as = w & 1;
-                if (w >= 2 && !mbar_wait(&bar.a_empty[as], ((w >> 1) - 1) & 1, abort_flag)) {
+                const int w = 2 * i + hc, as = w % kDAStages;
+                if (w >= kDAStages &&
+                    !mbar_wait(&bar.a_empty[as], ((w / kDAStages) - 1) & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
@@ -476,9 +486,9 @@ __device__ void delta_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Par
         const int fl = q4 * 32 + lane;
         for (int i = 0; i < nu; ++i) {
             const DeltaUnit du = delta_unit(u0 + i, NC);
-            const int s = i & 1;
+            const int s = i % kDAcc;
             // all epilogue threads leave together, so no named barrier is left half-joined
-            const bool got = mbar_wait(&bar.acc_full[s], (i >> 1) & 1, abort_flag);
+            const bool got = mbar_wait(&bar.acc_full[s], (i / kDAcc) & 1, abort_flag);
             if (!named_bar_and(2, 256, got)) break;
             tc_fence_after();
             const uint32_t lanebase = tmem + (uint32_t(q4 * 32) << 16) + s * 128;
@@ -957,13 +967,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 // bf16(sum_{c' < c} dS_c') for c >= 1, stored row-major as [80 n][64 f] per slice (the
 // readout's tensor copy swizzles it into the K-major B-operand layout; rows 65.. are never
 // read), final state = sum over all chunks.  Thread = (n, row pair).
+// The last z-plane of the grid instead builds the coefficient tables and the state header
+// (one block per query head), which the readout reads after this kernel.
 constexpr int kScanCols = 8;
 constexpr int kImgRows = 80;
 __global__ void __launch_bounds__(256) scan_kernel(const float* __restrict__ dS,
                                                    unsigned char* __restrict__ img,
-                                                   float* __restrict__ body, int NC)
+                                                   float* __restrict__ body, int NC,
+                                                   const int32_t* __restrict__ gid,
+                                                   const float* __restrict__ L,
+                                                   const int32_t* __restrict__ G, float eps,
+                                                   unsigned char* __restrict__ state, int B,
+                                                   int Hq, int Hkv, long long tokens)
 {
     grid_dep_launch();
+    if (blockIdx.z == gridDim.z - 1) {  // independent of the deltas: no wait
+        const int h = blockIdx.y * gridDim.x + blockIdx.x;
+        if (h < Hq) prep_head(h, gid, L, G, eps, state, B, Hq, Hkv, tokens);
+        return;
+    }
     grid_dep_wait();
     const int sl = blockIdx.x, bkv = blockIdx.z;
     const int nl = threadIdx.x >> 5, p = threadIdx.x & 31;
@@ -1167,8 +1189,9 @@ int launch_prefill_tc(const void* q, const void* k, const void* v, const int32_t
     {
         LaunchScope ls("scan", st);
         OAL_CUDA_TRY(launch_ex(tc::scan_kernel,
-                               dim3(tc::kSlices, tc::kImgRows / tc::kScanCols, B * Hkv),
-                               dim3(256), 0, st, overlap, (const float*)P.dS, P.img, body, NC));
+                               dim3(tc::kSlices, tc::kImgRows / tc::kScanCols, B * Hkv + 1),
+                               dim3(256), 0, st, overlap, (const float*)P.dS, P.img, body, NC,
+                               gid, L, G, eps, sb, B, Hq, Hkv, (long long)T));
     }
     {
         LaunchScope ls("readout_tc", st);
