@@ -158,6 +158,19 @@ int oal_dense_ref_gpu(const void* q, const void* k, const void* v, const int32_t
                       const float* L, const int32_t* G, float eps, float* out,
                       const oal_shape* s, void* stream);
 
+/* Contribution statistic of eq. (1) (same page, section 核心公式), per prompt p = (b, query
+ * head h) and dimension r:
+ *   chi[b][h][r] = (1/|Omega|) sum over causal pairs j <= i of |q_{b,h,i,r} k_{b,kv,j,r}| / sqrt(d_h)
+ * with kv = floor(h * Hkv / Hq) and |Omega| = T (T + 1) / 2, the number of causal pairs of the
+ * prompt (the page does not define Omega; this is the reading).  The page's chi_r is the mean
+ * of chi[b][h][r] over the prompts b of a head.  q [B][Hq][T][64], k [B][Hkv][T][64] in the
+ * dtype of `s`; chi [B][Hq][64] fp32; caller-owned device memory, 16-byte aligned.  Uses B, T,
+ * Hq, Hkv, dh and dtype of `s` (chunk is ignored).  Accumulates in fp64 (an O(T d) prefix scan
+ * of |k| per head).  B*T == 0 writes nothing and allows NULL pointers.  Errors: as
+ * oal_prefill (shape, NULL, alignment). */
+int oal_contribution_stat(const void* q, const void* k, float* chi, const oal_shape* s,
+                          void* stream);
+
 /* Launch mode of the tensor-core prefill (bf16, chunk 128), which runs as three kernels:
  * chunk deltas, the prefix scan over chunks, and the readout.  1 (default): the scan and the
  * readout are launched as programmatic dependents, so each is scheduled while its predecessor

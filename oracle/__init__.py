@@ -59,8 +59,9 @@ def _load():
                                                                        ctypes.c_double,
                                                                        ctypes.c_int, _I, _I, _I,
                                                                        _D]
+            lib.oal_oracle_chi.argtypes = [ctypes.c_int] * 5 + [_D, _D, _D]
             for f in (lib.oal_oracle_kappa, lib.oal_oracle_dense, lib.oal_oracle_recurrent,
-                      lib.oal_oracle_dense_rows):
+                      lib.oal_oracle_dense_rows, lib.oal_oracle_chi):
                 f.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -165,6 +166,19 @@ def recurrent(q, k, v, group_id, L, G, eps, state: State | None = None,
                                       *[_d(a) for a in outs], _d(y))
     _check(rc, "recurrent")
     return (y, out) if return_state else y
+
+
+def chi(q, k):
+    """Contribution statistic of eq. (1) per prompt (b, query head): [B, Hq, dh].  The
+    statistic chi_r of the page is chi(q, k).mean(axis=0) for the prompts of a head."""
+    q, k = _f64(q), _f64(k)
+    if q.ndim != 4 or k.ndim != 4 or k.shape[0] != q.shape[0] or k.shape[2:] != q.shape[2:]:
+        raise ValueError("q [B, Hq, T, dh] and k [B, Hkv, T, dh] expected")
+    B, Hq, T, dh = q.shape
+    out = np.zeros((B, Hq, dh), dtype=np.float64)
+    _check(_load().oal_oracle_chi(B, Hq, k.shape[1], T, dh, _d(q), _d(k), _d(out)),
+           "oal_oracle_chi")
+    return out
 
 
 def threads() -> int:

@@ -262,3 +262,33 @@ int oal_oracle_dense_rows(int B, int Hq, int Hkv, int T, int dh, int dv, const d
     }
     return status;
 }
+
+/*
+ * Contribution statistic, eq. (1) of the same section:
+ *   chi_{p,r} = (1/|Omega_p|) sum over causal pairs (i, j), j <= i, of |q_{p,i,r} k_{p,j,r}| / sqrt(d_h)
+ * for prompt p = (b, query head h); |Omega_p| = T (T + 1) / 2, the number of causal pairs
+ * (the page does not define Omega; this is the reading).  chi_r of eq. (1) is the mean of
+ * chi_{p,r} over prompts.  Plain double loop over every causal pair, O(T^2 dh) per head.
+ * Layouts: q [B][Hq][T][dh], k [B][Hkv][T][dh], chi [B][Hq][dh].
+ */
+int oal_oracle_chi(int B, int Hq, int Hkv, int T, int dh, const double* q, const double* k,
+                   double* chi)
+{
+    if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv || T < 1 || dh < 1) return -1;
+    const int group = Hq / Hkv;
+    const double pairs = 0.5 * (double)T * (double)(T + 1), rs = 1.0 / sqrt((double)dh);
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < Hq; ++h) {
+            const double* qh = q + ((size_t)b * Hq + h) * T * dh;
+            const double* kh = k + ((size_t)b * Hkv + h / group) * T * dh;
+            for (int r = 0; r < dh; ++r) {
+                double acc = 0.0;
+                for (int i = 0; i < T; ++i)
+                    for (int j = 0; j <= i; ++j)
+                        acc += fabs(qh[(size_t)i * dh + r] * kh[(size_t)j * dh + r] * rs);
+                chi[((size_t)b * Hq + h) * dh + r] = acc / pairs;
+            }
+        }
+    return 0;
+}

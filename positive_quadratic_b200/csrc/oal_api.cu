@@ -178,6 +178,18 @@ int oal_dense_ref_gpu(const void* q, const void* k, const void* v, const int32_t
                         static_cast<cudaStream_t>(stream));
 }
 
+int oal_contribution_stat(const void* q, const void* k, float* chi, const oal_shape* s,
+                          void* stream)
+{
+    int rc = check_common(s);
+    if (rc) return rc;
+    if ((long long)s->B * s->T == 0) return OAL_OK;
+    if (!q || !k || !chi) return OAL_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(chi)) return OAL_ERR_ALIGN;
+    return launch_chi(q, k, chi, s->B, s->T, s->Hq, s->Hkv, s->dtype,
+                      static_cast<cudaStream_t>(stream));
+}
+
 unsigned long long oal_launch_count(void) { return tracer().launches.load(); }
 
 int oal_set_prefill_overlap(int overlap) { return g_prefill_overlap.exchange(overlap ? 1 : 0); }

@@ -5,3 +5,4 @@
 #include "oal_tc.cu"
 #include "oal_api.cu"
 #include "oal_noalloc.cu"
+#include "oal_chi.cu"

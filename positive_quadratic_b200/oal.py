@@ -70,6 +70,7 @@ def lib() -> ctypes.CDLL:
             L.oal_prefill.argtypes = [_VP] * 6 + [ctypes.c_float, _VP, _VP, _VP, _SZ, _PS, _VP]
             L.oal_decode_step.argtypes = [_VP] * 6 + [_SZ, _PS, _VP]
             L.oal_dense_ref_gpu.argtypes = [_VP] * 6 + [ctypes.c_float, _VP, _PS, _VP]
+            L.oal_contribution_stat.argtypes = [_VP, _VP, _VP, _PS, _VP]
             L.oal_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), _VP]
             L.oal_launch_count.restype = ctypes.c_ulonglong
             L.oal_last_cuda_error.argtypes = [ctypes.c_char_p, ctypes.c_size_t]
@@ -83,7 +84,7 @@ def lib() -> ctypes.CDLL:
             L.oal_profile_read.restype = ctypes.c_int
             for name in ("oal_state_bytes", "oal_prefill_workspace_bytes",
                          "oal_decode_workspace_bytes", "oal_prefill", "oal_decode_step",
-                         "oal_dense_ref_gpu", "oal_device_error"):
+                         "oal_dense_ref_gpu", "oal_device_error", "oal_contribution_stat"):
                 getattr(L, name).restype = ctypes.c_int
             _lib = L
     return _lib
@@ -228,6 +229,22 @@ def dense_ref(q, k, v, group_id, L, G, eps: float, out=None, stream=None):
     rc = lib().oal_dense_ref_gpu(_ptr(q), _ptr(k), _ptr(v), _ptr(group_id), _ptr(L), _ptr(G),
                                  float(eps), _ptr(out), ctypes.byref(shape), _stream(stream))
     _check(rc, "oal_dense_ref_gpu")
+    return out
+
+
+def contribution_stat(q, k, out=None, stream=None):
+    """oal_contribution_stat: eq. (1)'s chi per prompt (b, query head) and dimension, [B, Hq, 64]
+    fp32; the page's chi_r is its mean over b."""
+    if q.dim() != 4 or k.dim() != 4 or k.dtype != q.dtype:
+        raise ValueError("q [B, Hq, T, d] and k [B, Hkv, T, d] of one dtype expected")
+    B, Hq, T, d = q.shape
+    shape = make_shape(B, T, Hq, k.shape[1], 128, _dtype_code(q), d)
+    if out is None:
+        out = torch.empty(B, Hq, d, dtype=torch.float32, device=q.device)
+    _contig_cuda(q, k, out)
+    rc = lib().oal_contribution_stat(_ptr(q), _ptr(k), _ptr(out), ctypes.byref(shape),
+                                     _stream(stream))
+    _check(rc, "oal_contribution_stat")
     return out
 
 

@@ -285,3 +285,30 @@ def test_tensor_schedules_agree(oal, cuda):
     finally:
         oal.set_prefill_overlap(prev)
     np.testing.assert_array_equal(y1, y2)
+
+
+# --- contribution statistic, eq. (1) -----------------------------------------------------------
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("T", [1, 7, 300, 1000])
+def test_contribution_stat(oal, cuda, T, dtype):
+    p = I.small_layer(900 + T, B=2, T=T, Hq=4, Hkv=2, dtype=dtype)
+    ref = oracle.chi(p.q, p.k)
+    q, k, *_ = dev_inputs(p, cuda)
+    chi = oal.contribution_stat(q, k).cpu().numpy()
+    assert oal.device_error() == 0
+    np.testing.assert_allclose(chi, ref, rtol=1e-5, atol=0)
+
+
+@pytest.mark.gpu
+def test_contribution_stat_config1(oal, cuda):
+    """Config-1 layer shape (14/2 heads, outliers), first 2048 tokens; the page's chi_r is
+    the mean over prompts, here the single prompt of each head."""
+    p = I.config1().slice_tokens(0, 2048)
+    ref = oracle.chi(p.q, p.k)
+    q, k, *_ = dev_inputs(p, cuda)
+    chi = oal.contribution_stat(q, k).cpu().numpy()
+    np.testing.assert_allclose(chi, ref, rtol=1e-5, atol=0)
+    # the outlier dimensions dominate the statistic, as the grouping assumes
+    assert np.all(chi.max(axis=-1) > 4 * np.median(chi, axis=-1))

@@ -313,3 +313,64 @@ def test_dense_rows_match_dense():
     yr = oracle.dense_rows(p.q, p.k, p.v, p.group_id, p.L, p.G, p.eps, rows)
     for n, (b, h, i) in enumerate(rows):
         np.testing.assert_array_equal(yr[n], y[b, h, i])
+
+
+# --- contribution statistic, eq. (1) ------------------------------------------------------------
+
+def test_chi_constant_inputs_closed_form():
+    """q = a and k = c everywhere: every causal pair contributes |a c| / sqrt(d), and the
+    pair count cancels |Omega| = T (T + 1) / 2, so chi = |a c| / 8 for d = 64."""
+    T, d = 37, 64
+    q = np.full((1, 1, T, d), -1.5)
+    k = np.full((1, 1, T, d), 0.75)
+    np.testing.assert_allclose(oracle.chi(q, k), abs(-1.5 * 0.75) / 8.0, rtol=1e-13)
+
+
+def test_chi_linear_keys_closed_form():
+    """q = 1, k_j = j + 1: sum_i sum_{j<=i} (j + 1) = T (T + 1)(T + 2) / 6, so chi =
+    (T + 2) / (3 sqrt(d)) after dividing by T (T + 1) / 2.  Summing over every j instead of
+    j <= i, or dividing by T^2, gives a different value."""
+    T, d = 50, 64
+    q = np.ones((1, 1, T, d))
+    k = np.broadcast_to((np.arange(T) + 1.0)[None, None, :, None], (1, 1, T, d)).copy()
+    np.testing.assert_allclose(oracle.chi(q, k), (T + 2) / (3.0 * 8.0), rtol=1e-12)
+
+
+def test_chi_is_causal_not_full():
+    """Only the last query sees the last key: a key spike at j = T - 1 contributes once."""
+    T, d = 16, 64
+    q = np.ones((1, 1, T, d))
+    k = np.zeros((1, 1, T, d))
+    k[0, 0, T - 1, 5] = 8.0
+    chi = oracle.chi(q, k)
+    pairs = T * (T + 1) / 2
+    assert chi[0, 0, 5] == pytest.approx(8.0 / 8.0 / pairs, rel=1e-13)
+    assert np.count_nonzero(chi) == 1
+
+
+def test_chi_invariances_and_gqa():
+    """Sign flips of q or k leave chi unchanged, scales multiply it, a permutation of the
+    dimensions permutes it, and query head h reads key head floor(h * Hkv / Hq)."""
+    rng = np.random.default_rng(11)
+    B, Hq, Hkv, T, d = 2, 4, 2, 23, 64
+    q = rng.standard_normal((B, Hq, T, d))
+    k = rng.standard_normal((B, Hkv, T, d))
+    base = oracle.chi(q, k)
+    np.testing.assert_allclose(oracle.chi(-q, k), base, rtol=1e-13)
+    np.testing.assert_allclose(oracle.chi(q, -2.0 * k), 2.0 * base, rtol=1e-13)
+    perm = rng.permutation(d)
+    np.testing.assert_allclose(oracle.chi(q[..., perm], k[..., perm]), base[..., perm],
+                               rtol=1e-13)
+    # GQA: heads 0, 1 read k head 0, heads 2, 3 read k head 1
+    k2 = np.concatenate([k[:, :1], k[:, :1], k[:, 1:], k[:, 1:]], axis=1)
+    np.testing.assert_allclose(oracle.chi(q, k2), base, rtol=1e-13)
+
+
+def test_chi_equals_prefix_sum_form():
+    """sum_i |q_i| (sum_{j<=i} |k_j|): a different evaluation route (cumulative sums)."""
+    rng = np.random.default_rng(12)
+    T, d = 40, 64
+    q = rng.standard_normal((1, 1, T, d))
+    k = rng.standard_normal((1, 1, T, d))
+    ref = (np.abs(q[0, 0]) * np.cumsum(np.abs(k[0, 0]), axis=0)).sum(0) / 8.0 / (T * (T + 1) / 2)
+    np.testing.assert_allclose(oracle.chi(q, k)[0, 0], ref, rtol=1e-12)
