@@ -135,7 +135,6 @@ struct Ctl {
     } bar;
     uint32_t tmem_base;
     int abort_flag;
-    int item;
     int G;
 };
 static_assert(sizeof(Ctl) <= 1024, "control block");
@@ -188,29 +187,9 @@ __device__ __forceinline__ void bounded_spin_done(uint64_t* bar, uint32_t parity
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
 __device__ __forceinline__ uint32_t pack2(float2 v) { return pack_bf16x2(v.x, v.y); }
 
-__device__ __forceinline__ void fence_proxy_async_global()
-{
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-}
 
-__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int* p)
-{
-    unsigned int v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
 
-__device__ __forceinline__ void red_release_gpu_add(unsigned int* p, unsigned int v)
-{
-    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
 
-__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d)
-{
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b),
-                 "f"(c), "f"(d)
-                 : "memory");
-}
 
 // MN-major SW128 atom whose N-element 0 is 1 for every K row (the [.; 1] column of [V; 1])
 __device__ __forceinline__ void init_ones_atom(unsigned char* atom)
