@@ -140,8 +140,8 @@ int oal_decode_step(const void* q, const void* k, const void* v, void* state, fl
  * cannot afford cudaMalloc's implicit device-wide synchronisation.
  * Same arguments and results as oal_decode_step, minus the workspace.  The scratch is a
  * fixed 4 MiB array inside the library (one copy on every GPU that loads the library, held
- * until the process exits).  A step needs align256(4*B*Hkv) + 1820*B*Hq bytes of it, so
- * B*Hq must stay at or below 2299 (batch 64 x 14 heads fits); larger problems return
+ * until the process exits).  A step needs align256(4*B*Hkv) + 2340*B*Hq bytes of it, so
+ * B*Hq must stay at or below 1788 (batch 64 x 14 heads fits); larger problems return
  * OAL_ERR_UNSUPPORTED without launching anything.
  * The first call on each device looks up the array's device address (cudaGetSymbolAddress);
  * make that first call before any stream capture.  Every call shares the one array and

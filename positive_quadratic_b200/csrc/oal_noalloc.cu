@@ -12,9 +12,9 @@
 
 namespace oal {
 
-// 4 MiB: room for the per-(b, kv) tickets and per-slab partial readouts (7 slabs x 65 fp32
-// per query head) of a decode step with B*Hq up to 2299 query heads (batch 64 x 14 heads
-// needs 1.6 MB).
+// 4 MiB: room for the per-(b, kv) tickets and per-slab partial readouts (9 slabs x 65 fp32
+// per query head) of a decode step with B*Hq up to 1788 query heads (batch 64 x 14 heads
+// needs 2.1 MB).
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];

@@ -349,21 +349,23 @@ __global__ void __launch_bounds__(256) readout_simt_kernel(
 }
 
 // ------------------------------------------------------------------------------------------
-// a11: decode step.  Block (slab, bkv) streams 320 packed rows of one (b, kv) state once:
+// a11: decode step.  Block (slab, bkv) streams 240 packed rows of one (b, kv) state once:
 // S_f += psi_f(k) [v; 1] (eq. (4) with one new token), then accumulates
 // u_h += phi_{h,f}(q_h) S_f for the Hq/Hkv query heads of that kv head (eq. (5)).  Row data
 // moves as 128-bit loads and stores (a half warp per 256-byte row).  Per-block partial u go
 // to the workspace; the last block of a (b, kv) (atomic ticket) sums them, writes yhat and
 // re-arms the ticket.
 // ------------------------------------------------------------------------------------------
-// 7 slabs of 320 packed rows per (b, kv) head: 256 threads with at most 80 registers, so
-// three blocks share an SM and a batch-64 step (896 blocks) runs in two full waves.
-constexpr int kDecRows = 320;
+// 9 slabs of 240 packed rows per (b, kv) head: 256 threads with at most 64 registers, so four
+// blocks share an SM (592 resident) and a batch-64 step (1152 blocks) takes 1.95 waves -- the
+// block count is chosen against the resident slots, since a last wave of a few blocks costs a
+// whole block time.
+constexpr int kDecRows = 240;
 constexpr int kDecThreads = 256;
-constexpr int kDecBatch = 5;  // rows in flight per thread (320 rows = 4 batches of 16 x 5)
+constexpr int kDecBatch = 4;  // rows in flight per thread (240 rows = 16 x (4 + 4 + 4 + 3))
 
 template <typename Tin, int kGrp>  // kGrp = Hq / Hkv query heads per kv head
-__global__ void __launch_bounds__(kDecThreads, 3) decode_kernel(const Tin* __restrict__ q,
+__global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const Tin* __restrict__ q,
                                                               const Tin* __restrict__ k,
                                                               const Tin* __restrict__ v,
                                                               unsigned char* __restrict__ state,
