@@ -889,7 +889,7 @@ __device__ void reader_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Pa
 
 // ------------------------------------------------------------------------------------------
 // kernels: 0 = chunk deltas (persistent: CTA i takes a contiguous range of units),
-// 1 = readers (grid NC x B*Hq).  Both may be launched as programmatic dependents of the
+// 1 = readers (one CTA per (b*h, chunk), B*Hq*NC in all).  Both may be launched as programmatic dependents of the
 // preceding kernel in the stream: griddepcontrol.wait orders every read of its outputs.
 // ------------------------------------------------------------------------------------------
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -931,7 +931,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int u1 = int((long long)units * (blockIdx.x + 1) / gridDim.x);
         if (u1 > u0) delta_item(sm, ctl, tmem, P, u0, u1);
     } else {
-        reader_item(sm, ctl, tmem, P, blockIdx.y, blockIdx.x);
+        // items with an inter-chunk part first, chunk-major with the heads of a chunk adjacent
+        // (they share the chunk's image in L2); the cheap chunk-0 items last, so that the
+        // final partial wave holds short items
+        const int nbh = P.B * P.Hq, heavy = nbh * (P.NC - 1), idx = blockIdx.x;
+        if (idx < heavy) reader_item(sm, ctl, tmem, P, idx % nbh, 1 + idx / nbh);
+        else reader_item(sm, ctl, tmem, P, idx - heavy, 0);
     }
 
     tc_fence_before();
@@ -1174,7 +1179,7 @@ int launch_prefill_tc(const void* q, const void* k, const void* v, const int32_t
     }
     {
         LaunchScope ls("readout_tc", st);
-        OAL_CUDA_TRY(launch_ex(tc::prefill_tc_kernel<1>, dim3(NC, B * Hq), dim3(tc::kThreads),
+        OAL_CUDA_TRY(launch_ex(tc::prefill_tc_kernel<1>, dim3(NC * B * Hq), dim3(tc::kThreads),
                                tc::kSmemBytes, st, overlap, mq, mk, mv, mi, P));
     }
     return OAL_OK;
