@@ -104,7 +104,9 @@ typedef struct {
 int oal_state_bytes(const oal_shape* s, size_t* bytes);
 
 /* Scratch needed by oal_prefill for `s` (all fields used).  The contents need no
- * initialisation and are meaningless after the call. */
+ * initialisation and are meaningless after the call.  On the tensor-core path (bf16, chunk
+ * 128) it holds the bf16 chunk-state images and the fp32 chunk deltas, 913,920 bytes per
+ * (b, kv head, chunk of 128 tokens); on the CUDA-core path the fp32 chunk states. */
 int oal_prefill_workspace_bytes(const oal_shape* s, size_t* bytes);
 
 /* Scratch needed by oal_decode_step for `s` (B, Hq, Hkv used).  It MUST be zero-filled once
@@ -117,8 +119,9 @@ int oal_decode_workspace_bytes(const oal_shape* s, size_t* bytes);
  * coefficients, ready for oal_decode_step.  Chunked evaluation: within each chunk of C tokens
  * the kernel kappa is evaluated densely (eqs. (2)-(3)); across chunks the exclusive prefix
  * state of eq. (4) is built and read out with eq. (5).  Linear in T for fixed d_h.
- * bf16 inputs run on tcgen05 tensor cores (fp32 accumulation); fp32 inputs run in fp32 on
- * CUDA cores.  `workspace` must hold oal_prefill_workspace_bytes(s) bytes. */
+ * bf16 inputs with chunk 128 run on tcgen05 tensor cores (bf16 operands, fp32 accumulation,
+ * exact fp32 final state); fp32 inputs, and bf16 with chunk 64 or 256, run on CUDA cores in
+ * fp32.  `workspace` must hold oal_prefill_workspace_bytes(s) bytes. */
 int oal_prefill(const void* q, const void* k, const void* v, const int32_t* group_id,
                 const float* L, const int32_t* G, float eps, float* out, void* state,
                 void* workspace, size_t workspace_bytes, const oal_shape* s, void* stream);
