@@ -126,6 +126,20 @@ int oal_prefill(const void* q, const void* k, const void* v, const int32_t* grou
                 const float* L, const int32_t* G, float eps, float* out, void* state,
                 void* workspace, size_t workspace_bytes, const oal_shape* s, void* stream);
 
+/* Prefill continuation: appends T tokens to the sequence whose prefix state `state` already
+ * holds (a previous oal_prefill / oal_prefill_continue / oal_decode_step of the same B, Hq,
+ * Hkv and the same group_id, L, G, eps).  out[b][h][t] is yhat of the t-th appended token,
+ * which attends causally to every earlier token of the sequence (eqs. (2)-(5) with the
+ * prefix sums of eq. (4) starting from the state); the state then holds the prefix after the
+ * last appended token and its token count grows by T.  Equivalent to one oal_prefill over
+ * the whole sequence, to the path's tolerance.  Only the tensor-core path (bf16, chunk 128)
+ * continues a prefix; other dtypes or chunk sizes return OAL_ERR_UNSUPPORTED.  T == 0 or
+ * B == 0 leaves the state untouched.  Other arguments and errors as oal_prefill. */
+int oal_prefill_continue(const void* q, const void* k, const void* v, const int32_t* group_id,
+                         const float* L, const int32_t* G, float eps, float* out, void* state,
+                         void* workspace, size_t workspace_bytes, const oal_shape* s,
+                         void* stream);
+
 /* One autoregressive step for every sequence of the batch: q [B][Hq][1][dh],
  * k [B][Hkv][1][dh], v [B][Hkv][1][dv] (dtype of s).  Adds the new token to `state`
  * (eq. (4), rank-one update of every packed row) and writes out [B][Hq][1][dv] = yhat of the

@@ -112,13 +112,17 @@ int oal_decode_workspace_bytes(const oal_shape* s, size_t* bytes)
     return OAL_OK;
 }
 
-int oal_prefill(const void* q, const void* k, const void* v, const int32_t* group_id,
-                const float* L, const int32_t* G, float eps, float* out, void* state,
-                void* workspace, size_t workspace_bytes, const oal_shape* s, void* stream)
+namespace {
+
+int prefill_impl(const void* q, const void* k, const void* v, const int32_t* group_id,
+                 const float* L, const int32_t* G, float eps, float* out, void* state,
+                 void* workspace, size_t workspace_bytes, const oal_shape* s, void* stream,
+                 bool cont)
 {
     int rc = check_common(s);
     if (rc) return rc;
     if ((rc = check_chunk(s))) return rc;
+    if (cont && !use_tensor_path(s)) return OAL_ERR_UNSUPPORTED;
     if (!group_id || !L || !G || !state) return OAL_ERR_NULL;
     if ((rc = check_io(s, q, k, v, out))) return rc;
     if (!aligned16(state) || !aligned16(group_id) || !aligned16(L) || !aligned16(G))
@@ -128,6 +132,7 @@ int oal_prefill(const void* q, const void* k, const void* v, const int32_t* grou
     if (!workspace || workspace_bytes < need) return OAL_ERR_WORKSPACE;
     if (!aligned16(workspace)) return OAL_ERR_ALIGN;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cont && (long long)s->B * s->T == 0) return OAL_OK;  // nothing appended
     // the tensor-core path builds the coefficient tables inside its scan kernel
     const bool tc = use_tensor_path(s) && s->B > 0 && s->T > 0;
     if (!tc) {
@@ -137,10 +142,29 @@ int oal_prefill(const void* q, const void* k, const void* v, const int32_t* grou
     if (s->B == 0) return OAL_OK;
     if (use_tensor_path(s))
         return launch_prefill_tc(q, k, v, group_id, L, G, eps, out, state, workspace, s->B, s->T,
-                                 s->Hq, s->Hkv, g_prefill_overlap.load() != 0, st);
+                                 s->Hq, s->Hkv, g_prefill_overlap.load() != 0, cont, st);
     return launch_prefill_simt(q, k, v, group_id, L, G, eps, out, state,
                                static_cast<float*>(workspace), s->B, s->T, s->Hq, s->Hkv,
                                s->chunk, s->dtype, st);
+}
+
+}  // namespace
+
+int oal_prefill(const void* q, const void* k, const void* v, const int32_t* group_id,
+                const float* L, const int32_t* G, float eps, float* out, void* state,
+                void* workspace, size_t workspace_bytes, const oal_shape* s, void* stream)
+{
+    return prefill_impl(q, k, v, group_id, L, G, eps, out, state, workspace,
+                             workspace_bytes, s, stream, false);
+}
+
+int oal_prefill_continue(const void* q, const void* k, const void* v, const int32_t* group_id,
+                         const float* L, const int32_t* G, float eps, float* out, void* state,
+                         void* workspace, size_t workspace_bytes, const oal_shape* s,
+                         void* stream)
+{
+    return prefill_impl(q, k, v, group_id, L, G, eps, out, state, workspace,
+                             workspace_bytes, s, stream, true);
 }
 
 int oal_decode_step(const void* q, const void* k, const void* v, void* state, float* out,

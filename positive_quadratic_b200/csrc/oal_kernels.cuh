@@ -32,7 +32,8 @@ size_t tc_image_bytes(int B, int Hkv, int T);
 size_t tc_workspace_bytes(int B, int Hkv, int T);
 int launch_prefill_tc(const void* q, const void* k, const void* v, const int32_t* gid,
                       const float* L, const int32_t* G, float eps, float* out, void* state,
-                      void* ws, int B, int T, int Hq, int Hkv, bool overlap, cudaStream_t st);
+                      void* ws, int B, int T, int Hq, int Hkv, bool overlap, bool cont,
+                      cudaStream_t st);
 
 int launch_chi(const void* q, const void* k, float* chi, int B, int T, int Hq, int Hkv,
                int dtype, cudaStream_t st);

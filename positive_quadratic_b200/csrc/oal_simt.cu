@@ -25,7 +25,7 @@ __device__ __forceinline__ void prep_head(int h, const int32_t* __restrict__ gid
                                           const float* __restrict__ L,
                                           const int32_t* __restrict__ G, float eps,
                                           unsigned char* __restrict__ state, int B, int Hq,
-                                          int Hkv, long long tokens)
+                                          int Hkv, long long tokens, bool add_tokens = false)
 {
     const int tid = threadIdx.x;
     __shared__ double M[kGM1][kGM1];
@@ -82,7 +82,7 @@ __device__ __forceinline__ void prep_head(int h, const int32_t* __restrict__ gid
         hd->dh = kD;
         hd->dv = kDV;
         hd->feat_pad = kFP;
-        hd->tokens = tokens;
+        hd->tokens = add_tokens ? hd->tokens + tokens : tokens;
         hd->eps = eps;
     }
 }

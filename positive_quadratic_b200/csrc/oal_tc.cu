@@ -155,6 +155,7 @@ struct Params {
     float* dS;               // chunk deltas [B*Hkv][NC][65][kFP] fp32
     float* out;
     int B, Hq, Hkv, T, NC;
+    int cont;                // 1: the state already holds a prefix; these tokens continue it
 };
 
 // ------------------------------------------------------------------------------------------
@@ -594,7 +595,7 @@ __device__ void reader_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Pa
     uint32_t* coefh = reinterpret_cast<uint32_t*>(sm + kRdOffCoefH);
     float* wch = reinterpret_cast<float*>(sm + kRdOffW);
     float* c0 = reinterpret_cast<float*>(sm + kRdOffC0);
-    const bool has_inter = c > 0;
+    const bool has_inter = c > 0 || P.cont;
 
     if (threadIdx.x == 0) {
         mbar_init(&bar.qkv_full, 1);
@@ -932,8 +933,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (u1 > u0) delta_item(sm, ctl, tmem, P, u0, u1);
     } else {
         // items with an inter-chunk part first, chunk-major with the heads of a chunk adjacent
-        // (they share the chunk's image in L2); the cheap chunk-0 items last, so that the
-        // final partial wave holds short items
+        // (they share the chunk's image in L2); the chunk-0 items last, so that the final
+        // partial wave holds short items (chunk 0 has no inter-chunk part unless the call
+        // continues a prefix)
         const int nbh = P.B * P.Hq, heavy = nbh * (P.NC - 1), idx = blockIdx.x;
         if (idx < heavy) reader_item(sm, ctl, tmem, P, idx % nbh, 1 + idx / nbh);
         else reader_item(sm, ctl, tmem, P, idx - heavy, 0);
@@ -962,12 +964,12 @@ __global__ void __launch_bounds__(256) scan_kernel(const float* __restrict__ dS,
                                                    const float* __restrict__ L,
                                                    const int32_t* __restrict__ G, float eps,
                                                    unsigned char* __restrict__ state, int B,
-                                                   int Hq, int Hkv, long long tokens)
+                                                   int Hq, int Hkv, long long tokens, int cont)
 {
     grid_dep_launch();
     if (blockIdx.z == gridDim.z - 1) {  // independent of the deltas: no wait
         const int h = blockIdx.y * gridDim.x + blockIdx.x;
-        if (h < Hq) prep_head(h, gid, L, G, eps, state, B, Hq, Hkv, tokens);
+        if (h < Hq) prep_head(h, gid, L, G, eps, state, B, Hq, Hkv, tokens, cont != 0);
         return;
     }
     grid_dep_wait();
@@ -975,11 +977,21 @@ __global__ void __launch_bounds__(256) scan_kernel(const float* __restrict__ dS,
     const int nl = threadIdx.x >> 5, p = threadIdx.x & 31;
     const int n = blockIdx.y * kScanCols + nl;
     __shared__ float fin[kScanCols][64 + 1];
+    float* unit = body + size_t(bkv) * kFP * kW;
+    // the prefix before this call: zero, or (continuation) the state's current contents
     float a0 = 0.f, a1 = 0.f;
+    const int f = sl * 64 + 2 * p, c_first = cont ? 0 : 1;
+    if (cont && n < kDV) {
+        a0 = unit[size_t(f) * kDV + n];
+        a1 = unit[size_t(f + 1) * kDV + n];
+    } else if (cont && n == kDV) {
+        a0 = unit[size_t(kFP) * kDV + f];
+        a1 = unit[size_t(kFP) * kDV + f + 1];
+    }
     if (n >= kW && n < kImgRows) {
         // rows 65..79 of every image: zero (the readout's N = 80 MMA reads them)
         unsigned char* dst = img + (size_t(bkv) * NC * kSlices + sl) * kImgSliceBytes + n * 128 + 4 * p;
-        for (int c = 1; c < NC; ++c)
+        for (int c = c_first; c < NC; ++c)
             *reinterpret_cast<uint32_t*>(dst + size_t(c) * kSlices * kImgSliceBytes) = 0u;
     }
     if (n < kW) {
@@ -995,7 +1007,7 @@ __global__ void __launch_bounds__(256) scan_kernel(const float* __restrict__ dS,
                 d[x] = __ldcs(reinterpret_cast<const float2*>(src + (c + x) * sstride));
 #pragma unroll
             for (int x = 0; x < 4; ++x) {
-                if (c + x >= 1)
+                if (c + x >= c_first)
                     *reinterpret_cast<uint32_t*>(dst + (c + x) * dstride) = pack_bf16x2(a0, a1);
                 a0 += d[x].x;
                 a1 += d[x].y;
@@ -1003,16 +1015,16 @@ __global__ void __launch_bounds__(256) scan_kernel(const float* __restrict__ dS,
         }
         for (; c < NC; ++c) {
             const float2 d = __ldcs(reinterpret_cast<const float2*>(src + c * sstride));
-            if (c >= 1) *reinterpret_cast<uint32_t*>(dst + c * dstride) = pack_bf16x2(a0, a1);
+            if (c >= c_first)
+                *reinterpret_cast<uint32_t*>(dst + c * dstride) = pack_bf16x2(a0, a1);
             a0 += d.x;
             a1 += d.y;
         }
     }
     fin[nl][2 * p] = a0;
     fin[nl][2 * p + 1] = a1;
-    __syncthreads();
+    __syncthreads();  // every read of the old state in this block precedes the writes below
     // final state of unit bkv: Hv[f][n] (n < 64), z[f] (n == 64)
-    float* unit = body + size_t(bkv) * kFP * kW;
     const int fl = threadIdx.x >> 2, cq = threadIdx.x & 3;
 #pragma unroll
     for (int x = 0; x < 2; ++x) {
@@ -1127,14 +1139,15 @@ cudaError_t launch_ex(void (*kern)(Args...), dim3 grid, dim3 block, size_t smem,
 
 int launch_prefill_tc(const void* q, const void* k, const void* v, const int32_t* gid,
                       const float* L, const int32_t* G, float eps, float* out, void* state,
-                      void* ws, int B, int T, int Hq, int Hkv, bool overlap, cudaStream_t st)
+                      void* ws, int B, int T, int Hq, int Hkv, bool overlap, bool cont,
+                      cudaStream_t st)
 {
     if (B == 0) return OAL_OK;
     const int NC = (T + tc::kC - 1) / tc::kC;
     unsigned char* sb = static_cast<unsigned char*>(state);
     float* body = reinterpret_cast<float*>(sb + kHeaderBytes + coef_bytes(Hq));
     if (T == 0) {
-        OAL_CUDA_TRY(cudaMemsetAsync(body, 0, size_t(B) * Hkv * state_unit_bytes(), st));
+        if (!cont) OAL_CUDA_TRY(cudaMemsetAsync(body, 0, size_t(B) * Hkv * state_unit_bytes(), st));
         return OAL_OK;
     }
     unsigned char* wsb = static_cast<unsigned char*>(ws);
@@ -1157,6 +1170,7 @@ int launch_prefill_tc(const void* q, const void* k, const void* v, const int32_t
     P.Hkv = Hkv;
     P.T = T;
     P.NC = NC;
+    P.cont = cont ? 1 : 0;
     const int units = B * Hkv * NC * tc::kNumSlabs;
     const int grid0 = std::max(1, std::min(sm_count(), units));
     OAL_CUDA_TRY(cudaFuncSetAttribute(tc::prefill_tc_kernel<0>,
@@ -1175,7 +1189,7 @@ int launch_prefill_tc(const void* q, const void* k, const void* v, const int32_t
         OAL_CUDA_TRY(launch_ex(tc::scan_kernel,
                                dim3(tc::kSlices, tc::kImgRows / tc::kScanCols, B * Hkv + 1),
                                dim3(256), 0, st, overlap, (const float*)P.dS, P.img, body, NC,
-                               gid, L, G, eps, sb, B, Hq, Hkv, (long long)T));
+                               gid, L, G, eps, sb, B, Hq, Hkv, (long long)T, P.cont));
     }
     {
         LaunchScope ls("readout_tc", st);

@@ -68,6 +68,7 @@ def lib() -> ctypes.CDLL:
                          "oal_decode_workspace_bytes"):
                 getattr(L, name).argtypes = [_PS, ctypes.POINTER(_SZ)]
             L.oal_prefill.argtypes = [_VP] * 6 + [ctypes.c_float, _VP, _VP, _VP, _SZ, _PS, _VP]
+            L.oal_prefill_continue.argtypes = L.oal_prefill.argtypes
             L.oal_decode_step.argtypes = [_VP] * 6 + [_SZ, _PS, _VP]
             L.oal_dense_ref_gpu.argtypes = [_VP] * 6 + [ctypes.c_float, _VP, _PS, _VP]
             L.oal_contribution_stat.argtypes = [_VP, _VP, _VP, _PS, _VP]
@@ -84,7 +85,8 @@ def lib() -> ctypes.CDLL:
             L.oal_profile_read.restype = ctypes.c_int
             for name in ("oal_state_bytes", "oal_prefill_workspace_bytes",
                          "oal_decode_workspace_bytes", "oal_prefill", "oal_decode_step",
-                         "oal_dense_ref_gpu", "oal_device_error", "oal_contribution_stat"):
+                         "oal_dense_ref_gpu", "oal_device_error", "oal_contribution_stat",
+                         "oal_prefill_continue"):
                 getattr(L, name).restype = ctypes.c_int
             _lib = L
     return _lib
@@ -196,6 +198,26 @@ def prefill(q, k, v, group_id, L, G, eps: float, chunk: int = 128, out=None, sta
                            _stream(stream))
     _check(rc, "oal_prefill")
     return out, state
+
+
+def prefill_continue(q, k, v, group_id, L, G, eps: float, state, out=None, workspace=None,
+                     stream=None):
+    """oal_prefill_continue: appends the T tokens of q/k/v to the sequence held by `state`
+    (bf16, chunk 128).  Returns out [B,Hq,T,dv] fp32; `state` is updated in place."""
+    shape = _shape_of(q, k, v, 128)
+    dev = q.device
+    if out is None:
+        out = torch.empty(q.shape[0], q.shape[1], q.shape[2], v.shape[3], dtype=torch.float32,
+                          device=dev)
+    if workspace is None:
+        workspace = empty_workspace(prefill_workspace_bytes(shape), dev)
+    _contig_cuda(q, k, v, group_id, L, G, out, state, workspace)
+    rc = lib().oal_prefill_continue(_ptr(q), _ptr(k), _ptr(v), _ptr(group_id), _ptr(L),
+                                    _ptr(G), float(eps), _ptr(out), _ptr(state),
+                                    _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                    ctypes.byref(shape), _stream(stream))
+    _check(rc, "oal_prefill_continue")
+    return out
 
 
 def decode_step(q, k, v, state, workspace, out=None, stream=None):

@@ -312,3 +312,37 @@ def test_contribution_stat_config1(oal, cuda):
     np.testing.assert_allclose(chi, ref, rtol=1e-5, atol=0)
     # the outlier dimensions dominate the statistic, as the grouping assumes
     assert np.all(chi.max(axis=-1) > 4 * np.median(chi, axis=-1))
+
+
+# --- prefill continuation ----------------------------------------------------------------------
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("T1,T2", [(200, 1), (256, 300), (129, 700), (1000, 128)])
+def test_prefill_continuation(oal, cuda, T1, T2):
+    """prefill(T1) then continue(T2) = one prefill of T1 + T2 tokens: outputs of the appended
+    tokens and the final state match the oracle run over the whole sequence."""
+    p = I.small_layer(700 + T1 + T2, B=2, T=T1 + T2, Hq=14, Hkv=2, dtype="bf16")
+    ref, st = oracle.recurrent(p.q, p.k, p.v, p.group_id, p.L, p.G, p.eps, return_state=True)
+    a, b = p.slice_tokens(0, T1), p.slice_tokens(T1, T1 + T2)
+    qa, ka, va, g, L, G = dev_inputs(a, cuda)
+    qb, kb, vb, *_ = dev_inputs(b, cuda)
+    _, state = oal.prefill(qa, ka, va, g, L, G, p.eps, 128)
+    yb = oal.prefill_continue(qb, kb, vb, g, L, G, p.eps, state)
+    torch.cuda.synchronize()
+    assert oal.device_error() == 0
+    assert row_rel_err(yb.cpu().numpy(), ref[:, :, T1:]) <= TOL_BF16
+    hdr, _, S = read_state(state.cpu().numpy(), 2, 14, 2)
+    assert hdr["tokens"] == T1 + T2
+    refS = pack_oracle_state(st)
+    assert np.max(np.abs(S[:, :, :F] - refS) / np.abs(refS).max(axis=2, keepdims=True)) < 1e-5
+
+
+@pytest.mark.gpu
+def test_prefill_continuation_unsupported_paths(oal, cuda):
+    """Continuation runs on the tensor-core path only; fp32 inputs are refused before any
+    launch."""
+    p = I.small_layer(31, B=1, T=64, Hq=4, Hkv=2, dtype="f32")
+    q, k, v, g, L, G = dev_inputs(p, cuda)
+    _, state = oal.prefill(q, k, v, g, L, G, p.eps, 128)
+    with pytest.raises(oal.OALError):
+        oal.prefill_continue(q, k, v, g, L, G, p.eps, state)
