@@ -121,7 +121,9 @@ int oal_decode_workspace_bytes(const oal_shape* s, size_t* bytes);
  * state of eq. (4) is built and read out with eq. (5).  Linear in T for fixed d_h.
  * bf16 inputs with chunk 128 run on tcgen05 tensor cores (bf16 operands, fp32 accumulation,
  * exact fp32 final state); fp32 inputs, and bf16 with chunk 64 or 256, run on CUDA cores in
- * fp32.  `workspace` must hold oal_prefill_workspace_bytes(s) bytes. */
+ * fp32.  `workspace` must hold oal_prefill_workspace_bytes(s) bytes.  out == NULL computes
+ * the state alone (no readout; q may then be NULL too), e.g. the per-segment state of a
+ * sequence-parallel prefill. */
 int oal_prefill(const void* q, const void* k, const void* v, const int32_t* group_id,
                 const float* L, const int32_t* G, float eps, float* out, void* state,
                 void* workspace, size_t workspace_bytes, const oal_shape* s, void* stream);

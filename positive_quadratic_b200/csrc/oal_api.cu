@@ -124,7 +124,8 @@ int prefill_impl(const void* q, const void* k, const void* v, const int32_t* gro
     if ((rc = check_chunk(s))) return rc;
     if (cont && !use_tensor_path(s)) return OAL_ERR_UNSUPPORTED;
     if (!group_id || !L || !G || !state) return OAL_ERR_NULL;
-    if ((rc = check_io(s, q, k, v, out))) return rc;
+    // out == NULL asks for the state alone (no readout); q is then not read either
+    if ((rc = check_io(s, out ? q : k, k, v, out ? out : v))) return rc;
     if (!aligned16(state) || !aligned16(group_id) || !aligned16(L) || !aligned16(G))
         return OAL_ERR_ALIGN;
     size_t need = 0;

@@ -84,6 +84,8 @@ __device__ __forceinline__ void prep_head(int h, const int32_t* __restrict__ gid
         hd->feat_pad = kFP;
         hd->tokens = add_tokens ? hd->tokens + tokens : tokens;
         hd->eps = eps;
+        for (int i = 0; i < int(sizeof(hd->reserved) / sizeof(hd->reserved[0])); ++i)
+            hd->reserved[i] = 0;  // every byte of the state is defined
     }
 }
 
@@ -535,7 +537,7 @@ static int launch_prefill_simt_t(const Tin* q, const Tin* k, const Tin* v,
                                                                          body);
         OAL_LAUNCH_CHECK();
     }
-    if (T == 0) return OAL_OK;
+    if (T == 0 || out == nullptr) return OAL_OK;  // no out: the state alone is wanted
     const size_t smem = sizeof(ReadoutSmem);
     auto kern = readout_simt_kernel<Tin, false>;
     OAL_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));

@@ -1152,7 +1152,9 @@ int launch_prefill_tc(const void* q, const void* k, const void* v, const int32_t
     }
     unsigned char* wsb = static_cast<unsigned char*>(ws);
     CUtensorMap mq, mk, mv, mi;
-    if (!make_map(&mq, q, T, B * Hq) || !make_map(&mk, k, T, B * Hkv) ||
+    // without out (state only) q is not read: its map then describes k and is never used
+    if (!(out ? make_map(&mq, q, T, B * Hq) : make_map(&mq, k, T, B * Hkv)) ||
+        !make_map(&mk, k, T, B * Hkv) ||
         !make_map(&mv, v, T, B * Hkv) ||
         !make_img_map(&mi, wsb, size_t(B) * Hkv * NC * tc::kSlices))
         return OAL_ERR_CUDA;
@@ -1191,6 +1193,7 @@ int launch_prefill_tc(const void* q, const void* k, const void* v, const int32_t
                                dim3(256), 0, st, overlap, (const float*)P.dS, P.img, body, NC,
                                gid, L, G, eps, sb, B, Hq, Hkv, (long long)T, P.cont));
     }
+    if (out == nullptr) return OAL_OK;  // no out: the state alone is wanted
     {
         LaunchScope ls("readout_tc", st);
         OAL_CUDA_TRY(launch_ex(tc::prefill_tc_kernel<1>, dim3(NC * B * Hq), dim3(tc::kThreads),

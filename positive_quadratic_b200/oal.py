@@ -200,6 +200,39 @@ def prefill(q, k, v, group_id, L, G, eps: float, chunk: int = 128, out=None, sta
     return out, state
 
 
+def prefill_state(k, v, group_id, L, G, eps: float, Hq: int, chunk: int = 128, state=None,
+                  workspace=None, stream=None):
+    """oal_prefill with out = NULL: the prefix state after the T tokens of k/v (and the
+    coefficient tables of Hq query heads), without computing outputs."""
+    B, Hkv, T, dh = k.shape
+    shape = make_shape(B, T, Hq, Hkv, chunk, _dtype_code(k), dh, v.shape[3])
+    dev = k.device
+    if state is None:
+        state = torch.empty(state_bytes(shape), dtype=torch.uint8, device=dev)
+    if workspace is None:
+        workspace = empty_workspace(prefill_workspace_bytes(shape), dev)
+    _contig_cuda(k, v, group_id, L, G, state, workspace)
+    rc = lib().oal_prefill(None, _ptr(k), _ptr(v), _ptr(group_id), _ptr(L), _ptr(G),
+                           float(eps), None, _ptr(state), _ptr(workspace),
+                           workspace.numel() * workspace.element_size(), ctypes.byref(shape),
+                           _stream(stream))
+    _check(rc, "oal_prefill (state only)")
+    return state
+
+
+def state_body(state: torch.Tensor, B: int, Hq: int, Hkv: int) -> torch.Tensor:
+    """fp32 view of the per-(b, kv) prefix states inside a state buffer (after the header and
+    the coefficient tables): B*Hkv units of Hv[2176][64] then z[2176]."""
+    off = 256 + ((Hq * FEATURES_PAD * 4 + 255) // 256) * 256
+    n = B * Hkv * FEATURES_PAD * (VALUE_DIM + 1)
+    return state[off:off + 4 * n].view(torch.float32)
+
+
+def set_state_tokens(state: torch.Tensor, tokens: int) -> None:
+    """Sets the token count in a state header (int64 at byte 32)."""
+    state[32:40].copy_(torch.tensor([int(tokens)], dtype=torch.int64).view(torch.uint8))
+
+
 def prefill_continue(q, k, v, group_id, L, G, eps: float, state, out=None, workspace=None,
                      stream=None):
     """oal_prefill_continue: appends the T tokens of q/k/v to the sequence held by `state`

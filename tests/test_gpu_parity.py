@@ -346,3 +346,23 @@ def test_prefill_continuation_unsupported_paths(oal, cuda):
     _, state = oal.prefill(q, k, v, g, L, G, p.eps, 128)
     with pytest.raises(oal.OALError):
         oal.prefill_continue(q, k, v, g, L, G, p.eps, state)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dtype,chunk", [("bf16", 128), ("bf16", 64), ("f32", 128)])
+def test_state_only_prefill(oal, cuda, dtype, chunk):
+    """out = NULL computes the same state as a full prefill, without the readout."""
+    p = I.small_layer(77, B=2, T=300, Hq=4, Hkv=2, dtype=dtype)
+    q, k, v, g, L, G = dev_inputs(p, cuda)
+    _, full = oal.prefill(q, k, v, g, L, G, p.eps, chunk)
+    oal.profile_read()
+    oal.profile_enable(True)
+    alone = oal.prefill_state(k, v, g, L, G, p.eps, 4, chunk)
+    oal.profile_enable(False)
+    names = set(oal.profile_read())
+    torch.cuda.synchronize()
+    assert oal.device_error() == 0
+    assert not any(n.startswith("readout") for n in names), names
+    # defined bytes: header fields (0..44), coefficient tables and prefix states (256..)
+    assert torch.equal(full[:44], alone[:44])
+    assert torch.equal(full[256:], alone[256:])
