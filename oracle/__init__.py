@@ -60,8 +60,14 @@ def _load():
                                                                        ctypes.c_int, _I, _I, _I,
                                                                        _D]
             lib.oal_oracle_chi.argtypes = [ctypes.c_int] * 5 + [_D, _D, _D]
+            lib.oal_oracle_hadamard_recurrent.argtypes = [ctypes.c_int] * 6 + [_D] * 14
+            lib.oal_oracle_hadamard_dense.argtypes = [ctypes.c_int] * 6 + [_D] * 8
+            lib.oal_oracle_dense_backward.argtypes = [ctypes.c_int] * 6 + [
+                _D, _D, _D, _I, _D, _I, ctypes.c_int, ctypes.c_double] + [_D] * 6
             for f in (lib.oal_oracle_kappa, lib.oal_oracle_dense, lib.oal_oracle_recurrent,
-                      lib.oal_oracle_dense_rows, lib.oal_oracle_chi):
+                      lib.oal_oracle_dense_rows, lib.oal_oracle_chi,
+                      lib.oal_oracle_hadamard_recurrent, lib.oal_oracle_hadamard_dense,
+                      lib.oal_oracle_dense_backward):
                 f.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -179,6 +185,84 @@ def chi(q, k):
     _check(_load().oal_oracle_chi(B, Hq, k.shape[1], T, dh, _d(q), _d(k), _d(out)),
            "oal_oracle_chi")
     return out
+
+
+def grouped_coefficients(group_id, L, G, eps):
+    """Coefficients (a [Hq], b [Hq, dh], C [Hq, dh, dh]) of eq. (5) that the grouped kernel of
+    eq. (3) expands into, with M = L L^T over each head's leading (G+1)x(G+1) block and
+    sbar_0 = 1: a = eps + M_00, b_r = 2 M_{0,g(r)}, C_rt = M_{g(r),g(t)}."""
+    group_id, G, L = _i32(group_id), _i32(G), _f64(L)
+    Hq, dh = group_id.shape
+    a, b, C = np.empty(Hq), np.empty((Hq, dh)), np.empty((Hq, dh, dh))
+    for h in range(Hq):
+        n = int(G[h]) + 1
+        M = L[h, :n, :n] @ L[h, :n, :n].T
+        g = group_id[h]
+        a[h] = eps + M[0, 0]
+        b[h] = 2.0 * M[0, g]
+        C[h] = M[np.ix_(g, g)]
+    return a, b, C
+
+
+def _hadamard_common(q, k, v, a, b, C):
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    if q.ndim != 4 or k.ndim != 4 or v.ndim != 4:
+        raise ValueError("q, k, v must be [B, H, T, d]")
+    B, Hq, T, dh = q.shape
+    Hkv, dv = k.shape[1], v.shape[3]
+    if k.shape != (B, Hkv, T, dh) or v.shape != (B, Hkv, T, dv):
+        raise ValueError("k/v shape mismatch")
+    a, b, C = _f64(np.reshape(a, (Hq,))), _f64(b), _f64(C)
+    if b.shape != (Hq, dh) or C.shape != (Hq, dh, dh):
+        raise ValueError("a [Hq], b [Hq, dh], C [Hq, dh, dh] expected")
+    return q, k, v, a, b, C, (B, Hq, Hkv, T, dh, dv)
+
+
+def hadamard_dense(q, k, v, a, b, C, return_u: bool = False):
+    """Ungrouped Hadamard form, dense: kappa = a + sum_r b_r x_r + sum_rt C_rt x_r x_t with
+    x = q*k/sqrt(dh), u_i = sum_{j<=i} kappa_ij [v_j; 1], yhat_i = u_i[:dv] / u_i[dv]."""
+    q, k, v, a, b, C, (B, Hq, Hkv, T, dh, dv) = _hadamard_common(q, k, v, a, b, C)
+    y = np.empty((B, Hq, T, dv))
+    u = np.empty((B, Hq, T, dv + 1)) if return_u else None
+    _check(_load().oal_oracle_hadamard_dense(B, Hq, Hkv, T, dh, dv, _d(q), _d(k), _d(v), _d(a),
+                                             _d(b), _d(C), _d(y), _d(u)), "hadamard_dense")
+    return (y, u) if return_u else y
+
+
+def hadamard_recurrent(q, k, v, a, b, C, state: State | None = None,
+                       return_state: bool = False, return_u: bool = False):
+    """Ungrouped Hadamard form through eqs. (4)-(5) with the given a, b, C.  Returns y, then
+    the state after the tokens (return_state) and u [B, Hq, T, dv+1] (return_u)."""
+    q, k, v, a, b, C, (B, Hq, Hkv, T, dh, dv) = _hadamard_common(q, k, v, a, b, C)
+    y = np.empty((B, Hq, T, dv))
+    u = np.empty((B, Hq, T, dv + 1)) if return_u else None
+    out = State.zeros(B, Hkv, dh, dv) if return_state else None
+    ins = (state.H0, state.H1, state.H2) if state is not None else (None, None, None)
+    outs = (out.H0, out.H1, out.H2) if out is not None else (None, None, None)
+    _check(_load().oal_oracle_hadamard_recurrent(B, Hq, Hkv, T, dh, dv, _d(q), _d(k), _d(v),
+                                                 _d(a), _d(b), _d(C), *[_d(x) for x in ins],
+                                                 *[_d(x) for x in outs], _d(y), _d(u)),
+           "hadamard_recurrent")
+    res = [y] + ([out] if return_state else []) + ([u] if return_u else [])
+    return res[0] if len(res) == 1 else tuple(res)
+
+
+def dense_backward(q, k, v, group_id, L, G, eps, dy):
+    """Gradients of the dense grouped form for upstream dy = dLoss/dyhat [B, Hq, T, dv]:
+    dict(dq, dk, dv, dL [Hq, Gmax+1, Gmax+1], deps)."""
+    q, k, v, group_id, L, G, (B, Hq, Hkv, T, dh, dv, Gmax) = _common(q, k, v, group_id, L, G)
+    dy = _f64(dy)
+    if dy.shape != (B, Hq, T, dv):
+        raise ValueError("dy must be [B, Hq, T, dv]")
+    dq, dk, dvv = np.empty(q.shape), np.empty(k.shape), np.empty(v.shape)
+    dL = np.empty(L.shape)
+    deps = np.zeros(1)
+    _check(_load().oal_oracle_dense_backward(B, Hq, Hkv, T, dh, dv, _d(q), _d(k), _d(v),
+                                             group_id.ctypes.data_as(_I), _d(L),
+                                             G.ctypes.data_as(_I), Gmax, float(eps), _d(dy),
+                                             _d(dq), _d(dk), _d(dvv), _d(dL), _d(deps)),
+           "dense_backward")
+    return dict(dq=dq, dk=dk, dv=dvv, dL=dL, deps=float(deps[0]))
 
 
 def threads() -> int:
