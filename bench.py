@@ -6,8 +6,10 @@ Headline (one JSON line on rank 0):
            2 key-value heads, d_h = dv = 64, bf16 inputs (seeded synthetic, same recipe as the
            parity tests), chunk 128.  One step = one oal_prefill call = the whole prefill
            hot path (coefficient expansion, chunk-state builder, readout with the intra-chunk
-           dense kernel).  Inputs are resident in HBM; L2 (126 MB) is flushed by writing a
-           256 MB buffer between steps, outside the timed events.
+           dense kernel).  Inputs are resident in HBM.  Between steps, outside the timed
+           events, a 256 MB buffer is written and another 256 MB read, so each timed step
+           starts on a cold L2 (126 MB) holding no dirty lines (--l2-flush write: the write
+           alone).
   e2e    = the same metric through the public Python API with pinned HOST buffers: every
            step copies q/k/v host->device, runs the prefill and copies yhat device->host.
   decode = autoregressive decode tokens/s: batch 64, 4096-token context prefilled into the
@@ -58,6 +60,12 @@ def parse():
     ap.add_argument("--no-overlap", action="store_true",
                     help="launch the prefill's scan and readout kernels in plain stream order "
                          "instead of as programmatic dependents")
+    ap.add_argument("--l2-flush", default="write+read", choices=["write+read", "write"],
+                    help="between timed steps: write a 256 MB buffer, then (default) read "
+                         "another 256 MB so that the write's dirty lines are written back "
+                         "outside the timed events")
+    ap.add_argument("--decode-variant", type=int, default=0, choices=[0, 1],
+                    help="decode kernel: 0 register-batched rows, 1 bulk-copied state slabs")
     ap.add_argument("--workload", default="config1", choices=["config1", "config3_16k",
                                                               "config3_32k", "config3_64k"],
                     help="prefill workload (config1 is the headline)")
@@ -260,6 +268,7 @@ def main():
     pk, pk_kind = peaks()
     oal.lib()
     oal.set_prefill_overlap(not args.no_overlap)
+    oal.set_decode_variant(args.decode_variant)
 
     p, desc = workload(args.workload)
     B, Hq, T, _ = p.q.shape
@@ -268,7 +277,7 @@ def main():
     out, state = oal.prefill(q, k, v, g, L, G, p.eps, args.chunk)
     ws = oal.empty_workspace(oal.prefill_workspace_bytes(
         oal.make_shape(B, T, Hq, Hkv, args.chunk, oal.OAL_BF16)), dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(torch, dev, args.l2_flush == "write+read")
     stream = torch.cuda.current_stream()
 
     def barrier():
@@ -280,7 +289,7 @@ def main():
 
     for _ in range(max(args.warmup, 3)):
         step()
-        flush.zero_()
+        flush()
     torch.cuda.synchronize()
     assert oal.device_error() == 0
 
@@ -297,7 +306,7 @@ def main():
             s0.record(stream)
             step()
             s1.record(stream)
-            flush.zero_()
+            flush()
         torch.cuda.synchronize()
     n_launch = oal.launch_count() - n0
     barrier()
@@ -344,7 +353,7 @@ def main():
         hout = torch.empty(out.shape, dtype=torch.float32, pin_memory=True)
         for _ in range(3):
             oal.prefill_host(hq, hk, hv, g, L, G, p.eps, args.chunk, bufs, hout)
-            flush.zero_()
+            flush()
         evs2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                 for _ in range(args.steps)]
         barrier()
@@ -353,7 +362,7 @@ def main():
             s0.record(stream)
             oal.prefill_host(hq, hk, hv, g, L, G, p.eps, args.chunk, bufs, hout)
             s1.record(stream)
-            flush.zero_()
+            flush()
         torch.cuda.synchronize()
         e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs2), world, dev)
         e2e = {"value": job_rate(world, args.steps * B * T, e_ms), "unit": UNIT,
@@ -377,7 +386,7 @@ def main():
                 "config": {"workload": desc, "chunk": args.chunk,
                            "schedule": "deltas, scan, readout" + (
                                "" if args.no_overlap else " (programmatic dependent launch)"),
-                           "l2": "flushed between steps (256 MB write, outside timed events)",
+                           "l2": flush.describe(),
                            "parallelism": f"replicas x{world}"},
                 "roofline": roof, "e2e": e2e, "gpu_launches": int(n_launch),
                 "clocks": clk.summary(), "decode": decode, "cpu_baseline": base,
@@ -386,6 +395,31 @@ def main():
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+class L2Flush:
+    """Evicts the 126 MB L2 between timed steps, outside the timed events.  A 256 MB write
+    alone leaves the L2 full of its own dirty lines, which the next timed kernel then has to
+    write back to HBM on top of its own traffic; the default therefore follows the write with
+    a read of a second 256 MB buffer, so the timed kernel starts on a cold L2 holding only
+    clean lines (as a profiler's cache flush leaves it)."""
+
+    def __init__(self, torch, dev, clean: bool):
+        self.torch, self.clean = torch, clean
+        self.wbuf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        self.rbuf = (torch.zeros((256 << 20) // 4, dtype=torch.float32, device=dev)
+                     if clean else None)
+        self.sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        self.wbuf.zero_()
+        if self.clean:
+            self.torch.sum(self.rbuf, dim=0, out=self.sink)
+
+    def describe(self) -> str:
+        return ("flushed between steps: 256 MB write, then 256 MB read so no dirty lines remain "
+                "(outside timed events)" if self.clean else
+                "flushed between steps: 256 MB write (outside timed events)")
 
 
 def run_decode(args, dev, torch, oal, pk, pk_kind, flush, world, barrier):
@@ -421,7 +455,7 @@ def run_decode(args, dev, torch, oal, pk, pk_kind, flush, world, barrier):
         s0.record(stream)
         oal.decode_step(qs[i], ks[i], vs[i], state, ws, out=out)
         s1.record(stream)
-        flush.zero_()
+        flush()
     torch.cuda.synchronize()
     oal.profile_enable(False)
     prof = oal.profile_read()
@@ -429,19 +463,21 @@ def run_decode(args, dev, torch, oal, pk, pk_kind, flush, world, barrier):
     ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world, dev)
     state_bytes = 2.0 * B * Hkv * F * W * 4   # every packed row read and written once
     io_bytes = B * (Hq + 2 * Hkv) * 64 * 2 + B * Hq * 64 * 4
-    kern = prof.get("decode")
+    kname = "decode_bulk" if args.decode_variant == 1 else "decode"
+    kern = prof.get(kname)
     roof = None
     if kern:
         per = kern[1] / kern[0]
         gbs = (state_bytes + io_bytes) / (per / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": gbs / pk["hbm_gbs"], "frac_of_8tbs": gbs / 8000.0, "traffic": None,
-                "kernel": "decode", "avg_launch_ms": per, "peak_kind": pk_kind,
+                "kernel": kname, "avg_launch_ms": per, "peak_kind": pk_kind,
                 "algorithmic_bytes_per_launch": state_bytes + io_bytes}
     return {"value": job_rate(world, B * nsteps, ms), "unit": UNIT,
             "ms_per_token_step": ms / nsteps, "batch": B, "context": 4096, "steps": nsteps,
             "roofline": roof,
-            "workload": "decode batch 64, context 4096, Hq=14 Hkv=2 d=64 bf16 q/k/v, fp32 state"}
+            "workload": "decode batch 64, context 4096, Hq=14 Hkv=2 d=64 bf16 q/k/v, fp32 state",
+            "kernel": kname}
 
 
 if __name__ == "__main__":

@@ -197,6 +197,14 @@ int oal_contribution_stat(const void* q, const void* k, float* chi, const oal_sh
  * results.  Process-wide; returns the previous setting. */
 int oal_set_prefill_overlap(int overlap);
 
+/* Decode kernel (oal_decode_step and oal_decode_step_noalloc).  0 (default): each thread
+ * keeps a batch of state rows in flight in registers.  1: each block streams its whole state
+ * slab into shared memory with bulk copies (cp.async.bulk) issued before it forms the feature
+ * weights.  Both use the same partition, workspace and summation order, so the results are
+ * identical.  Process-wide; returns the previous setting, or OAL_ERR_UNSUPPORTED (setting
+ * unchanged) for any other value. */
+int oal_set_decode_variant(int variant);
+
 /* Reads the device-side error word (OAL_OK or a negative oal_status set by a kernel since
  * the last read), synchronising `stream`, and clears it. */
 int oal_device_error(int* code, void* stream);

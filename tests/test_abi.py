@@ -90,3 +90,17 @@ def test_header_packed_order_is_complete():
     p = packed_pairs()
     assert len({(int(r), int(t)) for r, t in p}) == 2145
     assert all(r <= t for r, t in p)
+
+
+def test_decode_variant_switch():
+    """The decode-kernel switch is host state only: it accepts 0 and 1, returns the previous
+    value and refuses anything else without changing the setting."""
+    prev = oal.set_decode_variant(1)
+    try:
+        assert prev == 0
+        assert oal.set_decode_variant(1) == 1
+        with pytest.raises(oal.OALError):
+            oal.set_decode_variant(2)
+        assert oal.set_decode_variant(0) == 1
+    finally:
+        oal.set_decode_variant(prev)
