@@ -10,8 +10,10 @@ Headline (one JSON line on rank 0):
            events, a 256 MB buffer is written and another 256 MB read, so each timed step
            starts on a cold L2 (126 MB) holding no dirty lines (--l2-flush write: the write
            alone).
-  e2e    = the same metric through the public Python API with pinned HOST buffers: every
-           step copies q/k/v host->device, runs the prefill and copies yhat device->host.
+  e2e    = the same metric through the C ABI's host-buffer call (oal_prefill_host) with
+           pinned HOST buffers: every step copies q/k/v host->device, runs the prefill and
+           copies yhat device->host, the copies of one segment overlapping the kernels of the
+           next (checked once to reproduce the device-resident prefill bit for bit).
   decode = autoregressive decode tokens/s: batch 64, 4096-token context prefilled into the
            packed fp32 states, then single-token steps (L2 flushed between steps).
   roofline = the dominant prefill kernel's achieved rate from the library's CUDA-event trace
@@ -64,6 +66,8 @@ def parse():
                     help="between timed steps: write a 256 MB buffer, then (default) read "
                          "another 256 MB so that the write's dirty lines are written back "
                          "outside the timed events")
+    ap.add_argument("--e2e-segments", type=int, default=4,
+                    help="segments of the e2e host-buffer prefill (copies overlap kernels)")
     ap.add_argument("--decode-variant", type=int, default=0, choices=[0, 1],
                     help="decode kernel: 0 register-batched rows, 1 bulk-copied state slabs")
     ap.add_argument("--workload", default="config1", choices=["config1", "config3_16k",
@@ -343,16 +347,23 @@ def main():
                 "whole_step_frac_of_bf16_peak": prefill_flops(B, T, Hq, Hkv) /
                 (total_ms / args.steps / 1e3) / 1e12 / pk["bf16_tflops"]}
 
-    # ---- e2e through the public API with pinned host buffers ----
+    # ---- e2e through the C ABI with pinned host buffers (oal_prefill_host) ----
     e2e = None
     if not args.no_e2e:
         hq = q.cpu().pin_memory()
         hk = k.cpu().pin_memory()
         hv = v.cpu().pin_memory()
-        bufs = oal.alloc_prefill_buffers(hq, hk, hv, g, L, G, args.chunk, device=dev)
         hout = torch.empty(out.shape, dtype=torch.float32, pin_memory=True)
+        bufs = oal.host_prefill_buffers(hq, hk, hv, g, L, G, args.chunk, args.e2e_segments,
+                                        device=dev)
+        oal.prefill_from_host(hq, hk, hv, p.eps, bufs, hout)
+        torch.cuda.synchronize()
+        # the segmented call must reproduce the device-resident prefill exactly
+        same = bool(torch.equal(hout, out.cpu())) and oal.device_error() == 0
+        if not same:
+            bufs = oal.host_prefill_buffers(hq, hk, hv, g, L, G, args.chunk, 1, device=dev)
         for _ in range(3):
-            oal.prefill_host(hq, hk, hv, g, L, G, p.eps, args.chunk, bufs, hout)
+            oal.prefill_from_host(hq, hk, hv, p.eps, bufs, hout)
             flush()
         evs2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                 for _ in range(args.steps)]
@@ -360,14 +371,18 @@ def main():
         torch.cuda.synchronize()
         for s0, s1 in evs2:
             s0.record(stream)
-            oal.prefill_host(hq, hk, hv, g, L, G, p.eps, args.chunk, bufs, hout)
+            oal.prefill_from_host(hq, hk, hv, p.eps, bufs, hout)
             s1.record(stream)
             flush()
         torch.cuda.synchronize()
+        assert oal.device_error() == 0
         e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs2), world, dev)
         e2e = {"value": job_rate(world, args.steps * B * T, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": int(hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2),
-               "d2h_bytes_per_step": int(hout.numel() * 4)}
+               "d2h_bytes_per_step": int(hout.numel() * 4),
+               "api": "oal_prefill_host",
+               "segments": bufs["segments"] if same else 1,
+               "segmented_matches_device_prefill": same}
 
     # ---- decode ----
     decode = None

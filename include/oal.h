@@ -197,6 +197,37 @@ int oal_contribution_stat(const void* q, const void* k, float* chi, const oal_sh
  * results.  Process-wide; returns the previous setting. */
 int oal_set_prefill_overlap(int overlap);
 
+/* Scratch needed by oal_prefill_host for `s` cut into `segments` segments: device staging
+ * for q, k, v and yhat of the whole call plus the prefill workspace of the longest segment. */
+int oal_prefill_host_workspace_bytes(const oal_shape* s, int segments, size_t* bytes);
+
+/* Prefill from HOST memory, with the copies overlapped with the kernels.  q_host, k_host and
+ * v_host are host arrays in oal_prefill's layouts, and out_host receives yhat
+ * [B][Hq][T][dv] fp32 in host memory.  They should be page-locked, or the copies will not
+ * overlap.  group_id, L, G and state are device memory, as for oal_prefill.
+ * The T tokens are cut into `segments` contiguous segments whose boundaries fall on chunk
+ * boundaries (fewer when T is short). For each segment:
+ *  - it is copied to the device on `copy_in`;
+ *  - it is computed on `stream`: oal_prefill for the first segment, oal_prefill_continue for
+ *    the others;
+ *  - its yhat is copied back on `copy_out` while the next segment computes.
+ * The continued prefix scan adds the chunk deltas in the order one whole prefill does, so
+ * yhat and the state equal those of oal_prefill over the whole sequence.
+ * `workspace` is device memory of oal_prefill_host_workspace_bytes(s, segments) bytes,
+ * 256-byte aligned.  `stream`, `copy_in` and `copy_out` are caller-owned; a NULL copy stream
+ * means `stream` (no overlap on that side).  The call returns once everything is enqueued.
+ * The work is ordered after earlier work on `stream`, and later work on `stream` is ordered
+ * after the last copy back.  Synchronise `stream` before reading out_host or reusing the host
+ * inputs.
+ * Errors: as oal_prefill; OAL_ERR_UNSUPPORTED for segments > 1 off the tensor-core path
+ * (bf16, chunk 128); OAL_ERR_SHAPE for segments < 1; OAL_ERR_CUDA if a copy or event call
+ * fails. */
+int oal_prefill_host(const void* q_host, const void* k_host, const void* v_host,
+                     const int32_t* group_id, const float* L, const int32_t* G, float eps,
+                     float* out_host, void* state, void* workspace, size_t workspace_bytes,
+                     const oal_shape* s, int segments, void* stream, void* copy_in,
+                     void* copy_out);
+
 /* Decode kernel (oal_decode_step and oal_decode_step_noalloc).  0 (default): each thread
  * keeps a batch of state rows in flight in registers.  1: each block streams its whole state
  * slab into shared memory with bulk copies (cp.async.bulk) issued before it forms the feature

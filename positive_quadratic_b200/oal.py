@@ -78,6 +78,12 @@ def lib() -> ctypes.CDLL:
             L.oal_last_cuda_error.restype = ctypes.c_int
             L.oal_set_prefill_overlap.argtypes = [ctypes.c_int]
             L.oal_set_prefill_overlap.restype = ctypes.c_int
+            L.oal_prefill_host_workspace_bytes.argtypes = [_PS, ctypes.c_int,
+                                                           ctypes.POINTER(_SZ)]
+            L.oal_prefill_host.argtypes = [_VP] * 6 + [ctypes.c_float, _VP, _VP, _VP, _SZ, _PS,
+                                                       ctypes.c_int, _VP, _VP, _VP]
+            for name in ("oal_prefill_host_workspace_bytes", "oal_prefill_host"):
+                getattr(L, name).restype = ctypes.c_int
             L.oal_set_decode_variant.argtypes = [ctypes.c_int]
             L.oal_set_decode_variant.restype = ctypes.c_int
             L.oal_profile_enable.argtypes = [ctypes.c_int]
@@ -346,6 +352,47 @@ def alloc_prefill_buffers(q, k, v, group_id, L, G, chunk, device="cuda"):
     dstate = torch.empty(state_bytes(shape), dtype=torch.uint8, device=device)
     dws = empty_workspace(prefill_workspace_bytes(shape), device)
     return dq, dk, dv_, dg, dL, dG, dout, dstate, dws
+
+
+def host_prefill_buffers(q, k, v, group_id, L, G, chunk: int = 128, segments: int = 4,
+                         device="cuda") -> dict:
+    """Device memory and copy streams for prefill_from_host: group ids, L and G copied once,
+    the state, the oal_prefill_host workspace, and two copy streams."""
+    shape = _shape_of(q, k, v, chunk)
+    n = _SZ(0)
+    _check(lib().oal_prefill_host_workspace_bytes(ctypes.byref(shape), int(segments),
+                                                  ctypes.byref(n)),
+           "oal_prefill_host_workspace_bytes")
+    return dict(
+        g=group_id.to(device=device, dtype=torch.int32).contiguous(),
+        L=L.to(device=device, dtype=torch.float32).contiguous(),
+        G=G.to(device=device, dtype=torch.int32).contiguous(),
+        state=torch.empty(state_bytes(shape), dtype=torch.uint8, device=device),
+        ws=empty_workspace(n.value, device), chunk=int(chunk), segments=int(segments),
+        copy_in=torch.cuda.Stream(device=device), copy_out=torch.cuda.Stream(device=device))
+
+
+def prefill_from_host(q, k, v, eps: float, bufs: dict, out_host=None, stream=None):
+    """oal_prefill_host: q/k/v in (pinned) host memory, yhat back into host memory, with the
+    copies of one segment overlapped with the kernels of the next.  ``bufs`` comes from
+    host_prefill_buffers; the state ends in bufs["state"].  Returns the host output tensor,
+    valid once ``stream`` (default: the current stream) is synchronised."""
+    for t in (q, k, v):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous host tensors")
+    shape = _shape_of(q, k, v, bufs["chunk"])
+    if out_host is None:
+        out_host = torch.empty(q.shape[0], q.shape[1], q.shape[2], v.shape[3],
+                               dtype=torch.float32, pin_memory=True)
+    ws = bufs["ws"]
+    rc = lib().oal_prefill_host(_ptr(q), _ptr(k), _ptr(v), _ptr(bufs["g"]), _ptr(bufs["L"]),
+                                _ptr(bufs["G"]), float(eps), _ptr(out_host),
+                                _ptr(bufs["state"]), _ptr(ws), ws.numel() * ws.element_size(),
+                                ctypes.byref(shape), bufs["segments"], _stream(stream),
+                                ctypes.c_void_p(bufs["copy_in"].cuda_stream),
+                                ctypes.c_void_p(bufs["copy_out"].cuda_stream))
+    _check(rc, "oal_prefill_host")
+    return out_host
 
 
 def launch_count() -> int:

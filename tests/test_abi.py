@@ -104,3 +104,54 @@ def test_decode_variant_switch():
         assert oal.set_decode_variant(0) == 1
     finally:
         oal.set_decode_variant(prev)
+
+
+def _host_ws(L, s, segments):
+    n = ctypes.c_size_t(0)
+    rc = L.oal_prefill_host_workspace_bytes(ctypes.byref(s), segments, ctypes.byref(n))
+    return rc, n.value
+
+
+def _align256(x):
+    return (x + 255) // 256 * 256
+
+
+@pytest.mark.parametrize("T,segments", [(4096, 4), (300, 4), (128, 3), (1000, 1), (0, 2)])
+def test_prefill_host_workspace_layout(L, T, segments):
+    """Staging for q, k, v (bf16) and yhat (fp32) of the whole call, then the prefill
+    workspace of the longest segment: segments are whole chunks of 128 tokens."""
+    B, Hq, Hkv = 2, 14, 2
+    s = oal.make_shape(B, T, Hq, Hkv, 128, oal.OAL_BF16)
+    rc, n = _host_ws(L, s, segments)
+    assert rc == 0
+    seg_len = 0 if T == 0 else -(-(-(-T // segments)) // 128) * 128
+    seg = oal.make_shape(B, seg_len, Hq, Hkv, 128, oal.OAL_BF16)
+    pws = oal.prefill_workspace_bytes(seg)
+    staging = (_align256(B * Hq * T * 64 * 2) + 2 * _align256(B * Hkv * T * 64 * 2)
+               + _align256(B * Hq * T * 64 * 4))
+    assert n == staging + _align256(pws)
+
+
+def test_prefill_host_side_argument_errors(L):
+    s = oal.make_shape(1, 512, 2, 1, 128, oal.OAL_BF16)
+    assert _host_ws(L, s, 0)[0] == -2                      # segments < 1
+    f32 = oal.make_shape(1, 512, 2, 1, 128, oal.OAL_F32)
+    assert _host_ws(L, f32, 2)[0] == -3                    # no continuation off the tc path
+    assert _host_ws(L, f32, 1)[0] == 0
+    assert L.oal_prefill_host_workspace_bytes(ctypes.byref(s), 2, None) == -1
+    rc, need = _host_ws(L, s, 2)
+    P = _fake(1 << 20)
+    args = [P, P, P, P, P, P, ctypes.c_float(1e-6), P, P, _fake(1 << 24),
+            ctypes.c_size_t(need), ctypes.byref(s), 2, None, None, None]
+    bad = list(args)
+    bad[8] = None                                           # no state
+    assert L.oal_prefill_host(*bad) == -1
+    small = list(args)
+    small[10] = ctypes.c_size_t(need - 1)
+    assert L.oal_prefill_host(*small) == -8
+    mis = list(args)
+    mis[9] = _fake((1 << 24) + 16)                          # workspace not 256-aligned
+    assert L.oal_prefill_host(*mis) == -4
+    nohost = list(args)
+    nohost[0] = None
+    assert L.oal_prefill_host(*nohost) == -1

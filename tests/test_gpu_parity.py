@@ -366,3 +366,25 @@ def test_state_only_prefill(oal, cuda, dtype, chunk):
     # defined bytes: header fields (0..44), coefficient tables and prefix states (256..)
     assert torch.equal(full[:44], alone[:44])
     assert torch.equal(full[256:], alone[256:])
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("T,segments,B", [(1000, 4, 2), (512, 2, 1), (130, 4, 1), (256, 1, 2)])
+def test_prefill_from_host_buffers(oal, cuda, T, segments, B):
+    """oal_prefill_host: host q/k/v, segments copied in and yhat copied out on their own
+    streams while the next segment computes.  Chunk-aligned segments continue the prefix
+    scan in one prefill's order, so yhat and the state equal a device-resident oal_prefill
+    bit for bit; both match the oracle."""
+    p = I.small_layer(900 + T, B=B, T=T, Hq=14, Hkv=2, dtype="bf16")
+    q, k, v, g, L, G = dev_inputs(p, cuda)
+    ref_out, ref_state = oal.prefill(q, k, v, g, L, G, p.eps, 128)
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    bufs = oal.host_prefill_buffers(hq, hk, hv, g, L, G, 128, segments, device=cuda)
+    hout = oal.prefill_from_host(hq, hk, hv, p.eps, bufs)
+    torch.cuda.synchronize()
+    assert oal.device_error() == 0
+    assert torch.equal(hout, ref_out.cpu())
+    st, rs = bufs["state"], ref_state
+    assert torch.equal(st[:44], rs[:44]) and torch.equal(st[256:], rs[256:])
+    ref = oracle.recurrent(p.q, p.k, p.v, p.group_id, p.L, p.G, p.eps)
+    assert row_rel_err(hout.numpy(), ref) <= TOL_BF16
