@@ -68,8 +68,6 @@ def parse():
                          "outside the timed events")
     ap.add_argument("--e2e-segments", type=int, default=4,
                     help="segments of the e2e host-buffer prefill (copies overlap kernels)")
-    ap.add_argument("--decode-variant", type=int, default=0, choices=[0, 1],
-                    help="decode kernel: 0 register-batched rows, 1 bulk-copied state slabs")
     ap.add_argument("--workload", default="config1", choices=["config1", "config3_16k",
                                                               "config3_32k", "config3_64k"],
                     help="prefill workload (config1 is the headline)")
@@ -272,7 +270,6 @@ def main():
     pk, pk_kind = peaks()
     oal.lib()
     oal.set_prefill_overlap(not args.no_overlap)
-    oal.set_decode_variant(args.decode_variant)
 
     p, desc = workload(args.workload)
     B, Hq, T, _ = p.q.shape
@@ -478,7 +475,7 @@ def run_decode(args, dev, torch, oal, pk, pk_kind, flush, world, barrier):
     ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world, dev)
     state_bytes = 2.0 * B * Hkv * F * W * 4   # every packed row read and written once
     io_bytes = B * (Hq + 2 * Hkv) * 64 * 2 + B * Hq * 64 * 4
-    kname = "decode_bulk" if args.decode_variant == 1 else "decode"
+    kname = "decode"
     kern = prof.get(kname)
     roof = None
     if kern:

@@ -228,14 +228,6 @@ int oal_prefill_host(const void* q_host, const void* k_host, const void* v_host,
                      const oal_shape* s, int segments, void* stream, void* copy_in,
                      void* copy_out);
 
-/* Decode kernel (oal_decode_step and oal_decode_step_noalloc).  0 (default): each thread
- * keeps a batch of state rows in flight in registers.  1: each block streams its whole state
- * slab into shared memory with bulk copies (cp.async.bulk) issued before it forms the feature
- * weights.  Both use the same partition, workspace and summation order, so the results are
- * identical.  Process-wide; returns the previous setting, or OAL_ERR_UNSUPPORTED (setting
- * unchanged) for any other value. */
-int oal_set_decode_variant(int variant);
-
 /* Reads the device-side error word (OAL_OK or a negative oal_status set by a kernel since
  * the last read), synchronising `stream`, and clears it. */
 int oal_device_error(int* code, void* stream);

@@ -183,7 +183,7 @@ int oal_decode_step(const void* q, const void* k, const void* v, void* state, fl
     if (!workspace || workspace_bytes < need) return OAL_ERR_WORKSPACE;
     if (!aligned16(workspace)) return OAL_ERR_ALIGN;
     unsigned char* ws = static_cast<unsigned char*>(workspace);
-    return launch_decode_selected(q, k, v, state, out,
+    return launch_decode(q, k, v, state, out,
                          reinterpret_cast<float*>(ws + decode_ticket_bytes(s)),
                          reinterpret_cast<unsigned int*>(ws), s->B, s->Hq, s->Hkv, s->dtype,
                          static_cast<cudaStream_t>(stream));
@@ -218,12 +218,6 @@ int oal_contribution_stat(const void* q, const void* k, float* chi, const oal_sh
 unsigned long long oal_launch_count(void) { return tracer().launches.load(); }
 
 int oal_set_prefill_overlap(int overlap) { return g_prefill_overlap.exchange(overlap ? 1 : 0); }
-
-int oal_set_decode_variant(int variant)
-{
-    if (variant != 0 && variant != 1) return OAL_ERR_UNSUPPORTED;
-    return set_decode_variant(variant);
-}
 
 int oal_profile_enable(int on)
 {

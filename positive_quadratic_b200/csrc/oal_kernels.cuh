@@ -25,18 +25,6 @@ int launch_decode(const void* q, const void* k, const void* v, void* state, floa
                   float* part, unsigned int* tickets, int B, int Hq, int Hkv, int dtype,
                   cudaStream_t st);
 
-// the same step with each state slab streamed into shared memory by bulk copies
-// (oal_decode_bulk.cu); identical results, same workspace
-int launch_decode_bulk(const void* q, const void* k, const void* v, void* state, float* out,
-                       float* part, unsigned int* tickets, int B, int Hq, int Hkv, int dtype,
-                       cudaStream_t st);
-
-// the decode kernel chosen by oal_set_decode_variant
-int launch_decode_selected(const void* q, const void* k, const void* v, void* state, float* out,
-                           float* part, unsigned int* tickets, int B, int Hq, int Hkv,
-                           int dtype, cudaStream_t st);
-int set_decode_variant(int variant);
-
 int read_device_error(int* code, cudaStream_t st);
 
 // tensor-core (tcgen05) bf16 prefill, chunk 128

@@ -3,7 +3,6 @@
 #include "oal_common.cuh"
 #include "oal_simt.cu"
 #include "oal_tc.cu"
-#include "oal_decode_bulk.cu"
 #include "oal_api.cu"
 #include "oal_host.cu"
 #include "oal_noalloc.cu"

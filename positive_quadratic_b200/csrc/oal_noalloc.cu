@@ -66,7 +66,7 @@ extern "C" int oal_decode_step_noalloc(const void* q, const void* k, const void*
     unsigned char* ws = static_cast<unsigned char*>(scratch);
     // The array keeps whatever the previous call left; the tickets must start at zero.
     OAL_CUDA_TRY(cudaMemsetAsync(ws, 0, decode_ticket_bytes(s), st));
-    return launch_decode_selected(q, k, v, state, out,
+    return launch_decode(q, k, v, state, out,
                          reinterpret_cast<float*>(ws + decode_ticket_bytes(s)),
                          reinterpret_cast<unsigned int*>(ws), s->B, s->Hq, s->Hkv, s->dtype, st);
 }

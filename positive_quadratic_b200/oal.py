@@ -84,8 +84,6 @@ def lib() -> ctypes.CDLL:
                                                        ctypes.c_int, _VP, _VP, _VP]
             for name in ("oal_prefill_host_workspace_bytes", "oal_prefill_host"):
                 getattr(L, name).restype = ctypes.c_int
-            L.oal_set_decode_variant.argtypes = [ctypes.c_int]
-            L.oal_set_decode_variant.restype = ctypes.c_int
             L.oal_profile_enable.argtypes = [ctypes.c_int]
             L.oal_profile_enable.restype = ctypes.c_int
             L.oal_profile_read.argtypes = [ctypes.POINTER(KernelStat), ctypes.c_int,
@@ -417,12 +415,3 @@ def set_prefill_overlap(overlap: bool) -> bool:
     """Launch the tensor-core prefill's scan and readout kernels as programmatic dependents
     (True) or in plain stream order (False); returns the previous setting."""
     return bool(lib().oal_set_prefill_overlap(1 if overlap else 0))
-
-
-def set_decode_variant(variant: int) -> int:
-    """Decode kernel: 0 keeps state rows in flight in registers (default), 1 streams each
-    state slab into shared memory with bulk copies.  Identical results; returns the previous
-    setting."""
-    rc = lib().oal_set_decode_variant(int(variant))
-    _check(min(rc, 0), "oal_set_decode_variant")
-    return rc

@@ -92,20 +92,6 @@ def test_header_packed_order_is_complete():
     assert all(r <= t for r, t in p)
 
 
-def test_decode_variant_switch():
-    """The decode-kernel switch is host state only: it accepts 0 and 1, returns the previous
-    value and refuses anything else without changing the setting."""
-    prev = oal.set_decode_variant(1)
-    try:
-        assert prev == 0
-        assert oal.set_decode_variant(1) == 1
-        with pytest.raises(oal.OALError):
-            oal.set_decode_variant(2)
-        assert oal.set_decode_variant(0) == 1
-    finally:
-        oal.set_decode_variant(prev)
-
-
 def _host_ws(L, s, segments):
     n = ctypes.c_size_t(0)
     rc = L.oal_prefill_host_workspace_bytes(ctypes.byref(s), segments, ctypes.byref(n))
