@@ -351,8 +351,9 @@ def main():
         hk = k.cpu().pin_memory()
         hv = v.cpu().pin_memory()
         hout = torch.empty(out.shape, dtype=torch.float32, pin_memory=True)
-        bufs = oal.host_prefill_buffers(hq, hk, hv, g, L, G, args.chunk, args.e2e_segments,
-                                        device=dev)
+        # segments continue the prefix, which only the tensor-core path (chunk 128) does
+        nseg = args.e2e_segments if args.chunk == 128 else 1
+        bufs = oal.host_prefill_buffers(hq, hk, hv, g, L, G, args.chunk, nseg, device=dev)
         oal.prefill_from_host(hq, hk, hv, p.eps, bufs, hout)
         torch.cuda.synchronize()
         # the segmented call must reproduce the device-resident prefill exactly
@@ -375,10 +376,10 @@ def main():
         assert oal.device_error() == 0
         e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs2), world, dev)
         e2e = {"value": job_rate(world, args.steps * B * T, e_ms), "unit": UNIT,
-               "h2d_bytes_per_step": int(hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2),
+               "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in (hq, hk, hv))),
                "d2h_bytes_per_step": int(hout.numel() * 4),
                "api": "oal_prefill_host",
-               "segments": bufs["segments"] if same else 1,
+               "segments": bufs["segments"],
                "segmented_matches_device_prefill": same}
 
     # ---- decode ----
