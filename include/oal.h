@@ -18,8 +18,9 @@
  *
  * Conventions for every entry point:
  *  - All tensor arguments are DEVICE pointers to contiguous row-major arrays, allocated and
- *    owned by the caller (for example through PyTorch).  The library allocates no device
- *    memory and keeps no pointer after a call returns.
+ *    owned by the caller (for example through PyTorch), except the *_host arrays of
+ *    oal_prefill_host, which are host memory.  The library allocates no device memory and
+ *    keeps no pointer after a call returns.
  *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL = legacy
  *    default stream).  A return of OAL_OK means the work was validated and enqueued.
  *  - Return value: OAL_OK (0) or a negative oal_status.  Nothing aborts or throws.  Argument
@@ -99,7 +100,8 @@ typedef struct {
  * s_r = 1/sqrt(dh) for r < 64, s_64 = 1, plus eps on f = 2144; u = sum_f coef[h][f] *
  * qhat_r qhat_t * (Hv | z)[f].  The header holds magic 0x534C414F ("OALS"), the ABI version,
  * B, Hq, Hkv, dh, dv, OAL_FEATURES_PAD (int32 each), the token count (int64 at byte 32) and
- * eps (fp32 at byte 40).  The buffer is the resumable artifact of a sequence: copying it
+ * eps (fp32 at byte 40); bytes 44..255 are zero.  The buffer is the resumable artifact of
+ * a sequence: copying it
  * saves the sequence, copying it back resumes it. */
 int oal_state_bytes(const oal_shape* s, size_t* bytes);
 
