@@ -101,8 +101,7 @@ typedef struct {
  * qhat_r qhat_t * (Hv | z)[f].  The header holds magic 0x534C414F ("OALS"), the ABI version,
  * B, Hq, Hkv, dh, dv, OAL_FEATURES_PAD (int32 each), the token count (int64 at byte 32) and
  * eps (fp32 at byte 40); bytes 44..255 are zero.  The buffer is the resumable artifact of
- * a sequence: copying it
- * saves the sequence, copying it back resumes it. */
+ * a sequence: copying it saves the sequence, copying it back resumes it. */
 int oal_state_bytes(const oal_shape* s, size_t* bytes);
 
 /* Scratch needed by oal_prefill for `s` (all fields used).  The contents need no
