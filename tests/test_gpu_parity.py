@@ -231,6 +231,30 @@ def test_decode_continuation(oal, cuda, dtype):
     assert np.max(np.abs(S[:, :, :F] - ref) / np.abs(ref).max(axis=2, keepdims=True)) < 1e-5
 
 
+@pytest.mark.parametrize("Hq,Hkv,dtype", [(2, 2, "bf16"), (6, 2, "bf16"), (5, 1, "bf16"),
+                                           (8, 1, "bf16"), (8, 1, "f32")])
+def test_decode_group_sizes(oal, cuda, Hq, Hkv, dtype):
+    """Decode for every query-heads-per-kv-head count the kernel is specialised on that the
+    Qwen shape does not reach (1, 3, 5, 8): three steps after a ragged prefill."""
+    B, T0, n = 2, 150, 3
+    p = I.small_layer(320 + 10 * Hq + Hkv, B=B, T=T0 + n, Hq=Hq, Hkv=Hkv, dtype=dtype)
+    y_all, st_all = oracle.recurrent(p.q, p.k, p.v, p.group_id, p.L, p.G, p.eps,
+                                     return_state=True)
+    _, state = gpu_prefill(oal, p.slice_tokens(0, T0), cuda, 128)
+    ws = oal.decode_workspace(B, Hq, Hkv, cuda)
+    q, k, v, _, _, _ = dev_inputs(p, cuda)
+    for t in range(T0, T0 + n):
+        sl = lambda x: x[:, :, t:t + 1].contiguous()  # noqa: E731
+        y = oal.decode_step(sl(q), sl(k), sl(v), state, ws)
+        torch.cuda.synchronize()
+        assert row_rel_err(y.cpu().numpy()[:, :, 0], y_all[:, :, t]) <= tol(p)
+    assert oal.device_error() == 0
+    hdr, _, S = read_state(state.cpu().numpy(), B, Hq, Hkv)
+    assert hdr["tokens"] == T0 + n
+    ref = pack_oracle_state(st_all)
+    assert np.max(np.abs(S[:, :, :F] - ref) / np.abs(ref).max(axis=2, keepdims=True)) < 1e-5
+
+
 def test_chunk_size_independence(oal, cuda):
     p = I.small_layer(308, B=1, T=1000, Hq=4, Hkv=2, dtype="f32")
     ys = [gpu_prefill(oal, p, cuda, c)[0] for c in (64, 128, 256)]
