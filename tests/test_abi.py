@@ -141,3 +141,41 @@ def test_prefill_host_side_argument_errors(L):
     nohost = list(args)
     nohost[0] = None
     assert L.oal_prefill_host(*nohost) == -1
+
+
+def test_header_compiles_as_c_and_links(tmp_path):
+    """include/oal.h is plain C: a C99 program includes it, links liboal.so and calls the
+    host-only entry points (no GPU needed)."""
+    import os
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no gcc")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    libdir = os.path.dirname(build.build())
+    src = tmp_path / "abi.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <string.h>
+#include "oal.h"
+int main(void) {
+    oal_shape s = {1, 4096, 14, 2, OAL_HEAD_DIM, OAL_VALUE_DIM, 128, OAL_BF16};
+    size_t n = 0;
+    if (oal_abi_version() != OAL_ABI_VERSION) return 1;
+    if (oal_state_bytes(&s, &n) != OAL_OK || n == 0) return 2;
+    if (oal_prefill_workspace_bytes(&s, &n) != OAL_OK || n == 0) return 3;
+    if (oal_prefill_host_workspace_bytes(&s, 4, &n) != OAL_OK || n == 0) return 4;
+    s.chunk = 96;
+    if (oal_prefill_workspace_bytes(&s, &n) != OAL_ERR_UNSUPPORTED) return 5;
+    if (strlen(oal_status_string(OAL_ERR_ALIGN)) == 0) return 6;
+    printf("ok\n");
+    return 0;
+}
+''')
+    exe = tmp_path / "abi"
+    subprocess.check_call([gcc, "-std=c99", "-Wall", "-Werror", "-pedantic",
+                           "-I", os.path.join(root, "include"), str(src), "-o", str(exe),
+                           "-L", libdir, "-loal", "-Wl,-rpath," + libdir])
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
