@@ -198,6 +198,27 @@ int oal_contribution_stat(const void* q, const void* k, float* chi, const oal_sh
  * results.  Process-wide; returns the previous setting. */
 int oal_set_prefill_overlap(int overlap);
 
+/* Prefill with the ungrouped Hadamard form: eq. (5) with free coefficients, that is
+ *   kappa(q, k) = a + sum_r b_r x_r + sum_{r,t} C_rt x_r x_t,   x_r = q_r k_r / sqrt(d_h),
+ * the relaxation of the Taylor kernel's shared coefficients that the abstract of arXiv
+ * 2610.13674 describes (the grouped kernel of eq. (3) is the case a = eps + M_00,
+ * b_r = 2 M_{0,g(r)}, C_rt = M_{g(r),g(t)}).  a [Hq], b [Hq][64], C [Hq][64][64] (row r,
+ * column t) fp32 device arrays, 16-byte aligned; only the symmetric part of C matters.  The
+ * kernel need not be positive: yhat = u[:dv] / u[dv] is a plain IEEE division.
+ * Runs on CUDA cores in fp32 for both dtypes and every chunk size; the intra-chunk part costs
+ * O(T * chunk * d_h^2).  Other arguments, the state (eps = 0 in its header; a holds the
+ * constant), the workspace (oal_prefill_workspace_bytes) and errors as oal_prefill.
+ * oal_decode_step continues the sequence. */
+int oal_prefill_hadamard(const void* q, const void* k, const void* v, const float* a,
+                         const float* b, const float* C, float* out, void* state,
+                         void* workspace, size_t workspace_bytes, const oal_shape* s,
+                         void* stream);
+
+/* The dense O(T^2) form of the same kernel (causal, j <= i), fp32 on CUDA cores. */
+int oal_dense_hadamard_gpu(const void* q, const void* k, const void* v, const float* a,
+                           const float* b, const float* C, float* out, const oal_shape* s,
+                           void* stream);
+
 /* Scratch needed by oal_prefill_host for `s` cut into `segments` segments: device staging
  * for q, k, v and yhat of the whole call plus the prefill workspace of the longest segment. */
 int oal_prefill_host_workspace_bytes(const oal_shape* s, int segments, size_t* bytes);

@@ -25,6 +25,11 @@ int launch_decode(const void* q, const void* k, const void* v, void* state, floa
                   float* part, unsigned int* tickets, int B, int Hq, int Hkv, int dtype,
                   cudaStream_t st);
 
+// ungrouped Hadamard form (oal_hadamard.cu): prefill on CUDA cores, or the dense O(T^2) form
+int launch_hadamard(const void* q, const void* k, const void* v, const float* a, const float* b,
+                    const float* C, float* out, void* state, float* Hc, int B, int T, int Hq,
+                    int Hkv, int Cn, int dtype, bool dense, cudaStream_t st);
+
 int read_device_error(int* code, cudaStream_t st);
 
 // tensor-core (tcgen05) bf16 prefill, chunk 128

@@ -82,7 +82,10 @@ def lib() -> ctypes.CDLL:
                                                            ctypes.POINTER(_SZ)]
             L.oal_prefill_host.argtypes = [_VP] * 6 + [ctypes.c_float, _VP, _VP, _VP, _SZ, _PS,
                                                        ctypes.c_int, _VP, _VP, _VP]
-            for name in ("oal_prefill_host_workspace_bytes", "oal_prefill_host"):
+            L.oal_prefill_hadamard.argtypes = [_VP] * 7 + [_VP, _VP, _SZ, _PS, _VP]
+            L.oal_dense_hadamard_gpu.argtypes = [_VP] * 7 + [_PS, _VP]
+            for name in ("oal_prefill_host_workspace_bytes", "oal_prefill_host",
+                         "oal_prefill_hadamard", "oal_dense_hadamard_gpu"):
                 getattr(L, name).restype = ctypes.c_int
             L.oal_profile_enable.argtypes = [ctypes.c_int]
             L.oal_profile_enable.restype = ctypes.c_int
@@ -391,6 +394,52 @@ def prefill_from_host(q, k, v, eps: float, bufs: dict, out_host=None, stream=Non
                                 ctypes.c_void_p(bufs["copy_out"].cuda_stream))
     _check(rc, "oal_prefill_host")
     return out_host
+
+
+def _hadamard_coefs(q, a, b, C):
+    Hq = q.shape[1]
+    a, b, C = (t.to(device=q.device, dtype=torch.float32).contiguous() for t in (a, b, C))
+    if a.shape != (Hq,) or b.shape != (Hq, HEAD_DIM) or C.shape != (Hq, HEAD_DIM, HEAD_DIM):
+        raise ValueError("a [Hq], b [Hq, 64], C [Hq, 64, 64] expected")
+    return a, b, C
+
+
+def prefill_hadamard(q, k, v, a, b, C, chunk: int = 64, out=None, state=None, workspace=None,
+                     stream=None):
+    """oal_prefill_hadamard: causal prefill with kappa = a + b.x + x^T C x, x = q*k/sqrt(64)
+    (per query head a [Hq], b [Hq, 64], C [Hq, 64, 64]).  Returns (out, state); the state
+    continues with decode_step."""
+    shape = _shape_of(q, k, v, chunk)
+    dev = q.device
+    a, b, C = _hadamard_coefs(q, a, b, C)
+    if out is None:
+        out = torch.empty(q.shape[0], q.shape[1], q.shape[2], v.shape[3], dtype=torch.float32,
+                          device=dev)
+    if state is None:
+        state = torch.empty(state_bytes(shape), dtype=torch.uint8, device=dev)
+    if workspace is None:
+        workspace = empty_workspace(prefill_workspace_bytes(shape), dev)
+    _contig_cuda(q, k, v, a, b, C, out, state, workspace)
+    rc = lib().oal_prefill_hadamard(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(C),
+                                    _ptr(out), _ptr(state), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(),
+                                    ctypes.byref(shape), _stream(stream))
+    _check(rc, "oal_prefill_hadamard")
+    return out, state
+
+
+def dense_hadamard(q, k, v, a, b, C, out=None, stream=None):
+    """oal_dense_hadamard_gpu: the O(T^2) causal form of the same kernel."""
+    shape = _shape_of(q, k, v, 64)
+    a, b, C = _hadamard_coefs(q, a, b, C)
+    if out is None:
+        out = torch.empty(q.shape[0], q.shape[1], q.shape[2], v.shape[3], dtype=torch.float32,
+                          device=q.device)
+    _contig_cuda(q, k, v, a, b, C, out)
+    rc = lib().oal_dense_hadamard_gpu(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(C),
+                                      _ptr(out), ctypes.byref(shape), _stream(stream))
+    _check(rc, "oal_dense_hadamard_gpu")
+    return out
 
 
 def launch_count() -> int:

@@ -179,3 +179,24 @@ int main(void) {
                            "-L", libdir, "-loal", "-Wl,-rpath," + libdir])
     r = subprocess.run([str(exe)], capture_output=True, text=True)
     assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
+
+
+def test_hadamard_host_side_errors(L):
+    s = oal.make_shape(1, 256, 2, 1, 64, oal.OAL_F32)
+    P = _fake(1 << 20)
+    ws = ctypes.c_size_t(1 << 40)
+    # q, k, v, a, b, C, out, state, workspace, bytes, shape, stream
+    args = [P] * 9 + [ws, ctypes.byref(s), None]
+    for i in (3, 4, 5, 7):                       # a, b, C, state
+        bad = list(args)
+        bad[i] = None
+        assert L.oal_prefill_hadamard(*bad) == -1
+    mis = list(args)
+    mis[5] = _fake((1 << 20) + 8)                # C not 16-byte aligned
+    assert L.oal_prefill_hadamard(*mis) == -4
+    small = list(args)
+    small[9] = ctypes.c_size_t(16)
+    assert L.oal_prefill_hadamard(*small) == -8
+    odd = oal.make_shape(1, 256, 2, 1, 96, oal.OAL_F32)
+    assert L.oal_prefill_hadamard(*args[:10], ctypes.byref(odd), None) == -3
+    assert L.oal_dense_hadamard_gpu(P, P, P, None, P, P, P, ctypes.byref(s), None) == -1
