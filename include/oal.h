@@ -250,6 +250,30 @@ int oal_prefill_host(const void* q_host, const void* k_host, const void* v_host,
                      const oal_shape* s, int segments, void* stream, void* copy_in,
                      void* copy_out);
 
+/* Scratch needed by oal_prefill_varlen: n_streams slices of oal_prefill_workspace_bytes for
+ * the longest sequence, each rounded up to 256 bytes.  seq_lens is host memory. */
+int oal_prefill_varlen_workspace_bytes(const oal_shape* s, const int32_t* seq_lens, int n_seq,
+                                       int n_streams, size_t* bytes);
+
+/* Prefill of n_seq independent sequences of different lengths, packed back to back
+ * (a variable-length batch).  seq_lens [n_seq] (host int32, each >= 0) gives T_i; with
+ * o_i = T_0 + ... + T_{i-1}, sequence i is the B = 1 problem whose q block [Hq][T_i][dh]
+ * starts at element o_i*Hq*dh of q, k and v blocks [Hkv][T_i][dh|dv] at o_i*Hkv*dh, and out
+ * block [Hq][T_i][dv] (fp32) at o_i*Hq*dv.  Its state is written at states + i*state_stride
+ * (state_stride: a multiple of 256, at least oal_state_bytes for B = 1).  Every sequence is
+ * exactly an oal_prefill of its block; s gives Hq, Hkv, dh, dv, chunk and dtype (B and T are
+ * ignored).  streams [n_streams] (host array of caller-owned streams): sequence i runs on
+ * streams[i % n_streams] with workspace slice i % n_streams, so short sequences overlap.  The
+ * work is ordered after earlier work on streams[0], and later work on streams[0] is ordered
+ * after every sequence.  workspace: oal_prefill_varlen_workspace_bytes, 256-byte aligned.
+ * Errors: as oal_prefill, OAL_ERR_SHAPE for a negative length, n_streams < 1 or a bad
+ * stride. */
+int oal_prefill_varlen(const void* q, const void* k, const void* v, const int32_t* group_id,
+                       const float* L, const int32_t* G, float eps, float* out, void* states,
+                       size_t state_stride, void* workspace, size_t workspace_bytes,
+                       const oal_shape* s, const int32_t* seq_lens, int n_seq,
+                       void* const* streams, int n_streams);
+
 /* Reads the device-side error word (OAL_OK or a negative oal_status set by a kernel since
  * the last read), synchronising `stream`, and clears it. */
 int oal_device_error(int* code, void* stream);

@@ -6,5 +6,6 @@
 #include "oal_api.cu"
 #include "oal_host.cu"
 #include "oal_hadamard.cu"
+#include "oal_varlen.cu"
 #include "oal_noalloc.cu"
 #include "oal_chi.cu"

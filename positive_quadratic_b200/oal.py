@@ -84,8 +84,14 @@ def lib() -> ctypes.CDLL:
                                                        ctypes.c_int, _VP, _VP, _VP]
             L.oal_prefill_hadamard.argtypes = [_VP] * 7 + [_VP, _VP, _SZ, _PS, _VP]
             L.oal_dense_hadamard_gpu.argtypes = [_VP] * 7 + [_PS, _VP]
+            L.oal_prefill_varlen_workspace_bytes.argtypes = [_PS, _VP, ctypes.c_int,
+                                                             ctypes.c_int, ctypes.POINTER(_SZ)]
+            L.oal_prefill_varlen.argtypes = [_VP] * 6 + [ctypes.c_float, _VP, _VP, _SZ, _VP,
+                                                         _SZ, _PS, _VP, ctypes.c_int, _VP,
+                                                         ctypes.c_int]
             for name in ("oal_prefill_host_workspace_bytes", "oal_prefill_host",
-                         "oal_prefill_hadamard", "oal_dense_hadamard_gpu"):
+                         "oal_prefill_hadamard", "oal_dense_hadamard_gpu",
+                         "oal_prefill_varlen_workspace_bytes", "oal_prefill_varlen"):
                 getattr(L, name).restype = ctypes.c_int
             L.oal_profile_enable.argtypes = [ctypes.c_int]
             L.oal_profile_enable.restype = ctypes.c_int
@@ -440,6 +446,53 @@ def dense_hadamard(q, k, v, a, b, C, out=None, stream=None):
                                       _ptr(out), ctypes.byref(shape), _stream(stream))
     _check(rc, "oal_dense_hadamard_gpu")
     return out
+
+
+def prefill_varlen(qs, ks, vs, group_id, L, G, eps: float, chunk: int = 128, streams=None,
+                   states=None, workspace=None):
+    """oal_prefill_varlen over a list of sequences: qs[i] [Hq, T_i, 64], ks[i] / vs[i]
+    [Hkv, T_i, 64] (same dtype and device).  The blocks are packed back to back into one
+    buffer per tensor (the layout the call reads).  Returns (outs, states): outs[i] [Hq, T_i,
+    64] fp32, states [n, stride] uint8 with row i the state of sequence i (continue it with
+    decode_step).  ``streams`` (torch streams) run sequences side by side; default: the
+    current stream alone."""
+    n = len(qs)
+    if not (len(ks) == len(vs) == n) or n == 0:
+        raise ValueError("qs, ks, vs: equal, non-zero numbers of sequences")
+    seq = [int(t.shape[1]) for t in qs]
+    Hq, Hkv, dev = qs[0].shape[0], ks[0].shape[0], qs[0].device
+    pack = lambda ts: torch.cat([t.contiguous().reshape(-1) for t in ts])  # noqa: E731
+    q, k, v = pack(qs), pack(ks), pack(vs)
+    shape = make_shape(1, max(seq), Hq, Hkv, chunk, _dtype_code(q), qs[0].shape[-1],
+                       vs[0].shape[-1])
+    lens = (ctypes.c_int32 * n)(*seq)
+    if streams is None:
+        streams = [torch.cuda.current_stream(dev)]
+    handles = (ctypes.c_void_p * len(streams))(*[st.cuda_stream for st in streams])
+    nb = _SZ(0)
+    _check(lib().oal_prefill_varlen_workspace_bytes(ctypes.byref(shape), lens, n, len(streams),
+                                                    ctypes.byref(nb)),
+           "oal_prefill_varlen_workspace_bytes")
+    stride = (state_bytes(make_shape(1, 1, Hq, Hkv, chunk, _dtype_code(q))) + 255) // 256 * 256
+    out = torch.empty(Hq * sum(seq) * vs[0].shape[-1], dtype=torch.float32, device=dev)
+    if states is None:
+        states = torch.empty(n, stride, dtype=torch.uint8, device=dev)
+    if workspace is None:
+        workspace = empty_workspace(nb.value, dev)
+    _contig_cuda(q, k, v, group_id, L, G, out, states, workspace)
+    cur = torch.cuda.current_stream(dev)
+    streams[0].wait_stream(cur)  # the packed inputs were written on the current stream
+    rc = lib().oal_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(group_id), _ptr(L), _ptr(G),
+                                  float(eps), _ptr(out), _ptr(states), stride, _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(),
+                                  ctypes.byref(shape), lens, n, handles, len(streams))
+    _check(rc, "oal_prefill_varlen")
+    cur.wait_stream(streams[0])  # streams[0] already waits for every other stream
+    outs, off = [], 0
+    for t in seq:
+        outs.append(out[off * Hq * 64:(off + t) * Hq * 64].view(Hq, t, 64))
+        off += t
+    return outs, states
 
 
 def launch_count() -> int:

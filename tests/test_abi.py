@@ -200,3 +200,30 @@ def test_hadamard_host_side_errors(L):
     odd = oal.make_shape(1, 256, 2, 1, 96, oal.OAL_F32)
     assert L.oal_prefill_hadamard(*args[:10], ctypes.byref(odd), None) == -3
     assert L.oal_dense_hadamard_gpu(P, P, P, None, P, P, P, ctypes.byref(s), None) == -1
+
+
+def test_varlen_host_side_errors(L):
+    s = oal.make_shape(1, 0, 4, 2, 128, oal.OAL_BF16)
+    lens = (ctypes.c_int32 * 3)(100, 0, 300)
+    n = ctypes.c_size_t(0)
+    assert L.oal_prefill_varlen_workspace_bytes(ctypes.byref(s), lens, 3, 2, ctypes.byref(n)) == 0
+    one = oal.make_shape(1, 300, 4, 2, 128, oal.OAL_BF16)
+    assert n.value == 2 * ((oal.prefill_workspace_bytes(one) + 255) // 256 * 256)
+    bad = (ctypes.c_int32 * 2)(5, -1)
+    assert L.oal_prefill_varlen_workspace_bytes(ctypes.byref(s), bad, 2, 1, ctypes.byref(n)) == -2
+    assert L.oal_prefill_varlen_workspace_bytes(ctypes.byref(s), lens, 3, 0, ctypes.byref(n)) == -2
+    P = _fake(1 << 20)
+    sb = (oal.state_bytes(one) + 255) // 256 * 256
+    streams = (ctypes.c_void_p * 1)(None)
+    args = [P] * 6 + [ctypes.c_float(1e-6), P, _fake(1 << 24), ctypes.c_size_t(sb),
+                      _fake(1 << 25), ctypes.c_size_t(1 << 40), ctypes.byref(s), lens, 3,
+                      streams, 1]
+    stride = list(args)
+    stride[9] = ctypes.c_size_t(sb - 256)                 # smaller than one state
+    assert L.oal_prefill_varlen(*stride) == -2
+    nost = list(args)
+    nost[8] = None
+    assert L.oal_prefill_varlen(*nost) == -1
+    mis = list(args)
+    mis[10] = _fake((1 << 25) + 16)                       # workspace not 256-aligned
+    assert L.oal_prefill_varlen(*mis) == -4
