@@ -274,6 +274,25 @@ int oal_prefill_varlen(const void* q, const void* k, const void* v, const int32_
                        const oal_shape* s, const int32_t* seq_lens, int n_seq,
                        void* const* streams, int n_streams);
 
+/* Scratch needed by oal_dense_backward_gpu for `s` (B, T, Hq used): per row of every query
+ * head its normaliser, output, partial dM (81 floats) and partial deps. */
+int oal_dense_backward_workspace_bytes(const oal_shape* s, size_t* bytes);
+
+/* Gradients of the dense causal form (eqs. (2)-(3) summed over j <= i and normalised) for
+ * the joint training of the kernel coefficients with the model.  dy = dLoss/dyhat
+ * [B][Hq][T][dv] fp32.  Outputs (fp32, device): dq [B][Hq][T][dh]; dk [B][Hkv][T][dh] and
+ * dv [B][Hkv][T][dv], summed over the query heads of each group; dL [Hq][OAL_G_MAX+1]^2,
+ * zero outside each head's leading (G+1)x(G+1) block; deps, one float (eps is shared).
+ * By the chain rule: dkappa_ij = dy_i . (v_j - yhat_i) / D_i, dkappa/dsbar = 2 M sbar,
+ * dL = (dM + dM^T) L.  Deterministic: every output is summed in a fixed order.  O(B Hq T^2
+ * dh) on CUDA cores in fp32 for both input dtypes: a reference-scale gradient.  workspace:
+ * oal_dense_backward_workspace_bytes, 256-byte aligned.  Errors as oal_prefill. */
+int oal_dense_backward_gpu(const void* q, const void* k, const void* v, const int32_t* group_id,
+                           const float* L, const int32_t* G, float eps, const float* dy,
+                           float* dq, float* dk, float* dv, float* dL, float* deps,
+                           void* workspace, size_t workspace_bytes, const oal_shape* s,
+                           void* stream);
+
 /* Reads the device-side error word (OAL_OK or a negative oal_status set by a kernel since
  * the last read), synchronising `stream`, and clears it. */
 int oal_device_error(int* code, void* stream);

@@ -7,5 +7,6 @@
 #include "oal_host.cu"
 #include "oal_hadamard.cu"
 #include "oal_varlen.cu"
+#include "oal_backward.cu"
 #include "oal_noalloc.cu"
 #include "oal_chi.cu"

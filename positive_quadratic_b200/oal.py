@@ -89,6 +89,11 @@ def lib() -> ctypes.CDLL:
             L.oal_prefill_varlen.argtypes = [_VP] * 6 + [ctypes.c_float, _VP, _VP, _SZ, _VP,
                                                          _SZ, _PS, _VP, ctypes.c_int, _VP,
                                                          ctypes.c_int]
+            L.oal_dense_backward_workspace_bytes.argtypes = [_PS, ctypes.POINTER(_SZ)]
+            L.oal_dense_backward_gpu.argtypes = [_VP] * 6 + [ctypes.c_float] + [_VP] * 7 + [
+                _SZ, _PS, _VP]
+            for name in ("oal_dense_backward_workspace_bytes", "oal_dense_backward_gpu"):
+                getattr(L, name).restype = ctypes.c_int
             for name in ("oal_prefill_host_workspace_bytes", "oal_prefill_host",
                          "oal_prefill_hadamard", "oal_dense_hadamard_gpu",
                          "oal_prefill_varlen_workspace_bytes", "oal_prefill_varlen"):
@@ -493,6 +498,31 @@ def prefill_varlen(qs, ks, vs, group_id, L, G, eps: float, chunk: int = 128, str
         outs.append(out[off * Hq * 64:(off + t) * Hq * 64].view(Hq, t, 64))
         off += t
     return outs, states
+
+
+def dense_backward(q, k, v, group_id, L, G, eps: float, dy, stream=None) -> dict:
+    """oal_dense_backward_gpu: gradients of the dense causal form for dy = dLoss/dyhat
+    [B, Hq, T, 64] fp32.  Returns dict(dq, dk, dv, dL, deps) of fp32 device tensors."""
+    shape = _shape_of(q, k, v, 64)
+    dev = q.device
+    dy = dy.to(device=dev, dtype=torch.float32).contiguous()
+    dq = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    dk = torch.empty(k.shape, dtype=torch.float32, device=dev)
+    dv_ = torch.empty(v.shape, dtype=torch.float32, device=dev)
+    dL = torch.empty(L.shape, dtype=torch.float32, device=dev)
+    deps = torch.empty(4, dtype=torch.float32, device=dev)
+    n = _SZ(0)
+    _check(lib().oal_dense_backward_workspace_bytes(ctypes.byref(shape), ctypes.byref(n)),
+           "oal_dense_backward_workspace_bytes")
+    ws = empty_workspace(n.value, dev)
+    _contig_cuda(q, k, v, group_id, L, G, dy, dq, dk, dv_, dL, deps, ws)
+    rc = lib().oal_dense_backward_gpu(_ptr(q), _ptr(k), _ptr(v), _ptr(group_id), _ptr(L),
+                                      _ptr(G), float(eps), _ptr(dy), _ptr(dq), _ptr(dk),
+                                      _ptr(dv_), _ptr(dL), _ptr(deps), _ptr(ws),
+                                      ws.numel() * ws.element_size(), ctypes.byref(shape),
+                                      _stream(stream))
+    _check(rc, "oal_dense_backward_gpu")
+    return dict(dq=dq, dk=dk, dv=dv_, dL=dL, deps=deps[0])
 
 
 def launch_count() -> int:

@@ -227,3 +227,26 @@ def test_varlen_host_side_errors(L):
     mis = list(args)
     mis[10] = _fake((1 << 25) + 16)                       # workspace not 256-aligned
     assert L.oal_prefill_varlen(*mis) == -4
+
+
+def test_dense_backward_host_side_errors(L):
+    s = oal.make_shape(1, 64, 2, 1, 128, oal.OAL_F32)
+    n = ctypes.c_size_t(0)
+    assert L.oal_dense_backward_workspace_bytes(ctypes.byref(s), ctypes.byref(n)) == 0
+    rows = 1 * 2 * 64
+    a256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    assert n.value == 2 * a256(rows * 4) + a256(rows * 64 * 4) + a256(rows * 81 * 4) + a256(8)
+    P = _fake(1 << 20)
+    # q k v gid L G eps dy dq dk dv dL deps ws bytes shape stream
+    args = [P] * 6 + [ctypes.c_float(1e-6)] + [P] * 6 + [_fake(1 << 24), n, ctypes.byref(s),
+                                                         None]
+    for i in (3, 11, 12):                        # group_id, dL, deps
+        bad = list(args)
+        bad[i] = None
+        assert L.oal_dense_backward_gpu(*bad) == -1
+    small = list(args)
+    small[14] = ctypes.c_size_t(n.value - 1)
+    assert L.oal_dense_backward_gpu(*small) == -8
+    mis = list(args)
+    mis[13] = _fake((1 << 24) + 16)
+    assert L.oal_dense_backward_gpu(*mis) == -4
