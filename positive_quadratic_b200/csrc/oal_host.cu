@@ -11,9 +11,9 @@
 #pragma once
 
 #include <algorithm>
-#include <vector>
 
 #include "oal_common.cuh"
+#include "oal_events.cuh"
 #include "oal_kernels.cuh"
 
 namespace oal {
@@ -56,22 +56,6 @@ int plan_host(const oal_shape* s, int segments, HostPlan* p)
     *p = h;
     return OAL_OK;
 }
-
-// Events of one call; destroyed on every exit path (a destroyed event that is still pending
-// is released by the runtime once it completes).
-struct EventSet {
-    std::vector<cudaEvent_t> ev;
-    ~EventSet()
-    {
-        for (cudaEvent_t e : ev) cudaEventDestroy(e);
-    }
-    cudaError_t make(cudaEvent_t* out)
-    {
-        const cudaError_t e = cudaEventCreateWithFlags(out, cudaEventDisableTiming);
-        if (e == cudaSuccess) ev.push_back(*out);
-        return e;
-    }
-};
 
 // dst/src rows of `width` bytes: rows x width, with the given pitches
 cudaError_t copy_rows(void* dst, size_t dpitch, const void* src, size_t spitch, size_t width,
@@ -121,7 +105,7 @@ int oal_prefill_host(const void* q_host, const void* k_host, const void* v_host,
         return prefill_impl(ws, ws, ws, group_id, L, G, eps, reinterpret_cast<float*>(ws),
                             state, pws, p.ws_bytes, s, stream, false);
 
-    EventSet evs;
+    CallEvents evs;
     cudaEvent_t ev_start, ev_end;
     OAL_CUDA_TRY(evs.make(&ev_start));
     OAL_CUDA_TRY(evs.make(&ev_end));

@@ -10,9 +10,9 @@
 #pragma once
 
 #include <algorithm>
-#include <vector>
 
 #include "oal_common.cuh"
+#include "oal_events.cuh"
 #include "oal_kernels.cuh"
 
 namespace oal {
@@ -54,20 +54,6 @@ int plan_varlen(const oal_shape* s, const int32_t* seq_lens, int n_seq, int n_st
     return OAL_OK;
 }
 
-struct VarlenEvents {
-    std::vector<cudaEvent_t> ev;
-    ~VarlenEvents()
-    {
-        for (cudaEvent_t e : ev) cudaEventDestroy(e);
-    }
-    cudaError_t make(cudaEvent_t* out)
-    {
-        const cudaError_t e = cudaEventCreateWithFlags(out, cudaEventDisableTiming);
-        if (e == cudaSuccess) ev.push_back(*out);
-        return e;
-    }
-};
-
 }  // namespace
 }  // namespace oal
 
@@ -105,7 +91,7 @@ int oal_prefill_varlen(const void* q, const void* k, const void* v, const int32_
     const size_t es = s->dtype == OAL_BF16 ? 2 : 4, D = OAL_HEAD_DIM, DV = OAL_VALUE_DIM;
     const int nst = std::min(n_streams, n_seq);
     cudaStream_t first = static_cast<cudaStream_t>(streams[0]);
-    VarlenEvents evs;
+    CallEvents evs;
     cudaEvent_t ev_start;
     OAL_CUDA_TRY(evs.make(&ev_start));
     OAL_CUDA_TRY(cudaEventRecord(ev_start, first));
