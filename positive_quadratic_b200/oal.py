@@ -330,42 +330,6 @@ def device_error(stream=None) -> int:
     return code.value
 
 
-def prefill_host(q, k, v, group_id, L, G, eps: float, chunk: int = 128, dev_bufs=None,
-                 out_host=None, stream=None):
-    """End-to-end prefill from HOST tensors (pinned for overlap): copies q/k/v to the device,
-    runs oal_prefill, copies yhat back.  ``dev_bufs`` (from ``alloc_prefill_buffers``) reuses
-    device buffers across calls.  Returns the host output tensor."""
-    if dev_bufs is None:
-        dev_bufs = alloc_prefill_buffers(q, k, v, group_id, L, G, chunk)
-    dq, dk, dv_, dg, dL, dG, dout, dstate, dws = dev_bufs
-    s = torch.cuda.current_stream() if stream is None else stream
-    with torch.cuda.stream(s):
-        dq.copy_(q, non_blocking=True)
-        dk.copy_(k, non_blocking=True)
-        dv_.copy_(v, non_blocking=True)
-        prefill(dq, dk, dv_, dg, dL, dG, eps, chunk, dout, dstate, dws, s)
-        if out_host is None:
-            out_host = torch.empty(dout.shape, dtype=dout.dtype, pin_memory=True)
-        out_host.copy_(dout, non_blocking=True)
-    return out_host
-
-
-def alloc_prefill_buffers(q, k, v, group_id, L, G, chunk, device="cuda"):
-    """Device buffers for prefill_host (group ids, L and G are copied once here)."""
-    shape = _shape_of(q, k, v, chunk)
-    dq = torch.empty(q.shape, dtype=q.dtype, device=device)
-    dk = torch.empty(k.shape, dtype=k.dtype, device=device)
-    dv_ = torch.empty(v.shape, dtype=v.dtype, device=device)
-    dg = group_id.to(device=device, dtype=torch.int32).contiguous()
-    dL = L.to(device=device, dtype=torch.float32).contiguous()
-    dG = G.to(device=device, dtype=torch.int32).contiguous()
-    dout = torch.empty(q.shape[0], q.shape[1], q.shape[2], v.shape[3], dtype=torch.float32,
-                       device=device)
-    dstate = torch.empty(state_bytes(shape), dtype=torch.uint8, device=device)
-    dws = empty_workspace(prefill_workspace_bytes(shape), device)
-    return dq, dk, dv_, dg, dL, dG, dout, dstate, dws
-
-
 def host_prefill_buffers(q, k, v, group_id, L, G, chunk: int = 128, segments: int = 4,
                          device="cuda") -> dict:
     """Device memory and copy streams for prefill_from_host: group ids, L and G copied once,
