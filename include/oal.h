@@ -293,6 +293,15 @@ int oal_dense_backward_gpu(const void* q, const void* k, const void* v, const in
                            void* workspace, size_t workspace_bytes, const oal_shape* s,
                            void* stream);
 
+/* Sum of prefix states: out[i] = parts[0*n + i] + parts[1*n + i] + ... for the n_parts
+ * arrays of n floats stored back to back in `parts`, added in that order (the prefix state of
+ * eq. (4) is a sum over tokens, so summing the states of a sequence's first segments, each
+ * computed alone, gives the state after them).  Used on the fp32 body of state buffers (the
+ * part after the header and the coefficient tables) by the sequence-parallel prefill.
+ * n_parts = 0 writes zeros.  Device pointers, 16-byte aligned; n a multiple of 4 when
+ * n_parts > 0.  `out` must not overlap `parts`. */
+int oal_state_prefix_sum(const float* parts, int n_parts, size_t n, float* out, void* stream);
+
 /* Reads the device-side error word (OAL_OK or a negative oal_status set by a kernel since
  * the last read), synchronising `stream`, and clears it. */
 int oal_device_error(int* code, void* stream);

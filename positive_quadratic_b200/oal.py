@@ -89,6 +89,8 @@ def lib() -> ctypes.CDLL:
             L.oal_prefill_varlen.argtypes = [_VP] * 6 + [ctypes.c_float, _VP, _VP, _SZ, _VP,
                                                          _SZ, _PS, _VP, ctypes.c_int, _VP,
                                                          ctypes.c_int]
+            L.oal_state_prefix_sum.argtypes = [_VP, ctypes.c_int, _SZ, _VP, _VP]
+            L.oal_state_prefix_sum.restype = ctypes.c_int
             L.oal_dense_backward_workspace_bytes.argtypes = [_PS, ctypes.POINTER(_SZ)]
             L.oal_dense_backward_gpu.argtypes = [_VP] * 6 + [ctypes.c_float] + [_VP] * 7 + [
                 _SZ, _PS, _VP]
@@ -246,6 +248,19 @@ def state_body(state: torch.Tensor, B: int, Hq: int, Hkv: int) -> torch.Tensor:
     off = 256 + ((Hq * FEATURES_PAD * 4 + 255) // 256) * 256
     n = B * Hkv * FEATURES_PAD * (VALUE_DIM + 1)
     return state[off:off + 4 * n].view(torch.float32)
+
+
+def state_prefix_sum(parts: torch.Tensor, n_parts: int, out: torch.Tensor, stream=None):
+    """oal_state_prefix_sum: out = parts[0] + ... + parts[n_parts - 1] (rows of a contiguous
+    fp32 [rows, n] tensor, added in order)."""
+    if parts.dim() != 2 or parts.dtype != torch.float32 or out.dtype != torch.float32:
+        raise ValueError("parts [rows, n] and out [n] must be fp32")
+    if not 0 <= n_parts <= parts.shape[0] or out.numel() != parts.shape[1]:
+        raise ValueError("n_parts out of range or out of the wrong size")
+    _contig_cuda(parts, out)
+    _check(lib().oal_state_prefix_sum(_ptr(parts), int(n_parts), parts.shape[1], _ptr(out),
+                                      _stream(stream)), "oal_state_prefix_sum")
+    return out
 
 
 def set_state_tokens(state: torch.Tensor, tokens: int) -> None:

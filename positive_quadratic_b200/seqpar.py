@@ -6,12 +6,13 @@ before it.  Each rank
   1. computes the state of its own segment alone (a prefill without outputs),
   2. all-gathers the segment states (the one exchange step: B*Hkv*2176*65 fp32 per rank,
      1.1 MB for one Qwen2.5-0.5B layer, independent of the sequence length),
-  3. continues its segment from the sum of the earlier ranks' states (oal_prefill_continue),
+  3. writes the sum of the earlier ranks' states into its state buffer (oal_state_prefix_sum)
+     and continues its segment from there (oal_prefill_continue),
 which yields its tokens' outputs and the prefix state after its segment (the last rank holds
 the state of the whole sequence, ready for decode).
 
-The backend performs the three local operations; the default one is this library on the
-rank's GPU.  Ranks are torch.distributed ranks (NCCL on GPUs); `allgather` may be replaced
+The backend performs the local operations (segment state, state access, combine, continue);
+the default one is this library on the rank's GPU.  Ranks are torch.distributed ranks (NCCL on GPUs); `allgather` may be replaced
 (e.g. to run the ranks of one process for testing).
 """
 from __future__ import annotations
@@ -37,6 +38,10 @@ class LibraryBackend:
 
     def set_tokens(self, state, tokens):
         self.oal.set_state_tokens(state, tokens)
+
+    def combine(self, parts, n_parts, body):
+        """body = parts[0] + ... + parts[n_parts - 1], in the library (fixed order)."""
+        self.oal.state_prefix_sum(parts, n_parts, body)
 
     def continue_from(self, q, k, v, group_id, L, G, eps, state):
         return self.oal.prefill_continue(q, k, v, group_id, L, G, eps, state)
@@ -71,10 +76,9 @@ def sequence_parallel_prefill(q, k, v, group_id, L, G, eps: float, *, rank: int,
     parts = allgather(body.clone())
     if len(parts) != world:
         raise RuntimeError(f"all-gather returned {len(parts)} parts for {world} ranks")
-    prefix = torch.zeros_like(body)
-    for r in range(rank):
-        prefix += parts[r]
-    body.copy_(prefix)
+    if isinstance(parts, (list, tuple)):
+        parts = torch.stack(list(parts))  # one [world, n] buffer
+    backend.combine(parts, rank, body)
     backend.set_tokens(state, tokens_before)
     out = backend.continue_from(q, k, v, group_id, L, G, eps, state)
     return out, state

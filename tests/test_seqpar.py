@@ -34,6 +34,9 @@ class OracleBackend:
     def set_tokens(self, state, tokens):
         state["tokens"] = tokens
 
+    def combine(self, parts, n_parts, body):
+        body.copy_(parts[:n_parts].sum(dim=0))
+
     def continue_from(self, q, k, v, group_id, L, G, eps, state):
         st, flat = state["st"], state["_flat"].numpy()
         n0, n1 = st.H0.size, st.H1.size
@@ -125,3 +128,21 @@ def test_segments_on_one_gpu_match_whole_sequence(cuda):
         torch.cuda.synchronize()
         assert oal.device_error() == 0
         assert row_rel_err(y.cpu().numpy(), ref[:, :, r * seg:(r + 1) * seg]) <= TOL_BF16
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("n_parts", [0, 1, 3])
+def test_state_prefix_sum(cuda, n_parts):
+    """oal_state_prefix_sum adds the parts in order: equal, bit for bit, to fp32 additions in
+    the same order."""
+    from positive_quadratic_b200 import oal
+    n = 2 * 2176 * 65
+    g = torch.Generator().manual_seed(n_parts)
+    parts = torch.randn(4, n, generator=g).to(cuda)
+    out = torch.full((n,), float("nan"), device=cuda)
+    oal.state_prefix_sum(parts, n_parts, out)
+    ref = torch.zeros(n, device=cuda)
+    for r in range(n_parts):
+        ref = ref + parts[r]
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
