@@ -78,3 +78,33 @@ def test_decode_group_sizes(oal, cuda, Hq, Hkv, dtype):
     assert hdr["tokens"] == T0 + n
     ref = pack_oracle_state(st_all)
     assert np.max(np.abs(S[:, :, :F] - ref) / np.abs(ref).max(axis=2, keepdims=True)) < 1e-5
+
+
+def test_decode_step_in_a_cuda_graph(oal, cuda):
+    """A decode step captured once in a CUDA graph and replayed token after token (new
+    inputs copied into the captured buffers) continues the sequence like eager calls."""
+    B, Hq, Hkv, T0, n = 2, 14, 2, 140, 4
+    p = I.small_layer(330, B=B, T=T0 + n, Hq=Hq, Hkv=Hkv, dtype="bf16")
+    y_all = oracle.recurrent(p.q, p.k, p.v, p.group_id, p.L, p.G, p.eps)
+    _, state = gpu_prefill(oal, p.slice_tokens(0, T0), cuda, 128)
+    ws = oal.decode_workspace(B, Hq, Hkv, cuda)
+    q, k, v, _, _, _ = dev_inputs(p, cuda)
+    sq = q[:, :, T0:T0 + 1].clone()
+    sk = k[:, :, T0:T0 + 1].clone()
+    sv = v[:, :, T0:T0 + 1].clone()
+    out = torch.empty(B, Hq, 1, 64, dtype=torch.float32, device=cuda)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        oal.decode_step(sq, sk, sv, state, ws, out=out)
+    # capturing does not run the step: the state still holds T0 tokens
+    for t in range(T0, T0 + n):
+        sq.copy_(q[:, :, t:t + 1])
+        sk.copy_(k[:, :, t:t + 1])
+        sv.copy_(v[:, :, t:t + 1])
+        graph.replay()
+        torch.cuda.synchronize()
+        assert row_rel_err(out.cpu().numpy()[:, :, 0], y_all[:, :, t]) <= TOL_BF16
+    assert oal.device_error() == 0
+    hdr, _, _ = read_state(state.cpu().numpy(), B, Hq, Hkv)
+    assert hdr["tokens"] == T0 + n
