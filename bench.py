@@ -66,6 +66,9 @@ def parse():
                     help="between timed steps: write a 256 MB buffer, then (default) read "
                          "another 256 MB so that the write's dirty lines are written back "
                          "outside the timed events")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the small timings of the further paths (Hadamard prefill, "
+                         "variable-length batch, dense backward)")
     ap.add_argument("--e2e-segments", type=int, default=4,
                     help="segments of the e2e host-buffer prefill (copies overlap kernels)")
     ap.add_argument("--workload", default="config1", choices=["config1", "config3_16k",
@@ -347,46 +350,20 @@ def main():
     # ---- e2e through the C ABI with pinned host buffers (oal_prefill_host) ----
     e2e = None
     if not args.no_e2e:
-        hq = q.cpu().pin_memory()
-        hk = k.cpu().pin_memory()
-        hv = v.cpu().pin_memory()
-        hout = torch.empty(out.shape, dtype=torch.float32, pin_memory=True)
-        # segments continue the prefix, which only the tensor-core path (chunk 128) does
-        nseg = args.e2e_segments if args.chunk == 128 else 1
-        bufs = oal.host_prefill_buffers(hq, hk, hv, g, L, G, args.chunk, nseg, device=dev)
-        oal.prefill_from_host(hq, hk, hv, p.eps, bufs, hout)
-        torch.cuda.synchronize()
-        # the segmented call must reproduce the device-resident prefill exactly
-        same = bool(torch.equal(hout, out.cpu())) and oal.device_error() == 0
-        if not same:
-            bufs = oal.host_prefill_buffers(hq, hk, hv, g, L, G, args.chunk, 1, device=dev)
-        for _ in range(3):
-            oal.prefill_from_host(hq, hk, hv, p.eps, bufs, hout)
-            flush()
-        evs2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in range(args.steps)]
-        barrier()
-        torch.cuda.synchronize()
-        for s0, s1 in evs2:
-            s0.record(stream)
-            oal.prefill_from_host(hq, hk, hv, p.eps, bufs, hout)
-            s1.record(stream)
-            flush()
-        torch.cuda.synchronize()
-        assert oal.device_error() == 0
-        e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs2), world, dev)
-        e2e = {"value": job_rate(world, args.steps * B * T, e_ms), "unit": UNIT,
-               "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in (hq, hk, hv))),
-               "d2h_bytes_per_step": int(hout.numel() * 4),
-               "api": "oal_prefill_host",
-               "segments": bufs["segments"],
-               "segmented_matches_device_prefill": same}
+        try:
+            e2e = run_e2e(args, dev, torch, oal, p, q, k, v, g, L, G, out, B, T, flush,
+                          barrier, stream, world)
+        except Exception as exc:  # recorded in the line; the device-resident value stands
+            e2e = {"error": repr(exc)[:300]}
 
     # ---- decode ----
     decode = None
     if not args.no_decode:
         decode = run_decode(args, dev, torch, oal, pk, pk_kind, flush, world, barrier)
 
+    extras = None
+    if not args.no_extras:
+        extras = run_extras(dev, torch, oal)
     base = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         base = cpu_baseline(p)
@@ -402,7 +379,7 @@ def main():
                            "l2": flush.describe(),
                            "parallelism": f"replicas x{world}"},
                 "roofline": roof, "e2e": e2e, "gpu_launches": int(n_launch),
-                "clocks": clk.summary(), "decode": decode, "cpu_baseline": base,
+                "clocks": clk.summary(), "decode": decode, "extras": extras, "cpu_baseline": base,
                 "step_ms_min": min(step_ms), "step_ms_median": statistics.median(step_ms)}
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -433,6 +410,122 @@ class L2Flush:
         return ("flushed between steps: 256 MB write, then 256 MB read so no dirty lines remain "
                 "(outside timed events)" if self.clean else
                 "flushed between steps: 256 MB write (outside timed events)")
+
+
+def run_e2e(args, dev, torch, oal, p, q, k, v, g, L, G, out, B, T, flush, barrier, stream,
+            world):
+    """The prefill metric through the C ABI's host-buffer call (oal_prefill_host): pinned
+    host q/k/v in, fp32 yhat back, copies inside the timed events."""
+    hq = q.cpu().pin_memory()
+    hk = k.cpu().pin_memory()
+    hv = v.cpu().pin_memory()
+    hout = torch.empty(out.shape, dtype=torch.float32, pin_memory=True)
+    # segments continue the prefix, which only the tensor-core path (chunk 128) does
+    nseg = args.e2e_segments if args.chunk == 128 else 1
+    bufs = oal.host_prefill_buffers(hq, hk, hv, g, L, G, args.chunk, nseg, device=dev)
+    oal.prefill_from_host(hq, hk, hv, p.eps, bufs, hout)
+    torch.cuda.synchronize()
+    # the segmented call must reproduce the device-resident prefill exactly
+    same = bool(torch.equal(hout, out.cpu())) and oal.device_error() == 0
+    if not same:
+        bufs = oal.host_prefill_buffers(hq, hk, hv, g, L, G, args.chunk, 1, device=dev)
+    for _ in range(3):
+        oal.prefill_from_host(hq, hk, hv, p.eps, bufs, hout)
+        flush()
+    evs2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for s0, s1 in evs2:
+        s0.record(stream)
+        oal.prefill_from_host(hq, hk, hv, p.eps, bufs, hout)
+        s1.record(stream)
+        flush()
+    torch.cuda.synchronize()
+    assert oal.device_error() == 0
+    e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs2), world, dev)
+    e2e = {"value": job_rate(world, args.steps * B * T, e_ms), "unit": UNIT,
+           "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in (hq, hk, hv))),
+           "d2h_bytes_per_step": int(hout.numel() * 4),
+           "api": "oal_prefill_host",
+           "segments": bufs["segments"],
+           "segmented_matches_device_prefill": same}
+    return e2e
+
+
+def run_extras(dev, torch, oal):
+    """Small timings of the further paths on this rank (no cross-rank reduction): the
+    Hadamard-form prefill, a variable-length batch over four streams and the dense backward.
+    Each is timed with CUDA events after warm-up; a failure is recorded, not raised."""
+    from positive_quadratic_b200 import inputs as I
+    res = {}
+
+    def timed(fn, reps=5):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    def to(a, d=None):
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev, d)
+
+    try:  # ungrouped Hadamard form, CUDA cores, chunk 64
+        p = I.small_layer(901, B=1, T=2048, Hq=14, Hkv=2, dtype="bf16")
+        q, k, v = (to(x, torch.bfloat16) for x in (p.q, p.k, p.v))
+        a, b, C = (to(x, torch.float32) for x in oracle_free_hadamard_coefs(14))
+        ms = timed(lambda: oal.prefill_hadamard(q, k, v, a, b, C, 64))
+        res["hadamard_prefill"] = {"workload": "B=1 T=2048 Hq=14 Hkv=2 bf16, chunk 64",
+                                   "ms": ms, "tokens_per_s": 2048 / (ms / 1e3)}
+    except Exception as exc:
+        res["hadamard_prefill"] = {"error": repr(exc)[:300]}
+    try:  # variable-length batch: 16 sequences of 64..2048 tokens over 4 streams
+        rng = np.random.default_rng(902)
+        lens = [int(x) for x in rng.integers(64, 2049, size=16)]
+        base = I.small_layer(903, B=1, T=1, Hq=14, Hkv=2, dtype="bf16")
+        g, L, G = to(base.group_id), to(base.L), to(base.G)
+        seqs = [I.small_layer(904 + i, B=1, T=t, Hq=14, Hkv=2, dtype="bf16")
+                for i, t in enumerate(lens)]
+        qs = [to(s.q[0], torch.bfloat16) for s in seqs]
+        ks = [to(s.k[0], torch.bfloat16) for s in seqs]
+        vs = [to(s.v[0], torch.bfloat16) for s in seqs]
+        streams = [torch.cuda.Stream(device=dev) for _ in range(4)]
+        ms = timed(lambda: oal.prefill_varlen(qs, ks, vs, g, L, G, base.eps, 128,
+                                              streams=streams))
+        res["varlen_prefill"] = {"workload": f"16 sequences, {sum(lens)} tokens, 4 streams, "
+                                             "Hq=14 Hkv=2 bf16, chunk 128 (includes packing)",
+                                 "ms": ms, "tokens_per_s": sum(lens) / (ms / 1e3)}
+    except Exception as exc:
+        res["varlen_prefill"] = {"error": repr(exc)[:300]}
+    try:  # dense backward, reference scale
+        p = I.small_layer(905, B=1, T=256, Hq=14, Hkv=2, dtype="bf16")
+        q, k, v = (to(x, torch.bfloat16) for x in (p.q, p.k, p.v))
+        g, L, G = to(p.group_id), to(p.L), to(p.G)
+        dy = torch.randn(1, 14, 256, 64, device=dev)
+        ms = timed(lambda: oal.dense_backward(q, k, v, g, L, G, p.eps, dy), reps=3)
+        res["dense_backward"] = {"workload": "B=1 T=256 Hq=14 Hkv=2 bf16 (O(T^2) reference)",
+                                 "ms": ms}
+    except Exception as exc:
+        res["dense_backward"] = {"error": repr(exc)[:300]}
+    if oal.device_error() != 0:
+        res["device_error"] = True
+    return res
+
+
+def oracle_free_hadamard_coefs(Hq, d=64):
+    """Seeded Hadamard-form coefficients with a positive kernel: a in [2, 3), small b,
+    C = W W^T / d + I/2 (the benchmark's own draw; no oracle involved)."""
+    rng = np.random.default_rng(906)
+    a = 2.0 + rng.random(Hq)
+    b = 0.1 * rng.standard_normal((Hq, d))
+    W = rng.standard_normal((Hq, d, d))
+    C = W @ W.transpose(0, 2, 1) / d + 0.5 * np.eye(d)
+    return a, b, C
 
 
 def run_decode(args, dev, torch, oal, pk, pk_kind, flush, world, barrier):
