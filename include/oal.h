@@ -163,8 +163,11 @@ int oal_decode_step(const void* q, const void* k, const void* v, void* state, fl
  * until the process exits).  A step needs align256(4*B*Hkv) + 2340*B*Hq bytes of it, so
  * B*Hq must stay at or below 1788 (batch 64 x 14 heads fits); larger problems return
  * OAL_ERR_UNSUPPORTED without launching anything.
- * The first call on each device looks up the array's device address (cudaGetSymbolAddress);
- * make that first call before any stream capture.  Every call shares the one array and
+ * The first call on each device looks up the array's device address (cudaGetSymbolAddress)
+ * and caches it; make that first call before any stream capture.  cudaDeviceReset discards
+ * the library's device code and data on that device, and with them the array the cached
+ * address points to: do not call this entry point on a device after resetting it in the
+ * same process.  Every call shares the one array and
  * clears the part that must start at zero itself, so calls that overlap on the GPU (on
  * different streams, or from threads that do not order their calls) race and corrupt each
  * other's results: issue them one after another. */

@@ -113,16 +113,18 @@ int oal_prefill_varlen(const void* q, const void* k, const void* v, const int32_
         void* ws = static_cast<unsigned char*>(workspace) + size_t(j) * p.ws_slice;
         rc = prefill_impl(qi, ki, vi, group_id, L, G, eps, oi, st, ws, p.ws_one, &one,
                           streams[j], false);
-        if (rc) return rc;
+        if (rc) break;
         off += seq_lens[i];
     }
+    // join every side stream back into the first, also after a failed sequence, so that later
+    // work on streams[0] is ordered after everything already enqueued and no fork stays open
     for (int j = 1; j < nst; ++j) {
         cudaEvent_t ev;
         OAL_CUDA_TRY(evs.make(&ev));
         OAL_CUDA_TRY(cudaEventRecord(ev, static_cast<cudaStream_t>(streams[j])));
         OAL_CUDA_TRY(cudaStreamWaitEvent(first, ev, 0));
     }
-    return OAL_OK;
+    return rc;
 }
 
 }  // extern "C"

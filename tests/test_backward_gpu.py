@@ -1,7 +1,16 @@
 """GPU parity of the dense backward pass (oal_dense_backward_gpu) against the oracle's
 gradients (oracle.dense_backward, pinned by finite differences and exact identities in
 tests/test_oracle_backward_pins.py).  fp32 arithmetic on both input dtypes: each gradient
-within 1e-4 of the oracle, relative to its largest entry."""
+within 1e-4 of the oracle, relative to its largest entry, or to 1e-3 of the gradient's
+natural scale when that is larger.
+
+The floor matters only where a gradient vanishes in exact arithmetic.  At T = 1 the single
+row attends to itself alone, so yhat_0 = v_0 and every dkappa = dy . (v_0 - yhat_0) / D is
+zero: dq, dk and dL are exactly 0 (the oracle returns fp64 rounding, ~1e-18) and the fp32
+kernel returns fp32 rounding of the same cancellation (~1e-9).  A relative error against
+~1e-18 is meaningless there.  The natural scale of a gradient is the product of the
+magnitudes its chain-rule terms multiply: max|dy| max|v| max|q|,|k| for dq and dk (dkappa
+carries dy (v - yhat), dkappa/dq carries k), max|dy| for dv, max|dy| max|v| max|L| for dL."""
 import numpy as np
 import pytest
 
@@ -14,8 +23,17 @@ pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
 
 
-def _rel(a, b):
-    return float(np.abs(np.asarray(a, np.float64) - b).max() / max(np.abs(b).max(), 1e-30))
+def _rel(a, b, scale=0.0):
+    """max |a - b| over max(max |b|, 1e-3 * scale)."""
+    den = max(float(np.abs(b).max()), 1e-3 * scale, 1e-30)
+    return float(np.abs(np.asarray(a, np.float64) - b).max() / den)
+
+
+def _natural_scales(p, dy):
+    a = lambda x: float(np.abs(np.asarray(x, np.float64)).max()) if np.size(x) else 0.0  # noqa: E731
+    qk = max(a(p.q), a(p.k))
+    return {"dq": a(dy) * a(p.v) * qk, "dk": a(dy) * a(p.v) * qk, "dv": a(dy),
+            "dL": a(dy) * a(p.v) * a(p.L)}
 
 
 @pytest.mark.parametrize("dtype,B,T,Hq,Hkv", [("f32", 2, 70, 4, 2), ("bf16", 1, 131, 8, 1),
@@ -29,8 +47,9 @@ def test_dense_backward_matches_oracle(oal, cuda, dtype, B, T, Hq, Hkv):
     got = oal.dense_backward(q, k, v, g, L, G, p.eps, torch.from_numpy(dy).float())
     torch.cuda.synchronize()
     assert oal.device_error() == 0
+    scale = _natural_scales(p, dy)
     for name in ("dq", "dk", "dv", "dL"):
-        assert _rel(got[name].cpu().numpy(), ref[name]) <= 1e-4, name
+        assert _rel(got[name].cpu().numpy(), ref[name], scale[name]) <= 1e-4, name
     dL = got["dL"].cpu().numpy()
     for h in range(Hq):  # zero outside each head's live block
         n = int(p.G[h]) + 1
