@@ -97,7 +97,7 @@ int oal_prefill_workspace_bytes(const oal_shape* s, size_t* bytes)
     if (rc) return rc;
     if ((rc = check_chunk(s))) return rc;
     if (!bytes) return OAL_ERR_NULL;
-    const size_t tc = use_tensor_path(s) ? tc_workspace_bytes(s->B, s->Hkv, s->T) : 0;
+    const size_t tc = use_tensor_path(s) ? tc_workspace_bytes(s->B, s->Hq, s->Hkv, s->T) : 0;
     *bytes = simt_chunk_state_bytes(s) > tc ? simt_chunk_state_bytes(s) : tc;
     if (*bytes == 0) *bytes = 256;
     return OAL_OK;

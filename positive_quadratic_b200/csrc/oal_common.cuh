@@ -43,6 +43,15 @@ constexpr int kLinStart = 2080;
 constexpr int kConstRow = 2144;
 constexpr int kMaxGroup = 8;            // Hq / Hkv supported
 
+// Per-query-head table of the tensor-core readout, written into the prefill workspace by the
+// coefficient expansion (a1) and copied into shared memory once per readout item:
+constexpr uint32_t kTabCoefH = 0;      // bf16 [1792]: coefficients of the off-diagonal rows
+constexpr uint32_t kTabCoefT = 3584;   // fp32 [384]: coefficients of rows 1792..2175
+constexpr uint32_t kTabW = 5120;       // fp32 [9][64]: L_{g(r),m} / sqrt(d_h) (0 for m > G)
+constexpr uint32_t kTabC0 = 7424;      // fp32 [9]: L_{0,m} (0 for m > G)
+constexpr uint32_t kTabG = 7460;       // int32: G of the head (clamped to 1..8)
+constexpr uint32_t kTabBytes = 7680;   // a multiple of 256
+
 constexpr uint32_t kStateMagic = 0x534C414Fu;  // "OALS"
 constexpr size_t kHeaderBytes = 256;
 

@@ -34,7 +34,7 @@ int read_device_error(int* code, cudaStream_t st);
 
 // tensor-core (tcgen05) bf16 prefill, chunk 128
 size_t tc_image_bytes(int B, int Hkv, int T);
-size_t tc_workspace_bytes(int B, int Hkv, int T);
+size_t tc_workspace_bytes(int B, int Hq, int Hkv, int T);
 int launch_prefill_tc(const void* q, const void* k, const void* v, const int32_t* gid,
                       const float* L, const int32_t* G, float eps, float* out, void* state,
                       void* ws, int B, int T, int Hq, int Hkv, bool overlap, bool cont,

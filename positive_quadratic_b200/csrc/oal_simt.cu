@@ -25,7 +25,8 @@ __device__ __forceinline__ void prep_head(int h, const int32_t* __restrict__ gid
                                           const float* __restrict__ L,
                                           const int32_t* __restrict__ G, float eps,
                                           unsigned char* __restrict__ state, int B, int Hq,
-                                          int Hkv, long long tokens, bool add_tokens = false)
+                                          int Hkv, long long tokens, bool add_tokens = false,
+                                          unsigned char* __restrict__ rtab = nullptr)
 {
     const int tid = threadIdx.x;
     __shared__ double M[kGM1][kGM1];
@@ -71,6 +72,26 @@ __device__ __forceinline__ void prep_head(int h, const int32_t* __restrict__ gid
             if (f == kConstRow) val += double(eps);
         }
         coef[f] = float(val);
+        if (rtab) {  // the readout table: bf16 off-diagonal coefficients, fp32 for the rest
+            unsigned char* tb = rtab + size_t(h) * kTabBytes;
+            if (f < kOffDiagRows)
+                reinterpret_cast<__nv_bfloat16*>(tb + kTabCoefH)[f] = __float2bfloat16_rn(float(val));
+            else
+                reinterpret_cast<float*>(tb + kTabCoefT)[f - kOffDiagRows] = float(val);
+        }
+    }
+    if (rtab) {
+        // score-tile weights of the factored intra-chunk kernel, eq. (3) as
+        // kappa = eps + sum_m (L_0m + sum_r q_r k_r L_{g(r),m} / sqrt(d_h))^2
+        unsigned char* tb = rtab + size_t(h) * kTabBytes;
+        const float* Lh = L + size_t(h) * kGM1 * kGM1;
+        for (int e = tid; e < kGM1 * kD; e += blockDim.x) {
+            const int m = e / kD, r = e % kD;
+            reinterpret_cast<float*>(tb + kTabW)[e] = m <= Gh ? Lh[g[r] * kGM1 + m] * 0.125f : 0.f;
+        }
+        if (tid < kGM1) reinterpret_cast<float*>(tb + kTabC0)[tid] = tid <= Gh ? Lh[tid] : 0.f;
+        if (tid == 0) *reinterpret_cast<int*>(tb + kTabG) = Gh;
+        for (uint32_t b = kTabG + 4 + tid; b < kTabBytes; b += blockDim.x) tb[b] = 0;
     }
     if (h == 0 && tid == 0) {
         StateHeader* hd = reinterpret_cast<StateHeader*>(state);

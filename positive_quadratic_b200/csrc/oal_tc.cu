@@ -58,18 +58,6 @@ constexpr uint32_t kTmemCols = 512;
 static_assert(kFP % kSlabRows == 0 && kFP % 64 == 0, "feature padding");
 
 // ---- shared memory (offsets from a 1024-aligned base) ---------------------------------------
-// reader
-constexpr uint32_t kRdOffK = 0;           // K tile (score B operand, K-major)
-constexpr uint32_t kRdOffV = 16384;       // V tile (PV B operand, MN-major)
-constexpr uint32_t kRdOffQ = 32768;       // Q tile (bf16, K-major): phi and Aq read it
-constexpr uint32_t kRdOffAq = 49152;      // Aq0 | Aq1 (score A operands); the P tile aliases
-constexpr uint32_t kRdOffA = 81920;       // 4 x 16 KB phi stages (readout A operand, K-major)
-constexpr uint32_t kRdOffB = 147456;      // 2 x 20 KB state-image stages of 2 slices (B operand)
-constexpr uint32_t kRdOffCoef = 188416;   // 2176 fp32 coefficients
-constexpr uint32_t kRdOffCoefH = 197120;  // 1792 bf16 coefficients of the off-diagonal rows
-constexpr uint32_t kRdOffW = 200704;      // 9 x 64 fp32
-constexpr uint32_t kRdOffC0 = 203008;     // 9 fp32
-constexpr uint32_t kRdOffOnes = 203776;   // 16 KB ones atom; then image stage 2 (20 KB) reuses it
 // chunk-delta builder
 constexpr uint32_t kStOffKV = 0;          // 3 x (K 16 KB + V 16 KB)
 constexpr uint32_t kStOffA = 98304;       // 3 x (hi 16 KB + lo 16 KB) psi stages
@@ -78,58 +66,21 @@ constexpr uint32_t kOffOnes = 196608;     // 16 KB ones atom
 constexpr uint32_t kOffCtl = 224256;      // barriers and control words
 constexpr uint32_t kSmemBytes = kOffCtl + 1024 + 1024;
 
-constexpr int kPhiSets = 4;                                // reader warps (w >> 2) per slice
-// phi stages (SMEM, 1 slice): two per warp set (stages kq and kq + 4), so that every wait on
-// a stage barrier is for the phase right after the one the waiter last saw complete (parity
-// waits cannot tell phases two apart).  Stages 0..3 have their own region; stages 4..7 reuse
-// the K, V and Aq | P tiles once the intra-chunk MMAs that read them have completed.
-constexpr int kRdStages = 2 * kPhiSets;
-// image stages (SMEM, 2 slices each): stages 0, 1 have their own region, stage 2 reuses the
-// ones atom once the intra-chunk P [V | 1] MMAs have completed
-constexpr int kBStages = 3;
 constexpr uint32_t kImgPairBytes = 2 * kImgSliceBytes;     // one tensor copy: 160 rows
-constexpr uint32_t kPhiTileBytes = kC * 64 * 2;            // 128 rows x 64 packed rows, bf16
 constexpr int kKVStages = 3;
 constexpr int kDAStages = 3;  // psi stages (hi + lo tiles of one half chunk)
 constexpr int kDAcc = 4;      // TMEM accumulators of the delta builder (128 columns each)
 constexpr uint32_t kStATile = 64 * kSlabRows * 2;          // 64 tokens x 128 rows = 16 KB
-// reader TMEM map: U in [0, 80); score tiles S0 | S1 in [128, 384).  phi stays in shared
-// memory: warp stores into tensor memory stall concurrent MMAs, shared-memory stores do not.
-constexpr uint32_t kColU = 0, kColS0 = 128;
 static_assert(kStOffKV + kKVStages * 2 * kTileBytes <= kStOffA &&
                   kStOffA + kDAStages * 2 * kStATile <= kOffOnes &&
                   kOffOnes + kOnesAtomBytes <= kOffCtl && kDAcc * 128 <= int(kTmemCols),
               "delta builder shared-memory and TMEM map");
-__host__ __device__ constexpr uint32_t rd_stage_off(int st)
-{
-    return st < kPhiSets ? kRdOffA + uint32_t(st) * kPhiTileBytes
-                         : (st == 4 ? kRdOffK : st == 5 ? kRdOffV : kRdOffAq + (st - 6) * kTileBytes);
-}
-static_assert(kRdOffK + kTileBytes <= kRdOffV && kRdOffV + kTileBytes <= kRdOffQ &&
-                  kRdOffAq + 2 * kTileBytes <= kRdOffA && kTileBytes == kPhiTileBytes,
-              "reused phi stages");
-__host__ __device__ constexpr uint32_t rd_bstage_off(int bs)
-{
-    return bs < 2 ? kRdOffB + uint32_t(bs) * kImgPairBytes : kRdOffOnes;
-}
-static_assert(kRdOffA + kPhiSets * kPhiTileBytes <= kRdOffB &&
-                  kRdOffB + 2 * kImgPairBytes <= kRdOffCoef && kRdOffC0 + 64 <= kRdOffOnes &&
-                  kRdOffOnes % 1024 == 0 && kRdOffOnes + kImgPairBytes <= kOffCtl &&
-                  kOnesAtomBytes <= kImgPairBytes,
-              "reader shared-memory map");
-
-struct RdBars {
-    uint64_t qkv_full, aq_full[2], s_full[2], s_empty[2], p_full, pv_done;
-    uint64_t a_full[kRdStages], a_empty[kRdStages], b_full[kBStages], b_empty[kBStages];
-    uint64_t u_full, done;
-};
 struct StBars {
     uint64_t kv_full[kKVStages], kv_empty[kKVStages], a_full[kDAStages], a_empty[kDAStages];
     uint64_t acc_full[kDAcc], acc_empty[kDAcc], done;
 };
 struct Ctl {
     union {
-        RdBars rd;
         StBars st;
         uint64_t raw[64];
     } bar;
@@ -138,8 +89,7 @@ struct Ctl {
     int G;
 };
 static_assert(sizeof(Ctl) <= 1024, "control block");
-static_assert(sizeof(RdBars) <= sizeof(uint64_t) * 64 && sizeof(StBars) <= sizeof(uint64_t) * 64,
-              "barrier block");
+static_assert(sizeof(StBars) <= sizeof(uint64_t) * 64, "barrier block");
 
 struct Params {
     const CUtensorMap* tm_q;
@@ -150,7 +100,7 @@ struct Params {
     const float* L;
     const int32_t* G;
     float eps;
-    const float* coef_all;   // state header coefficient table [Hq][kFP]
+    const unsigned char* rtab;  // per-head readout tables [Hq][kTabBytes] (workspace)
     unsigned char* img;      // chunk-state images [B*Hkv][NC][34 slices][80 n][64 f] bf16
     float* dS;               // chunk deltas [B*Hkv][NC][65][kFP] fp32
     float* out;
@@ -527,397 +477,31 @@ constexpr bool phi_chunk_needed(int ch)  // 8-dim chunk of the q row
     return false;
 }
 
-// diagonal / linear / constant slices: 64 rows with compile-time (r, t); fp32 products,
-// one rounding
-template <int F0>
-__device__ __forceinline__ void phi_static(const unsigned char* qt, const float* coef, int row,
-                                           uint32_t (&w)[32])
-{
-    float q[66];
-    static_for<8>([&](auto CH) {
-        constexpr int ch = decltype(CH)::value;
-        if constexpr (phi_chunk_needed<F0>(ch)) {
-            const uint4 v = *reinterpret_cast<const uint4*>(qt + kmajor_chunk(row, ch));
-            q[8 * ch + 0] = bf16lo_to_f32(v.x);
-            q[8 * ch + 1] = bf16hi_to_f32(v.x);
-            q[8 * ch + 2] = bf16lo_to_f32(v.y);
-            q[8 * ch + 3] = bf16hi_to_f32(v.y);
-            q[8 * ch + 4] = bf16lo_to_f32(v.z);
-            q[8 * ch + 5] = bf16hi_to_f32(v.z);
-            q[8 * ch + 6] = bf16lo_to_f32(v.w);
-            q[8 * ch + 7] = bf16hi_to_f32(v.w);
-        }
-    });
-    q[64] = 1.f;
-    q[65] = 0.f;
-    static_for<8>([&](auto X) {
-        constexpr int x = decltype(X)::value;
-        const float4 c0 = *reinterpret_cast<const float4*>(coef + F0 + 8 * x);
-        const float4 c1 = *reinterpret_cast<const float4*>(coef + F0 + 8 * x + 4);
-        const float cf[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-        static_for<4>([&](auto E) {
-            constexpr int e = decltype(E)::value;
-            constexpr RT a = feature_rt(F0 + 8 * x + 2 * e);
-            constexpr RT b = feature_rt(F0 + 8 * x + 2 * e + 1);
-            w[4 * x + e] =
-                pack_bf16x2(cf[2 * e] * (q[a.r] * q[a.t]), cf[2 * e + 1] * (q[b.r] * q[b.t]));
-        });
-    });
-}
-
-__device__ __forceinline__ void phi_diag(const unsigned char* qt, const float* coef, int s,
-                                         int row, uint32_t (&w)[32])
-{
-    const int sel = s - kOffDiagSlices;
-    static_for<kSlices - kOffDiagSlices>([&](auto I) {
-        constexpr int i = decltype(I)::value;
-        if (sel == i) phi_static<kOffDiagRows + i * 64>(qt, coef, row, w);
-    });
-}
-
 // ------------------------------------------------------------------------------------------
-// reader item: (bh, chunk c).  Warps 0-15 (row quarter qw = w & 3, set kq = w >> 2):
-//   intra-chunk phase: Aq tiles (dims [16 kq, 16 kq + 16)), kappa over keys
-//   [32 kq, 32 kq + 32) of score tiles S_0..S_G, P tile;
-//   inter-chunk phase: phi of slices s = kq (mod 4) into TMEM stages;
-//   epilogue: yhat columns [16 kq, 16 kq + 16).
-// Warp 16: TMA, warp 17: MMA (S_0..S_G, then P [V; 1], then the 34 readout slices).
-// ------------------------------------------------------------------------------------------
-__device__ void reader_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Params& P, int bh,
-                            int c)
-{
-    RdBars& bar = ctl.bar.rd;
-    volatile int* abort_flag = &ctl.abort_flag;
-    const int Hq = P.Hq, Hkv = P.Hkv, T = P.T, NC = P.NC;
-    const int b = bh / Hq, h = bh % Hq, kv = h / (Hq / Hkv), bkv = b * Hkv + kv;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    float* coef = reinterpret_cast<float*>(sm + kRdOffCoef);
-    uint32_t* coefh = reinterpret_cast<uint32_t*>(sm + kRdOffCoefH);
-    float* wch = reinterpret_cast<float*>(sm + kRdOffW);
-    float* c0 = reinterpret_cast<float*>(sm + kRdOffC0);
-    const bool has_inter = c > 0 || P.cont;
-
-    if (threadIdx.x == 0) {
-        mbar_init(&bar.qkv_full, 1);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&bar.aq_full[i], 16);
-            mbar_init(&bar.s_full[i], 1);
-            mbar_init(&bar.s_empty[i], 16);
-        }
-        mbar_init(&bar.p_full, 16);
-        mbar_init(&bar.pv_done, 1);
-        for (int i = 0; i < kRdStages; ++i) {
-            mbar_init(&bar.a_full[i], 4);
-            mbar_init(&bar.a_empty[i], 1);
-        }
-        for (int i = 0; i < kBStages; ++i) {
-            mbar_init(&bar.b_full[i], 1);
-            mbar_init(&bar.b_empty[i], 1);
-        }
-        mbar_init(&bar.u_full, 1);
-        mbar_init(&bar.done, 1);
-        ctl.abort_flag = 0;
-        int Gh = P.G[h];
-        if (Gh < 1 || Gh > kGMax) {
-            raise_error(OAL_ERR_GROUPS);
-            Gh = Gh < 1 ? 1 : kGMax;
-        }
-        ctl.G = Gh;
-        fence_mbar_init();
-    }
-    __syncthreads();
-    const int G = ctl.G;
-    if (warp == kTmaWarp && lane == 0) {
-        // tiles and the coefficient table first: they do not depend on the setup below
-        mbar_expect_tx(&bar.qkv_full, 3 * kTileBytes + kFP * 4);
-        tma_load_3d(sm + kRdOffQ, P.tm_q, &bar.qkv_full, 0, c * kC, bh);
-        tma_load_3d(sm + kRdOffK, P.tm_k, &bar.qkv_full, 0, c * kC, bkv);
-        tma_load_3d(sm + kRdOffV, P.tm_v, &bar.qkv_full, 0, c * kC, bkv);
-        bulk_g2s(coef, P.coef_all + size_t(h) * kFP, kFP * 4, &bar.qkv_full);
-    }
-    for (int e = threadIdx.x; e < kGM1 * 64; e += blockDim.x) {
-        const int m = e >> 6, r = e & 63;
-        int g = P.gid[h * kD + r];
-        if (g < 1 || g > G) {
-            raise_error(OAL_ERR_GROUPS);
-            g = g < 1 ? 1 : G;
-        }
-        wch[e] = (m <= G) ? P.L[size_t(h) * kGM1 * kGM1 + g * kGM1 + m] * 0.125f : 0.f;
-    }
-    if (threadIdx.x < kGM1) c0[threadIdx.x] = P.L[size_t(h) * kGM1 * kGM1 + threadIdx.x];
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-
-    if (warp == kTmaWarp) {
-        if (lane == 0) {
-            int issued = 0;
-            bool ok = true;
-            if (has_inter && ok) {
-                // slices 2u, 2u + 1 of image (bkv, c) in one copy of 160 rows
-                const int row0 = (bkv * NC + c) * kSlices * 80;
-                for (int u = 0; u < kSlices / 2; ++u) {
-                    const int bs = u % kBStages;
-                    if (u >= kBStages &&
-                        !mbar_wait(&bar.b_empty[bs], ((u / kBStages) - 1) & 1, abort_flag))
-                        break;
-                    // stage 2 is the ones atom until the P [V | 1] MMAs are done
-                    if (u == 2 && !mbar_wait(&bar.pv_done, 0, abort_flag)) break;
-                    mbar_expect_tx(&bar.b_full[bs], kImgPairBytes);
-                    tma_load_2d(sm + rd_bstage_off(bs), P.tm_img, &bar.b_full[bs], 0,
-                                row0 + 160 * u);
-                    ++issued;
-                }
-            }
-            bounded_spin_done(&bar.qkv_full, 0);
-            for (int u = max(0, issued - kBStages); u < issued; ++u)
-                bounded_spin_done(&bar.b_full[u % kBStages], (u / kBStages) & 1);
-        }
-        __syncwarp();
-    } else if (warp == kMmaWarp) {
-        // the whole warp runs the issue loop (waits by every lane); one elected lane issues
-        constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);
-        constexpr uint32_t id_u = idesc_bf16(128, 80, false, false);   // A, B K-major
-        constexpr uint32_t id_pv = idesc_bf16(128, 80, false, true);   // B = [V | ones] MN
-        const uint32_t aq0 = smem_u32(sm + kRdOffAq), kt = smem_u32(sm + kRdOffK);
-        const uint32_t vt = smem_u32(sm + kRdOffV), ones = smem_u32(sm + kRdOffOnes);
-        const uint32_t sm0 = smem_u32(sm);
-        bool ok = mbar_wait(&bar.qkv_full, 0, abort_flag);
-        // grouped score tiles S_m = (Q o w_m) K^T, double-buffered in TMEM
-        for (int m = 0; m <= G && ok; ++m) {
-            const int sb = m & 1;
-            ok = mbar_wait(&bar.aq_full[sb], (m >> 1) & 1, abort_flag);
-            if (ok && m >= 2) ok = mbar_wait(&bar.s_empty[sb], ((m >> 1) - 1) & 1, abort_flag);
-            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-            tc_fence_after();
-            if (elect_one()) {
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16(tmem + kColS0 + sb * 128,
-                             sdesc_sw128(aq0 + sb * kTileBytes + ks * 32, 16, 1024),
-                             sdesc_sw128(kt + ks * 32, 16, 1024), id_s, ks > 0 ? 1u : 0u);
-                mma_commit(&bar.s_full[sb]);
-            }
-            __syncwarp();
-        }
-        // intra-chunk term: U = P [V | 1]
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar.p_full, 0, abort_flag));
-        if (ok) {
-            tc_fence_after();
-            if (elect_one()) {
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    mma_bf16(tmem + kColU,
-                             sdesc_sw128(aq0 + (ks >> 2) * kTileBytes + (ks & 3) * 32, 16, 1024),
-                             sdesc_sw128(vt + ks * 2048, ones - vt, 1024), id_pv,
-                             ks > 0 ? 1u : 0u);
-                mma_commit(&bar.pv_done);  // K, V, Aq | P are free for phi stages 4..7
-            }
-            __syncwarp();
-        }
-        // inter-chunk readout U += phi(Q_c) S_c, two slices (one image stage) per round:
-        // A = phi slices 2u, 2u + 1 (stages (2u) % 8, (2u + 1) % 8), B = image pair u
-        for (int u = 0; u < kSlices / 2 && ok && has_inter; ++u) {
-            const int s0 = 2 * u, bs = u % kBStages;
-            ok = mbar_wait(&bar.a_full[s0 % kRdStages], (s0 / kRdStages) & 1, abort_flag) &&
-                 mbar_wait(&bar.a_full[(s0 + 1) % kRdStages], ((s0 + 1) / kRdStages) & 1,
-                           abort_flag) &&
-                 mbar_wait(&bar.b_full[bs], (u / kBStages) & 1, abort_flag);
-            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-            tc_fence_after();
-            if (elect_one()) {
-#pragma unroll
-                for (int x = 0; x < 2; ++x) {
-                    const int st = (s0 + x) % kRdStages;
-                    const uint32_t bsl = sm0 + rd_bstage_off(bs) + x * kImgSliceBytes;
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_bf16(tmem + kColU,
-                                 sdesc_sw128(sm0 + rd_stage_off(st) + ks * 32, 16, 1024),
-                                 sdesc_sw128(bsl + ks * 32, 16, 1024), id_u, 1u);
-                    mma_commit(&bar.a_empty[st]);
-                }
-                mma_commit(&bar.b_empty[bs]);
-            }
-            __syncwarp();
-        }
-        if (elect_one()) {
-            if (ok) mma_commit(&bar.u_full);
-            mma_commit(&bar.done);
-        }
-        __syncwarp();
-        if (lane == 0) bounded_spin_done(&bar.done, 0);
-        __syncwarp();
-    } else {
-        const int qw = warp & 3, kq = warp >> 2, row = qw * 32 + lane;
-        const unsigned char* qt = sm + kRdOffQ;
-        const uint32_t aq0 = smem_u32(sm + kRdOffAq);
-        const uint32_t lanebase = tmem + (uint32_t(qw * 32) << 16);
-        bool ok = mbar_wait(&bar.qkv_full, 0, abort_flag);
-
-
-        // ---- intra-chunk phase ----
-        // Aq_m = Q o w_m (bf16, K-major); this warp writes dims [16 kq, 16 kq + 16)
-        auto produce_aq = [&](int m) {
-            const uint32_t base = aq0 + (m & 1) * kTileBytes;
-            const float* w = wch + m * 64;
-#pragma unroll
-            for (int x = 0; x < 2; ++x) {
-                const int ch = 2 * kq + x;
-                const uint4 qv = *reinterpret_cast<const uint4*>(qt + kmajor_chunk(row, ch));
-                const float4 wa = *reinterpret_cast<const float4*>(w + 8 * ch);
-                const float4 wb = *reinterpret_cast<const float4*>(w + 8 * ch + 4);
-                sts128(base + kmajor_chunk(row, ch),
-                       pack2(__fmul2_rn(f2(bf16lo_to_f32(qv.x), bf16hi_to_f32(qv.x)), f2(wa.x, wa.y))),
-                       pack2(__fmul2_rn(f2(bf16lo_to_f32(qv.y), bf16hi_to_f32(qv.y)), f2(wa.z, wa.w))),
-                       pack2(__fmul2_rn(f2(bf16lo_to_f32(qv.z), bf16hi_to_f32(qv.z)), f2(wb.x, wb.y))),
-                       pack2(__fmul2_rn(f2(bf16lo_to_f32(qv.w), bf16hi_to_f32(qv.w)), f2(wb.z, wb.w))));
-            }
-            fence_proxy_async();
-            warp_arrive(&bar.aq_full[m & 1]);
-        };
-        // phi slice s of this row -> shared stage s % 8 (kq or kq + 4; K-major, 128B-swizzled
-        // rows)
-        const uint32_t sm0 = smem_u32(sm);
-        auto produce_phi = [&](int s) -> bool {
-            const int st = s % kRdStages;
-            uint32_t w[32];
-            if (s < kOffDiagSlices) phi_offdiag(qt, coefh, s, row, w);
-            else phi_diag(qt, coef, s, row, w);
-            if (s >= kRdStages &&
-                !mbar_wait(&bar.a_empty[st], ((s / kRdStages) - 1) & 1, abort_flag))
-                return false;
-            // first use of a reused stage: the intra-chunk MMAs must be done with it
-            if (s >= kPhiSets && s < kRdStages && !mbar_wait(&bar.pv_done, 0, abort_flag))
-                return false;
-            const uint32_t base = sm0 + rd_stage_off(st);
-#pragma unroll
-            for (int x = 0; x < 8; ++x)
-                sts128(base + kmajor_chunk(row, x), w[4 * x], w[4 * x + 1], w[4 * x + 2],
-                       w[4 * x + 3]);
-            fence_proxy_async();
-            warp_arrive(&bar.a_full[st]);
-            return true;
-        };
-        if (ok) {
-            // bf16 copy of the off-diagonal coefficients (read by phi)
-            for (int i = threadIdx.x; i < kOffDiagRows / 2; i += 16 * 32)
-                coefh[i] = pack_bf16x2(coef[2 * i], coef[2 * i + 1]);
-        }
-        named_bar_sync(1, 16 * 32);
-        if (ok) {
-            // the first phi slice of this set is staged before the intra-chunk phase, so the
-            // readout MMAs can start as soon as the intra-chunk ones are issued
-            if (has_inter) ok = produce_phi(kq);
-            produce_aq(0);
-            if (G >= 1) produce_aq(1);
-        }
-        const bool live = kq <= qw;  // keys [32 kq, 32 kq + 32) vs rows [32 qw, 32 qw + 32)
-        float acc[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) acc[j] = 0.f;
-        for (int m = 0; m <= G && ok; ++m) {
-            const int sb = m & 1;
-            if (!mbar_wait(&bar.s_full[sb], (m >> 1) & 1, abort_flag)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            if (live) {
-                const float cm = c0[m];
-                const uint32_t taddr = lanebase + kColS0 + sb * 128 + 32 * kq;
-                float v[32];
-                tmem_ld16(taddr, *reinterpret_cast<float(*)[16]>(&v[0]));
-                tmem_ld16(taddr + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
-                tmem_ld_wait();
-#pragma unroll
-                for (int i = 0; i < 32; i += 2) {
-                    const float2 t = __fadd2_rn(f2(cm, cm), f2(v[i], v[i + 1]));
-                    const float2 a = __ffma2_rn(t, t, f2(acc[i], acc[i + 1]));
-                    acc[i] = a.x;
-                    acc[i + 1] = a.y;
-                }
-            }
-            tc_fence_before();
-            warp_arrive(&bar.s_empty[sb]);
-            if (m + 2 <= G) produce_aq(m + 2);
-        }
-        if (ok) {
-            // P tile (K-major, 2 K-atoms over the 128 keys; aliases Aq0 | Aq1): keys
-            // [32 kq, 32 kq + 32) are chunks 4 (kq & 1) .. + 3 of atom kq >> 1
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {
-                uint32_t wv[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int j0 = 32 * kq + 8 * x + 2 * e;
-                    const float k0 = (j0 <= row) ? P.eps + acc[8 * x + 2 * e] : 0.f;
-                    const float k1 = (j0 + 1 <= row) ? P.eps + acc[8 * x + 2 * e + 1] : 0.f;
-                    wv[e] = pack_bf16x2(k0, k1);
-                }
-                sts128(aq0 + (kq >> 1) * kTileBytes + kmajor_chunk(row, 4 * (kq & 1) + x),
-                       wv[0], wv[1], wv[2], wv[3]);
-            }
-            fence_proxy_async();
-            warp_arrive(&bar.p_full);
-        }
-        // ---- inter-chunk phase: phi(Q_c) slices kq + 4, kq + 8, ... ----
-        for (int s = kq + kPhiSets; s < kSlices && ok && has_inter; s += kPhiSets)
-            ok = produce_phi(s);
-
-        // ---- epilogue: yhat = u[:64] / u[64], columns [16 kq, 16 kq + 16) of this row ----
-        if (ok) ok = mbar_wait(&bar.u_full, 0, abort_flag);
-        if (ok) {
-            tc_fence_after();
-            float u[16], dz[16];
-            tmem_ld16(lanebase + kColU + 16 * kq, u);
-            tmem_ld16(lanebase + kColU + 64, dz);
-            tmem_ld_wait();
-            const int irow = c * kC + row;
-            if (irow < T) {
-                const float inv = 1.f / dz[0];
-                float4* o = reinterpret_cast<float4*>(P.out + (size_t(bh) * T + irow) * kDV +
-                                                      16 * kq);
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    o[i] = make_float4(u[4 * i] * inv, u[4 * i + 1] * inv, u[4 * i + 2] * inv,
-                                       u[4 * i + 3] * inv);
-            }
-        }
-    }
-}
-
-// ------------------------------------------------------------------------------------------
-// kernels: 0 = chunk deltas (persistent: CTA i takes a contiguous range of units),
-// 1 = readers (one CTA per (b*h, chunk), B*Hq*NC in all).  Both may be launched as programmatic dependents of the
-// preceding kernel in the stream: griddepcontrol.wait orders every read of its outputs.
+// Kernels.  Chunk deltas: persistent, CTA i takes a contiguous range of units.  The scan and
+// the readout may be launched as programmatic dependents of the preceding kernel in the
+// stream: griddepcontrol.wait orders every read of its outputs.
 // ------------------------------------------------------------------------------------------
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
-template <int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
-    prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
-                      const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v,
-                      const __grid_constant__ CUtensorMap tm_img, Params P)
+    delta_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                 Params P)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Ctl& ctl = *reinterpret_cast<Ctl*>(sm + kOffCtl);
     const int warp = threadIdx.x >> 5;
-    P.tm_q = &tm_q;
     P.tm_k = &tm_k;
     P.tm_v = &tm_v;
-    P.tm_img = &tm_img;
 
     if (warp == kMmaWarp) {
         tmem_alloc(&ctl.tmem_base, kTmemCols);
         tmem_relinquish();
     }
-    init_ones_atom(sm + (kMode == 0 ? kOffOnes : kRdOffOnes));
+    init_ones_atom(sm + kOffOnes);
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
@@ -926,20 +510,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     grid_dep_launch();  // the next kernel may start its prologue
     grid_dep_wait();    // outputs of the previous kernel are visible from here on
 
-    if (kMode == 0) {
-        const int units = P.B * P.Hkv * P.NC * kNumSlabs;
-        const int u0 = int((long long)units * blockIdx.x / gridDim.x);
-        const int u1 = int((long long)units * (blockIdx.x + 1) / gridDim.x);
-        if (u1 > u0) delta_item(sm, ctl, tmem, P, u0, u1);
-    } else {
-        // items with an inter-chunk part first, chunk-major with the heads of a chunk adjacent
-        // (they share the chunk's image in L2); the chunk-0 items last, so that the final
-        // partial wave holds short items (chunk 0 has no inter-chunk part unless the call
-        // continues a prefix)
-        const int nbh = P.B * P.Hq, heavy = nbh * (P.NC - 1), idx = blockIdx.x;
-        if (idx < heavy) reader_item(sm, ctl, tmem, P, idx % nbh, 1 + idx / nbh);
-        else reader_item(sm, ctl, tmem, P, idx - heavy, 0);
-    }
+    const int units = P.B * P.Hkv * P.NC * kNumSlabs;
+    const int u0 = int((long long)units * blockIdx.x / gridDim.x);
+    const int u1 = int((long long)units * (blockIdx.x + 1) / gridDim.x);
+    if (u1 > u0) delta_item(sm, ctl, tmem, P, u0, u1);
 
     tc_fence_before();
     __syncthreads();
@@ -948,6 +522,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_dealloc(tmem, kTmemCols);
     }
 }
+
+// A barrier wait by a whole warp (every lane waits; true only if the phase completed for all).
+__device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, volatile int* abort_flag)
+{
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+}
+
+// The same for warps whose waits are long or off the critical path: suspended while waiting.
+__device__ __forceinline__ bool wait_all_sleep(uint64_t* bar, uint32_t parity,
+                                               volatile int* abort_flag)
+{
+    return __all_sync(0xffffffffu, mbar_wait_sleep(bar, parity, abort_flag));
+}
+
+#include "oal_tc_intra.cuh"
+#include "oal_tc_readout.cuh"
 
 // Exclusive prefix over chunks of one (bkv, 64-row slice, 8 columns): image_c =
 // bf16(sum_{c' < c} dS_c') for c >= 1, stored row-major as [80 n][64 f] per slice (the
@@ -964,12 +554,13 @@ __global__ void __launch_bounds__(256) scan_kernel(const float* __restrict__ dS,
                                                    const float* __restrict__ L,
                                                    const int32_t* __restrict__ G, float eps,
                                                    unsigned char* __restrict__ state, int B,
-                                                   int Hq, int Hkv, long long tokens, int cont)
+                                                   int Hq, int Hkv, long long tokens, int cont,
+                                                   unsigned char* __restrict__ rtab)
 {
     grid_dep_launch();
     if (blockIdx.z == gridDim.z - 1) {  // independent of the deltas: no wait
         const int h = blockIdx.y * gridDim.x + blockIdx.x;
-        if (h < Hq) prep_head(h, gid, L, G, eps, state, B, Hq, Hkv, tokens, cont != 0);
+        if (h < Hq) prep_head(h, gid, L, G, eps, state, B, Hq, Hkv, tokens, cont != 0, rtab);
         return;
     }
     grid_dep_wait();
@@ -1076,16 +667,15 @@ bool make_map(CUtensorMap* m, const void* base, int T, int heads)
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// chunk-state images [slices][80 rows][64] bf16 viewed as 2D {64, slices * 80}; box {64, 160}
-// = two consecutive slices per copy (copies from L2 cost about the same per copy from 8 to
-// 20 KB, so fewer and larger ones); 128B swizzle on the way in.
+// chunk-state images [slices][80 rows][64] bf16 viewed as 2D {64, slices * 80}; box {64, 80}
+// = one slice per copy; 128B swizzle on the way in.
 bool make_img_map(CUtensorMap* m, const void* base, size_t slices)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[2] = {64, cuuint64_t(slices) * 80};
     const cuuint64_t strides[1] = {128};
-    const cuuint32_t box[2] = {64, 160};
+    const cuuint32_t box[2] = {64, 80};
     const cuuint32_t estr[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -1108,10 +698,19 @@ size_t tc_image_bytes(int B, int Hkv, int T)
     return size_t(B) * Hkv * NC * tc::kImgChunkBytes;
 }
 
-size_t tc_workspace_bytes(int B, int Hkv, int T)
+static size_t tc_delta_bytes(int B, int Hkv, int T)
 {
     const size_t NC = size_t((T + tc::kC - 1) / tc::kC);
-    return tc_image_bytes(B, Hkv, T) + size_t(B) * Hkv * NC * kW * kFP * 4;
+    return size_t(B) * Hkv * NC * kW * kFP * 4;
+}
+
+// normalisers of the intra-chunk sums, [B*Hq][T] fp32
+static size_t tc_zin_bytes(int B, int Hq, int T) { return align256(size_t(B) * Hq * T * 4); }
+
+size_t tc_workspace_bytes(int B, int Hq, int Hkv, int T)
+{
+    return tc_image_bytes(B, Hkv, T) + tc_delta_bytes(B, Hkv, T) + size_t(Hq) * kTabBytes +
+           tc_zin_bytes(B, Hq, T);
 }
 
 namespace {
@@ -1163,9 +762,11 @@ int launch_prefill_tc(const void* q, const void* k, const void* v, const int32_t
     P.L = L;
     P.G = G;
     P.eps = eps;
-    P.coef_all = reinterpret_cast<const float*>(sb + kHeaderBytes);
     P.img = wsb;
     P.dS = reinterpret_cast<float*>(wsb + tc_image_bytes(B, Hkv, T));
+    unsigned char* rtab = wsb + tc_image_bytes(B, Hkv, T) + tc_delta_bytes(B, Hkv, T);
+    P.rtab = rtab;
+    float* zin = reinterpret_cast<float*>(rtab + size_t(Hq) * kTabBytes);
     P.out = out;
     P.B = B;
     P.Hq = Hq;
@@ -1174,30 +775,46 @@ int launch_prefill_tc(const void* q, const void* k, const void* v, const int32_t
     P.NC = NC;
     P.cont = cont ? 1 : 0;
     const int units = B * Hkv * NC * tc::kNumSlabs;
-    const int grid0 = std::max(1, std::min(sm_count(), units));
-    OAL_CUDA_TRY(cudaFuncSetAttribute(tc::prefill_tc_kernel<0>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const int nsm = sm_count();
+    const int grid0 = std::max(1, std::min(nsm, units));
+    OAL_CUDA_TRY(cudaFuncSetAttribute(tc::delta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       int(tc::kSmemBytes)));
-    OAL_CUDA_TRY(cudaFuncSetAttribute(tc::prefill_tc_kernel<1>,
+    OAL_CUDA_TRY(cudaFuncSetAttribute(tc::intra::intra_kernel,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      int(tc::kSmemBytes)));
+                                      int(tc::intra::kSmemBytes)));
+    OAL_CUDA_TRY(cudaFuncSetAttribute(tc::rd::readout_kernel,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      int(tc::rd::kSmemBytes)));
+    // two intra-chunk CTAs per SM need the whole shared-memory carve-out
+    OAL_CUDA_TRY(cudaFuncSetAttribute(tc::intra::intra_kernel,
+                                      cudaFuncAttributePreferredSharedMemoryCarveout, 100));
+    if (out != nullptr) {
+        // intra-chunk sums first: they need only q, k, v; chunk 0 of a fresh prefill is final
+        LaunchScope ls("intra_tc", st);
+        OAL_CUDA_TRY(launch_ex(tc::intra::intra_kernel, dim3(NC * B * Hq),
+                               dim3(tc::intra::kThreads), tc::intra::kSmemBytes, st, false, mq, mk,
+                               mv, P, zin));
+    }
     {
         LaunchScope ls("delta_tc", st);
-        OAL_CUDA_TRY(launch_ex(tc::prefill_tc_kernel<0>, dim3(grid0), dim3(tc::kThreads),
-                               tc::kSmemBytes, st, false, mq, mk, mv, mi, P));
+        OAL_CUDA_TRY(launch_ex(tc::delta_kernel, dim3(grid0), dim3(tc::kThreads), tc::kSmemBytes,
+                               st, overlap && out != nullptr, mk, mv, P));
     }
     {
         LaunchScope ls("scan", st);
         OAL_CUDA_TRY(launch_ex(tc::scan_kernel,
                                dim3(tc::kSlices, tc::kImgRows / tc::kScanCols, B * Hkv + 1),
                                dim3(256), 0, st, overlap, (const float*)P.dS, P.img, body, NC,
-                               gid, L, G, eps, sb, B, Hq, Hkv, (long long)T, P.cont));
+                               gid, L, G, eps, sb, B, Hq, Hkv, (long long)T, P.cont, rtab));
     }
     if (out == nullptr) return OAL_OK;  // no out: the state alone is wanted
-    {
+    const int items = B * Hq * (cont ? NC : NC - 1);
+    if (items > 0) {
+        // persistent: one CTA per SM walks the items (b*h, chunk) with an inter-chunk part
+        const int grid2 = std::max(1, std::min(nsm, items));
         LaunchScope ls("readout_tc", st);
-        OAL_CUDA_TRY(launch_ex(tc::prefill_tc_kernel<1>, dim3(NC * B * Hq), dim3(tc::kThreads),
-                               tc::kSmemBytes, st, overlap, mq, mk, mv, mi, P));
+        OAL_CUDA_TRY(launch_ex(tc::rd::readout_kernel, dim3(grid2), dim3(tc::rd::kThreads),
+                               tc::rd::kSmemBytes, st, overlap, mq, mi, P, (const float*)zin));
     }
     return OAL_OK;
 }
