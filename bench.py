@@ -74,6 +74,10 @@ def parse():
     ap.add_argument("--workload", default="config1", choices=["config1", "config3_16k",
                                                               "config3_32k", "config3_64k"],
                     help="prefill workload (config1 is the headline)")
+    ap.add_argument("--no-config2", action="store_true",
+                    help="skip the batched 18-layer prefill (B=8, T=4096) measurement")
+    ap.add_argument("--config2-steps", type=int, default=3,
+                    help="timed passes over the 18 layers of the batched prefill")
     return ap.parse_args()
 
 
@@ -146,10 +150,11 @@ class ClockSampler:
 
 def profiled_traffic(workload_name):
     """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the kernels
-    captured with ncu on the config-1 workload, from the committed profile summary."""
+    captured with ncu on the config-1 workload, from the committed profile summary of the
+    current kernels (none: null)."""
     if workload_name != "config1":
         return {}
-    path = os.path.join(ROOT, "profiles", "readout_tc_config1_full.md")
+    path = os.path.join(ROOT, "profiles", "prefill_tc_config1_kernels.md")
     out = {}
     if os.path.exists(path):
         with open(path) as f:
@@ -203,6 +208,69 @@ def prefill_flops(B, T, Hq, Hkv):
     """Algorithmic prefill work: the eq. (4) state update per key/value head plus the eq. (5)
     readout per query head over D = 2145 packed features and dv + 1 = 65 columns."""
     return 2.0 * B * T * F * W * (Hq + Hkv)
+
+
+def kernel_work(p, chunk=128):
+    """Algorithmic work of each kernel of one tensor-core prefill call (bf16, chunk 128):
+    name -> (amount, 'flop' | 'byte').
+      delta_tc   eq. (4) chunk deltas: 2 F W flop per token and key/value head
+      readout_tc eq. (5) over the prefix state: 2 F W flop per query row with an inter-chunk
+                 part (every chunk but the first)
+      intra_tc   eqs. (2)-(3) inside a chunk: per causal pair (i, j <= i in the same chunk)
+                 2 * 64 (G + 1) flop for the G + 1 factored score products and 2 * 65 for
+                 kappa [v; 1]
+      scan       bytes: fp32 deltas read once, bf16 state images written once (80 rows of
+                 64 per 64 packed rows), the fp32 final state written once"""
+    B, Hq, T, _ = p.q.shape
+    Hkv = p.k.shape[1]
+    NC = -(-T // chunk)
+    rows_inter = max(0, T - chunk)
+    pairs = 0
+    for c in range(NC):
+        n = min(chunk, T - c * chunk)
+        pairs += n * (n + 1) // 2
+    per_pair = sum(2.0 * 64 * (int(g) + 1) + 2.0 * W for g in p.G)  # summed over heads
+    slices = 2176 // 64
+    return {
+        "delta_tc": (2.0 * B * Hkv * T * F * W, "flop"),
+        "readout_tc": (2.0 * B * Hq * rows_inter * F * W, "flop"),
+        "intra_tc": (B * pairs * per_pair, "flop"),
+        "scan": (B * Hkv * (NC * W * 2176 * 4 + (NC - 1) * slices * 80 * 64 * 2
+                            + 2176 * W * 4), "byte"),
+    }
+
+
+def kernel_rooflines(prof, work, pk, pk_kind, n_steps):
+    """Per-kernel achieved rate from the library's CUDA-event trace (name -> (launches, ms))
+    against the measured peaks: tensor-core kernels against the bf16 peak, the scan against
+    HBM copy bandwidth (its data stays in the L2, so it can read above 1), CUDA-core kernels
+    against the fp32 ALU peak."""
+    out = {}
+    total = sum(t for _, t in prof.values()) or 1.0
+    for name, (nl, ms) in prof.items():
+        per = ms / nl
+        amount, kind = work.get(name, (None, None))
+        if amount is None:
+            alu = 148 * 128 * 2 * pk.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+            out[name] = {"bound": "alu", "avg_launch_ms": per, "peak": alu, "unit": "TFLOP/s",
+                         "share": t_share(ms, total)}
+            continue
+        if kind == "flop":
+            ach = amount / (per / 1e3) / 1e12
+            out[name] = {"bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops"],
+                         "algorithmic_per_launch": amount, "avg_launch_ms": per,
+                         "share": t_share(ms, total), "peak_kind": pk_kind}
+        else:
+            ach = amount / (per / 1e3) / 1e9
+            out[name] = {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": ach / pk["hbm_gbs"], "algorithmic_per_launch": amount,
+                         "avg_launch_ms": per, "share": t_share(ms, total), "peak_kind": pk_kind}
+    return out
+
+
+def t_share(ms, total):
+    return round(ms / total, 4)
 
 
 def cpu_baseline(p, budget_s=12.0):
@@ -320,30 +388,20 @@ def main():
     total_ms = max_over_ranks(sum(step_ms), world, dev)
     value = job_rate(world, args.steps * B * T, total_ms)
 
-    # roofline of the dominant prefill kernel
-    flops_state = 2.0 * B * T * F * W * Hkv
-    flops_read = 2.0 * B * T * F * W * Hq
-    dom = max(prof.items(), key=lambda kv: kv[1][1]) if prof else None
+    # roofline of the dominant prefill kernel (largest share of the device time)
+    per_kernel = kernel_rooflines(prof, kernel_work(p, args.chunk), pk, pk_kind, args.steps)
     roof = None
-    if dom is not None:
-        name, (nl, ms) = dom
-        per = ms / nl
-        algo = flops_read if name.startswith("readout") else (
-            flops_state if name.startswith(("state", "delta")) else prefill_flops(B, T, Hq, Hkv))
-        tensor = name.endswith("_tc")
-        if tensor:
-            peak, unit, bound = pk["bf16_tflops"], "TFLOP/s", "tensor"
-        else:
-            # fp32 FMA on CUDA cores: 148 SMs x 128 lanes x 2 flop x max SM clock
-            peak, unit, bound = 148 * 128 * 2 * pk.get("sm_max_mhz", 1965.0) * 1e6 / 1e12, \
-                "TFLOP/s", "alu"
-        ach = algo / (per / 1e3) / 1e12
-        roof = {"bound": bound, "achieved": ach, "peak": peak, "unit": unit, "frac": ach / peak,
+    if per_kernel:
+        name = max(per_kernel, key=lambda n: per_kernel[n]["share"])
+        d = per_kernel[name]
+        roof = {"bound": d["bound"], "achieved": d.get("achieved"), "peak": d["peak"],
+                "unit": d["unit"], "frac": d.get("frac"),
                 "traffic": profiled_traffic(args.workload).get(name), "kernel": name,
-                "avg_launch_ms": per,
-                "algorithmic_flop_per_launch": algo, "peak_kind": pk_kind,
-                "kernel_shares": {n: round(t / sum(x[1] for x in prof.values()), 4)
-                                  for n, (c, t) in prof.items()},
+                "avg_launch_ms": d["avg_launch_ms"],
+                "algorithmic_per_launch": d.get("algorithmic_per_launch"),
+                "peak_kind": pk_kind,
+                "kernel_shares": {n: v["share"] for n, v in per_kernel.items()},
+                "kernels": per_kernel,
                 "whole_step_frac_of_bf16_peak": prefill_flops(B, T, Hq, Hkv) /
                 (total_ms / args.steps / 1e3) / 1e12 / pk["bf16_tflops"]}
 
@@ -360,6 +418,13 @@ def main():
     decode = None
     if not args.no_decode:
         decode = run_decode(args, dev, torch, oal, pk, pk_kind, flush, world, barrier)
+
+    config2 = None
+    if not args.no_config2:
+        try:
+            config2 = run_config2(args, dev, torch, oal, pk, pk_kind, flush, world, barrier)
+        except Exception as exc:  # recorded in the line; the headline value stands
+            config2 = {"error": repr(exc)[:300]}
 
     extras = None
     if not args.no_extras:
@@ -379,7 +444,8 @@ def main():
                            "l2": flush.describe(),
                            "parallelism": f"replicas x{world}"},
                 "roofline": roof, "e2e": e2e, "gpu_launches": int(n_launch),
-                "clocks": clk.summary(), "decode": decode, "extras": extras, "cpu_baseline": base,
+                "clocks": clk.summary(), "decode": decode, "config2": config2, "extras": extras,
+                "cpu_baseline": base,
                 "step_ms_min": min(step_ms), "step_ms_median": statistics.median(step_ms)}
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -526,6 +592,63 @@ def oracle_free_hadamard_coefs(Hq, d=64):
     W = rng.standard_normal((Hq, d, d))
     C = W @ W.transpose(0, 2, 1) / d + 0.5 * np.eye(d)
     return a, b, C
+
+
+def run_config2(args, dev, torch, oal, pk, pk_kind, flush, world, barrier):
+    """Batched prefill of the 18 converted layers (3-20) of a Qwen2.5-0.5B-shaped model:
+    B=8, T=4096, 14/2 heads, bf16, each layer with its own seeded inputs, groups and L.  One
+    pass = one oal_prefill per layer; tokens/s = B*T tokens through all 18 layers per pass.
+    Inputs resident in HBM, the L2 flushed between passes (outside the timed events)."""
+    from positive_quadratic_b200 import inputs as I
+    layers = []
+    for l in range(18):
+        p = I.config2_layer(l)
+        layers.append(to_dev(p, dev, torch) + (p.eps,))
+    q0 = layers[0][0]
+    B, Hq, T, _ = q0.shape
+    Hkv = layers[0][1].shape[1]
+    out = torch.empty(B, Hq, T, 64, dtype=torch.float32, device=dev)
+    shape = oal.make_shape(B, T, Hq, Hkv, 128, oal.OAL_BF16)
+    ws = oal.empty_workspace(oal.prefill_workspace_bytes(shape), dev)
+    states = [oal.prefill(*layers[l][:6], layers[l][6], 128, out=out, workspace=ws)[1]
+              for l in range(18)]
+
+    def one_pass():
+        for l in range(18):
+            q, k, v, g, L, G, eps = layers[l]
+            oal.prefill(q, k, v, g, L, G, eps, 128, out=out, state=states[l], workspace=ws)
+
+    one_pass()
+    flush()
+    torch.cuda.synchronize()
+    assert oal.device_error() == 0
+    stream = torch.cuda.current_stream()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.config2_steps)]
+    oal.profile_read()
+    oal.profile_enable(True)
+    barrier()
+    torch.cuda.synchronize()
+    for s0, s1 in evs:
+        s0.record(stream)
+        one_pass()
+        s1.record(stream)
+        flush()
+    torch.cuda.synchronize()
+    oal.profile_enable(False)
+    prof = oal.profile_read()
+    assert oal.device_error() == 0
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world, dev)
+    per_pass = ms / args.config2_steps
+    flops = 18 * prefill_flops(B, T, Hq, Hkv)
+    total = sum(t for _, t in prof.values()) or 1.0
+    return {"value": job_rate(world, args.config2_steps * B * T, ms), "unit": UNIT,
+            "ms_per_pass": per_pass, "passes": args.config2_steps,
+            "workload": "18 layers, B=8 T=4096 Hq=14 Hkv=2 d=64 bf16, chunk 128; tokens/s "
+                        "through all 18 layers",
+            "whole_pass_frac_of_bf16_peak": flops / (per_pass / 1e3) / 1e12 / pk["bf16_tflops"],
+            "algorithmic_flop_per_pass": flops, "peak_kind": pk_kind,
+            "kernel_shares": {n: round(t / total, 4) for n, (c, t) in prof.items()}}
 
 
 def run_decode(args, dev, torch, oal, pk, pk_kind, flush, world, barrier):

@@ -375,9 +375,12 @@ __global__ void __launch_bounds__(256) readout_simt_kernel(
 // a11: decode step.  Block (slab, bkv) streams 240 packed rows of one (b, kv) state once:
 // S_f += psi_f(k) [v; 1] (eq. (4) with one new token), then accumulates
 // u_h += phi_{h,f}(q_h) S_f for the Hq/Hkv query heads of that kv head (eq. (5)).  Row data
-// moves as 128-bit loads and stores (a half warp per 256-byte row).  Per-block partial u go
-// to the workspace; the last block of a (b, kv) (atomic ticket) sums them, writes yhat and
-// re-arms the ticket.
+// moves as 128-bit loads and stores (a half warp per 256-byte row), the first rows requested
+// before the per-row weights are formed and every batch of rows prefetched while the previous
+// one is computed.  Per-block partial u go to the workspace in a fixed order (warp partials
+// summed in shared memory, no float atomics); the last block of a (b, kv) (atomic ticket)
+// sums the slab partials in slab order, writes yhat and re-arms the ticket.  Every sum has a
+// fixed order, so a step is bit-reproducible.
 // ------------------------------------------------------------------------------------------
 // 9 slabs of 240 packed rows per (b, kv) head: 256 threads with at most 64 registers, so four
 // blocks share an SM (592 resident) and a batch-64 step (1152 blocks) takes 1.95 waves -- the
@@ -385,7 +388,8 @@ __global__ void __launch_bounds__(256) readout_simt_kernel(
 // whole block time.
 constexpr int kDecRows = 240;
 constexpr int kDecThreads = 256;
-constexpr int kDecBatch = 4;  // rows in flight per thread (240 rows = 16 x (4 + 4 + 4 + 3))
+constexpr int kDecBatch = 2;   // rows per thread per batch (a half warp per row); the next batch is in flight
+constexpr int kDecWarps = kDecThreads / 32;
 
 template <typename Tin, int kGrp>  // kGrp = Hq / Hkv query heads per kv head
 __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const Tin* __restrict__ q,
@@ -400,7 +404,7 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const Tin* __res
     const int slab = blockIdx.x, bkv = blockIdx.y, nslab = gridDim.x;
     constexpr int grp = kGrp;
     const int b = bkv / Hkv, kv = bkv % Hkv, h0 = kv * grp;
-    const int tid = threadIdx.x, lane4 = tid & 15, rsub = tid >> 4;
+    const int tid = threadIdx.x, lane4 = tid & 15, rsub = tid >> 4, warp = tid >> 5;
     const float* coef = reinterpret_cast<const float*>(state + kHeaderBytes);
     float* unit = reinterpret_cast<float*>(state + kHeaderBytes + coef_bytes(Hq)) +
                   size_t(bkv) * kFP * kW;
@@ -410,11 +414,25 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const Tin* __res
     __shared__ __align__(16) float vh[kW + 3];
     __shared__ float kh[kDA];
     __shared__ float qh[kMaxGroup][kDA];
-    __shared__ float phis[kDecRows][kMaxGroup + 1];
-    __shared__ float psis[kDecRows];
-    __shared__ float red[kMaxGroup][kW];
+    // per row: phi of the query heads (columns 0..grp-1) and psi (column kPsi); one 32-byte
+    // record up to 7 heads, 48 bytes for 8
+    constexpr int kRec = kGrp <= 7 ? 8 : 12, kPsi = kGrp <= 7 ? 7 : 8;
+    __shared__ __align__(16) float wrow[kDecRows][kRec];
+    __shared__ float red[kDecWarps][kMaxGroup][kW];
     __shared__ float ufin[kMaxGroup][kW];
     __shared__ int s_last;
+
+    const int f0 = slab * kDecRows;
+    const int nrows = max(0, min(kDecRows, kF - f0));
+    constexpr int kRowStep = kDecThreads / 16;  // rows one pass of the block covers
+    // the first batch of rows is requested before anything else
+    float4 hv[kDecBatch];
+#pragma unroll
+    for (int x = 0; x < kDecBatch; ++x) {
+        const int row = rsub + kRowStep * x;
+        if (row < nrows)
+            hv[x] = __ldcs(reinterpret_cast<const float4*>(Hv + size_t(f0 + row) * kDV) + lane4);
+    }
 
     if (tid < kD) {
         kh[tid] = to_f32(k[size_t(bkv) * kD + tid]);
@@ -428,16 +446,18 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const Tin* __res
         const int g = e / kDA, r = e % kDA;
         qh[g][r] = r < kD ? to_f32(q[(size_t(b) * Hq + h0 + g) * kD + r]) : (r == kD ? 1.f : 0.f);
     }
-    for (int e = tid; e < kMaxGroup * kW; e += kDecThreads) (&red[0][0])[e] = 0.f;
     __syncthreads();
-    const int f0 = slab * kDecRows;
-    const int nrows = max(0, min(kDecRows, kF - f0));
     for (int row = tid; row < nrows; row += kDecThreads) {
         const int f = f0 + row;
         const RT rt = feature_rt(f);
-        psis[row] = kh[rt.r] * kh[rt.t];
-        for (int g = 0; g < grp; ++g)
-            phis[row][g] = coef[size_t(h0 + g) * kFP + f] * qh[g][rt.r] * qh[g][rt.t];
+        float w[kRec];
+#pragma unroll
+        for (int g = 0; g < kRec; ++g)
+            w[g] = g < grp ? coef[size_t(h0 + g) * kFP + f] * qh[g][rt.r] * qh[g][rt.t] : 0.f;
+        w[kPsi] = kh[rt.r] * kh[rt.t];
+#pragma unroll
+        for (int x = 0; x < kRec; x += 4)
+            *reinterpret_cast<float4*>(&wrow[row][x]) = make_float4(w[x], w[x + 1], w[x + 2], w[x + 3]);
     }
     __syncthreads();
 
@@ -446,23 +466,30 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const Tin* __res
 #pragma unroll
     for (int g = 0; g < kGrp; ++g) acc[g][0] = acc[g][1] = acc[g][2] = acc[g][3] = 0.f;
     const float4 v4 = *reinterpret_cast<const float4*>(&vh[lane4 * 4]);
-    // rows in batches of kDecBatch: every load of a batch is issued before any store (the
-    // compiler cannot move a load past a store to a possibly aliasing row by itself)
-    constexpr int kRowStep = kDecThreads / 16;
 #pragma unroll 1
     for (int base = rsub; base < nrows; base += kRowStep * kDecBatch) {
-        float4 hv[kDecBatch];
+        // prefetch the next batch (all loads of a batch are issued before its stores)
+        float4 nx[kDecBatch];
 #pragma unroll
         for (int x = 0; x < kDecBatch; ++x) {
-            const int row = base + kRowStep * x;
+            const int row = base + kRowStep * (kDecBatch + x);
             if (row < nrows)
-                hv[x] = __ldcs(reinterpret_cast<const float4*>(Hv + size_t(f0 + row) * kDV) + lane4);
+                nx[x] = __ldcs(reinterpret_cast<const float4*>(Hv + size_t(f0 + row) * kDV) + lane4);
         }
 #pragma unroll
         for (int x = 0; x < kDecBatch; ++x) {
             const int row = base + kRowStep * x;
             if (row < nrows) {
-                const float psi = psis[row];
+                float ph[kRec];
+#pragma unroll
+                for (int y = 0; y < kRec; y += 4) {
+                    const float4 w4 = *reinterpret_cast<const float4*>(&wrow[row][y]);
+                    ph[y] = w4.x;
+                    ph[y + 1] = w4.y;
+                    ph[y + 2] = w4.z;
+                    ph[y + 3] = w4.w;
+                }
+                const float psi = ph[kPsi];
                 float4 h = hv[x];
                 h.x = fmaf(psi, v4.x, h.x);
                 h.y = fmaf(psi, v4.y, h.y);
@@ -471,26 +498,28 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const Tin* __res
                 __stcs(reinterpret_cast<float4*>(Hv + size_t(f0 + row) * kDV) + lane4, h);
 #pragma unroll
                 for (int g = 0; g < kGrp; ++g) {
-                    const float ph = phis[row][g];
-                    acc[g][0] = fmaf(ph, h.x, acc[g][0]);
-                    acc[g][1] = fmaf(ph, h.y, acc[g][1]);
-                    acc[g][2] = fmaf(ph, h.z, acc[g][2]);
-                    acc[g][3] = fmaf(ph, h.w, acc[g][3]);
+                    acc[g][0] = fmaf(ph[g], h.x, acc[g][0]);
+                    acc[g][1] = fmaf(ph[g], h.y, acc[g][1]);
+                    acc[g][2] = fmaf(ph[g], h.z, acc[g][2]);
+                    acc[g][3] = fmaf(ph[g], h.w, acc[g][3]);
                 }
             }
         }
+#pragma unroll
+        for (int x = 0; x < kDecBatch; ++x) hv[x] = nx[x];
     }
     float accz[kGrp];
 #pragma unroll
     for (int g = 0; g < kGrp; ++g) accz[g] = 0.f;
     for (int row = tid; row < nrows; row += kDecThreads) {
-        const float zz = z[f0 + row] + psis[row];
+        const float zz = z[f0 + row] + wrow[row][kPsi];
         z[f0 + row] = zz;
+        const float* ph = wrow[row];
 #pragma unroll
-        for (int g = 0; g < kGrp; ++g) accz[g] = fmaf(phis[row][g], zz, accz[g]);
+        for (int g = 0; g < kGrp; ++g) accz[g] = fmaf(ph[g], zz, accz[g]);
     }
-    // reduce: the two half-warps of a warp hold the same columns; warps meet in shared
-    // memory through atomic adds
+    // fixed-order reduction: the two half-warps of a warp hold the same columns; every warp
+    // writes its partial, then one thread per (head, column) sums the warps in order
 #pragma unroll
     for (int g = 0; g < kGrp; ++g) {
 #pragma unroll
@@ -500,13 +529,18 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const Tin* __res
         for (int o = 16; o > 0; o >>= 1) zz += __shfl_xor_sync(0xffffffffu, zz, o);
         if ((tid & 31) < 16) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) atomicAdd(&red[g][lane4 * 4 + c], acc[g][c]);
+            for (int c = 0; c < 4; ++c) red[warp][g][lane4 * 4 + c] = acc[g][c];
         }
-        if ((tid & 31) == 0) atomicAdd(&red[g][kDV], zz);
+        if ((tid & 31) == 0) red[warp][g][kDV] = zz;
     }
     __syncthreads();
     float* mypart = part + (size_t(bkv) * nslab + slab) * grp * kW;
-    for (int e = tid; e < grp * kW; e += kDecThreads) mypart[e] = red[e / kW][e % kW];
+    for (int e = tid; e < grp * kW; e += kDecThreads) {
+        float sum = 0.f;
+#pragma unroll
+        for (int w = 0; w < kDecWarps; ++w) sum += red[w][e / kW][e % kW];
+        mypart[e] = sum;
+    }
     __threadfence();
     __syncthreads();
     if (tid == 0) {
