@@ -31,6 +31,7 @@
 #include <cuda.h>
 
 #include "oal_common.cuh"
+#include "oal_events.cuh"
 #include "oal_kernels.cuh"
 #include "oal_tc_util.cuh"
 
@@ -49,10 +50,11 @@ constexpr uint32_t kTileBytes = kC * 64 * 2;               // 16384: one 128 x 6
 constexpr uint32_t kOnesAtomBytes = kC * 128;              // 16384: 128 rows x 128 B
 constexpr uint16_t kBf16One = 0x3F80;
 
-constexpr int kWarps = 18;
+constexpr int kWarps = 19;
 constexpr int kThreads = kWarps * 32;
 constexpr int kTmaWarp = 16;
-constexpr int kMmaWarp = 17;
+constexpr int kMmaWarp = 17;   // MMA issuer of the even units (and tensor-memory owner)
+constexpr int kMmaWarpB = 18;  // MMA issuer of the odd units
 constexpr uint32_t kTmemCols = 512;
 
 static_assert(kFP % kSlabRows == 0 && kFP % 64 == 0, "feature padding");
@@ -77,7 +79,7 @@ static_assert(kStOffKV + kKVStages * 2 * kTileBytes <= kStOffA &&
               "delta builder shared-memory and TMEM map");
 struct StBars {
     uint64_t kv_full[kKVStages], kv_empty[kKVStages], a_full[kDAStages], a_empty[kDAStages];
-    uint64_t acc_full[kDAcc], acc_empty[kDAcc], done;
+    uint64_t acc_full[kDAcc], acc_empty[kDAcc], done, done_b;
 };
 struct Ctl {
     union {
@@ -315,6 +317,7 @@ __device__ void delta_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Par
             mbar_init(&bar.acc_empty[i], 8);
         }
         mbar_init(&bar.done, 1);
+        mbar_init(&bar.done_b, 1);
         ctl.abort_flag = 0;
         fence_mbar_init();
     }
@@ -341,13 +344,17 @@ __device__ void delta_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Par
                 bounded_spin_done(&bar.kv_full[i % kKVStages], (i / kKVStages) & 1);
         }
         __syncwarp();
-    } else if (warp == kMmaWarp) {
-        // the whole warp runs the issue loop; one elected lane issues
+    } else if (warp == kMmaWarp || warp == kMmaWarpB) {
+        // two issuers, even and odd units (each unit has its own accumulator): a barrier wait
+        // or commit stalls the issuing thread while the tensor pipe drains its short queue,
+        // and the other issuer's MMAs fill that gap.  The whole warp runs the issue loop; one
+        // elected lane issues.
         constexpr uint32_t id = idesc_bf16(128, 80, true, true);
         const uint32_t a0 = smem_u32(sm + kStOffA), kv0 = smem_u32(sm + kStOffKV);
         const uint32_t ones = smem_u32(sm + kOffOnes);
+        uint64_t* done = warp == kMmaWarp ? &bar.done : &bar.done_b;
         bool ok = true;
-        for (int i = 0; i < nu && ok; ++i) {
+        for (int i = warp == kMmaWarp ? 0 : 1; i < nu && ok; i += 2) {
             const int s = i % kDAcc, st = i % kKVStages;
             if (i >= kDAcc) ok = mbar_wait(&bar.acc_empty[s], ((i / kDAcc) - 1) & 1, abort_flag);
             if (ok) ok = mbar_wait(&bar.kv_full[st], (i / kKVStages) & 1, abort_flag);
@@ -381,9 +388,9 @@ __device__ void delta_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Par
             }
             __syncwarp();
         }
-        if (elect_one()) mma_commit(&bar.done);
+        if (elect_one()) mma_commit(done);
         __syncwarp();
-        if (lane == 0) bounded_spin_done(&bar.done, 0);
+        if (lane == 0) bounded_spin_done(done, 0);
         __syncwarp();
     } else if (warp < 8) {
         const int t = threadIdx.x, j = t & 63, qf = t >> 6;
@@ -682,6 +689,21 @@ bool make_img_map(CUtensorMap* m, const void* base, size_t slices)
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// One helper stream per device, created on first use and kept for the process: the
+// intra-chunk kernel runs on it, forked from and joined back into the caller's stream.
+cudaStream_t helper_stream()
+{
+    constexpr int kMaxDev = 64;
+    static std::mutex mu;
+    static cudaStream_t streams[kMaxDev] = {};
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
+    std::lock_guard<std::mutex> g(mu);
+    if (!streams[dev] && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess)
+        streams[dev] = nullptr;
+    return streams[dev];
+}
+
 int sm_count()
 {
     int dev = 0, n = 0;
@@ -788,17 +810,28 @@ int launch_prefill_tc(const void* q, const void* k, const void* v, const int32_t
     // two intra-chunk CTAs per SM need the whole shared-memory carve-out
     OAL_CUDA_TRY(cudaFuncSetAttribute(tc::intra::intra_kernel,
                                       cudaFuncAttributePreferredSharedMemoryCarveout, 100));
-    if (out != nullptr) {
-        // intra-chunk sums first: they need only q, k, v; chunk 0 of a fresh prefill is final
-        LaunchScope ls("intra_tc", st);
-        OAL_CUDA_TRY(launch_ex(tc::intra::intra_kernel, dim3(NC * B * Hq),
-                               dim3(tc::intra::kThreads), tc::intra::kSmemBytes, st, false, mq, mk,
-                               mv, P, zin));
-    }
+    CallEvents evs;
+    cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+    cudaStream_t st2 = out != nullptr ? helper_stream() : nullptr;
+    if (out != nullptr && st2 == nullptr) return OAL_ERR_CUDA;
+    if (out != nullptr) OAL_CUDA_TRY(evs.make(&ev_fork));
+    if (out != nullptr) OAL_CUDA_TRY(evs.make(&ev_join));
+    if (out != nullptr) OAL_CUDA_TRY(cudaEventRecord(ev_fork, st));
     {
         LaunchScope ls("delta_tc", st);
         OAL_CUDA_TRY(launch_ex(tc::delta_kernel, dim3(grid0), dim3(tc::kThreads), tc::kSmemBytes,
-                               st, overlap && out != nullptr, mk, mv, P));
+                               st, false, mk, mv, P));
+    }
+    if (out != nullptr) {
+        // the intra-chunk sums need only q, k, v: they run on the helper stream beside the
+        // chunk deltas and the scan (latency-bound, they fill SMs the memory-bound scan
+        // leaves idle); chunk 0 of a fresh prefill is final there
+        OAL_CUDA_TRY(cudaStreamWaitEvent(st2, ev_fork, 0));
+        LaunchScope ls("intra_tc", st2);
+        OAL_CUDA_TRY(launch_ex(tc::intra::intra_kernel, dim3(NC * B * Hq),
+                               dim3(tc::intra::kThreads), tc::intra::kSmemBytes, st2, false, mq,
+                               mk, mv, P, zin));
+        OAL_CUDA_TRY(cudaEventRecord(ev_join, st2));
     }
     {
         LaunchScope ls("scan", st);
@@ -809,6 +842,7 @@ int launch_prefill_tc(const void* q, const void* k, const void* v, const int32_t
     }
     if (out == nullptr) return OAL_OK;  // no out: the state alone is wanted
     const int items = B * Hq * (cont ? NC : NC - 1);
+    OAL_CUDA_TRY(cudaStreamWaitEvent(st, ev_join, 0));  // the intra-chunk sums are complete
     if (items > 0) {
         // persistent: one CTA per SM walks the items (b*h, chunk) with an inter-chunk part
         const int grid2 = std::max(1, std::min(nsm, items));
