@@ -201,6 +201,15 @@ int oal_contribution_stat(const void* q, const void* k, float* chi, const oal_sh
  * results.  Process-wide; returns the previous setting. */
 int oal_set_prefill_overlap(int overlap);
 
+/* Test hook for the failure path of the tensor-core kernels.  While on, the inter-chunk
+ * readout kernel of the tensor-core prefill (bf16, chunk 128, T > 128 or a continuation)
+ * issues none of its copies, so every bounded wait in it runs out: after about one second the
+ * kernel sets OAL_ERR_TIMEOUT in the device error word and every role leaves its loop (no copy
+ * or MMA left in flight, tensor memory freed), and the context stays usable.  The output of
+ * that call is undefined; the state and later calls are not affected.  Process-wide; returns
+ * the previous setting.  Off by default; not for production use. */
+int oal_set_debug_skip_copies(int on);
+
 /* Prefill with the ungrouped Hadamard form: eq. (5) with free coefficients, that is
  *   kappa(q, k) = a + sum_r b_r x_r + sum_{r,t} C_rt x_r x_t,   x_r = q_r k_r / sqrt(d_h),
  * the relaxation of the Taylor kernel's shared coefficients that the abstract of arXiv

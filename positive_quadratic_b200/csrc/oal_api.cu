@@ -219,6 +219,8 @@ unsigned long long oal_launch_count(void) { return tracer().launches.load(); }
 
 int oal_set_prefill_overlap(int overlap) { return g_prefill_overlap.exchange(overlap ? 1 : 0); }
 
+int oal_set_debug_skip_copies(int on) { return oal::g_skip_copies.exchange(on ? 1 : 0); }
+
 int oal_profile_enable(int on)
 {
     Tracer& t = tracer();

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cstddef>
+#include <atomic>
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -39,6 +40,9 @@ int launch_prefill_tc(const void* q, const void* k, const void* v, const int32_t
                       const float* L, const int32_t* G, float eps, float* out, void* state,
                       void* ws, int B, int T, int Hq, int Hkv, bool overlap, bool cont,
                       cudaStream_t st);
+
+// test hook of oal_set_debug_skip_copies
+extern std::atomic<int> g_skip_copies;
 
 int launch_chi(const void* q, const void* k, float* chi, int B, int T, int Hq, int Hkv,
                int dtype, cudaStream_t st);

@@ -108,6 +108,7 @@ struct Params {
     float* out;
     int B, Hq, Hkv, T, NC;
     int cont;                // 1: the state already holds a prefix; these tokens continue it
+    int skip_copies;         // test hook: the readout issues no copies, so its waits run out
 };
 
 // ------------------------------------------------------------------------------------------
@@ -704,6 +705,13 @@ cudaStream_t helper_stream()
     return streams[dev];
 }
 
+}  // namespace
+
+// Test hook of oal_set_debug_skip_copies (process-wide).
+std::atomic<int> g_skip_copies{0};
+
+namespace {
+
 int sm_count()
 {
     int dev = 0, n = 0;
@@ -796,6 +804,7 @@ int launch_prefill_tc(const void* q, const void* k, const void* v, const int32_t
     P.T = T;
     P.NC = NC;
     P.cont = cont ? 1 : 0;
+    P.skip_copies = g_skip_copies.load() ? 1 : 0;
     const int units = B * Hkv * NC * tc::kNumSlabs;
     const int nsm = sm_count();
     const int grid0 = std::max(1, std::min(nsm, units));

@@ -238,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      uint32_t(nrows) * kDV * 4, &bar.ui_full);
         };
         int last_pf = -1;  // item index j of the last U_intra copy issued, if not waited for
-        if (qw == 0 && lane == 0 && int(blockIdx.x) < n_items) {
+        if (qw == 0 && lane == 0 && int(blockIdx.x) < n_items && !P.skip_copies) {
             prefetch(blockIdx.x);
             last_pf = 0;
         }
@@ -301,7 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // the staged rows are free for the next copy once all four warps are done
             if (!named_bar_and(1, 128, got)) break;
             const int nidx = idx + gridDim.x;
-            if (qw == 0 && lane == 0 && nidx < n_items) {
+            if (qw == 0 && lane == 0 && nidx < n_items && !P.skip_copies) {
                 prefetch(nidx);
                 last_pf = j + 1;
             }
@@ -356,6 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int issued = 0, lq = -1;
             bool ok = true;
             auto load_q = [&](int jj, int qidx) {
+                if (P.skip_copies) return;
                 int bh, c;
                 item_of(qidx, P, bh, c);
                 const int qb = jj & 1;
@@ -382,10 +383,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
-                    mbar_expect_tx(&bar.b_full[st], kImgSliceBytes);
-                    tma_load_2d(sm + kOffB + st * kImgPairBytes + x * kImgSliceBytes, P.tm_img,
-                                &bar.b_full[st], 0, row0 + 160 * p + 80 * x);
-                    issued = g + 1;
+                    if (!P.skip_copies) {
+                        mbar_expect_tx(&bar.b_full[st], kImgSliceBytes);
+                        tma_load_2d(sm + kOffB + st * kImgPairBytes + x * kImgSliceBytes,
+                                    P.tm_img, &bar.b_full[st], 0, row0 + 160 * p + 80 * x);
+                        issued = g + 1;
+                    }
                     if (x == 0 && p == kSlots && j >= 1 && nidx < n_items) {
                         // buffer (j + 1) & 1 is free once the producers finished item j - 1,
                         // which they have by the time this item's first slot is reused

@@ -78,6 +78,8 @@ def lib() -> ctypes.CDLL:
             L.oal_last_cuda_error.restype = ctypes.c_int
             L.oal_set_prefill_overlap.argtypes = [ctypes.c_int]
             L.oal_set_prefill_overlap.restype = ctypes.c_int
+            L.oal_set_debug_skip_copies.argtypes = [ctypes.c_int]
+            L.oal_set_debug_skip_copies.restype = ctypes.c_int
             L.oal_prefill_host_workspace_bytes.argtypes = [_PS, ctypes.c_int,
                                                            ctypes.POINTER(_SZ)]
             L.oal_prefill_host.argtypes = [_VP] * 6 + [ctypes.c_float, _VP, _VP, _VP, _SZ, _PS,
@@ -526,3 +528,9 @@ def set_prefill_overlap(overlap: bool) -> bool:
     """Launch the tensor-core prefill's scan and readout kernels as programmatic dependents
     (True) or in plain stream order (False); returns the previous setting."""
     return bool(lib().oal_set_prefill_overlap(1 if overlap else 0))
+
+
+def set_debug_skip_copies(on: bool) -> bool:
+    """Test hook: while on, the tensor-core readout issues no copies, so its bounded waits run
+    out and it reports OAL_ERR_TIMEOUT (see include/oal.h); returns the previous setting."""
+    return bool(lib().oal_set_debug_skip_copies(1 if on else 0))
