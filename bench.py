@@ -148,13 +148,13 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def profiled_traffic(workload_name):
+def profiled_traffic(workload_name, summary="prefill_tc_config1_kernels.md"):
     """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the kernels
-    captured with ncu on the config-1 workload, from the committed profile summary of the
+    captured with ncu on the bench workload, from the committed profile summary of the
     current kernels (none: null)."""
     if workload_name != "config1":
         return {}
-    path = os.path.join(ROOT, "profiles", "prefill_tc_config1_kernels.md")
+    path = os.path.join(ROOT, "profiles", summary)
     out = {}
     if os.path.exists(path):
         with open(path) as f:
@@ -704,7 +704,8 @@ def run_decode(args, dev, torch, oal, pk, pk_kind, flush, world, barrier):
         per = kern[1] / kern[0]
         gbs = (state_bytes + io_bytes) / (per / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": gbs / pk["hbm_gbs"], "frac_of_8tbs": gbs / 8000.0, "traffic": None,
+                "frac": gbs / pk["hbm_gbs"], "frac_of_8tbs": gbs / 8000.0,
+                "traffic": profiled_traffic("config1", "decode_batch64_sections.md").get(kname),
                 "kernel": kname, "avg_launch_ms": per, "peak_kind": pk_kind,
                 "algorithmic_bytes_per_launch": state_bytes + io_bytes}
     return {"value": job_rate(world, B * nsteps, ms), "unit": UNIT,
