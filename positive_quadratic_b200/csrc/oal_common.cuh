@@ -50,6 +50,7 @@ constexpr uint32_t kTabCoefT = 3584;   // fp32 [384]: coefficients of rows 1792.
 constexpr uint32_t kTabW = 5120;       // fp32 [9][64]: L_{g(r),m} / sqrt(d_h) (0 for m > G)
 constexpr uint32_t kTabC0 = 7424;      // fp32 [9]: L_{0,m} (0 for m > G)
 constexpr uint32_t kTabG = 7460;       // int32: G of the head (clamped to 1..8)
+constexpr uint32_t kTabPure = 7464;    // uint8 [8]: 1 if the 8 dims of block R share one group
 constexpr uint32_t kTabBytes = 7680;   // a multiple of 256
 
 constexpr uint32_t kStateMagic = 0x534C414Fu;  // "OALS"

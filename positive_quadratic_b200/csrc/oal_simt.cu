@@ -91,7 +91,12 @@ __device__ __forceinline__ void prep_head(int h, const int32_t* __restrict__ gid
         }
         if (tid < kGM1) reinterpret_cast<float*>(tb + kTabC0)[tid] = tid <= Gh ? Lh[tid] : 0.f;
         if (tid == 0) *reinterpret_cast<int*>(tb + kTabG) = Gh;
-        for (uint32_t b = kTabG + 4 + tid; b < kTabBytes; b += blockDim.x) tb[b] = 0;
+        if (tid < 8) {  // block R of 8 dims in a single group: its phi weights depend on t only
+            bool pure = true;
+            for (int a = 1; a < 8; ++a) pure = pure && g[8 * tid + a] == g[8 * tid];
+            tb[kTabPure + tid] = pure ? 1 : 0;
+        }
+        for (uint32_t b = kTabPure + 8 + tid; b < kTabBytes; b += blockDim.x) tb[b] = 0;
     }
     if (h == 0 && tid == 0) {
         StateHeader* hd = reinterpret_cast<StateHeader*>(state);

@@ -456,6 +456,28 @@ __device__ void delta_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Par
 // arithmetic: phi = bf16(bf16(q_r q_t) c) with c rounded to bf16 -- three roundings of 2^-9,
 // the same order as the bf16 operand rounding the tensor core sees anyway, and no fp32 ->
 // bf16 conversions (which issue at a quarter of the FMA rate).
+// The same slice when the 8 dims of block R share one group: the weight of (a, b) is then
+// c_b for every a, so phi = bf16(q_a bf16(c_b q_b)) -- one packed product per pair of rows
+// after the 4 that form c o q over block T (two roundings, as above).
+__device__ __forceinline__ void phi_offdiag_pure(const unsigned char* qt, const uint32_t* coefh,
+                                                 int s, int row, uint32_t (&w)[32])
+{
+    const int rt = c_block_rt[s];
+    const uint4 qr = *reinterpret_cast<const uint4*>(qt + kmajor_chunk(row, rt >> 3));
+    const uint4 qc = *reinterpret_cast<const uint4*>(qt + kmajor_chunk(row, rt & 7));
+    const uint4 c = *reinterpret_cast<const uint4*>(coefh + 32 * s);  // row a = 0 of the slice
+    const uint32_t y[4] = {bmul2(c.x, qc.x), bmul2(c.y, qc.y), bmul2(c.z, qc.z), bmul2(c.w, qc.w)};
+    const uint32_t rr[4] = {qr.x, qr.y, qr.z, qr.w};
+#pragma unroll
+    for (int a = 0; a < 8; ++a) {
+        const uint32_t xa = (a & 1) ? dup_hi(rr[a >> 1]) : dup_lo(rr[a >> 1]);
+        w[4 * a + 0] = bmul2(xa, y[0]);
+        w[4 * a + 1] = bmul2(xa, y[1]);
+        w[4 * a + 2] = bmul2(xa, y[2]);
+        w[4 * a + 3] = bmul2(xa, y[3]);
+    }
+}
+
 __device__ __forceinline__ void phi_offdiag(const unsigned char* qt, const uint32_t* coefh, int s,
                                             int row, uint32_t (&w)[32])
 {

@@ -136,7 +136,11 @@ __device__ __forceinline__ void phi_slice(const unsigned char* qt, const unsigne
                                           int row, uint32_t (&w)[32])
 {
     if (s < kOffDiagSlices) {
-        phi_offdiag(qt, reinterpret_cast<const uint32_t*>(tab + kTabCoefH), s, row, w);
+        const uint32_t* ch = reinterpret_cast<const uint32_t*>(tab + kTabCoefH);
+        if (tab[kTabPure + (c_block_rt[s] >> 3)])  // the same for the whole item
+            phi_offdiag_pure(qt, ch, s, row, w);
+        else
+            phi_offdiag(qt, ch, s, row, w);
         return;
     }
     const float* ct = reinterpret_cast<const float*>(tab + kTabCoefT);
