@@ -569,14 +569,17 @@ __device__ __forceinline__ bool wait_all_sleep(uint64_t* bar, uint32_t parity,
 #include "oal_tc_intra.cuh"
 #include "oal_tc_readout.cuh"
 
-// Exclusive prefix over chunks of one (bkv, 64-row slice, 8 columns): image_c =
+// Exclusive prefix over chunks of one (bkv, 64-row slice, 16 columns): image_c =
 // bf16(sum_{c' < c} dS_c') for c >= 1, stored row-major as [80 n][64 f] per slice (the
-// readout's tensor copy swizzles it into the K-major B-operand layout; rows 65.. are never
-// read), final state = sum over all chunks.  Thread = (n, row pair).
+// readout's tensor copy swizzles rows 0..64 into the K-major B-operand layout; rows 65..79
+// are never written or read -- the readout keeps them zero in shared memory), final state =
+// sum over all chunks.  Thread = (column n, 4 consecutive rows): 16-byte loads, 8 chunks in
+// flight, 8-byte image stores.
 // The last z-plane of the grid instead builds the coefficient tables and the state header
 // (one block per query head), which the readout reads after this kernel.
-constexpr int kScanCols = 8;
+constexpr int kScanCols = 16;
 constexpr int kImgRows = 80;
+constexpr int kScanColGroups = (kW + kScanCols - 1) / kScanCols;  // 5
 __global__ void __launch_bounds__(256) scan_kernel(const float* __restrict__ dS,
                                                    unsigned char* __restrict__ img,
                                                    float* __restrict__ body, int NC,
@@ -595,63 +598,59 @@ __global__ void __launch_bounds__(256) scan_kernel(const float* __restrict__ dS,
     }
     grid_dep_wait();
     const int sl = blockIdx.x, bkv = blockIdx.z;
-    const int nl = threadIdx.x >> 5, p = threadIdx.x & 31;
+    const int nl = threadIdx.x >> 4, rq = threadIdx.x & 15;
     const int n = blockIdx.y * kScanCols + nl;
-    __shared__ float fin[kScanCols][64 + 1];
+    __shared__ float fin[kScanCols][64 + 4];
     float* unit = body + size_t(bkv) * kFP * kW;
     // the prefix before this call: zero, or (continuation) the state's current contents
-    float a0 = 0.f, a1 = 0.f;
-    const int f = sl * 64 + 2 * p, c_first = cont ? 0 : 1;
+    float a[4] = {0.f, 0.f, 0.f, 0.f};
+    const int f = sl * 64 + 4 * rq, c_first = cont ? 0 : 1;
     if (cont && n < kDV) {
-        a0 = unit[size_t(f) * kDV + n];
-        a1 = unit[size_t(f + 1) * kDV + n];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) a[e] = unit[size_t(f + e) * kDV + n];
     } else if (cont && n == kDV) {
-        a0 = unit[size_t(kFP) * kDV + f];
-        a1 = unit[size_t(kFP) * kDV + f + 1];
-    }
-    if (n >= kW && n < kImgRows) {
-        // rows 65..79 of every image: zero (the readout's N = 80 MMA reads them)
-        unsigned char* dst = img + (size_t(bkv) * NC * kSlices + sl) * kImgSliceBytes + n * 128 + 4 * p;
-        for (int c = c_first; c < NC; ++c)
-            *reinterpret_cast<uint32_t*>(dst + size_t(c) * kSlices * kImgSliceBytes) = 0u;
+        const float4 z4 = *reinterpret_cast<const float4*>(unit + size_t(kFP) * kDV + f);
+        a[0] = z4.x; a[1] = z4.y; a[2] = z4.z; a[3] = z4.w;
     }
     if (n < kW) {
-        const float* src = dS + (size_t(bkv) * NC * kW + n) * kFP + sl * 64 + 2 * p;
+        const float* src = dS + (size_t(bkv) * NC * kW + n) * kFP + f;
         unsigned char* dst = img + (size_t(bkv) * NC * kSlices + sl) * kImgSliceBytes +
-                             n * 128 + 4 * p;
+                             n * 128 + 8 * rq;
         const size_t sstride = size_t(kW) * kFP, dstride = size_t(kSlices) * kImgSliceBytes;
-        int c = 0;
-        for (; c + 4 <= NC; c += 4) {
-            float2 d[4];
+        constexpr int kDepth = 8;
+        for (int c0 = 0; c0 < NC; c0 += kDepth) {
+            float4 d[kDepth];
 #pragma unroll
-            for (int x = 0; x < 4; ++x)
-                d[x] = __ldcs(reinterpret_cast<const float2*>(src + (c + x) * sstride));
+            for (int x = 0; x < kDepth; ++x)
+                if (c0 + x < NC)
+                    d[x] = __ldcs(reinterpret_cast<const float4*>(src + (c0 + x) * sstride));
 #pragma unroll
-            for (int x = 0; x < 4; ++x) {
-                if (c + x >= c_first)
-                    *reinterpret_cast<uint32_t*>(dst + (c + x) * dstride) = pack_bf16x2(a0, a1);
-                a0 += d[x].x;
-                a1 += d[x].y;
+            for (int x = 0; x < kDepth; ++x) {
+                const int c = c0 + x;
+                if (c < NC) {
+                    if (c >= c_first)
+                        *reinterpret_cast<uint2*>(dst + c * dstride) =
+                            make_uint2(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]));
+                    a[0] += d[x].x;
+                    a[1] += d[x].y;
+                    a[2] += d[x].z;
+                    a[3] += d[x].w;
+                }
             }
         }
-        for (; c < NC; ++c) {
-            const float2 d = __ldcs(reinterpret_cast<const float2*>(src + c * sstride));
-            if (c >= c_first)
-                *reinterpret_cast<uint32_t*>(dst + c * dstride) = pack_bf16x2(a0, a1);
-            a0 += d.x;
-            a1 += d.y;
-        }
     }
-    fin[nl][2 * p] = a0;
-    fin[nl][2 * p + 1] = a1;
-    __syncthreads();  // every read of the old state in this block precedes the writes below
-    // final state of unit bkv: Hv[f][n] (n < 64), z[f] (n == 64)
-    const int fl = threadIdx.x >> 2, cq = threadIdx.x & 3;
 #pragma unroll
-    for (int x = 0; x < 2; ++x) {
-        const int nn = blockIdx.y * kScanCols + 2 * cq + x;
-        if (nn < kDV) unit[size_t(sl * 64 + fl) * kDV + nn] = fin[2 * cq + x][fl];
-        else if (nn == kDV) unit[size_t(kFP) * kDV + sl * 64 + fl] = fin[2 * cq + x][fl];
+    for (int e = 0; e < 4; ++e) fin[nl][4 * rq + e] = a[e];
+    __syncthreads();  // every read of the old state in this block precedes the writes below
+    // final state of unit bkv: Hv[f][n] (n < 64), z[f] (n == 64); thread = (row, 4 columns)
+    const int fl = threadIdx.x >> 2, cq = threadIdx.x & 3;
+    const int nn0 = blockIdx.y * kScanCols + 4 * cq;
+    if (nn0 + 3 < kDV) {
+        *reinterpret_cast<float4*>(unit + size_t(sl * 64 + fl) * kDV + nn0) =
+            make_float4(fin[4 * cq][fl], fin[4 * cq + 1][fl], fin[4 * cq + 2][fl],
+                        fin[4 * cq + 3][fl]);
+    } else if (nn0 == kDV) {
+        unit[size_t(kFP) * kDV + sl * 64 + fl] = fin[4 * cq][fl];
     }
 }
 
@@ -697,15 +696,16 @@ bool make_map(CUtensorMap* m, const void* base, int T, int heads)
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// chunk-state images [slices][80 rows][64] bf16 viewed as 2D {64, slices * 80}; box {64, 80}
-// = one slice per copy; 128B swizzle on the way in.
+// chunk-state images [slices][80 rows][64] bf16 viewed as 2D {64, slices * 80}; box {64, 65}
+// = rows 0..64 of one slice per copy (rows 65..79 are kept zero in shared memory by the
+// readout and never written by the scan); 128B swizzle on the way in.
 bool make_img_map(CUtensorMap* m, const void* base, size_t slices)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[2] = {64, cuuint64_t(slices) * 80};
     const cuuint64_t strides[1] = {128};
-    const cuuint32_t box[2] = {64, 80};
+    const cuuint32_t box[2] = {64, kW};
     const cuuint32_t estr[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -867,7 +867,7 @@ int launch_prefill_tc(const void* q, const void* k, const void* v, const int32_t
     {
         LaunchScope ls("scan", st);
         OAL_CUDA_TRY(launch_ex(tc::scan_kernel,
-                               dim3(tc::kSlices, tc::kImgRows / tc::kScanCols, B * Hkv + 1),
+                               dim3(tc::kSlices, tc::kScanColGroups, B * Hkv + 1),
                                dim3(256), 0, st, overlap, (const float*)P.dS, P.img, body, NC,
                                gid, L, G, eps, sb, B, Hq, Hkv, (long long)T, P.cont, rtab));
     }

@@ -189,6 +189,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_alloc(&ctl.tmem_base, kTmemCols);
         tmem_relinquish();
     }
+    // image stages: copies fill rows 0..64 of each slice; rows 65..79 (the N = 80 padding of
+    // the MMA) stay zero from here on
+    for (int i = threadIdx.x; i < int(kSlots * kImgPairBytes / 16); i += blockDim.x)
+        reinterpret_cast<uint4*>(sm + kOffB)[i] = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -388,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     if (!P.skip_copies) {
-                        mbar_expect_tx(&bar.b_full[st], kImgSliceBytes);
+                        mbar_expect_tx(&bar.b_full[st], kImgLoadBytes);
                         tma_load_2d(sm + kOffB + st * kImgPairBytes + x * kImgSliceBytes,
                                     P.tm_img, &bar.b_full[st], 0, row0 + 160 * p + 80 * x);
                         issued = g + 1;
