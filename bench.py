@@ -433,7 +433,7 @@ def main():
 
     extras = None
     if not args.no_extras:
-        extras = run_extras(dev, torch, oal)
+        extras = run_extras(dev, torch, oal, pk)
     base = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         base = cpu_baseline(p)
@@ -524,9 +524,10 @@ def run_e2e(args, dev, torch, oal, p, q, k, v, g, L, G, out, B, T, flush, barrie
     return e2e
 
 
-def run_extras(dev, torch, oal):
+def run_extras(dev, torch, oal, pk):
     """Small timings of the further paths on this rank (no cross-rank reduction): the
-    Hadamard-form prefill, a variable-length batch over four streams and the dense backward.
+    Hadamard-form prefill, a variable-length batch over four streams, long-context prefill
+    with its chunk-size sweep, and the dense backward.
     Each is timed with CUDA events after warm-up; a failure is recorded, not raised."""
     from positive_quadratic_b200 import inputs as I
     res = {}
@@ -573,6 +574,33 @@ def run_extras(dev, torch, oal):
                                  "ms": ms, "tokens_per_s": sum(lens) / (ms / 1e3)}
     except Exception as exc:
         res["varlen_prefill"] = {"error": repr(exc)[:300]}
+    try:  # long-context prefill (config 3) and its chunk-size sweep
+        sweep = {}
+        for T, chunks in ((16384, (64, 128, 256)), (32768, (128,)), (65536, (128,))):
+            p = I.config3(T)
+            q, k, v, g, L, G = to_dev(p, dev, torch)
+            out = torch.empty(1, 14, T, 64, dtype=torch.float32, device=dev)
+            for C in chunks:
+                ws = oal.empty_workspace(oal.prefill_workspace_bytes(
+                    oal.make_shape(1, T, 14, 2, C, oal.OAL_BF16)), dev)
+                st = oal.prefill(q, k, v, g, L, G, p.eps, C, out=out, workspace=ws)[1]
+                ms = timed(lambda: oal.prefill(q, k, v, g, L, G, p.eps, C, out=out, state=st,
+                                               workspace=ws), reps=3)
+                sweep[f"T{T}_C{C}"] = {
+                    "ms": ms, "tokens_per_s": T / (ms / 1e3),
+                    "path": "tensor cores (bf16 operands, fp32 accumulation)"
+                    if oal.prefill_path(oal.make_shape(1, T, 14, 2, C, oal.OAL_BF16))
+                    == oal.OAL_PATH_TENSOR else "CUDA cores (fp32)",
+                    "frac_of_bf16_peak": prefill_flops(1, T, 14, 2) / (ms / 1e3) / 1e12
+                    / pk["bf16_tflops"]}
+                del ws
+            del q, k, v, out
+        res["config3_long_context"] = {
+            "workload": "B=1 Hq=14 Hkv=2 d=64 bf16, chunk swept at T=16384 (64 and 256 run on "
+                        "the fp32 CUDA-core path; 128 is the tensor-core tile height)",
+            "points": sweep}
+    except Exception as exc:
+        res["config3_long_context"] = {"error": repr(exc)[:300]}
     try:  # dense backward, reference scale
         p = I.small_layer(905, B=1, T=256, Hq=14, Hkv=2, dtype="bf16")
         q, k, v = (to(x, torch.bfloat16) for x in (p.q, p.k, p.v))

@@ -107,8 +107,18 @@ int oal_state_bytes(const oal_shape* s, size_t* bytes);
 /* Scratch needed by oal_prefill for `s` (all fields used).  The contents need no
  * initialisation and are meaningless after the call.  On the tensor-core path (bf16, chunk
  * 128) it holds the bf16 chunk-state images and the fp32 chunk deltas, 913,920 bytes per
- * (b, kv head, chunk of 128 tokens); on the CUDA-core path the fp32 chunk states. */
+ * (b, kv head, chunk of 128 tokens), plus one 7,680-byte readout table per query head and
+ * the fp32 intra-chunk normalisers (4 bytes per (b, query head, token)); on the CUDA-core
+ * path the fp32 chunk states. */
 int oal_prefill_workspace_bytes(const oal_shape* s, size_t* bytes);
+
+/* Which kernels oal_prefill, oal_prefill_continue and oal_prefill_host run for `s`:
+ * *path = OAL_PATH_TENSOR (bf16 inputs, chunk 128: tcgen05 tensor cores, bf16 operands and
+ * fp32 accumulation) or OAL_PATH_CUDA_CORE (fp32 inputs, or chunk 64 or 256: fp32 CUDA-core
+ * kernels).  Both compute eqs. (2)-(5); the choice changes speed and rounding, not the
+ * result's definition.  Returns the shape-validation status of oal_prefill_workspace_bytes. */
+typedef enum { OAL_PATH_CUDA_CORE = 0, OAL_PATH_TENSOR = 1 } oal_path;
+int oal_prefill_path(const oal_shape* s, int* path);
 
 /* Scratch needed by oal_decode_step for `s` (B, Hq, Hkv used).  It MUST be zero-filled once
  * before the first decode call.  Its first 256-byte-aligned block holds one completion ticket

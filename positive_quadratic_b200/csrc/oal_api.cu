@@ -103,6 +103,16 @@ int oal_prefill_workspace_bytes(const oal_shape* s, size_t* bytes)
     return OAL_OK;
 }
 
+int oal_prefill_path(const oal_shape* s, int* path)
+{
+    int rc = check_common(s);
+    if (rc) return rc;
+    if ((rc = check_chunk(s))) return rc;
+    if (!path) return OAL_ERR_NULL;
+    *path = use_tensor_path(s) ? OAL_PATH_TENSOR : OAL_PATH_CUDA_CORE;
+    return OAL_OK;
+}
+
 int oal_decode_workspace_bytes(const oal_shape* s, size_t* bytes)
 {
     const int rc = check_common(s);

@@ -4,22 +4,24 @@
 // section 核心公式, numbered in order of appearance: (2) grouped score, (3) kernel kappa,
 // (4) prefix states, (5) readout.  With the packed feature map of oal_common.cuh, the state
 // of a (b, kv) head after token i is S_i = sum_{j<=i} psi(k_j) [v_j; 1] (2176 x 65) and
-// u_i = phi(q_i)^T S_i.  Chunked with C = 128 tokens, the prefill runs as three kernels:
+// u_i = phi(q_i)^T S_i.  Chunked with C = 128 tokens, the prefill runs as four kernels:
 //
 //   chunk deltas (b, kv, chunk c, slab of 128 packed rows; every unit independent):
 //     producer warps build psi(K_c)^T (MN-major, bf16) in shared memory, split exactly into
-//     hi = bf16(psi) and lo = psi - hi; N=80 MMAs accumulate dS_c = psi(K_c)^T [V_c; 1] in
-//     TMEM (the [.; 1] column comes from a constant "ones" atom addressed through the B
-//     descriptor's leading byte offset) and epilogue warps store it in fp32.
-//   prefix scan (SIMT, memory bound): S_c = sum_{c' < c} dS_c' for every chunk, written as
-//     bf16 K-major B-operand images, and the final state S_NC in fp32 (eq. 4 in chunk form).
-//   readout (b, h, chunk c): 128 query rows of one head.  The intra-chunk kernel runs first
-//     on tensor cores in the factored form of eq. (3),
+//     hi = bf16(psi) and lo = psi - hi; N=80 MMAs, issued by two warps (even and odd units),
+//     accumulate dS_c = psi(K_c)^T [V_c; 1] in TMEM (the [.; 1] column comes from a constant
+//     "ones" atom addressed through the B descriptor's leading byte offset) and epilogue
+//     warps store it in fp32.
+//   intra-chunk part (oal_tc_intra.cuh; b, h, chunk c), on a helper stream beside the deltas
+//     and the scan: the factored form of eq. (3),
 //       kappa = eps + sum_m (L_0m + (q o w_m) . k)^2,   w_m[r] = L_{g(r),m} / sqrt(d)
 //     (= ||L^T sbar||^2): score tiles S_m = (Q o w_m) K^T in TMEM, kappa accumulated in
-//     registers, masked causally and multiplied into [V_c; 1].  Then phi(Q_c) is written
-//     straight into tensor memory (tcgen05.st) slice by slice and multiplied with the image
-//     of S_c by N=80 MMAs reading A from TMEM, into the same accumulator; finally
+//     registers, masked causally and multiplied into [V_c; 1].
+//   prefix scan (SIMT, memory bound): S_c = sum_{c' < c} dS_c' for every chunk, written as
+//     bf16 images of the B operand, and the final state S_NC in fp32 (eq. 4 in chunk form).
+//   inter-chunk readout (oal_tc_readout.cuh; persistent over items b, h, chunk c): phi(Q_c)
+//     is written into tensor memory slice pair by slice pair and multiplied with the image of
+//     S_c by N=80 MMAs reading A from TMEM; the epilogue adds the intra-chunk sum and writes
 //     yhat = u[:64] / u[64] (eq. 5).
 //
 // Every wait is bounded (1 s); one that runs out sets OAL_ERR_TIMEOUT and the CTA leaves its
@@ -97,7 +99,7 @@ struct Params {
     const CUtensorMap* tm_q;
     const CUtensorMap* tm_k;
     const CUtensorMap* tm_v;
-    const CUtensorMap* tm_img;  // chunk-state images as {64 f, slices * 80 rows}, box {64, 160}
+    const CUtensorMap* tm_img;  // chunk-state images as {64 f, slices * 80 rows}, box {64, 65}
     const int32_t* gid;
     const float* L;
     const int32_t* G;
@@ -294,7 +296,7 @@ __device__ __forceinline__ DeltaUnit delta_unit(int u, int NC)
 // ------------------------------------------------------------------------------------------
 // chunk-delta item: units [u0, u1), each dS_c = psi(K_c)^T [V_c; 1] for the 128 packed rows
 // of one slab, stored in fp32 as dS[bkv][c][n][f] (n = column of [v; 1]).
-// Warps 0-7 psi producers, 8-15 epilogue, 16 TMA, 17 MMA.
+// Warps 0-7 psi producers, 8-15 epilogue, 16 TMA, 17 and 18 MMA (even and odd units).
 // ------------------------------------------------------------------------------------------
 __device__ void delta_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Params& P, int u0,
                            int u1)

@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(HERE, "liboal.so")
 HEADER = os.path.join(os.path.dirname(HERE), "include", "oal.h")
 
 OAL_F32, OAL_BF16 = 0, 1
+OAL_PATH_CUDA_CORE, OAL_PATH_TENSOR = 0, 1
 HEAD_DIM = VALUE_DIM = 64
 G_MAX = 8
 FEATURES, FEATURES_PAD = 2145, 2176
@@ -67,6 +68,8 @@ def lib() -> ctypes.CDLL:
             for name in ("oal_state_bytes", "oal_prefill_workspace_bytes",
                          "oal_decode_workspace_bytes"):
                 getattr(L, name).argtypes = [_PS, ctypes.POINTER(_SZ)]
+            L.oal_prefill_path.argtypes = [_PS, ctypes.POINTER(ctypes.c_int)]
+            L.oal_prefill_path.restype = ctypes.c_int
             L.oal_prefill.argtypes = [_VP] * 6 + [ctypes.c_float, _VP, _VP, _VP, _SZ, _PS, _VP]
             L.oal_prefill_continue.argtypes = L.oal_prefill.argtypes
             L.oal_decode_step.argtypes = [_VP] * 6 + [_SZ, _PS, _VP]
@@ -177,6 +180,13 @@ def prefill_workspace_bytes(shape: Shape) -> int:
     _check(lib().oal_prefill_workspace_bytes(ctypes.byref(shape), ctypes.byref(n)),
            "oal_prefill_workspace_bytes")
     return n.value
+
+
+def prefill_path(shape: Shape) -> int:
+    """OAL_PATH_TENSOR or OAL_PATH_CUDA_CORE: the kernels oal_prefill runs for `shape`."""
+    p = ctypes.c_int()
+    _check(lib().oal_prefill_path(ctypes.byref(shape), ctypes.byref(p)), "oal_prefill_path")
+    return p.value
 
 
 def decode_workspace_bytes(shape: Shape) -> int:

@@ -45,6 +45,19 @@ def test_shape_validation(field, value, code):
     assert oal.lib().oal_prefill_workspace_bytes(ctypes.byref(s), ctypes.byref(n)) == code
 
 
+def test_prefill_path_query():
+    assert oal.prefill_path(oal.make_shape(1, 4096, 14, 2, 128, oal.OAL_BF16)) == \
+        oal.OAL_PATH_TENSOR
+    for chunk, dt in ((64, oal.OAL_BF16), (256, oal.OAL_BF16), (128, oal.OAL_F32)):
+        assert oal.prefill_path(oal.make_shape(1, 4096, 14, 2, chunk, dt)) == \
+            oal.OAL_PATH_CUDA_CORE
+    s = oal.make_shape(1, 256, 14, 2, 96, oal.OAL_BF16)
+    p = ctypes.c_int()
+    assert oal.lib().oal_prefill_path(ctypes.byref(s), ctypes.byref(p)) == -3
+    s.chunk = 128
+    assert oal.lib().oal_prefill_path(ctypes.byref(s), None) == -1
+
+
 def test_group_size_limit():
     s = oal.make_shape(1, 16, 16, 1)
     n = ctypes.c_size_t()
