@@ -552,8 +552,16 @@ def run_extras(dev, torch, oal, pk):
         q, k, v = (to(x, torch.bfloat16) for x in (p.q, p.k, p.v))
         a, b, C = (to(x, torch.float32) for x in oracle_free_hadamard_coefs(14))
         ms = timed(lambda: oal.prefill_hadamard(q, k, v, a, b, C, 64))
-        res["hadamard_prefill"] = {"workload": "B=1 T=2048 Hq=14 Hkv=2 bf16, chunk 64",
+        res["hadamard_prefill"] = {"workload": "B=1 T=2048 Hq=14 Hkv=2 bf16, chunk 64 "
+                                               "(CUDA cores, fp32)",
                                    "ms": ms, "tokens_per_s": 2048 / (ms / 1e3)}
+        p = I.small_layer(907, B=1, T=4096, Hq=14, Hkv=2, dtype="bf16")
+        q, k, v = (to(x, torch.bfloat16) for x in (p.q, p.k, p.v))
+        ms = timed(lambda: oal.prefill_hadamard(q, k, v, a, b, C, 128))
+        res["hadamard_prefill_tc"] = {"workload": "B=1 T=4096 Hq=14 Hkv=2 bf16, chunk 128 "
+                                                  "(tensor cores; intra-chunk part through the "
+                                                  "feature map)",
+                                      "ms": ms, "tokens_per_s": 4096 / (ms / 1e3)}
     except Exception as exc:
         res["hadamard_prefill"] = {"error": repr(exc)[:300]}
     try:  # variable-length batch: 16 sequences of 64..2048 tokens over 4 streams

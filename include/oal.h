@@ -227,8 +227,11 @@ int oal_set_debug_skip_copies(int on);
  * b_r = 2 M_{0,g(r)}, C_rt = M_{g(r),g(t)}).  a [Hq], b [Hq][64], C [Hq][64][64] (row r,
  * column t) fp32 device arrays, 16-byte aligned; only the symmetric part of C matters.  The
  * kernel need not be positive: yhat = u[:dv] / u[dv] is a plain IEEE division.
- * Runs on CUDA cores in fp32 for both dtypes and every chunk size; the intra-chunk part costs
- * O(T * chunk * d_h^2).  Other arguments, the state (eps = 0 in its header; a holds the
+ * bf16 inputs with chunk 128 run on tcgen05 tensor cores: the chunk states, prefix scan and
+ * inter-chunk readout of oal_prefill with this coefficient table, and the intra-chunk part as
+ * Phi(Q_c) Psi(K_c)^T over the 2176 packed rows (bf16 operands, fp32 accumulation).  fp32
+ * inputs, and other chunk sizes, run on CUDA cores in fp32 with an O(T * chunk * d_h^2)
+ * intra-chunk part.  Other arguments, the state (eps = 0 in its header; a holds the
  * constant), the workspace (oal_prefill_workspace_bytes) and errors as oal_prefill.
  * oal_decode_step continues the sequence. */
 int oal_prefill_hadamard(const void* q, const void* k, const void* v, const float* a,

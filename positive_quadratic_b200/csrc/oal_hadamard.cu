@@ -31,7 +31,8 @@ __global__ void __launch_bounds__(256) prep_hadamard_kernel(const float* __restr
                                                             const float* __restrict__ C,
                                                             unsigned char* __restrict__ state,
                                                             int B, int Hq, int Hkv,
-                                                            long long tokens)
+                                                            long long tokens,
+                                                            unsigned char* __restrict__ rtab)
 {
     const int h = blockIdx.x, tid = threadIdx.x;
     const float* bh = b + size_t(h) * kD;
@@ -47,6 +48,17 @@ __global__ void __launch_bounds__(256) prep_hadamard_kernel(const float* __restr
             else val = (double(Ch[rt.r * kD + rt.t]) + double(Ch[rt.t * kD + rt.r])) / 64.0;
         }
         coef[f] = float(val);
+        if (rtab) {  // tensor-core readout table: bf16 off-diagonal coefficients, fp32 the rest
+            unsigned char* tb = rtab + size_t(h) * kTabBytes;
+            if (f < kOffDiagRows)
+                reinterpret_cast<__nv_bfloat16*>(tb + kTabCoefH)[f] = __float2bfloat16_rn(float(val));
+            else
+                reinterpret_cast<float*>(tb + kTabCoefT)[f - kOffDiagRows] = float(val);
+        }
+    }
+    if (rtab) {  // no 8-dim block shares its weights across rows ("pure" flags 0), rest zero
+        unsigned char* tb = rtab + size_t(h) * kTabBytes;
+        for (uint32_t x = kTabW + tid; x < kTabBytes; x += blockDim.x) tb[x] = 0;
     }
     if (h == 0 && tid == 0) {
         StateHeader* hd = reinterpret_cast<StateHeader*>(state);
@@ -209,7 +221,7 @@ static int launch_hadamard_t(const Tin* q, const Tin* k, const Tin* v, const flo
         {
             LaunchScope ls("prep_hadamard", st);
             prep_hadamard_kernel<<<Hq, 256, 0, st>>>(a, b, C, static_cast<unsigned char*>(state),
-                                                    B, Hq, Hkv, T);
+                                                    B, Hq, Hkv, T, nullptr);
             OAL_LAUNCH_CHECK();
         }
         if (B == 0) return OAL_OK;
@@ -275,9 +287,26 @@ int oal_prefill_hadamard(const void* q, const void* k, const void* v, const floa
     if (!a || !b || !C || !state) return OAL_ERR_NULL;
     if ((rc = check_io(s, q, k, v, out))) return rc;
     if (!aligned16(a) || !aligned16(b) || !aligned16(C) || !aligned16(state)) return OAL_ERR_ALIGN;
-    const size_t need = simt_chunk_state_bytes(s);
+    const bool tensor = use_tensor_path(s) && out != nullptr;
+    const size_t need = tensor ? tc_workspace_bytes(s->B, s->Hq, s->Hkv, s->T)
+                               : simt_chunk_state_bytes(s);
     if (need > 0 && (!workspace || workspace_bytes < need)) return OAL_ERR_WORKSPACE;
     if (workspace && !aligned16(workspace)) return OAL_ERR_ALIGN;
+    if (tensor) {
+        // the coefficient tables (state and readout) first; then the tensor-core prefill with
+        // the intra-chunk part through the feature map
+        cudaStream_t st = static_cast<cudaStream_t>(stream);
+        {
+            LaunchScope ls("prep_hadamard", st);
+            prep_hadamard_kernel<<<s->Hq, 256, 0, st>>>(
+                a, b, C, static_cast<unsigned char*>(state), s->B, s->Hq, s->Hkv, s->T,
+                tc_rtab(workspace, s->B, s->Hkv, s->T));
+            OAL_LAUNCH_CHECK();
+        }
+        return launch_prefill_tc(q, k, v, nullptr, nullptr, nullptr, 0.f, out, state, workspace,
+                                 s->B, s->T, s->Hq, s->Hkv, g_prefill_overlap.load() != 0, false,
+                                 st, true);
+    }
     return launch_hadamard(q, k, v, a, b, C, out, state, static_cast<float*>(workspace), s->B,
                            s->T, s->Hq, s->Hkv, s->chunk, s->dtype, false,
                            static_cast<cudaStream_t>(stream));

@@ -33,13 +33,16 @@ int launch_hadamard(const void* q, const void* k, const void* v, const float* a,
 
 int read_device_error(int* code, cudaStream_t st);
 
-// tensor-core (tcgen05) bf16 prefill, chunk 128
+// tensor-core (tcgen05) bf16 prefill, chunk 128.  fm_intra: the coefficient tables and the
+// state header were written by the caller (free coefficients; gid, L, G unused) and the
+// intra-chunk part goes through the feature map.
 size_t tc_image_bytes(int B, int Hkv, int T);
 size_t tc_workspace_bytes(int B, int Hq, int Hkv, int T);
+unsigned char* tc_rtab(void* ws, int B, int Hkv, int T);  // per-head readout tables in ws
 int launch_prefill_tc(const void* q, const void* k, const void* v, const int32_t* gid,
                       const float* L, const int32_t* G, float eps, float* out, void* state,
                       void* ws, int B, int T, int Hq, int Hkv, bool overlap, bool cont,
-                      cudaStream_t st);
+                      cudaStream_t st, bool fm_intra = false);
 
 // test hook of oal_set_debug_skip_copies
 extern std::atomic<int> g_skip_copies;

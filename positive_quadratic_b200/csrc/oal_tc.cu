@@ -570,6 +570,7 @@ __device__ __forceinline__ bool wait_all_sleep(uint64_t* bar, uint32_t parity,
 
 #include "oal_tc_intra.cuh"
 #include "oal_tc_readout.cuh"
+#include "oal_tc_intra_fm.cuh"
 
 // Exclusive prefix over chunks of one (bkv, 64-row slice, 16 columns): image_c =
 // bf16(sum_{c' < c} dS_c') for c >= 1, stored row-major as [80 n][64 f] per slice (the
@@ -577,8 +578,9 @@ __device__ __forceinline__ bool wait_all_sleep(uint64_t* bar, uint32_t parity,
 // are never written or read -- the readout keeps them zero in shared memory), final state =
 // sum over all chunks.  Thread = (column n, 4 consecutive rows): 16-byte loads, 8 chunks in
 // flight, 8-byte image stores.
-// The last z-plane of the grid instead builds the coefficient tables and the state header
-// (one block per query head), which the readout reads after this kernel.
+// With `prep`, the last z-plane of the grid instead builds the coefficient tables and the
+// state header (one block per query head), which the readout reads after this kernel; without
+// it (free coefficients) the caller has written them before the prefill.
 constexpr int kScanCols = 16;
 constexpr int kImgRows = 80;
 constexpr int kScanColGroups = (kW + kScanCols - 1) / kScanCols;  // 5
@@ -590,10 +592,10 @@ __global__ void __launch_bounds__(256) scan_kernel(const float* __restrict__ dS,
                                                    const int32_t* __restrict__ G, float eps,
                                                    unsigned char* __restrict__ state, int B,
                                                    int Hq, int Hkv, long long tokens, int cont,
-                                                   unsigned char* __restrict__ rtab)
+                                                   unsigned char* __restrict__ rtab, int prep)
 {
     grid_dep_launch();
-    if (blockIdx.z == gridDim.z - 1) {  // independent of the deltas: no wait
+    if (prep && blockIdx.z == gridDim.z - 1) {  // independent of the deltas: no wait
         const int h = blockIdx.y * gridDim.x + blockIdx.x;
         if (h < Hq) prep_head(h, gid, L, G, eps, state, B, Hq, Hkv, tokens, cont != 0, rtab);
         return;
@@ -767,6 +769,11 @@ size_t tc_workspace_bytes(int B, int Hq, int Hkv, int T)
            tc_zin_bytes(B, Hq, T);
 }
 
+unsigned char* tc_rtab(void* ws, int B, int Hkv, int T)
+{
+    return static_cast<unsigned char*>(ws) + tc_image_bytes(B, Hkv, T) + tc_delta_bytes(B, Hkv, T);
+}
+
 namespace {
 
 // Launch with the programmatic-dependent attribute: the kernel may be scheduled while its
@@ -793,7 +800,7 @@ cudaError_t launch_ex(void (*kern)(Args...), dim3 grid, dim3 block, size_t smem,
 int launch_prefill_tc(const void* q, const void* k, const void* v, const int32_t* gid,
                       const float* L, const int32_t* G, float eps, float* out, void* state,
                       void* ws, int B, int T, int Hq, int Hkv, bool overlap, bool cont,
-                      cudaStream_t st)
+                      cudaStream_t st, bool fm_intra)
 {
     if (B == 0) return OAL_OK;
     const int NC = (T + tc::kC - 1) / tc::kC;
@@ -818,7 +825,7 @@ int launch_prefill_tc(const void* q, const void* k, const void* v, const int32_t
     P.eps = eps;
     P.img = wsb;
     P.dS = reinterpret_cast<float*>(wsb + tc_image_bytes(B, Hkv, T));
-    unsigned char* rtab = wsb + tc_image_bytes(B, Hkv, T) + tc_delta_bytes(B, Hkv, T);
+    unsigned char* rtab = tc_rtab(ws, B, Hkv, T);
     P.rtab = rtab;
     float* zin = reinterpret_cast<float*>(rtab + size_t(Hq) * kTabBytes);
     P.out = out;
@@ -837,6 +844,9 @@ int launch_prefill_tc(const void* q, const void* k, const void* v, const int32_t
     OAL_CUDA_TRY(cudaFuncSetAttribute(tc::intra::intra_kernel,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       int(tc::intra::kSmemBytes)));
+    OAL_CUDA_TRY(cudaFuncSetAttribute(tc::fm::intra_fm_kernel,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      int(tc::fm::kSmemBytes)));
     OAL_CUDA_TRY(cudaFuncSetAttribute(tc::rd::readout_kernel,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       int(tc::rd::kSmemBytes)));
@@ -860,18 +870,26 @@ int launch_prefill_tc(const void* q, const void* k, const void* v, const int32_t
         // chunk deltas and the scan (latency-bound, they fill SMs the memory-bound scan
         // leaves idle); chunk 0 of a fresh prefill is final there
         OAL_CUDA_TRY(cudaStreamWaitEvent(st2, ev_fork, 0));
-        LaunchScope ls("intra_tc", st2);
-        OAL_CUDA_TRY(launch_ex(tc::intra::intra_kernel, dim3(NC * B * Hq),
-                               dim3(tc::intra::kThreads), tc::intra::kSmemBytes, st2, false, mq,
-                               mk, mv, P, zin));
+        if (fm_intra) {  // free coefficients: Phi(Q_c) Psi(K_c)^T through the feature map
+            LaunchScope ls("intra_fm_tc", st2);
+            OAL_CUDA_TRY(launch_ex(tc::fm::intra_fm_kernel, dim3(NC * B * Hq),
+                                   dim3(tc::fm::kThreads), tc::fm::kSmemBytes, st2, false, mq,
+                                   mk, mv, P, zin));
+        } else {
+            LaunchScope ls("intra_tc", st2);
+            OAL_CUDA_TRY(launch_ex(tc::intra::intra_kernel, dim3(NC * B * Hq),
+                                   dim3(tc::intra::kThreads), tc::intra::kSmemBytes, st2, false,
+                                   mq, mk, mv, P, zin));
+        }
         OAL_CUDA_TRY(cudaEventRecord(ev_join, st2));
     }
     {
         LaunchScope ls("scan", st);
+        const int prep = fm_intra ? 0 : 1;
         OAL_CUDA_TRY(launch_ex(tc::scan_kernel,
-                               dim3(tc::kSlices, tc::kScanColGroups, B * Hkv + 1),
+                               dim3(tc::kSlices, tc::kScanColGroups, B * Hkv + prep),
                                dim3(256), 0, st, overlap, (const float*)P.dS, P.img, body, NC,
-                               gid, L, G, eps, sb, B, Hq, Hkv, (long long)T, P.cont, rtab));
+                               gid, L, G, eps, sb, B, Hq, Hkv, (long long)T, P.cont, rtab, prep));
     }
     if (out == nullptr) return OAL_OK;  // no out: the state alone is wanted
     const int items = B * Hq * (cont ? NC : NC - 1);

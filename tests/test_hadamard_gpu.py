@@ -2,13 +2,14 @@
 eq. (5) of "OAL: 按 QK 离群贡献分组的正二次注意力核" (section 核心公式) with free a, b_r, C_rt,
 the relaxation the abstract of arXiv 2610.13674 describes.  The oracle is
 oracle.hadamard_recurrent / hadamard_dense (pinned in tests/test_oracle_hadamard_pins.py).
-The path computes in fp32 for both input dtypes, so the fp32 tolerance applies."""
+bf16 inputs with chunk 128 run on tensor cores (bf16 operands, fp32 accumulation: the bf16
+tolerance); every other case computes in fp32 on CUDA cores (the fp32 tolerance)."""
 import numpy as np
 import pytest
 
 import oracle
 from positive_quadratic_b200 import inputs as I
-from tests._metrics import TOL_F32, row_rel_err
+from tests._metrics import TOL_BF16, TOL_F32, row_rel_err
 from tests.test_gpu_parity import dev_inputs, oal  # noqa: F401 (fixture)
 
 pytestmark = pytest.mark.gpu
@@ -32,8 +33,14 @@ def _t(x, dev):
     return torch.from_numpy(np.ascontiguousarray(x)).to(dev)
 
 
-@pytest.mark.parametrize("dtype,chunk", [("f32", 64), ("f32", 128), ("bf16", 128),
-                                         ("bf16", 256)])
+def _tol(oal, p, chunk):
+    shape = oal.make_shape(p.q.shape[0], p.q.shape[2], p.q.shape[1], p.k.shape[1], chunk,
+                           oal.OAL_BF16 if p.dtype == "bf16" else oal.OAL_F32)
+    return TOL_BF16 if oal.prefill_path(shape) == oal.OAL_PATH_TENSOR else TOL_F32
+
+
+@pytest.mark.parametrize("dtype,chunk", [("f32", 64), ("f32", 128), ("bf16", 64),
+                                         ("bf16", 128), ("bf16", 256)])
 def test_prefill_hadamard_matches_oracle(oal, cuda, dtype, chunk):
     p = I.small_layer(500 + chunk, B=2, T=301, Hq=4, Hkv=2, dtype=dtype)
     a, b, C = _coefs(7, 4)
@@ -42,7 +49,52 @@ def test_prefill_hadamard_matches_oracle(oal, cuda, dtype, chunk):
     y, _ = oal.prefill_hadamard(q, k, v, _t(a, cuda), _t(b, cuda), _t(C, cuda), chunk)
     torch.cuda.synchronize()
     assert oal.device_error() == 0
-    assert row_rel_err(y.cpu().numpy(), ref) <= TOL_F32
+    assert row_rel_err(y.cpu().numpy(), ref) <= _tol(oal, p, chunk)
+
+
+@pytest.mark.parametrize("T", [1, 127, 128, 129, 640])
+def test_tensor_hadamard_edges(oal, cuda, T):
+    """Tensor-core path at a single token, one partial and one full chunk, a one-token second
+    chunk and five chunks; GQA 7 query heads per kv head."""
+    p = I.small_layer(520 + T, B=1, T=T, Hq=7, Hkv=1, dtype="bf16")
+    a, b, C = _coefs(11, 7)
+    ref = oracle.hadamard_recurrent(p.q, p.k, p.v, a, b, C)
+    q, k, v, *_ = dev_inputs(p, cuda)
+    y, _ = oal.prefill_hadamard(q, k, v, _t(a, cuda), _t(b, cuda), _t(C, cuda), 128)
+    torch.cuda.synchronize()
+    assert oal.device_error() == 0
+    assert row_rel_err(y.cpu().numpy(), ref) <= TOL_BF16
+
+
+def test_tensor_hadamard_full_layer(oal, cuda):
+    """A Qwen2.5-0.5B-shaped layer (B=1, T=4096, 14 query / 2 kv heads), every row against
+    the oracle's recurrence."""
+    p = I.small_layer(530, B=1, T=4096, Hq=14, Hkv=2, dtype="bf16")
+    a, b, C = _coefs(12, 14)
+    ref = oracle.hadamard_recurrent(p.q, p.k, p.v, a, b, C)
+    q, k, v, *_ = dev_inputs(p, cuda)
+    y, _ = oal.prefill_hadamard(q, k, v, _t(a, cuda), _t(b, cuda), _t(C, cuda), 128)
+    torch.cuda.synchronize()
+    assert oal.device_error() == 0
+    assert row_rel_err(y.cpu().numpy(), ref) <= TOL_BF16
+
+
+def test_tensor_hadamard_state_matches_cuda_core_state(oal, cuda):
+    """Both paths leave the same coefficient table (bit for bit: one prep kernel) and the same
+    fp32 prefix state (the chunk deltas are exact on both; only the summation order differs)."""
+    p = I.small_layer(531, B=2, T=700, Hq=4, Hkv=2, dtype="bf16")
+    a, b, C = _coefs(13, 4)
+    q, k, v, *_ = dev_inputs(p, cuda)
+    ta, tb, tC = _t(a, cuda), _t(b, cuda), _t(C, cuda)
+    _, s_tc = oal.prefill_hadamard(q, k, v, ta, tb, tC, 128)
+    _, s_cc = oal.prefill_hadamard(q, k, v, ta, tb, tC, 64)
+    torch.cuda.synchronize()
+    assert oal.device_error() == 0
+    head = 256 + ((4 * 2176 * 4 + 255) // 256) * 256
+    assert torch.equal(s_tc[:head], s_cc[:head])
+    x = s_tc[head:].view(torch.float32).double()
+    y = s_cc[head:].view(torch.float32).double()
+    assert float((x - y).abs().max() / y.abs().max()) <= 1e-5
 
 
 def test_dense_hadamard_matches_oracle(oal, cuda):
