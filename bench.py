@@ -219,8 +219,8 @@ def kernel_work(p, chunk=128):
       intra_tc   eqs. (2)-(3) inside a chunk: per causal pair (i, j <= i in the same chunk)
                  2 * 64 (G + 1) flop for the G + 1 factored score products and 2 * 65 for
                  kappa [v; 1]
-      scan       bytes: fp32 deltas read once, bf16 state images written once (80 rows of
-                 64 per 64 packed rows), the fp32 final state written once"""
+      scan       bytes: fp32 deltas read once, bf16 state images written once (the 65 live
+                 rows of 64 per 64 packed rows), the fp32 final state written once"""
     B, Hq, T, _ = p.q.shape
     Hkv = p.k.shape[1]
     NC = -(-T // chunk)
@@ -235,7 +235,7 @@ def kernel_work(p, chunk=128):
         "delta_tc": (2.0 * B * Hkv * T * F * W, "flop"),
         "readout_tc": (2.0 * B * Hq * rows_inter * F * W, "flop"),
         "intra_tc": (B * pairs * per_pair, "flop"),
-        "scan": (B * Hkv * (NC * W * 2176 * 4 + (NC - 1) * slices * 80 * 64 * 2
+        "scan": (B * Hkv * (NC * W * 2176 * 4 + (NC - 1) * slices * W * 64 * 2
                             + 2176 * W * 4), "byte"),
     }
 
@@ -515,12 +515,44 @@ def run_e2e(args, dev, torch, oal, p, q, k, v, g, L, G, out, B, T, flush, barrie
     torch.cuda.synchronize()
     assert oal.device_error() == 0
     e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs2), world, dev)
+    # the copies alone, as the call issues them (in on one stream, out on another, both at
+    # once): the PCIe bound the end-to-end number is measured against
+    dq, dk, dv = (torch.empty_like(t, device=dev) for t in (hq, hk, hv))
+    dout = torch.empty(out.shape, dtype=torch.float32, device=dev)
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+
+    def copies(which):
+        if which in ("in", "both"):
+            with torch.cuda.stream(s_in):
+                for d_, h_ in ((dq, hq), (dk, hk), (dv, hv)):
+                    d_.copy_(h_, non_blocking=True)
+        if which in ("out", "both"):
+            with torch.cuda.stream(s_out):
+                hout.copy_(dout, non_blocking=True)
+
+    copy_ms = {}
+    for which in ("in", "out", "both"):
+        copies(which)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            copies(which)
+        torch.cuda.synchronize()
+        copy_ms[which] = (time.perf_counter() - t0) * 1e3 / args.steps
+    h2d = int(sum(t.numel() * t.element_size() for t in (hq, hk, hv)))
+    d2h = int(hout.numel() * 4)
     e2e = {"value": job_rate(world, args.steps * B * T, e_ms), "unit": UNIT,
-           "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in (hq, hk, hv))),
-           "d2h_bytes_per_step": int(hout.numel() * 4),
+           "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h,
            "api": "oal_prefill_host",
            "segments": bufs["segments"],
-           "segmented_matches_device_prefill": same}
+           "segmented_matches_device_prefill": same,
+           "ms_per_step": e_ms / args.steps,
+           "copies_alone": {
+               "what": "the same pinned copies without kernels, in and out on two streams "
+                       "(host wall clock per step)",
+               "h2d_ms": copy_ms["in"], "d2h_ms": copy_ms["out"], "both_ms": copy_ms["both"],
+               "h2d_gbs": h2d / copy_ms["in"] / 1e6, "d2h_gbs": d2h / copy_ms["out"] / 1e6}}
     return e2e
 
 
