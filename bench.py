@@ -612,6 +612,27 @@ def run_extras(dev, torch, oal, pk):
         res["varlen_prefill"] = {"workload": f"16 sequences, {sum(lens)} tokens, 4 streams, "
                                              "Hq=14 Hkv=2 bf16, chunk 128 (includes packing)",
                                  "ms": ms, "tokens_per_s": sum(lens) / (ms / 1e3)}
+        # the same batch, packed once, in one launch per kernel
+        q, k, v, _ = oal.pack_sequences(qs, ks, vs)
+        ms = timed(lambda: oal.prefill_packed(q, k, v, lens, 14, 2, g, L, G, base.eps))
+        res["packed_prefill"] = {"workload": f"the same 16 sequences, {sum(lens)} tokens, "
+                                             "one launch per kernel (oal_prefill_packed)",
+                                 "ms": ms, "tokens_per_s": sum(lens) / (ms / 1e3)}
+        # many short sequences: 64 of 64..320 tokens
+        lens2 = [int(x) for x in rng.integers(64, 321, size=64)]
+        seqs2 = [I.small_layer(950 + i, B=1, T=t, Hq=14, Hkv=2, dtype="bf16")
+                 for i, t in enumerate(lens2)]
+        qs2 = [to(s_.q[0], torch.bfloat16) for s_ in seqs2]
+        ks2 = [to(s_.k[0], torch.bfloat16) for s_ in seqs2]
+        vs2 = [to(s_.v[0], torch.bfloat16) for s_ in seqs2]
+        ms_v = timed(lambda: oal.prefill_varlen(qs2, ks2, vs2, g, L, G, base.eps, 128,
+                                                streams=streams))
+        q2, k2, v2, _ = oal.pack_sequences(qs2, ks2, vs2)
+        ms_p = timed(lambda: oal.prefill_packed(q2, k2, v2, lens2, 14, 2, g, L, G, base.eps))
+        res["short_sequences"] = {"workload": f"64 sequences of 64..320 tokens ({sum(lens2)} "
+                                              "tokens), Hq=14 Hkv=2 bf16, chunk 128",
+                                  "varlen_4_streams_ms": ms_v, "packed_one_launch_ms": ms_p,
+                                  "packed_tokens_per_s": sum(lens2) / (ms_p / 1e3)}
     except Exception as exc:
         res["varlen_prefill"] = {"error": repr(exc)[:300]}
     try:  # long-context prefill (config 3) and its chunk-size sweep

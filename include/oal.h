@@ -299,6 +299,28 @@ int oal_prefill_varlen(const void* q, const void* k, const void* v, const int32_
                        const oal_shape* s, const int32_t* seq_lens, int n_seq,
                        void* const* streams, int n_streams);
 
+/* Scratch needed by oal_prefill_packed: the chunk states of every sequence (913,920 bytes per
+ * (sequence, kv head, chunk of 128 tokens)), one 7,680-byte readout table per query head, the
+ * intra-chunk normalisers (4 bytes per (token, query head)), 32 bytes of descriptor and three
+ * 128-byte tensor maps per sequence.  seq_lens is host memory. */
+int oal_prefill_packed_workspace_bytes(const oal_shape* s, const int32_t* seq_lens, int n_seq,
+                                       size_t* bytes);
+
+/* The variable-length batch of oal_prefill_varlen (same packed layout of q, k, v, out and the
+ * states, same meaning of every argument) computed by one launch of each tensor-core kernel
+ * for the whole batch on `stream`: the chunk deltas, intra-chunk sums, prefix scans and
+ * readouts of all sequences share one grid each, so many short sequences fill the GPU
+ * together.  Each sequence's results are those of an oal_prefill of its block (the same
+ * per-chunk arithmetic and summation order).  Tensor-core path only: bf16 inputs with chunk
+ * 128, else OAL_ERR_UNSUPPORTED.  workspace: oal_prefill_packed_workspace_bytes, 256-byte
+ * aligned; states 256-byte aligned.  The descriptors and tensor maps are copied into the
+ * workspace on `stream` from host memory that the call owns, so seq_lens may be reused on
+ * return.  Errors: as oal_prefill_varlen. */
+int oal_prefill_packed(const void* q, const void* k, const void* v, const int32_t* group_id,
+                       const float* L, const int32_t* G, float eps, float* out, void* states,
+                       size_t state_stride, void* workspace, size_t workspace_bytes,
+                       const oal_shape* s, const int32_t* seq_lens, int n_seq, void* stream);
+
 /* Scratch needed by oal_dense_backward_gpu for `s` (B, T, Hq used): per row of every query
  * head its normaliser, output, partial dM (81 floats) and partial deps. */
 int oal_dense_backward_workspace_bytes(const oal_shape* s, size_t* bytes);

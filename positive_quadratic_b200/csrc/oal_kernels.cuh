@@ -44,6 +44,21 @@ int launch_prefill_tc(const void* q, const void* k, const void* v, const int32_t
                       void* ws, int B, int T, int Hq, int Hkv, bool overlap, bool cont,
                       cudaStream_t st, bool fm_intra = false);
 
+// The same kernels over a packed variable-length batch in one launch each: sequence i is the
+// B = 1 problem of lens[i] tokens whose q block [Hq][T_i][64] starts at row tok_i * Hq (tok_i:
+// tokens before it), likewise k, v ([Hkv]) and out; its state is at states + i * stride.
+// The workspace holds the chunk states of every sequence, one readout table per head, the
+// intra-chunk normalisers, the sequence descriptors and three tensor maps per sequence.
+struct TcPackedLayout {
+    size_t img, dS, rtab, zin, seqs, maps, total;  // byte offsets and total size
+    long long chunks, tokens;                      // sums over the sequences
+};
+TcPackedLayout tc_packed_layout(int Hq, int Hkv, const int32_t* lens, int n);
+int launch_prefill_tc_packed(const void* q, const void* k, const void* v, const int32_t* gid,
+                             const float* L, const int32_t* G, float eps, float* out,
+                             unsigned char* states, size_t stride, void* ws, const int32_t* lens,
+                             int n, int Hq, int Hkv, bool overlap, cudaStream_t st);
+
 // test hook of oal_set_debug_skip_copies
 extern std::atomic<int> g_skip_copies;
 

@@ -27,8 +27,10 @@
 // Every wait is bounded (1 s); one that runs out sets OAL_ERR_TIMEOUT and the CTA leaves its
 // loops in order (copies drained, MMAs committed, TMEM freed) instead of hanging.
 #include <algorithm>
+#include <cstring>
 #include <mutex>
 #include <utility>
+#include <vector>
 
 #include <cuda.h>
 
@@ -95,6 +97,20 @@ struct Ctl {
 static_assert(sizeof(Ctl) <= 1024, "control block");
 static_assert(sizeof(StBars) <= sizeof(uint64_t) * 64, "barrier block");
 
+// One sequence of a packed variable-length batch (all counts are sums over the sequences
+// before it, so that a flat unit or item index finds its sequence by binary search).
+struct SeqDesc {
+    int T, NC;    // tokens and chunks of the sequence
+    int tok;      // tokens before it: its q block starts at row tok * Hq of [rows][64]
+    int chunk0;   // its first chunk-state index (images, deltas): sum of Hkv * NC
+    int unit0;    // its first chunk-delta unit: sum of Hkv * NC * 17
+    int intra0;   // its first intra-chunk item: sum of Hq * NC
+    int read0;    // its first readout item: sum of Hq * max(NC - 1, 0)
+    int pad;
+};
+static_assert(sizeof(SeqDesc) == 32, "descriptor layout");
+constexpr int kSdUnit0 = 4, kSdIntra0 = 5, kSdRead0 = 6;  // int offsets in SeqDesc
+
 struct Params {
     const CUtensorMap* tm_q;
     const CUtensorMap* tm_k;
@@ -111,6 +127,12 @@ struct Params {
     int B, Hq, Hkv, T, NC;
     int cont;                // 1: the state already holds a prefix; these tokens continue it
     int skip_copies;         // test hook: the readout issues no copies, so its waits run out
+    int n_units, n_intra, n_read;  // chunk-delta units, intra-chunk items, readout items
+    // packed variable-length batch (nseq > 0): B, T and NC above are unused; sequence i has
+    // descriptor seqs[i] and tensor maps maps[3 i + {0, 1, 2}] (q, k, v) in global memory
+    int nseq;
+    const SeqDesc* seqs;
+    const CUtensorMap* maps;
 };
 
 // ------------------------------------------------------------------------------------------
@@ -283,14 +305,101 @@ __device__ __forceinline__ void psi_tile(int slab, int qf, const unsigned char* 
     });
 }
 
-// unit u -> (bkv, chunk c, slab); slabs of one chunk are consecutive
-struct DeltaUnit {
-    int bkv, c, slab;
-};
-__device__ __forceinline__ DeltaUnit delta_unit(int u, int NC)
+// The sequence of a packed batch whose run of indices (field f of the descriptors: first
+// unit or item) contains idx; sequences with an empty run are skipped.
+__device__ __forceinline__ int seq_of(const SeqDesc* sd, int n, int idx, int f)
 {
-    const int rest = u / kNumSlabs;
-    return DeltaUnit{rest / NC, rest % NC, u % kNumSlabs};
+    const int* p = reinterpret_cast<const int*>(sd) + f;
+    int lo = 0, hi = n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (__ldg(p + 8 * mid) <= idx) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+// Order this thread's later tensor copies after the host's write of a tensor map that lives
+// in global memory (the maps of a packed batch).
+__device__ __forceinline__ void tmap_acquire(const CUtensorMap* m)
+{
+    asm volatile("fence.proxy.tensormap::generic.acquire.sys [%0], 128;" ::"l"(m) : "memory");
+}
+
+// unit u -> (kv head, chunk c, slab); slabs of one chunk are consecutive.  mk / mv and kvz:
+// the tensor maps and z coordinate of the unit's K and V tiles; T: the sequence's tokens;
+// chunk: its chunk-state index (deltas, images).
+struct DeltaUnit {
+    int c, slab, T, kvz;
+    size_t chunk;
+    const CUtensorMap *mk, *mv;
+};
+__device__ __forceinline__ DeltaUnit delta_unit(int u, const Params& P)
+{
+    if (P.nseq == 0) {
+        const int rest = u / kNumSlabs, bkv = rest / P.NC, c = rest % P.NC;
+        return DeltaUnit{c, u % kNumSlabs, P.T, bkv, size_t(bkv) * P.NC + c, P.tm_k, P.tm_v};
+    }
+    const int i = seq_of(P.seqs, P.nseq, u, kSdUnit0);
+    const SeqDesc sd = P.seqs[i];
+    const int lu = u - sd.unit0, rest = lu / kNumSlabs, kv = rest / sd.NC, c = rest % sd.NC;
+    return DeltaUnit{c, lu % kNumSlabs, sd.T, kv, size_t(sd.chunk0) + size_t(kv) * sd.NC + c,
+                     P.maps + 3 * i + 1, P.maps + 3 * i + 2};
+}
+
+// An item (query head h of one sequence, chunk c) of the intra-chunk kernels (intra = true)
+// or of the inter-chunk readout.  mq / mk / mv and qz / kvz: tensor maps and z coordinates of
+// its Q, K, V tiles; orow: row of the sequence's token 0 of head h in out [rows][64] and in
+// the normalisers; chunk: chunk-state index of (sequence, kv head, c).
+struct ItemRef {
+    const CUtensorMap *mq, *mk, *mv;
+    int qz, kvz, c, T, h;
+    size_t orow, chunk;
+};
+__device__ __forceinline__ ItemRef item_ref(int idx, const Params& P, bool intra)
+{
+    ItemRef r;
+    if (P.nseq == 0) {
+        const int nbh = P.B * P.Hq;
+        int bh, c;
+        if (P.cont || !intra) {
+            bh = idx % nbh;
+            c = idx / nbh + (P.cont || intra ? 0 : 1);
+        } else if (idx < nbh * (P.NC - 1)) {  // chunks with an inter-chunk part first
+            bh = idx % nbh;
+            c = 1 + idx / nbh;
+        } else {
+            bh = idx - nbh * (P.NC - 1);
+            c = 0;
+        }
+        const int b = bh / P.Hq, h = bh % P.Hq, bkv = b * P.Hkv + h / (P.Hq / P.Hkv);
+        r.mq = P.tm_q;
+        r.mk = P.tm_k;
+        r.mv = P.tm_v;
+        r.qz = bh;
+        r.kvz = bkv;
+        r.c = c;
+        r.T = P.T;
+        r.h = h;
+        r.orow = size_t(bh) * P.T;
+        r.chunk = size_t(bkv) * P.NC + c;
+        return r;
+    }
+    const int i = seq_of(P.seqs, P.nseq, idx, intra ? kSdIntra0 : kSdRead0);
+    const SeqDesc sd = P.seqs[i];
+    const int l = idx - (intra ? sd.intra0 : sd.read0);
+    const int h = l % P.Hq, c = l / P.Hq + (intra ? 0 : 1), kv = h / (P.Hq / P.Hkv);
+    r.mq = P.maps + 3 * i;
+    r.mk = P.maps + 3 * i + 1;
+    r.mv = P.maps + 3 * i + 2;
+    r.qz = h;
+    r.kvz = kv;
+    r.c = c;
+    r.T = sd.T;
+    r.h = h;
+    r.orow = size_t(sd.tok) * P.Hq + size_t(h) * sd.T;
+    r.chunk = size_t(sd.chunk0) + size_t(kv) * sd.NC + c;
+    return r;
 }
 
 // ------------------------------------------------------------------------------------------
@@ -304,7 +413,7 @@ __device__ void delta_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Par
     StBars& bar = ctl.bar.st;
     volatile int* abort_flag = &ctl.abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int NC = P.NC, T = P.T, nu = u1 - u0;
+    const int nu = u1 - u0;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kKVStages; ++i) {
@@ -332,15 +441,19 @@ __device__ void delta_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Par
         if (lane == 0) {
             int issued = 0;
             for (int i = 0; i < nu; ++i) {
-                const DeltaUnit du = delta_unit(u0 + i, NC);
+                const DeltaUnit du = delta_unit(u0 + i, P);
                 const int s = i % kKVStages;
                 if (i >= kKVStages &&
                     !mbar_wait(&bar.kv_empty[s], ((i / kKVStages) - 1) & 1, abort_flag))
                     break;
                 unsigned char* kvs = sm + kStOffKV + s * 2 * kTileBytes;
+                if (P.nseq) {
+                    tmap_acquire(du.mk);
+                    tmap_acquire(du.mv);
+                }
                 mbar_expect_tx(&bar.kv_full[s], 2 * kTileBytes);
-                tma_load_3d(kvs, P.tm_k, &bar.kv_full[s], 0, du.c * kC, du.bkv);
-                tma_load_3d(kvs + kTileBytes, P.tm_v, &bar.kv_full[s], 0, du.c * kC, du.bkv);
+                tma_load_3d(kvs, du.mk, &bar.kv_full[s], 0, du.c * kC, du.kvz);
+                tma_load_3d(kvs + kTileBytes, du.mv, &bar.kv_full[s], 0, du.c * kC, du.kvz);
                 ++issued;
             }
             for (int i = max(0, issued - kKVStages); i < issued; ++i)
@@ -399,7 +512,7 @@ __device__ void delta_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Par
         const int t = threadIdx.x, j = t & 63, qf = t >> 6;
         const uint32_t a0 = smem_u32(sm + kStOffA);
         for (int i = 0; i < nu; ++i) {
-            const DeltaUnit du = delta_unit(u0 + i, NC);
+            const DeltaUnit du = delta_unit(u0 + i, P);
             const int st = i % kKVStages;
             if (!mbar_wait(&bar.kv_full[st], (i / kKVStages) & 1, abort_flag)) break;
             const unsigned char* kt = sm + kStOffKV + st * 2 * kTileBytes;
@@ -412,7 +525,7 @@ __device__ void delta_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Par
                     break;
                 }
                 const int trow = hc * 64 + j;
-                const float one = (du.c * kC + trow < T) ? 1.f : 0.f;
+                const float one = (du.c * kC + trow < du.T) ? 1.f : 0.f;
                 psi_tile(du.slab, qf, kt, trow, one, a0 + as * 2 * kStATile, j);
                 fence_proxy_async();
                 warp_arrive(&bar.a_full[as]);
@@ -425,7 +538,7 @@ __device__ void delta_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Par
         const int q4 = warp & 3, hfe = (warp - 8) >> 2;
         const int fl = q4 * 32 + lane;
         for (int i = 0; i < nu; ++i) {
-            const DeltaUnit du = delta_unit(u0 + i, NC);
+            const DeltaUnit du = delta_unit(u0 + i, P);
             const int s = i % kDAcc;
             // all epilogue threads leave together, so no named barrier is left half-joined
             const bool got = mbar_wait(&bar.acc_full[s], (i / kDAcc) & 1, abort_flag);
@@ -439,7 +552,7 @@ __device__ void delta_item(unsigned char* sm, Ctl& ctl, uint32_t tmem, const Par
             tmem_ld_wait();
             tc_fence_before();
             warp_arrive(&bar.acc_empty[s]);
-            float* dst = P.dS + (size_t(du.bkv) * NC + du.c) * kW * kFP + du.slab * kSlabRows + fl;
+            float* dst = P.dS + du.chunk * kW * kFP + du.slab * kSlabRows + fl;
 #pragma unroll
             for (int x = 0; x < 16; ++x) {
                 dst[size_t(hfe * 32 + x) * kFP] = v0[x];
@@ -542,7 +655,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     grid_dep_launch();  // the next kernel may start its prologue
     grid_dep_wait();    // outputs of the previous kernel are visible from here on
 
-    const int units = P.B * P.Hkv * P.NC * kNumSlabs;
+    const int units = P.n_units;
     const int u0 = int((long long)units * blockIdx.x / gridDim.x);
     const int u1 = int((long long)units * (blockIdx.x + 1) / gridDim.x);
     if (u1 > u0) delta_item(sm, ctl, tmem, P, u0, u1);
@@ -592,20 +705,45 @@ __global__ void __launch_bounds__(256) scan_kernel(const float* __restrict__ dS,
                                                    const int32_t* __restrict__ G, float eps,
                                                    unsigned char* __restrict__ state, int B,
                                                    int Hq, int Hkv, long long tokens, int cont,
-                                                   unsigned char* __restrict__ rtab, int prep)
+                                                   unsigned char* __restrict__ rtab, int prep,
+                                                   const SeqDesc* __restrict__ seqs, int nseq,
+                                                   size_t state_stride)
 {
     grid_dep_launch();
     if (prep && blockIdx.z == gridDim.z - 1) {  // independent of the deltas: no wait
-        const int h = blockIdx.y * gridDim.x + blockIdx.x;
-        if (h < Hq) prep_head(h, gid, L, G, eps, state, B, Hq, Hkv, tokens, cont != 0, rtab);
+        const int nb = gridDim.x * gridDim.y, e0 = blockIdx.y * gridDim.x + blockIdx.x;
+        if (nseq == 0) {
+            for (int e = e0; e < Hq; e += nb)
+                prep_head(e, gid, L, G, eps, state, B, Hq, Hkv, tokens, cont != 0, rtab);
+        } else {  // a packed batch: every sequence's state (B = 1) gets a header and the tables
+            for (int e = e0; e < Hq * nseq; e += nb) {
+                const int i = e / Hq;
+                prep_head(e % Hq, gid, L, G, eps, state + size_t(i) * state_stride, 1, Hq, Hkv,
+                          seqs[i].T, false, i == 0 ? rtab : nullptr);
+            }
+        }
         return;
     }
     grid_dep_wait();
-    const int sl = blockIdx.x, bkv = blockIdx.z;
+    const int sl = blockIdx.x;
     const int nl = threadIdx.x >> 4, rq = threadIdx.x & 15;
     const int n = blockIdx.y * kScanCols + nl;
     __shared__ float fin[kScanCols][64 + 4];
-    float* unit = body + size_t(bkv) * kFP * kW;
+    // this block's (b, kv) unit: its chunk-state index base and its part of the final state
+    size_t chunk0;
+    float* unit;
+    if (nseq == 0) {
+        const int bkv = blockIdx.z;
+        chunk0 = size_t(bkv) * NC;
+        unit = body + size_t(bkv) * kFP * kW;
+    } else {
+        const int i = blockIdx.z / Hkv, kv = blockIdx.z % Hkv;
+        const SeqDesc sd = seqs[i];
+        NC = sd.NC;
+        chunk0 = size_t(sd.chunk0) + size_t(kv) * sd.NC;
+        unit = reinterpret_cast<float*>(state + size_t(i) * state_stride + kHeaderBytes +
+                                        coef_bytes(Hq)) + size_t(kv) * kFP * kW;
+    }
     // the prefix before this call: zero, or (continuation) the state's current contents
     float a[4] = {0.f, 0.f, 0.f, 0.f};
     const int f = sl * 64 + 4 * rq, c_first = cont ? 0 : 1;
@@ -617,9 +755,8 @@ __global__ void __launch_bounds__(256) scan_kernel(const float* __restrict__ dS,
         a[0] = z4.x; a[1] = z4.y; a[2] = z4.z; a[3] = z4.w;
     }
     if (n < kW) {
-        const float* src = dS + (size_t(bkv) * NC * kW + n) * kFP + f;
-        unsigned char* dst = img + (size_t(bkv) * NC * kSlices + sl) * kImgSliceBytes +
-                             n * 128 + 8 * rq;
+        const float* src = dS + (chunk0 * kW + n) * kFP + f;
+        unsigned char* dst = img + (chunk0 * kSlices + sl) * kImgSliceBytes + n * 128 + 8 * rq;
         const size_t sstride = size_t(kW) * kFP, dstride = size_t(kSlices) * kImgSliceBytes;
         constexpr int kDepth = 8;
         for (int c0 = 0; c0 < NC; c0 += kDepth) {
@@ -797,6 +934,102 @@ cudaError_t launch_ex(void (*kern)(Args...), dim3 grid, dim3 block, size_t smem,
 
 }  // namespace
 
+namespace {
+
+// What the scan kernel needs besides Params: the state (or, for a packed batch, the first of
+// the per-sequence states and their stride) and the prep plane's inputs.
+struct ScanArgs {
+    float* body;
+    unsigned char* state;
+    size_t stride;
+    const int32_t* gid;
+    const float* L;
+    const int32_t* G;
+    float eps;
+    long long tokens;
+    int prep;
+};
+
+// The kernel sequence shared by a uniform batch and a packed one: chunk deltas -> (helper
+// stream: intra-chunk sums) -> scan -> join -> inter-chunk readout.  P carries the unit and
+// item counts; grids follow from them.
+int run_prefill_tc(tc::Params& P, const CUtensorMap& mq, const CUtensorMap& mk,
+                   const CUtensorMap& mv, const CUtensorMap& mi, float* zin, const ScanArgs& sa,
+                   int scan_planes, bool fm_intra, bool overlap, cudaStream_t st)
+{
+    const bool with_out = P.out != nullptr;
+    const int nsm = sm_count();
+    OAL_CUDA_TRY(cudaFuncSetAttribute(tc::delta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      int(tc::kSmemBytes)));
+    OAL_CUDA_TRY(cudaFuncSetAttribute(tc::intra::intra_kernel,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      int(tc::intra::kSmemBytes)));
+    OAL_CUDA_TRY(cudaFuncSetAttribute(tc::fm::intra_fm_kernel,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      int(tc::fm::kSmemBytes)));
+    OAL_CUDA_TRY(cudaFuncSetAttribute(tc::rd::readout_kernel,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      int(tc::rd::kSmemBytes)));
+    // two intra-chunk CTAs per SM need the whole shared-memory carve-out
+    OAL_CUDA_TRY(cudaFuncSetAttribute(tc::intra::intra_kernel,
+                                      cudaFuncAttributePreferredSharedMemoryCarveout, 100));
+    CallEvents evs;
+    cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+    const bool intra = with_out && P.n_intra > 0;
+    cudaStream_t st2 = intra ? helper_stream() : nullptr;
+    if (intra && st2 == nullptr) return OAL_ERR_CUDA;
+    if (intra) {
+        OAL_CUDA_TRY(evs.make(&ev_fork));
+        OAL_CUDA_TRY(evs.make(&ev_join));
+        OAL_CUDA_TRY(cudaEventRecord(ev_fork, st));
+    }
+    if (P.n_units > 0) {
+        const int grid0 = std::max(1, std::min(nsm, P.n_units));
+        LaunchScope ls("delta_tc", st);
+        OAL_CUDA_TRY(launch_ex(tc::delta_kernel, dim3(grid0), dim3(tc::kThreads), tc::kSmemBytes,
+                               st, false, mk, mv, P));
+    }
+    if (intra) {
+        // the intra-chunk sums need only q, k, v: they run on the helper stream beside the
+        // chunk deltas and the scan (latency-bound, they fill SMs the memory-bound scan
+        // leaves idle); chunk 0 of a fresh prefill is final there
+        OAL_CUDA_TRY(cudaStreamWaitEvent(st2, ev_fork, 0));
+        if (fm_intra) {  // free coefficients: Phi(Q_c) Psi(K_c)^T through the feature map
+            LaunchScope ls("intra_fm_tc", st2);
+            OAL_CUDA_TRY(launch_ex(tc::fm::intra_fm_kernel, dim3(P.n_intra),
+                                   dim3(tc::fm::kThreads), tc::fm::kSmemBytes, st2, false, mq,
+                                   mk, mv, P, zin));
+        } else {
+            LaunchScope ls("intra_tc", st2);
+            OAL_CUDA_TRY(launch_ex(tc::intra::intra_kernel, dim3(P.n_intra),
+                                   dim3(tc::intra::kThreads), tc::intra::kSmemBytes, st2, false,
+                                   mq, mk, mv, P, zin));
+        }
+        OAL_CUDA_TRY(cudaEventRecord(ev_join, st2));
+    }
+    {
+        LaunchScope ls("scan", st);
+        OAL_CUDA_TRY(launch_ex(tc::scan_kernel,
+                               dim3(tc::kSlices, tc::kScanColGroups, scan_planes + sa.prep),
+                               dim3(256), 0, st, overlap && P.n_units > 0, (const float*)P.dS,
+                               P.img, sa.body, P.NC, sa.gid, sa.L, sa.G, sa.eps, sa.state, P.B,
+                               P.Hq, P.Hkv, sa.tokens, P.cont, const_cast<unsigned char*>(P.rtab), sa.prep,
+                               (const tc::SeqDesc*)P.seqs, P.nseq, sa.stride));
+    }
+    if (!with_out) return OAL_OK;  // no out: the state alone is wanted
+    if (intra) OAL_CUDA_TRY(cudaStreamWaitEvent(st, ev_join, 0));  // intra-chunk sums complete
+    if (P.n_read > 0) {
+        // persistent: one CTA per SM walks the items (b*h, chunk) with an inter-chunk part
+        const int grid2 = std::max(1, std::min(nsm, P.n_read));
+        LaunchScope ls("readout_tc", st);
+        OAL_CUDA_TRY(launch_ex(tc::rd::readout_kernel, dim3(grid2), dim3(tc::rd::kThreads),
+                               tc::rd::kSmemBytes, st, overlap, mq, mi, P, (const float*)zin));
+    }
+    return OAL_OK;
+}
+
+}  // namespace
+
 int launch_prefill_tc(const void* q, const void* k, const void* v, const int32_t* gid,
                       const float* L, const int32_t* G, float eps, float* out, void* state,
                       void* ws, int B, int T, int Hq, int Hkv, bool overlap, bool cont,
@@ -836,72 +1069,102 @@ int launch_prefill_tc(const void* q, const void* k, const void* v, const int32_t
     P.NC = NC;
     P.cont = cont ? 1 : 0;
     P.skip_copies = g_skip_copies.load() ? 1 : 0;
-    const int units = B * Hkv * NC * tc::kNumSlabs;
-    const int nsm = sm_count();
-    const int grid0 = std::max(1, std::min(nsm, units));
-    OAL_CUDA_TRY(cudaFuncSetAttribute(tc::delta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      int(tc::kSmemBytes)));
-    OAL_CUDA_TRY(cudaFuncSetAttribute(tc::intra::intra_kernel,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      int(tc::intra::kSmemBytes)));
-    OAL_CUDA_TRY(cudaFuncSetAttribute(tc::fm::intra_fm_kernel,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      int(tc::fm::kSmemBytes)));
-    OAL_CUDA_TRY(cudaFuncSetAttribute(tc::rd::readout_kernel,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      int(tc::rd::kSmemBytes)));
-    // two intra-chunk CTAs per SM need the whole shared-memory carve-out
-    OAL_CUDA_TRY(cudaFuncSetAttribute(tc::intra::intra_kernel,
-                                      cudaFuncAttributePreferredSharedMemoryCarveout, 100));
-    CallEvents evs;
-    cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
-    cudaStream_t st2 = out != nullptr ? helper_stream() : nullptr;
-    if (out != nullptr && st2 == nullptr) return OAL_ERR_CUDA;
-    if (out != nullptr) OAL_CUDA_TRY(evs.make(&ev_fork));
-    if (out != nullptr) OAL_CUDA_TRY(evs.make(&ev_join));
-    if (out != nullptr) OAL_CUDA_TRY(cudaEventRecord(ev_fork, st));
-    {
-        LaunchScope ls("delta_tc", st);
-        OAL_CUDA_TRY(launch_ex(tc::delta_kernel, dim3(grid0), dim3(tc::kThreads), tc::kSmemBytes,
-                               st, false, mk, mv, P));
+    P.n_units = B * Hkv * NC * tc::kNumSlabs;
+    P.n_intra = NC * B * Hq;
+    P.n_read = B * Hq * (cont ? NC : NC - 1);
+    P.nseq = 0;
+    ScanArgs sa{body, sb, 0, gid, L, G, eps, (long long)T, fm_intra ? 0 : 1};
+    return run_prefill_tc(P, mq, mk, mv, mi, zin, sa, B * Hkv, fm_intra, overlap, st);
+}
+
+// ---- packed variable-length batch ----------------------------------------------------------
+
+TcPackedLayout tc_packed_layout(int Hq, int Hkv, const int32_t* lens, int n)
+{
+    TcPackedLayout l{};
+    long long chunks = 0, tokens = 0;
+    for (int i = 0; i < n; ++i) {
+        chunks += (lens[i] + tc::kC - 1) / tc::kC;
+        tokens += lens[i];
     }
-    if (out != nullptr) {
-        // the intra-chunk sums need only q, k, v: they run on the helper stream beside the
-        // chunk deltas and the scan (latency-bound, they fill SMs the memory-bound scan
-        // leaves idle); chunk 0 of a fresh prefill is final there
-        OAL_CUDA_TRY(cudaStreamWaitEvent(st2, ev_fork, 0));
-        if (fm_intra) {  // free coefficients: Phi(Q_c) Psi(K_c)^T through the feature map
-            LaunchScope ls("intra_fm_tc", st2);
-            OAL_CUDA_TRY(launch_ex(tc::fm::intra_fm_kernel, dim3(NC * B * Hq),
-                                   dim3(tc::fm::kThreads), tc::fm::kSmemBytes, st2, false, mq,
-                                   mk, mv, P, zin));
-        } else {
-            LaunchScope ls("intra_tc", st2);
-            OAL_CUDA_TRY(launch_ex(tc::intra::intra_kernel, dim3(NC * B * Hq),
-                                   dim3(tc::intra::kThreads), tc::intra::kSmemBytes, st2, false,
-                                   mq, mk, mv, P, zin));
+    l.chunks = chunks;
+    l.tokens = tokens;
+    l.img = 0;
+    l.dS = l.img + size_t(chunks) * Hkv * tc::kImgChunkBytes;
+    l.rtab = l.dS + size_t(chunks) * Hkv * kW * kFP * 4;
+    l.zin = l.rtab + size_t(Hq) * kTabBytes;
+    l.seqs = l.zin + align256(size_t(tokens) * Hq * 4);
+    l.maps = l.seqs + align256(size_t(n) * sizeof(tc::SeqDesc));
+    l.total = std::max<size_t>(256, l.maps + align256(size_t(n) * 3 * sizeof(CUtensorMap)));
+    return l;
+}
+
+int launch_prefill_tc_packed(const void* q, const void* k, const void* v, const int32_t* gid,
+                             const float* L, const int32_t* G, float eps, float* out,
+                             unsigned char* states, size_t stride, void* ws, const int32_t* lens,
+                             int n, int Hq, int Hkv, bool overlap, cudaStream_t st)
+{
+    if (n == 0) return OAL_OK;
+    const TcPackedLayout lay = tc_packed_layout(Hq, Hkv, lens, n);
+    unsigned char* wsb = static_cast<unsigned char*>(ws);
+    std::vector<tc::SeqDesc> sd(static_cast<size_t>(n));
+    std::vector<CUtensorMap> maps(size_t(n) * 3);
+    std::memset(maps.data(), 0, maps.size() * sizeof(CUtensorMap));
+    const size_t rq = size_t(Hq) * OAL_HEAD_DIM * 2, rkv = size_t(Hkv) * OAL_HEAD_DIM * 2;
+    int tok = 0, chunk0 = 0, unit0 = 0, intra0 = 0, read0 = 0;
+    for (int i = 0; i < n; ++i) {
+        const int T = lens[i], NC = (T + tc::kC - 1) / tc::kC;
+        sd[size_t(i)] = tc::SeqDesc{T, NC, tok, chunk0, unit0, intra0, read0, 0};
+        if (T > 0) {  // a sequence without tokens has no units or items: its maps stay unused
+            const unsigned char* qi = static_cast<const unsigned char*>(q) + size_t(tok) * rq;
+            const unsigned char* ki = static_cast<const unsigned char*>(k) + size_t(tok) * rkv;
+            const unsigned char* vi = static_cast<const unsigned char*>(v) + size_t(tok) * rkv;
+            if (!make_map(&maps[3 * size_t(i)], qi, T, Hq) ||
+                !make_map(&maps[3 * size_t(i) + 1], ki, T, Hkv) ||
+                !make_map(&maps[3 * size_t(i) + 2], vi, T, Hkv))
+                return OAL_ERR_CUDA;
         }
-        OAL_CUDA_TRY(cudaEventRecord(ev_join, st2));
+        tok += T;
+        chunk0 += Hkv * NC;
+        unit0 += Hkv * NC * tc::kNumSlabs;
+        intra0 += Hq * NC;
+        read0 += Hq * std::max(NC - 1, 0);
     }
-    {
-        LaunchScope ls("scan", st);
-        const int prep = fm_intra ? 0 : 1;
-        OAL_CUDA_TRY(launch_ex(tc::scan_kernel,
-                               dim3(tc::kSlices, tc::kScanColGroups, B * Hkv + prep),
-                               dim3(256), 0, st, overlap, (const float*)P.dS, P.img, body, NC,
-                               gid, L, G, eps, sb, B, Hq, Hkv, (long long)T, P.cont, rtab, prep));
-    }
-    if (out == nullptr) return OAL_OK;  // no out: the state alone is wanted
-    const int items = B * Hq * (cont ? NC : NC - 1);
-    OAL_CUDA_TRY(cudaStreamWaitEvent(st, ev_join, 0));  // the intra-chunk sums are complete
-    if (items > 0) {
-        // persistent: one CTA per SM walks the items (b*h, chunk) with an inter-chunk part
-        const int grid2 = std::max(1, std::min(nsm, items));
-        LaunchScope ls("readout_tc", st);
-        OAL_CUDA_TRY(launch_ex(tc::rd::readout_kernel, dim3(grid2), dim3(tc::rd::kThreads),
-                               tc::rd::kSmemBytes, st, overlap, mq, mi, P, (const float*)zin));
-    }
-    return OAL_OK;
+    CUtensorMap mi, none;
+    std::memset(&none, 0, sizeof(none));
+    if (lay.chunks > 0 && !make_img_map(&mi, wsb, size_t(lay.chunks) * Hkv * tc::kSlices))
+        return OAL_ERR_CUDA;
+    if (lay.chunks == 0) mi = none;
+    // descriptors and tensor maps into the workspace, ahead of the kernels on the same stream
+    OAL_CUDA_TRY(cudaMemcpyAsync(wsb + lay.seqs, sd.data(), sd.size() * sizeof(tc::SeqDesc),
+                                 cudaMemcpyHostToDevice, st));
+    OAL_CUDA_TRY(cudaMemcpyAsync(wsb + lay.maps, maps.data(), maps.size() * sizeof(CUtensorMap),
+                                 cudaMemcpyHostToDevice, st));
+    tc::Params P{};
+    P.gid = gid;
+    P.L = L;
+    P.G = G;
+    P.eps = eps;
+    P.img = wsb + lay.img;
+    P.dS = reinterpret_cast<float*>(wsb + lay.dS);
+    P.rtab = wsb + lay.rtab;
+    float* zin = reinterpret_cast<float*>(wsb + lay.zin);
+    P.out = out;
+    P.B = n;
+    P.Hq = Hq;
+    P.Hkv = Hkv;
+    P.T = 0;
+    P.NC = 0;
+    P.cont = 0;
+    P.skip_copies = g_skip_copies.load() ? 1 : 0;
+    P.n_units = unit0;
+    P.n_intra = intra0;
+    P.n_read = read0;
+    P.nseq = n;
+    P.seqs = reinterpret_cast<const tc::SeqDesc*>(wsb + lay.seqs);
+    P.maps = reinterpret_cast<const CUtensorMap*>(wsb + lay.maps);
+    ScanArgs sa{nullptr, states, stride, gid, L, G, eps, 0, 1};
+    return run_prefill_tc(P, none, none, none, mi, zin, sa, n * Hkv, false, overlap, st);
 }
 
 }  // namespace oal

@@ -62,21 +62,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int* abort_flag = &ctl.abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // item: chunks with an inter-chunk part first, the heads of a chunk adjacent
-    const int nbh = P.B * P.Hq, idx = blockIdx.x;
-    int bh, c;
-    if (P.cont) {
-        bh = idx % nbh;
-        c = idx / nbh;
-    } else if (idx < nbh * (P.NC - 1)) {
-        bh = idx % nbh;
-        c = 1 + idx / nbh;
-    } else {
-        bh = idx - nbh * (P.NC - 1);
-        c = 0;
-    }
+    P.tm_q = &tm_q;
+    P.tm_k = &tm_k;
+    P.tm_v = &tm_v;
+    const ItemRef it = item_ref(blockIdx.x, P, true);
+    const int c = it.c, h = it.h;
     const bool final_out = (c == 0) && !P.cont;
-    const int b = bh / P.Hq, h = bh % P.Hq, bkv = b * P.Hkv + h / (P.Hq / P.Hkv);
 
     if (threadIdx.x == 0) {
         mbar_init(&ctl.qkv_full, 1);
@@ -115,9 +106,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     grid_dep_launch();
     if (warp == kLdWarp && lane == 0) {
         mbar_expect_tx(&ctl.qkv_full, 3 * kTileBytes + kTabBytes);
-        tma_load_3d(sm + kOffQ, &tm_q, &ctl.qkv_full, 0, c * kC, bh);
-        tma_load_3d(sm + kOffK, &tm_k, &ctl.qkv_full, 0, c * kC, bkv);
-        tma_load_3d(sm + kOffV, &tm_v, &ctl.qkv_full, 0, c * kC, bkv);
+        if (P.nseq) {
+            tmap_acquire(it.mq);
+            tmap_acquire(it.mk);
+            tmap_acquire(it.mv);
+        }
+        tma_load_3d(sm + kOffQ, it.mq, &ctl.qkv_full, 0, c * kC, it.qz);
+        tma_load_3d(sm + kOffK, it.mk, &ctl.qkv_full, 0, c * kC, it.kvz);
+        tma_load_3d(sm + kOffV, it.mv, &ctl.qkv_full, 0, c * kC, it.kvz);
         bulk_g2s(sm + kOffTab, P.rtab + size_t(h) * kTabBytes, kTabBytes, &ctl.qkv_full);
     }
 
@@ -188,15 +184,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float z = tmem_ld1(lanebase + kColU + 64);
                 tmem_ld_wait();
                 const int irow = c * kC + row;
-                if (irow < P.T) {
-                    float4* o = reinterpret_cast<float4*>(P.out + (size_t(bh) * P.T + irow) * kDV +
-                                                          32 * kh);
+                if (irow < it.T) {
+                    float4* o = reinterpret_cast<float4*>(P.out + (it.orow + irow) * kDV + 32 * kh);
                     const float inv = final_out ? 1.f / z : 1.f;
 #pragma unroll
                     for (int i = 0; i < 8; ++i)
                         o[i] = make_float4(u[4 * i] * inv, u[4 * i + 1] * inv, u[4 * i + 2] * inv,
                                            u[4 * i + 3] * inv);
-                    if (!final_out && kh == 0) zin[size_t(bh) * P.T + irow] = z;
+                    if (!final_out && kh == 0) zin[it.orow + irow] = z;
                 }
             }
         }

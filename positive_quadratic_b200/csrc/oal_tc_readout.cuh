@@ -67,14 +67,8 @@ struct Ctl {
 };
 static_assert(sizeof(Ctl) <= 1024, "control block");
 
-// Items of the inter-chunk readout: chunk-major, the query heads of a chunk adjacent (they
-// read the same state image, which then stays in L2).
-__device__ __forceinline__ void item_of(int idx, const Params& P, int& bh, int& c)
-{
-    const int nbh = P.B * P.Hq;
-    bh = idx % nbh;
-    c = idx / nbh + (P.cont ? 0 : 1);
-}
+// Items of the inter-chunk readout (item_ref): chunk-major within a sequence, the query heads
+// of a chunk adjacent (they read the same state image, which then stays in L2).
 
 // 8-dim chunks of the q row that the packed rows [F, F + n) read
 template <int F, int n>
@@ -163,7 +157,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     Bars& bar = ctl.bar;
     volatile int* abort_flag = &ctl.abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_items = P.B * P.Hq * (P.cont ? P.NC : P.NC - 1);
+    const int n_items = P.n_read;
     P.tm_q = &tm_q;
     P.tm_img = &tm_img;
 
@@ -239,11 +233,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float* ui = reinterpret_cast<const float*>(sm + kOffUI) + row * kDV;
         // the U_intra rows of item jj (one bulk copy of up to 32 KB, rows 256 B apart)
         auto prefetch = [&](int idx) {
-            int bh, c;
-            item_of(idx, P, bh, c);
-            const int nrows = min(kC, P.T - c * kC);
+            const ItemRef it = item_ref(idx, P, false);
+            const int nrows = min(kC, it.T - it.c * kC);
             mbar_expect_tx(&bar.ui_full, uint32_t(nrows) * kDV * 4);
-            bulk_g2s(sm + kOffUI, P.out + (size_t(bh) * P.T + size_t(c) * kC) * kDV,
+            bulk_g2s(sm + kOffUI, P.out + (it.orow + size_t(it.c) * kC) * kDV,
                      uint32_t(nrows) * kDV * 4, &bar.ui_full);
         };
         int last_pf = -1;  // item index j of the last U_intra copy issued, if not waited for
@@ -253,11 +246,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // all four warps run the same iterations and leave together (named barrier below)
         for (int j = 0, idx = blockIdx.x; idx < n_items; ++j, idx += gridDim.x) {
-            int bh, c;
-            item_of(idx, P, bh, c);
-            const int irow = c * kC + row;
-            const bool valid = irow < P.T;
-            const size_t ro = size_t(bh) * P.T + irow;
+            const ItemRef it = item_ref(idx, P, false);
+            const int irow = it.c * kC + row;
+            const bool valid = irow < it.T;
+            const size_t ro = it.orow + irow;
             const float zi = valid ? zin[ro] : 0.f;  // in flight while the item runs
             const bool got = wait_all_sleep(&bar.ui_full, j & 1, abort_flag) &&
                              wait_all_sleep(&bar.u_full, j & 1, abort_flag);
@@ -366,12 +358,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             auto load_q = [&](int jj, int qidx) {
                 if (P.skip_copies) return;
-                int bh, c;
-                item_of(qidx, P, bh, c);
+                const ItemRef it = item_ref(qidx, P, false);
                 const int qb = jj & 1;
+                if (P.nseq) tmap_acquire(it.mq);
                 mbar_expect_tx(&bar.q_full[qb], kTileBytes + kTabBytes);
-                tma_load_3d(sm + kOffQ + qb * kTileBytes, P.tm_q, &bar.q_full[qb], 0, c * kC, bh);
-                bulk_g2s(sm + kOffTab + qb * kTabBytes, P.rtab + size_t(bh % P.Hq) * kTabBytes,
+                tma_load_3d(sm + kOffQ + qb * kTileBytes, it.mq, &bar.q_full[qb], 0, it.c * kC,
+                            it.qz);
+                bulk_g2s(sm + kOffTab + qb * kTabBytes, P.rtab + size_t(it.h) * kTabBytes,
                          kTabBytes, &bar.q_full[qb]);
                 lq = jj;
             };
@@ -381,11 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             for (int j = 0, idx = blockIdx.x; idx < n_items && ok; ++j, idx += gridDim.x) {
                 const int nidx = idx + gridDim.x;
-                int bh, c;
-                item_of(idx, P, bh, c);
-                const int b = bh / P.Hq, h = bh % P.Hq;
-                const int bkv = b * P.Hkv + h / (P.Hq / P.Hkv);
-                const int row0 = (bkv * P.NC + c) * kSlices * 80;
+                const int row0 = int(item_ref(idx, P, false).chunk) * kSlices * 80;
                 for (int p = 0; p < kPairs; ++p) {
                     const int g = j * kPairs + p, st = g % kSlots, use = g / kSlots;
                     if (use >= 1 && !mbar_wait_sleep(&bar.e[st], (use - 1) & 1, abort_flag)) {

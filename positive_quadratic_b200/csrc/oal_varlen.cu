@@ -54,10 +54,75 @@ int plan_varlen(const oal_shape* s, const int32_t* seq_lens, int n_seq, int n_st
     return OAL_OK;
 }
 
+// The packed batch in one launch per kernel: the tensor-core path only (bf16, chunk 128).
+int plan_packed(const oal_shape* s, const int32_t* seq_lens, int n_seq, TcPackedLayout* lay,
+                size_t* state_one)
+{
+    if (!s || (n_seq > 0 && !seq_lens)) return OAL_ERR_NULL;
+    if (n_seq < 0) return OAL_ERR_SHAPE;
+    oal_shape one = *s;
+    one.B = 1;
+    int tmax = 0;
+    long long total = 0;
+    for (int i = 0; i < n_seq; ++i) {
+        if (seq_lens[i] < 0) return OAL_ERR_SHAPE;
+        tmax = std::max(tmax, int(seq_lens[i]));
+        total += seq_lens[i];
+    }
+    if (total * (long long)s->Hq >= (1LL << 31)) return OAL_ERR_SHAPE;
+    one.T = tmax;
+    int rc = check_common(&one);
+    if (rc) return rc;
+    if ((rc = check_chunk(&one))) return rc;
+    if (!use_tensor_path(&one)) return OAL_ERR_UNSUPPORTED;
+    *lay = tc_packed_layout(s->Hq, s->Hkv, seq_lens, n_seq);
+    // tensor-copy row coordinates of the chunk-state images are 32-bit
+    if (lay->chunks * s->Hkv * 34 * 80 >= (1LL << 31)) return OAL_ERR_SHAPE;
+    return oal_state_bytes(&one, state_one);
+}
+
 }  // namespace
 }  // namespace oal
 
 extern "C" {
+
+int oal_prefill_packed_workspace_bytes(const oal_shape* s, const int32_t* seq_lens, int n_seq,
+                                       size_t* bytes)
+{
+    using namespace oal;
+    if (!bytes) return OAL_ERR_NULL;
+    TcPackedLayout lay;
+    size_t state_one = 0;
+    const int rc = plan_packed(s, seq_lens, n_seq, &lay, &state_one);
+    if (rc) return rc;
+    *bytes = lay.total;
+    return OAL_OK;
+}
+
+int oal_prefill_packed(const void* q, const void* k, const void* v, const int32_t* group_id,
+                       const float* L, const int32_t* G, float eps, float* out, void* states,
+                       size_t state_stride, void* workspace, size_t workspace_bytes,
+                       const oal_shape* s, const int32_t* seq_lens, int n_seq, void* stream)
+{
+    using namespace oal;
+    TcPackedLayout lay;
+    size_t state_one = 0;
+    int rc = plan_packed(s, seq_lens, n_seq, &lay, &state_one);
+    if (rc) return rc;
+    if (!states || !group_id || !L || !G) return OAL_ERR_NULL;
+    if (state_stride < state_one || state_stride % 256 != 0) return OAL_ERR_SHAPE;
+    if (!workspace || workspace_bytes < lay.total) return OAL_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return OAL_ERR_ALIGN;
+    if ((reinterpret_cast<uintptr_t>(states) & 255) != 0) return OAL_ERR_ALIGN;
+    if (lay.tokens > 0 && (!q || !k || !v || !out)) return OAL_ERR_NULL;
+    if (lay.tokens > 0 && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)))
+        return OAL_ERR_ALIGN;
+    if (!aligned16(group_id) || !aligned16(L) || !aligned16(G)) return OAL_ERR_ALIGN;
+    return launch_prefill_tc_packed(q, k, v, group_id, L, G, eps, out,
+                                    static_cast<unsigned char*>(states), state_stride, workspace,
+                                    seq_lens, n_seq, s->Hq, s->Hkv, g_prefill_overlap.load() != 0,
+                                    static_cast<cudaStream_t>(stream));
+}
 
 int oal_prefill_varlen_workspace_bytes(const oal_shape* s, const int32_t* seq_lens, int n_seq,
                                        int n_streams, size_t* bytes)

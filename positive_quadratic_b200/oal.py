@@ -94,6 +94,12 @@ def lib() -> ctypes.CDLL:
             L.oal_prefill_varlen.argtypes = [_VP] * 6 + [ctypes.c_float, _VP, _VP, _SZ, _VP,
                                                          _SZ, _PS, _VP, ctypes.c_int, _VP,
                                                          ctypes.c_int]
+            L.oal_prefill_packed_workspace_bytes.argtypes = [_PS, _VP, ctypes.c_int,
+                                                             ctypes.POINTER(_SZ)]
+            L.oal_prefill_packed_workspace_bytes.restype = ctypes.c_int
+            L.oal_prefill_packed.argtypes = [_VP] * 6 + [ctypes.c_float, _VP, _VP, _SZ, _VP,
+                                                         _SZ, _PS, _VP, ctypes.c_int, _VP]
+            L.oal_prefill_packed.restype = ctypes.c_int
             L.oal_state_prefix_sum.argtypes = [_VP, ctypes.c_int, _SZ, _VP, _VP]
             L.oal_state_prefix_sum.restype = ctypes.c_int
             L.oal_dense_backward_workspace_bytes.argtypes = [_PS, ctypes.POINTER(_SZ)]
@@ -489,6 +495,46 @@ def prefill_varlen(qs, ks, vs, group_id, L, G, eps: float, chunk: int = 128, str
         outs.append(out[off * Hq * 64:(off + t) * Hq * 64].view(Hq, t, 64))
         off += t
     return outs, states
+
+
+def pack_sequences(qs, ks, vs):
+    """The packed layout of a variable-length batch: qs[i] [Hq, T_i, 64], ks[i] / vs[i]
+    [Hkv, T_i, 64] concatenated block after block into flat q, k, v; returns (q, k, v, lens)."""
+    n = len(qs)
+    if not (len(ks) == len(vs) == n) or n == 0:
+        raise ValueError("qs, ks, vs: equal, non-zero numbers of sequences")
+    pack = lambda ts: torch.cat([t.contiguous().reshape(-1) for t in ts])  # noqa: E731
+    return pack(qs), pack(ks), pack(vs), [int(t.shape[1]) for t in qs]
+
+
+def prefill_packed(q, k, v, lens, Hq: int, Hkv: int, group_id, L, G, eps: float, out=None,
+                   states=None, workspace=None, stream=None):
+    """oal_prefill_packed: the variable-length batch (packed as pack_sequences lays it out)
+    in one launch per tensor-core kernel.  bf16 only (chunk 128).  Returns (out, states):
+    out flat fp32 [Hq * sum(lens) * 64] (sequence i's [Hq, T_i, 64] block after the blocks
+    before it), states [n, stride] uint8."""
+    n = len(lens)
+    dev = q.device
+    shape = make_shape(1, max(lens) if n else 0, Hq, Hkv, 128, _dtype_code(q))
+    c_lens = (ctypes.c_int32 * max(n, 1))(*lens)
+    nb = _SZ(0)
+    _check(lib().oal_prefill_packed_workspace_bytes(ctypes.byref(shape), c_lens, n,
+                                                    ctypes.byref(nb)),
+           "oal_prefill_packed_workspace_bytes")
+    stride = (state_bytes(make_shape(1, 1, Hq, Hkv, 128, _dtype_code(q))) + 255) // 256 * 256
+    if out is None:
+        out = torch.empty(Hq * sum(lens) * 64, dtype=torch.float32, device=dev)
+    if states is None:
+        states = torch.empty(n, stride, dtype=torch.uint8, device=dev)
+    if workspace is None:
+        workspace = empty_workspace(nb.value, dev)
+    _contig_cuda(q, k, v, group_id, L, G, out, states, workspace)
+    rc = lib().oal_prefill_packed(_ptr(q), _ptr(k), _ptr(v), _ptr(group_id), _ptr(L), _ptr(G),
+                                  float(eps), _ptr(out), _ptr(states), stride, _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(),
+                                  ctypes.byref(shape), c_lens, n, _stream(stream))
+    _check(rc, "oal_prefill_packed")
+    return out, states
 
 
 def dense_backward(q, k, v, group_id, L, G, eps: float, dy, stream=None) -> dict:

@@ -58,6 +58,35 @@ def test_prefill_path_query():
     assert oal.lib().oal_prefill_path(ctypes.byref(s), None) == -1
 
 
+def test_packed_batch_host_checks():
+    """The one-launch packed batch runs only on the tensor-core path; sizes and arguments are
+    checked on the host before anything reaches the device."""
+    lens = (ctypes.c_int32 * 3)(300, 0, 129)
+    n = ctypes.c_size_t()
+    s = oal.make_shape(1, 300, 14, 2, 128, oal.OAL_BF16)
+    assert oal.lib().oal_prefill_packed_workspace_bytes(ctypes.byref(s), lens, 3,
+                                                        ctypes.byref(n)) == 0
+    chunks, toks = 3 + 0 + 2, 429
+    tail = ((toks * 14 * 4 + 255) // 256 * 256 + 256 + (3 * 3 * 128 + 255) // 256 * 256)
+    assert n.value == chunks * 2 * 913920 + 14 * 7680 + tail
+    for chunk, dt in ((64, oal.OAL_BF16), (128, oal.OAL_F32)):
+        s2 = oal.make_shape(1, 300, 14, 2, chunk, dt)
+        assert oal.lib().oal_prefill_packed_workspace_bytes(ctypes.byref(s2), lens, 3,
+                                                            ctypes.byref(n)) == -3
+    bad = (ctypes.c_int32 * 2)(10, -1)
+    assert oal.lib().oal_prefill_packed_workspace_bytes(ctypes.byref(s), bad, 2,
+                                                        ctypes.byref(n)) == -2
+    P = _fake(1 << 20)
+    ws = _fake(1 << 24)
+    # workspace too small, misaligned workspace, missing states
+    assert oal.lib().oal_prefill_packed(P, P, P, P, P, P, 0.0, P, P, 1 << 21, ws, 256,
+                                        ctypes.byref(s), lens, 3, None) == -8
+    assert oal.lib().oal_prefill_packed(P, P, P, P, P, P, 0.0, P, P, 1 << 21, _fake(4096 + 16),
+                                        1 << 40, ctypes.byref(s), lens, 3, None) == -4
+    assert oal.lib().oal_prefill_packed(P, P, P, P, P, P, 0.0, P, None, 1 << 21, ws, 1 << 40,
+                                        ctypes.byref(s), lens, 3, None) == -1
+
+
 def test_group_size_limit():
     s = oal.make_shape(1, 16, 16, 1)
     n = ctypes.c_size_t()
