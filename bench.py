@@ -558,8 +558,8 @@ def run_e2e(args, dev, torch, oal, p, q, k, v, g, L, G, out, B, T, flush, barrie
 
 def run_extras(dev, torch, oal, pk):
     """Small timings of the further paths on this rank (no cross-rank reduction): the
-    Hadamard-form prefill, a variable-length batch over four streams, long-context prefill
-    with its chunk-size sweep, and the dense backward.
+    Hadamard-form prefill, variable-length batches (four streams; one launch per kernel),
+    long-context prefill with its chunk-size sweep, and the dense and chunked backward.
     Each is timed with CUDA events after warm-up; a failure is recorded, not raised."""
     from positive_quadratic_b200 import inputs as I
     res = {}
@@ -670,6 +670,16 @@ def run_extras(dev, torch, oal, pk):
         ms = timed(lambda: oal.dense_backward(q, k, v, g, L, G, p.eps, dy), reps=3)
         res["dense_backward"] = {"workload": "B=1 T=256 Hq=14 Hkv=2 bf16 (O(T^2) reference)",
                                  "ms": ms}
+        pc = I.config1()
+        q, k, v = (to(x, torch.bfloat16) for x in (pc.q, pc.k, pc.v))
+        g, L, G = to(pc.group_id), to(pc.L), to(pc.G)
+        dy = torch.randn(1, 14, 4096, 64, device=dev)
+        ws = oal.backward_workspace(q, k, v)
+        ms = timed(lambda: oal.backward(q, k, v, g, L, G, pc.eps, dy, workspace=ws), reps=3)
+        res["backward"] = {"workload": "B=1 T=4096 Hq=14 Hkv=2 bf16, chunked O(T) gradients "
+                                       "(dq, dk, dv, dL, deps) on CUDA cores in fp32, including "
+                                       "the fp32 forward it recomputes",
+                           "ms": ms, "tokens_per_s": 4096 / (ms / 1e3)}
     except Exception as exc:
         res["dense_backward"] = {"error": repr(exc)[:300]}
     if oal.device_error() != 0:

@@ -340,6 +340,29 @@ int oal_dense_backward_gpu(const void* q, const void* k, const void* v, const in
                            void* workspace, size_t workspace_bytes, const oal_shape* s,
                            void* stream);
 
+/* Scratch needed by oal_backward for `s` (B, T, Hq, Hkv used): the fp32 prefix and suffix
+ * chunk states (2 x 565,760 bytes per (b, kv head, chunk of 64 tokens)), per row of every
+ * query head its normaliser, output, upstream gradient of u, partial dM and deps, and one
+ * partial dC' (2176 floats) per (b, query head, chunk). */
+int oal_backward_workspace_bytes(const oal_shape* s, size_t* bytes);
+
+/* Training-scale gradients: the same outputs, layouts and conventions as
+ * oal_dense_backward_gpu (dq, dk, dv, dL, deps for dy = dLoss/dyhat), computed as the chunked
+ * reverse of the prefill in O(T) per head instead of O(T^2).  With g_i = dLoss/du_i =
+ * [dy_i / D_i ; -(dy_i . yhat_i) / D_i] and the packed feature map of eq. (5), pairs inside a
+ * 64-token chunk are differentiated directly (eqs. (2)-(3)); pairs across chunks through the
+ * exclusive prefix states S_c = sum psi_j [v_j; 1]^T (eq. (4), as in the prefill) and the
+ * exclusive suffix states R_c = sum phi_i g_i^T of the readout gradient: dphi(q_i) = S_c g_i,
+ * dpsi(k_j) = R_c [v_j; 1], d[v_j; 1] += R_c^T psi(k_j), and dC' = sum_i dphi(q_i) o
+ * (qhat_r qhat_t) mapped through C' = (2 - [r = t]) M_{g(r)g(t)} s_r s_t (+ eps) to dM and
+ * dL = (dM + dM^T) L.  It recomputes yhat and D_i with the fp32 prefill first.  fp32 on CUDA
+ * cores for both input dtypes; deterministic (every sum in a fixed order).  workspace:
+ * oal_backward_workspace_bytes, 256-byte aligned.  Errors as oal_dense_backward_gpu. */
+int oal_backward(const void* q, const void* k, const void* v, const int32_t* group_id,
+                 const float* L, const int32_t* G, float eps, const float* dy, float* dq,
+                 float* dk, float* dv, float* dL, float* deps, void* workspace,
+                 size_t workspace_bytes, const oal_shape* s, void* stream);
+
 /* Sum of prefix states: out[i] = parts[0*n + i] + parts[1*n + i] + ... for the n_parts
  * arrays of n floats stored back to back in `parts`, added in that order (the prefix state of
  * eq. (4) is a sum over tokens, so summing the states of a sequence's first segments, each

@@ -8,6 +8,7 @@
 #include "oal_hadamard.cu"
 #include "oal_varlen.cu"
 #include "oal_backward.cu"
+#include "oal_backward_chunked.cu"
 #include "oal_stateops.cu"
 #include "oal_noalloc.cu"
 #include "oal_chi.cu"

@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(256) state_simt_kernel(const Tin* __restrict__
 // inter (prefill only): u_i += phi(q_i)^T S_c with phi_f(q) = Cp_f qhat_r qhat_t (eq. (5));
 // intra: u_i += sum_j kappa(q_i, k_j) [v_j; 1] over j in [j0, i] with kappa from eqs.
 // (2)-(3) (j0 = start of the chunk for prefill, 0 for the dense form); then
-// yhat_i = u_i[0:64] / u_i[64].
+// yhat_i = u_i[0:64] / u_i[64] (and, when den_out is given, D_i = u_i[64]).
 // ------------------------------------------------------------------------------------------
 struct ReadoutSmem {
     float qs[64][kDA + 1];
@@ -222,7 +222,8 @@ __global__ void __launch_bounds__(256) readout_simt_kernel(
     const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
     const int32_t* __restrict__ gid, const float* __restrict__ L, const int32_t* __restrict__ G,
     float eps, const float* __restrict__ coef, const float* __restrict__ Hc,
-    float* __restrict__ out, int Hq, int Hkv, int T, int C, int NC)
+    float* __restrict__ out, int Hq, int Hkv, int T, int C, int NC,
+    float* __restrict__ den_out)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     ReadoutSmem& sm = *reinterpret_cast<ReadoutSmem*>(smem_raw);
@@ -373,6 +374,7 @@ __global__ void __launch_bounds__(256) readout_simt_kernel(
         const float den = sm.ps[ri][kDV];
         float* o = out + (size_t(bh) * T + i) * kDV;
         for (int n = cg; n < kDV; n += 4) o[n] = sm.ps[ri][n] / den;
+        if (den_out && cg == 0) den_out[size_t(bh) * T + i] = den;  // the normaliser D_i
     }
 }
 
@@ -603,7 +605,7 @@ static int launch_prefill_simt_t(const Tin* q, const Tin* k, const Tin* v,
     OAL_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
     LaunchScope ls("readout_simt", st);
     kern<<<dim3((T + 63) / 64, B * Hq), 256, smem, st>>>(q, k, v, gid, L, G, eps, coef, Hc, out,
-                                                         Hq, Hkv, T, C, NC);
+                                                         Hq, Hkv, T, C, NC, nullptr);
     OAL_LAUNCH_CHECK();
     return OAL_OK;
 }
@@ -634,7 +636,8 @@ static int launch_dense_t(const Tin* q, const Tin* k, const Tin* v, const int32_
     OAL_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
     LaunchScope ls("dense_simt", st);
     kern<<<dim3((T + 63) / 64, B * Hq), 256, smem, st>>>(q, k, v, gid, L, G, eps, nullptr,
-                                                         nullptr, out, Hq, Hkv, T, 64, 1);
+                                                         nullptr, out, Hq, Hkv, T, 64, 1,
+                                                         nullptr);
     OAL_LAUNCH_CHECK();
     return OAL_OK;
 }

@@ -102,10 +102,12 @@ def lib() -> ctypes.CDLL:
             L.oal_prefill_packed.restype = ctypes.c_int
             L.oal_state_prefix_sum.argtypes = [_VP, ctypes.c_int, _SZ, _VP, _VP]
             L.oal_state_prefix_sum.restype = ctypes.c_int
-            L.oal_dense_backward_workspace_bytes.argtypes = [_PS, ctypes.POINTER(_SZ)]
-            L.oal_dense_backward_gpu.argtypes = [_VP] * 6 + [ctypes.c_float] + [_VP] * 7 + [
-                _SZ, _PS, _VP]
-            for name in ("oal_dense_backward_workspace_bytes", "oal_dense_backward_gpu"):
+            for pre in ("oal_dense_backward", "oal_backward"):
+                getattr(L, pre + "_workspace_bytes").argtypes = [_PS, ctypes.POINTER(_SZ)]
+                getattr(L, pre + "_workspace_bytes").restype = ctypes.c_int
+            for name in ("oal_dense_backward_gpu", "oal_backward"):
+                getattr(L, name).argtypes = [_VP] * 6 + [ctypes.c_float] + [_VP] * 7 + [
+                    _SZ, _PS, _VP]
                 getattr(L, name).restype = ctypes.c_int
             for name in ("oal_prefill_host_workspace_bytes", "oal_prefill_host",
                          "oal_prefill_hadamard", "oal_dense_hadamard_gpu",
@@ -537,9 +539,19 @@ def prefill_packed(q, k, v, lens, Hq: int, Hkv: int, group_id, L, G, eps: float,
     return out, states
 
 
+def backward(q, k, v, group_id, L, G, eps: float, dy, stream=None, workspace=None) -> dict:
+    """oal_backward: the training-scale (chunked, O(T)) gradients for dy = dLoss/dyhat
+    [B, Hq, T, 64] fp32.  Returns dict(dq, dk, dv, dL, deps) of fp32 device tensors."""
+    return _backward("oal_backward", q, k, v, group_id, L, G, eps, dy, stream, workspace)
+
+
 def dense_backward(q, k, v, group_id, L, G, eps: float, dy, stream=None) -> dict:
     """oal_dense_backward_gpu: gradients of the dense causal form for dy = dLoss/dyhat
     [B, Hq, T, 64] fp32.  Returns dict(dq, dk, dv, dL, deps) of fp32 device tensors."""
+    return _backward("oal_dense_backward_gpu", q, k, v, group_id, L, G, eps, dy, stream, None)
+
+
+def _backward(name, q, k, v, group_id, L, G, eps, dy, stream, ws) -> dict:
     shape = _shape_of(q, k, v, 64)
     dev = q.device
     dy = dy.to(device=dev, dtype=torch.float32).contiguous()
@@ -548,18 +560,27 @@ def dense_backward(q, k, v, group_id, L, G, eps: float, dy, stream=None) -> dict
     dv_ = torch.empty(v.shape, dtype=torch.float32, device=dev)
     dL = torch.empty(L.shape, dtype=torch.float32, device=dev)
     deps = torch.empty(4, dtype=torch.float32, device=dev)
-    n = _SZ(0)
-    _check(lib().oal_dense_backward_workspace_bytes(ctypes.byref(shape), ctypes.byref(n)),
-           "oal_dense_backward_workspace_bytes")
-    ws = empty_workspace(n.value, dev)
+    if ws is None:
+        n = _SZ(0)
+        query = "oal_backward_workspace_bytes" if name == "oal_backward" else \
+            "oal_dense_backward_workspace_bytes"
+        _check(getattr(lib(), query)(ctypes.byref(shape), ctypes.byref(n)), query)
+        ws = empty_workspace(n.value, dev)
     _contig_cuda(q, k, v, group_id, L, G, dy, dq, dk, dv_, dL, deps, ws)
-    rc = lib().oal_dense_backward_gpu(_ptr(q), _ptr(k), _ptr(v), _ptr(group_id), _ptr(L),
-                                      _ptr(G), float(eps), _ptr(dy), _ptr(dq), _ptr(dk),
-                                      _ptr(dv_), _ptr(dL), _ptr(deps), _ptr(ws),
-                                      ws.numel() * ws.element_size(), ctypes.byref(shape),
-                                      _stream(stream))
-    _check(rc, "oal_dense_backward_gpu")
+    rc = getattr(lib(), name)(_ptr(q), _ptr(k), _ptr(v), _ptr(group_id), _ptr(L), _ptr(G),
+                              float(eps), _ptr(dy), _ptr(dq), _ptr(dk), _ptr(dv_), _ptr(dL),
+                              _ptr(deps), _ptr(ws), ws.numel() * ws.element_size(),
+                              ctypes.byref(shape), _stream(stream))
+    _check(rc, name)
     return dict(dq=dq, dk=dk, dv=dv_, dL=dL, deps=deps[0])
+
+
+def backward_workspace(q, k, v) -> torch.Tensor:
+    """A workspace for backward() on inputs of these shapes (reusable across calls)."""
+    n = _SZ(0)
+    _check(lib().oal_backward_workspace_bytes(ctypes.byref(_shape_of(q, k, v, 64)),
+                                              ctypes.byref(n)), "oal_backward_workspace_bytes")
+    return empty_workspace(n.value, q.device)
 
 
 def launch_count() -> int:

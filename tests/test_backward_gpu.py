@@ -69,3 +69,63 @@ def test_dense_backward_is_reproducible(oal, cuda):
     torch.cuda.synchronize()
     for name in ("dq", "dk", "dv", "dL", "deps"):
         assert torch.equal(a[name], b[name]), name
+
+
+# ---- the training-scale (chunked) backward: oal_backward ---------------------------------
+
+@pytest.mark.parametrize("dtype,B,T,Hq,Hkv", [("f32", 2, 70, 4, 2), ("bf16", 1, 131, 8, 1),
+                                              ("f32", 1, 1, 2, 2), ("f32", 1, 64, 2, 1),
+                                              ("f32", 1, 65, 2, 1), ("bf16", 1, 300, 7, 1)])
+def test_chunked_backward_matches_oracle(oal, cuda, dtype, B, T, Hq, Hkv):
+    """Chunk boundaries at 64 tokens: one partial chunk, exactly one chunk, a one-token
+    second chunk, several chunks; GQA up to 8 query heads per kv head."""
+    p = I.small_layer(800 + T, B=B, T=T, Hq=Hq, Hkv=Hkv, dtype=dtype)
+    rng = np.random.default_rng(T + 1)
+    dy = rng.standard_normal((B, Hq, T, 64))
+    ref = oracle.dense_backward(p.q, p.k, p.v, p.group_id, p.L, p.G, p.eps, dy)
+    q, k, v, g, L, G = dev_inputs(p, cuda)
+    got = oal.backward(q, k, v, g, L, G, p.eps, torch.from_numpy(dy).float())
+    torch.cuda.synchronize()
+    assert oal.device_error() == 0
+    scale = _natural_scales(p, dy)
+    for name in ("dq", "dk", "dv", "dL"):
+        assert _rel(got[name].cpu().numpy(), ref[name], scale[name]) <= 1e-4, name
+    assert abs(float(got["deps"]) - ref["deps"]) <= 1e-4 * max(1.0, abs(ref["deps"]))
+
+
+def test_chunked_backward_matches_dense_gpu(oal, cuda):
+    """Against the dense GPU gradient (independent pair sums) on a longer sequence."""
+    p = I.small_layer(820, B=1, T=700, Hq=14, Hkv=2, dtype="bf16")
+    q, k, v, g, L, G = dev_inputs(p, cuda)
+    dy = torch.randn(1, 14, 700, 64, generator=torch.Generator().manual_seed(5))
+    a = oal.backward(q, k, v, g, L, G, p.eps, dy)
+    b = oal.dense_backward(q, k, v, g, L, G, p.eps, dy)
+    torch.cuda.synchronize()
+    assert oal.device_error() == 0
+    for name in ("dq", "dk", "dv", "dL"):
+        x, y = a[name].double(), b[name].double()
+        assert float((x - y).abs().max() / y.abs().max()) <= 1e-4, name
+    assert abs(float(a["deps"]) - float(b["deps"])) <= 1e-4 * max(1.0, abs(float(b["deps"])))
+
+
+def test_chunked_backward_full_layer_identities(oal, cuda):
+    """A Qwen2.5-0.5B-shaped layer (B=1, T=4096, 14/2 heads, bf16) at training scale: the
+    gradients are reproducible bit for bit and satisfy identities that hold at any size --
+    <dL, L> = -2 eps deps (kappa(cL) = eps + c^2 (kappa - eps), and yhat is a kappa-weighted
+    mean) and sum_j dv_j = sum over tokens and group heads of dy (yhat(v + c) = yhat(v) + c)."""
+    p = I.config1()
+    q, k, v, g, L, G = dev_inputs(p, cuda)
+    dy = torch.randn(1, 14, 4096, 64, generator=torch.Generator().manual_seed(6))
+    ws = oal.backward_workspace(q, k, v)
+    a = oal.backward(q, k, v, g, L, G, p.eps, dy, workspace=ws)
+    b = oal.backward(q, k, v, g, L, G, p.eps, dy, workspace=ws)
+    torch.cuda.synchronize()
+    assert oal.device_error() == 0
+    for name in ("dq", "dk", "dv", "dL", "deps"):
+        assert torch.equal(a[name], b[name]), name
+        assert bool(torch.isfinite(a[name]).all()), name
+    lhs = float((a["dL"].double() * L.double()).sum())
+    assert abs(lhs + 2 * p.eps * float(a["deps"])) <= 1e-3 * float(a["dL"].abs().max())
+    per_kv = dy.double().reshape(1, 2, 7, 4096, 64).sum(dim=(2, 3))
+    got = a["dv"].double().cpu().sum(dim=2)
+    assert float((got - per_kv).abs().max()) <= 1e-3 * float(per_kv.abs().max())
