@@ -38,13 +38,17 @@ namespace rd {
 constexpr int kPhiWarps = 16, kEpiWarp0 = 16, kMmaA = 20, kMmaB = 21, kImgWarp0 = 22;
 constexpr int kWarps = 24;
 constexpr int kThreads = kWarps * 32;
-constexpr int kSlots = 4;            // pair slots (phi in tensor memory + image stage)
+constexpr int kSlots = 4;            // pair slots of phi in tensor memory
+// image stages (pair g in stage g % kStages).  Even and at least kSlots: the next use of the
+// stage holding pair g - 4 is then pair g - 4 + kStages, issued by pair g's MMA issuer after
+// pair g, so a barrier of that stage is never two phases ahead of a waiter (see below).
+constexpr int kStages = 6;
 constexpr int kPairs = kSlices / 2;  // 17
 
 // shared memory (offsets from a 1024-aligned base)
 constexpr uint32_t kOffQ = 0;                                     // 2 x 16 KB Q tiles
-constexpr uint32_t kOffB = 32768;                                 // 4 x 20 KB image stages
-constexpr uint32_t kOffTab = kOffB + kSlots * kImgPairBytes;      // 2 x per-head tables
+constexpr uint32_t kOffB = 32768;                                 // 6 x 20 KB image stages
+constexpr uint32_t kOffTab = kOffB + kStages * kImgPairBytes;     // 2 x per-head tables
 constexpr uint32_t kOffCtl = kOffTab + 2 * kTabBytes;
 constexpr uint32_t kOffUI = kOffCtl + 1024;                       // U_intra rows [128][64] fp32
 constexpr uint32_t kSmemBytes = kOffUI + kC * kDV * 4 + 1024;
@@ -57,7 +61,8 @@ static_assert(kColPhi + kSlots * 64 <= kTmemCols && kColUB + 80 <= kColPhi, "ten
 
 struct Bars {
     uint64_t q_full[2], q_empty[2];
-    uint64_t f_full[kSlots], b_full[kSlots], e[kSlots];  // phi published, image landed, slot free
+    uint64_t f_full[kSlots];                    // phi of the slot's pair published
+    uint64_t b_full[kStages], done_mma[kStages];  // image landed; the stage's pair multiplied
     uint64_t u_full, u_empty, done_a, done_b, ui_full;
 };
 struct Ctl {
@@ -166,10 +171,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bar.q_full[i], 1);
             mbar_init(&bar.q_empty[i], kPhiWarps);
         }
-        for (int i = 0; i < kSlots; ++i) {
-            mbar_init(&bar.f_full[i], 4);
+        for (int i = 0; i < kSlots; ++i) mbar_init(&bar.f_full[i], 4);
+        for (int i = 0; i < kStages; ++i) {
             mbar_init(&bar.b_full[i], 2);
-            mbar_init(&bar.e[i], 1);
+            mbar_init(&bar.done_mma[i], 1);
         }
         mbar_init(&bar.u_full, 2);
         mbar_init(&bar.u_empty, 4);
@@ -185,7 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // image stages: copies fill rows 0..64 of each slice; rows 65..79 (the N = 80 padding of
     // the MMA) stay zero from here on
-    for (int i = threadIdx.x; i < int(kSlots * kImgPairBytes / 16); i += blockDim.x)
+    for (int i = threadIdx.x; i < int(kStages * kImgPairBytes / 16); i += blockDim.x)
         reinterpret_cast<uint4*>(sm + kOffB)[i] = make_uint4(0u, 0u, 0u, 0u);
     fence_proxy_async();
     tc_fence_before();
@@ -209,16 +214,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             const unsigned char* tab = sm + kOffTab + qb * kTabBytes;
             // this set's pairs of the item: g = gp0 + p with g % 4 == set
             for (int p = (set - gp0 % kSlots + kSlots) % kSlots; p < kPairs && ok; p += kSlots) {
-                const int g = gp0 + p, use = g / kSlots;
+                const int g = gp0 + p;
                 uint32_t w[32];
                 phi_slice(qt, tab, 2 * p, row, w);
-                ok = use == 0 || wait_all(&bar.e[set], (use - 1) & 1, abort_flag);
+                // the slot is free once pair g - 4 has been multiplied (the next completion of
+                // that stage's barrier is pair g - 4 + kStages, after pair g on the same issuer)
+                ok = g < kSlots || wait_all(&bar.done_mma[(g - kSlots) % kStages],
+                                            ((g - kSlots) / kStages) & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
                 tmem_st32(slotcol, w);
                 phi_slice(qt, tab, 2 * p + 1, row, w);
                 tmem_st32(slotcol + 32, w);
-                ok = wait_all(&bar.b_full[set], use & 1, abort_flag);
+                ok = wait_all(&bar.b_full[g % kStages], (g / kStages) & 1, abort_flag);
                 if (!ok) break;
                 tmem_st_wait();
                 tc_fence_before();
@@ -327,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 tc_fence_after();
                 if (elect_one()) {
-                    const uint32_t bst = sm0 + kOffB + slot * kImgPairBytes;
+                    const uint32_t bst = sm0 + kOffB + (g % kStages) * kImgPairBytes;
 #pragma unroll
                     for (int x = 0; x < 2; ++x)
 #pragma unroll
@@ -335,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             mma_bf16_ts(ucol, tmem + kColPhi + slot * 64 + x * 32 + ks * 8,
                                         sdesc_sw128(bst + x * kImgSliceBytes + ks * 32, 16, 1024),
                                         id_u, (p > 1 || x > 0 || ks > 0) ? 1u : 0u);
-                    mma_commit(&bar.e[slot]);
+                    mma_commit(&bar.done_mma[g % kStages]);
                 }
                 __syncwarp();
             }
@@ -376,8 +384,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int nidx = idx + gridDim.x;
                 const int row0 = int(item_ref(idx, P, false).chunk) * kSlices * 80;
                 for (int p = 0; p < kPairs; ++p) {
-                    const int g = j * kPairs + p, st = g % kSlots, use = g / kSlots;
-                    if (use >= 1 && !mbar_wait_sleep(&bar.e[st], (use - 1) & 1, abort_flag)) {
+                    // stage st is free once pair g - kStages has been multiplied; the next
+                    // completion of its barrier is pair g's, which needs this copy
+                    const int g = j * kPairs + p, st = g % kStages, use = g / kStages;
+                    if (use >= 1 &&
+                        !mbar_wait_sleep(&bar.done_mma[st], (use - 1) & 1, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -400,8 +411,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             // no copy may still be in flight when the CTA exits
-            for (int g = max(0, issued - kSlots); g < issued; ++g)
-                bounded_spin_done(&bar.b_full[g % kSlots], (g / kSlots) & 1);
+            for (int g = max(0, issued - kStages); g < issued; ++g)
+                bounded_spin_done(&bar.b_full[g % kStages], (g / kStages) & 1);
             for (int i = max(0, lq - 1); i <= lq; ++i)
                 bounded_spin_done(&bar.q_full[i & 1], (i >> 1) & 1);
         }
