@@ -27,6 +27,7 @@
 // Every wait is bounded (1 s); one that runs out sets OAL_ERR_TIMEOUT and the CTA leaves its
 // loops in order (copies drained, MMAs committed, TMEM freed) instead of hanging.
 #include <algorithm>
+#include <atomic>
 #include <cstring>
 #include <mutex>
 #include <utility>
@@ -877,10 +878,37 @@ namespace {
 
 int sm_count()
 {
+    constexpr int kMaxDev = 64;
+    static std::atomic<int> cached[kMaxDev] = {};
     int dev = 0, n = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (dev >= 0 && dev < kMaxDev && (n = cached[dev].load(std::memory_order_relaxed)) > 0)
+        return n;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    if (dev >= 0 && dev < kMaxDev) cached[dev].store(n, std::memory_order_relaxed);
     return n;
+}
+
+// The kernel attributes of the tensor-core prefill, set once per device (they are properties
+// of the kernels in the current device's context).
+cudaError_t set_tc_attributes_once();
+
+// A fork and a join event per host thread and device, reused by every call of that thread
+// (a stream wait takes the event's most recent record at the time it is enqueued).
+bool fork_join_events(cudaEvent_t* fork, cudaEvent_t* join)
+{
+    constexpr int kMaxDev = 64;
+    thread_local cudaEvent_t ev[kMaxDev][2] = {};
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return false;
+    for (int i = 0; i < 2; ++i)
+        if (!ev[dev][i] && cudaEventCreateWithFlags(&ev[dev][i], cudaEventDisableTiming) != cudaSuccess) {
+            ev[dev][i] = nullptr;
+            return false;
+        }
+    *fork = ev[dev][0];
+    *join = ev[dev][1];
+    return true;
 }
 
 }  // namespace
@@ -936,6 +964,33 @@ cudaError_t launch_ex(void (*kern)(Args...), dim3 grid, dim3 block, size_t smem,
 
 namespace {
 
+cudaError_t set_tc_attributes_once()
+{
+    constexpr int kMaxDev = 64;
+    static std::atomic<int> done[kMaxDev] = {};
+    static std::mutex mu;
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < kMaxDev && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    std::lock_guard<std::mutex> g(mu);
+    const std::pair<const void*, int> smem[] = {
+        {reinterpret_cast<const void*>(tc::delta_kernel), int(tc::kSmemBytes)},
+        {reinterpret_cast<const void*>(tc::intra::intra_kernel), int(tc::intra::kSmemBytes)},
+        {reinterpret_cast<const void*>(tc::fm::intra_fm_kernel), int(tc::fm::kSmemBytes)},
+        {reinterpret_cast<const void*>(tc::rd::readout_kernel), int(tc::rd::kSmemBytes)}};
+    for (const auto& k : smem)
+        if ((e = cudaFuncSetAttribute(k.first, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      k.second)) != cudaSuccess)
+            return e;
+    // two intra-chunk CTAs per SM need the whole shared-memory carve-out
+    if ((e = cudaFuncSetAttribute(reinterpret_cast<const void*>(tc::intra::intra_kernel),
+                                  cudaFuncAttributePreferredSharedMemoryCarveout, 100)) != cudaSuccess)
+        return e;
+    if (dev >= 0 && dev < kMaxDev) done[dev].store(1, std::memory_order_release);
+    return cudaSuccess;
+}
+
 // What the scan kernel needs besides Params: the state (or, for a packed batch, the first of
 // the per-sequence states and their stride) and the prep plane's inputs.
 struct ScanArgs {
@@ -959,28 +1014,13 @@ int run_prefill_tc(tc::Params& P, const CUtensorMap& mq, const CUtensorMap& mk,
 {
     const bool with_out = P.out != nullptr;
     const int nsm = sm_count();
-    OAL_CUDA_TRY(cudaFuncSetAttribute(tc::delta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      int(tc::kSmemBytes)));
-    OAL_CUDA_TRY(cudaFuncSetAttribute(tc::intra::intra_kernel,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      int(tc::intra::kSmemBytes)));
-    OAL_CUDA_TRY(cudaFuncSetAttribute(tc::fm::intra_fm_kernel,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      int(tc::fm::kSmemBytes)));
-    OAL_CUDA_TRY(cudaFuncSetAttribute(tc::rd::readout_kernel,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      int(tc::rd::kSmemBytes)));
-    // two intra-chunk CTAs per SM need the whole shared-memory carve-out
-    OAL_CUDA_TRY(cudaFuncSetAttribute(tc::intra::intra_kernel,
-                                      cudaFuncAttributePreferredSharedMemoryCarveout, 100));
-    CallEvents evs;
+    OAL_CUDA_TRY(set_tc_attributes_once());
     cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
     const bool intra = with_out && P.n_intra > 0;
     cudaStream_t st2 = intra ? helper_stream() : nullptr;
     if (intra && st2 == nullptr) return OAL_ERR_CUDA;
     if (intra) {
-        OAL_CUDA_TRY(evs.make(&ev_fork));
-        OAL_CUDA_TRY(evs.make(&ev_join));
+        if (!fork_join_events(&ev_fork, &ev_join)) return OAL_ERR_CUDA;
         OAL_CUDA_TRY(cudaEventRecord(ev_fork, st));
     }
     if (P.n_units > 0) {
