@@ -404,13 +404,13 @@ def main():
     prof = oal.profile_read()
     traced_ms = sum(a.elapsed_time(b) for a, b in evs2) / args.steps
 
-    # roofline of the dominant prefill kernel: the largest share of the kernels that run one
-    # after another on the caller's stream (chunk deltas, scan, readout); the intra-chunk
-    # kernel runs beside the deltas and the scan on the library's helper stream
+    # roofline of the dominant prefill kernel: the largest share of the four kernels, which run
+    # one after another on the caller's stream (deltas, scan, intra-chunk sums, readout; each
+    # a programmatic dependent of the one before)
     per_kernel = kernel_rooflines(prof, kernel_work(p, args.chunk), pk, pk_kind, args.steps)
     roof = None
     if per_kernel:
-        serial = [n for n in per_kernel if n != "intra_tc"] or list(per_kernel)
+        serial = list(per_kernel)
         name = max(serial, key=lambda n: per_kernel[n]["share"])
         d = per_kernel[name]
         roof = {"bound": d["bound"], "achieved": d.get("achieved"), "peak": d["peak"],

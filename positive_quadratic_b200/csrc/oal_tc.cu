@@ -12,13 +12,16 @@
 //     accumulate dS_c = psi(K_c)^T [V_c; 1] in TMEM (the [.; 1] column comes from a constant
 //     "ones" atom addressed through the B descriptor's leading byte offset) and epilogue
 //     warps store it in fp32.
-//   intra-chunk part (oal_tc_intra.cuh; b, h, chunk c), on a helper stream beside the deltas
-//     and the scan: the factored form of eq. (3),
+//   intra-chunk part (oal_tc_intra.cuh; b, h, chunk c), launched after the scan as its
+//     programmatic dependent (it needs only q, k, v, so its CTAs fill SMs as the scan's
+//     blocks retire): the factored form of eq. (3),
 //       kappa = eps + sum_m (L_0m + (q o w_m) . k)^2,   w_m[r] = L_{g(r),m} / sqrt(d)
 //     (= ||L^T sbar||^2): score tiles S_m = (Q o w_m) K^T in TMEM, kappa accumulated in
 //     registers, masked causally and multiplied into [V_c; 1].
 //   prefix scan (SIMT, memory bound): S_c = sum_{c' < c} dS_c' for every chunk, written as
 //     bf16 images of the B operand, and the final state S_NC in fp32 (eq. 4 in chunk form).
+//     (Launch order: deltas, scan, intra-chunk part, readout, each a programmatic dependent of
+//     the one before on the caller's stream.)
 //   inter-chunk readout (oal_tc_readout.cuh; persistent over items b, h, chunk c): phi(Q_c)
 //     is written into tensor memory slice pair by slice pair and multiplied with the image of
 //     S_c by N=80 MMAs reading A from TMEM; the epilogue adds the intra-chunk sum and writes
@@ -36,7 +39,6 @@
 #include <cuda.h>
 
 #include "oal_common.cuh"
-#include "oal_events.cuh"
 #include "oal_kernels.cuh"
 #include "oal_tc_util.cuh"
 
@@ -887,20 +889,6 @@ bool make_map_uncached(CUtensorMap* m, const void* base, int T, int heads)
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// One helper stream per device, created on first use and kept for the process: the
-// intra-chunk kernel runs on it, forked from and joined back into the caller's stream.
-cudaStream_t helper_stream()
-{
-    constexpr int kMaxDev = 64;
-    static std::mutex mu;
-    static cudaStream_t streams[kMaxDev] = {};
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
-    std::lock_guard<std::mutex> g(mu);
-    if (!streams[dev] && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess)
-        streams[dev] = nullptr;
-    return streams[dev];
-}
 
 }  // namespace
 
@@ -926,23 +914,6 @@ int sm_count()
 // of the kernels in the current device's context).
 cudaError_t set_tc_attributes_once();
 
-// A fork and a join event per host thread and device, reused by every call of that thread
-// (a stream wait takes the event's most recent record at the time it is enqueued).
-bool fork_join_events(cudaEvent_t* fork, cudaEvent_t* join)
-{
-    constexpr int kMaxDev = 64;
-    thread_local cudaEvent_t ev[kMaxDev][2] = {};
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return false;
-    for (int i = 0; i < 2; ++i)
-        if (!ev[dev][i] && cudaEventCreateWithFlags(&ev[dev][i], cudaEventDisableTiming) != cudaSuccess) {
-            ev[dev][i] = nullptr;
-            return false;
-        }
-    *fork = ev[dev][0];
-    *join = ev[dev][1];
-    return true;
-}
 
 }  // namespace
 
@@ -1048,37 +1019,16 @@ int run_prefill_tc(tc::Params& P, const CUtensorMap& mq, const CUtensorMap& mk,
     const bool with_out = P.out != nullptr;
     const int nsm = sm_count();
     OAL_CUDA_TRY(set_tc_attributes_once());
-    cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
-    const bool intra = with_out && P.n_intra > 0;
-    cudaStream_t st2 = intra ? helper_stream() : nullptr;
-    if (intra && st2 == nullptr) return OAL_ERR_CUDA;
-    if (intra) {
-        if (!fork_join_events(&ev_fork, &ev_join)) return OAL_ERR_CUDA;
-        OAL_CUDA_TRY(cudaEventRecord(ev_fork, st));
-    }
+    // One stream, each kernel a programmatic dependent of the one before: chunk deltas ->
+    // scan -> intra-chunk sums -> readout.  The intra-chunk kernel needs only q, k, v, so its
+    // CTAs fill SMs as the memory-bound scan's blocks retire instead of waiting for the scan;
+    // it waits for the scan only at its very end, so that its completion (what the readout
+    // waits for) implies the scan's.
     if (P.n_units > 0) {
         const int grid0 = std::max(1, std::min(nsm, P.n_units));
         LaunchScope ls("delta_tc", st);
         OAL_CUDA_TRY(launch_ex(tc::delta_kernel, dim3(grid0), dim3(tc::kThreads), tc::kSmemBytes,
                                st, false, mk, mv, P));
-    }
-    if (intra) {
-        // the intra-chunk sums need only q, k, v: they run on the helper stream beside the
-        // chunk deltas and the scan (latency-bound, they fill SMs the memory-bound scan
-        // leaves idle); chunk 0 of a fresh prefill is final there
-        OAL_CUDA_TRY(cudaStreamWaitEvent(st2, ev_fork, 0));
-        if (fm_intra) {  // free coefficients: Phi(Q_c) Psi(K_c)^T through the feature map
-            LaunchScope ls("intra_fm_tc", st2);
-            OAL_CUDA_TRY(launch_ex(tc::fm::intra_fm_kernel, dim3(P.n_intra),
-                                   dim3(tc::fm::kThreads), tc::fm::kSmemBytes, st2, false, mq,
-                                   mk, mv, P, zin));
-        } else {
-            LaunchScope ls("intra_tc", st2);
-            OAL_CUDA_TRY(launch_ex(tc::intra::intra_kernel, dim3(P.n_intra),
-                                   dim3(tc::intra::kThreads), tc::intra::kSmemBytes, st2, false,
-                                   mq, mk, mv, P, zin));
-        }
-        OAL_CUDA_TRY(cudaEventRecord(ev_join, st2));
     }
     {
         LaunchScope ls("scan", st);
@@ -1090,7 +1040,20 @@ int run_prefill_tc(tc::Params& P, const CUtensorMap& mq, const CUtensorMap& mk,
                                (const tc::SeqDesc*)P.seqs, P.nseq, sa.stride));
     }
     if (!with_out) return OAL_OK;  // no out: the state alone is wanted
-    if (intra) OAL_CUDA_TRY(cudaStreamWaitEvent(st, ev_join, 0));  // intra-chunk sums complete
+    if (P.n_intra > 0) {
+        // chunk 0 of a fresh prefill is final here
+        if (fm_intra) {  // free coefficients: Phi(Q_c) Psi(K_c)^T through the feature map
+            LaunchScope ls("intra_fm_tc", st);
+            OAL_CUDA_TRY(launch_ex(tc::fm::intra_fm_kernel, dim3(P.n_intra),
+                                   dim3(tc::fm::kThreads), tc::fm::kSmemBytes, st, overlap, mq,
+                                   mk, mv, P, zin));
+        } else {
+            LaunchScope ls("intra_tc", st);
+            OAL_CUDA_TRY(launch_ex(tc::intra::intra_kernel, dim3(P.n_intra),
+                                   dim3(tc::intra::kThreads), tc::intra::kSmemBytes, st, overlap,
+                                   mq, mk, mv, P, zin));
+        }
+    }
     if (P.n_read > 0) {
         // persistent: one CTA per SM walks the items (b*h, chunk) with an inter-chunk part
         const int grid2 = std::max(1, std::min(nsm, P.n_read));

@@ -9,8 +9,9 @@
 // One CTA per item (b*h, chunk c), two CTAs per SM so that one CTA's tensor work fills the
 // other's latency chain.  Warps 0-7 (row quarter qw = warp & 3, key half kh = warp >> 2):
 // Aq_m = Q o w_m tiles (dims [32 kh, 32 kh + 32)), kappa over keys [64 kh, 64 kh + 64) of each
-// score tile S_m = Aq_m K^T (tensor memory), the causal P tile, and the epilogue.  Warp 8
-// issues the MMAs (S_m, then U = P [V | 1]); warp 9 loads Q, K, V.
+// score tile S_m = Aq_m K^T (tensor memory, two buffers: tile m + 1 is computed while tile m is
+// read), the causal P tile, and the epilogue.  Warp 8 issues the MMAs (S_m, then
+// U = P [V | 1]); warp 9 loads Q, K, V.
 // Output: a chunk without an inter-chunk part (chunk 0 of a fresh prefill) is complete, so
 // yhat = U[:64] / U[64] goes to `out`; otherwise U[:64] goes to `out` and U[64] to `zin`, and
 // the inter-chunk readout adds phi(q) S_c before normalising.
@@ -21,7 +22,9 @@ constexpr int kWarps = 10;
 constexpr int kThreads = kWarps * 32;
 constexpr int kMmaWarp = 8, kLdWarp = 9;
 constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColS = 0, kColU = 128;
+// score tiles S_m alternate between [0, 128) and [128, 256), so tile m + 1 is computed while
+// tile m is read; U = P [V | 1] reuses [0, 80) once every tile has been read
+constexpr uint32_t kColS = 0, kColU = 0;
 
 // shared memory (offsets from a 1024-aligned base)
 constexpr uint32_t kOffK = 0, kOffV = 16384, kOffQ = 32768, kOffAq = 49152, kOffOnes = 81920;
@@ -32,7 +35,7 @@ constexpr uint32_t kSmemBytes = kOffCtl + 512 + 1024;
 static_assert(kOffCtl % 8 == 0 && 2 * (kSmemBytes + 1024) <= 233472, "two CTAs per SM");
 
 struct Ctl {
-    uint64_t qkv_full, aq_full[2], s_full, s_empty, p_full, u_full, done;
+    uint64_t qkv_full, aq_full[2], s_full[2], s_empty[2], p_full, u_full, done;
     uint32_t tmem_base;
     int abort_flag;
     int G;
@@ -62,8 +65,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         mbar_init(&ctl.qkv_full, 1);
         mbar_init(&ctl.aq_full[0], 8);
         mbar_init(&ctl.aq_full[1], 8);
-        mbar_init(&ctl.s_full, 1);
-        mbar_init(&ctl.s_empty, 8);
+        mbar_init(&ctl.s_full[0], 1);
+        mbar_init(&ctl.s_full[1], 1);
+        mbar_init(&ctl.s_empty[0], 8);
+        mbar_init(&ctl.s_empty[1], 8);
         mbar_init(&ctl.p_full, 8);
         mbar_init(&ctl.u_full, 1);
         mbar_init(&ctl.done, 1);
@@ -147,7 +152,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
         for (int x = 0; x < 64; ++x) acc[x] = 0.f;
         for (int m = 0; m <= G && ok; ++m) {
-            ok = wait_all_sleep(&ctl.s_full, m & 1, abort_flag);
+            ok = wait_all_sleep(&ctl.s_full[m & 1], (m >> 1) & 1, abort_flag);
             if (!ok) break;
             tc_fence_after();
             if (live) {
@@ -155,7 +160,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
                 for (int x = 0; x < 4; ++x) {
                     float v[16];
-                    tmem_ld16(lanebase + kColS + 64 * kh + 16 * x, v);
+                    tmem_ld16(lanebase + kColS + (m & 1) * 128 + 64 * kh + 16 * x, v);
                     tmem_ld_wait();
 #pragma unroll
                     for (int i = 0; i < 16; i += 2) {
@@ -167,7 +172,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 }
             }
             tc_fence_before();
-            warp_arrive(&ctl.s_empty);
+            warp_arrive(&ctl.s_empty[m & 1]);
             if (m + 2 <= G) produce_aq(m + 2);  // S_m completed: its Aq buffer is free
         }
         if (ok) {
@@ -215,16 +220,19 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint32_t vt = smem_u32(sm + kOffV), ones = smem_u32(sm + kOffOnes);
         bool ok = wait_all(&ctl.qkv_full, 0, abort_flag);
         for (int m = 0; m <= G && ok; ++m) {
+            // tile buffer m & 1 is free once tile m - 2 has been read (the next completion of
+            // that barrier is tile m's read, after this MMA)
             ok = wait_all(&ctl.aq_full[m & 1], (m >> 1) & 1, abort_flag);
-            if (ok && m >= 1) ok = wait_all(&ctl.s_empty, (m - 1) & 1, abort_flag);
+            if (ok && m >= 2) ok = wait_all(&ctl.s_empty[m & 1], ((m - 2) >> 1) & 1, abort_flag);
             if (!ok) break;
             tc_fence_after();
             if (elect_one()) {
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16(tmem + kColS, sdesc_sw128(aq0 + (m & 1) * kTileBytes + ks * 32, 16, 1024),
+                    mma_bf16(tmem + kColS + (m & 1) * 128,
+                             sdesc_sw128(aq0 + (m & 1) * kTileBytes + ks * 32, 16, 1024),
                              sdesc_sw128(kt + ks * 32, 16, 1024), id_s, ks > 0 ? 1u : 0u);
-                mma_commit(&ctl.s_full);
+                mma_commit(&ctl.s_full[m & 1]);
             }
             __syncwarp();
         }
@@ -250,6 +258,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         bounded_spin_done(&ctl.qkv_full, 0);  // no copy in flight at exit
     }
 
+    // launched as a dependent of the scan without reading its outputs: complete only after it
+    grid_dep_wait();
     tc_fence_before();
     __syncthreads();
     if (warp == kMmaWarp) {

@@ -250,6 +250,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         bounded_spin_done(&ctl.qkv_full, 0);  // no copy in flight at exit
     }
 
+    // launched as a dependent of the scan without reading its outputs: complete only after it
+    grid_dep_wait();
     tc_fence_before();
     __syncthreads();
     if (warp == kMmaA) {
