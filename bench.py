@@ -462,8 +462,9 @@ def main():
                 "ms_per_step": total_ms / args.steps, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": {"workload": desc, "chunk": args.chunk,
-                           "schedule": "deltas, scan, readout" + (
-                               "" if args.no_overlap else " (programmatic dependent launch)"),
+                           "schedule": "deltas, scan, intra-chunk sums, readout on one stream"
+                           + ("" if args.no_overlap else
+                              ", each a programmatic dependent launch of the one before"),
                            "l2": flush.describe(),
                            "parallelism": f"replicas x{world}"},
                 "roofline": roof, "e2e": e2e, "gpu_launches": int(n_launch),
