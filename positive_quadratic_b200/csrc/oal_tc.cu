@@ -118,13 +118,13 @@ struct Params {
     const CUtensorMap* tm_q;
     const CUtensorMap* tm_k;
     const CUtensorMap* tm_v;
+    const CUtensorMap* tm_img;  // chunk-state images as {64 f, slices * 80 rows}, box {64, 65}
     const int32_t* gid;
     const float* L;
     const int32_t* G;
     float eps;
     const unsigned char* rtab;  // per-head readout tables [Hq][kTabBytes] (workspace)
-    unsigned char* img;      // chunk-state images [B*Hkv][NC][34 slices][80 n][64 f] bf16,
-                             // each 1 KB row group in the 128-byte-swizzled K-major order
+    unsigned char* img;      // chunk-state images [B*Hkv][NC][34 slices][80 n][64 f] bf16
     float* dS;               // chunk deltas [B*Hkv][NC][65][kFP] fp32
     float* out;
     int B, Hq, Hkv, T, NC;
@@ -689,10 +689,10 @@ __device__ __forceinline__ bool wait_all_sleep(uint64_t* bar, uint32_t parity,
 #include "oal_tc_intra_fm.cuh"
 
 // Exclusive prefix over chunks of one (bkv, 64-row slice, 16 columns): image_c =
-// bf16(sum_{c' < c} dS_c') for c >= 1, stored as [80 n][64 f] per slice in the swizzled
-// K-major B-operand layout of the readout's shared-memory stages (rows 65..79 are never
-// written or read -- the readout keeps them zero in shared memory), final state = sum over
-// all chunks.  Thread = (column n, 4 consecutive rows): 16-byte loads, 8 chunks in
+// bf16(sum_{c' < c} dS_c') for c >= 1, stored row-major as [80 n][64 f] per slice (the
+// readout's tensor copy swizzles rows 0..64 into the K-major B-operand layout; rows 65..79
+// are never written or read -- the readout keeps them zero in shared memory), final state =
+// sum over all chunks.  Thread = (column n, 4 consecutive rows): 16-byte loads, 8 chunks in
 // flight, 8-byte image stores.
 // With `prep`, the last z-plane of the grid instead builds the coefficient tables and the
 // state header (one block per query head), which the readout reads after this kernel; without
@@ -715,14 +715,19 @@ __global__ void __launch_bounds__(256) scan_kernel(const float* __restrict__ dS,
     grid_dep_launch();
     if (prep && blockIdx.z == gridDim.z - 1) {  // independent of the deltas: no wait
         const int nb = gridDim.x * gridDim.y, e0 = blockIdx.y * gridDim.x + blockIdx.x;
+        // prep_head keeps its group table in shared memory: every pass of a block's loop ends
+        // with a barrier before the next pass overwrites it
         if (nseq == 0) {
-            for (int e = e0; e < Hq; e += nb)
+            for (int e = e0; e < Hq; e += nb) {
                 prep_head(e, gid, L, G, eps, state, B, Hq, Hkv, tokens, cont != 0, rtab);
+                __syncthreads();
+            }
         } else {  // a packed batch: every sequence's state (B = 1) gets a header and the tables
             for (int e = e0; e < Hq * nseq; e += nb) {
                 const int i = e / Hq;
                 prep_head(e % Hq, gid, L, G, eps, state + size_t(i) * state_stride, 1, Hq, Hkv,
                           seqs[i].T, false, i == 0 ? rtab : nullptr);
+                __syncthreads();
             }
         }
         return;
@@ -759,11 +764,7 @@ __global__ void __launch_bounds__(256) scan_kernel(const float* __restrict__ dS,
     }
     if (n < kW) {
         const float* src = dS + (chunk0 * kW + n) * kFP + f;
-        // row n of the slice image holds packed rows 64 sl .. 64 sl + 63 of column n, stored in
-        // the 128-byte-swizzled order of the readout's shared-memory stage (16-byte chunk c of
-        // row n at chunk position c ^ (n & 7)), so that a plain copy lands it ready for the MMA
-        unsigned char* dst = img + (chunk0 * kSlices + sl) * kImgSliceBytes + n * 128 +
-                             ((((rq >> 1) ^ (n & 7)) << 4) | ((rq & 1) << 3));
+        unsigned char* dst = img + (chunk0 * kSlices + sl) * kImgSliceBytes + n * 128 + 8 * rq;
         const size_t sstride = size_t(kW) * kFP, dstride = size_t(kSlices) * kImgSliceBytes;
         constexpr int kDepth = 8;
         for (int c0 = 0; c0 < NC; c0 += kDepth) {
@@ -832,6 +833,7 @@ EncodeTiledFn encode_fn()
 // [heads][T][64] bf16 viewed as 3D {64, T, heads}; box {64, 128, 1}; 128B swizzle; rows past
 // T read as zero.
 bool make_map_uncached(CUtensorMap* m, const void* base, int T, int heads);
+bool make_img_map_uncached(CUtensorMap* m, const void* base, size_t slices);
 
 // Tensor maps are pure functions of (base address, sizes): the last few of each host thread
 // are kept, so repeated calls on the same buffers skip the encoding.
@@ -889,6 +891,31 @@ bool make_map_uncached(CUtensorMap* m, const void* base, int T, int heads)
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// chunk-state images [slices][80 rows][64] bf16 viewed as 2D {64, slices * 80}; box {64, 65}
+// = rows 0..64 of one slice per copy (rows 65..79 are kept zero in shared memory by the
+// readout and never written by the scan); 128B swizzle on the way in.
+bool make_img_map(CUtensorMap* m, const void* base, size_t slices)
+{
+    MapCacheEntry* slot = nullptr;
+    if (map_cache_get(1, base, (unsigned long long)slices, 0ull, m, &slot)) return true;
+    if (!make_img_map_uncached(m, base, slices)) return false;
+    slot->map = *m;
+    slot->kind = 2;
+    return true;
+}
+
+bool make_img_map_uncached(CUtensorMap* m, const void* base, size_t slices)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {64, cuuint64_t(slices) * 80};
+    const cuuint64_t strides[1] = {128};
+    const cuuint32_t box[2] = {64, kW};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 }  // namespace
 
@@ -1013,7 +1040,7 @@ struct ScanArgs {
 // stream: intra-chunk sums) -> scan -> join -> inter-chunk readout.  P carries the unit and
 // item counts; grids follow from them.
 int run_prefill_tc(tc::Params& P, const CUtensorMap& mq, const CUtensorMap& mk,
-                   const CUtensorMap& mv, float* zin, const ScanArgs& sa,
+                   const CUtensorMap& mv, const CUtensorMap& mi, float* zin, const ScanArgs& sa,
                    int scan_planes, bool fm_intra, bool overlap, cudaStream_t st)
 {
     const bool with_out = P.out != nullptr;
@@ -1059,7 +1086,7 @@ int run_prefill_tc(tc::Params& P, const CUtensorMap& mq, const CUtensorMap& mk,
         const int grid2 = std::max(1, std::min(nsm, P.n_read));
         LaunchScope ls("readout_tc", st);
         OAL_CUDA_TRY(launch_ex(tc::rd::readout_kernel, dim3(grid2), dim3(tc::rd::kThreads),
-                               tc::rd::kSmemBytes, st, overlap, mq, P, (const float*)zin));
+                               tc::rd::kSmemBytes, st, overlap, mq, mi, P, (const float*)zin));
     }
     return OAL_OK;
 }
@@ -1080,11 +1107,12 @@ int launch_prefill_tc(const void* q, const void* k, const void* v, const int32_t
         return OAL_OK;
     }
     unsigned char* wsb = static_cast<unsigned char*>(ws);
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mi;
     // without out (state only) q is not read: its map then describes k and is never used
     if (!(out ? make_map(&mq, q, T, B * Hq) : make_map(&mq, k, T, B * Hkv)) ||
         !make_map(&mk, k, T, B * Hkv) ||
-        !make_map(&mv, v, T, B * Hkv))
+        !make_map(&mv, v, T, B * Hkv) ||
+        !make_img_map(&mi, wsb, size_t(B) * Hkv * NC * tc::kSlices))
         return OAL_ERR_CUDA;
     tc::Params P{};
     P.gid = gid;
@@ -1109,7 +1137,7 @@ int launch_prefill_tc(const void* q, const void* k, const void* v, const int32_t
     P.n_read = B * Hq * (cont ? NC : NC - 1);
     P.nseq = 0;
     ScanArgs sa{body, sb, 0, gid, L, G, eps, (long long)T, fm_intra ? 0 : 1};
-    return run_prefill_tc(P, mq, mk, mv, zin, sa, B * Hkv, fm_intra, overlap, st);
+    return run_prefill_tc(P, mq, mk, mv, mi, zin, sa, B * Hkv, fm_intra, overlap, st);
 }
 
 // ---- packed variable-length batch ----------------------------------------------------------
@@ -1165,8 +1193,11 @@ int launch_prefill_tc_packed(const void* q, const void* k, const void* v, const 
         intra0 += Hq * NC;
         read0 += Hq * std::max(NC - 1, 0);
     }
-    CUtensorMap none;
+    CUtensorMap mi, none;
     std::memset(&none, 0, sizeof(none));
+    if (lay.chunks > 0 && !make_img_map(&mi, wsb, size_t(lay.chunks) * Hkv * tc::kSlices))
+        return OAL_ERR_CUDA;
+    if (lay.chunks == 0) mi = none;
     // descriptors and tensor maps into the workspace, ahead of the kernels on the same stream
     OAL_CUDA_TRY(cudaMemcpyAsync(wsb + lay.seqs, sd.data(), sd.size() * sizeof(tc::SeqDesc),
                                  cudaMemcpyHostToDevice, st));
@@ -1196,7 +1227,7 @@ int launch_prefill_tc_packed(const void* q, const void* k, const void* v, const 
     P.seqs = reinterpret_cast<const tc::SeqDesc*>(wsb + lay.seqs);
     P.maps = reinterpret_cast<const CUtensorMap*>(wsb + lay.maps);
     ScanArgs sa{nullptr, states, stride, gid, L, G, eps, 0, 1};
-    return run_prefill_tc(P, none, none, none, zin, sa, n * Hkv, false, overlap, st);
+    return run_prefill_tc(P, none, none, none, mi, zin, sa, n * Hkv, false, overlap, st);
 }
 
 }  // namespace oal

@@ -25,10 +25,10 @@
 //                barrier wait, fence or commit stalls the issuing thread for a few hundred
 //                cycles while the tensor pipe drains its short queue; with two issuers one
 //                issues while the other waits.  U_A + U_B is summed in a fixed order.
-//   warps 22, 23 state-image copies of the even and odd pairs: one plain bulk copy per pair
-//                (the issuing warps compete with the producers for issue slots, so the copy
-//                path is kept to a few instructions per pair).  Warp 22 also loads the Q tile
-//                and per-head coefficient table one item ahead (double-buffered).
+//   warps 22, 23 state-image copies, one slice (10 KB) of each pair each: a single thread's
+//                bulk-copy queue moves about 40 B/clk, two threads twice that.  Warp 22 also
+//                loads the Q tile and per-head coefficient table one item ahead
+//                (double-buffered).
 // Tensor memory (512 columns): U_A [0, 80), U_B [96, 176), phi slots [192, 448).
 // Every wait is bounded; one that runs out sets OAL_ERR_TIMEOUT and every role leaves its loop
 // in order (copies drained, MMAs committed, tensor memory freed by the allocating warp).
@@ -43,8 +43,6 @@ constexpr int kSlots = 4;            // pair slots of phi in tensor memory
 // stage holding pair g - 4 is then pair g - 4 + kStages, issued by pair g's MMA issuer after
 // pair g, so a barrier of that stage is never two phases ahead of a waiter (see below).
 constexpr int kStages = 6;
-// one pair's copy: slice 2p (80 rows) and the 65 live rows of slice 2p + 1
-constexpr uint32_t kImgPairLoadBytes = kImgSliceBytes + kImgLoadBytes;
 constexpr int kPairs = kSlices / 2;  // 17
 
 // shared memory (offsets from a 1024-aligned base)
@@ -153,7 +151,8 @@ __device__ __forceinline__ void phi_slice(const unsigned char* qt, const unsigne
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    readout_kernel(const __grid_constant__ CUtensorMap tm_q, Params P,
+    readout_kernel(const __grid_constant__ CUtensorMap tm_q,
+                   const __grid_constant__ CUtensorMap tm_img, Params P,
                    const float* __restrict__ zin)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -165,6 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_items = P.n_read;
     P.tm_q = &tm_q;
+    P.tm_img = &tm_img;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int i = 0; i < kSlots; ++i) mbar_init(&bar.f_full[i], 4);
         for (int i = 0; i < kStages; ++i) {
-            mbar_init(&bar.b_full[i], 1);
+            mbar_init(&bar.b_full[i], 2);
             mbar_init(&bar.done_mma[i], 1);
         }
         mbar_init(&bar.u_full, 2);
@@ -358,15 +358,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) bounded_spin_done(done, 0);
         __syncwarp();
     } else if (warp < kImgWarp0 + 2) {
-        // ---- state-image copies: warp x = warp - kImgWarp0 copies the pairs p = x (mod 2), one
-        // plain bulk copy of both slices (the second slice's 65 live rows and the first's 80 rows;
-        // the scan stores each slice in the swizzled order of the shared-memory stage, and the
-        // first slice's padding rows only reach unused accumulator columns).  Lane 0 of warp
-        // x = 0 also loads the Q tile and table of item j + 1 while item j's images stream ----
+        // ---- state-image copies: slice x = warp - kImgWarp0 of every pair (80 rows, 10 KB);
+        // warp x = 0 also loads Q tile + table of item j + 1 while item j's images stream ----
         const int x = warp - kImgWarp0;
         if (lane == 0) {
-            int lq = -1, nm = 0;
-            int mine[3] = {0, 0, 0};  // this warp's last three copies (distinct stages)
+            int issued = 0, lq = -1;
             bool ok = true;
             auto load_q = [&](int jj, int qidx) {
                 if (P.skip_copies) return;
@@ -386,8 +382,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             for (int j = 0, idx = blockIdx.x; idx < n_items && ok; ++j, idx += gridDim.x) {
                 const int nidx = idx + gridDim.x;
-                const unsigned char* src = P.img + item_ref(idx, P, false).chunk * kImgChunkBytes;
-                for (int p = x; p < kPairs; p += 2) {
+                const int row0 = int(item_ref(idx, P, false).chunk) * kSlices * 80;
+                for (int p = 0; p < kPairs; ++p) {
                     // stage st is free once pair g - kStages has been multiplied; the next
                     // completion of its barrier is pair g's, which needs this copy
                     const int g = j * kPairs + p, st = g % kStages, use = g / kStages;
@@ -397,11 +393,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     if (!P.skip_copies) {
-                        mbar_expect_tx(&bar.b_full[st], kImgPairLoadBytes);
-                        bulk_g2s(sm + kOffB + st * kImgPairBytes, src + size_t(p) * kImgPairBytes,
-                                 kImgPairLoadBytes, &bar.b_full[st]);
-                        mine[nm % 3] = g;
-                        ++nm;
+                        mbar_expect_tx(&bar.b_full[st], kImgLoadBytes);
+                        tma_load_2d(sm + kOffB + st * kImgPairBytes + x * kImgSliceBytes,
+                                    P.tm_img, &bar.b_full[st], 0, row0 + 160 * p + 80 * x);
+                        issued = g + 1;
                     }
                     if (x == 0 && p == kSlots && j >= 1 && nidx < n_items) {
                         // buffer (j + 1) & 1 is free once the producers finished item j - 1,
@@ -416,8 +411,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             // no copy may still be in flight when the CTA exits
-            for (int i = max(0, nm - 3); i < nm; ++i)
-                bounded_spin_done(&bar.b_full[mine[i % 3] % kStages], (mine[i % 3] / kStages) & 1);
+            for (int g = max(0, issued - kStages); g < issued; ++g)
+                bounded_spin_done(&bar.b_full[g % kStages], (g / kStages) & 1);
             for (int i = max(0, lq - 1); i <= lq; ++i)
                 bounded_spin_done(&bar.q_full[i & 1], (i >> 1) & 1);
         }

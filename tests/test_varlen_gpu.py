@@ -60,9 +60,13 @@ def _layer_batch(cuda, lens, Hq, Hkv, seed):
     return base, g, L, G, probs, qs, ks, vs
 
 
+_SHORT64 = [int(x) for x in np.random.default_rng(7).integers(64, 321, size=64)]
+
+
 @pytest.mark.parametrize("lens,Hq,Hkv", [([300, 0, 129, 1000, 1, 128, 127, 640], 14, 2),
                                          ([5] * 40 + [700, 0, 0, 33], 4, 2),
-                                         ([2048, 64, 1500], 8, 1)])
+                                         ([2048, 64, 1500], 8, 1),
+                                         (_SHORT64, 14, 2)])
 def test_packed_equals_separate_prefills(oal, cuda, lens, Hq, Hkv):
     """One launch per kernel for the whole batch gives each sequence exactly what an
     oal_prefill of it alone gives (same per-chunk arithmetic and summation order), outputs
