@@ -8,9 +8,10 @@
 // (U_intra[:64] in `out`, U_intra[64] in the workspace).
 //
 // One CTA per SM walks a static list of items (b*h, chunk c >= 1, or every chunk when the call
-// continues a prefix).  Work moves in slice pairs: a pair is 2 x 64 packed rows, its phi in a
-// tensor-memory slot of 64 columns and its state image in a 20 KB shared-memory stage with the
-// same index g % 4 (g counts pairs over all items of the CTA).
+// continues a prefix).  Work moves in slice pairs: a pair is 2 x 64 packed rows, its phi in
+// tensor-memory slot g % 4 (64 columns) and its state image in 20 KB shared-memory stage g % 6
+// (g counts pairs over all items of the CTA), so the image copies run two pairs ahead of the
+// phi slots.
 // Roles (24 warps):
 //   warps 0-15   phi producers: set = warp >> 2 produces the pairs g = set (mod 4) into slot
 //                `set`, row quarter = warp & 3; phi of both slices, then (after the slot and
@@ -25,10 +26,10 @@
 //                barrier wait, fence or commit stalls the issuing thread for a few hundred
 //                cycles while the tensor pipe drains its short queue; with two issuers one
 //                issues while the other waits.  U_A + U_B is summed in a fixed order.
-//   warps 22, 23 state-image copies, one slice (10 KB) of each pair each: a single thread's
-//                bulk-copy queue moves about 40 B/clk, two threads twice that.  Warp 22 also
-//                loads the Q tile and per-head coefficient table one item ahead
-//                (double-buffered).
+//   warps 22, 23 state-image copies, one slice of each pair each: one tiled tensor copy of
+//                the slice's 65 live rows (the 15 padding rows of the N = 80 operand stay zero
+//                from the CTA's start).  Warp 22 also loads the Q tile and per-head
+//                coefficient table one item ahead (double-buffered).
 // Tensor memory (512 columns): U_A [0, 80), U_B [96, 176), phi slots [192, 448).
 // Every wait is bounded; one that runs out sets OAL_ERR_TIMEOUT and every role leaves its loop
 // in order (copies drained, MMAs committed, tensor memory freed by the allocating warp).
@@ -358,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) bounded_spin_done(done, 0);
         __syncwarp();
     } else if (warp < kImgWarp0 + 2) {
-        // ---- state-image copies: slice x = warp - kImgWarp0 of every pair (80 rows, 10 KB);
+        // ---- state-image copies: slice x = warp - kImgWarp0 of every pair (65 of its 80 rows);
         // warp x = 0 also loads Q tile + table of item j + 1 while item j's images stream ----
         const int x = warp - kImgWarp0;
         if (lane == 0) {
