@@ -1075,8 +1075,10 @@ int run_prefill_tc(tc::Params& P, const CUtensorMap& mq, const CUtensorMap& mk,
                                    dim3(tc::fm::kThreads), tc::fm::kSmemBytes, st, overlap, mq,
                                    mk, mv, P, zin));
         } else {
+            // persistent: two CTAs per SM walk the items (b*h, chunk)
+            const int grid1 = std::max(1, std::min(tc::intra::kCtasPerSm * nsm, P.n_intra));
             LaunchScope ls("intra_tc", st);
-            OAL_CUDA_TRY(launch_ex(tc::intra::intra_kernel, dim3(P.n_intra),
+            OAL_CUDA_TRY(launch_ex(tc::intra::intra_kernel, dim3(grid1),
                                    dim3(tc::intra::kThreads), tc::intra::kSmemBytes, st, overlap,
                                    mq, mk, mv, P, zin));
         }
