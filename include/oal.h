@@ -120,9 +120,10 @@ int oal_prefill_workspace_bytes(const oal_shape* s, size_t* bytes);
 typedef enum { OAL_PATH_CUDA_CORE = 0, OAL_PATH_TENSOR = 1 } oal_path;
 int oal_prefill_path(const oal_shape* s, int* path);
 
-/* Scratch needed by oal_decode_step for `s` (B, Hq, Hkv used).  It MUST be zero-filled once
- * before the first decode call.  Its first 256-byte-aligned block holds one completion ticket
- * per (b, kv) that every completed call returns to zero; the rest is per-call scratch. */
+/* Scratch needed by oal_decode_step for `s` (B, Hq, Hkv used): per-call partial readouts
+ * (one per 240-row slab of each (b, kv) and query head), written and then read by the same
+ * call, so its contents between calls do not matter.  (Its first 256-byte-aligned block is
+ * reserved; earlier versions kept completion tickets there.) */
 int oal_decode_workspace_bytes(const oal_shape* s, size_t* bytes);
 
 /* Causal prefill of T tokens: writes out = yhat for every token (eqs. (2)-(5)) and fills
@@ -177,8 +178,7 @@ int oal_decode_step(const void* q, const void* k, const void* v, void* state, fl
  * and caches it; make that first call before any stream capture.  cudaDeviceReset discards
  * the library's device code and data on that device, and with them the array the cached
  * address points to: do not call this entry point on a device after resetting it in the
- * same process.  Every call shares the one array and
- * clears the part that must start at zero itself, so calls that overlap on the GPU (on
+ * same process.  Every call shares the one array, so calls that overlap on the GPU (on
  * different streams, or from threads that do not order their calls) race and corrupt each
  * other's results: issue them one after another. */
 int oal_decode_step_noalloc(const void* q, const void* k, const void* v, void* state,

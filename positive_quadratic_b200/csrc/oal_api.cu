@@ -194,9 +194,8 @@ int oal_decode_step(const void* q, const void* k, const void* v, void* state, fl
     if (!aligned16(workspace)) return OAL_ERR_ALIGN;
     unsigned char* ws = static_cast<unsigned char*>(workspace);
     return launch_decode(q, k, v, state, out,
-                         reinterpret_cast<float*>(ws + decode_ticket_bytes(s)),
-                         reinterpret_cast<unsigned int*>(ws), s->B, s->Hq, s->Hkv, s->dtype,
-                         static_cast<cudaStream_t>(stream));
+                         reinterpret_cast<float*>(ws + decode_ticket_bytes(s)), s->B, s->Hq,
+                         s->Hkv, s->dtype, static_cast<cudaStream_t>(stream));
 }
 
 int oal_dense_ref_gpu(const void* q, const void* k, const void* v, const int32_t* group_id,

@@ -23,7 +23,7 @@ int launch_dense(const void* q, const void* k, const void* v, const int32_t* gid
 int decode_slabs();
 
 int launch_decode(const void* q, const void* k, const void* v, void* state, float* out,
-                  float* part, unsigned int* tickets, int B, int Hq, int Hkv, int dtype,
+                  float* part, int B, int Hq, int Hkv, int dtype,
                   cudaStream_t st);
 
 // ungrouped Hadamard form (oal_hadamard.cu): prefill on CUDA cores, or the dense O(T^2) form

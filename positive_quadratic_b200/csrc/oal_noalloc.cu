@@ -12,8 +12,8 @@
 
 namespace oal {
 
-// 4 MiB: room for the per-(b, kv) tickets and per-slab partial readouts (9 slabs x 65 fp32
-// per query head) of a decode step with B*Hq up to 1788 query heads (batch 64 x 14 heads
+// 4 MiB: room for the reserved leading block and the per-slab partial readouts (9 slabs x 65
+// fp32 per query head) of a decode step with B*Hq up to 1788 query heads (batch 64 x 14 heads
 // needs 2.1 MB).
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
 
@@ -64,9 +64,8 @@ extern "C" int oal_decode_step_noalloc(const void* q, const void* k, const void*
     if ((rc = noalloc_scratch(&scratch))) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     unsigned char* ws = static_cast<unsigned char*>(scratch);
-    // The array keeps whatever the previous call left; the tickets must start at zero.
-    OAL_CUDA_TRY(cudaMemsetAsync(ws, 0, decode_ticket_bytes(s), st));
+    // every word of the scratch that a step reads, the step itself wrote first
     return launch_decode(q, k, v, state, out,
-                         reinterpret_cast<float*>(ws + decode_ticket_bytes(s)),
-                         reinterpret_cast<unsigned int*>(ws), s->B, s->Hq, s->Hkv, s->dtype, st);
+                         reinterpret_cast<float*>(ws + decode_ticket_bytes(s)), s->B, s->Hq,
+                         s->Hkv, s->dtype, st);
 }

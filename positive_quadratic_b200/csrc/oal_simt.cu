@@ -385,9 +385,9 @@ __global__ void __launch_bounds__(256) readout_simt_kernel(
 // moves as 128-bit loads and stores (a half warp per 256-byte row), the first rows requested
 // before the per-row weights are formed and every batch of rows prefetched while the previous
 // one is computed.  Per-block partial u go to the workspace in a fixed order (warp partials
-// summed in shared memory, no float atomics); the last block of a (b, kv) (atomic ticket)
-// sums the slab partials in slab order, writes yhat and re-arms the ticket.  Every sum has a
-// fixed order, so a step is bit-reproducible.
+// summed in shared memory, no float atomics); decode_finish_kernel, launched as a
+// programmatic dependent, sums the slab partials in slab order and writes yhat.  Every sum
+// has a fixed order, so a step is bit-reproducible.
 // ------------------------------------------------------------------------------------------
 // 9 slabs of 240 packed rows per (b, kv) head: 256 threads with at most 64 registers, so four
 // blocks share an SM (592 resident) and a batch-64 step (1152 blocks) takes 1.95 waves -- the
@@ -405,7 +405,6 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const Tin* __res
                                                               unsigned char* __restrict__ state,
                                                               float* __restrict__ out,
                                                               float* __restrict__ part,
-                                                              unsigned int* __restrict__ tickets,
                                                               int Hq, int Hkv)
 {
     const int slab = blockIdx.x, bkv = blockIdx.y, nslab = gridDim.x;
@@ -426,8 +425,6 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const Tin* __res
     constexpr int kRec = kGrp <= 7 ? 8 : 12, kPsi = kGrp <= 7 ? 7 : 8;
     __shared__ __align__(16) float wrow[kDecRows][kRec];
     __shared__ float red[kDecWarps][kMaxGroup][kW];
-    __shared__ float ufin[kMaxGroup][kW];
-    __shared__ int s_last;
 
     const int f0 = slab * kDecRows;
     const int nrows = max(0, min(kDecRows, kF - f0));
@@ -441,6 +438,18 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const Tin* __res
             hv[x] = __ldcs(reinterpret_cast<const float4*>(Hv + size_t(f0 + row) * kDV) + lane4);
     }
 
+    // this thread's row of the slab (kDecRows < kDecThreads: at most one): its readout
+    // coefficients and z entry are requested now too, so that their latency overlaps the
+    // loads of q, k, v below
+    static_assert(kDecRows <= kDecThreads, "one prologue row per thread");
+    const bool has_row = tid < nrows;
+    float cpre[kGrp];
+    float zpre = 0.f;
+    if (has_row) {
+#pragma unroll
+        for (int g = 0; g < kGrp; ++g) cpre[g] = coef[size_t(h0 + g) * kFP + f0 + tid];
+        zpre = z[f0 + tid];
+    }
     if (tid < kD) {
         kh[tid] = to_f32(k[size_t(bkv) * kD + tid]);
         vh[tid] = to_f32(v[size_t(bkv) * kDV + tid]);
@@ -454,13 +463,13 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const Tin* __res
         qh[g][r] = r < kD ? to_f32(q[(size_t(b) * Hq + h0 + g) * kD + r]) : (r == kD ? 1.f : 0.f);
     }
     __syncthreads();
-    for (int row = tid; row < nrows; row += kDecThreads) {
-        const int f = f0 + row;
-        const RT rt = feature_rt(f);
+    if (has_row) {
+        const int row = tid;
+        const RT rt = feature_rt(f0 + row);
         float w[kRec];
 #pragma unroll
         for (int g = 0; g < kRec; ++g)
-            w[g] = g < grp ? coef[size_t(h0 + g) * kFP + f] * qh[g][rt.r] * qh[g][rt.t] : 0.f;
+            w[g] = g < grp ? cpre[g < grp ? g : 0] * qh[g][rt.r] * qh[g][rt.t] : 0.f;
         w[kPsi] = kh[rt.r] * kh[rt.t];
 #pragma unroll
         for (int x = 0; x < kRec; x += 4)
@@ -518,8 +527,9 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const Tin* __res
     float accz[kGrp];
 #pragma unroll
     for (int g = 0; g < kGrp; ++g) accz[g] = 0.f;
-    for (int row = tid; row < nrows; row += kDecThreads) {
-        const float zz = z[f0 + row] + wrow[row][kPsi];
+    if (has_row) {
+        const int row = tid;
+        const float zz = zpre + wrow[row][kPsi];
         z[f0 + row] = zz;
         const float* ph = wrow[row];
 #pragma unroll
@@ -548,31 +558,38 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const Tin* __res
         for (int w = 0; w < kDecWarps; ++w) sum += red[w][e / kW][e % kW];
         mypart[e] = sum;
     }
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-        const unsigned int prev = atomicAdd(&tickets[bkv], 1u);
-        s_last = (prev == unsigned(nslab - 1));
-    }
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
+    // the finishing kernel (a programmatic dependent) may launch once every block is here; it
+    // waits for this grid's completion before reading the partials
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// The end of a decode step: per (b, kv) the slab partials summed in slab order, yhat =
+// u[:64] / u[64] for the Hq/Hkv query heads, and the token count of the state header.
+// One block per (b, kv); launched as a programmatic dependent of decode_kernel.
+template <int kGrp>
+__global__ void __launch_bounds__(256) decode_finish_kernel(const float* __restrict__ part,
+                                                            float* __restrict__ out,
+                                                            unsigned char* __restrict__ state,
+                                                            int Hq, int Hkv, int nslab)
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // the partials are complete
+    constexpr int grp = kGrp;
+    const int bkv = blockIdx.x, b = bkv / Hkv, kv = bkv % Hkv, h0 = kv * grp;
+    __shared__ float ufin[kMaxGroup][kW];
     const float* allpart = part + size_t(bkv) * nslab * grp * kW;
-    for (int e = tid; e < grp * kW; e += kDecThreads) {
+    for (int e = threadIdx.x; e < grp * kW; e += blockDim.x) {
         float s = 0.f;
-        for (int sl = 0; sl < nslab; ++sl) s += __ldcg(allpart + size_t(sl) * grp * kW + e);
+        for (int sl = 0; sl < nslab; ++sl) s += allpart[size_t(sl) * grp * kW + e];
         ufin[e / kW][e % kW] = s;
     }
     __syncthreads();
-    for (int e = tid; e < grp * kDV; e += kDecThreads) {
+    for (int e = threadIdx.x; e < grp * kDV; e += blockDim.x) {
         const int g = e / kDV, n = e % kDV;
         out[(size_t(b) * Hq + h0 + g) * kDV + n] = ufin[g][n] / ufin[g][kDV];
     }
-    if (tid == 0) {
-        tickets[bkv] = 0u;
-        if (bkv == 0) reinterpret_cast<StateHeader*>(state)->tokens += 1;
-    }
+    if (threadIdx.x == 0 && bkv == 0) reinterpret_cast<StateHeader*>(state)->tokens += 1;
 }
+
 int launch_prep(const int32_t* gid, const float* L, const int32_t* G, float eps, void* state,
                 int B, int Hq, int Hkv, long long tokens, cudaStream_t st)
 {
@@ -658,38 +675,54 @@ int launch_dense(const void* q, const void* k, const void* v, const int32_t* gid
 int decode_slabs() { return (kF + kDecRows - 1) / kDecRows; }
 
 int launch_decode(const void* q, const void* k, const void* v, void* state, float* out,
-                  float* part, unsigned int* tickets, int B, int Hq, int Hkv, int dtype,
-                  cudaStream_t st)
+                  float* part, int B, int Hq, int Hkv, int dtype, cudaStream_t st)
 {
     if (B == 0) return OAL_OK;
     const dim3 grid(decode_slabs(), B * Hkv);
     unsigned char* s = static_cast<unsigned char*>(state);
-    LaunchScope ls("decode", st);
     const int grp = Hq / Hkv;
     const bool bf = dtype == OAL_BF16;
-    auto go = [&](auto G) {
+    auto go = [&](auto G) -> cudaError_t {
         constexpr int g = decltype(G)::value;
-        if (bf)
-            decode_kernel<__nv_bfloat16, g><<<grid, kDecThreads, 0, st>>>(
-                static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-                static_cast<const __nv_bfloat16*>(v), s, out, part, tickets, Hq, Hkv);
-        else
-            decode_kernel<float, g><<<grid, kDecThreads, 0, st>>>(
-                static_cast<const float*>(q), static_cast<const float*>(k),
-                static_cast<const float*>(v), s, out, part, tickets, Hq, Hkv);
+        {
+            LaunchScope ls("decode", st);
+            if (bf)
+                decode_kernel<__nv_bfloat16, g><<<grid, kDecThreads, 0, st>>>(
+                    static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                    static_cast<const __nv_bfloat16*>(v), s, out, part, Hq, Hkv);
+            else
+                decode_kernel<float, g><<<grid, kDecThreads, 0, st>>>(
+                    static_cast<const float*>(q), static_cast<const float*>(k),
+                    static_cast<const float*>(v), s, out, part, Hq, Hkv);
+            const cudaError_t e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+        }
+        LaunchScope ls("decode_finish", st);
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3(B * Hkv);
+        cfg.blockDim = dim3(256);
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, decode_finish_kernel<g>, static_cast<const float*>(part),
+                                  out, s, Hq, Hkv, int(grid.x));
     };
+    cudaError_t e;
     switch (grp) {
-        case 1: go(std::integral_constant<int, 1>{}); break;
-        case 2: go(std::integral_constant<int, 2>{}); break;
-        case 3: go(std::integral_constant<int, 3>{}); break;
-        case 4: go(std::integral_constant<int, 4>{}); break;
-        case 5: go(std::integral_constant<int, 5>{}); break;
-        case 6: go(std::integral_constant<int, 6>{}); break;
-        case 7: go(std::integral_constant<int, 7>{}); break;
-        case 8: go(std::integral_constant<int, 8>{}); break;
+        case 1: e = go(std::integral_constant<int, 1>{}); break;
+        case 2: e = go(std::integral_constant<int, 2>{}); break;
+        case 3: e = go(std::integral_constant<int, 3>{}); break;
+        case 4: e = go(std::integral_constant<int, 4>{}); break;
+        case 5: e = go(std::integral_constant<int, 5>{}); break;
+        case 6: e = go(std::integral_constant<int, 6>{}); break;
+        case 7: e = go(std::integral_constant<int, 7>{}); break;
+        case 8: e = go(std::integral_constant<int, 8>{}); break;
         default: return OAL_ERR_UNSUPPORTED;
     }
-    OAL_LAUNCH_CHECK();
+    OAL_CUDA_TRY(e);
     return OAL_OK;
 }
 

@@ -324,7 +324,7 @@ def decode_step(q, k, v, state, workspace, out=None, stream=None):
 
 
 def decode_workspace(B, Hq, Hkv, device) -> torch.Tensor:
-    """Zero-filled decode workspace (the ABI requires zeros before the first step)."""
+    """Decode workspace (zero-filled; a step writes every scratch word before reading it)."""
     n = decode_workspace_bytes(make_shape(B, 1, Hq, Hkv))
     return torch.zeros(max(n, 256), dtype=torch.uint8, device=device)
 

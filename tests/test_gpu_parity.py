@@ -184,11 +184,30 @@ def test_decode_continuation(oal, cuda, dtype):
         torch.cuda.synchronize()
         assert row_rel_err(y.cpu().numpy()[:, :, 0], y_all[:, :, t]) <= tol(p)
     assert oal.device_error() == 0
-    assert torch.all(ws[:256] == 0)  # completion tickets return to zero
+    assert torch.all(ws[:256] == 0)  # the reserved leading block is never written
     hdr, _, S = read_state(state.cpu().numpy(), 3, 14, 2)
     assert hdr["tokens"] == T0 + n
     ref = pack_oracle_state(st_all)
     assert np.max(np.abs(S[:, :, :F] - ref) / np.abs(ref).max(axis=2, keepdims=True)) < 1e-5
+
+
+def test_decode_workspace_contents_do_not_matter(oal, cuda):
+    """A decode step writes every scratch word it reads: a workspace full of garbage gives the
+    same outputs and state, bit for bit, as a zero-filled one."""
+    p = I.small_layer(309, B=2, T=65, Hq=14, Hkv=2, dtype="bf16")
+    pre = p.slice_tokens(0, 64)
+    q, k, v, _, _, _ = dev_inputs(p, cuda)
+    sl = lambda x: x[:, :, 64:65].contiguous()  # noqa: E731
+    res = []
+    for fill in (0, 0xFF):
+        _, state = gpu_prefill(oal, pre, cuda, 128)
+        ws = oal.decode_workspace(2, 14, 2, cuda)
+        ws.fill_(fill)
+        y = oal.decode_step(sl(q), sl(k), sl(v), state, ws)
+        torch.cuda.synchronize()
+        res.append((y.clone(), state.clone()))
+    assert oal.device_error() == 0
+    assert torch.equal(res[0][0], res[1][0]) and torch.equal(res[0][1], res[1][1])
 
 
 def test_chunk_size_independence(oal, cuda):
