@@ -577,9 +577,17 @@ __global__ void __launch_bounds__(256) decode_finish_kernel(const float* __restr
     const int bkv = blockIdx.x, b = bkv / Hkv, kv = bkv % Hkv, h0 = kv * grp;
     __shared__ float ufin[kMaxGroup][kW];
     const float* allpart = part + size_t(bkv) * nslab * grp * kW;
+    constexpr int kSlabs = (kF + kDecRows - 1) / kDecRows;  // the grid's slab count
     for (int e = threadIdx.x; e < grp * kW; e += blockDim.x) {
+        // every slab's partial requested at once, then summed in slab order
+        float pv[kSlabs];
+#pragma unroll
+        for (int sl = 0; sl < kSlabs; ++sl)
+            pv[sl] = sl < nslab ? allpart[size_t(sl) * grp * kW + e] : 0.f;
         float s = 0.f;
-        for (int sl = 0; sl < nslab; ++sl) s += allpart[size_t(sl) * grp * kW + e];
+#pragma unroll
+        for (int sl = 0; sl < kSlabs; ++sl)
+            if (sl < nslab) s += pv[sl];
         ufin[e / kW][e % kW] = s;
     }
     __syncthreads();
