@@ -22,7 +22,8 @@
 //   forward  : coefficients, exclusive prefix states S_c (fp32), yhat and D for every row;
 //   g        : the upstream gradient rows g_i;
 //   intra    : rows (dq, the row's dM and deps) and keys (dk, dv) over within-chunk pairs;
-//   suffix   : R_c for every chunk (a reverse exclusive scan over chunks);
+//   suffix   : R_c for every chunk (each chunk's sum, chunk-parallel, then a reverse exclusive
+//              scan over chunks);
 //   inter    : rows add S_c g_i through phi to dq and leave per-(head, chunk) partial dC';
 //              keys add R_c w_j through psi to dk and R_c^T psi_j to dv;
 //   heads    : dM from the row partials and dC', dL, deps.
@@ -182,13 +183,16 @@ __global__ void __launch_bounds__(kBwdThreads) cb_intra_keys_kernel(const Tin* _
     for (int n = 0; n < kDV; ++n) A.dv[(size_t(bkv) * A.T + j) * kDV + n] = dvr[n];
 }
 
-// Exclusive suffix states R_c = sum over rows of later chunks and the group's query heads of
-// phi_h(q_i) g_i^T.  Block (64 packed rows, b*kv) walks the chunks backwards; thread =
-// (packed row, column group of 17 columns of [.; 1]).  Layout [bkv][c][n][f] like S_c.
+// Suffix states R_c = sum over rows of later chunks and the group's query heads of
+// phi_h(q_i) g_i^T, in two passes: cb_chunk_agg_kernel writes each chunk's own sum to R[c]
+// (block = 64 packed rows x chunk x (b, kv); thread = (packed row, column group of 17 columns
+// of [.; 1])), then chunk_scan_kernel (reverse) makes it the exclusive suffix in place.
+// Layout [bkv][c][n][f] like S_c.
 template <typename Tin>
-__global__ void __launch_bounds__(256) cb_suffix_kernel(const Tin* __restrict__ q, CbArgs A)
+__global__ void __launch_bounds__(256) cb_chunk_agg_kernel(const Tin* __restrict__ q, CbArgs A)
 {
-    const int slab = blockIdx.x, bkv = blockIdx.y, b = bkv / A.Hkv, kv = bkv % A.Hkv;
+    const int slab = blockIdx.x, bkv = blockIdx.z;
+    const int b = bkv / A.Hkv, kv = bkv % A.Hkv;
     const int grp = A.Hq / A.Hkv;
     const int tid = threadIdx.x, fi = tid & 63, cg = tid >> 6;
     const int f = slab * 64 + fi;
@@ -196,16 +200,8 @@ __global__ void __launch_bounds__(256) cb_suffix_kernel(const Tin* __restrict__ 
     __shared__ float qs[64][kDA + 1];
     __shared__ float gs[64][kW];
     const float* coef = cb_coef(A);
-    float run[17], acc[17];
-#pragma unroll
-    for (int u = 0; u < 17; ++u) run[u] = 0.f;
-    for (int c = A.NC - 1; c >= 0; --c) {
-        float* dst = A.R + (size_t(bkv) * A.NC + c) * kW * kFP;
-#pragma unroll
-        for (int u = 0; u < 17; ++u) {
-            const int n = cg + 4 * u;
-            if (n < kW) dst[size_t(n) * kFP + f] = run[u];
-        }
+    for (int c = blockIdx.y; c < A.NC; c += gridDim.y) {  // (gridDim.y < NC only past 65535)
+        float acc[17];
 #pragma unroll
         for (int u = 0; u < 17; ++u) acc[u] = 0.f;
         const int t0 = c * kCbC;
@@ -236,8 +232,12 @@ __global__ void __launch_bounds__(256) cb_suffix_kernel(const Tin* __restrict__ 
             }
             __syncthreads();
         }
+        float* dst = A.R + (size_t(bkv) * A.NC + c) * kW * kFP;
 #pragma unroll
-        for (int u = 0; u < 17; ++u) run[u] += acc[u];
+        for (int u = 0; u < 17; ++u) {
+            const int n = cg + 4 * u;
+            if (n < kW) dst[size_t(n) * kFP + f] = acc[u];
+        }
     }
 }
 
@@ -504,9 +504,8 @@ static int launch_backward_chunked_t(const Tin* q, const Tin* k, const Tin* v, C
         float* body = reinterpret_cast<float*>(A.st + kHeaderBytes + coef_bytes(Hq));
         {
             LaunchScope ls("backward_state", st);
-            state_simt_kernel<Tin><<<dim3(kFP / 64, B * Hkv), 256, 0, st>>>(k, v, T, kCbC, NC,
-                                                                             A.Hc, body);
-            OAL_LAUNCH_CHECK();
+            const int rc2 = launch_chunk_states_simt(k, v, T, kCbC, NC, A.Hc, body, B * Hkv, st);
+            if (rc2) return rc2;
         }
         {
             const size_t smem = sizeof(ReadoutSmem);
@@ -539,7 +538,11 @@ static int launch_backward_chunked_t(const Tin* q, const Tin* k, const Tin* v, C
         }
         {
             LaunchScope ls("backward_suffix", st);
-            cb_suffix_kernel<Tin><<<dim3(kFP / 64, B * Hkv), 256, 0, st>>>(q, A);
+            cb_chunk_agg_kernel<Tin><<<dim3(kFP / 64, std::min(NC, 65535), B * Hkv), 256, 0,
+                                       st>>>(q, A);
+            OAL_LAUNCH_CHECK();
+            chunk_scan_kernel<<<dim3((kW * kFP + 255) / 256, B * Hkv), 256, 0, st>>>(A.R, NC, 1,
+                                                                                   nullptr);
             OAL_LAUNCH_CHECK();
         }
         const size_t smem = sizeof(CbRowSmem);

@@ -230,9 +230,8 @@ static int launch_hadamard_t(const Tin* q, const Tin* k, const Tin* v, const flo
         const int NC = (T + Cn - 1) / Cn;
         {
             LaunchScope ls("state_simt", st);
-            state_simt_kernel<Tin><<<dim3(kFP / 64, B * Hkv), 256, 0, st>>>(k, v, T, Cn, NC, Hc,
-                                                                             body);
-            OAL_LAUNCH_CHECK();
+            const int rc = launch_chunk_states_simt(k, v, T, Cn, NC, Hc, body, B * Hkv, st);
+            if (rc) return rc;
         }
         if (T == 0) return OAL_OK;
         const float* coef = reinterpret_cast<const float*>(static_cast<unsigned char*>(state) +

@@ -608,6 +608,121 @@ int launch_prep(const int32_t* gid, const float* L, const int32_t* G, float eps,
     return OAL_OK;
 }
 
+// ------------------------------------------------------------------------------------------
+// The same chunk states, chunk-parallel: chunk_delta_simt_kernel writes each chunk's own sum
+// psi(k_j) [v_j; 1] over its tokens to Hc[bkv][c] (block = 64 packed rows x chunk x (b, kv),
+// the per-chunk arithmetic of state_simt_kernel), then chunk_scan_kernel turns Hc into the
+// exclusive prefix in place, adding the chunks in order, and writes the inclusive state: the
+// same sums in the same order as state_simt_kernel, so the same bits, with every chunk's
+// products computed at once instead of one chunk after another.
+// ------------------------------------------------------------------------------------------
+template <typename Tin>
+__global__ void __launch_bounds__(256) chunk_delta_simt_kernel(const Tin* __restrict__ k,
+                                                               const Tin* __restrict__ v, int T,
+                                                               int C, int NC,
+                                                               float* __restrict__ Hc)
+{
+    const int slab = blockIdx.x, bkv = blockIdx.z;
+    const int tid = threadIdx.x, fi = tid & 63, cg = tid >> 6;
+    const int f = slab * 64 + fi;
+    const RT rt = feature_rt(f);
+    __shared__ float ks[64][kDA + 1];
+    __shared__ float vs[64][kW];
+    const Tin* kb = k + size_t(bkv) * T * kD;
+    const Tin* vb = v + size_t(bkv) * T * kDV;
+    for (int c = blockIdx.y; c < NC; c += gridDim.y) {  // (gridDim.y < NC only past 65535)
+        float acc[17];
+#pragma unroll
+        for (int u = 0; u < 17; ++u) acc[u] = 0.f;
+        const int t0 = c * C, t1 = min(t0 + C, T);
+        for (int s0 = t0; s0 < t1; s0 += 64) {
+            for (int e = tid; e < 64 * kD; e += 256) {
+                const int j = e / kD, r = e % kD, tok = s0 + j;
+                ks[j][r] = tok < t1 ? to_f32(kb[size_t(tok) * kD + r]) : 0.f;
+                vs[j][r] = tok < t1 ? to_f32(vb[size_t(tok) * kDV + r]) : 0.f;
+            }
+            if (tid < 64) {
+                const bool ok = s0 + tid < t1;
+                ks[tid][kD] = ok ? 1.f : 0.f;
+                ks[tid][kD + 1] = 0.f;
+                vs[tid][kDV] = ok ? 1.f : 0.f;
+            }
+            __syncthreads();
+            for (int j = 0; j < 64; ++j) {
+                const float psi = ks[j][rt.r] * ks[j][rt.t];
+#pragma unroll
+                for (int u = 0; u < 17; ++u) {
+                    const int n = cg + 4 * u;
+                    if (n < kW) acc[u] = fmaf(psi, vs[j][n], acc[u]);
+                }
+            }
+            __syncthreads();
+        }
+        float* dst = Hc + (size_t(bkv) * NC + c) * kW * kFP;
+#pragma unroll
+        for (int u = 0; u < 17; ++u) {
+            const int n = cg + 4 * u;
+            if (n < kW) dst[size_t(n) * kFP + f] = acc[u];
+        }
+    }
+}
+
+// In place over X[bkv][c][n][f] (fp32, [65][2176] per chunk): the exclusive prefix over chunks
+// (reverse = 0: X_c <- sum_{c' < c} X_c') or suffix (reverse = 1: X_c <- sum_{c' > c} X_c'),
+// the chunks added one at a time in that order.  With `body`, the sum over all chunks goes to
+// the state of (b, kv) (rows [f][64], then z[f]).  Thread = one (n, f) entry of one (b, kv).
+__global__ void __launch_bounds__(256) chunk_scan_kernel(float* __restrict__ X, int NC,
+                                                         int reverse, float* __restrict__ body)
+{
+    constexpr int kPer = kW * kFP;
+    const int e = blockIdx.x * blockDim.x + threadIdx.x, bkv = blockIdx.y;
+    if (e >= kPer) return;
+    float* x = X + size_t(bkv) * NC * kPer + e;
+    constexpr int kAhead = 8;  // chunks requested ahead of the running sum
+    float run = 0.f;
+    for (int i0 = 0; i0 < NC; i0 += kAhead) {
+        float d[kAhead];
+#pragma unroll
+        for (int u = 0; u < kAhead; ++u) {
+            const int i = i0 + u, c = reverse ? NC - 1 - i : i;
+            d[u] = i < NC ? x[size_t(c) * kPer] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kAhead; ++u) {
+            const int i = i0 + u, c = reverse ? NC - 1 - i : i;
+            if (i < NC) {
+                x[size_t(c) * kPer] = run;
+                run += d[u];
+            }
+        }
+    }
+    if (body) {
+        const int n = e / kFP, f = e - n * kFP;
+        float* unit = body + size_t(bkv) * kFP * kW;
+        if (n < kDV) unit[size_t(f) * kDV + n] = run;
+        else unit[size_t(kFP) * kDV + f] = run;
+    }
+}
+
+// The chunk states of the fp32 path: chunk-parallel when there is an Hc to hold the chunk
+// sums, else the walking kernel (the final state alone).
+template <typename Tin>
+int launch_chunk_states_simt(const Tin* k, const Tin* v, int T, int C, int NC, float* Hc,
+                             float* body, int nbkv, cudaStream_t st)
+{
+    if (Hc == nullptr || NC <= 1 || nbkv > 65535) {
+        state_simt_kernel<Tin><<<dim3(kFP / 64, nbkv), 256, 0, st>>>(k, v, T, C, NC, Hc, body);
+        OAL_LAUNCH_CHECK();
+        return OAL_OK;
+    }
+    chunk_delta_simt_kernel<Tin><<<dim3(kFP / 64, std::min(NC, 65535), nbkv), 256, 0, st>>>(
+        k, v, T, C, NC, Hc);
+    OAL_LAUNCH_CHECK();
+    chunk_scan_kernel<<<dim3((kW * kFP + 255) / 256, nbkv), 256, 0, st>>>(Hc, NC, 0, body);
+    OAL_LAUNCH_CHECK();
+    return OAL_OK;
+}
+
 template <typename Tin>
 static int launch_prefill_simt_t(const Tin* q, const Tin* k, const Tin* v,
                                  const int32_t* gid, const float* L, const int32_t* G,
@@ -620,9 +735,8 @@ static int launch_prefill_simt_t(const Tin* q, const Tin* k, const Tin* v,
                                            coef_bytes(Hq));
     {
         LaunchScope ls("state_simt", st);
-        state_simt_kernel<Tin><<<dim3(kFP / 64, B * Hkv), 256, 0, st>>>(k, v, T, C, NC, Hc,
-                                                                         body);
-        OAL_LAUNCH_CHECK();
+        const int rc = launch_chunk_states_simt(k, v, T, C, NC, Hc, body, B * Hkv, st);
+        if (rc) return rc;
     }
     if (T == 0 || out == nullptr) return OAL_OK;  // no out: the state alone is wanted
     const size_t smem = sizeof(ReadoutSmem);
