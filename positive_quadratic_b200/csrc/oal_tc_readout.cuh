@@ -87,13 +87,17 @@ constexpr bool rows_need_chunk(int ch)
     return false;
 }
 
-// phi of the diagonal / linear / constant slices (64 rows with compile-time (r, t)); fp32
-// products, one rounding.  coef_t holds the coefficients of rows 1792.. .  The q values are
-// loaded per group of 8 rows, so that only the chunks a group reads are live at a time.
+// phi of the diagonal / linear / constant slices (64 rows with compile-time (r, t)), in
+// packed bf16 like the off-diagonal slices: phi = bf16(bf16(q_r q_t) * bf16(c)).  coef_t holds
+// the (fp32) coefficients of rows 1792.. .  The q values are loaded per group of 8 rows, so
+// that only the chunks a group reads are live at a time; each pair of rows takes its two q_r
+// and its two q_t into one bf16x2 register each with one byte permute (q_64 = 1 and q_65 = 0
+// come from a constant word).
 template <int F0>
 __device__ __forceinline__ void phi_tail_static(const unsigned char* qt, const float* coef_t,
                                                 int row, uint32_t (&w)[32])
 {
+    constexpr uint32_t kOneZero = 0x00003F80u;  // bf16 halves (1, 0)
     static_for<8>([&](auto X) {
         constexpr int x = decltype(X)::value;
         constexpr int F = F0 + 8 * x;
@@ -108,26 +112,30 @@ __device__ __forceinline__ void phi_tail_static(const unsigned char* qt, const f
                 qp[4 * ch + 3] = v.w;
             }
         });
-        // q_r as fp32 (r = 64: the constant 1)
-        auto qv = [&](auto R) -> float {
+        // the 32-bit word holding q_r, and the half of it (r = 64, 65: the constant word)
+        auto word = [&](auto R) -> uint32_t {
             constexpr int r = decltype(R)::value;
-            if constexpr (r >= 64) return r == 64 ? 1.f : 0.f;
-            else if constexpr (r & 1) return bf16hi_to_f32(qp[r >> 1]);
-            else return bf16lo_to_f32(qp[r >> 1]);
+            if constexpr (r >= 64) return kOneZero;
+            else return qp[r >> 1];
         };
+        auto half = [](int r) constexpr -> int { return r >= 64 ? r - 64 : (r & 1); };
         const float* cp = coef_t + (F - kOffDiagRows);
         const float4 c0 = *reinterpret_cast<const float4*>(cp);
         const float4 c1 = *reinterpret_cast<const float4*>(cp + 4);
-        const float cf[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        const uint32_t cw[4] = {pack_bf16x2(c0.x, c0.y), pack_bf16x2(c0.z, c0.w),
+                                pack_bf16x2(c1.x, c1.y), pack_bf16x2(c1.z, c1.w)};
         static_for<4>([&](auto E) {
             constexpr int e = decltype(E)::value;
             constexpr RT a = feature_rt(F + 2 * e);
             constexpr RT b = feature_rt(F + 2 * e + 1);
-            const float pa = qv(std::integral_constant<int, a.r>{}) *
-                             qv(std::integral_constant<int, a.t>{});
-            const float pb = qv(std::integral_constant<int, b.r>{}) *
-                             qv(std::integral_constant<int, b.t>{});
-            w[4 * x + e] = pack_bf16x2(cf[2 * e] * pa, cf[2 * e + 1] * pb);
+            // low half from the first word, high half from the second (bytes 4..7)
+            constexpr uint32_t sr = (half(a.r) ? 0x32u : 0x10u) | ((half(b.r) ? 0x76u : 0x54u) << 8);
+            constexpr uint32_t st = (half(a.t) ? 0x32u : 0x10u) | ((half(b.t) ? 0x76u : 0x54u) << 8);
+            const uint32_t xr = __byte_perm(word(std::integral_constant<int, a.r>{}),
+                                            word(std::integral_constant<int, b.r>{}), sr);
+            const uint32_t xt = __byte_perm(word(std::integral_constant<int, a.t>{}),
+                                            word(std::integral_constant<int, b.t>{}), st);
+            w[4 * x + e] = bmul2(bmul2(xr, xt), cw[e]);
         });
     });
 }
