@@ -134,16 +134,16 @@ __global__ void __launch_bounds__(kBwdThreads) cb_intra_rows_kernel(const Tin* _
     A.rowE[row] = de;
 }
 
-// Within-chunk pairs, keys: thread = key j, rows i in [j, end of j's chunk) of every query
-// head of the group.  Writes dk and dv (the inter pass adds to them).
+// Within-chunk pairs, keys: thread = (key j, query head x of the group), rows i in [j, end of
+// j's chunk); the eight lanes of a key (x = lane & 7, heads past the group's contribute zero)
+// add their dk and dv with a fixed butterfly.  Writes dk and dv (the inter pass adds to them).
+constexpr int kKeysPerBlock = 16;
 template <typename Tin>
-__global__ void __launch_bounds__(kBwdThreads) cb_intra_keys_kernel(const Tin* __restrict__ q,
-                                                                    const Tin* __restrict__ k,
-                                                                    const Tin* __restrict__ v,
-                                                                    CbArgs A)
+__global__ void __launch_bounds__(8 * kKeysPerBlock) cb_intra_keys_kernel(
+    const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v, CbArgs A)
 {
     const int bkv = blockIdx.y, b = bkv / A.Hkv, kv = bkv % A.Hkv, grp = A.Hq / A.Hkv;
-    const int j = blockIdx.x * kBwdThreads + threadIdx.x;
+    const int x = threadIdx.x & 7, j = blockIdx.x * kKeysPerBlock + (threadIdx.x >> 3);
     __shared__ float m[kMaxGroup][kMM];
     __shared__ int g[kMaxGroup][kD];
     __shared__ int sG[kMaxGroup];
@@ -156,14 +156,13 @@ __global__ void __launch_bounds__(kBwdThreads) cb_intra_keys_kernel(const Tin* _
                                          g[threadIdx.x]);
     }
     __syncthreads();
-    if (j >= A.T) return;
-    const Tin* kj = k + (size_t(bkv) * A.T + j) * kD;
-    const Tin* vj = v + (size_t(bkv) * A.T + j) * kDV;
-    const int iend = min(A.T, (j / kCbC + 1) * kCbC);
     float dkr[kD], dvr[kDV], sb[kGM1], ms[kGM1];
     for (int r = 0; r < kD; ++r) dkr[r] = 0.f;
     for (int n = 0; n < kDV; ++n) dvr[n] = 0.f;
-    for (int x = 0; x < grp; ++x) {
+    if (j < A.T && x < grp) {
+        const Tin* kj = k + (size_t(bkv) * A.T + j) * kD;
+        const Tin* vj = v + (size_t(bkv) * A.T + j) * kDV;
+        const int iend = min(A.T, (j / kCbC + 1) * kCbC);
         const int h = kv * grp + x, bh = b * A.Hq + h;
         for (int i = j; i < iend; ++i) {
             const size_t row = size_t(bh) * A.T + i;
@@ -179,8 +178,18 @@ __global__ void __launch_bounds__(kBwdThreads) cb_intra_keys_kernel(const Tin* _
                 dkr[r] = fmaf(dk_ * 2.f * ms[g[x][r]] * 0.125f, to_f32(qi[r]), dkr[r]);
         }
     }
-    for (int r = 0; r < kD; ++r) A.dk[(size_t(bkv) * A.T + j) * kD + r] = dkr[r];
-    for (int n = 0; n < kDV; ++n) A.dv[(size_t(bkv) * A.T + j) * kDV + n] = dvr[n];
+    // sum over the group's heads: lanes x, x ^ 4, x ^ 2, x ^ 1 of the key, a fixed order
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) {
+#pragma unroll
+        for (int r = 0; r < kD; ++r) dkr[r] += __shfl_xor_sync(0xffffffffu, dkr[r], o);
+#pragma unroll
+        for (int n = 0; n < kDV; ++n) dvr[n] += __shfl_xor_sync(0xffffffffu, dvr[n], o);
+    }
+    if (j < A.T && x == 0) {
+        for (int r = 0; r < kD; ++r) A.dk[(size_t(bkv) * A.T + j) * kD + r] = dkr[r];
+        for (int n = 0; n < kDV; ++n) A.dv[(size_t(bkv) * A.T + j) * kDV + n] = dvr[n];
+    }
 }
 
 // Suffix states R_c = sum over rows of later chunks and the group's query heads of
@@ -393,6 +402,37 @@ __global__ void __launch_bounds__(256) cb_inter_keys_kernel(const Tin* __restric
     }
 }
 
+// Per (b*h, chunk): the chunk's rows' dM and deps partials, summed in row order into the
+// chunk's first row (each thread owns one of the 81 dM entries, thread 81 deps).
+__global__ void __launch_bounds__(96) cb_rowsum_kernel(CbArgs A)
+{
+    const int c = blockIdx.x, bh = blockIdx.y, e = threadIdx.x;
+    const size_t r0 = size_t(bh) * A.T + size_t(c) * kCbC;
+    const int n = min(kCbC, A.T - c * kCbC);
+    if (e < kMM) {
+        float s = 0.f;
+        for (int i = 0; i < n; ++i) s += A.rowM[(r0 + i) * kMM + e];
+        A.rowM[r0 * kMM + e] = s;
+    } else if (e == kMM) {
+        float s = 0.f;
+        for (int i = 0; i < n; ++i) s += A.rowE[r0 + i];
+        A.rowE[r0] = s;
+    }
+}
+
+// Per (head, packed row f): the partial dC'_f of every (b, chunk), summed in that order into
+// the (b = 0, chunk 0) slot.
+__global__ void __launch_bounds__(256) cb_dcsum_kernel(CbArgs A)
+{
+    const int f = blockIdx.x * blockDim.x + threadIdx.x, h = blockIdx.y;
+    if (f >= kF) return;
+    float acc = 0.f;
+    for (int b = 0; b < A.B; ++b)
+        for (int c = 0; c < A.NC; ++c)
+            acc += A.dcp[((size_t(b) * A.Hq + h) * A.NC + c) * kFP + f];
+    A.dcp[size_t(h) * A.NC * kFP + f] = acc;
+}
+
 // dM_h = the rows' within-chunk partials plus dC'_h mapped through C'_f = (2 - [r = t])
 // M_{g(r)g(t)} s_r s_t (each ordered pair (r, t) carries half of an off-diagonal row), summed in
 // a fixed order; dL_h = (dM + dM^T) L; deps_h = within-chunk partials + dC' of the constant row.
@@ -415,18 +455,14 @@ __global__ void __launch_bounds__(kMM) cb_heads_kernel(CbArgs A)
     } else if (e < kDA) {
         g[e] = 0;  // the constant slot belongs to sbar_0
     }
-    // dC'_h: the partials of every (b, chunk), summed in order
-    for (int f = e; f < kF; f += kMM) {
-        float acc = 0.f;
-        for (int b = 0; b < A.B; ++b)
-            for (int c = 0; c < A.NC; ++c)
-                acc += A.dcp[((size_t(b) * A.Hq + h) * A.NC + c) * kFP + f];
-        dC[f] = acc;
-    }
+    // dC'_h: cb_dcsum_kernel left the sum over every (b, chunk) in the (b = 0, chunk 0) slot
+    const bool any = A.B > 0 && A.NC > 0;
+    for (int f = e; f < kF; f += kMM) dC[f] = any ? A.dcp[size_t(h) * A.NC * kFP + f] : 0.f;
+    // the rows' partials: cb_rowsum_kernel left each chunk's sum in the chunk's first row
     float s = 0.f, de = 0.f;
     for (int b = 0; b < A.B; ++b)
-        for (int i = 0; i < A.T; ++i) {
-            const size_t row = (size_t(b) * A.Hq + h) * A.T + i;
+        for (int c = 0; c < A.NC; ++c) {
+            const size_t row = (size_t(b) * A.Hq + h) * A.T + size_t(c) * kCbC;
             s += A.rowM[row * kMM + e];
             if (e == 0) de += A.rowE[row];
         }
@@ -532,8 +568,8 @@ static int launch_backward_chunked_t(const Tin* q, const Tin* k, const Tin* v, C
         }
         {
             LaunchScope ls("backward_intra_keys", st);
-            cb_intra_keys_kernel<Tin><<<dim3((T + kBwdThreads - 1) / kBwdThreads, B * Hkv),
-                                        kBwdThreads, 0, st>>>(q, k, v, A);
+            cb_intra_keys_kernel<Tin><<<dim3((T + kKeysPerBlock - 1) / kKeysPerBlock, B * Hkv),
+                                        8 * kKeysPerBlock, 0, st>>>(q, k, v, A);
             OAL_LAUNCH_CHECK();
         }
         {
@@ -565,6 +601,12 @@ static int launch_backward_chunked_t(const Tin* q, const Tin* k, const Tin* v, C
     }
     {
         LaunchScope ls("backward_heads", st);
+        if (B > 0 && T > 0) {
+            cb_rowsum_kernel<<<dim3(NC, B * Hq), 96, 0, st>>>(A);
+            OAL_LAUNCH_CHECK();
+            cb_dcsum_kernel<<<dim3((kF + 255) / 256, Hq), 256, 0, st>>>(A);
+            OAL_LAUNCH_CHECK();
+        }
         cb_heads_kernel<<<Hq, kMM, 0, st>>>(A);
         OAL_LAUNCH_CHECK();
     }
