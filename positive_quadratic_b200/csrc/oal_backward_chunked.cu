@@ -308,7 +308,7 @@ __global__ void __launch_bounds__(256) cb_inter_rows_kernel(const Tin* __restric
         // dq: thread (row ri, cg) owns the dims d = cg (mod 4)
         for (int fl = 0; fl < 64; ++fl) {
             const int f = slab * 64 + fl;
-            const RT rt = feature_rt(f);
+            const RT rt = feature_rt_tab(f);
             const float w = sm.ps[ri][fl] * cf[f];
             if (rt.r < kD && (rt.r & 3) == cg)
                 sm.ds[ri][rt.r] += rt.r == rt.t ? 2.f * w * sm.qs[ri][rt.r] : w * sm.qs[ri][rt.t];
@@ -316,7 +316,7 @@ __global__ void __launch_bounds__(256) cb_inter_rows_kernel(const Tin* __restric
         }
         // partial dC' of the slab's rows: thread (f, row group)
         {
-            const RT rt = feature_rt(slab * 64 + ri);
+            const RT rt = feature_rt_tab(slab * 64 + ri);
             float part = 0.f;
             for (int j = cg; j < 64; j += 4)
                 part = fmaf(sm.ps[j][ri], sm.qs[j][rt.r] * sm.qs[j][rt.t], part);
@@ -374,7 +374,7 @@ __global__ void __launch_bounds__(256) cb_inter_keys_kernel(const Tin* __restric
             sm.ps[rj][fl] = d;
         }
         for (int fl = 0; fl < 64; ++fl) {
-            const RT rt = feature_rt(slab * 64 + fl);
+            const RT rt = feature_rt_tab(slab * 64 + fl);
             const float psi = sm.qs[rj][rt.r] * sm.qs[rj][rt.t];
 #pragma unroll
             for (int u = 0; u < 17; ++u) {
@@ -384,7 +384,7 @@ __global__ void __launch_bounds__(256) cb_inter_keys_kernel(const Tin* __restric
         }
         __syncthreads();
         for (int fl = 0; fl < 64; ++fl) {
-            const RT rt = feature_rt(slab * 64 + fl);
+            const RT rt = feature_rt_tab(slab * 64 + fl);
             const float w = sm.ps[rj][fl];
             if (rt.r < kD && (rt.r & 3) == cg)
                 sm.ds[rj][rt.r] += rt.r == rt.t ? 2.f * w * sm.qs[rj][rt.r] : w * sm.qs[rj][rt.t];
@@ -471,7 +471,7 @@ __global__ void __launch_bounds__(kMM) cb_heads_kernel(CbArgs A)
     float sc = 0.f;  // dC' reaching M_{a mm}
     if (a <= Gh && mm <= Gh) {
         for (int f = 0; f < kF; ++f) {
-            const RT rt = feature_rt(f);
+            const RT rt = feature_rt_tab(f);
             const int ga = g[rt.r], gb = g[rt.t];
             float wgt = (ga == a && gb == mm) ? 1.f : 0.f;
             if (rt.r != rt.t && gb == a && ga == mm) wgt += 1.f;

@@ -13,6 +13,28 @@
 
 namespace oal {
 
+// (r, t) of every packed row as r | t << 8: a table for the loops that visit many rows, which
+// would otherwise walk the block structure of feature_rt once per row.
+struct RtTable {
+    uint16_t v[kF];
+};
+constexpr RtTable make_rt_table()
+{
+    RtTable tab{};
+    for (int f = 0; f < kF; ++f) {
+        const RT rt = feature_rt(f);
+        tab.v[f] = uint16_t(rt.r | (rt.t << 8));
+    }
+    return tab;
+}
+__device__ const RtTable c_rt_tab = make_rt_table();
+__device__ __forceinline__ RT feature_rt_tab(int f)
+{
+    if (f >= kF) return RT{kD + 1, kD + 1};
+    const uint32_t x = c_rt_tab.v[f];
+    return RT{int(x & 255u), int(x >> 8)};
+}
+
 // ------------------------------------------------------------------------------------------
 // a1: coefficient expansion.  M = L L^T (fp64), then the packed readout coefficients
 // Cp_f (oal_common.cuh) per query head, written into the state buffer's coefficient table;
@@ -293,7 +315,7 @@ __global__ void __launch_bounds__(256) readout_simt_kernel(
         for (int slab = 0; slab < kFP / 64; ++slab) {
             const int f = slab * 64 + ri;
             for (int n = cg; n < kW; n += 4) sm.u.hs[n][ri] = Hs[size_t(n) * kFP + f];
-            const RT rt = feature_rt(f);
+            const RT rt = feature_rt_tab(f);
             const float cfv = cf[f];
             for (int row = cg; row < 64; row += 4)
                 sm.ps[row][ri] = cfv * sm.qs[row][rt.r] * sm.qs[row][rt.t];
