@@ -81,7 +81,7 @@ struct HadamardSmem {
     float qs[64][kDA + 1];
     float ps[64][65];
     union {
-        float hs[kW][64];
+        InterTiles t;
         struct {
             float ks[64][kD + 1];
             float vs[64][kW];
@@ -133,26 +133,14 @@ __global__ void __launch_bounds__(256) readout_hadamard_kernel(
 
     const int c = i0 / Cn;
     if (!kDense && c > 0) {
-        const float* Hs = Hc + (size_t(bkv) * NC + c) * kW * kFP;
-        const float* cf = coef + size_t(h) * kFP;
-        for (int slab = 0; slab < kFP / 64; ++slab) {
-            const int f = slab * 64 + ri;
-            for (int n = cg; n < kW; n += 4) sm.u.hs[n][ri] = Hs[size_t(n) * kFP + f];
-            const RT rt = feature_rt(f);
-            const float cfv = cf[f];
-            for (int row = cg; row < 64; row += 4)
-                sm.ps[row][ri] = cfv * sm.qs[row][rt.r] * sm.qs[row][rt.t];
-            __syncthreads();
-            for (int ff = 0; ff < 64; ++ff) {
-                const float p = sm.ps[ri][ff];
+        inter_tile_simt(sm, Hc + (size_t(bkv) * NC + c) * kW * kFP, coef + size_t(h) * kFP,
+                        sm.ps);
 #pragma unroll
-                for (int u = 0; u < 17; ++u) {
-                    const int n = cg + 4 * u;
-                    if (n < kW) acc[u] = fmaf(p, sm.u.hs[n][ff], acc[u]);
-                }
-            }
-            __syncthreads();
+        for (int u = 0; u < 17; ++u) {
+            const int n = cg + 4 * u;
+            if (n < kW) acc[u] = sm.ps[ri][n];
         }
+        __syncthreads();  // ps is the intra-chunk weights' buffer from here on
     }
 
     const int j0 = kDense ? 0 : c * Cn;

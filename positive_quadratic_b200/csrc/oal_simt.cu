@@ -223,11 +223,19 @@ __global__ void __launch_bounds__(256) state_simt_kernel(const Tin* __restrict__
 // (2)-(3) (j0 = start of the chunk for prefill, 0 for the dense form); then
 // yhat_i = u_i[0:64] / u_i[64] (and, when den_out is given, D_i = u_i[64]).
 // ------------------------------------------------------------------------------------------
+// The inter-chunk tile's operands, transposed: phi of the 64 rows and a 64-row slab of S_c,
+// each [f][row or n] with rows 16-byte aligned (68 floats), so that a thread reads four
+// consecutive rows or columns as one vector.
+struct InterTiles {
+    float psT[64][68];
+    float hsT[64][68];
+};
+
 struct ReadoutSmem {
     float qs[64][kDA + 1];
     float ps[64][65];
     union {
-        float hs[kW][64];
+        InterTiles t;
         struct {
             float ks[64][kD + 1];
             float vs[64][kW];
@@ -238,6 +246,59 @@ struct ReadoutSmem {
     int gstart[kGM1 + 1];
     int G;
 };
+
+// Inter-chunk part of a 64-row readout tile: res[row][n] = sum_f phi_f(q_row) S_c[n][f] with
+// phi_f = cf_f qhat_r qhat_t (eq. (5)), the sum running over the 64-row slabs of S_c and the
+// rows f of each slab in order.  256 threads; in the products, thread t owns rows
+// 4 (t & 15) .. + 3 and columns 4 (t >> 4) .. + 3 (and column 64 for t < 16), reading four
+// phi values and four S values per f as two vectors.  Ends with res complete and synchronised.
+template <class Smem>
+__device__ __forceinline__ void inter_tile_simt(Smem& sm, const float* __restrict__ Hs,
+                                                const float* __restrict__ cf,
+                                                float (*res)[65])
+{
+    const int tid = threadIdx.x, ri = tid & 63, cg = tid >> 6;
+    const int rg = tid & 15, cq = tid >> 4;
+    float t4[4][4], tn[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        tn[i] = 0.f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) t4[i][j] = 0.f;
+    }
+    for (int slab = 0; slab < kFP / 64; ++slab) {
+        const int f = slab * 64 + ri;
+        for (int n = cg; n < kW; n += 4) sm.u.t.hsT[ri][n] = Hs[size_t(n) * kFP + f];
+        const RT rt = feature_rt_tab(f);
+        const float cfv = cf[f];
+        for (int row = cg; row < 64; row += 4)
+            sm.u.t.psT[ri][row] = cfv * sm.qs[row][rt.r] * sm.qs[row][rt.t];
+        __syncthreads();
+#pragma unroll 4
+        for (int ff = 0; ff < 64; ++ff) {
+            const float4 a = *reinterpret_cast<const float4*>(&sm.u.t.psT[ff][4 * rg]);
+            const float4 b = *reinterpret_cast<const float4*>(&sm.u.t.hsT[ff][4 * cq]);
+            const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) t4[i][j] = fmaf(av[i], bv[j], t4[i][j]);
+            if (cq == 0) {
+                const float bn = sm.u.t.hsT[ff][kDV];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) tn[i] = fmaf(av[i], bn, tn[i]);
+            }
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) res[4 * rg + i][4 * cq + j] = t4[i][j];
+        if (cq == 0) res[4 * rg + i][kDV] = tn[i];
+    }
+    __syncthreads();
+}
 
 template <typename Tin, bool kDense>
 __global__ void __launch_bounds__(256) readout_simt_kernel(
@@ -310,26 +371,14 @@ __global__ void __launch_bounds__(256) readout_simt_kernel(
 
     const int c = i0 / C;
     if (!kDense && c > 0) {
-        const float* Hs = Hc + (size_t(bkv) * NC + c) * kW * kFP;
-        const float* cf = coef + size_t(h) * kFP;
-        for (int slab = 0; slab < kFP / 64; ++slab) {
-            const int f = slab * 64 + ri;
-            for (int n = cg; n < kW; n += 4) sm.u.hs[n][ri] = Hs[size_t(n) * kFP + f];
-            const RT rt = feature_rt_tab(f);
-            const float cfv = cf[f];
-            for (int row = cg; row < 64; row += 4)
-                sm.ps[row][ri] = cfv * sm.qs[row][rt.r] * sm.qs[row][rt.t];
-            __syncthreads();
-            for (int ff = 0; ff < 64; ++ff) {
-                const float p = sm.ps[ri][ff];
+        inter_tile_simt(sm, Hc + (size_t(bkv) * NC + c) * kW * kFP, coef + size_t(h) * kFP,
+                        sm.ps);
 #pragma unroll
-                for (int u = 0; u < 17; ++u) {
-                    const int n = cg + 4 * u;
-                    if (n < kW) acc[u] = fmaf(p, sm.u.hs[n][ff], acc[u]);
-                }
-            }
-            __syncthreads();
+        for (int u = 0; u < 17; ++u) {
+            const int n = cg + 4 * u;
+            if (n < kW) acc[u] = sm.ps[ri][n];
         }
+        __syncthreads();  // ps is the intra-chunk weights' buffer from here on
     }
 
     const int j0 = kDense ? 0 : c * C;
