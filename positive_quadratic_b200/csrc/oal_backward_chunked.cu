@@ -253,6 +253,7 @@ __global__ void __launch_bounds__(256) cb_chunk_agg_kernel(const Tin* __restrict
 struct CbRowSmem {
     float qs[64][kDA + 1];   // qhat rows (the tile's query rows, or the chunk's key rows)
     float gs[64][kW];        // g rows, or [v; 1] rows
+    float gT[kW][68];        // gs transposed, rows 16-byte aligned
     float hs[kW][64];        // a 64-row slab of S_c or R_c, [n][f]
     float ps[64][65];        // dphi or dpsi of the slab, [row][f]
     float ds[64][kD + 1];    // dq or dk of the tile's rows
@@ -289,20 +290,42 @@ __global__ void __launch_bounds__(256) cb_inter_rows_kernel(const Tin* __restric
         sm.qs[tid][kD] = 1.f;
         sm.qs[tid][kD + 1] = 0.f;
     }
+    for (int e = tid; e < 64 * kW; e += 256) {
+        const int j = e / kW, n = e % kW;
+        sm.gT[n][j] = i0 + j < A.T ? A.Gr[(r0 + j) * kW + n] : 0.f;
+    }
     __syncthreads();
     const float* Hs = A.Hc + (size_t(bkv) * A.NC + c) * kW * kFP;
     const float* cf = cb_coef(A) + size_t(h) * kFP;
+    // dphi tile: thread owns rows 4 (tid & 15) .. + 3 and packed rows 4 (tid >> 4) .. + 3 of
+    // the slab, the sum over n in order
+    const int rg = tid & 15, fq = tid >> 4;
     for (int slab = 0; slab < kFP / 64; ++slab) {
         for (int e = tid; e < kW * 64; e += 256) {
             const int n = e / 64, fl = e % 64;
             sm.hs[n][fl] = Hs[size_t(n) * kFP + slab * 64 + fl];
         }
         __syncthreads();
-        for (int u = 0; u < 16; ++u) {
-            const int fl = cg + 4 * u;
-            float d = 0.f;
-            for (int n = 0; n < kW; ++n) d = fmaf(sm.hs[n][fl], sm.gs[ri][n], d);
-            sm.ps[ri][fl] = d;
+        {
+            float t4[4][4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) t4[i][jj] = 0.f;
+#pragma unroll 5
+            for (int n = 0; n < kW; ++n) {
+                const float4 hv = *reinterpret_cast<const float4*>(&sm.hs[n][4 * fq]);
+                const float4 gv = *reinterpret_cast<const float4*>(&sm.gT[n][4 * rg]);
+                const float hf[4] = {hv.x, hv.y, hv.z, hv.w}, gr[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) t4[i][jj] = fmaf(hf[jj], gr[i], t4[i][jj]);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) sm.ps[4 * rg + i][4 * fq + jj] = t4[i][jj];
         }
         __syncthreads();
         // dq: thread (row ri, cg) owns the dims d = cg (mod 4)
