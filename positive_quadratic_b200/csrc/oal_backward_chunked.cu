@@ -197,22 +197,32 @@ __global__ void __launch_bounds__(8 * kKeysPerBlock) cb_intra_keys_kernel(
 // (block = 64 packed rows x chunk x (b, kv); thread = (packed row, column group of 17 columns
 // of [.; 1])), then chunk_scan_kernel (reverse) makes it the exclusive suffix in place.
 // Layout [bkv][c][n][f] like S_c.
+struct CbAggSmem {
+    float qs[64][kDA + 1];  // qhat rows of the chunk for one query head (and 1, 0)
+    float A[64][68];        // phi of the rows, [row][packed row of the slab]
+    float B[64][68];        // g rows
+};
+
 template <typename Tin>
 __global__ void __launch_bounds__(256) cb_chunk_agg_kernel(const Tin* __restrict__ q, CbArgs A)
 {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    CbAggSmem& sm = *reinterpret_cast<CbAggSmem*>(smem_raw);
     const int slab = blockIdx.x, bkv = blockIdx.z;
     const int b = bkv / A.Hkv, kv = bkv % A.Hkv;
     const int grp = A.Hq / A.Hkv;
     const int tid = threadIdx.x, fi = tid & 63, cg = tid >> 6;
     const int f = slab * 64 + fi;
     const RT rt = feature_rt(f);
-    __shared__ float qs[64][kDA + 1];
-    __shared__ float gs[64][kW];
     const float* coef = cb_coef(A);
     for (int c = blockIdx.y; c < A.NC; c += gridDim.y) {  // (gridDim.y < NC only past 65535)
-        float acc[17];
+        float t4[4][4], tn[4];
 #pragma unroll
-        for (int u = 0; u < 17; ++u) acc[u] = 0.f;
+        for (int i = 0; i < 4; ++i) {
+            tn[i] = 0.f;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) t4[i][jj] = 0.f;
+        }
         const int t0 = c * kCbC;
         for (int x = 0; x < grp; ++x) {
             const int h = kv * grp + x;
@@ -220,33 +230,23 @@ __global__ void __launch_bounds__(256) cb_chunk_agg_kernel(const Tin* __restrict
             const float cf = coef[size_t(h) * kFP + f];
             for (int e = tid; e < 64 * kD; e += 256) {
                 const int j = e / kD, r = e % kD;
-                qs[j][r] = t0 + j < A.T ? to_f32(q[(r0 + j) * kD + r]) : 0.f;
+                sm.qs[j][r] = t0 + j < A.T ? to_f32(q[(r0 + j) * kD + r]) : 0.f;
             }
             for (int e = tid; e < 64 * kW; e += 256) {
                 const int j = e / kW, n = e % kW;
-                gs[j][n] = t0 + j < A.T ? A.Gr[(r0 + j) * kW + n] : 0.f;
+                sm.B[j][n] = t0 + j < A.T ? A.Gr[(r0 + j) * kW + n] : 0.f;
             }
             if (tid < 64) {
-                qs[tid][kD] = 1.f;
-                qs[tid][kD + 1] = 0.f;
+                sm.qs[tid][kD] = 1.f;
+                sm.qs[tid][kD + 1] = 0.f;
             }
             __syncthreads();
-            for (int j = 0; j < 64; ++j) {
-                const float phi = cf * qs[j][rt.r] * qs[j][rt.t];
-#pragma unroll
-                for (int u = 0; u < 17; ++u) {
-                    const int n = cg + 4 * u;
-                    if (n < kW) acc[u] = fmaf(phi, gs[j][n], acc[u]);
-                }
-            }
+            for (int j = cg; j < 64; j += 4) sm.A[j][fi] = cf * sm.qs[j][rt.r] * sm.qs[j][rt.t];
+            __syncthreads();
+            tile_acc_simt(sm.A, sm.B, t4, tn);
             __syncthreads();
         }
-        float* dst = A.R + (size_t(bkv) * A.NC + c) * kW * kFP;
-#pragma unroll
-        for (int u = 0; u < 17; ++u) {
-            const int n = cg + 4 * u;
-            if (n < kW) dst[size_t(n) * kFP + f] = acc[u];
-        }
+        tile_store_simt(A.R + (size_t(bkv) * A.NC + c) * kW * kFP, slab * 64, t4, tn);
     }
 }
 
@@ -597,8 +597,11 @@ static int launch_backward_chunked_t(const Tin* q, const Tin* k, const Tin* v, C
         }
         {
             LaunchScope ls("backward_suffix", st);
-            cb_chunk_agg_kernel<Tin><<<dim3(kFP / 64, std::min(NC, 65535), B * Hkv), 256, 0,
-                                       st>>>(q, A);
+            OAL_CUDA_TRY(cudaFuncSetAttribute(cb_chunk_agg_kernel<Tin>,
+                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              int(sizeof(CbAggSmem))));
+            cb_chunk_agg_kernel<Tin><<<dim3(kFP / 64, std::min(NC, 65535), B * Hkv), 256,
+                                       sizeof(CbAggSmem), st>>>(q, A);
             OAL_LAUNCH_CHECK();
             chunk_scan_kernel<<<dim3((kW * kFP + 255) / 256, B * Hkv), 256, 0, st>>>(A.R, NC, 1,
                                                                                    nullptr);

@@ -687,54 +687,90 @@ int launch_prep(const int32_t* gid, const float* L, const int32_t* G, float eps,
 // same sums in the same order as state_simt_kernel, so the same bits, with every chunk's
 // products computed at once instead of one chunk after another.
 // ------------------------------------------------------------------------------------------
+// out[n][f] += sum over the 64 rows j of A[j][f] B[j][n], in row order, for one 64-row tile.
+// 256 threads: thread t owns f = 4 (t & 15) .. + 3 and n = 4 (t >> 4) .. + 3 (and n = 64 for
+// t < 16), reading four A and four B values per row as vectors.
+__device__ __forceinline__ void tile_acc_simt(const float (*A)[68], const float (*B)[68],
+                                              float (&t4)[4][4], float (&tn)[4])
+{
+    const int fg = threadIdx.x & 15, nq = threadIdx.x >> 4;
+#pragma unroll 4
+    for (int j = 0; j < 64; ++j) {
+        const float4 a = *reinterpret_cast<const float4*>(&A[j][4 * fg]);
+        const float4 b = *reinterpret_cast<const float4*>(&B[j][4 * nq]);
+        const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) t4[i][jj] = fmaf(av[i], bv[jj], t4[i][jj]);
+        if (nq == 0) {
+            const float bn = B[j][kDV];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) tn[i] = fmaf(av[i], bn, tn[i]);
+        }
+    }
+}
+
+// The tile's sums to dst[n * kFP + f0 + f] (65 columns n, 64 packed rows f).
+__device__ __forceinline__ void tile_store_simt(float* __restrict__ dst, int f0,
+                                                const float (&t4)[4][4], const float (&tn)[4])
+{
+    const int fg = threadIdx.x & 15, nq = threadIdx.x >> 4;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) dst[size_t(4 * nq + jj) * kFP + f0 + 4 * fg + i] = t4[i][jj];
+        if (nq == 0) dst[size_t(kDV) * kFP + f0 + 4 * fg + i] = tn[i];
+    }
+}
+
+struct DeltaSmem {
+    float ks[64][kDA + 1];  // k rows of the tile (and the constant 1, 0)
+    float A[64][68];        // psi of the tile's rows, [token][packed row of the slab]
+    float B[64][68];        // [v; 1] of the tile's rows
+};
+
 template <typename Tin>
 __global__ void __launch_bounds__(256) chunk_delta_simt_kernel(const Tin* __restrict__ k,
                                                                const Tin* __restrict__ v, int T,
                                                                int C, int NC,
                                                                float* __restrict__ Hc)
 {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    DeltaSmem& sm = *reinterpret_cast<DeltaSmem*>(smem_raw);
     const int slab = blockIdx.x, bkv = blockIdx.z;
     const int tid = threadIdx.x, fi = tid & 63, cg = tid >> 6;
-    const int f = slab * 64 + fi;
-    const RT rt = feature_rt(f);
-    __shared__ float ks[64][kDA + 1];
-    __shared__ float vs[64][kW];
+    const RT rt = feature_rt(slab * 64 + fi);
     const Tin* kb = k + size_t(bkv) * T * kD;
     const Tin* vb = v + size_t(bkv) * T * kDV;
     for (int c = blockIdx.y; c < NC; c += gridDim.y) {  // (gridDim.y < NC only past 65535)
-        float acc[17];
+        float t4[4][4], tn[4];
 #pragma unroll
-        for (int u = 0; u < 17; ++u) acc[u] = 0.f;
+        for (int i = 0; i < 4; ++i) {
+            tn[i] = 0.f;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) t4[i][jj] = 0.f;
+        }
         const int t0 = c * C, t1 = min(t0 + C, T);
         for (int s0 = t0; s0 < t1; s0 += 64) {
             for (int e = tid; e < 64 * kD; e += 256) {
                 const int j = e / kD, r = e % kD, tok = s0 + j;
-                ks[j][r] = tok < t1 ? to_f32(kb[size_t(tok) * kD + r]) : 0.f;
-                vs[j][r] = tok < t1 ? to_f32(vb[size_t(tok) * kDV + r]) : 0.f;
+                sm.ks[j][r] = tok < t1 ? to_f32(kb[size_t(tok) * kD + r]) : 0.f;
+                sm.B[j][r] = tok < t1 ? to_f32(vb[size_t(tok) * kDV + r]) : 0.f;
             }
             if (tid < 64) {
                 const bool ok = s0 + tid < t1;
-                ks[tid][kD] = ok ? 1.f : 0.f;
-                ks[tid][kD + 1] = 0.f;
-                vs[tid][kDV] = ok ? 1.f : 0.f;
+                sm.ks[tid][kD] = ok ? 1.f : 0.f;
+                sm.ks[tid][kD + 1] = 0.f;
+                sm.B[tid][kDV] = ok ? 1.f : 0.f;
             }
             __syncthreads();
-            for (int j = 0; j < 64; ++j) {
-                const float psi = ks[j][rt.r] * ks[j][rt.t];
-#pragma unroll
-                for (int u = 0; u < 17; ++u) {
-                    const int n = cg + 4 * u;
-                    if (n < kW) acc[u] = fmaf(psi, vs[j][n], acc[u]);
-                }
-            }
+            for (int j = cg; j < 64; j += 4) sm.A[j][fi] = sm.ks[j][rt.r] * sm.ks[j][rt.t];
+            __syncthreads();
+            tile_acc_simt(sm.A, sm.B, t4, tn);
             __syncthreads();
         }
-        float* dst = Hc + (size_t(bkv) * NC + c) * kW * kFP;
-#pragma unroll
-        for (int u = 0; u < 17; ++u) {
-            const int n = cg + 4 * u;
-            if (n < kW) dst[size_t(n) * kFP + f] = acc[u];
-        }
+        tile_store_simt(Hc + (size_t(bkv) * NC + c) * kW * kFP, slab * 64, t4, tn);
     }
 }
 
@@ -786,8 +822,11 @@ int launch_chunk_states_simt(const Tin* k, const Tin* v, int T, int C, int NC, f
         OAL_LAUNCH_CHECK();
         return OAL_OK;
     }
-    chunk_delta_simt_kernel<Tin><<<dim3(kFP / 64, std::min(NC, 65535), nbkv), 256, 0, st>>>(
-        k, v, T, C, NC, Hc);
+    OAL_CUDA_TRY(cudaFuncSetAttribute(chunk_delta_simt_kernel<Tin>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      int(sizeof(DeltaSmem))));
+    chunk_delta_simt_kernel<Tin><<<dim3(kFP / 64, std::min(NC, 65535), nbkv), 256,
+                                   sizeof(DeltaSmem), st>>>(k, v, T, C, NC, Hc);
     OAL_LAUNCH_CHECK();
     chunk_scan_kernel<<<dim3((kW * kFP + 255) / 256, nbkv), 256, 0, st>>>(Hc, NC, 0, body);
     OAL_LAUNCH_CHECK();
