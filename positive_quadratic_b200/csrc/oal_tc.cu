@@ -254,29 +254,32 @@ constexpr bool psi_chunk_needed(int ch)
     return false;
 }
 
-// diagonal / linear / constant slabs: 32 rows with compile-time (r, t); fp32 products (exact)
-// split into hi and lo
+// diagonal / linear / constant slabs: 32 rows with compile-time (r, t), split exactly into hi
+// and lo like the off-diagonal ones: each pair of rows gathers its two k_r and its two k_t
+// into one bf16x2 register each with one byte permute (k_64 = `one`, k_65 = 0 from a constant
+// word), then hi = bf16(k_r k_t) and lo = the exact remainder.
 template <int F0>
 __device__ __forceinline__ void psi_static(const unsigned char* ktile, int trow, float one,
                                            uint32_t abase, int j)
 {
-    float k[66];
+    uint32_t kw[32];  // packed bf16 pairs of the k chunks these rows read
     static_for<8>([&](auto CH) {
         constexpr int ch = decltype(CH)::value;
         if constexpr (psi_chunk_needed<F0>(ch)) {
             const uint4 w = *reinterpret_cast<const uint4*>(ktile + kmajor_chunk(trow, ch));
-            k[ch * 8 + 0] = bf16lo_to_f32(w.x);
-            k[ch * 8 + 1] = bf16hi_to_f32(w.x);
-            k[ch * 8 + 2] = bf16lo_to_f32(w.y);
-            k[ch * 8 + 3] = bf16hi_to_f32(w.y);
-            k[ch * 8 + 4] = bf16lo_to_f32(w.z);
-            k[ch * 8 + 5] = bf16hi_to_f32(w.z);
-            k[ch * 8 + 6] = bf16lo_to_f32(w.w);
-            k[ch * 8 + 7] = bf16hi_to_f32(w.w);
+            kw[ch * 4 + 0] = w.x;
+            kw[ch * 4 + 1] = w.y;
+            kw[ch * 4 + 2] = w.z;
+            kw[ch * 4 + 3] = w.w;
         }
     });
-    k[64] = one;
-    k[65] = 0.f;
+    const uint32_t onez = pack_bf16x2(one, 0.f);  // bf16 halves (k_64, k_65) = (one, 0)
+    auto word = [&](auto R) -> uint32_t {
+        constexpr int r = decltype(R)::value;
+        if constexpr (r >= 64) return onez;
+        else return kw[r >> 1];
+    };
+    auto half = [](int r) constexpr -> int { return r >= 64 ? r - 64 : (r & 1); };
     constexpr int m0 = F0 % kSlabRows;
     static_for<4>([&](auto CH) {
         constexpr int ch = decltype(CH)::value;
@@ -285,9 +288,15 @@ __device__ __forceinline__ void psi_static(const unsigned char* ktile, int trow,
             constexpr int e = decltype(E)::value;
             constexpr RT a = feature_rt(F0 + ch * 8 + 2 * e);
             constexpr RT b = feature_rt(F0 + ch * 8 + 2 * e + 1);
-            const float pa = k[a.r] * k[a.t], pb = k[b.r] * k[b.t];
-            h[e] = pack_bf16x2(pa, pb);
-            l[e] = pack_bf16x2(pa - bf16lo_to_f32(h[e]), pb - bf16hi_to_f32(h[e]));
+            // low half from the first word, high half from the second (bytes 4..7)
+            constexpr uint32_t sr = (half(a.r) ? 0x32u : 0x10u) | ((half(b.r) ? 0x76u : 0x54u) << 8);
+            constexpr uint32_t st = (half(a.t) ? 0x32u : 0x10u) | ((half(b.t) ? 0x76u : 0x54u) << 8);
+            const uint32_t xr = __byte_perm(word(std::integral_constant<int, a.r>{}),
+                                            word(std::integral_constant<int, b.r>{}), sr);
+            const uint32_t xt = __byte_perm(word(std::integral_constant<int, a.t>{}),
+                                            word(std::integral_constant<int, b.t>{}), st);
+            h[e] = bmul2(xr, xt);
+            l[e] = bfma2(xr, xt, h[e] ^ 0x80008000u);
         });
         sts128(abase + st_a_off(m0 + 8 * ch, j), h[0], h[1], h[2], h[3]);
         sts128(abase + kStATile + st_a_off(m0 + 8 * ch, j), l[0], l[1], l[2], l[3]);
