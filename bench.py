@@ -610,6 +610,24 @@ def run_extras(dev, torch, oal, pk):
     def to(a, d=None):
         return torch.from_numpy(np.ascontiguousarray(a)).to(dev, d)
 
+    try:  # dense O(T^2) form against the linear-time prefill; the contribution statistic
+        pc = I.config1()
+        q, k, v = (to(x, torch.bfloat16) for x in (pc.q, pc.k, pc.v))
+        g, L, G = to(pc.group_id), to(pc.L), to(pc.G)
+        pts = {}
+        for T in (1024, 4096):
+            qq, kk, vv = (x[:, :, :T].contiguous() for x in (q, k, v))
+            ms_d = timed(lambda: oal.dense_ref(qq, kk, vv, g, L, G, pc.eps), reps=2)
+            ms_l = timed(lambda: oal.prefill(qq, kk, vv, g, L, G, pc.eps, 128))
+            pts[f"T{T}"] = {"dense_ms": ms_d, "linear_ms": ms_l}
+        res["dense_vs_linear"] = {"workload": "B=1 Hq=14 Hkv=2 bf16 inputs; oal_dense_ref_gpu "
+                                              "(O(T^2), CUDA cores, fp32) against oal_prefill "
+                                              "(tensor cores, chunk 128)", "points": pts}
+        ms = timed(lambda: oal.contribution_stat(q, k))
+        res["contribution_stat"] = {"workload": "eq. (1) chi over B=1 T=4096 Hq=14 Hkv=2 bf16",
+                                    "ms": ms}
+    except Exception as exc:
+        res["dense_vs_linear"] = {"error": repr(exc)[:300]}
     try:  # ungrouped Hadamard form, CUDA cores, chunk 64
         p = I.small_layer(901, B=1, T=2048, Hq=14, Hkv=2, dtype="bf16")
         q, k, v = (to(x, torch.bfloat16) for x in (p.q, p.k, p.v))
