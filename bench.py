@@ -289,6 +289,40 @@ def cpu_baseline(p, budget_s=12.0):
                       f"{el:.1f} s", "seconds": el}
 
 
+def cpu_baseline_decode(p, steps=16):
+    """The fp64 oracle's decode step on this host's cores: batch and heads of `p`, the state
+    of a 16-token prefix (a step's cost does not depend on the context length: the state has
+    a fixed size), then `steps` single-token steps continuing it."""
+    import oracle
+    pre = 16
+    sl = lambda a, t0, t1: np.ascontiguousarray(a[:, :, t0:t1])  # noqa: E731
+    _, st = oracle.recurrent(sl(p.q, 0, pre), sl(p.k, 0, pre), sl(p.v, 0, pre), p.group_id,
+                             p.L, p.G, p.eps, return_state=True)
+    t0 = time.perf_counter()
+    for t in range(pre, pre + steps):
+        _, st = oracle.recurrent(sl(p.q, t, t + 1), sl(p.k, t, t + 1), sl(p.v, t, t + 1),
+                                 p.group_id, p.L, p.G, p.eps, state=st, return_state=True)
+    el = time.perf_counter() - t0
+    B = p.q.shape[0]
+    return {"value": B * steps / el, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"fp64 oracle recurrence, batch {B}, {steps} single-token steps after a "
+                      f"{pre}-token prefix (a step's cost does not depend on the context), "
+                      f"{el:.1f} s", "seconds": el}
+
+
+def cpu_baseline_long(T=16384):
+    """The fp64 oracle on one long-context layer (config 3's shape at T), one run."""
+    import oracle
+    from positive_quadratic_b200 import inputs as I
+    p = I.config3(T)
+    t0 = time.perf_counter()
+    oracle.recurrent(p.q, p.k, p.v, p.group_id, p.L, p.G, p.eps)
+    el = time.perf_counter() - t0
+    return {"value": T / el, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"fp64 oracle recurrence on the full layer B=1 T={T} Hq=14, one run, "
+                      f"{el:.1f} s", "seconds": el}
+
+
 def run_reference(args):
     """The reference arm: the fp64 oracle timed on this host's cores (rank 0 only)."""
     rank = int(os.environ.get("RANK", "0"))
@@ -465,6 +499,12 @@ def main():
     base = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         base = cpu_baseline(p)
+        from positive_quadratic_b200 import inputs as I
+        if isinstance(decode, dict):
+            decode["cpu_baseline"] = cpu_baseline_decode(I.config4(batch=64, context=20,
+                                                                   steps=0))
+        if isinstance(extras, dict) and isinstance(extras.get("config3_long_context"), dict):
+            extras["config3_long_context"]["cpu_baseline_T16384"] = cpu_baseline_long(16384)
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
