@@ -499,12 +499,15 @@ def main():
     base = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         base = cpu_baseline(p)
-        from positive_quadratic_b200 import inputs as I
-        if isinstance(decode, dict):
-            decode["cpu_baseline"] = cpu_baseline_decode(I.config4(batch=64, context=20,
-                                                                   steps=0))
-        if isinstance(extras, dict) and isinstance(extras.get("config3_long_context"), dict):
-            extras["config3_long_context"]["cpu_baseline_T16384"] = cpu_baseline_long(16384)
+        try:  # recorded in the line; the headline value stands either way
+            from positive_quadratic_b200 import inputs as I
+            if isinstance(decode, dict):
+                decode["cpu_baseline"] = cpu_baseline_decode(
+                    I.config4(batch=64, context=20, steps=0))
+            if isinstance(extras, dict) and isinstance(extras.get("config3_long_context"), dict):
+                extras["config3_long_context"]["cpu_baseline_T16384"] = cpu_baseline_long(16384)
+        except Exception as exc:
+            base["extra_error"] = repr(exc)[:300]
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
