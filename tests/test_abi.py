@@ -126,6 +126,15 @@ def test_decode_and_dense_host_side_errors(L):
     assert L.oal_device_error(None, None) == -1
 
 
+@pytest.mark.parametrize("B,Hq,Hkv", [(1, 14, 2), (64, 14, 2), (3, 8, 1), (5, 6, 3)])
+def test_decode_workspace_size(B, Hq, Hkv):
+    """The decode scratch is the reserved leading block plus one partial readout (65 fp32) per
+    slab (9 of 240 packed rows) and query head: align256(4 B Hkv) + 2340 B Hq bytes, the
+    size include/oal.h states for the no-alloc entry point."""
+    n = oal.decode_workspace_bytes(oal.make_shape(B, 1, Hq, Hkv))
+    assert n == (4 * B * Hkv + 255) // 256 * 256 + 2340 * B * Hq
+
+
 def test_header_packed_order_is_complete():
     """The packed order written in include/oal.h covers every pair r <= t of 65 exactly once."""
     from tests._packed import packed_pairs
