@@ -2,8 +2,7 @@
 
 Callers that cannot allocate device memory (a serving engine that owns all GPU memory, a
 plugin interface that passes only inputs and outputs) use oal_decode_step_noalloc, whose
-scratch lives in a fixed array inside the library.  This file is collected last so that a
-run that stops at the first failure has already run every other test."""
+scratch lives in a fixed array inside the library."""
 import ctypes
 
 import numpy as np
