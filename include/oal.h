@@ -171,9 +171,9 @@ int oal_decode_step(const void* q, const void* k, const void* v, void* state, fl
  * cannot afford cudaMalloc's implicit device-wide synchronisation.
  * Same arguments and results as oal_decode_step, minus the workspace.  The scratch is a
  * fixed 4 MiB array inside the library (one copy on every GPU that loads the library, held
- * until the process exits).  A step needs align256(4*B*Hkv) + 2340*B*Hq bytes of it, so
- * B*Hq must stay at or below 1788 (batch 64 x 14 heads fits); larger problems return
- * OAL_ERR_UNSUPPORTED without launching anything.
+ * until the process exits).  A step needs align256(4*B*Hkv) + 2340*B*Hq bytes of it; a step
+ * that needs more than 4 MiB returns OAL_ERR_UNSUPPORTED without launching anything.  Every
+ * B*Hq up to 1789 fits, whatever Hkv (batch 64 x 14 heads needs 2.1 MB).
  * The first call on each device looks up the array's device address (cudaGetSymbolAddress)
  * and caches it; make that first call before any stream capture.  cudaDeviceReset discards
  * the library's device code and data on that device, and with them the array the cached
@@ -340,10 +340,12 @@ int oal_dense_backward_gpu(const void* q, const void* k, const void* v, const in
                            void* workspace, size_t workspace_bytes, const oal_shape* s,
                            void* stream);
 
-/* Scratch needed by oal_backward for `s` (B, T, Hq, Hkv used): the fp32 prefix and suffix
- * chunk states (2 x 565,760 bytes per (b, kv head, chunk of 64 tokens)), per row of every
- * query head its normaliser, output, upstream gradient of u, partial dM and deps, and one
- * partial dC' (2176 floats) per (b, query head, chunk). */
+/* Scratch needed by oal_backward for `s` (B, T, Hq, Hkv used): a state buffer
+ * (oal_state_bytes), the fp32 prefix and suffix chunk states (2 x 565,760 bytes per
+ * (b, kv head, chunk of 64 tokens)), per row of every query head its normaliser (1 float),
+ * output (64), upstream gradient of u (65), partial dM (81) and deps (1), one partial dC'
+ * (2176 floats) per (b, query head, chunk) and one float per query head; each part starts
+ * on a 256-byte boundary. */
 int oal_backward_workspace_bytes(const oal_shape* s, size_t* bytes);
 
 /* Training-scale gradients: the same outputs, layouts and conventions as

@@ -13,8 +13,8 @@
 namespace oal {
 
 // 4 MiB: room for the reserved leading block and the per-slab partial readouts (9 slabs x 65
-// fp32 per query head) of a decode step with B*Hq up to 1788 query heads (batch 64 x 14 heads
-// needs 2.1 MB).
+// fp32 per query head) of a decode step with B*Hq up to 1789 query heads, whatever Hkv
+// (batch 64 x 14 heads needs 2.1 MB).
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];

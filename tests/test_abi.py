@@ -301,3 +301,120 @@ def test_dense_backward_host_side_errors(L):
     mis = list(args)
     mis[13] = _fake((1 << 24) + 16)
     assert L.oal_dense_backward_gpu(*mis) == -4
+
+
+@pytest.mark.parametrize("B,T,Hq,Hkv", [(1, 4096, 14, 2), (2, 100, 4, 2), (1, 64, 8, 1),
+                                        (3, 0, 6, 3)])
+def test_backward_workspace_size(L, B, T, Hq, Hkv):
+    """The chunked backward's scratch as include/oal.h lists it, part by part."""
+    s = oal.make_shape(B, T, Hq, Hkv, 128, oal.OAL_F32)
+    n = ctypes.c_size_t(0)
+    assert L.oal_backward_workspace_bytes(ctypes.byref(s), ctypes.byref(n)) == 0
+    NC, rows = -(-T // 64), B * Hq * T
+    parts = [oal.state_bytes(s), B * Hkv * NC * 565760, B * Hkv * NC * 565760, rows * 4,
+             rows * 64 * 4, rows * 65 * 4, B * Hq * NC * 2176 * 4, rows * 81 * 4, rows * 4,
+             Hq * 4]
+    assert n.value == max(256, sum(_align256(x) for x in parts))
+    assert L.oal_backward_workspace_bytes(ctypes.byref(s), None) == -1
+
+
+def test_backward_host_side_errors(L):
+    s = oal.make_shape(1, 64, 2, 1, 128, oal.OAL_F32)
+    n = ctypes.c_size_t(0)
+    assert L.oal_backward_workspace_bytes(ctypes.byref(s), ctypes.byref(n)) == 0
+    P = _fake(1 << 20)
+    # q k v gid L G eps dy dq dk dv dL deps ws bytes shape stream
+    args = [P] * 6 + [ctypes.c_float(1e-6)] + [P] * 6 + [_fake(1 << 24), n, ctypes.byref(s),
+                                                         None]
+    for i in (0, 3, 4, 5, 7, 8, 9, 10, 11, 12):   # every pointer the call reads or writes
+        bad = list(args)
+        bad[i] = None
+        assert L.oal_backward(*bad) == -1, i
+    for i in (0, 7, 9, 11):                        # q, dy, dk, dL not 16-byte aligned
+        mis = list(args)
+        mis[i] = _fake((1 << 20) + 4)
+        assert L.oal_backward(*mis) == -4, i
+    small = list(args)
+    small[14] = ctypes.c_size_t(n.value - 1)
+    assert L.oal_backward(*small) == -8
+    nows = list(args)
+    nows[13] = None
+    assert L.oal_backward(*nows) == -8
+    mis_ws = list(args)
+    mis_ws[13] = _fake((1 << 24) + 16)             # workspace not 256-byte aligned
+    assert L.oal_backward(*mis_ws) == -4
+    wide = oal.make_shape(1, 64, 18, 2, 128, oal.OAL_F32)   # 9 query heads per kv head
+    assert L.oal_backward(*args[:15], ctypes.byref(wide), None) == -3
+
+
+def test_prefill_continue_host_side_checks(L):
+    """A continuation exists only on the tensor-core path (bf16, chunk 128); appending no
+    tokens returns at once, before any device work."""
+    P = _fake(1 << 20)
+    ws = ctypes.c_size_t(1 << 40)
+    for dtype, chunk in ((oal.OAL_F32, 128), (oal.OAL_BF16, 64), (oal.OAL_BF16, 256)):
+        s = oal.make_shape(1, 256, 2, 1, chunk, dtype)
+        assert L.oal_prefill_continue(*[P] * 6, ctypes.c_float(1e-6), P, P, P, ws,
+                                      ctypes.byref(s), None) == -3
+    s = oal.make_shape(1, 256, 2, 1, 128, oal.OAL_BF16)
+    assert L.oal_prefill_continue(*[P] * 6, ctypes.c_float(1e-6), P, None, P, ws,
+                                  ctypes.byref(s), None) == -1
+    empty = oal.make_shape(1, 0, 2, 1, 128, oal.OAL_BF16)
+    assert L.oal_prefill_continue(None, None, None, P, P, P, ctypes.c_float(1e-6), None, P, P,
+                                  ws, ctypes.byref(empty), None) == 0
+    odd = oal.make_shape(1, 256, 2, 1, 96, oal.OAL_BF16)
+    assert L.oal_prefill_continue(*[P] * 6, ctypes.c_float(1e-6), P, P, P, ws,
+                                  ctypes.byref(odd), None) == -3
+
+
+def test_noalloc_decode_host_side_checks(L):
+    """The allocation-free decode refuses a step whose scratch would exceed its fixed 4 MiB
+    array before it touches the device; B*Hq = 1789 fits whatever Hkv."""
+    fn = L.oal_decode_step_noalloc
+    fn.argtypes = [ctypes.c_void_p] * 5 + [ctypes.POINTER(oal.Shape), ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    P = _fake(1 << 20)
+    assert _align256(4 * 1789) + 2340 * 1789 <= 4 << 20                 # Hkv = Hq, the worst
+    assert _align256(4 * 128 * 2) + 2340 * 128 * 14 == 4 << 20          # exactly full
+    for B, Hq, Hkv in ((129, 14, 2), (1790, 1, 1), (225, 8, 1)):
+        need = _align256(4 * B * Hkv) + 2340 * B * Hq
+        assert need > 4 << 20
+        big = oal.make_shape(B, 1, Hq, Hkv, 128, oal.OAL_BF16)
+        assert fn(P, P, P, P, P, ctypes.byref(big), None) == -3
+    s = oal.make_shape(64, 1, 14, 2, 128, oal.OAL_BF16)
+    assert fn(P, P, P, None, P, ctypes.byref(s), None) == -1      # no state
+    assert fn(P, None, P, P, P, ctypes.byref(s), None) == -1      # no k
+    assert fn(P, P, P, _fake((1 << 20) + 8), P, ctypes.byref(s), None) == -4
+    assert fn(P, P, P, P, P, None, None) == -1
+
+
+def test_contribution_stat_host_side_checks(L):
+    P = _fake(1 << 20)
+    s = oal.make_shape(2, 300, 14, 2, 128, oal.OAL_BF16)
+    assert L.oal_contribution_stat(P, None, P, ctypes.byref(s), None) == -1
+    assert L.oal_contribution_stat(P, P, _fake((1 << 20) + 4), ctypes.byref(s), None) == -4
+    empty = oal.make_shape(2, 0, 14, 2, 128, oal.OAL_BF16)      # nothing to write
+    assert L.oal_contribution_stat(None, None, None, ctypes.byref(empty), None) == 0
+    bad = oal.make_shape(2, 300, 14, 3, 128, oal.OAL_BF16)      # Hq not a multiple of Hkv
+    assert L.oal_contribution_stat(P, P, P, ctypes.byref(bad), None) == -2
+
+
+def test_state_prefix_sum_host_side_checks(L):
+    P = _fake(1 << 20)
+    n = ctypes.c_size_t(1024)
+    assert L.oal_state_prefix_sum(P, -1, n, P, None) == -2
+    assert L.oal_state_prefix_sum(None, 2, ctypes.c_size_t(0), None, None) == 0
+    assert L.oal_state_prefix_sum(None, 2, n, P, None) == -1
+    assert L.oal_state_prefix_sum(P, 2, n, None, None) == -1
+    assert L.oal_state_prefix_sum(P, 2, ctypes.c_size_t(1022), P, None) == -4
+    assert L.oal_state_prefix_sum(_fake((1 << 20) + 4), 2, n, P, None) == -4
+
+
+def test_overlap_switch_returns_previous_setting(L):
+    prev = L.oal_set_prefill_overlap(0)
+    try:
+        assert prev in (0, 1)
+        assert L.oal_set_prefill_overlap(7) == 0
+        assert L.oal_set_prefill_overlap(1) == 1
+    finally:
+        L.oal_set_prefill_overlap(prev)
