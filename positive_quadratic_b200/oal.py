@@ -414,11 +414,12 @@ def _hadamard_coefs(q, a, b, C):
     return a, b, C
 
 
-def prefill_hadamard(q, k, v, a, b, C, chunk: int = 64, out=None, state=None, workspace=None,
+def prefill_hadamard(q, k, v, a, b, C, chunk: int = 128, out=None, state=None, workspace=None,
                      stream=None):
     """oal_prefill_hadamard: causal prefill with kappa = a + b.x + x^T C x, x = q*k/sqrt(64)
-    (per query head a [Hq], b [Hq, 64], C [Hq, 64, 64]).  Returns (out, state); the state
-    continues with decode_step."""
+    (per query head a [Hq], b [Hq, 64], C [Hq, 64, 64]).  bf16 with chunk 128 (the default,
+    as for prefill) runs on tensor cores.  Returns (out, state); the state continues with
+    decode_step."""
     shape = _shape_of(q, k, v, chunk)
     dev = q.device
     a, b, C = _hadamard_coefs(q, a, b, C)
