@@ -119,3 +119,37 @@ def test_scan_traffic_is_close_to_its_algorithmic_bytes():
     alg = bench.kernel_work(p, 128)["scan"][0]
     got = bench.profiled_traffic("config1")["scan"]
     assert 0.5 * alg <= got <= 1.25 * alg
+
+
+def _run_bench(env_extra, *argv):
+    import json
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, **env_extra)
+    r = subprocess.run([sys.executable, str(ROOT / "bench.py"), *argv], cwd=ROOT, env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    return [json.loads(ln) for ln in lines]
+
+
+def test_reference_arm_prints_one_contract_line():
+    """bench.py --impl reference times the fp64 oracle on the host (no GPU needed) and prints
+    one JSON line with the keys of the benchmark contract."""
+    (out,) = _run_bench({"RANK": "0", "WORLD_SIZE": "1"}, "--impl", "reference", "--steps",
+                        "2", "--warmup", "3")
+    assert out["impl"] == "reference" and out["n_gpus"] == 1
+    assert out["steps"] == 2 and out["warmup"] == 3
+    assert out["value"] > 0 and out["unit"] == "tokens/s" and out["higher_is_better"] is True
+    assert out["ms_per_step"] == pytest.approx(512 / out["value"] * 1e3, rel=1e-6)
+    assert out["cpu_baseline"]["kind"] == "oracle" and out["cpu_baseline"]["cores"] >= 1
+    assert out["cpu_baseline"]["value"] == out["value"]
+    assert out["e2e"] == {"value": out["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                          "d2h_bytes_per_step": 0}
+    assert "T=4096" in out["config"]["workload"]
+
+
+def test_reference_arm_other_ranks_do_no_work():
+    assert _run_bench({"RANK": "1", "WORLD_SIZE": "2"}, "--impl", "reference", "--gpus", "2",
+                      "--steps", "2", "--warmup", "3") == []
