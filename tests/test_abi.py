@@ -418,3 +418,30 @@ def test_overlap_switch_returns_previous_setting(L):
         assert L.oal_set_prefill_overlap(1) == 1
     finally:
         L.oal_set_prefill_overlap(prev)
+
+
+def test_binding_refuses_host_tensors():
+    """The Python binding has no CPU path: host tensors are refused before the library is
+    called, so nothing can silently compute elsewhere than in the CUDA kernels."""
+    import torch
+    B, Hq, Hkv, T = 1, 4, 2, 16
+    q = torch.zeros(B, Hq, T, 64, dtype=torch.bfloat16)
+    k = torch.zeros(B, Hkv, T, 64, dtype=torch.bfloat16)
+    v = torch.zeros(B, Hkv, T, 64, dtype=torch.bfloat16)
+    gid = torch.zeros(Hq, 64, dtype=torch.int32)
+    Lm = torch.eye(9, dtype=torch.float32).expand(Hq, 9, 9).contiguous()
+    G = torch.ones(Hq, dtype=torch.int32)
+    a, b, C = torch.ones(Hq), torch.zeros(Hq, 64), torch.zeros(Hq, 64, 64)
+    calls = [
+        lambda: oal.prefill(q, k, v, gid, Lm, G, 1e-6),
+        lambda: oal.dense_ref(q, k, v, gid, Lm, G, 1e-6),
+        lambda: oal.contribution_stat(q, k),
+        lambda: oal.prefill_hadamard(q, k, v, a, b, C),
+        lambda: oal.backward(q, k, v, gid, Lm, G, 1e-6, torch.zeros(B, Hq, T, 64)),
+        lambda: oal.decode_step(q[:, :, :1].contiguous(), k[:, :, :1].contiguous(),
+                                v[:, :, :1].contiguous(), torch.zeros(1 << 20, dtype=torch.uint8),
+                                oal.decode_workspace(B, Hq, Hkv, "cpu")),
+    ]
+    for call in calls:
+        with pytest.raises(ValueError, match="CUDA"):
+            call()
