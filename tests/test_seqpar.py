@@ -103,6 +103,51 @@ def test_gloo_ranks_match_whole_sequence(world):
     np.testing.assert_allclose(res[world - 1][1], st.H2, rtol=1e-10, atol=1e-12)
 
 
+def _rank_main_uneven(rank, world, port, bounds, out):
+    import torch.distributed as dist
+    from datetime import timedelta
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        p = _problem()
+        t0, t1 = bounds[rank], bounds[rank + 1]
+        s = p.slice_tokens(t0, t1)
+        y, state = seqpar.sequence_parallel_prefill(
+            torch.from_numpy(s.q), torch.from_numpy(s.k), torch.from_numpy(s.v), p.group_id,
+            p.L, p.G, p.eps, rank=rank, world=world, tokens_before=t0,
+            backend=OracleBackend())
+        out[rank] = (y.numpy(), state["st"].H2.copy(), state["tokens"])
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_gloo_ranks_uneven_segments_cover_the_sequence():
+    """Four ranks hold segments of 9, 0, 40 and 25 tokens (one empty) of a 74-token sequence:
+    together they give every token's output and, on the last rank, the whole state."""
+    import torch.multiprocessing as mp
+    world, bounds = 4, [0, 9, 9, 49, 74]
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        out = mgr.dict()
+        procs = [ctx.Process(target=_rank_main_uneven, args=(r, world, port, bounds, out))
+                 for r in range(world)]
+        for pr in procs:
+            pr.start()
+        for pr in procs:
+            pr.join(180)
+        assert all(pr.exitcode == 0 for pr in procs), [pr.exitcode for pr in procs]
+        res = dict(out)
+    p = _problem()
+    ref, st = oracle.recurrent(p.q, p.k, p.v, p.group_id, p.L, p.G, p.eps, return_state=True)
+    y = np.concatenate([res[r][0] for r in range(world)], axis=2)
+    assert y.shape == ref.shape
+    np.testing.assert_allclose(y, ref, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(res[world - 1][1], st.H2, rtol=1e-10, atol=1e-12)
+    assert [res[r][2] for r in range(world)] == bounds[:-1]
+
+
 @pytest.mark.gpu
 def test_segments_on_one_gpu_match_whole_sequence(cuda):
     """Three ranks run in this process on the library: each rank's output equals the
