@@ -388,6 +388,45 @@ def test_prefill_continuation(oal, cuda, T1, T2):
 
 
 @pytest.mark.gpu
+def test_state_saved_to_a_file_resumes_the_sequence(oal, cuda, tmp_path):
+    """The state buffer is the resumable artifact of a sequence: written to a file after a
+    prefill and read back into another device buffer (at another address), it continues the
+    sequence exactly as the original buffer does -- a prefill continuation, then decode
+    steps -- outputs and state bit for bit."""
+    T1, T2, n = 256, 300, 3
+    p = I.small_layer(733, B=2, T=T1 + T2 + n, Hq=14, Hkv=2, dtype="bf16")
+    a, b = p.slice_tokens(0, T1), p.slice_tokens(T1, T1 + T2)
+    qa, ka, va, g, L, G = dev_inputs(a, cuda)
+    qb, kb, vb, *_ = dev_inputs(b, cuda)
+    q, k, v, *_ = dev_inputs(p, cuda)
+    _, state = oal.prefill(qa, ka, va, g, L, G, p.eps, 128)
+    torch.cuda.synchronize()
+    path = tmp_path / "sequence.state"
+    state.cpu().numpy().tofile(path)
+    raw = torch.from_numpy(np.fromfile(path, dtype=np.uint8))
+    arena = torch.zeros(raw.numel() + 1024, dtype=torch.uint8, device=cuda)
+    resumed = arena[512:512 + raw.numel()]
+    resumed.copy_(raw.to(cuda))
+    assert torch.equal(resumed, state)
+    ws = oal.decode_workspace(2, 14, 2, cuda)
+    runs = []
+    for st in (state, resumed):
+        ys = [oal.prefill_continue(qb, kb, vb, g, L, G, p.eps, st)]
+        for t in range(T1 + T2, T1 + T2 + n):
+            sl = lambda x: x[:, :, t:t + 1].contiguous()  # noqa: E731
+            ys.append(oal.decode_step(sl(q), sl(k), sl(v), st, ws))
+        torch.cuda.synchronize()
+        runs.append(([y.clone() for y in ys], st.clone()))
+    assert oal.device_error() == 0
+    for y0, y1 in zip(runs[0][0], runs[1][0]):
+        assert torch.equal(y0, y1)
+    assert torch.equal(runs[0][1], runs[1][1])
+    assert torch.all(arena[:512] == 0) and torch.all(arena[512 + raw.numel():] == 0)
+    hdr, _, _ = read_state(runs[1][1].cpu().numpy(), 2, 14, 2)
+    assert hdr["tokens"] == T1 + T2 + n
+
+
+@pytest.mark.gpu
 def test_prefill_continuation_unsupported_paths(oal, cuda):
     """Continuation runs on the tensor-core path only; fp32 inputs are refused before any
     launch."""
