@@ -70,7 +70,12 @@ typedef enum {
     OAL_ERR_STATE = -9        /* state buffer does not match the shape */
 } oal_status;
 
-/* Problem description shared by every call. */
+/* Problem description shared by every call.  Size limits checked on the host (OAL_ERR_SHAPE):
+ * B*Hq*max(T, 1) < 2^31 rows; and, because a grid holds at most 65535 blocks in its y and z
+ * dimensions, B*Hq <= 65535 for the CUDA-core prefill, the Hadamard and dense forms and both
+ * backward passes, B*Hkv <= 65535 for the decode step, and B*Hkv + 1 <= 65535 for the
+ * tensor-core prefill (n_seq*Hkv + 1 for the packed batch).  The size queries
+ * (*_workspace_bytes) apply the same limits. */
 typedef struct {
     int32_t B;     /* batch */
     int32_t T;     /* tokens per sequence (oal_decode_step: ignored, one token) */

@@ -41,6 +41,13 @@ int check_chunk(const oal_shape* s)
                                                                    : OAL_ERR_UNSUPPORTED;
 }
 
+// A grid's y and z dimensions hold at most 65535 blocks.  The CUDA-core kernels put the
+// B*Hq query-head planes there, the decode step the B*Hkv state planes, and the tensor-core
+// scan the B*Hkv state planes plus one for the coefficient tables.
+constexpr long long kMaxGridPlanes = 65535;
+
+int check_planes(long long planes) { return planes > kMaxGridPlanes ? OAL_ERR_SHAPE : OAL_OK; }
+
 size_t simt_chunk_state_bytes(const oal_shape* s)
 {
     const size_t NC = s->T > 0 ? size_t((s->T + s->chunk - 1) / s->chunk) : 0;
@@ -49,6 +56,13 @@ size_t simt_chunk_state_bytes(const oal_shape* s)
 
 // bf16 inputs with chunk 128 run on the tcgen05 kernels; everything else on CUDA cores.
 bool use_tensor_path(const oal_shape* s) { return s->dtype == OAL_BF16 && s->chunk == 128; }
+
+// The prefill's grid planes on the path the shape takes.
+int check_prefill_planes(const oal_shape* s)
+{
+    return check_planes(use_tensor_path(s) ? (long long)s->B * s->Hkv + 1
+                                           : (long long)s->B * s->Hq);
+}
 
 std::atomic<int> g_prefill_overlap{1};
 
@@ -96,6 +110,7 @@ int oal_prefill_workspace_bytes(const oal_shape* s, size_t* bytes)
     int rc = check_common(s);
     if (rc) return rc;
     if ((rc = check_chunk(s))) return rc;
+    if ((rc = check_prefill_planes(s))) return rc;
     if (!bytes) return OAL_ERR_NULL;
     const size_t tc = use_tensor_path(s) ? tc_workspace_bytes(s->B, s->Hq, s->Hkv, s->T) : 0;
     *bytes = simt_chunk_state_bytes(s) > tc ? simt_chunk_state_bytes(s) : tc;
@@ -115,8 +130,9 @@ int oal_prefill_path(const oal_shape* s, int* path)
 
 int oal_decode_workspace_bytes(const oal_shape* s, size_t* bytes)
 {
-    const int rc = check_common(s);
+    int rc = check_common(s);
     if (rc) return rc;
+    if ((rc = check_planes((long long)s->B * s->Hkv))) return rc;
     if (!bytes) return OAL_ERR_NULL;
     *bytes = decode_ticket_bytes(s) + decode_part_bytes(s);
     return OAL_OK;
@@ -133,6 +149,7 @@ int prefill_impl(const void* q, const void* k, const void* v, const int32_t* gro
     if (rc) return rc;
     if ((rc = check_chunk(s))) return rc;
     if (cont && !use_tensor_path(s)) return OAL_ERR_UNSUPPORTED;
+    if ((rc = check_prefill_planes(s))) return rc;
     if (!group_id || !L || !G || !state) return OAL_ERR_NULL;
     // out == NULL asks for the state alone (no readout); q is then not read either
     if ((rc = check_io(s, out ? q : k, k, v, out ? out : v))) return rc;
@@ -183,6 +200,7 @@ int oal_decode_step(const void* q, const void* k, const void* v, void* state, fl
 {
     int rc = check_common(s);
     if (rc) return rc;
+    if ((rc = check_planes((long long)s->B * s->Hkv))) return rc;
     oal_shape one = *s;
     one.T = 1;
     if (!state) return OAL_ERR_NULL;
@@ -204,6 +222,7 @@ int oal_dense_ref_gpu(const void* q, const void* k, const void* v, const int32_t
 {
     int rc = check_common(s);
     if (rc) return rc;
+    if ((rc = check_planes((long long)s->B * s->Hq))) return rc;
     if (!group_id || !L || !G) return OAL_ERR_NULL;
     if ((rc = check_io(s, q, k, v, out))) return rc;
     if (!aligned16(group_id) || !aligned16(L) || !aligned16(G)) return OAL_ERR_ALIGN;

@@ -649,8 +649,9 @@ extern "C" {
 int oal_backward_workspace_bytes(const oal_shape* s, size_t* bytes)
 {
     using namespace oal;
-    const int rc = check_common(s);
+    int rc = check_common(s);
     if (rc) return rc;
+    if ((rc = check_planes((long long)s->B * s->Hq))) return rc;
     if (!bytes) return OAL_ERR_NULL;
     *bytes = cb_layout(s->B, s->T, s->Hq, s->Hkv).total;
     return OAL_OK;
@@ -664,6 +665,7 @@ int oal_backward(const void* q, const void* k, const void* v, const int32_t* gro
     using namespace oal;
     int rc = check_common(s);
     if (rc) return rc;
+    if ((rc = check_planes((long long)s->B * s->Hq))) return rc;
     if (!group_id || !L || !G || !dL || !deps) return OAL_ERR_NULL;
     if ((rc = check_io(s, q, k, v, dq))) return rc;
     if ((long long)s->B * s->T > 0 && (!dy || !dk || !dv)) return OAL_ERR_NULL;

@@ -271,10 +271,12 @@ int oal_prefill_hadamard(const void* q, const void* k, const void* v, const floa
     int rc = check_common(s);
     if (rc) return rc;
     if ((rc = check_chunk(s))) return rc;
+    const bool tensor = use_tensor_path(s) && out != nullptr;
+    if ((rc = check_planes(tensor ? (long long)s->B * s->Hkv + 1 : (long long)s->B * s->Hq)))
+        return rc;
     if (!a || !b || !C || !state) return OAL_ERR_NULL;
     if ((rc = check_io(s, q, k, v, out))) return rc;
     if (!aligned16(a) || !aligned16(b) || !aligned16(C) || !aligned16(state)) return OAL_ERR_ALIGN;
-    const bool tensor = use_tensor_path(s) && out != nullptr;
     const size_t need = tensor ? tc_workspace_bytes(s->B, s->Hq, s->Hkv, s->T)
                                : simt_chunk_state_bytes(s);
     if (need > 0 && (!workspace || workspace_bytes < need)) return OAL_ERR_WORKSPACE;
@@ -306,6 +308,7 @@ int oal_dense_hadamard_gpu(const void* q, const void* k, const void* v, const fl
     using namespace oal;
     int rc = check_common(s);
     if (rc) return rc;
+    if ((rc = check_planes((long long)s->B * s->Hq))) return rc;
     if (!a || !b || !C) return OAL_ERR_NULL;
     if ((rc = check_io(s, q, k, v, out))) return rc;
     if (!aligned16(a) || !aligned16(b) || !aligned16(C)) return OAL_ERR_ALIGN;

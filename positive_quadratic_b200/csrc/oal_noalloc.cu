@@ -52,6 +52,7 @@ extern "C" int oal_decode_step_noalloc(const void* q, const void* k, const void*
     using namespace oal;
     int rc = check_common(s);
     if (rc) return rc;
+    if ((rc = check_planes((long long)s->B * s->Hkv))) return rc;
     oal_shape one = *s;
     one.T = 1;
     if (!state) return OAL_ERR_NULL;

@@ -75,6 +75,8 @@ int plan_packed(const oal_shape* s, const int32_t* seq_lens, int n_seq, TcPacked
     if (rc) return rc;
     if ((rc = check_chunk(&one))) return rc;
     if (!use_tensor_path(&one)) return OAL_ERR_UNSUPPORTED;
+    // the scan's grid planes: every sequence's kv heads and the coefficient tables
+    if ((rc = check_planes((long long)n_seq * s->Hkv + 1))) return rc;
     *lay = tc_packed_layout(s->Hq, s->Hkv, seq_lens, n_seq);
     // tensor-copy row coordinates of the chunk-state images are 32-bit
     if (lay->chunks * s->Hkv * 34 * 80 >= (1LL << 31)) return OAL_ERR_SHAPE;

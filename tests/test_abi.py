@@ -445,3 +445,62 @@ def test_binding_refuses_host_tensors():
     for call in calls:
         with pytest.raises(ValueError, match="CUDA"):
             call()
+
+
+def _ws(L, fn, s):
+    n = ctypes.c_size_t(0)
+    return getattr(L, fn)(ctypes.byref(s), ctypes.byref(n))
+
+
+def test_grid_plane_limits():
+    """Grids hold at most 65535 blocks in y and z: B*Hq for the CUDA-core kernels (prefill,
+    Hadamard and dense forms, both backward passes), B*Hkv for the decode step and B*Hkv + 1
+    for the tensor-core prefill's scan.  Larger problems are refused on the host with
+    OAL_ERR_SHAPE, at the size query and at the call, before any device work.  The calls
+    get NULL pointers, so a missing size check would show as OAL_ERR_NULL instead."""
+    L = oal.lib()
+    F32, BF16 = oal.OAL_F32, oal.OAL_BF16
+    P = None
+    eps = ctypes.c_float(1e-6)
+    big = ctypes.c_size_t(1 << 45)
+    # CUDA-core prefill: B*Hq planes
+    assert _ws(L, "oal_prefill_workspace_bytes", oal.make_shape(13107, 1, 5, 5, 64, F32)) == 0
+    over = oal.make_shape(6554, 1, 10, 2, 64, F32)                # 65540 planes
+    assert _ws(L, "oal_prefill_workspace_bytes", over) == -2
+    assert L.oal_prefill(None, None, None, None, None, None, eps, None, None, None, big,
+                         ctypes.byref(over), None) == -2
+    # tensor-core prefill: B*Hkv + 1 planes (B*Hq does not matter there)
+    assert _ws(L, "oal_prefill_workspace_bytes", oal.make_shape(6554, 1, 10, 2, 128, BF16)) == 0
+    assert _ws(L, "oal_prefill_workspace_bytes", oal.make_shape(32767, 1, 2, 2, 128, BF16)) == 0
+    tc_over = oal.make_shape(32768, 1, 2, 2, 128, BF16)             # 65536 + 1 planes
+    assert _ws(L, "oal_prefill_workspace_bytes", tc_over) == -2
+    assert L.oal_prefill_continue(None, None, None, None, None, None, eps, None, None, None,
+                                  big, ctypes.byref(tc_over), None) == -2
+    assert _host_ws(L, tc_over, 1)[0] == -2
+    # decode: B*Hkv planes, both entry points
+    assert _ws(L, "oal_decode_workspace_bytes", oal.make_shape(32767, 1, 4, 2)) == 0
+    dec_over = oal.make_shape(32768, 1, 4, 2)                       # 65536 planes
+    assert _ws(L, "oal_decode_workspace_bytes", dec_over) == -2
+    assert L.oal_decode_step(P, P, P, P, P, P, big, ctypes.byref(dec_over), None) == -2
+    fn = L.oal_decode_step_noalloc
+    fn.argtypes = [ctypes.c_void_p] * 5 + [ctypes.POINTER(oal.Shape), ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    assert fn(P, P, P, P, P, ctypes.byref(dec_over), None) == -2
+    # dense form, Hadamard forms, backward passes: B*Hq planes
+    assert L.oal_dense_ref_gpu(P, P, P, P, P, P, eps, P, ctypes.byref(over), None) == -2
+    assert L.oal_dense_hadamard_gpu(P, P, P, P, P, P, P, ctypes.byref(over), None) == -2
+    assert L.oal_prefill_hadamard(P, P, P, P, P, P, P, P, P, big, ctypes.byref(over),
+                                  None) == -2
+    for name in ("oal_backward", "oal_dense_backward_gpu"):
+        assert _ws(L, name.replace("_gpu", "") + "_workspace_bytes", over) == -2
+        assert getattr(L, name)(*[P] * 6, eps, *[P] * 6, P, big, ctypes.byref(over),
+                                None) == -2
+    assert _ws(L, "oal_backward_workspace_bytes", oal.make_shape(13107, 1, 5, 5, 64, F32)) == 0
+    # packed batch: every sequence's kv heads plus one plane
+    lens = (ctypes.c_int32 * 32768)(*([1] * 32768))
+    n = ctypes.c_size_t(0)
+    s = oal.make_shape(1, 0, 2, 2, 128, BF16)
+    assert L.oal_prefill_packed_workspace_bytes(ctypes.byref(s), lens, 32767,
+                                                ctypes.byref(n)) == 0
+    assert L.oal_prefill_packed_workspace_bytes(ctypes.byref(s), lens, 32768,
+                                                ctypes.byref(n)) == -2
