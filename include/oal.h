@@ -74,8 +74,10 @@ typedef enum {
  * B*Hq*max(T, 1) < 2^31 rows; and, because a grid holds at most 65535 blocks in its y and z
  * dimensions, B*Hq <= 65535 for the CUDA-core prefill, the Hadamard and dense forms and both
  * backward passes, B*Hkv <= 65535 for the decode step, and B*Hkv + 1 <= 65535 for the
- * tensor-core prefill (n_seq*Hkv + 1 for the packed batch).  The size queries
- * (*_workspace_bytes) apply the same limits. */
+ * tensor-core prefill (n_seq*Hkv + 1 for the packed batch).  The tensor-core prefill also
+ * needs B*Hkv*ceil(T/128)*34*80 < 2^31 (32-bit row coordinates of its chunk-state images;
+ * chunks*Hkv*34*80 for the packed batch).  The size queries (*_workspace_bytes) apply the
+ * same limits. */
 typedef struct {
     int32_t B;     /* batch */
     int32_t T;     /* tokens per sequence (oal_decode_step: ignored, one token) */

@@ -57,11 +57,16 @@ size_t simt_chunk_state_bytes(const oal_shape* s)
 // bf16 inputs with chunk 128 run on the tcgen05 kernels; everything else on CUDA cores.
 bool use_tensor_path(const oal_shape* s) { return s->dtype == OAL_BF16 && s->chunk == 128; }
 
-// The prefill's grid planes on the path the shape takes.
+// The prefill's size limits on the path the shape takes: its grid planes, and on tensor cores
+// the 32-bit row coordinate (tc::kImgRows rows per slice) of the chunk-state images that the
+// readout loads.
 int check_prefill_planes(const oal_shape* s)
 {
-    return check_planes(use_tensor_path(s) ? (long long)s->B * s->Hkv + 1
-                                           : (long long)s->B * s->Hq);
+    if (!use_tensor_path(s)) return check_planes((long long)s->B * s->Hq);
+    const long long NC = (s->T + tc::kC - 1) / tc::kC;
+    if ((long long)s->B * s->Hkv * NC * tc::kSlices * tc::kImgRows >= (1LL << 31))
+        return OAL_ERR_SHAPE;
+    return check_planes((long long)s->B * s->Hkv + 1);
 }
 
 std::atomic<int> g_prefill_overlap{1};

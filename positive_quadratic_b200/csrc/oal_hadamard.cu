@@ -272,7 +272,7 @@ int oal_prefill_hadamard(const void* q, const void* k, const void* v, const floa
     if (rc) return rc;
     if ((rc = check_chunk(s))) return rc;
     const bool tensor = use_tensor_path(s) && out != nullptr;
-    if ((rc = check_planes(tensor ? (long long)s->B * s->Hkv + 1 : (long long)s->B * s->Hq)))
+    if ((rc = tensor ? check_prefill_planes(s) : check_planes((long long)s->B * s->Hq)))
         return rc;
     if (!a || !b || !C || !state) return OAL_ERR_NULL;
     if ((rc = check_io(s, q, k, v, out))) return rc;

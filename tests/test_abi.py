@@ -477,6 +477,14 @@ def test_grid_plane_limits():
     assert L.oal_prefill_continue(None, None, None, None, None, None, eps, None, None, None,
                                   big, ctypes.byref(tc_over), None) == -2
     assert _host_ws(L, tc_over, 1)[0] == -2
+    # tensor-core prefill: the chunk-state images' 32-bit row coordinate (34 slices of 80 rows
+    # per chunk and kv head)
+    assert _ws(L, "oal_prefill_workspace_bytes", oal.make_shape(1, 98689 * 128, 8, 8, 128,
+                                                                BF16)) == 0
+    long_tc = oal.make_shape(1, 98690 * 128, 8, 8, 128, BF16)
+    assert 8 * 98689 * 34 * 80 < 1 << 31 <= 8 * 98690 * 34 * 80
+    assert _ws(L, "oal_prefill_workspace_bytes", long_tc) == -2
+    assert L.oal_prefill(P, P, P, P, P, P, eps, P, P, P, big, ctypes.byref(long_tc), None) == -2
     # decode: B*Hkv planes, both entry points
     assert _ws(L, "oal_decode_workspace_bytes", oal.make_shape(32767, 1, 4, 2)) == 0
     dec_over = oal.make_shape(32768, 1, 4, 2)                       # 65536 planes
