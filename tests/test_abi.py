@@ -2,6 +2,7 @@
 header declares, and rejects bad arguments on the host before touching the device."""
 import ctypes
 
+import numpy as np
 import pytest
 
 from positive_quadratic_b200 import build, oal
@@ -512,3 +513,31 @@ def test_grid_plane_limits():
                                                 ctypes.byref(n)) == 0
     assert L.oal_prefill_packed_workspace_bytes(ctypes.byref(s), lens, 32768,
                                                 ctypes.byref(n)) == -2
+
+
+def test_library_packed_order_matches_header(tmp_path):
+    """The library's packed feature order (its feature_rt, compiled for the host from the CUDA
+    sources) is the order include/oal.h documents, row for row; the padding rows map past the
+    last dimension (65, 65)."""
+    import os
+    import subprocess
+    from tests._packed import F, FP, packed_pairs
+    csrc = os.path.join(os.path.dirname(oal.LIB_PATH), "csrc")
+    src = tmp_path / "rt.cu"
+    src.write_text('#include "oal_common.cuh"\n#include <cstdio>\n'
+                   "int main() {\n"
+                   "    for (int f = 0; f < oal::kFP; ++f) {\n"
+                   "        const oal::RT rt = oal::feature_rt(f);\n"
+                   '        std::printf("%d %d\\n", rt.r, rt.t);\n'
+                   "    }\n"
+                   "    return 0;\n"
+                   "}\n")
+    exe = tmp_path / "rt"
+    nvcc = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
+    subprocess.check_call([nvcc, "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a",
+                           "-I", csrc, str(src), "-o", str(exe)])
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout
+    rt = np.array([[int(x) for x in ln.split()] for ln in out.splitlines()])
+    assert rt.shape == (FP, 2)
+    assert np.array_equal(rt[:F], packed_pairs())
+    assert np.all(rt[F:] == 65)
