@@ -66,3 +66,22 @@ def pack_oracle_state(st, pairs=None):
         else:
             out[:, :, f] = st.H0
     return out
+
+
+def coef_from_header(group_id, L, G, eps):
+    """Readout weights [Hq, FP] of the packed rows as include/oal.h states them:
+    (r == t ? 1 : 2) * M_{g(r),g(t)} * s_r * s_t with M = L L^T, g(64) = 0, s_r = 1/8 for
+    r < 64 and s_64 = 1, plus eps on the constant row 2144; zero on the padding rows."""
+    pairs = packed_pairs()
+    Hq = G.shape[0]
+    out = np.zeros((Hq, FP))
+    for h in range(Hq):
+        Gh = int(G[h])
+        Lh = L[h, :Gh + 1, :Gh + 1].astype(np.float64)
+        M = Lh @ Lh.T
+        g = np.concatenate([group_id[h], [0]])
+        s = np.concatenate([np.full(64, 0.125), [1.0]])
+        r, t = pairs[:, 0], pairs[:, 1]
+        out[h, :F] = np.where(r == t, 1.0, 2.0) * M[g[r], g[t]] * s[r] * s[t]
+        out[h, 2144] += eps
+    return out

@@ -9,7 +9,7 @@ import pytest
 import oracle
 from positive_quadratic_b200 import inputs as I
 from tests._metrics import TOL_BF16, TOL_F32, row_rel_err
-from tests._packed import F, FP, pack_oracle_state, packed_pairs, read_state
+from tests._packed import F, FP, coef_from_header, pack_oracle_state, read_state
 
 pytestmark = pytest.mark.gpu
 
@@ -137,19 +137,7 @@ def test_bad_group_id_sets_error_word(oal, cuda):
 
 def _coef_reference(p):
     """Readout weights of the packed rows per include/oal.h, from L and the group ids."""
-    pairs = packed_pairs()
-    Hq = p.G.shape[0]
-    out = np.zeros((Hq, FP))
-    for h in range(Hq):
-        Gh = int(p.G[h])
-        Lh = p.L[h, :Gh + 1, :Gh + 1].astype(np.float64)
-        M = Lh @ Lh.T
-        g = np.concatenate([p.group_id[h], [0]])
-        s = np.concatenate([np.full(64, 0.125), [1.0]])
-        r, t = pairs[:, 0], pairs[:, 1]
-        out[h, :F] = np.where(r == t, 1.0, 2.0) * M[g[r], g[t]] * s[r] * s[t]
-        out[h, 2144] += p.eps
-    return out
+    return coef_from_header(p.group_id, p.L, p.G, p.eps)
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
