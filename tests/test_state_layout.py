@@ -47,3 +47,29 @@ def test_coefficient_rows_by_hand():
     g = int(p.group_id[h, out])
     assert coef[h, pairs.index((out, 64))] == pytest.approx(2 * M[g, 0] / 8)
     assert coef[h, pairs.index((64, 64))] == pytest.approx(M[0, 0] + p.eps)
+
+
+def test_hadamard_state_reads_out_with_its_coefficients():
+    """The state of the Hadamard form has the same packed rows; its readout weights follow
+    from kappa = a + b.x + x^T C x with x_r = q_r k_r / 8: a on the constant row, b_r / 8 on
+    the linear row of r, (C_rt + C_tr) / 64 on a cross row r < t and C_rr / 64 on a square."""
+    rng = np.random.default_rng(25)
+    p = I.small_layer(25, B=1, T=21, Hq=4, Hkv=2, dtype="f32")
+    Hq = 4
+    a = rng.uniform(1.0, 2.0, Hq)
+    b = rng.normal(0.0, 0.5, (Hq, 64))
+    C = rng.normal(0.0, 0.2, (Hq, 64, 64))
+    y, st = oracle.hadamard_recurrent(p.q, p.k, p.v, a, b, C, return_state=True)
+    S = pack_oracle_state(st)
+    pairs = packed_pairs()
+    r, t = pairs[:, 0], pairs[:, 1]
+    T = p.q.shape[2]
+    for h in range(Hq):
+        cr = np.where(t == 64, 0, np.minimum(r, 63))
+        ct = np.minimum(t, 63)
+        coef = np.where(r == t, C[h, cr, ct], C[h, cr, ct] + C[h, ct, cr]) / 64.0
+        coef = np.where(t == 64, b[h, np.minimum(r, 63)] / 8.0, coef)
+        coef = np.where((r == 64) & (t == 64), a[h], coef)
+        qhat = np.concatenate([p.q[0, h, T - 1].astype(np.float64), [1.0]])
+        u = (coef * qhat[r] * qhat[t]) @ S[0, h // 2]
+        np.testing.assert_allclose(u[:64] / u[64], y[0, h, T - 1], rtol=1e-9, atol=1e-12)
