@@ -191,3 +191,48 @@ def test_state_prefix_sum(cuda, n_parts):
         ref = ref + parts[r]
     torch.cuda.synchronize()
     assert torch.equal(out, ref)
+
+
+def _rank_main_failing(rank, world, port, out):
+    import torch.distributed as dist
+    from datetime import timedelta
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=10))
+    if rank == 1:  # this rank fails before its exchange step and leaves
+        raise SystemExit(3)
+    p = _problem()
+    s = p.slice_tokens(0, 37)
+    try:
+        seqpar.sequence_parallel_prefill(
+            torch.from_numpy(s.q), torch.from_numpy(s.k), torch.from_numpy(s.v), p.group_id,
+            p.L, p.G, p.eps, rank=rank, world=world, tokens_before=0, backend=OracleBackend())
+        out[rank] = "returned"
+    except Exception as exc:  # the collective reports the lost peer
+        out[rank] = "error: " + type(exc).__name__
+
+
+def test_a_failed_rank_ends_the_others_exchange_with_an_error():
+    """A rank that leaves before the exchange step makes the other ranks' all-gather end with
+    an error (the peer's closed connection or the process group's short timeout), not a hang."""
+    import time
+    import torch.multiprocessing as mp
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    t0 = time.monotonic()
+    with ctx.Manager() as mgr:
+        out = mgr.dict()
+        procs = [ctx.Process(target=_rank_main_failing, args=(r, world, port, out))
+                 for r in range(world)]
+        for pr in procs:
+            pr.start()
+        for pr in procs:
+            pr.join(120)
+        alive = [pr.is_alive() for pr in procs]
+        for pr in procs:
+            if pr.is_alive():
+                pr.kill()
+        res = dict(out)
+    assert not any(alive), "a rank hung"
+    assert procs[1].exitcode == 3
+    assert res.get(0, "").startswith("error"), res
+    assert time.monotonic() - t0 < 120
